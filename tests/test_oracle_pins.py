@@ -1,0 +1,413 @@
+"""Pins the fp64 oracle to facts that do not come from the oracle itself.
+
+Closed forms, brute force on tiny inputs, hand-worked examples from
+tests/golden and identities of the mathematics.  Each check is chosen so that
+a plausible slip in the oracle (a dropped term, a wrong sign or index, a
+transposed operand) fails it.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import mamba as om
+from oracle import moe as omoe
+from oracle import native
+from synthetic import MambaShape, mamba_params, mamba_input
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _rand_scan(rng, B=2, L=9, C=5, N=4, a_neg=True):
+    x = rng.standard_normal((B, L, C))
+    dt = np.log1p(np.exp(rng.standard_normal((B, L, C)) - 2.0))
+    A = -np.exp(rng.standard_normal((C, N))) if a_neg else rng.standard_normal((C, N))
+    Bm = rng.standard_normal((B, L, N))
+    Cm = rng.standard_normal((B, L, N))
+    D = rng.standard_normal(C)
+    z = rng.standard_normal((B, L, C))
+    return x, dt, A, Bm, Cm, D, z
+
+
+# ----------------------------------------------------------------- scan pins
+
+def test_scan_hand_example():
+    g = _golden("scan_hand_example.json")
+    ln2 = math.log(2.0)
+    x = np.array(g["x"])[None, :, None]
+    L = x.shape[1]
+    dt = np.full((1, L, 1), ln2)
+    A = np.array(g["A"])[None, :]
+    Bm = np.tile(np.array(g["B"]), (1, L, 1))
+    Cm = np.tile(np.array(g["C"]), (1, L, 1))
+    D = np.array([g["D"]])
+    want = np.array(g["y_ln2_coef"]) * ln2 + np.array(g["y_const"])
+    want_h = np.array(g["h_last_ln2_coef"]) * ln2
+    for fn in (om.selective_scan, om.selective_scan_c):
+        y, h = fn(x, dt, A, Bm, Cm, D)
+        np.testing.assert_allclose(y[0, :, 0], want, rtol=1e-14)
+        np.testing.assert_allclose(h[0, 0], want_h, rtol=1e-14)
+
+
+def test_scan_A_zero_is_cumsum():
+    rng = np.random.default_rng(1)
+    x, dt, A, Bm, Cm, D, z = _rand_scan(rng)
+    A = np.zeros_like(A)
+    # h_t[c, n] = sum_{s<=t} dt_s[c] B_s[n] x_s[c]
+    contrib = dt[..., None] * Bm[:, :, None, :] * x[..., None]      # [B, L, C, N]
+    hcum = np.cumsum(contrib, axis=1)
+    want = (np.einsum("blcn,bln->blc", hcum, Cm) + D * x) * (z / (1 + np.exp(-z)))
+    for fn in (om.selective_scan, om.selective_scan_c):
+        y, h = fn(x, dt, A, Bm, Cm, D, z)
+        np.testing.assert_allclose(y, want, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(h, hcum[:, -1], rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("L", [1, 2, 3, 5])
+def test_scan_bruteforce_unrolled(L):
+    """y_t = sum_{s<=t} sum_n C_t[n] (prod_{r=s+1..t} e^{dt_r A_n}) dt_s B_s[n] x_s + D x_t."""
+    rng = np.random.default_rng(10 + L)
+    x, dt, A, Bm, Cm, D, z = _rand_scan(rng, B=1, L=L, C=3, N=3)
+    want = np.zeros((1, L, 3))
+    for c in range(3):
+        for t in range(L):
+            acc = 0.0
+            for s in range(t + 1):
+                for n in range(3):
+                    decay = 1.0
+                    for r in range(s + 1, t + 1):
+                        decay *= math.exp(dt[0, r, c] * A[c, n])
+                    acc += Cm[0, t, n] * decay * dt[0, s, c] * Bm[0, s, n] * x[0, s, c]
+            want[0, t, c] = acc + D[c] * x[0, t, c]
+    for fn in (om.selective_scan, om.selective_scan_c):
+        y, _ = fn(x, dt, A, Bm, Cm, D)
+        np.testing.assert_allclose(y, want, rtol=1e-12, atol=1e-13)
+
+
+def test_scan_constant_input_geometric_series():
+    L, C, N = 40, 2, 3
+    dtv, xv = 0.3, 1.7
+    A = np.array([[-0.5, -1.0, -2.0], [-0.1, -0.2, -3.0]])
+    Bv = np.array([0.4, -1.1, 2.0])
+    x = np.full((1, L, C), xv)
+    dt = np.full((1, L, C), dtv)
+    Bm = np.tile(Bv, (1, L, 1))
+    Cm = np.tile(np.array([1.0, 0.0, 0.0]), (1, L, 1))
+    D = np.zeros(C)
+    _, h = om.selective_scan(x, dt, A, Bm, Cm, D)
+    a = np.exp(dtv * A)                                   # [C, N]
+    want = dtv * Bv[None] * xv * (1 - a ** L) / (1 - a)
+    np.testing.assert_allclose(h[0], want, rtol=1e-13)
+
+
+def test_scan_C_zero_gives_skip_times_gate():
+    rng = np.random.default_rng(3)
+    x, dt, A, Bm, Cm, D, z = _rand_scan(rng)
+    y, _ = om.selective_scan(x, dt, A, Bm, np.zeros_like(Cm), D, z)
+    np.testing.assert_allclose(y, D * x * z / (1 + np.exp(-z)), rtol=1e-14)
+
+
+def test_scan_linear_in_x():
+    rng = np.random.default_rng(4)
+    x, dt, A, Bm, Cm, D, z = _rand_scan(rng)
+    x2 = rng.standard_normal(x.shape)
+    y1, h1 = om.selective_scan(x, dt, A, Bm, Cm, D, z)
+    y2, h2 = om.selective_scan(x2, dt, A, Bm, Cm, D, z)
+    y3, h3 = om.selective_scan(2.0 * x - 3.0 * x2, dt, A, Bm, Cm, D, z)
+    np.testing.assert_allclose(y3, 2.0 * y1 - 3.0 * y2, rtol=1e-11, atol=1e-11)
+    np.testing.assert_allclose(h3, 2.0 * h1 - 3.0 * h2, rtol=1e-11, atol=1e-11)
+
+
+def test_scan_initial_state_is_zero_input_prefix():
+    """Starting from h0 equals scanning a prefix that produced h0."""
+    rng = np.random.default_rng(5)
+    x, dt, A, Bm, Cm, D, z = _rand_scan(rng, L=12)
+    y_all, h_all = om.selective_scan(x, dt, A, Bm, Cm, D, z)
+    _, h_mid = om.selective_scan(x[:, :5], dt[:, :5], A, Bm[:, :5], Cm[:, :5], D)
+    y_tail, h_tail = om.selective_scan(x[:, 5:], dt[:, 5:], A, Bm[:, 5:], Cm[:, 5:], D,
+                                       z[:, 5:], h0=h_mid)
+    np.testing.assert_allclose(y_tail, y_all[:, 5:], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(h_tail, h_all, rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("chunk", [1, 7, 64, 300])
+def test_scan_chunked_equals_sequential(chunk):
+    rng = np.random.default_rng(6)
+    x, dt, A, Bm, Cm, D, z = _rand_scan(rng, B=2, L=150, C=4, N=16)
+    h0 = rng.standard_normal((2, 4, 16))
+    y1, h1 = om.selective_scan(x, dt, A, Bm, Cm, D, z, h0)
+    y2, h2 = om.selective_scan_chunked(x, dt, A, Bm, Cm, D, z, h0, chunk=chunk)
+    np.testing.assert_allclose(y2, y1, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(h2, h1, rtol=1e-12, atol=1e-12)
+
+
+def test_scan_c_matches_numpy_on_random():
+    rng = np.random.default_rng(7)
+    x, dt, A, Bm, Cm, D, z = _rand_scan(rng, B=2, L=64, C=6, N=16)
+    h0 = rng.standard_normal((2, 6, 16))
+    y1, h1 = om.selective_scan(x, dt, A, Bm, Cm, D, z, h0)
+    y2, h2 = native.scan(x, dt, A, Bm, Cm, D, z, h0)
+    np.testing.assert_allclose(y2, y1, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(h2, h1, rtol=1e-13, atol=1e-13)
+
+
+# ----------------------------------------------------------------- conv pins
+
+def test_conv_hand_example():
+    g = _golden("conv_hand_example.json")
+    x = np.array(g["x"])[None, :, None]
+    w = np.array(g["w"])[None, :]
+    out, st = om.causal_conv1d(x, w, np.array([g["b"]]))
+    np.testing.assert_allclose(out[0, :, 0], g["out_pre_activation"], rtol=0, atol=0)
+    np.testing.assert_allclose(st[0, 0], g["state_after"], rtol=0, atol=0)
+
+
+def test_conv_delta_kernels():
+    rng = np.random.default_rng(8)
+    x = rng.standard_normal((2, 10, 3))
+    ident = np.tile([0.0, 0.0, 0.0, 1.0], (3, 1))
+    out, _ = om.causal_conv1d(x, ident, np.zeros(3))
+    np.testing.assert_array_equal(out, x)
+    shift = np.tile([1.0, 0.0, 0.0, 0.0], (3, 1))
+    out, st = om.causal_conv1d(x, shift, np.zeros(3))
+    np.testing.assert_array_equal(out[:, 3:], x[:, :-3])
+    np.testing.assert_array_equal(out[:, :3], 0.0)
+    np.testing.assert_array_equal(st, np.transpose(x[:, -3:], (0, 2, 1)))
+
+
+def test_conv_vs_torch_conv1d():
+    rng = np.random.default_rng(9)
+    B, L, C, K = 2, 17, 5, 4
+    x = rng.standard_normal((B, L, C))
+    w = rng.standard_normal((C, K))
+    b = rng.standard_normal(C)
+    out, _ = om.causal_conv1d(x, w, b)
+    t = torch.nn.functional.conv1d(torch.from_numpy(x).permute(0, 2, 1),
+                                   torch.from_numpy(w)[:, None, :], torch.from_numpy(b),
+                                   padding=K - 1, groups=C)[..., :L]
+    np.testing.assert_allclose(out, t.permute(0, 2, 1).numpy(), rtol=1e-13, atol=1e-13)
+
+
+def test_conv_state_continues_sequence():
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((1, 9, 4))
+    w = rng.standard_normal((4, 4))
+    b = rng.standard_normal(4)
+    full, st_full = om.causal_conv1d(x, w, b)
+    a, st = om.causal_conv1d(x[:, :2], w, b)         # shorter than the window
+    rest, st2 = om.causal_conv1d(x[:, 2:], w, b, st)
+    np.testing.assert_allclose(np.concatenate([a, rest], 1), full, rtol=1e-14)
+    np.testing.assert_array_equal(st2, st_full)
+
+
+# ------------------------------------------------------ elementwise and norms
+
+def test_linear_vs_triple_loop():
+    rng = np.random.default_rng(12)
+    x = rng.standard_normal((3, 4))
+    W = rng.standard_normal((5, 4))
+    want = [[sum(x[i, k] * W[j, k] for k in range(4)) for j in range(5)] for i in range(3)]
+    np.testing.assert_allclose(om.linear(x, W), np.array(want), rtol=1e-14)
+    np.testing.assert_array_equal(om.linear(x, np.eye(4)), x)
+
+
+def test_rmsnorm_identities():
+    rng = np.random.default_rng(13)
+    w = rng.standard_normal(8)
+    c = np.full((2, 8), -3.5)                       # constant vector -> w * sign
+    np.testing.assert_allclose(om.rmsnorm(c, w, 0.0), -np.tile(w, (2, 1)), rtol=1e-15)
+    x = rng.standard_normal((3, 8))
+    np.testing.assert_allclose(om.rmsnorm(7.0 * x, w, 0.0), om.rmsnorm(x, w, 0.0), rtol=1e-14)
+    # unit weights: mean of squares of the output is 1
+    y = om.rmsnorm(x, np.ones(8), 0.0)
+    np.testing.assert_allclose(np.mean(y * y, axis=-1), 1.0, rtol=1e-14)
+    # eps enters under the root
+    e = 0.25
+    np.testing.assert_allclose(om.rmsnorm(x, np.ones(8), e),
+                               x / np.sqrt(np.mean(x * x, -1, keepdims=True) + e), rtol=1e-15)
+
+
+def test_softplus_silu_identities():
+    v = np.linspace(-30, 30, 61)
+    sp = om.softplus(v)
+    np.testing.assert_allclose(sp, [math.log1p(math.exp(t)) for t in v], rtol=1e-14)
+    np.testing.assert_allclose(sp - om.softplus(-v), v, rtol=1e-13, atol=1e-13)
+    assert om.softplus(np.array([0.0]))[0] == pytest.approx(math.log(2.0), rel=1e-15)
+    s = om.silu(v)
+    np.testing.assert_allclose(s - om.silu(-v), v, rtol=1e-13, atol=1e-13)
+    assert om.silu(np.array([0.0]))[0] == 0.0
+    np.testing.assert_allclose(s, [t / (1 + math.exp(-t)) for t in v], rtol=1e-14)
+
+
+# --------------------------------------------------------------- mixer pins
+
+def _tiny_shape(inner_norm):
+    return MambaShape(d_model=8, d_inner=12, d_state=16, d_conv=4, dt_rank=3,
+                      dtype="f32", inner_norm=inner_norm)
+
+
+@pytest.mark.parametrize("inner_norm", [False, True])
+def test_step_equals_prefill_of_L_plus_1(inner_norm):
+    sh = _tiny_shape(inner_norm)
+    p = om.params64(mamba_params(sh, seed=3, a_init="random", norm_init="random",
+                                 d_init="random"))
+    u = om.to64(mamba_input(sh, batch=2, seqlen=10, seed=3))
+    full = om.mamba_prefill(p, u, sh)
+    part = om.mamba_prefill(p, u[:, :7], sh)
+    cs, ss = part["conv_state"], part["ssm_state"]
+    for t in range(7, 10):
+        o, cs, ss = om.mamba_step(p, u[:, t], sh, cs, ss)
+        np.testing.assert_allclose(o, full["out"][:, t], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(cs, full["conv_state"], rtol=1e-14)
+    np.testing.assert_allclose(ss, full["ssm_state"], rtol=1e-12, atol=1e-13)
+
+
+def test_prefill_continues_from_states():
+    sh = _tiny_shape(True)
+    p = om.params64(mamba_params(sh, seed=4))
+    u = om.to64(mamba_input(sh, batch=1, seqlen=12, seed=4))
+    full = om.mamba_prefill(p, u, sh)
+    a = om.mamba_prefill(p, u[:, :5], sh)
+    b = om.mamba_prefill(p, u[:, 5:], sh, a["conv_state"], a["ssm_state"])
+    np.testing.assert_allclose(b["out"], full["out"][:, 5:], rtol=1e-12, atol=1e-13)
+
+
+def test_prefill_step_order_by_hand():
+    """The composed layer against the same steps written out with torch fp64."""
+    sh = _tiny_shape(True)
+    p = mamba_params(sh, seed=5, norm_init="random", d_init="random")
+    u = mamba_input(sh, batch=1, seqlen=6, seed=5).double()[0]
+    P = {k: v.double() for k, v in p.items()}
+    di, N, R = sh.d_inner, sh.d_state, sh.dt_rank
+    xz = u @ P["in_proj"].T
+    x, z = xz[:, :di], xz[:, di:]
+    conv = torch.nn.functional.conv1d(x.T[None], P["conv_w"][:, None, :], P["conv_b"],
+                                      padding=3, groups=di)[0, :, :6].T
+    xc = torch.nn.functional.silu(conv)
+    pr = xc @ P["x_proj"].T
+    rn = lambda a, w: a * torch.rsqrt((a * a).mean(-1, keepdim=True) + sh.eps) * w
+    dtl, Bm, Cm = rn(pr[:, :R], P["norm_dt"]), rn(pr[:, R:R + N], P["norm_B"]), \
+        rn(pr[:, R + N:], P["norm_C"])
+    dt = torch.nn.functional.softplus(dtl @ P["dt_proj"].T + P["dt_bias"])
+    h = torch.zeros(di, N, dtype=torch.float64)
+    ys = []
+    for t in range(6):
+        h = torch.exp(dt[t, :, None] * P["A"]) * h + dt[t, :, None] * Bm[t][None] * xc[t, :, None]
+        ys.append((h @ Cm[t] + P["D"] * xc[t]) * torch.nn.functional.silu(z[t]))
+    want = torch.stack(ys) @ P["out_proj"].T
+    got = om.mamba_prefill(om.params64(p), om.to64(u[None]), sh)["out"][0]
+    np.testing.assert_allclose(got, want.numpy(), rtol=1e-12, atol=1e-13)
+
+
+# ------------------------------------------------------------------ MoE pins
+
+def test_router_vs_bruteforce_sort():
+    facts = _golden("page_facts.json")
+    E, K = facts["n_experts"], facts["top_k"]
+    rng = np.random.default_rng(14)
+    v = rng.standard_normal((40, 6))
+    W = rng.standard_normal((E, 6))
+    idx, w, logits = omoe.router(v, W, K)
+    for t in range(40):
+        lg = [sum(v[t, j] * W[e, j] for j in range(6)) for e in range(E)]
+        order = sorted(range(E), key=lambda e: (-lg[e], e))[:K]
+        assert list(idx[t]) == order
+        den = sum(math.exp(l) for l in lg)
+        np.testing.assert_allclose(w[t], [math.exp(lg[e]) / den for e in order], rtol=1e-12)
+
+
+def test_router_ties_go_to_lower_index():
+    W = np.zeros((16, 4))
+    W[3] = W[9] = W[12] = [1.0, 0, 0, 0]            # three equal winners
+    v = np.array([[2.0, 0, 0, 0], [-1.0, 0, 0, 0]])
+    idx, w, _ = omoe.router(v, W, 2)
+    assert list(idx[0]) == [3, 9]
+    # negative logit for the three: the 13 zero-logit experts win, lowest first
+    assert list(idx[1]) == [0, 1]
+    np.testing.assert_allclose(w[1], 1.0 / (13 + 3 * math.exp(-1.0)), rtol=1e-14)
+
+
+def test_router_constructed_winners():
+    E = 16
+    W = np.eye(E)
+    v = np.zeros((E, E))
+    for t in range(E):
+        v[t, t] = 5.0
+        v[t, (t + 7) % E] = 3.0
+    idx, _, _ = omoe.router(v, W, 2)
+    np.testing.assert_array_equal(idx[:, 0], np.arange(E))
+    np.testing.assert_array_equal(idx[:, 1], (np.arange(E) + 7) % E)
+
+
+def test_permutation_invariants():
+    rng = np.random.default_rng(15)
+    T, E, K = 97, 16, 2
+    idx = np.stack([rng.choice(E, 2, replace=False) for _ in range(T)]).astype(np.int32)
+    counts, offsets, perm = omoe.permute(idx, E)
+    assert counts.sum() == T * K
+    assert sorted(perm.tolist()) == list(range(T * K))
+    keys = [(idx.reshape(-1)[f], f // K, f % K) for f in perm]
+    assert keys == sorted(keys)
+    for e in range(E):
+        seg = perm[offsets[e]:offsets[e + 1]]
+        assert all(idx.reshape(-1)[f] == e for f in seg)
+    inv = np.empty_like(perm)
+    inv[perm] = np.arange(T * K)
+    np.testing.assert_array_equal(perm[inv], np.arange(T * K))
+
+
+def test_swiglu_expert_vs_loop():
+    rng = np.random.default_rng(16)
+    v = rng.standard_normal((2, 3))
+    g, u, d = rng.standard_normal((4, 3)), rng.standard_normal((4, 3)), rng.standard_normal((3, 4))
+    want = np.zeros((2, 3))
+    for t in range(2):
+        a = []
+        for j in range(4):
+            gv = sum(v[t, k] * g[j, k] for k in range(3))
+            uv = sum(v[t, k] * u[j, k] for k in range(3))
+            a.append(gv / (1 + math.exp(-gv)) * uv)
+        for o in range(3):
+            want[t, o] = sum(a[j] * d[o, j] for j in range(4))
+    np.testing.assert_allclose(omoe.swiglu_expert(v, g, u, d), want, rtol=1e-13)
+
+
+def test_moe_identical_experts():
+    rng = np.random.default_rng(17)
+    E, dm, dff = 16, 6, 5
+    g, u, d = rng.standard_normal((dff, dm)), rng.standard_normal((dff, dm)), rng.standard_normal((dm, dff))
+    p = dict(router=rng.standard_normal((E, dm)), w_gate=np.stack([g] * E),
+             w_up=np.stack([u] * E), w_down=np.stack([d] * E))
+    v = rng.standard_normal((11, dm))
+    r = omoe.moe_forward(p, v, 2)
+    want = r["w"].sum(1)[:, None] * omoe.swiglu_expert(v, g, u, d)
+    np.testing.assert_allclose(r["out"], want, rtol=1e-12, atol=1e-13)
+    # sampling tokens gives the same rows
+    r2 = omoe.moe_forward(p, v, 2, tokens=[3, 7])
+    np.testing.assert_allclose(r2["out"], r["out"][[3, 7]], rtol=1e-14)
+
+
+def test_moe_single_expert_routing_by_hand():
+    """Only experts 0 and 1 can win: out = p0 * f0(v) + p1 * f1(v)."""
+    rng = np.random.default_rng(18)
+    E, dm, dff = 16, 4, 3
+    R = np.full((E, dm), 0.0)
+    R[0, 0], R[1, 1] = 10.0, 9.0
+    v = np.abs(rng.standard_normal((5, dm))) + 1.0
+    v[:, 1] = v[:, 0]                                  # expert 0 logit > expert 1 logit
+    p = dict(router=R, w_gate=rng.standard_normal((E, dff, dm)),
+             w_up=rng.standard_normal((E, dff, dm)), w_down=rng.standard_normal((E, dm, dff)))
+    r = omoe.moe_forward(p, v, 2)
+    assert (r["idx"][:, 0] == 0).all() and (r["idx"][:, 1] == 1).all()
+    f = lambda e: omoe.swiglu_expert(v, p["w_gate"][e], p["w_up"][e], p["w_down"][e])
+    want = r["w"][:, :1] * f(0) + r["w"][:, 1:] * f(1)
+    np.testing.assert_allclose(r["out"], want, rtol=1e-13)
