@@ -1,0 +1,390 @@
+#!/usr/bin/env python
+"""Throughput of the Jamba Mamba mixer on B200: one JSON line on rank 0.
+
+A step is one prefill of a 131072-token sequence (batch 1) through the whole
+mixer at Jamba width (d_model 4096, d_inner 8192, d_state 16, dt_rank 256,
+inner RMSNorm): in_proj, conv+SiLU, x_proj, inner norms, dt_proj+softplus,
+selective scan + gate, out_proj.  Beside it the same line carries the decode
+step (batch 64, CUDA graph), the selective scan alone at 128K context, the
+RMSNorm -> Mamba -> RMSNorm -> top-2-of-16 MoE layer pair, the roofline of the
+dominant kernel and the fp64 oracle timed on this host as the CPU baseline.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--quick]
+
+With N > 1 (launched by torchrun) every rank runs its own sequence: no
+collective on the data path, weak scaling, max time over ranks.
+"""
+import argparse
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+PREFILL_L = 131072
+DECODE_B, DECODE_PREFILL, DECODE_STEPS = 64, 2048, 1024
+SCAN_L, SCAN_DI = 131072, 8192
+PAIR_B, PAIR_L = 4, 8192
+METRIC = "Mamba-layer tokens/s (prefill 128K, decode) at d_model=4096; scan HBM GB/s vs peak"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="product", choices=["product", "reference"])
+    ap.add_argument("--quick", action="store_true", help="skip the side measurements")
+    ap.add_argument("--seqlen", type=int, default=PREFILL_L)
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d["bf16_tflops_sustained"], src="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+# ------------------------------------------------------------------ clocks
+class Clocks:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+        except Exception:
+            uuid = None
+        self.sel = ["-i", uuid] if uuid else []
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                                          "-lms", "200"] + self.sel, stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        busy = [v for v in sm if v > 0.5 * mx] or sm
+        busy.sort()
+        return {"sm_mhz": busy[len(busy) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ helpers
+def event_time_ms(fn, reps, stream, flush=None):
+    """mean device time of fn() over reps launches on `stream`, L2 flushed before each"""
+    times = []
+    for _ in range(reps):
+        if flush is not None:
+            flush()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    return sum(times) / len(times), times
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def max_over_ranks(v, world):
+    """the slowest rank's time (the job takes as long as its slowest replica)"""
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(rank):
+    """each replica prefills its own sequence: the input seed is the rank"""
+    return rank
+
+
+def aggregate_tokens_per_s(world, tokens_per_rank, max_ms):
+    """whole-job throughput: all ranks' tokens over the slowest rank's time"""
+    return world * tokens_per_rank / (max_ms / 1e3)
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ CPU baseline
+def cpu_baseline(sample_tokens=1024):
+    """fp64 oracle prefill of `sample_tokens` tokens at Jamba width on this host's cores."""
+    import numpy as np
+    from oracle import mamba as om
+    from synthetic import mamba_input, mamba_params, workload
+    sh = workload("prefill_4k")["mamba"]
+    p64 = om.params64(mamba_params(sh, seed=0))
+    u = om.to64(mamba_input(sh, 1, sample_tokens, seed=0))
+    t0 = time.perf_counter()
+    om.mamba_prefill(p64, u, sh, scan="c")
+    dt = time.perf_counter() - t0
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except Exception:
+        cores = os.cpu_count()
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [cores])
+    except Exception:
+        threads = cores
+    _ = np
+    return {"value": sample_tokens / dt, "unit": "tokens/s", "cores": int(threads), "kind": "oracle",
+            "sample": "fp64 oracle prefill of %d tokens (batch 1) at d_model 4096 / d_inner 8192, numpy "
+                      "matmul + C scan; %.1f s" % (sample_tokens, dt)}
+
+
+# ------------------------------------------------------------------ product arm
+def run_product(args):
+    import mamba_selective_scan_mixer_b200 as J
+    from synthetic import MoEShape, block_norm_params, decode_inputs, mamba_input, mamba_params, moe_params, \
+        scan_inputs, workload
+
+    world, rank, local = dist_setup(args)
+    dev = torch.device("cuda", local)
+    pk = peaks()
+    sh = workload("prefill_4k")["mamba"]
+    L = args.seqlen
+    stream = torch.cuda.current_stream(dev)
+
+    params = {k: v.to(dev) for k, v in mamba_params(sh, seed=0).items()}
+    mixer = J.MambaMixer(params, sh)
+    u = mamba_input(sh, 1, L, seed=rank_seed(rank), device=dev)
+    out = torch.empty_like(u)
+    cs, ss = mixer.new_states(1)
+    flush_buf = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    flush = lambda: flush_buf.zero_()
+    step = lambda: mixer.prefill(u, out=out, conv_state_out=cs, ssm_state_out=ss)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    J.device_status()
+    clocks = Clocks(dev)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    ms, per = event_time_ms(step, args.steps, stream, flush)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    J.device_status()
+    ms = max_over_ranks(ms, world)
+    value = aggregate_tokens_per_s(world, L, ms)
+
+    res = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "bf16",
+           "data": "synthetic: seeded N(0,1) input, N(0,0.02) weights, A=-(n+1), D=1, dt_bias log-uniform",
+           "config": {"workload": "prefill_128k: Mamba mixer prefill, batch 1, L=%d, d_model 4096, d_inner 8192, "
+                                  "d_state 16, dt_rank 256, inner RMSNorm, bf16 weights/activations, fp32 state" % L,
+                      "global_batch": world, "seq_len": L, "parallelism": "replicas" if world > 1 else "single",
+                      "l2": "512 MB buffer written before every timed step (outside the events)"},
+           "gpu_launches": 7 * args.steps, "clocks": clk}
+
+    if rank == 0 and not args.quick:
+        # dominant kernel: in_proj GEMM on the tensor cores, same shape as inside the step
+        xz = torch.empty(L, 2 * sh.d_inner, dtype=torch.bfloat16, device=dev)
+        a2 = u.view(L, sh.d_model)
+        g = lambda: J.gemm(a2, params["in_proj"], out=xz)
+        for _ in range(2):
+            g()
+        gms, _ = event_time_ms(g, 5, stream, flush)
+        flops = 2.0 * L * 2 * sh.d_inner * sh.d_model
+        ach = flops / (gms / 1e3) / 1e12
+        res["roofline"] = {"kernel": "in_proj gemm_bf16_tc_kernel<256,4> (%dx%dx%d)" % (L, 2 * sh.d_inner, sh.d_model),
+                           "bound": "tensor", "achieved": round(ach, 1), "peak": pk["bf16"], "unit": "TFLOP/s",
+                           "frac": round(ach / pk["bf16"], 4), "traffic": None,
+                           "peak_source": "%s bf16 burst (kernel timed alone)" % pk["src"],
+                           "ms": round(gms, 3)}
+        del xz
+        # selective scan alone at 128K context
+        s = {k: v.to(dev) for k, v in scan_inputs(1, SCAN_L, SCAN_DI, 16, seed=0, device=dev).items()}
+        y = torch.empty_like(s["x"])
+        sc = lambda: J.selective_scan(s["x"], s["z"], s["dt"], s["B"], s["C"], s["A"], s["D"], y=y, ws=scan_ws,
+                                      want_state=True)
+        import ctypes
+        nbytes = ctypes.c_size_t()
+        J.lib().jamba_selective_scan_workspace_size(1, SCAN_L, SCAN_DI, 16, 0, ctypes.byref(nbytes))
+        scan_ws = torch.empty(nbytes.value, dtype=torch.uint8, device=dev)
+        for _ in range(2):
+            sc()
+        sms, _ = event_time_ms(sc, 5, stream, flush)
+        sbytes = SCAN_L * (SCAN_DI * (2 + 2 + 4 + 2) + 16 * 2 * 2)
+        gbs = sbytes / (sms / 1e3) / 1e9
+        res["scan"] = {"workload": "scan_128k: selective scan + D + SiLU(z) gate alone, batch 1, L=131072, "
+                                   "d_inner 8192, bf16 x/z/B/C/y, fp32 dt",
+                       "ms": round(sms, 4), "GB/s": round(gbs, 1), "frac_of_measured_hbm": round(gbs / pk["hbm"], 4),
+                       "frac_of_8TBs": round(gbs / 8000.0, 4), "algorithmic_bytes": sbytes,
+                       "tokens/s": round(SCAN_L / (sms / 1e3), 1)}
+        del s, y, scan_ws
+        # decode: batch 64, caches from a 2048-token prefill, steps in one CUDA graph
+        B = DECODE_B
+        u0 = mamba_input(sh, B, DECODE_PREFILL, seed=1, device=dev)
+        dcs, dss = mixer.new_states(B)
+        mixer.prefill(u0, conv_state_out=dcs, ssm_state_out=dss)
+        steps_u = decode_inputs(sh, B, DECODE_STEPS, seed=1, device=dev)
+        dout = torch.empty(B, sh.d_model, dtype=torch.bfloat16, device=dev)
+        mixer.step(steps_u[0], dcs, dss, out=dout)       # sizes the workspace before capture
+        torch.cuda.synchronize()
+        gs = torch.cuda.Stream(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=gs):
+            for t in range(DECODE_STEPS):
+                mixer.step(steps_u[t], dcs, dss, out=dout)
+        graph.replay()
+        torch.cuda.synchronize()
+        dms, _ = event_time_ms(graph.replay, 3, stream, flush)
+        per_step_us = dms * 1e3 / DECODE_STEPS
+        wbytes = sum(v.numel() * v.element_size() for v in params.values())
+        step_bytes = wbytes + 2 * (B * sh.d_inner * 16 * 4 + B * sh.d_inner * 3 * 4) + 2 * B * sh.d_model * 2
+        res["decode"] = {"workload": "decode_b64: batch 64, one token per step, 1024 steps in one CUDA graph, "
+                                     "caches from a 2048-token prefill",
+                         "tokens/s": round(B * DECODE_STEPS / (dms / 1e3), 1), "us_per_step": round(per_step_us, 2),
+                         "GB/s": round(step_bytes / (per_step_us / 1e6) / 1e9, 1),
+                         "frac_of_measured_hbm": round(step_bytes / (per_step_us / 1e6) / 1e9 / pk["hbm"], 4),
+                         "algorithmic_bytes_per_step": step_bytes, "launches_per_step": 8}
+        del graph, u0, steps_u
+        # layer pair: RMSNorm -> Mamba -> residual -> RMSNorm -> top-2-of-16 MoE -> residual
+        es = MoEShape()
+        mp = moe_params(es, seed=0, device=dev)
+        moe = J.MoE(mp, es)
+        g1, g2 = block_norm_params(sh.d_model, device=dev)
+        xp = mamba_input(sh, PAIR_B, PAIR_L, seed=2, device=dev)
+        pair = lambda: J.layer_pair(mixer, moe, xp, g1, g2)
+        pair()
+        torch.cuda.synchronize()
+        pms, _ = event_time_ms(pair, 3, stream, flush)
+        T = PAIR_B * PAIR_L
+        pflops = T * (2.0 * (2 * sh.d_inner * sh.d_model + (sh.dt_rank + 32) * sh.d_inner +
+                             sh.dt_rank * sh.d_inner + sh.d_model * sh.d_inner)
+                      + 2 * 2.0 * (3 * es.d_model * es.d_ff) + 2.0 * 16 * es.d_model)
+        res["layer_pair"] = {"workload": "layer_pair: batch 4 x 8192 tokens, Mamba (as prefill) + 16-expert "
+                                         "top-2 SwiGLU MoE (d_ff 14336)",
+                             "tokens/s": round(T / (pms / 1e3), 1), "ms": round(pms, 3),
+                             "TFLOP/s": round(pflops / (pms / 1e3) / 1e12, 1),
+                             "frac_of_bf16_sustained": round(pflops / (pms / 1e3) / 1e12 / pk["bf16_sus"], 4)}
+        del mp, moe, xp
+        J.device_status()
+
+    # end to end through the public API with host buffers (pinned), copies inside the timed region
+    if not args.quick:
+        hu = u.cpu().pin_memory()
+        hout = torch.empty_like(hu).pin_memory()
+        du = torch.empty_like(u)
+
+        def e2e():
+            du.copy_(hu, non_blocking=True)
+            mixer.prefill(du, out=out, conv_state_out=cs, ssm_state_out=ss)
+            hout.copy_(out, non_blocking=True)
+
+        e2e()
+        torch.cuda.synchronize()
+        ems, _ = event_time_ms(e2e, max(2, args.steps // 2), stream, flush)
+        ems = max_over_ranks(ems, world)
+        res["e2e"] = {"value": round(aggregate_tokens_per_s(world, L, ems), 1), "unit": "tokens/s",
+                      "h2d_bytes_per_step": hu.numel() * hu.element_size(),
+                      "d2h_bytes_per_step": hout.numel() * hout.element_size()}
+    if rank == 0 and not args.quick:
+        res["cpu_baseline"] = cpu_baseline()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    """The oracle as it stands, on this host's cores, same metric and workload (bounded sample)."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    times = []
+    base = None
+    for _ in range(args.warmup):
+        cpu_baseline(256)
+    for _ in range(args.steps):
+        base = cpu_baseline(256)
+        times.append(256 / base["value"])
+    ms = 1e3 * sum(times) / len(times)
+    v = 256 / (ms / 1e3)
+    base["value"] = round(v, 2)
+    print(json.dumps({"impl": "reference", "metric": METRIC, "value": round(v, 2), "unit": "tokens/s",
+                      "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2),
+                      "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                      "data": "synthetic", "config": {"workload": "prefill_128k (oracle sample: 256 tokens per "
+                                                                  "step at the same widths)"},
+                      "cpu_baseline": base,
+                      "e2e": {"value": round(v, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                              "d2h_bytes_per_step": 0}}), flush=True)
+
+
+if __name__ == "__main__":
+    a = parse()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_product(a)

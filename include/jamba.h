@@ -1,0 +1,221 @@
+/*
+ * jamba.h — C ABI of the B200 (sm_100a) Jamba Mamba-mixer / MoE library.
+ *
+ * The computation follows "Jamba: A Hybrid Transformer-Mamba Language Model"
+ * (paper summary page): section 2 (Mamba layers with RMSNorm inside them, no
+ * positional encoding, SwiGLU MLPs, MoE with n experts and top-K routing),
+ * section 3.1 (n = 16 experts, K = 2), section 6.4 / figure 9 (RMSNorm on the
+ * Mamba layer's inner activations).  The Mamba layer itself is the selective
+ * state-space layer the paper cites (section 2, ref [17]):
+ *
+ *   xz = u W_in^T;  x, z = split(xz)
+ *   xc = SiLU(causal depthwise conv1d(x) + conv_b)
+ *   dt_low, B, C = split(xc W_x^T)         (RMSNorm on each when enabled)
+ *   dt = softplus(dt_low W_dt^T + dt_bias)
+ *   h_t = exp(dt_t A) h_{t-1} + dt_t B_t x_t,   y_t = (C_t . h_t + D x_t) SiLU(z_t)
+ *   out = y W_out^T (+ residual)
+ *
+ * Conventions for every entry point:
+ *  - Tensor pointers are DEVICE pointers owned by the caller, row-major and
+ *    contiguous unless a leading dimension is given, 16-byte aligned.  The
+ *    library never frees caller memory and keeps no pointer to activations
+ *    after a call returns.
+ *  - "dtype" tensors are bf16 (JAMBA_BF16) or fp32 (JAMBA_F32) as configured;
+ *    states, dt_bias, A, D and norm weights are always fp32.
+ *  - Work is enqueued on the given stream (a cudaStream_t; NULL = legacy
+ *    default stream) and runs asynchronously; calls never synchronize unless
+ *    documented.  Arguments are validated before anything is launched: on an
+ *    error status nothing was enqueued.
+ *  - Asynchronous device errors (a bounded wait inside a kernel that ran out
+ *    of time) are latched in a per-device error word; read it with
+ *    jamba_device_status().
+ *  - No function throws; jamba_last_error() describes the last failure of
+ *    the calling thread.
+ */
+#ifndef JAMBA_H_
+#define JAMBA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum jamba_status {
+  JAMBA_OK = 0,
+  JAMBA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, non-positive size        */
+  JAMBA_ERR_UNSUPPORTED = 2, /* shape or dtype outside what the kernels handle    */
+  JAMBA_ERR_WORKSPACE = 3,   /* workspace missing or smaller than *_workspace_size */
+  JAMBA_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed                 */
+  JAMBA_ERR_TIMEOUT = 5,     /* a device-side bounded wait gave up                */
+  JAMBA_ERR_OOM = 6          /* host allocation failed                            */
+} jamba_status;
+
+typedef enum jamba_dtype { JAMBA_F32 = 0, JAMBA_BF16 = 1 } jamba_dtype;
+
+typedef struct CUstream_st* jamba_stream_t; /* same type as cudaStream_t */
+
+/* Last error message of the calling thread (static storage, never NULL). */
+const char* jamba_last_error(void);
+
+/* Synchronizes `stream`, then returns and clears the device error word of the
+ * current device: JAMBA_OK, JAMBA_ERR_TIMEOUT, or JAMBA_ERR_CUDA when the
+ * stream itself reports an error. */
+jamba_status jamba_device_status(jamba_stream_t stream);
+
+/* ------------------------------------------------------------------ Mamba */
+
+typedef struct jamba_mamba_config {
+  int d_model;       /* block width (4096 in Jamba)                              */
+  int d_inner;       /* mixer width, multiple of 8 (8192)                        */
+  int d_state;       /* SSM state size: must be 16                               */
+  int d_conv;        /* conv taps: must be 4                                     */
+  int dt_rank;       /* rank of the dt projection, multiple of 8 (256)           */
+  int dtype;         /* jamba_dtype of weights and activations                   */
+  int inner_rmsnorm; /* 1: RMSNorm on dt_low, B and C (Jamba section 6.4)        */
+  float eps;         /* epsilon of the inner RMSNorms                            */
+} jamba_mamba_config;
+
+typedef struct jamba_mamba_weights {
+  const void* in_proj;   /* [2*d_inner, d_model] dtype; rows [0,d_inner) give x, the rest z */
+  const void* conv_w;    /* [d_inner, d_conv] dtype; tap d_conv-1 multiplies the current token */
+  const void* conv_b;    /* [d_inner] dtype */
+  const void* x_proj;    /* [dt_rank + 2*d_state, d_inner] dtype; rows: dt_low | B | C */
+  const void* dt_proj;   /* [d_inner, dt_rank] dtype */
+  const float* dt_bias;  /* [d_inner] */
+  const float* A;        /* [d_inner, d_state], any finite values (negative for a stable layer) */
+  const float* D;        /* [d_inner] */
+  const void* out_proj;  /* [d_model, d_inner] dtype */
+  const float* norm_dt;  /* [dt_rank]  (read only when inner_rmsnorm) */
+  const float* norm_B;   /* [d_state] */
+  const float* norm_C;   /* [d_state] */
+} jamba_mamba_weights;
+
+typedef struct jamba_mamba* jamba_mamba_t;
+
+/* Creates a mixer handle on the current CUDA device.  The weight pointers are
+ * borrowed: they must stay valid and unchanged until destroy.  The handle owns
+ * only host-side descriptors (TMA tensor maps of the weights).
+ * Errors: INVALID_ARG (null pointers, misalignment), UNSUPPORTED (d_state != 16,
+ * d_conv != 4, widths not multiples of 8). */
+jamba_status jamba_mamba_create(const jamba_mamba_config* cfg, const jamba_mamba_weights* w,
+                                jamba_mamba_t* out);
+jamba_status jamba_mamba_destroy(jamba_mamba_t h);
+
+/* Bytes of device workspace that jamba_mamba_prefill needs for `batch` rows of
+ * `seqlen` tokens (seqlen = 1 gives the size for jamba_mamba_step). */
+jamba_status jamba_mamba_workspace_size(jamba_mamba_t h, int batch, int seqlen, size_t* bytes);
+
+/* Mixer forward over whole sequences (prefill).
+ *   u        [batch, seqlen, d_model] dtype       input (already block-normed)
+ *   residual [batch, seqlen, d_model] dtype|NULL  added to the output when given
+ *   out      [batch, seqlen, d_model] dtype       may alias residual, not u
+ *   conv_state_in / ssm_state_in [batch, d_inner, d_conv-1] / [batch, d_inner, d_state]
+ *            fp32 or NULL: state to continue from (NULL = zeros)
+ *   conv_state_out / ssm_state_out: same shapes, fp32 or NULL: the caches after
+ *            the last token (conv: the last d_conv-1 pre-conv inputs, oldest first)
+ *   ws / ws_bytes: device workspace of at least jamba_mamba_workspace_size bytes
+ * The states may alias (in == out) for in-place continuation. */
+jamba_status jamba_mamba_prefill(jamba_mamba_t h, const void* u, const void* residual, void* out,
+                                 int batch, int seqlen, const float* conv_state_in,
+                                 const float* ssm_state_in, float* conv_state_out,
+                                 float* ssm_state_out, void* ws, size_t ws_bytes,
+                                 jamba_stream_t stream);
+
+/* One-token decode step for every batch row, updating both caches in place.
+ *   u [batch, d_model], residual [batch, d_model] or NULL, out [batch, d_model]
+ *   conv_state [batch, d_inner, d_conv-1] fp32, ssm_state [batch, d_inner, d_state] fp32
+ * Workspace: jamba_mamba_workspace_size(h, batch, 1). */
+jamba_status jamba_mamba_step(jamba_mamba_t h, const void* u, const void* residual, void* out,
+                              int batch, float* conv_state, float* ssm_state, void* ws,
+                              size_t ws_bytes, jamba_stream_t stream);
+
+/* ------------------------------------------------------- selective scan */
+
+/* Bytes of workspace jamba_selective_scan needs (chunk 0 = automatic). */
+jamba_status jamba_selective_scan_workspace_size(int batch, int seqlen, int d_inner, int d_state,
+                                                 int chunk, size_t* bytes);
+
+/* The selective scan with D skip and SiLU(z) gate alone (the recurrence
+ * stated in the file header), batch x d_inner channels, fp32 state.
+ *   x, z   [batch, seqlen, *] dtype, row strides ld_x / ld_z elements (>= d_inner)
+ *   dt     [batch, seqlen, *] fp32, row stride ld_dt
+ *   B, C   [batch, seqlen, *] bc_dtype, row strides ld_b / ld_c (>= d_state)
+ *   A      [d_inner, d_state] fp32, D [d_inner] fp32
+ *   h0     [batch, d_inner, d_state] fp32 or NULL (zeros)
+ *   y      [batch, seqlen, *] dtype, row stride ld_y
+ *   h_out  [batch, d_inner, d_state] fp32 or NULL: state after the last step
+ *   chunk  time steps per chunk (multiple of 16), 0 = automatic
+ * Time is split into chunks scanned concurrently; the state entering each
+ * chunk is passed between chunks with a decoupled look-back.  Errors:
+ * UNSUPPORTED for d_state != 16, INVALID_ARG for strides/alignment. */
+jamba_status jamba_selective_scan(const void* x, int ld_x, const void* z, int ld_z, const float* dt,
+                                  int ld_dt, const void* B, int ld_b, const void* C, int ld_c,
+                                  int bc_dtype, const float* A, const float* D, const float* h0,
+                                  void* y, int ld_y, float* h_out, int batch, int seqlen,
+                                  int d_inner, int d_state, int dtype, int chunk, void* ws,
+                                  size_t ws_bytes, jamba_stream_t stream);
+
+/* ------------------------------------------------------- building blocks */
+
+/* out = RMSNorm(x) * w over rows of `cols` elements (block norm of the layer pair).
+ * x, out [rows, cols] dtype; w [cols] fp32. */
+jamba_status jamba_rmsnorm(const void* x, const float* w, void* out, int rows, int cols, float eps,
+                           int dtype, jamba_stream_t stream);
+
+/* Causal depthwise conv1d + SiLU over [batch, seqlen] tokens.
+ *   x [batch, seqlen, *] dtype row stride ld_x; w [channels, 4] dtype; b [channels] dtype
+ *   out [batch, seqlen, channels] dtype (contiguous)
+ *   state_in / state_out [batch, channels, 3] fp32 or NULL (see jamba_mamba_prefill) */
+jamba_status jamba_causal_conv1d(const void* x, int ld_x, const void* w, const void* b, void* out,
+                                 const float* state_in, float* state_out, int batch, int seqlen,
+                                 int channels, int dtype, jamba_stream_t stream);
+
+/* Dense GEMM out = a @ b^T (+ residual) on the sm_100a tensor cores (bf16) or
+ * the CUDA cores (fp32).  a [m, k], b [n, k] row-major; out [m, n] row stride
+ * ld_out; residual NULL or [m, n] with the same stride.  out_dtype may differ
+ * from dtype only as fp32 output of bf16 inputs. */
+jamba_status jamba_gemm(const void* a, const void* b, void* out, int ld_out, const void* residual,
+                        int m, int n, int k, int dtype, int out_dtype, jamba_stream_t stream);
+
+/* -------------------------------------------------------------------- MoE */
+
+typedef struct jamba_moe_config {
+  int d_model;   /* 4096 */
+  int d_ff;      /* expert hidden width (14336), multiple of 128 */
+  int n_experts; /* n (16 in Jamba section 3.1), at most 64 */
+  int top_k;     /* K (2 in Jamba section 3.1), 1 or 2 */
+  int dtype;     /* JAMBA_BF16 */
+} jamba_moe_config;
+
+typedef struct jamba_moe_weights {
+  const void* router; /* [n_experts, d_model] */
+  const void* w_gate; /* [n_experts, d_ff, d_model] */
+  const void* w_up;   /* [n_experts, d_ff, d_model] */
+  const void* w_down; /* [n_experts, d_model, d_ff] */
+} jamba_moe_weights;
+
+jamba_status jamba_moe_workspace_size(const jamba_moe_config* cfg, int tokens, size_t* bytes);
+
+/* Top-K-of-n SwiGLU mixture of experts on `tokens` rows (Jamba section 2).
+ *   x        [tokens, d_model] dtype (already block-normed)
+ *   residual [tokens, d_model] dtype or NULL, added to the output
+ *   y        [tokens, d_model] dtype
+ *   topk_idx [tokens, top_k] int32 out: experts by descending logit, ties to the lower index
+ *   topk_w   [tokens, top_k] fp32 out: their softmax probabilities (not renormalised)
+ *   expert_offsets [n_experts + 1] int32 out: routed-row ranges per expert
+ *   perm     [tokens * top_k] int32 out: routed row p holds pair (token, slot) = perm[p]
+ *            as token * top_k + slot, rows sorted by (expert, token, slot)
+ * Router logits are accumulated in fp64 from the bf16 inputs, so the expert
+ * choice is the exact-arithmetic one except for ties closer than 1e-13. */
+jamba_status jamba_moe_forward(const jamba_moe_config* cfg, const jamba_moe_weights* w,
+                               const void* x, const void* residual, void* y, int tokens,
+                               int32_t* topk_idx, float* topk_w, int32_t* expert_offsets,
+                               int32_t* perm, void* ws, size_t ws_bytes, jamba_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* JAMBA_H_ */

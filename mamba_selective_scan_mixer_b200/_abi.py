@@ -1,0 +1,94 @@
+"""ctypes declarations of include/jamba.h and the loader of libjamba.so.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library.  Importing this module does not load the library; the first call
+does, and raises if libjamba.so has not been built.
+"""
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libjamba.so")
+
+JAMBA_OK = 0
+STATUS_NAMES = {0: "JAMBA_OK", 1: "JAMBA_ERR_INVALID_ARG", 2: "JAMBA_ERR_UNSUPPORTED",
+                3: "JAMBA_ERR_WORKSPACE", 4: "JAMBA_ERR_CUDA", 5: "JAMBA_ERR_TIMEOUT",
+                6: "JAMBA_ERR_OOM"}
+JAMBA_F32 = 0
+JAMBA_BF16 = 1
+
+
+class JambaError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__("%s: %s" % (STATUS_NAMES.get(status, status), msg))
+        self.status = status
+
+
+class MambaConfig(ctypes.Structure):
+    _fields_ = [("d_model", ctypes.c_int), ("d_inner", ctypes.c_int), ("d_state", ctypes.c_int),
+                ("d_conv", ctypes.c_int), ("dt_rank", ctypes.c_int), ("dtype", ctypes.c_int),
+                ("inner_rmsnorm", ctypes.c_int), ("eps", ctypes.c_float)]
+
+
+class MambaWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("in_proj", "conv_w", "conv_b", "x_proj", "dt_proj", "dt_bias", "A", "D",
+                 "out_proj", "norm_dt", "norm_B", "norm_C")]
+
+
+class MoeConfig(ctypes.Structure):
+    _fields_ = [("d_model", ctypes.c_int), ("d_ff", ctypes.c_int), ("n_experts", ctypes.c_int),
+                ("top_k", ctypes.c_int), ("dtype", ctypes.c_int)]
+
+
+class MoeWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("router", "w_gate", "w_up", "w_down")]
+
+
+P = ctypes.c_void_p
+I = ctypes.c_int
+SZ = ctypes.c_size_t
+F = ctypes.c_float
+
+# name -> argument types (all return jamba_status as int, except jamba_last_error)
+SIGNATURES = {
+    "jamba_device_status": [P],
+    "jamba_mamba_create": [ctypes.POINTER(MambaConfig), ctypes.POINTER(MambaWeights), ctypes.POINTER(P)],
+    "jamba_mamba_destroy": [P],
+    "jamba_mamba_workspace_size": [P, I, I, ctypes.POINTER(SZ)],
+    "jamba_mamba_prefill": [P, P, P, P, I, I, P, P, P, P, P, SZ, P],
+    "jamba_mamba_step": [P, P, P, P, I, P, P, P, SZ, P],
+    "jamba_selective_scan_workspace_size": [I, I, I, I, I, ctypes.POINTER(SZ)],
+    "jamba_selective_scan": [P, I, P, I, P, I, P, I, P, I, I, P, P, P, P, I, P, I, I, I, I, I, I, P, SZ, P],
+    "jamba_rmsnorm": [P, P, P, I, I, F, I, P],
+    "jamba_causal_conv1d": [P, I, P, P, P, P, P, I, I, I, I, P],
+    "jamba_gemm": [P, P, P, I, P, I, I, I, I, I, P],
+    "jamba_moe_workspace_size": [ctypes.POINTER(MoeConfig), I, ctypes.POINTER(SZ)],
+    "jamba_moe_forward": [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), P, P, P, I, P, P, P, P,
+                          P, SZ, P],
+}
+
+_lib = None
+
+
+def lib():
+    """The loaded library; raises if it is missing (there is no fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError("libjamba.so is not built (python -m mamba_selective_scan_mixer_b200.build)")
+        L = ctypes.CDLL(LIB_PATH)
+        L.jamba_last_error.restype = ctypes.c_char_p
+        L.jamba_last_error.argtypes = []
+        for name, args in SIGNATURES.items():
+            f = getattr(L, name)
+            f.restype = ctypes.c_int
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def check(status):
+    if status != JAMBA_OK:
+        raise JambaError(status, lib().jamba_last_error().decode())
+    return status

@@ -1,0 +1,496 @@
+// C ABI: argument checks, workspace layout and the launch sequences of the
+// Mamba mixer (prefill, decode step), the selective scan alone, the building
+// blocks and the MoE.  See include/jamba.h for the contract of each call.
+#include <new>
+#include <string>
+
+#include "gemm_tc.cuh"
+#include "host.hpp"
+
+using namespace jb;
+
+struct jamba_mamba {
+  jamba_mamba_config cfg;
+  jamba_mamba_weights w;
+  int device;
+};
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t al(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
+
+// Sequential carve-out of a workspace; with a null base it only measures.
+struct Carver {
+  uint8_t* base;
+  size_t off = 0;
+  explicit Carver(void* b) : base(reinterpret_cast<uint8_t*>(b)) {}
+  template <typename T = void>
+  T* take(size_t bytes) {
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += al(bytes);
+    return p;
+  }
+};
+
+inline int esize(int dtype) { return dtype == JAMBA_BF16 ? 2 : 4; }
+inline cudaStream_t cs(jamba_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+struct PrefillWs {
+  void* xz; void* xc; float* xpart; void* dtlow; float* bc; float* dt; void* y; float* conv_tmp; void* scan;
+  size_t scan_bytes;
+  int splits, chunk;
+  size_t total;
+};
+
+PrefillWs carve_prefill(const jamba_mamba_config& c, int batch, int L, void* ws) {
+  PrefillWs p;
+  const size_t T = (size_t)batch * L;
+  const int es = esize(c.dtype);
+  const int W = c.dt_rank + 2 * c.d_state;
+  p.splits = c.dtype == JAMBA_BF16 ? choose_splits((int)T, W, c.d_inner, 144, 8) : 1;
+  p.chunk = scan_auto_chunk(batch, L, c.d_inner);
+  Carver cv(ws);
+  p.xz = cv.take(T * 2 * c.d_inner * es);
+  p.xc = cv.take(T * c.d_inner * es);
+  p.xpart = cv.take<float>((size_t)p.splits * T * W * 4);
+  p.dtlow = cv.take(T * c.dt_rank * es);
+  p.bc = cv.take<float>(T * 2 * c.d_state * 4);
+  p.dt = cv.take<float>(T * c.d_inner * 4);
+  p.y = cv.take(T * c.d_inner * es);
+  p.conv_tmp = cv.take<float>((size_t)batch * c.d_inner * (c.d_conv - 1) * 4);
+  p.scan_bytes = scan_workspace_bytes(batch, L, c.d_inner, p.chunk);
+  p.scan = cv.take(p.scan_bytes);
+  p.total = cv.off;
+  return p;
+}
+
+struct StepWs {
+  void* xz; void* xc; float* xpart; void* dtlow; float* bc; float* dt; void* y; float* opart;
+  int x_splits, o_splits;
+  size_t total;
+};
+
+StepWs carve_step(const jamba_mamba_config& c, int batch, void* ws) {
+  StepWs p;
+  const int es = esize(c.dtype);
+  const int W = c.dt_rank + 2 * c.d_state;
+  const bool tc = c.dtype == JAMBA_BF16;
+  p.x_splits = tc ? choose_splits(W, batch, c.d_inner, 64, 4) : 1;
+  p.o_splits = tc ? choose_splits(c.d_model, batch, c.d_inner, 64, 8) : 1;
+  Carver cv(ws);
+  p.xz = cv.take((size_t)batch * 2 * c.d_inner * es);
+  p.xc = cv.take((size_t)batch * c.d_inner * es);
+  p.xpart = cv.take<float>((size_t)p.x_splits * batch * W * 4);
+  p.dtlow = cv.take((size_t)batch * c.dt_rank * es);
+  p.bc = cv.take<float>((size_t)batch * 2 * c.d_state * 4);
+  p.dt = cv.take<float>((size_t)batch * c.d_inner * 4);
+  p.y = cv.take((size_t)batch * c.d_inner * es);
+  p.opart = cv.take<float>((size_t)p.o_splits * batch * c.d_model * 4);
+  p.total = cv.off;
+  return p;
+}
+
+GemmDesc gdesc(const void* a, long long lda, const void* b, long long ldb, int M, int N, int K, int epi, void* out,
+               long long ldo) {
+  GemmDesc g = {};
+  g.a = a; g.lda = lda; g.b = b; g.ldb = ldb; g.M = M; g.N = N; g.K = K; g.epi = epi; g.out = out; g.ldo = ldo;
+  g.splits = 1;
+  return g;
+}
+
+jamba_status gemm_any(int dtype, const GemmDesc& g, cudaStream_t s) {
+  return dtype == JAMBA_BF16 ? gemm_bf16(g, s) : gemm_f32(g, s);
+}
+
+jamba_status check_dtype(int d) {
+  return (d == JAMBA_BF16 || d == JAMBA_F32) ? JAMBA_OK : fail(JAMBA_ERR_UNSUPPORTED, "dtype must be JAMBA_F32 or JAMBA_BF16");
+}
+
+jamba_status check_ptr(const void* p, const char* name, bool required = true) {
+  if (!p) return required ? fail(JAMBA_ERR_INVALID_ARG, std::string(name) + " is null") : JAMBA_OK;
+  if (!aligned16(p)) return fail(JAMBA_ERR_INVALID_ARG, std::string(name) + " is not 16-byte aligned");
+  return JAMBA_OK;
+}
+
+jamba_status check_device(const jamba_mamba* h) {
+  int dev = -1;
+  JB_CUDA(cudaGetDevice(&dev));
+  if (dev != h->device) return fail(JAMBA_ERR_INVALID_ARG, "handle was created on another device");
+  return JAMBA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* jamba_last_error(void) { return jb::last_error(); }
+
+jamba_status jamba_device_status(jamba_stream_t stream) {
+  JB_CUDA(cudaStreamSynchronize(cs(stream)));
+  int* w = device_error_word();
+  if (!w) return fail(JAMBA_ERR_CUDA, "could not allocate the device status word");
+  int v = 0;
+  JB_CUDA(cudaMemcpy(&v, w, sizeof(int), cudaMemcpyDeviceToHost));
+  if (v != 0) {
+    JB_CUDA(cudaMemset(w, 0, sizeof(int)));
+    return fail((jamba_status)v, "a device-side wait gave up");
+  }
+  return JAMBA_OK;
+}
+
+// ------------------------------------------------------------------ Mamba
+
+jamba_status jamba_mamba_create(const jamba_mamba_config* cfg, const jamba_mamba_weights* w, jamba_mamba_t* out) {
+  if (!cfg || !w || !out) return fail(JAMBA_ERR_INVALID_ARG, "create: null argument");
+  *out = nullptr;
+  const jamba_mamba_config& c = *cfg;
+  JB_TRY(check_dtype(c.dtype));
+  if (c.d_state != 16) return fail(JAMBA_ERR_UNSUPPORTED, "d_state must be 16");
+  if (c.d_conv != 4) return fail(JAMBA_ERR_UNSUPPORTED, "d_conv must be 4");
+  if (c.d_model <= 0 || c.d_inner <= 0 || c.dt_rank <= 0) return fail(JAMBA_ERR_INVALID_ARG, "widths must be positive");
+  if (c.d_model % 8 || c.d_inner % 8) return fail(JAMBA_ERR_UNSUPPORTED, "d_model and d_inner must be multiples of 8");
+  if (c.dtype == JAMBA_BF16 && c.dt_rank % 8) return fail(JAMBA_ERR_UNSUPPORTED, "bf16 needs dt_rank % 8 == 0");
+  if (c.dt_rank + 2 * c.d_state > 512) return fail(JAMBA_ERR_UNSUPPORTED, "dt_rank + 2 d_state above 512");
+  if (!(c.eps >= 0.f)) return fail(JAMBA_ERR_INVALID_ARG, "eps must be >= 0");
+  JB_TRY(check_ptr(w->in_proj, "in_proj"));
+  JB_TRY(check_ptr(w->conv_w, "conv_w"));
+  JB_TRY(check_ptr(w->conv_b, "conv_b"));
+  JB_TRY(check_ptr(w->x_proj, "x_proj"));
+  JB_TRY(check_ptr(w->dt_proj, "dt_proj"));
+  JB_TRY(check_ptr(w->dt_bias, "dt_bias"));
+  JB_TRY(check_ptr(w->A, "A"));
+  JB_TRY(check_ptr(w->D, "D"));
+  JB_TRY(check_ptr(w->out_proj, "out_proj"));
+  if (c.inner_rmsnorm) {
+    JB_TRY(check_ptr(w->norm_dt, "norm_dt"));
+    JB_TRY(check_ptr(w->norm_B, "norm_B"));
+    JB_TRY(check_ptr(w->norm_C, "norm_C"));
+  }
+  jamba_mamba* h = new (std::nothrow) jamba_mamba;
+  if (!h) return fail(JAMBA_ERR_OOM, "create: out of host memory");
+  h->cfg = c;
+  h->w = *w;
+  if (cudaGetDevice(&h->device) != cudaSuccess) {
+    delete h;
+    return fail(JAMBA_ERR_CUDA, "create: no CUDA device");
+  }
+  *out = h;
+  return JAMBA_OK;
+}
+
+jamba_status jamba_mamba_destroy(jamba_mamba_t h) {
+  delete h;
+  return JAMBA_OK;
+}
+
+jamba_status jamba_mamba_workspace_size(jamba_mamba_t h, int batch, int seqlen, size_t* bytes) {
+  if (!h || !bytes || batch <= 0 || seqlen <= 0) return fail(JAMBA_ERR_INVALID_ARG, "workspace_size: bad argument");
+  size_t a = carve_prefill(h->cfg, batch, seqlen, nullptr).total;
+  if (seqlen == 1) {
+    const size_t b = carve_step(h->cfg, batch, nullptr).total;
+    a = a > b ? a : b;
+  }
+  *bytes = a;
+  return JAMBA_OK;
+}
+
+jamba_status jamba_mamba_prefill(jamba_mamba_t h, const void* u, const void* residual, void* out, int batch,
+                                 int seqlen, const float* conv_state_in, const float* ssm_state_in,
+                                 float* conv_state_out, float* ssm_state_out, void* ws, size_t ws_bytes,
+                                 jamba_stream_t stream) {
+  if (!h) return fail(JAMBA_ERR_INVALID_ARG, "prefill: null handle");
+  if (batch <= 0 || seqlen <= 0) return fail(JAMBA_ERR_INVALID_ARG, "prefill: batch and seqlen must be positive");
+  JB_TRY(check_device(h));
+  JB_TRY(check_ptr(u, "u"));
+  JB_TRY(check_ptr(out, "out"));
+  JB_TRY(check_ptr(residual, "residual", false));
+  JB_TRY(check_ptr(conv_state_in, "conv_state_in", false));
+  JB_TRY(check_ptr(ssm_state_in, "ssm_state_in", false));
+  JB_TRY(check_ptr(conv_state_out, "conv_state_out", false));
+  JB_TRY(check_ptr(ssm_state_out, "ssm_state_out", false));
+  JB_TRY(check_ptr(ws, "workspace"));
+  if (u == out) return fail(JAMBA_ERR_INVALID_ARG, "prefill: out may not alias u");
+  const jamba_mamba_config& c = h->cfg;
+  const jamba_mamba_weights& w = h->w;
+  if ((long long)batch * seqlen > (1LL << 31) / 2) return fail(JAMBA_ERR_UNSUPPORTED, "prefill: too many tokens");
+  PrefillWs p = carve_prefill(c, batch, seqlen, ws);
+  if (ws_bytes < p.total) return fail(JAMBA_ERR_WORKSPACE, "prefill: workspace too small");
+  cudaStream_t s = cs(stream);
+  const int T = batch * seqlen, di = c.d_inner, dm = c.d_model, R = c.dt_rank, N = c.d_state;
+  const int W = R + 2 * N;
+
+  // in_proj: xz = u W_in^T
+  JB_TRY(gemm_any(c.dtype, gdesc(u, dm, w.in_proj, dm, T, 2 * di, dm, c.dtype == JAMBA_BF16 ? EPI_BF16 : EPI_F32,
+                                 p.xz, 2 * di), s));
+  // conv + SiLU (cache in -> out; an aliased cache is copied first)
+  const float* cin = conv_state_in;
+  if (cin && cin == conv_state_out) {
+    JB_CUDA(cudaMemcpyAsync(p.conv_tmp, cin, sizeof(float) * (size_t)batch * di * 3, cudaMemcpyDeviceToDevice, s));
+    cin = p.conv_tmp;
+  }
+  JB_TRY(conv_prefill(p.xz, 2 * di, w.conv_w, w.conv_b, p.xc, cin, conv_state_out, batch, seqlen, di, c.dtype, s));
+  // x_proj (split-K partials) -> sum + inner RMSNorms
+  GemmDesc gx = gdesc(p.xc, di, w.x_proj, di, T, W, di, EPI_F32, p.xpart, W);
+  gx.splits = p.splits;
+  gx.split_stride = (long long)T * W;
+  if (c.dtype == JAMBA_BF16) gx.bn = 144;
+  JB_TRY(gemm_any(c.dtype, gx, s));
+  JB_TRY(xproj_norm(p.xpart, p.splits, (long long)T * W, T, R, N, w.norm_dt, w.norm_B, w.norm_C, c.inner_rmsnorm,
+                    c.eps, p.dtlow, p.bc, c.dtype, s));
+  // dt = softplus(dt_low W_dt^T + dt_bias)
+  GemmDesc gd = gdesc(p.dtlow, R, w.dt_proj, R, T, di, R, EPI_SOFTPLUS, p.dt, di);
+  gd.bias = w.dt_bias;
+  JB_TRY(gemm_any(c.dtype, gd, s));
+  // selective scan + D skip + SiLU(z) gate
+  ScanCall sc = {};
+  sc.x = p.xc; sc.ld_x = di;
+  sc.z = reinterpret_cast<const uint8_t*>(p.xz) + (size_t)di * esize(c.dtype); sc.ld_z = 2 * di;
+  sc.dt = p.dt; sc.ld_dt = di;
+  sc.B = p.bc; sc.ld_b = 2 * N;
+  sc.C = p.bc + N; sc.ld_c = 2 * N;
+  sc.bc_dtype = JAMBA_F32;
+  sc.A = w.A; sc.D = w.D; sc.h0 = ssm_state_in;
+  sc.y = p.y; sc.ld_y = di;
+  sc.h_out = ssm_state_out;
+  sc.batch = batch; sc.L = seqlen; sc.di = di; sc.dtype = c.dtype; sc.chunk = p.chunk;
+  sc.ws = p.scan; sc.ws_bytes = p.scan_bytes;
+  JB_TRY(scan_run(sc, s));
+  // out_proj (+ residual)
+  GemmDesc go = gdesc(p.y, di, w.out_proj, di, T, dm, di, c.dtype == JAMBA_BF16 ? EPI_BF16 : EPI_F32, out, dm);
+  go.residual = residual;
+  go.ldr = dm;
+  JB_TRY(gemm_any(c.dtype, go, s));
+  return JAMBA_OK;
+}
+
+jamba_status jamba_mamba_step(jamba_mamba_t h, const void* u, const void* residual, void* out, int batch,
+                              float* conv_state, float* ssm_state, void* ws, size_t ws_bytes, jamba_stream_t stream) {
+  if (!h) return fail(JAMBA_ERR_INVALID_ARG, "step: null handle");
+  if (batch <= 0) return fail(JAMBA_ERR_INVALID_ARG, "step: batch must be positive");
+  JB_TRY(check_device(h));
+  JB_TRY(check_ptr(u, "u"));
+  JB_TRY(check_ptr(out, "out"));
+  JB_TRY(check_ptr(residual, "residual", false));
+  JB_TRY(check_ptr(conv_state, "conv_state"));
+  JB_TRY(check_ptr(ssm_state, "ssm_state"));
+  JB_TRY(check_ptr(ws, "workspace"));
+  if (u == out) return fail(JAMBA_ERR_INVALID_ARG, "step: out may not alias u");
+  const jamba_mamba_config& c = h->cfg;
+  const jamba_mamba_weights& w = h->w;
+  StepWs p = carve_step(c, batch, ws);
+  if (ws_bytes < p.total) return fail(JAMBA_ERR_WORKSPACE, "step: workspace too small");
+  cudaStream_t s = cs(stream);
+  const int di = c.d_inner, dm = c.d_model, R = c.dt_rank, N = c.d_state, W = R + 2 * N;
+  if (c.dtype == JAMBA_BF16) {
+    // weights stream through the tensor cores as the 128-row side; the token batch is the N side
+    GemmDesc g1 = gdesc(w.in_proj, dm, u, dm, 2 * di, batch, dm, EPI_BF16, p.xz, 2 * di);
+    g1.transpose_out = 1;
+    g1.bn = 64;
+    JB_TRY(gemm_bf16(g1, s));
+    JB_TRY(conv_step(p.xz, 2 * di, w.conv_w, w.conv_b, p.xc, conv_state, batch, di, c.dtype, s));
+    GemmDesc g2 = gdesc(w.x_proj, di, p.xc, di, W, batch, di, EPI_F32, p.xpart, W);
+    g2.transpose_out = 1;
+    g2.bn = 64;
+    g2.splits = p.x_splits;
+    g2.split_stride = (long long)batch * W;
+    JB_TRY(gemm_bf16(g2, s));
+    JB_TRY(xproj_norm(p.xpart, p.x_splits, (long long)batch * W, batch, R, N, w.norm_dt, w.norm_B, w.norm_C,
+                      c.inner_rmsnorm, c.eps, p.dtlow, p.bc, c.dtype, s));
+    GemmDesc g3 = gdesc(w.dt_proj, R, p.dtlow, R, di, batch, R, EPI_SOFTPLUS, p.dt, di);
+    g3.transpose_out = 1;
+    g3.bn = 64;
+    g3.bias = w.dt_bias;
+    JB_TRY(gemm_bf16(g3, s));
+    JB_TRY(ssm_step(p.xc, reinterpret_cast<const uint8_t*>(p.xz) + (size_t)di * 2, 2 * di, p.dt, p.bc, 2 * N, w.A,
+                    w.D, ssm_state, p.y, batch, di, c.dtype, s));
+    GemmDesc g4 = gdesc(w.out_proj, di, p.y, di, dm, batch, di, EPI_F32, p.opart, dm);
+    g4.transpose_out = 1;
+    g4.bn = 64;
+    g4.splits = p.o_splits;
+    g4.split_stride = (long long)batch * dm;
+    JB_TRY(gemm_bf16(g4, s));
+    JB_TRY(splitk_reduce(p.opart, p.o_splits, (long long)batch * dm, (long long)batch * dm, residual, out, c.dtype, s));
+  } else {
+    JB_TRY(gemm_f32(gdesc(u, dm, w.in_proj, dm, batch, 2 * di, dm, EPI_F32, p.xz, 2 * di), s));
+    JB_TRY(conv_step(p.xz, 2 * di, w.conv_w, w.conv_b, p.xc, conv_state, batch, di, c.dtype, s));
+    JB_TRY(gemm_f32(gdesc(p.xc, di, w.x_proj, di, batch, W, di, EPI_F32, p.xpart, W), s));
+    JB_TRY(xproj_norm(p.xpart, 1, 0, batch, R, N, w.norm_dt, w.norm_B, w.norm_C, c.inner_rmsnorm, c.eps, p.dtlow,
+                      p.bc, c.dtype, s));
+    GemmDesc g3 = gdesc(p.dtlow, R, w.dt_proj, R, batch, di, R, EPI_SOFTPLUS, p.dt, di);
+    g3.bias = w.dt_bias;
+    JB_TRY(gemm_f32(g3, s));
+    JB_TRY(ssm_step(p.xc, reinterpret_cast<const uint8_t*>(p.xz) + (size_t)di * 4, 2 * di, p.dt, p.bc, 2 * N, w.A,
+                    w.D, ssm_state, p.y, batch, di, c.dtype, s));
+    GemmDesc g4 = gdesc(p.y, di, w.out_proj, di, batch, dm, di, EPI_F32, out, dm);
+    g4.residual = residual;
+    g4.ldr = dm;
+    JB_TRY(gemm_f32(g4, s));
+  }
+  return JAMBA_OK;
+}
+
+// --------------------------------------------------------- selective scan
+
+jamba_status jamba_selective_scan_workspace_size(int batch, int seqlen, int d_inner, int d_state, int chunk,
+                                                 size_t* bytes) {
+  if (!bytes || batch <= 0 || seqlen <= 0 || d_inner <= 0) return fail(JAMBA_ERR_INVALID_ARG, "scan workspace: bad argument");
+  if (d_state != 16) return fail(JAMBA_ERR_UNSUPPORTED, "d_state must be 16");
+  if (chunk == 0) chunk = scan_auto_chunk(batch, seqlen, d_inner);
+  if (chunk < 0 || chunk % 16) return fail(JAMBA_ERR_INVALID_ARG, "chunk must be a multiple of 16");
+  *bytes = scan_workspace_bytes(batch, seqlen, d_inner, chunk);
+  return JAMBA_OK;
+}
+
+jamba_status jamba_selective_scan(const void* x, int ld_x, const void* z, int ld_z, const float* dt, int ld_dt,
+                                  const void* B, int ld_b, const void* C, int ld_c, int bc_dtype, const float* A,
+                                  const float* D, const float* h0, void* y, int ld_y, float* h_out, int batch,
+                                  int seqlen, int d_inner, int d_state, int dtype, int chunk, void* ws,
+                                  size_t ws_bytes, jamba_stream_t stream) {
+  JB_TRY(check_dtype(dtype));
+  JB_TRY(check_dtype(bc_dtype));
+  if (d_state != 16) return fail(JAMBA_ERR_UNSUPPORTED, "d_state must be 16");
+  if (batch <= 0 || seqlen <= 0 || d_inner <= 0) return fail(JAMBA_ERR_INVALID_ARG, "scan: sizes must be positive");
+  JB_TRY(check_ptr(x, "x"));
+  JB_TRY(check_ptr(z, "z"));
+  JB_TRY(check_ptr(dt, "dt"));
+  JB_TRY(check_ptr(B, "B"));
+  JB_TRY(check_ptr(C, "C"));
+  JB_TRY(check_ptr(A, "A"));
+  JB_TRY(check_ptr(D, "D"));
+  JB_TRY(check_ptr(h0, "h0", false));
+  JB_TRY(check_ptr(y, "y"));
+  JB_TRY(check_ptr(h_out, "h_out", false));
+  if (chunk == 0) chunk = scan_auto_chunk(batch, seqlen, d_inner);
+  ScanCall sc = {};
+  sc.x = x; sc.ld_x = ld_x; sc.z = z; sc.ld_z = ld_z; sc.dt = dt; sc.ld_dt = ld_dt;
+  sc.B = B; sc.ld_b = ld_b; sc.C = C; sc.ld_c = ld_c; sc.bc_dtype = bc_dtype;
+  sc.A = A; sc.D = D; sc.h0 = h0; sc.y = y; sc.ld_y = ld_y; sc.h_out = h_out;
+  sc.batch = batch; sc.L = seqlen; sc.di = d_inner; sc.dtype = dtype; sc.chunk = chunk;
+  sc.ws = ws; sc.ws_bytes = ws_bytes;
+  return scan_run(sc, cs(stream));
+}
+
+// --------------------------------------------------------- building blocks
+
+jamba_status jamba_rmsnorm(const void* x, const float* w, void* out, int rows, int cols, float eps, int dtype,
+                           jamba_stream_t stream) {
+  JB_TRY(check_dtype(dtype));
+  if (rows <= 0 || cols <= 0) return fail(JAMBA_ERR_INVALID_ARG, "rmsnorm: sizes must be positive");
+  JB_TRY(check_ptr(x, "x"));
+  JB_TRY(check_ptr(w, "w"));
+  JB_TRY(check_ptr(out, "out"));
+  return rmsnorm(x, w, out, rows, cols, eps, dtype, cs(stream));
+}
+
+jamba_status jamba_causal_conv1d(const void* x, int ld_x, const void* w, const void* b, void* out,
+                                 const float* state_in, float* state_out, int batch, int seqlen, int channels,
+                                 int dtype, jamba_stream_t stream) {
+  JB_TRY(check_dtype(dtype));
+  if (batch <= 0 || seqlen <= 0 || channels <= 0 || ld_x < channels)
+    return fail(JAMBA_ERR_INVALID_ARG, "conv: bad sizes");
+  JB_TRY(check_ptr(x, "x"));
+  JB_TRY(check_ptr(w, "w"));
+  JB_TRY(check_ptr(b, "b"));
+  JB_TRY(check_ptr(out, "out"));
+  if (state_in && state_in == state_out)
+    return fail(JAMBA_ERR_INVALID_ARG, "conv: state_in and state_out may not alias here");
+  return conv_prefill(x, ld_x, w, b, out, state_in, state_out, batch, seqlen, channels, dtype, cs(stream));
+}
+
+jamba_status jamba_gemm(const void* a, const void* b, void* out, int ld_out, const void* residual, int m, int n,
+                        int k, int dtype, int out_dtype, jamba_stream_t stream) {
+  JB_TRY(check_dtype(dtype));
+  JB_TRY(check_dtype(out_dtype));
+  if (m <= 0 || n <= 0 || k <= 0 || ld_out < n) return fail(JAMBA_ERR_INVALID_ARG, "gemm: bad sizes");
+  if (dtype == JAMBA_F32 && out_dtype != JAMBA_F32) return fail(JAMBA_ERR_UNSUPPORTED, "gemm: fp32 inputs give fp32 output");
+  if (residual && out_dtype != dtype) return fail(JAMBA_ERR_UNSUPPORTED, "gemm: residual needs out_dtype == dtype");
+  GemmDesc g = gdesc(a, k, b, k, m, n, k, out_dtype == JAMBA_BF16 ? EPI_BF16 : EPI_F32, out, ld_out);
+  g.residual = residual;
+  g.ldr = ld_out;
+  return gemm_any(dtype, g, cs(stream));
+}
+
+// -------------------------------------------------------------------- MoE
+
+namespace {
+struct MoeWs {
+  int* counts; int* inv; void* xperm; void* act; float* Y;
+  size_t total;
+};
+MoeWs carve_moe(const jamba_moe_config& c, int T, void* ws) {
+  MoeWs m;
+  const size_t rows = (size_t)T * c.top_k;
+  Carver cv(ws);
+  m.counts = cv.take<int>(sizeof(int) * 64);
+  m.inv = cv.take<int>(sizeof(int) * rows);
+  m.xperm = cv.take(rows * c.d_model * 2);
+  m.act = cv.take(rows * c.d_ff * 2);
+  m.Y = cv.take<float>(rows * c.d_model * 4);
+  m.total = cv.off;
+  return m;
+}
+jamba_status check_moe_cfg(const jamba_moe_config* c) {
+  if (!c) return fail(JAMBA_ERR_INVALID_ARG, "moe: null config");
+  if (c->dtype != JAMBA_BF16) return fail(JAMBA_ERR_UNSUPPORTED, "moe: bf16 only");
+  if (c->n_experts < 1 || c->n_experts > 64) return fail(JAMBA_ERR_UNSUPPORTED, "moe: 1..64 experts");
+  if (c->top_k < 1 || c->top_k > 2 || c->top_k > c->n_experts) return fail(JAMBA_ERR_UNSUPPORTED, "moe: top_k must be 1 or 2");
+  if (c->d_model <= 0 || c->d_model % 256) return fail(JAMBA_ERR_UNSUPPORTED, "moe: d_model must be a multiple of 256");
+  if (c->d_ff <= 0 || c->d_ff % 128) return fail(JAMBA_ERR_UNSUPPORTED, "moe: d_ff must be a multiple of 128");
+  return JAMBA_OK;
+}
+}  // namespace
+
+jamba_status jamba_moe_workspace_size(const jamba_moe_config* cfg, int tokens, size_t* bytes) {
+  JB_TRY(check_moe_cfg(cfg));
+  if (!bytes || tokens <= 0) return fail(JAMBA_ERR_INVALID_ARG, "moe workspace: bad argument");
+  *bytes = carve_moe(*cfg, tokens, nullptr).total;
+  return JAMBA_OK;
+}
+
+jamba_status jamba_moe_forward(const jamba_moe_config* cfg, const jamba_moe_weights* w, const void* x,
+                               const void* residual, void* y, int tokens, int32_t* topk_idx, float* topk_w,
+                               int32_t* expert_offsets, int32_t* perm, void* ws, size_t ws_bytes,
+                               jamba_stream_t stream) {
+  JB_TRY(check_moe_cfg(cfg));
+  if (!w || tokens <= 0) return fail(JAMBA_ERR_INVALID_ARG, "moe: bad argument");
+  JB_TRY(check_ptr(w->router, "router"));
+  JB_TRY(check_ptr(w->w_gate, "w_gate"));
+  JB_TRY(check_ptr(w->w_up, "w_up"));
+  JB_TRY(check_ptr(w->w_down, "w_down"));
+  JB_TRY(check_ptr(x, "x"));
+  JB_TRY(check_ptr(y, "y"));
+  JB_TRY(check_ptr(residual, "residual", false));
+  JB_TRY(check_ptr(topk_idx, "topk_idx"));
+  JB_TRY(check_ptr(topk_w, "topk_w"));
+  JB_TRY(check_ptr(expert_offsets, "expert_offsets"));
+  JB_TRY(check_ptr(perm, "perm"));
+  JB_TRY(check_ptr(ws, "workspace"));
+  const jamba_moe_config& c = *cfg;
+  MoeWs m = carve_moe(c, tokens, ws);
+  if (ws_bytes < m.total) return fail(JAMBA_ERR_WORKSPACE, "moe: workspace too small");
+  cudaStream_t s = cs(stream);
+  const int E = c.n_experts, K = c.top_k, dm = c.d_model, dff = c.d_ff;
+  const int rows = tokens * K;
+  JB_TRY(moe_route(x, w->router, tokens, dm, E, K, topk_idx, topk_w, m.counts, expert_offsets, perm, m.inv, s));
+  JB_TRY(moe_gather(x, perm, rows, K, dm, m.xperm, s));
+  // gate | up with SwiGLU: act = SiLU(x W_g^T) * (x W_u^T), per expert
+  GemmDesc g1 = gdesc(m.xperm, dm, w->w_gate, dm, rows, dff, dm, EPI_SWIGLU, m.act, dff);
+  g1.b2 = w->w_up;
+  g1.grouped = 1;
+  g1.offsets = expert_offsets;
+  g1.num_groups = E;
+  g1.b_rows = dff;
+  JB_TRY(gemm_bf16(g1, s));
+  // down: Y = act W_d^T, fp32 rows in routed order
+  GemmDesc g2 = gdesc(m.act, dff, w->w_down, dff, rows, dm, dff, EPI_F32, m.Y, dm);
+  g2.grouped = 1;
+  g2.offsets = expert_offsets;
+  g2.num_groups = E;
+  g2.b_rows = dm;
+  JB_TRY(gemm_bf16(g2, s));
+  JB_TRY(moe_combine(m.Y, m.inv, topk_w, tokens, K, dm, residual, y, s));
+  return JAMBA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,165 @@
+// Causal depthwise conv1d (d_conv = 4) + SiLU, prefill and decode step.
+//
+// Mamba layer used by Jamba ("Jamba: A Hybrid Transformer-Mamba Language
+// Model", section 2, ref [17]): xc[t, c] = SiLU(b[c] + sum_k w[c, k] x[t-3+k, c]),
+// x at negative times taken from the cache (the last three pre-conv inputs,
+// oldest first) or zero.
+//
+// Prefill: each thread owns 16 bytes of channels (8 bf16 or 4 fp32) over a run
+// of 64 time steps, keeping the three previous inputs in registers, so every
+// input row is read once (plus a 3-row halo per run) with 16-byte loads that
+// are contiguous across the warp.
+#include "common.cuh"
+#include "host.hpp"
+
+namespace jb {
+
+constexpr int CONV_TQ = 64;
+constexpr int CONV_THREADS = 128;
+
+template <typename T> struct Vec16;
+template <> struct Vec16<bf16> {
+  static constexpr int N = 8;
+  static __device__ __forceinline__ void load(const bf16* p, float* v) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(h[i]);
+      v[2 * i] = f.x;
+      v[2 * i + 1] = f.y;
+    }
+  }
+  static __device__ __forceinline__ void store(bf16* p, const float* v) {
+    uint4 u;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+    *reinterpret_cast<uint4*>(p) = u;
+  }
+};
+template <> struct Vec16<float> {
+  static constexpr int N = 4;
+  static __device__ __forceinline__ void load(const float* p, float* v) {
+    const float4 u = *reinterpret_cast<const float4*>(p);
+    v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
+  }
+  static __device__ __forceinline__ void store(float* p, const float* v) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  }
+};
+
+template <typename T>
+__global__ void __launch_bounds__(CONV_THREADS)
+conv_prefill_kernel(const T* __restrict__ x, long long ld_x, const T* __restrict__ w, const T* __restrict__ bias,
+                    T* __restrict__ out, const float* __restrict__ st_in, float* __restrict__ st_out, int L,
+                    int C) {
+  constexpr int V = Vec16<T>::N;
+  const int c0 = (blockIdx.x * CONV_THREADS + threadIdx.x) * V;
+  if (c0 >= C) return;
+  const int b = blockIdx.z;
+  const int t0 = blockIdx.y * CONV_TQ;
+  const int t1 = min(L, t0 + CONV_TQ);
+  float wk[4][V], bv[V];
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) wk[k][i] = to_f(w[(long long)(c0 + i) * 4 + k]);
+    bv[i] = to_f(bias[c0 + i]);
+  }
+  const T* xb = x + (long long)b * L * ld_x;
+  float win[3][V];
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    const int t = t0 - 3 + k;
+    if (t >= 0) {
+      Vec16<T>::load(xb + (long long)t * ld_x + c0, win[k]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < V; ++i)
+        win[k][i] = st_in ? st_in[((long long)b * C + c0 + i) * 3 + (3 + t)] : 0.f;
+    }
+  }
+  T* ob = out + (long long)b * L * C;
+  for (int t = t0; t < t1; ++t) {
+    float cur[V], o[V];
+    Vec16<T>::load(xb + (long long)t * ld_x + c0, cur);
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+      float acc = bv[i];
+      acc = fmaf(wk[0][i], win[0][i], acc);
+      acc = fmaf(wk[1][i], win[1][i], acc);
+      acc = fmaf(wk[2][i], win[2][i], acc);
+      acc = fmaf(wk[3][i], cur[i], acc);
+      o[i] = silu(acc);
+      win[0][i] = win[1][i];
+      win[1][i] = win[2][i];
+      win[2][i] = cur[i];
+    }
+    Vec16<T>::store(ob + (long long)t * C + c0, o);
+  }
+  if (st_out && t1 == L) {
+#pragma unroll
+    for (int i = 0; i < V; ++i)
+#pragma unroll
+      for (int k = 0; k < 3; ++k) st_out[((long long)b * C + c0 + i) * 3 + k] = win[k][i];
+  }
+}
+
+// decode: one thread per (batch row, channel); the cache shifts in place
+template <typename T>
+__global__ void __launch_bounds__(256)
+conv_step_kernel(const T* __restrict__ x, long long ld_x, const T* __restrict__ w, const T* __restrict__ bias,
+                 T* __restrict__ out, float* __restrict__ state, int batch, int C) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long long)batch * C) return;
+  const int b = (int)(i / C), c = (int)(i - (long long)b * C);
+  float* s = state + i * 3;
+  const float s0 = s[0], s1 = s[1], s2 = s[2];
+  const float xv = to_f(x[(long long)b * ld_x + c]);
+  float acc = to_f(bias[c]);
+  acc = fmaf(to_f(w[(long long)c * 4 + 0]), s0, acc);
+  acc = fmaf(to_f(w[(long long)c * 4 + 1]), s1, acc);
+  acc = fmaf(to_f(w[(long long)c * 4 + 2]), s2, acc);
+  acc = fmaf(to_f(w[(long long)c * 4 + 3]), xv, acc);
+  out[i] = from_f<T>(silu(acc));
+  s[0] = s1;
+  s[1] = s2;
+  s[2] = xv;
+}
+
+jamba_status conv_prefill(const void* x, long long ld_x, const void* w, const void* b, void* out,
+                          const float* st_in, float* st_out, int batch, int L, int C, int dtype, cudaStream_t s) {
+  const int V = dtype == JAMBA_BF16 ? 8 : 4;
+  if (C % V || ld_x % V || !aligned16(x) || !aligned16(out))
+    return fail(JAMBA_ERR_INVALID_ARG, "conv: channels and row stride must fill 16-byte vectors");
+  dim3 grid((C / V + CONV_THREADS - 1) / CONV_THREADS, (L + CONV_TQ - 1) / CONV_TQ, batch);
+  if (dtype == JAMBA_BF16)
+    conv_prefill_kernel<bf16><<<grid, CONV_THREADS, 0, s>>>(
+        reinterpret_cast<const bf16*>(x), ld_x, reinterpret_cast<const bf16*>(w), reinterpret_cast<const bf16*>(b),
+        reinterpret_cast<bf16*>(out), st_in, st_out, L, C);
+  else
+    conv_prefill_kernel<float><<<grid, CONV_THREADS, 0, s>>>(
+        reinterpret_cast<const float*>(x), ld_x, reinterpret_cast<const float*>(w),
+        reinterpret_cast<const float*>(b), reinterpret_cast<float*>(out), st_in, st_out, L, C);
+  JB_CUDA(cudaGetLastError());
+  return JAMBA_OK;
+}
+
+jamba_status conv_step(const void* x, long long ld_x, const void* w, const void* b, void* out, float* state,
+                       int batch, int C, int dtype, cudaStream_t s) {
+  const long long n = (long long)batch * C;
+  const unsigned grid = (unsigned)((n + 255) / 256);
+  if (dtype == JAMBA_BF16)
+    conv_step_kernel<bf16><<<grid, 256, 0, s>>>(reinterpret_cast<const bf16*>(x), ld_x,
+                                               reinterpret_cast<const bf16*>(w), reinterpret_cast<const bf16*>(b),
+                                               reinterpret_cast<bf16*>(out), state, batch, C);
+  else
+    conv_step_kernel<float><<<grid, 256, 0, s>>>(reinterpret_cast<const float*>(x), ld_x,
+                                                reinterpret_cast<const float*>(w), reinterpret_cast<const float*>(b),
+                                                reinterpret_cast<float*>(out), state, batch, C);
+  JB_CUDA(cudaGetLastError());
+  return JAMBA_OK;
+}
+
+}  // namespace jb

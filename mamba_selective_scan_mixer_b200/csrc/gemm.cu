@@ -1,0 +1,183 @@
+// GEMM launchers: the tcgen05 kernel for bf16 and a CUDA-core kernel for the
+// fp32 path (fp32 inputs must keep ~1e-5 accuracy, which TF32 would not).
+#include <string>
+
+#include "gemm_tc.cuh"
+#include "host.hpp"
+
+namespace jb {
+
+template <int BN, int STAGES>
+static jamba_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb2,
+                              const GemmParams& p, int grid, cudaStream_t s) {
+  using S = GemmSmem<BN, STAGES>;
+  static bool configured[64] = {false};
+  int dev = 0;
+  JB_CUDA(cudaGetDevice(&dev));
+  if (dev < 64 && !configured[dev]) {
+    JB_CUDA(cudaFuncSetAttribute(gemm_bf16_tc_kernel<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)S::BYTES));
+    configured[dev] = true;
+  }
+  gemm_bf16_tc_kernel<BN, STAGES><<<grid, 192, S::BYTES, s>>>(ma, mb, mb2, p);
+  JB_CUDA(cudaGetLastError());
+  return JAMBA_OK;
+}
+
+jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
+  if (g.M <= 0 || g.N <= 0 || g.K <= 0) return fail(JAMBA_ERR_INVALID_ARG, "gemm: sizes must be positive");
+  if (!g.a || !g.b || !g.out) return fail(JAMBA_ERR_INVALID_ARG, "gemm: null operand");
+  if (g.K % 8 || g.lda % 8 || g.ldb % 8 || !aligned16(g.a) || !aligned16(g.b))
+    return fail(JAMBA_ERR_INVALID_ARG, "gemm: K and leading dimensions must be multiples of 8, operands 16-byte aligned");
+  if (!g.transpose_out && !aligned16(g.out)) return fail(JAMBA_ERR_INVALID_ARG, "gemm: output must be 16-byte aligned");
+  if (!g.transpose_out && ((g.epi == EPI_BF16 || g.epi == EPI_SWIGLU) ? g.ldo % 8 : g.ldo % 4))
+    return fail(JAMBA_ERR_INVALID_ARG, "gemm: output leading dimension breaks 16-byte rows");
+  if (g.residual && (g.transpose_out || g.epi != EPI_BF16 || g.ldr % 8 || !aligned16(g.residual)))
+    return fail(JAMBA_ERR_INVALID_ARG, "gemm: residual only with aligned non-transposed bf16 output");
+  if (g.splits > 1 && (g.epi != EPI_F32 || g.grouped))
+    return fail(JAMBA_ERR_INVALID_ARG, "gemm: split-K writes fp32 partials only");
+  if (g.epi == EPI_SWIGLU && (!g.grouped || !g.b2))
+    return fail(JAMBA_ERR_INVALID_ARG, "gemm: SwiGLU needs grouped gate and up weights");
+
+  int bn = g.bn;
+  if (bn == 0) {
+    if (g.epi == EPI_SWIGLU) bn = 256;
+    else if (g.N <= 64) bn = 64;
+    else if (g.N <= 128) bn = 128;
+    else if (g.N <= 144 || g.N == 288) bn = 144;
+    else bn = 256;
+  }
+  const int bn_out = g.epi == EPI_SWIGLU ? bn / 2 : bn;
+  const int b_box = g.epi == EPI_SWIGLU ? bn / 2 : bn;
+
+  CUtensorMap ma, mb, mb2;
+  const uint64_t a_rows = (uint64_t)g.M;
+  JB_TRY(make_map_2d(&ma, g.a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)g.K, a_rows,
+                     (uint64_t)g.lda * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B));
+  if (!g.grouped) {
+    JB_TRY(make_map_2d(&mb, g.b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)g.K, (uint64_t)g.N,
+                       (uint64_t)g.ldb * 2, 64, (uint32_t)b_box, CU_TENSOR_MAP_SWIZZLE_128B));
+    mb2 = mb;
+  } else {
+    const uint64_t rs = (uint64_t)g.ldb * 2, os = rs * (uint64_t)g.b_rows;
+    JB_TRY(make_map_3d(&mb, g.b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)g.K, (uint64_t)g.b_rows,
+                       (uint64_t)g.num_groups, rs, os, 64, (uint32_t)b_box, CU_TENSOR_MAP_SWIZZLE_128B));
+    if (g.b2) {
+      JB_TRY(make_map_3d(&mb2, g.b2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)g.K, (uint64_t)g.b_rows,
+                         (uint64_t)g.num_groups, rs, os, 64, (uint32_t)b_box, CU_TENSOR_MAP_SWIZZLE_128B));
+    } else {
+      mb2 = mb;
+    }
+  }
+
+  GemmParams p;
+  p.M = g.M;
+  p.N = g.N;
+  p.K = g.K;
+  p.k_tiles = (g.K + 63) / 64;
+  p.splits = g.splits < 1 ? 1 : g.splits;
+  p.k_tiles_per_split = (p.k_tiles + p.splits - 1) / p.splits;
+  p.splits = (p.k_tiles + p.k_tiles_per_split - 1) / p.k_tiles_per_split;
+  p.m_tiles = (g.M + 127) / 128;
+  p.n_tiles = (g.N + bn_out - 1) / bn_out;
+  p.grouped = g.grouped;
+  p.offsets = g.offsets;
+  p.num_groups = g.num_groups;
+  p.epi = g.epi;
+  p.transpose_out = g.transpose_out;
+  p.out = g.out;
+  p.ldo = g.ldo;
+  p.split_stride = g.split_stride;
+  p.residual = g.residual;
+  p.ldr = g.ldr;
+  p.bias = g.bias;
+  p.err = device_error_word();
+  if (!p.err) return fail(JAMBA_ERR_CUDA, "could not allocate the device status word");
+
+  long long tiles = g.grouped ? (long long)(p.m_tiles + g.num_groups) * p.n_tiles
+                              : (long long)p.m_tiles * p.n_tiles * p.splits;
+  const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
+  switch (bn) {
+    case 64: return launch_tc<64, 8>(ma, mb, mb2, p, grid, s);
+    case 128: return launch_tc<128, 6>(ma, mb, mb2, p, grid, s);
+    case 144: return launch_tc<144, 6>(ma, mb, mb2, p, grid, s);
+    case 256: return launch_tc<256, 4>(ma, mb, mb2, p, grid, s);
+    default: return fail(JAMBA_ERR_UNSUPPORTED, "gemm: tile width " + std::to_string(bn));
+  }
+}
+
+// ---------------------------------------------------------------- fp32 path
+// 64 x 64 output tile per 256-thread block, 4 x 4 per thread, k-steps of 16.
+__global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__ A, long long lda,
+                                                       const float* __restrict__ B, long long ldb, int M, int N,
+                                                       int K, GemmParams p) {
+  __shared__ float As[16][64 + 4];
+  __shared__ float Bs[16][64 + 4];
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < K; k0 += 16) {
+    for (int i = threadIdx.x; i < 64 * 16; i += 256) {
+      const int r = i >> 4, k = i & 15;
+      As[k][r] = (m0 + r < M && k0 + k < K) ? A[(long long)(m0 + r) * lda + k0 + k] : 0.f;
+      Bs[k][r] = (n0 + r < N && k0 + k < K) ? B[(long long)(n0 + r) * ldb + k0 + k] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        a[i] = As[k][ty * 4 + i];
+        b[i] = Bs[k][tx * 4 + i];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  float* out = reinterpret_cast<float*>(p.out);
+  const float* res = reinterpret_cast<const float*>(p.residual);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int m = m0 + ty * 4 + i;
+    if (m >= M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + tx * 4 + j;
+      if (n >= N) continue;
+      float v = acc[i][j];
+      if (p.epi == EPI_SOFTPLUS) v = softplus(v + p.bias[p.transpose_out ? m : n]);
+      if (p.transpose_out) {
+        out[(long long)n * p.ldo + m] = v;
+      } else {
+        if (res) v += res[(long long)m * p.ldr + n];
+        out[(long long)m * p.ldo + n] = v;
+      }
+    }
+  }
+}
+
+jamba_status gemm_f32(const GemmDesc& g, cudaStream_t s) {
+  if (g.M <= 0 || g.N <= 0 || g.K <= 0) return fail(JAMBA_ERR_INVALID_ARG, "gemm: sizes must be positive");
+  if (!g.a || !g.b || !g.out) return fail(JAMBA_ERR_INVALID_ARG, "gemm: null operand");
+  if (g.grouped || g.splits > 1 || (g.epi != EPI_F32 && g.epi != EPI_SOFTPLUS))
+    return fail(JAMBA_ERR_UNSUPPORTED, "fp32 gemm: dense, unsplit, fp32 or softplus epilogue only");
+  GemmParams p = {};
+  p.epi = g.epi;
+  p.transpose_out = g.transpose_out;
+  p.out = g.out;
+  p.ldo = g.ldo;
+  p.residual = g.residual;
+  p.ldr = g.ldr;
+  p.bias = g.bias;
+  dim3 grid((g.N + 63) / 64, (g.M + 63) / 64);
+  gemm_f32_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const float*>(g.a), g.lda,
+                                       reinterpret_cast<const float*>(g.b), g.ldb, g.M, g.N, g.K, p);
+  JB_CUDA(cudaGetLastError());
+  return JAMBA_OK;
+}
+
+}  // namespace jb

@@ -1,0 +1,353 @@
+// tcgen05 / TMEM GEMM for sm_100a: D[m, n] = sum_k A[m, k] * B[n, k], bf16
+// inputs, fp32 accumulation in tensor memory.
+//
+// One persistent CTA per SM, 6 warps:
+//   warp 0     TMA producer: 128 x 64 A tile and BN x 64 B tile per k-step
+//              (128-byte swizzle) into a STAGES-deep shared-memory ring;
+//   warp 1     allocates TMEM and issues tcgen05.mma (one thread), M = 128,
+//              N = BN, K = 16 per instruction, into one of two TMEM
+//              accumulators so the epilogue of tile i overlaps tile i + 1;
+//   warps 2-5  epilogue: tcgen05.ld of their 32-lane quarter, fused
+//              elementwise op, stores to global memory.
+// Used for in_proj, x_proj, dt_proj (+bias+softplus), out_proj (+residual),
+// the decode projections (swap-AB: weights as A so the 64-row token batch is
+// the N side, stored transposed) and the grouped MoE expert GEMMs (SwiGLU
+// epilogue).  Every wait is bounded (see common.cuh).
+#pragma once
+#include "common.cuh"
+
+namespace jb {
+
+enum EpiKind : int { EPI_BF16 = 0, EPI_F32 = 1, EPI_SOFTPLUS = 2, EPI_SWIGLU = 3 };
+
+struct GemmParams {
+  int M, N, K;           // N counts output columns (SwiGLU: d_ff)
+  int k_tiles;           // ceil(K / 64)
+  int splits, k_tiles_per_split;
+  int m_tiles, n_tiles;  // dense mode
+  int grouped;           // A rows split by offsets[], B is [groups, rows, K]
+  const int* offsets;
+  int num_groups;
+  int epi;
+  int transpose_out;     // store out[n * ldo + m]
+  void* out;
+  long long ldo, split_stride;
+  const void* residual;  // bf16, same layout as out (non-transposed only)
+  long long ldr;
+  const float* bias;     // indexed by n (or by m when transposed)
+  int* err;
+};
+
+struct TileInfo {
+  int m0, m_end, n0, kt0, kt1, group, split;
+};
+
+template <int BN>
+__device__ __forceinline__ int total_tiles(const GemmParams& p) {
+  if (!p.grouped) return p.m_tiles * p.n_tiles * p.splits;
+  int tot = 0;
+  for (int g = 0; g < p.num_groups; ++g) {
+    int cnt = __ldg(p.offsets + g + 1) - __ldg(p.offsets + g);
+    tot += ((cnt + 127) >> 7) * p.n_tiles;
+  }
+  return tot;
+}
+
+template <int BN>
+__device__ __forceinline__ void decode_tile(const GemmParams& p, int t, TileInfo& ti) {
+  const int bn_out = (p.epi == EPI_SWIGLU) ? BN / 2 : BN;
+  if (!p.grouped) {
+    const int per_split = p.m_tiles * p.n_tiles;
+    const int s = t / per_split;
+    const int r = t - s * per_split;
+    // rasterise in bands of 16 m-tiles so concurrent CTAs share A and B tiles in L2
+    constexpr int G = 16;
+    const int span = G * p.n_tiles;
+    const int gi = r / span;
+    const int first_m = gi * G;
+    const int gsize = min(p.m_tiles - first_m, G);
+    const int rr = r - gi * span;
+    const int mb = first_m + rr % gsize;
+    const int nb = rr / gsize;
+    ti.m0 = mb * 128;
+    ti.m_end = p.M;
+    ti.n0 = nb * bn_out;
+    ti.kt0 = s * p.k_tiles_per_split;
+    ti.kt1 = min(p.k_tiles, ti.kt0 + p.k_tiles_per_split);
+    ti.group = 0;
+    ti.split = s;
+  } else {
+    for (int g = 0; g < p.num_groups; ++g) {
+      const int o0 = __ldg(p.offsets + g), o1 = __ldg(p.offsets + g + 1);
+      const int mt = (o1 - o0 + 127) >> 7;
+      const int tg = mt * p.n_tiles;
+      if (t < tg) {
+        const int mb = t % mt, nb = t / mt;  // m fastest: neighbours share the weight tile
+        ti.m0 = o0 + mb * 128;
+        ti.m_end = o1;
+        ti.n0 = nb * bn_out;
+        ti.kt0 = 0;
+        ti.kt1 = p.k_tiles;
+        ti.group = g;
+        ti.split = 0;
+        return;
+      }
+      t -= tg;
+    }
+    ti.m0 = ti.m_end = ti.n0 = ti.kt0 = ti.kt1 = ti.group = ti.split = 0;
+  }
+}
+
+__device__ __forceinline__ void store_bf16x8(bf16* dst, const float* v) {
+  uint4 u;
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+  *reinterpret_cast<uint4*>(dst) = u;
+}
+
+// Epilogue for one 32-column chunk held by this thread (row m, columns n..n+31).
+__device__ __forceinline__ void epi_chunk(const GemmParams& p, const TileInfo& ti, int m, int n, float* v) {
+  if (m >= ti.m_end) return;
+  if (!p.transpose_out) {
+    if (p.epi == EPI_BF16) {
+      bf16* o = reinterpret_cast<bf16*>(p.out) + (long long)m * p.ldo;
+      const bf16* r = p.residual ? reinterpret_cast<const bf16*>(p.residual) + (long long)m * p.ldr : nullptr;
+#pragma unroll
+      for (int c = 0; c < 32; c += 8) {
+        const int nn = n + c;
+        if (nn + 8 <= p.N) {
+          float w[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) w[i] = v[c + i];
+          if (r) {
+            uint4 rv = *reinterpret_cast<const uint4*>(r + nn);
+            const bf16* rb = reinterpret_cast<const bf16*>(&rv);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) w[i] += __bfloat162float(rb[i]);
+          }
+          store_bf16x8(o + nn, w);
+        } else {
+          for (int i = 0; i < 8 && nn + i < p.N; ++i) {
+            float w = v[c + i] + (r ? __bfloat162float(r[nn + i]) : 0.f);
+            o[nn + i] = __float2bfloat16_rn(w);
+          }
+        }
+      }
+    } else {  // EPI_F32 / EPI_SOFTPLUS
+      float* o = reinterpret_cast<float*>(p.out) + (long long)ti.split * p.split_stride + (long long)m * p.ldo;
+      const bool sp = p.epi == EPI_SOFTPLUS;
+#pragma unroll
+      for (int c = 0; c < 32; c += 4) {
+        const int nn = n + c;
+        float w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          w[i] = v[c + i];
+          if (sp && nn + i < p.N) w[i] = softplus(w[i] + __ldg(p.bias + nn + i));
+        }
+        if (nn + 4 <= p.N) {
+          *reinterpret_cast<float4*>(o + nn) = make_float4(w[0], w[1], w[2], w[3]);
+        } else {
+          for (int i = 0; i < 4 && nn + i < p.N; ++i) o[nn + i] = w[i];
+        }
+      }
+    }
+  } else {
+    // swap-AB: row m is an output feature, column n a token; lanes hold consecutive m
+    if (p.epi == EPI_BF16) {
+      bf16* o = reinterpret_cast<bf16*>(p.out);
+#pragma unroll 8
+      for (int c = 0; c < 32; ++c)
+        if (n + c < p.N) o[(long long)(n + c) * p.ldo + m] = __float2bfloat16_rn(v[c]);
+    } else {
+      float* o = reinterpret_cast<float*>(p.out) + (long long)ti.split * p.split_stride;
+      const float b = (p.epi == EPI_SOFTPLUS) ? __ldg(p.bias + m) : 0.f;
+#pragma unroll 8
+      for (int c = 0; c < 32; ++c) {
+        if (n + c < p.N) {
+          float w = v[c];
+          if (p.epi == EPI_SOFTPLUS) w = softplus(w + b);
+          o[(long long)(n + c) * p.ldo + m] = w;
+        }
+      }
+    }
+  }
+}
+
+template <int BN, int STAGES>
+struct GemmSmem {
+  static constexpr uint32_t A_BYTES = 128 * 128;
+  static constexpr uint32_t B_BYTES = BN * 128;
+  static constexpr uint32_t BAR_OFF = STAGES * (A_BYTES + B_BYTES);
+  static constexpr uint32_t BYTES = BAR_OFF + 256 + 1024;  // + barriers + alignment slack
+  // barrier slots: full[STAGES], empty[STAGES], tmem_full[2], tmem_empty[2], drain, tmem holder
+  static constexpr uint32_t TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
+                                        : (2 * BN <= 256) ? 256 : 512;
+};
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(192, 1)
+gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmB2, const GemmParams p) {
+  using S = GemmSmem<BN, STAGES>;
+  static_assert(BN % 16 == 0 && BN >= 32 && BN <= 256, "UMMA N for M = 128");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * S::A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::BAR_OFF);
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES);
+  const uint32_t tfull0 = smem_u32(bars + 2 * STAGES), tempty0 = smem_u32(bars + 2 * STAGES + 2);
+  const uint32_t drain = smem_u32(bars + 2 * STAGES + 4);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(tfull0 + 8 * i, 1);
+      mbar_init(tempty0 + 8 * i, 4);
+    }
+    mbar_init(drain, 1);
+    mbar_fence_init();
+    tma_prefetch(&tmA);
+    tma_prefetch(&tmB);
+    if (p.epi == EPI_SWIGLU) tma_prefetch(&tmB2);
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_holder), S::TMEM_COLS);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_holder;
+  const int ntiles = total_tiles<BN>(p);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        TileInfo ti;
+        decode_tile<BN>(p, t, ti);
+        for (int kt = ti.kt0; kt < ti.kt1; ++kt) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, p.err)) { ok = false; break; }
+          const uint32_t fb = full0 + 8 * stage;
+          mbar_arrive_tx(fb, S::A_BYTES + S::B_BYTES);
+          const uint32_t a_dst = smem_u32(sA + stage * S::A_BYTES);
+          const uint32_t b_dst = smem_u32(sB + stage * S::B_BYTES);
+          tma_load_2d(a_dst, &tmA, fb, kt * 64, ti.m0);
+          if (!p.grouped) {
+            tma_load_2d(b_dst, &tmB, fb, kt * 64, ti.n0);
+          } else if (p.epi != EPI_SWIGLU) {
+            tma_load_3d(b_dst, &tmB, fb, kt * 64, ti.n0, ti.group);
+          } else {
+            tma_load_3d(b_dst, &tmB, fb, kt * 64, ti.n0, ti.group);
+            tma_load_3d(b_dst + (BN / 2) * 128, &tmB2, fb, kt * 64, ti.n0, ti.group);
+          }
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_bf16(128, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int it = 0;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++it) {
+        TileInfo ti;
+        decode_tile<BN>(p, t, ti);
+        const int acc = it & 1;
+        const uint32_t use = (uint32_t)(it >> 1);
+        if (!mbar_wait(tempty0 + 8 * acc, (use & 1) ^ 1, p.err)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tbase + acc * BN;
+        for (int kt = ti.kt0; kt < ti.kt1; ++kt) {
+          if (!mbar_wait(full0 + 8 * stage, phase, p.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t ad = sw128_desc(smem_u32(sA + stage * S::A_BYTES));
+          const uint64_t bd = sw128_desc(smem_u32(sB + stage * S::B_BYTES));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(d_tmem, ad + 2 * kk, bd + 2 * kk, IDESC, (kt > ti.kt0 || kk > 0) ? 1u : 0u);
+          umma_commit(empty0 + 8 * stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        umma_commit(tfull0 + 8 * acc);
+      }
+      // drain: no MMA may still be writing TMEM when the CTA frees it
+      umma_commit(drain);
+      mbar_wait(drain, 0, p.err);
+    }
+  } else {
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    int it = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
+      TileInfo ti;
+      decode_tile<BN>(p, t, ti);
+      const int acc = it & 1;
+      const uint32_t use = (uint32_t)(it >> 1);
+      if (!mbar_wait(tfull0 + 8 * acc, use & 1, p.err)) break;
+      tc_fence_after();
+      const int m = ti.m0 + q * 32 + lane;
+      const uint32_t tl = tbase + ((uint32_t)(q * 32) << 16) + acc * BN;
+      if (p.epi != EPI_SWIGLU) {
+#pragma unroll 1
+        for (int j = 0; j < BN / 32; ++j) {
+          float v[32];
+          tmem_ld32(tl + j * 32, v);
+          tmem_wait_ld();
+          epi_chunk(p, ti, m, ti.n0 + j * 32, v);
+        }
+        if constexpr (BN % 32 != 0) {
+          float v[16];
+          tmem_ld16(tl + (BN / 32) * 32, v);
+          tmem_wait_ld();
+          float w[32];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) { w[i] = v[i]; w[16 + i] = 0.f; }
+          // only 16 valid columns here: clamp N for this chunk
+          GemmParams q2 = p;
+          q2.N = min(p.N, ti.n0 + (BN / 32) * 32 + 16);
+          epi_chunk(q2, ti, m, ti.n0 + (BN / 32) * 32, w);
+        }
+      } else {
+        bf16* o = reinterpret_cast<bf16*>(p.out) + (long long)m * p.ldo;
+#pragma unroll 1
+        for (int j = 0; j < BN / 64; ++j) {
+          float g[32], u[32];
+          tmem_ld32(tl + j * 32, g);
+          tmem_ld32(tl + BN / 2 + j * 32, u);
+          tmem_wait_ld();
+          if (m < ti.m_end) {
+            const int n = ti.n0 + j * 32;
+#pragma unroll
+            for (int c = 0; c < 32; c += 8) {
+              float w[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) w[i] = silu(g[c + i]) * u[c + i];
+              if (n + c + 8 <= p.N) store_bf16x8(o + n + c, w);
+              else
+                for (int i = 0; i < 8 && n + c + i < p.N; ++i) o[n + c + i] = __float2bfloat16_rn(w[i]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, S::TMEM_COLS);
+  }
+}
+
+}  // namespace jb

@@ -1,0 +1,115 @@
+// Host-side internals shared by the launchers: error reporting, device
+// properties, TMA tensor-map encoding, per-device error word.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "../../include/jamba.h"
+
+namespace jb {
+
+jamba_status fail(jamba_status st, const std::string& msg);
+const char* last_error();
+jamba_status cuda_fail(cudaError_t e, const char* what);
+#define JB_CUDA(call)                                       \
+  do {                                                      \
+    cudaError_t e_ = (call);                                \
+    if (e_ != cudaSuccess) return ::jb::cuda_fail(e_, #call); \
+  } while (0)
+#define JB_TRY(expr)                         \
+  do {                                       \
+    jamba_status s_ = (expr);                \
+    if (s_ != JAMBA_OK) return s_;           \
+  } while (0)
+
+int num_sms();                 // of the current device
+int* device_error_word();      // per-device status word (allocated on first use)
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// 2-D tensor map over a row-major matrix: `inner` elements per row (the
+// extent TMA treats as valid), `rows` rows, `row_stride` bytes between rows.
+jamba_status make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes,
+                         uint64_t inner, uint64_t rows, uint64_t row_stride, uint32_t box_inner,
+                         uint32_t box_rows, CUtensorMapSwizzle sw);
+// 3-D tensor map over [outer][rows][inner].
+jamba_status make_map_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes,
+                         uint64_t inner, uint64_t rows, uint64_t outer, uint64_t row_stride,
+                         uint64_t outer_stride, uint32_t box_inner, uint32_t box_rows,
+                         CUtensorMapSwizzle sw);
+
+// ---------------------------------------------------------------- GEMM
+struct GemmDesc {
+  const void* a;   // [M, K] bf16, row stride lda elements
+  long long lda;
+  const void* b;   // dense: [N, K] row stride ldb; grouped: [groups, b_rows, K] contiguous
+  long long ldb;
+  const void* b2;  // SwiGLU "up" weights, same shape as b
+  int M, N, K;
+  int b_rows;      // grouped: rows of each group's B matrix
+  int grouped;
+  const int* offsets;
+  int num_groups;
+  int epi;         // EpiKind
+  int transpose_out;
+  void* out;
+  long long ldo, split_stride;
+  const void* residual;
+  long long ldr;
+  const float* bias;
+  int splits;      // >= 1; more than one only with fp32 partial outputs
+  int bn;          // 0 = automatic
+};
+jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s);
+jamba_status gemm_f32(const GemmDesc& g, cudaStream_t s);
+
+// Splits so that m_tiles * n_tiles * splits fills the SMs, each split keeping
+// at least `min_k_tiles` 64-wide k-steps.
+int choose_splits(int M, int N, int K, int bn, int min_k_tiles);
+
+// ---------------------------------------------------------------- scan
+struct ScanCall {
+  const void* x; long long ld_x;
+  const void* z; long long ld_z;
+  const float* dt; long long ld_dt;
+  const void* B; long long ld_b;
+  const void* C; long long ld_c;
+  int bc_dtype;
+  const float* A; const float* D; const float* h0;
+  void* y; long long ld_y;
+  float* h_out;
+  int batch, L, di, dtype, chunk;
+  void* ws; size_t ws_bytes;
+};
+jamba_status scan_run(const ScanCall& s, cudaStream_t st);
+size_t scan_workspace_bytes(int batch, int L, int di, int chunk_len);
+int scan_auto_chunk(int batch, int L, int di);
+jamba_status ssm_step(const void* xc, const void* z, long long ld_z, const float* dt, const float* bc,
+                      long long ld_bc, const float* A, const float* D, float* state, void* y, int batch, int di,
+                      int dtype, cudaStream_t st);
+
+// ---------------------------------------------------------------- conv / norms
+jamba_status conv_prefill(const void* x, long long ld_x, const void* w, const void* b, void* out,
+                          const float* st_in, float* st_out, int batch, int L, int C, int dtype, cudaStream_t s);
+jamba_status conv_step(const void* x, long long ld_x, const void* w, const void* b, void* out, float* state,
+                       int batch, int C, int dtype, cudaStream_t s);
+jamba_status rmsnorm(const void* x, const float* w, void* out, int rows, int cols, float eps, int dtype,
+                     cudaStream_t s);
+jamba_status xproj_norm(const float* part, int splits, long long split_stride, int T, int R, int N,
+                        const float* w_dt, const float* w_B, const float* w_C, int inner_norm, float eps,
+                        void* dtlow, float* bc, int dtype, cudaStream_t s);
+jamba_status splitk_reduce(const float* part, int splits, long long split_stride, long long n,
+                           const void* residual, void* out, int dtype, cudaStream_t s);
+
+// ---------------------------------------------------------------- MoE
+jamba_status moe_route(const void* x, const void* W, int T, int dm, int E, int K, int* idx, float* w, int* counts,
+                       int* offsets, int* perm, int* inv, cudaStream_t s);
+jamba_status moe_gather(const void* x, const int* perm, int rows, int K, int dm, void* out, cudaStream_t s);
+jamba_status moe_combine(const float* Y, const int* inv, const float* w, int T, int K, int dm, const void* residual,
+                         void* out, cudaStream_t s);
+
+}  // namespace jb

@@ -1,0 +1,201 @@
+// MoE routing: router logits, softmax and top-K, the expert-sorted
+// permutation, the row gather in front of the expert GEMMs and the weighted
+// combine behind them.
+//
+// "Jamba: A Hybrid Transformer-Mamba Language Model" (summary page),
+// section 2: MoE layers with n experts, the router picks the top K per token;
+// section 3.1: n = 16, K = 2.  Expert choice is an integer decided by
+// floating point, so the logits are accumulated in fp64 from products of the
+// bf16 inputs (each product is exact in fp32): the choice then matches the
+// exact-arithmetic one except for logit ties closer than about 1e-13.
+#include "common.cuh"
+#include "host.hpp"
+
+namespace jb {
+
+constexpr int ROUTER_EG = 16;  // experts per register group
+
+// one warp per token
+__global__ void __launch_bounds__(256)
+router_kernel(const bf16* __restrict__ x, const bf16* __restrict__ W, int T, int dm, int E, int K,
+              int* __restrict__ idx_out, float* __restrict__ w_out, int* __restrict__ counts) {
+  const int warps = gridDim.x * 8;
+  const int lane = threadIdx.x & 31;
+  double logit[64];
+  for (int t = blockIdx.x * 8 + (threadIdx.x >> 5); t < T; t += warps) {
+    const bf16* xr = x + (long long)t * dm;
+    for (int e0 = 0; e0 < E; e0 += ROUTER_EG) {
+      double acc[ROUTER_EG];
+#pragma unroll
+      for (int e = 0; e < ROUTER_EG; ++e) acc[e] = 0.0;
+      for (int k0 = lane * 8; k0 < dm; k0 += 256) {
+        const uint4 xv = *reinterpret_cast<const uint4*>(xr + k0);
+        const __nv_bfloat162* xh = reinterpret_cast<const __nv_bfloat162*>(&xv);
+        float xf[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __bfloat1622float2(xh[i]);
+          xf[2 * i] = f.x;
+          xf[2 * i + 1] = f.y;
+        }
+#pragma unroll
+        for (int e = 0; e < ROUTER_EG; ++e) {
+          if (e0 + e >= E) break;
+          const uint4 wv = __ldg(reinterpret_cast<const uint4*>(W + (long long)(e0 + e) * dm + k0));
+          const __nv_bfloat162* wh = reinterpret_cast<const __nv_bfloat162*>(&wv);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(wh[i]);
+            acc[e] += (double)(xf[2 * i] * f.x);      // exact product of two bf16 values
+            acc[e] += (double)(xf[2 * i + 1] * f.y);
+          }
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < ROUTER_EG; ++e) {
+        double v = acc[e];
+#pragma unroll
+        for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (e0 + e < E) logit[e0 + e] = v;
+      }
+    }
+    if (lane == 0) {
+      double mx = logit[0];
+      for (int e = 1; e < E; ++e) mx = logit[e] > mx ? logit[e] : mx;
+      double den = 0.0;
+      for (int e = 0; e < E; ++e) den += exp(logit[e] - mx);
+      unsigned long long taken = 0ull;
+      for (int k = 0; k < K; ++k) {
+        int best = -1;
+        for (int e = 0; e < E; ++e) {
+          if (taken >> e & 1ull) continue;
+          if (best < 0 || logit[e] > logit[best]) best = e;  // strict: ties keep the lower index
+        }
+        taken |= 1ull << best;
+        idx_out[(long long)t * K + k] = best;
+        w_out[(long long)t * K + k] = (float)(exp(logit[best] - mx) / den);
+        atomicAdd(counts + best, 1);
+      }
+    }
+  }
+}
+
+// One block per expert: stable positions of that expert's (token, slot)
+// pairs in flat order, i.e. routed rows sorted by (expert, token, slot).
+__global__ void __launch_bounds__(1024)
+permute_kernel(const int* __restrict__ idx, int TK, int E, const int* __restrict__ counts, int* __restrict__ offsets,
+               int* __restrict__ perm, int* __restrict__ inv) {
+  const int e = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  __shared__ int s_warp[32];
+  __shared__ int s_base;
+  if (tid == 0) {
+    int o = 0;
+    for (int i = 0; i < e; ++i) o += counts[i];
+    s_base = o;
+    if (e == 0) {
+      int acc = 0;
+      offsets[0] = 0;
+      for (int i = 0; i < E; ++i) {
+        acc += counts[i];
+        offsets[i + 1] = acc;
+      }
+    }
+  }
+  __syncthreads();
+  int run = s_base;
+  for (int f0 = 0; f0 < TK; f0 += 1024) {
+    const int f = f0 + tid;
+    const bool hit = f < TK && idx[f] == e;
+    const unsigned bal = __ballot_sync(0xffffffffu, hit);
+    if (lane == 0) s_warp[warp] = __popc(bal);
+    __syncthreads();
+    if (warp == 0) {
+      const int v = s_warp[lane];
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+      }
+      s_warp[lane] = incl - v;  // exclusive prefix per warp
+      if (lane == 31) s_base = incl;  // block total (read after the next barrier)
+    }
+    __syncthreads();
+    if (hit) {
+      const int pos = run + s_warp[warp] + __popc(bal & ((1u << lane) - 1u));
+      perm[pos] = f;
+      inv[f] = pos;
+    }
+    run += s_base;
+    __syncthreads();
+  }
+}
+
+// routed row p <- token perm[p] / K
+__global__ void __launch_bounds__(256)
+gather_rows_kernel(const bf16* __restrict__ x, const int* __restrict__ perm, int K, int dm, bf16* __restrict__ out) {
+  const long long p = blockIdx.x;
+  const int t = perm[p] / K;
+  const uint4* src = reinterpret_cast<const uint4*>(x + (long long)t * dm);
+  uint4* dst = reinterpret_cast<uint4*>(out + p * dm);
+  for (int i = threadIdx.x; i < dm / 8; i += 256) dst[i] = src[i];
+}
+
+// out[t] = residual[t] + sum_k w[t, k] * Y[inv[t K + k]], slot 0 first, fp32
+__global__ void __launch_bounds__(256)
+combine_kernel(const float* __restrict__ Y, const int* __restrict__ inv, const float* __restrict__ w, int K, int dm,
+               const bf16* __restrict__ residual, bf16* __restrict__ out) {
+  const long long t = blockIdx.x;
+  for (int c = threadIdx.x * 4; c < dm; c += 1024) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int k = 0; k < K; ++k) {
+      const float wk = w[t * K + k];
+      const float4 y = *reinterpret_cast<const float4*>(Y + (long long)inv[t * K + k] * dm + c);
+      acc[0] = fmaf(wk, y.x, acc[0]);
+      acc[1] = fmaf(wk, y.y, acc[1]);
+      acc[2] = fmaf(wk, y.z, acc[2]);
+      acc[3] = fmaf(wk, y.w, acc[3]);
+    }
+    __nv_bfloat162 o[2];
+    float r[4] = {0.f, 0.f, 0.f, 0.f};
+    if (residual) {
+      const uint2 rv = *reinterpret_cast<const uint2*>(residual + t * dm + c);
+      const __nv_bfloat162* rh = reinterpret_cast<const __nv_bfloat162*>(&rv);
+      const float2 a = __bfloat1622float2(rh[0]), b = __bfloat1622float2(rh[1]);
+      r[0] = a.x; r[1] = a.y; r[2] = b.x; r[3] = b.y;
+    }
+    o[0] = __floats2bfloat162_rn(acc[0] + r[0], acc[1] + r[1]);
+    o[1] = __floats2bfloat162_rn(acc[2] + r[2], acc[3] + r[3]);
+    *reinterpret_cast<uint2*>(out + t * dm + c) = *reinterpret_cast<uint2*>(o);
+  }
+}
+
+jamba_status moe_route(const void* x, const void* W, int T, int dm, int E, int K, int* idx, float* w, int* counts,
+                       int* offsets, int* perm, int* inv, cudaStream_t s) {
+  JB_CUDA(cudaMemsetAsync(counts, 0, sizeof(int) * E, s));
+  int blocks = (T + 7) / 8;
+  const int cap = 8 * num_sms();
+  if (blocks > cap) blocks = cap;
+  router_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const bf16*>(x), reinterpret_cast<const bf16*>(W), T, dm, E,
+                                       K, idx, w, counts);
+  JB_CUDA(cudaGetLastError());
+  permute_kernel<<<E, 1024, 0, s>>>(idx, T * K, E, counts, offsets, perm, inv);
+  JB_CUDA(cudaGetLastError());
+  return JAMBA_OK;
+}
+
+jamba_status moe_gather(const void* x, const int* perm, int rows, int K, int dm, void* out, cudaStream_t s) {
+  gather_rows_kernel<<<rows, 256, 0, s>>>(reinterpret_cast<const bf16*>(x), perm, K, dm, reinterpret_cast<bf16*>(out));
+  JB_CUDA(cudaGetLastError());
+  return JAMBA_OK;
+}
+
+jamba_status moe_combine(const float* Y, const int* inv, const float* w, int T, int K, int dm, const void* residual,
+                         void* out, cudaStream_t s) {
+  combine_kernel<<<T, 256, 0, s>>>(Y, inv, w, K, dm, reinterpret_cast<const bf16*>(residual),
+                                   reinterpret_cast<bf16*>(out));
+  JB_CUDA(cudaGetLastError());
+  return JAMBA_OK;
+}
+
+}  // namespace jb

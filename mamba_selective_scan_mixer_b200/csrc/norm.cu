@@ -1,0 +1,154 @@
+// RMSNorms and split-K reductions.
+//
+// Jamba ("Jamba: A Hybrid Transformer-Mamba Language Model", section 2 and
+// section 6.4 / figure 9) adds RMSNorm inside the Mamba layer; here it acts on
+// the three parts of the x_proj output separately (dt_low over dt_rank
+// columns, B and C over d_state columns each), fused with the sum of the
+// split-K partials of x_proj.  The block RMSNorm in front of the mixer and the
+// MoE is a plain row norm.
+#include "common.cuh"
+#include "host.hpp"
+
+namespace jb {
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// one 256-thread block per row
+template <typename T>
+__global__ void __launch_bounds__(256)
+rmsnorm_kernel(const T* __restrict__ x, const float* __restrict__ w, T* __restrict__ out, int cols, float eps) {
+  const long long row = blockIdx.x;
+  const T* xr = x + row * cols;
+  T* orow = out + row * cols;
+  float ss = 0.f;
+  for (int c = threadIdx.x; c < cols; c += 256) {
+    const float v = to_f(xr[c]);
+    ss = fmaf(v, v, ss);
+  }
+  __shared__ float red[8];
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < 8 ? red[threadIdx.x] : 0.f;
+    v = warp_sum(v);
+    if (threadIdx.x == 0) red[0] = v;
+  }
+  __syncthreads();
+  const float inv = rsqrtf(red[0] / (float)cols + eps);
+  for (int c = threadIdx.x; c < cols; c += 256) orow[c] = from_f<T>(to_f(xr[c]) * inv * w[c]);
+}
+
+// x_proj output: sum the split-K partials [splits][T][R + 2N], then the three
+// inner RMSNorms; dt_low goes out in the GEMM dtype, B | C in fp32.
+template <typename TD>
+__global__ void __launch_bounds__(256)
+xproj_norm_kernel(const float* __restrict__ part, int splits, long long split_stride, int T, int R, int N,
+                  const float* __restrict__ w_dt, const float* __restrict__ w_B, const float* __restrict__ w_C,
+                  int inner_norm, float eps, TD* __restrict__ dtlow, float* __restrict__ bc) {
+  const int warp = (blockIdx.x * 256 + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= T) return;
+  const int W = R + 2 * N;
+  constexpr int MAXPER = 16;  // up to 512 columns
+  float v[MAXPER];
+  float s_dt = 0.f, s_b = 0.f, s_c = 0.f;
+#pragma unroll
+  for (int k = 0; k < MAXPER; ++k) {
+    const int col = lane + 32 * k;
+    float acc = 0.f;
+    if (col < W) {
+      for (int s = 0; s < splits; ++s) acc += part[s * split_stride + (long long)warp * W + col];
+      if (col < R) s_dt = fmaf(acc, acc, s_dt);
+      else if (col < R + N) s_b = fmaf(acc, acc, s_b);
+      else s_c = fmaf(acc, acc, s_c);
+    }
+    v[k] = acc;
+  }
+  float i_dt = 1.f, i_b = 1.f, i_c = 1.f;
+  if (inner_norm) {
+    i_dt = rsqrtf(warp_sum(s_dt) / (float)R + eps);
+    i_b = rsqrtf(warp_sum(s_b) / (float)N + eps);
+    i_c = rsqrtf(warp_sum(s_c) / (float)N + eps);
+  }
+#pragma unroll
+  for (int k = 0; k < MAXPER; ++k) {
+    const int col = lane + 32 * k;
+    if (col >= W) continue;
+    if (col < R) {
+      const float o = inner_norm ? v[k] * i_dt * w_dt[col] : v[k];
+      dtlow[(long long)warp * R + col] = from_f<TD>(o);
+    } else if (col < R + N) {
+      bc[(long long)warp * 2 * N + (col - R)] = inner_norm ? v[k] * i_b * w_B[col - R] : v[k];
+    } else {
+      bc[(long long)warp * 2 * N + (col - R)] = inner_norm ? v[k] * i_c * w_C[col - R - N] : v[k];
+    }
+  }
+}
+
+// out[r, c] = sum_s part[s][r][c] (+ residual[r, c])
+template <typename T>
+__global__ void __launch_bounds__(256)
+splitk_reduce_kernel(const float* __restrict__ part, int splits, long long split_stride, long long n,
+                     const T* __restrict__ residual, T* __restrict__ out) {
+  const long long i = ((long long)blockIdx.x * 256 + threadIdx.x) * 4;
+  if (i >= n) return;
+  float4 acc = *reinterpret_cast<const float4*>(part + i);
+  for (int s = 1; s < splits; ++s) {
+    const float4 p = *reinterpret_cast<const float4*>(part + s * split_stride + i);
+    acc.x += p.x; acc.y += p.y; acc.z += p.z; acc.w += p.w;
+  }
+  float r[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    if (residual) r[k] += to_f(residual[i + k]);
+    out[i + k] = from_f<T>(r[k]);
+  }
+}
+
+jamba_status rmsnorm(const void* x, const float* w, void* out, int rows, int cols, float eps, int dtype,
+                     cudaStream_t s) {
+  if (dtype == JAMBA_BF16)
+    rmsnorm_kernel<bf16><<<rows, 256, 0, s>>>(reinterpret_cast<const bf16*>(x), w, reinterpret_cast<bf16*>(out),
+                                             cols, eps);
+  else
+    rmsnorm_kernel<float><<<rows, 256, 0, s>>>(reinterpret_cast<const float*>(x), w, reinterpret_cast<float*>(out),
+                                              cols, eps);
+  JB_CUDA(cudaGetLastError());
+  return JAMBA_OK;
+}
+
+jamba_status xproj_norm(const float* part, int splits, long long split_stride, int T, int R, int N,
+                        const float* w_dt, const float* w_B, const float* w_C, int inner_norm, float eps,
+                        void* dtlow, float* bc, int dtype, cudaStream_t s) {
+  if (R + 2 * N > 512) return fail(JAMBA_ERR_UNSUPPORTED, "x_proj width above 512");
+  const unsigned grid = (unsigned)(((long long)T * 32 + 255) / 256);
+  if (dtype == JAMBA_BF16)
+    xproj_norm_kernel<bf16><<<grid, 256, 0, s>>>(part, splits, split_stride, T, R, N, w_dt, w_B, w_C, inner_norm,
+                                                eps, reinterpret_cast<bf16*>(dtlow), bc);
+  else
+    xproj_norm_kernel<float><<<grid, 256, 0, s>>>(part, splits, split_stride, T, R, N, w_dt, w_B, w_C, inner_norm,
+                                                 eps, reinterpret_cast<float*>(dtlow), bc);
+  JB_CUDA(cudaGetLastError());
+  return JAMBA_OK;
+}
+
+jamba_status splitk_reduce(const float* part, int splits, long long split_stride, long long n,
+                           const void* residual, void* out, int dtype, cudaStream_t s) {
+  if (n % 4) return fail(JAMBA_ERR_INVALID_ARG, "split-K reduce: size must be a multiple of 4");
+  const unsigned grid = (unsigned)((n / 4 + 255) / 256);
+  if (dtype == JAMBA_BF16)
+    splitk_reduce_kernel<bf16><<<grid, 256, 0, s>>>(part, splits, split_stride, n,
+                                                   reinterpret_cast<const bf16*>(residual), reinterpret_cast<bf16*>(out));
+  else
+    splitk_reduce_kernel<float><<<grid, 256, 0, s>>>(part, splits, split_stride, n,
+                                                    reinterpret_cast<const float*>(residual),
+                                                    reinterpret_cast<float*>(out));
+  JB_CUDA(cudaGetLastError());
+  return JAMBA_OK;
+}
+
+}  // namespace jb

@@ -1,0 +1,232 @@
+"""Torch-tensor front end of the C ABI (marshalling only).
+
+Tensors must already live on the CUDA device; workspaces are allocated with
+torch and passed down as raw pointers.  Names follow include/jamba.h.
+"""
+import ctypes
+
+import torch
+
+from . import _abi
+from ._abi import check, lib
+
+_DT = {torch.bfloat16: _abi.JAMBA_BF16, torch.float32: _abi.JAMBA_F32}
+_TORCH_DT = {"bf16": torch.bfloat16, "f32": torch.float32}
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("libjamba works on CUDA tensors only")
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _contig(t, name):
+    if t is not None and not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+class _Workspace:
+    def __init__(self):
+        self.buf = None
+
+    def get(self, nbytes, device):
+        if self.buf is None or self.buf.numel() < nbytes or self.buf.device != device:
+            self.buf = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+        return self.buf
+
+
+def device_status(stream=None):
+    """Synchronizes the stream and raises if a kernel's bounded wait gave up."""
+    check(lib().jamba_device_status(_stream(stream)))
+
+
+class MambaMixer:
+    """One Mamba mixer layer (prefill and decode) over borrowed weight tensors.
+
+    params: dict with in_proj, conv_w, conv_b, x_proj, dt_proj, dt_bias, A, D,
+    out_proj, norm_dt, norm_B, norm_C (the layout of jamba_mamba_weights).
+    """
+
+    def __init__(self, params, shape):
+        self.shape = shape
+        self.dtype = _TORCH_DT[shape.dtype]
+        self.params = {k: v.contiguous() for k, v in params.items()}
+        _cuda(*self.params.values())
+        self.device = self.params["in_proj"].device
+        cfg = _abi.MambaConfig(shape.d_model, shape.d_inner, shape.d_state, shape.d_conv, shape.dt_rank,
+                               _DT[self.dtype], int(shape.inner_norm), float(shape.eps))
+        w = _abi.MambaWeights(*[ctypes.c_void_p(self.params[k].data_ptr()) for k in
+                                ("in_proj", "conv_w", "conv_b", "x_proj", "dt_proj", "dt_bias", "A", "D",
+                                 "out_proj", "norm_dt", "norm_B", "norm_C")])
+        self._cfg = cfg
+        h = ctypes.c_void_p()
+        with torch.cuda.device(self.device):
+            check(lib().jamba_mamba_create(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(h)))
+        self.handle = h
+        self.ws = _Workspace()
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h is not None and h.value and _abi._lib is not None:
+            _abi._lib.jamba_mamba_destroy(h)
+            self.handle = None
+
+    def workspace_size(self, batch, seqlen):
+        n = ctypes.c_size_t()
+        check(lib().jamba_mamba_workspace_size(self.handle, batch, seqlen, ctypes.byref(n)))
+        return n.value
+
+    def new_states(self, batch):
+        sh = self.shape
+        return (torch.zeros(batch, sh.d_inner, sh.d_conv - 1, device=self.device),
+                torch.zeros(batch, sh.d_inner, sh.d_state, device=self.device))
+
+    def prefill(self, u, residual=None, conv_state_in=None, ssm_state_in=None, conv_state_out=None,
+                ssm_state_out=None, out=None, stream=None):
+        """u [B, L, d_model] -> (out, conv_state_out, ssm_state_out)."""
+        _cuda(u, residual)
+        _contig(u, "u")
+        _contig(residual, "residual")
+        B, L, _ = u.shape
+        if out is None:
+            out = torch.empty_like(u)
+        if conv_state_out is None or ssm_state_out is None:
+            cs, ss = self.new_states(B)
+            conv_state_out = cs if conv_state_out is None else conv_state_out
+            ssm_state_out = ss if ssm_state_out is None else ssm_state_out
+        nbytes = self.workspace_size(B, L)
+        ws = self.ws.get(nbytes, u.device)
+        check(lib().jamba_mamba_prefill(self.handle, _p(u), _p(residual), _p(out), B, L, _p(conv_state_in),
+                                        _p(ssm_state_in), _p(conv_state_out), _p(ssm_state_out), _p(ws),
+                                        ws.numel(), _stream(stream)))
+        return out, conv_state_out, ssm_state_out
+
+    def step(self, u, conv_state, ssm_state, residual=None, out=None, stream=None):
+        """u [B, d_model]; updates both caches in place; returns out [B, d_model]."""
+        _cuda(u, conv_state, ssm_state, residual)
+        _contig(u, "u")
+        B = u.shape[0]
+        if out is None:
+            out = torch.empty_like(u)
+        nbytes = self.workspace_size(B, 1)
+        ws = self.ws.get(nbytes, u.device)
+        check(lib().jamba_mamba_step(self.handle, _p(u), _p(residual), _p(out), B, _p(conv_state),
+                                     _p(ssm_state), _p(ws), ws.numel(), _stream(stream)))
+        return out
+
+
+def selective_scan(x, z, dt, B, C, A, D, h0=None, chunk=0, want_state=True, y=None, ws=None, stream=None):
+    """x, z, dt [batch, L, d_inner] (row strides taken from the tensors);
+    B, C [batch, L, 16]; A [d_inner, 16]; D [d_inner]; h0 [batch, d_inner, 16] or None.
+    Returns (y, h_out)."""
+    _cuda(x, z, dt, B, C, A, D, h0)
+    batch, L, di = x.shape
+    N = A.shape[1]
+    for t, n in ((x, "x"), (z, "z"), (dt, "dt"), (B, "B"), (C, "C")):
+        if t.stride(-1) != 1 or t.stride(0) != L * t.stride(1):
+            raise ValueError("%s: rows must be unit-stride and evenly spaced" % n)
+    if y is None:
+        y = torch.empty(batch, L, di, dtype=x.dtype, device=x.device)
+    h_out = torch.empty(batch, di, N, dtype=torch.float32, device=x.device) if want_state else None
+    n = ctypes.c_size_t()
+    check(lib().jamba_selective_scan_workspace_size(batch, L, di, N, chunk, ctypes.byref(n)))
+    if ws is None or ws.numel() < n.value:
+        ws = torch.empty(max(n.value, 256), dtype=torch.uint8, device=x.device)
+    check(lib().jamba_selective_scan(_p(x), x.stride(1), _p(z), z.stride(1), _p(dt), dt.stride(1), _p(B),
+                                     B.stride(1), _p(C), C.stride(1), _DT[B.dtype], _p(A), _p(D), _p(h0),
+                                     _p(y), y.stride(1), _p(h_out), batch, L, di, N, _DT[x.dtype], chunk,
+                                     _p(ws), ws.numel(), _stream(stream)))
+    return y, h_out
+
+
+def rmsnorm(x, w, eps=1e-6, out=None, stream=None):
+    _cuda(x, w)
+    _contig(x, "x")
+    out = torch.empty_like(x) if out is None else out
+    cols = x.shape[-1]
+    check(lib().jamba_rmsnorm(_p(x), _p(w), _p(out), x.numel() // cols, cols, float(eps), _DT[x.dtype],
+                              _stream(stream)))
+    return out
+
+
+def causal_conv1d(x, w, b, state_in=None, want_state=True, stream=None):
+    """x [batch, L, C] (row stride from the tensor) -> (SiLU(conv), state_out)."""
+    _cuda(x, w, b, state_in)
+    batch, L, C = x.shape
+    out = torch.empty(batch, L, C, dtype=x.dtype, device=x.device)
+    st = torch.empty(batch, C, 3, dtype=torch.float32, device=x.device) if want_state else None
+    check(lib().jamba_causal_conv1d(_p(x), x.stride(1), _p(w), _p(b), _p(out), _p(state_in), _p(st), batch, L,
+                                    C, _DT[x.dtype], _stream(stream)))
+    return out, st
+
+
+def gemm(a, b, residual=None, out_dtype=None, out=None, stream=None):
+    """a [m, k] @ b[n, k]^T (+ residual) on the tensor cores (bf16) or CUDA cores (fp32)."""
+    _cuda(a, b, residual, out)
+    _contig(a, "a")
+    _contig(b, "b")
+    m, k = a.shape
+    n = b.shape[0]
+    od = out.dtype if out is not None else (out_dtype or a.dtype)
+    if out is None:
+        out = torch.empty(m, n, dtype=od, device=a.device)
+    _contig(out, "out")
+    check(lib().jamba_gemm(_p(a), _p(b), _p(out), n, _p(residual), m, n, k, _DT[a.dtype], _DT[od],
+                           _stream(stream)))
+    return out
+
+
+class MoE:
+    """Top-K SwiGLU mixture of experts over borrowed weights (router, w_gate, w_up, w_down)."""
+
+    def __init__(self, params, shape):
+        self.shape = shape
+        self.params = {k: v.contiguous() for k, v in params.items()}
+        _cuda(*self.params.values())
+        self.cfg = _abi.MoeConfig(shape.d_model, shape.d_ff, shape.n_experts, shape.top_k, _abi.JAMBA_BF16)
+        self.w = _abi.MoeWeights(*[ctypes.c_void_p(self.params[k].data_ptr())
+                                   for k in ("router", "w_gate", "w_up", "w_down")])
+        self.ws = _Workspace()
+
+    def workspace_size(self, tokens):
+        n = ctypes.c_size_t()
+        check(lib().jamba_moe_workspace_size(ctypes.byref(self.cfg), tokens, ctypes.byref(n)))
+        return n.value
+
+    def forward(self, x, residual=None, out=None, stream=None):
+        """x [T, d_model] -> dict(out, idx, w, offsets, perm)."""
+        _cuda(x, residual)
+        _contig(x, "x")
+        T = x.shape[0]
+        K, E = self.shape.top_k, self.shape.n_experts
+        dev = x.device
+        out = torch.empty_like(x) if out is None else out
+        idx = torch.empty(T, K, dtype=torch.int32, device=dev)
+        w = torch.empty(T, K, dtype=torch.float32, device=dev)
+        offs = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        perm = torch.empty(T * K, dtype=torch.int32, device=dev)
+        ws = self.ws.get(self.workspace_size(T), dev)
+        check(lib().jamba_moe_forward(ctypes.byref(self.cfg), ctypes.byref(self.w), _p(x), _p(residual),
+                                      _p(out), T, _p(idx), _p(w), _p(offs), _p(perm), _p(ws), ws.numel(),
+                                      _stream(stream)))
+        return dict(out=out, idx=idx, w=w, offsets=offs, perm=perm)
+
+
+def layer_pair(mixer, moe, x, g1, g2, eps=1e-6, stream=None):
+    """RMSNorm -> Mamba -> residual -> RMSNorm -> MoE -> residual on x [B, L, d_model]."""
+    B, L, dm = x.shape
+    u = rmsnorm(x, g1, eps, stream=stream)
+    h, _, _ = mixer.prefill(u, residual=x, stream=stream)
+    v = rmsnorm(h, g2, eps, stream=stream)
+    r = moe.forward(v.view(B * L, dm), residual=h.view(B * L, dm), stream=stream)
+    r["h"] = h
+    return r

@@ -1,0 +1,132 @@
+"""Mamba mixer parity through the C ABI: prefill, decode step, caches and the
+step-equals-prefill property, against the fp64 oracle on seeded inputs."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import mamba as om
+from synthetic import MambaShape, decode_inputs, mamba_input, mamba_params, workload
+from tests.helpers import TOL_BF16, TOL_F32, cuda_or_skip, rel_l2, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dev():
+    d = cuda_or_skip()
+    import mamba_selective_scan_mixer_b200 as J
+    J.lib()
+    return d
+
+
+def _mixer(shape, seed, dev, **kw):
+    import mamba_selective_scan_mixer_b200 as J
+    p = mamba_params(shape, seed=seed, **kw)
+    return J.MambaMixer({k: v.to(dev) for k, v in p.items()}, shape), om.params64(p)
+
+
+def test_tiny_fp32_prefill_and_16_steps(dev):
+    """tiny fp32 mixer: prefill of 256 tokens then 16 decode steps, fp32 bar"""
+    wl = workload("tiny_fp32")
+    sh = wl["mamba"]
+    mix, p64 = _mixer(sh, 0, dev)
+    u = mamba_input(sh, 1, wl["seqlen"] + wl["steps"], seed=0)
+    u64 = to_np(u)
+    out, cs, ss = mix.prefill(u[:, :wl["seqlen"]].contiguous().to(dev))
+    ref = om.mamba_prefill(p64, u64[:, :wl["seqlen"]], sh)
+    assert rel_l2(to_np(out), ref["out"]) < TOL_F32
+    assert rel_l2(to_np(cs), ref["conv_state"]) < TOL_F32
+    assert rel_l2(to_np(ss), ref["ssm_state"]) < TOL_F32
+    rcs, rss = ref["conv_state"], ref["ssm_state"]
+    outs, wants = [], []
+    for t in range(wl["steps"]):
+        o = mix.step(u[:, wl["seqlen"] + t].contiguous().to(dev), cs, ss)
+        w, rcs, rss = om.mamba_step(p64, u64[:, wl["seqlen"] + t], sh, rcs, rss)
+        outs.append(to_np(o))
+        wants.append(w)
+    assert rel_l2(np.stack(outs), np.stack(wants)) < TOL_F32
+    assert rel_l2(to_np(ss), rss) < TOL_F32
+    assert rel_l2(to_np(cs), rcs) < TOL_F32
+
+
+@pytest.mark.parametrize("inner_norm", [True, False])
+def test_bf16_prefill_small_widths(dev, inner_norm):
+    sh = MambaShape(d_model=256, d_inner=512, dt_rank=32, dtype="bf16", inner_norm=inner_norm)
+    mix, p64 = _mixer(sh, 1, dev, norm_init="random", d_init="random")
+    u = mamba_input(sh, 2, 300, seed=1)
+    out, cs, ss = mix.prefill(u.to(dev))
+    ref = om.mamba_prefill(p64, to_np(u), sh)
+    assert rel_l2(to_np(out), ref["out"]) < TOL_BF16
+    assert rel_l2(to_np(ss), ref["ssm_state"]) < TOL_BF16
+    assert rel_l2(to_np(cs), ref["conv_state"]) < TOL_BF16
+
+
+def test_bf16_prefill_residual_and_continuation(dev):
+    """prefill continues from given caches; residual added in the out_proj epilogue"""
+    sh = MambaShape(d_model=256, d_inner=512, dt_rank=32, dtype="bf16")
+    mix, p64 = _mixer(sh, 2, dev, a_init="random")
+    u = mamba_input(sh, 1, 200, seed=2)
+    res = mamba_input(sh, 1, 200, seed=3)
+    ud = u.to(dev)
+    _, cs, ss = mix.prefill(ud[:, :120].contiguous())
+    out, cs2, ss2 = mix.prefill(ud[:, 120:].contiguous(), residual=res[:, 120:].contiguous().to(dev),
+                                conv_state_in=cs, ssm_state_in=ss)
+    ref = om.mamba_prefill(p64, to_np(u), sh)
+    assert rel_l2(to_np(out), ref["out"][:, 120:] + to_np(res)[:, 120:]) < TOL_BF16
+    assert rel_l2(to_np(ss2), ref["ssm_state"]) < TOL_BF16
+    # in-place continuation: caches in == out
+    cs3, ss3 = cs.clone(), ss.clone()
+    mix.prefill(ud[:, 120:].contiguous(), conv_state_in=cs3, ssm_state_in=ss3, conv_state_out=cs3,
+                ssm_state_out=ss3)
+    assert torch.equal(cs3, cs2)
+    assert rel_l2(to_np(ss3), to_np(ss2)) < 1e-6
+
+
+def test_bf16_decode_steps_match_oracle_and_prefill(dev):
+    sh = MambaShape(d_model=512, d_inner=1024, dt_rank=64, dtype="bf16")
+    mix, p64 = _mixer(sh, 4, dev)
+    B, L0, S = 5, 40, 12
+    u = mamba_input(sh, B, L0, seed=4)
+    steps = decode_inputs(sh, B, S, seed=4)
+    _, cs, ss = mix.prefill(u.to(dev))
+    outs = [to_np(mix.step(steps[t].to(dev), cs, ss)) for t in range(S)]
+    full = torch.cat([u, steps.transpose(0, 1)], dim=1)
+    ref = om.mamba_prefill(p64, to_np(full), sh)
+    assert rel_l2(np.stack(outs, 1), ref["out"][:, L0:]) < TOL_BF16
+    assert rel_l2(to_np(ss), ref["ssm_state"]) < TOL_BF16
+    # GPU step == GPU prefill of the longer sequence
+    out_full, _, ss_full = mix.prefill(full.contiguous().to(dev))
+    assert rel_l2(np.stack(outs, 1), to_np(out_full)[:, L0:]) < TOL_BF16
+
+
+@pytest.mark.slow
+def test_prefill_4k_full_width(dev):
+    """Jamba-width prefill of 4096 tokens with inner RMSNorm, whole output vs the oracle"""
+    wl = workload("prefill_4k")
+    sh = wl["mamba"]
+    mix, p64 = _mixer(sh, 0, dev)
+    u = mamba_input(sh, wl["batch"], wl["seqlen"], seed=0)
+    out, cs, ss = mix.prefill(u.to(dev))
+    ref = om.mamba_prefill(p64, to_np(u), sh, scan="c")
+    assert rel_l2(to_np(out), ref["out"]) < TOL_BF16
+    assert rel_l2(to_np(ss), ref["ssm_state"]) < TOL_BF16
+
+
+@pytest.mark.slow
+def test_decode_b64_full_width_sampled_rows(dev):
+    """batch-64 decode at Jamba width: 2048-token prefill then steps; sampled batch
+    rows checked against the oracle's prefill of the same token sequence"""
+    wl = workload("decode_b64")
+    sh = wl["mamba"]
+    mix, p64 = _mixer(sh, 0, dev)
+    B, L0, S = wl["batch"], wl["prefill"], 32
+    u = mamba_input(sh, B, L0, seed=0)
+    steps = decode_inputs(sh, B, S, seed=0)
+    _, cs, ss = mix.prefill(u.to(dev))
+    sd = steps.to(dev)
+    outs = torch.stack([mix.step(sd[t], cs, ss) for t in range(S)], 1)
+    rows = [0, 37, 63]
+    full = torch.cat([u[rows], steps[:, rows].transpose(0, 1)], dim=1)
+    ref = om.mamba_prefill(p64, to_np(full), sh, scan="c")
+    assert rel_l2(to_np(outs[rows]), ref["out"][:, L0:]) < TOL_BF16
+    assert rel_l2(to_np(ss[rows]), ref["ssm_state"]) < TOL_BF16
