@@ -49,7 +49,7 @@ PrefillWs carve_prefill(const jamba_mamba_config& c, int batch, int L, void* ws)
   const int es = esize(c.dtype);
   const int W = c.dt_rank + 2 * c.d_state;
   p.splits = c.dtype == JAMBA_BF16 ? choose_splits((int)T, W, c.d_inner, 144, 8) : 1;
-  p.chunk = scan_auto_chunk(batch, L, c.d_inner);
+  p.chunk = scan_auto_chunk(batch, L, c.d_inner, c.dtype, JAMBA_F32);
   Carver cv(ws);
   p.xz = cv.take(T * 2 * c.d_inner * es);
   p.xc = cv.take(T * c.d_inner * es);
@@ -336,8 +336,15 @@ jamba_status jamba_selective_scan_workspace_size(int batch, int seqlen, int d_in
                                                  size_t* bytes) {
   if (!bytes || batch <= 0 || seqlen <= 0 || d_inner <= 0) return fail(JAMBA_ERR_INVALID_ARG, "scan workspace: bad argument");
   if (d_state != 16) return fail(JAMBA_ERR_UNSUPPORTED, "d_state must be 16");
-  if (chunk == 0) chunk = scan_auto_chunk(batch, seqlen, d_inner);
   if (chunk < 0 || chunk % 16) return fail(JAMBA_ERR_INVALID_ARG, "chunk must be a multiple of 16");
+  // the automatic chunk does not depend on the dtypes by more than the
+  // resident-CTA count; size for the smallest chunk any dtype would pick
+  if (chunk == 0) {
+    const int a = scan_auto_chunk(batch, seqlen, d_inner, JAMBA_BF16, JAMBA_BF16);
+    const int b = scan_auto_chunk(batch, seqlen, d_inner, JAMBA_BF16, JAMBA_F32);
+    const int c = scan_auto_chunk(batch, seqlen, d_inner, JAMBA_F32, JAMBA_F32);
+    chunk = a < b ? (a < c ? a : c) : (b < c ? b : c);
+  }
   *bytes = scan_workspace_bytes(batch, seqlen, d_inner, chunk);
   return JAMBA_OK;
 }
@@ -361,7 +368,7 @@ jamba_status jamba_selective_scan(const void* x, int ld_x, const void* z, int ld
   JB_TRY(check_ptr(h0, "h0", false));
   JB_TRY(check_ptr(y, "y"));
   JB_TRY(check_ptr(h_out, "h_out", false));
-  if (chunk == 0) chunk = scan_auto_chunk(batch, seqlen, d_inner);
+  if (chunk == 0) chunk = scan_auto_chunk(batch, seqlen, d_inner, dtype, bc_dtype);
   ScanCall sc = {};
   sc.x = x; sc.ld_x = ld_x; sc.z = z; sc.ld_z = ld_z; sc.dt = dt; sc.ld_dt = ld_dt;
   sc.B = B; sc.ld_b = ld_b; sc.C = C; sc.ld_c = ld_c; sc.bc_dtype = bc_dtype;

@@ -128,9 +128,12 @@ __device__ __forceinline__ void epi_chunk(const GemmParams& p, const TileInfo& t
           }
           store_bf16x8(o + nn, w);
         } else {
-          for (int i = 0; i < 8 && nn + i < p.N; ++i) {
-            float w = v[c + i] + (r ? __bfloat162float(r[nn + i]) : 0.f);
-            o[nn + i] = __float2bfloat16_rn(w);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            if (nn + i < p.N) {
+              const float w = v[c + i] + (r ? __bfloat162float(r[nn + i]) : 0.f);
+              o[nn + i] = __float2bfloat16_rn(w);
+            }
           }
         }
       }
@@ -149,7 +152,9 @@ __device__ __forceinline__ void epi_chunk(const GemmParams& p, const TileInfo& t
         if (nn + 4 <= p.N) {
           *reinterpret_cast<float4*>(o + nn) = make_float4(w[0], w[1], w[2], w[3]);
         } else {
-          for (int i = 0; i < 4 && nn + i < p.N; ++i) o[nn + i] = w[i];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            if (nn + i < p.N) o[nn + i] = w[i];
         }
       }
     }
@@ -157,13 +162,13 @@ __device__ __forceinline__ void epi_chunk(const GemmParams& p, const TileInfo& t
     // swap-AB: row m is an output feature, column n a token; lanes hold consecutive m
     if (p.epi == EPI_BF16) {
       bf16* o = reinterpret_cast<bf16*>(p.out);
-#pragma unroll 8
+#pragma unroll
       for (int c = 0; c < 32; ++c)
         if (n + c < p.N) o[(long long)(n + c) * p.ldo + m] = __float2bfloat16_rn(v[c]);
     } else {
       float* o = reinterpret_cast<float*>(p.out) + (long long)ti.split * p.split_stride;
       const float b = (p.epi == EPI_SOFTPLUS) ? __ldg(p.bias + m) : 0.f;
-#pragma unroll 8
+#pragma unroll
       for (int c = 0; c < 32; ++c) {
         if (n + c < p.N) {
           float w = v[c];
@@ -331,9 +336,13 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
               float w[8];
 #pragma unroll
               for (int i = 0; i < 8; ++i) w[i] = silu(g[c + i]) * u[c + i];
-              if (n + c + 8 <= p.N) store_bf16x8(o + n + c, w);
-              else
-                for (int i = 0; i < 8 && n + c + i < p.N; ++i) o[n + c + i] = __float2bfloat16_rn(w[i]);
+              if (n + c + 8 <= p.N) {
+                store_bf16x8(o + n + c, w);
+              } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                  if (n + c + i < p.N) o[n + c + i] = __float2bfloat16_rn(w[i]);
+              }
             }
           }
         }

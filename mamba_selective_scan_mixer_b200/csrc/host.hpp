@@ -87,7 +87,7 @@ struct ScanCall {
 };
 jamba_status scan_run(const ScanCall& s, cudaStream_t st);
 size_t scan_workspace_bytes(int batch, int L, int di, int chunk_len);
-int scan_auto_chunk(int batch, int L, int di);
+int scan_auto_chunk(int batch, int L, int di, int dtype, int bc_dtype);
 jamba_status ssm_step(const void* xc, const void* z, long long ld_z, const float* dt, const float* bc,
                       long long ld_bc, const float* A, const float* D, float* state, void* y, int batch, int di,
                       int dtype, cudaStream_t st);

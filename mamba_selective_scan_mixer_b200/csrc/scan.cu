@@ -6,22 +6,31 @@
 // state n:  h_t = exp(dt_t A) h_{t-1} + dt_t B_t x_t,
 //           y_t = (C_t . h_t + D x_t) * SiLU(z_t).
 //
-// Prefill kernel layout: a CTA owns 256 channels (2 per thread, all 16 states
-// of each in fp32 registers) of one batch row and one time chunk.  x, z, dt, B
-// and C arrive through a 4-stage TMA ring of 4-step tiles.  Chunks run
-// concurrently; CTAs take tickets in (chunk, group) order and pass the state
-// between chunks with a decoupled look-back over per-chunk records
-// (aggregate: decay product P and local end state; inclusive: true end state).
-// Until the carried-in state is known, a chunk's outputs depend on it through
-// C_t . (P_t * h_in); those steps are written as fp32 pre-gate values and
-// finished once h_in arrives.  P_t only shrinks towards zero: once it is
-// exactly zero for every channel of a warp, later steps no longer depend on
-// h_in and are gated and stored directly.
+// Prefill kernel.  A CTA owns 256 channels of one batch row over one time
+// chunk: four consumer warps (2 channels per thread, all 16 states of each
+// in fp32 registers, packed fp32x2 arithmetic) and one producer warp that
+// streams x, z, dt, B, C through a 3-stage ring of 8-step TMA tiles and widens
+// B|C to fp32.  Consumers never meet at a CTA barrier inside the time loop.
 //
-// When every channel of the CTA has A[c, n] == (n + 1) * A[c, 0] (the
-// initialisation used by Mamba layers), exp(dt A_n) = r^(n+1) with
-// r = exp(dt A_0): one exponential and 15 products per step instead of 16
-// exponentials.  Other A take the general path.
+// Chunks of the same channels run concurrently.  Before the state entering a
+// chunk is known, its outputs depend on it through C_t . (P_t * h_in), P_t the
+// decay product since the chunk start.  P_t only shrinks, and once it is
+// exactly zero for every channel of a warp the warp's later outputs no longer
+// depend on h_in: the first pass therefore runs the chunk's head (the steps
+// before that point) in state-only mode and writes final outputs after it.
+// At the chunk end the CTA publishes (P, local end state) -- or its true end
+// state if every warp's P died -- and looks back over its predecessors'
+// records (decoupled look-back, (P2, h2) o (P1, h1) = (P2 P1, P2 h1 + h2)).
+// A second pass then replays the head from the true incoming state.  CTAs
+// take tickets in (chunk, group) order, so a predecessor has always started.
+//
+// Decay factors: when every channel of the CTA has A[c, n] == (n + 1) A[c, 0]
+// (the initialisation of Mamba layers) exp(dt A_n) = r^(n+1) with
+// r = exp(dt A_0): one exponential and 15 products per step (bf16 activations
+// only: the power form multiplies the rounding of r by up to 16, which the
+// fp32 path's accuracy bar does not allow).  Other A take the general kernel
+// with one exponential per state.  Both kernels are launched; each CTA runs
+// only if its channels belong to its kind.
 #include <string>
 
 #include "common.cuh"
@@ -29,36 +38,35 @@
 
 namespace jb {
 
-constexpr int SCAN_THREADS = 128;
-constexpr int SCAN_CH = 256;   // channels per CTA (2 per thread)
-constexpr int SCAN_Q = 4;      // time steps per pipeline stage
-constexpr int SCAN_STAGES = 4;
-constexpr int NS = 16;         // d_state
+constexpr int SCAN_CONSUMERS = 128;                 // 4 warps x 32 threads x 2 channels
+constexpr int SCAN_THREADS = SCAN_CONSUMERS + 32;   // + producer warp
+constexpr int SCAN_CH = 256;                        // channels per CTA
+constexpr int SCAN_Q = 8;                           // time steps per stage
+constexpr int SCAN_STAGES = 3;
+constexpr int NS = 16;                              // d_state
 constexpr float LOG2E = 1.4426950408889634f;
+constexpr int REC = 3 * SCAN_CH * NS;               // floats per chunk record: P, h, inclusive h
 
 __host__ __device__ constexpr int al128(int v) { return (v + 127) & ~127; }
 
-template <typename TX, typename TBC>
+template <typename TX, typename TBC, bool FAST>
 struct ScanLayout {
   static constexpr int X = SCAN_Q * SCAN_CH * (int)sizeof(TX);
   static constexpr int DT = SCAN_Q * SCAN_CH * 4;
   static constexpr int BCB = SCAN_Q * NS * (int)sizeof(TBC);
-  static constexpr int STAGE_TX = 2 * X + DT + 2 * BCB;  // bytes landed per stage
+  static constexpr int STAGE_TX = 2 * X + DT + 2 * BCB;  // bytes TMA lands per stage
   static constexpr int OFF_Z = X, OFF_DT = 2 * X, OFF_B = 2 * X + DT, OFF_C = OFF_B + al128(BCB);
-  static constexpr int STAGE = OFF_C + al128(BCB);
-  static constexpr int OFF_BCF = SCAN_STAGES * STAGE;                 // fp32 B|C [STAGES][Q][32]
-  static constexpr int OFF_A2 = OFF_BCF + SCAN_STAGES * SCAN_Q * 32 * 4;  // A*log2(e) [256][16]
-  static constexpr int OFF_BAR = OFF_A2 + SCAN_CH * NS * 4;
-  static constexpr int BYTES = OFF_BAR + 128 + 128;                  // + alignment slack
-  static_assert(SCAN_Q * 32 == SCAN_THREADS, "one B|C element per thread per stage");
-  static_assert(2 * SCAN_CH * NS * 4 <= SCAN_STAGES * STAGE, "look-back scratch fits the stage ring");
+  static constexpr int OFF_BCF = OFF_C + al128(BCB);      // fp32 B|C [Q][32]
+  static constexpr int STAGE = OFF_BCF + SCAN_Q * 32 * 4;
+  static constexpr int OFF_A2 = SCAN_STAGES * STAGE;      // general kernel: A * log2(e) [256][16]
+  static constexpr int A2_BYTES = FAST ? 0 : SCAN_CH * NS * 4;
+  static constexpr int OFF_BAR = OFF_A2 + A2_BYTES;       // full[S], ready[S], empty[S]
+  static constexpr int BYTES = OFF_BAR + 3 * SCAN_STAGES * 8 + 128 + 128;
+  static_assert(2 * SCAN_CH * NS * 4 <= SCAN_STAGES * STAGE, "look-back scratch fits in the stage ring");
 };
 
 struct ScanArgs {
-  long long ld_x, ld_z, ld_dt, ld_b, ld_c, ld_y;
-  const float* dt;       // for the fix-up pass
-  const void* z;
-  const void* C;
+  long long ld_y;
   const float* A;
   const float* D;
   const float* h0;
@@ -66,10 +74,9 @@ struct ScanArgs {
   float* h_out;
   int batch, L, di;
   int chunk_len, n_chunks, cgroups;
-  int* ticket;
+  int* ticket;           // [2]: one counter per kernel kind
   int* flags;            // [batch * cgroups * n_chunks]
-  float* rec;            // per record: P[256][16], h[256][16], incl[256][16]
-  float* ylocal;         // [batch * L, di] fp32
+  float* rec;            // per record: P[256][16], h[256][16], inclusive h[256][16]
   int* err;
 };
 
@@ -102,171 +109,289 @@ template <> struct Pair<float> {
 __device__ __forceinline__ void powers16(float r, float* pw) {
   pw[0] = r;
   pw[1] = r * r;
-  float2 p34 = fmul2(make_float2(pw[1], pw[1]), make_float2(pw[0], pw[1]));
+  const float2 p34 = fmul2(make_float2(pw[1], pw[1]), make_float2(pw[0], pw[1]));
   pw[2] = p34.x; pw[3] = p34.y;
-  float2 p56 = fmul2(make_float2(pw[3], pw[3]), make_float2(pw[0], pw[1]));
-  float2 p78 = fmul2(make_float2(pw[3], pw[3]), make_float2(pw[2], pw[3]));
+  const float2 p56 = fmul2(make_float2(pw[3], pw[3]), make_float2(pw[0], pw[1]));
+  const float2 p78 = fmul2(make_float2(pw[3], pw[3]), make_float2(pw[2], pw[3]));
   pw[4] = p56.x; pw[5] = p56.y; pw[6] = p78.x; pw[7] = p78.y;
 #pragma unroll
   for (int i = 0; i < 8; i += 2) {
-    float2 q = fmul2(make_float2(pw[7], pw[7]), make_float2(pw[i], pw[i + 1]));
+    const float2 q = fmul2(make_float2(pw[7], pw[7]), make_float2(pw[i], pw[i + 1]));
     pw[8 + i] = q.x; pw[9 + i] = q.y;
   }
 }
 
-template <typename TX, typename TBC, bool FAST>
-__device__ __forceinline__ void scan_chunk(const CUtensorMap* mx, const CUtensorMap* mz, const CUtensorMap* mdt,
-                                           const CUtensorMap* mB, const CUtensorMap* mC, const ScanArgs& a,
-                                           uint8_t* smem, int b, int cg, int chunk, int grp) {
-  using Lyt = ScanLayout<TX, TBC>;
-  const int tid = threadIdx.x, lane = tid & 31;
-  const int c_base = cg * SCAN_CH;
-  const int cl = tid * 2;            // local channel of this thread's first channel
-  const int c = c_base + cl;
-  const bool valid = c < a.di;       // d_inner is a multiple of 8: both channels valid or neither
-  const int t0 = chunk * a.chunk_len;
-  const int t1 = min(a.L, t0 + a.chunk_len);
-  const long long row0 = (long long)b * a.L;
-  float* sBCf = reinterpret_cast<float*>(smem + Lyt::OFF_BCF);
-  const float* sA2 = reinterpret_cast<const float*>(smem + Lyt::OFF_A2);
-  const uint32_t full0 = smem_u32(smem + Lyt::OFF_BAR);
-  __shared__ int s_flag;
+// Per-CTA context shared by the passes.
+struct ScanCtx {
+  int b, cg, chunk, grp;
+  int t0, t1;
+  long long row0;
+  int c_base;
+};
 
-  float A2_0[2], Dv[2];
+// Producer warp: streams the stages of one pass (window starting at `ts`,
+// `nsub` stages) into the ring and widens B|C.  `g0` counts the stages this
+// CTA already used, so the mbarrier phases continue across passes.
+template <typename TX, typename TBC, bool FAST>
+__device__ __forceinline__ bool producer_pass(const CUtensorMap* mx, const CUtensorMap* mz, const CUtensorMap* mdt,
+                                              const CUtensorMap* mB, const CUtensorMap* mC, uint8_t* smem,
+                                              const ScanCtx& cx, int ts, int nsub, int g0, int* err) {
+  using Lyt = ScanLayout<TX, TBC, FAST>;
+  const int lane = threadIdx.x & 31;
+  const uint32_t full0 = smem_u32(smem + Lyt::OFF_BAR);
+  const uint32_t ready0 = full0 + 8 * SCAN_STAGES, empty0 = ready0 + 8 * SCAN_STAGES;
+  bool ok = true;
+  auto issue = [&](int g) -> bool {  // lane 0 only
+    const int slot = g % SCAN_STAGES, use = g / SCAN_STAGES;
+    if (use > 0 && !mbar_wait(empty0 + 8 * slot, (uint32_t)((use - 1) & 1), err)) return false;
+    uint8_t* st = smem + slot * Lyt::STAGE;
+    const uint32_t bar = full0 + 8 * slot;
+    const int row = (int)(cx.row0 + ts + (g - g0) * SCAN_Q);
+    mbar_arrive_tx(bar, Lyt::STAGE_TX);
+    tma_load_2d(smem_u32(st), mx, bar, cx.c_base, row);
+    tma_load_2d(smem_u32(st + Lyt::OFF_Z), mz, bar, cx.c_base, row);
+    tma_load_2d(smem_u32(st + Lyt::OFF_DT), mdt, bar, cx.c_base, row);
+    tma_load_2d(smem_u32(st + Lyt::OFF_B), mB, bar, 0, row);
+    tma_load_2d(smem_u32(st + Lyt::OFF_C), mC, bar, 0, row);
+    return true;
+  };
+  if (lane == 0)
+    for (int i = 0; i < SCAN_STAGES - 1 && i < nsub && ok; ++i) ok = issue(g0 + i);
+  ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
+  for (int i = 0; i < nsub && ok; ++i) {
+    const int g = g0 + i, slot = g % SCAN_STAGES;
+    ok = mbar_wait(full0 + 8 * slot, (uint32_t)((g / SCAN_STAGES) & 1), err);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok) break;
+    uint8_t* st = smem + slot * Lyt::STAGE;
+    const TBC* sb = reinterpret_cast<const TBC*>(st + (lane < 16 ? Lyt::OFF_B : Lyt::OFF_C));
+    float* bcf = reinterpret_cast<float*>(st + Lyt::OFF_BCF);
+#pragma unroll
+    for (int q = 0; q < SCAN_Q; ++q) bcf[q * 32 + lane] = to_f(sb[q * NS + (lane & 15)]);
+    mbar_arrive(ready0 + 8 * slot);  // every lane: each releases its own writes
+    if (lane == 0 && i + SCAN_STAGES - 1 < nsub) ok = issue(g + SCAN_STAGES - 1);
+    ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
+  }
+  return ok;
+}
+
+// One time step for this thread's two channels: updates h (and, while `head`,
+// the decay trackers) and returns the two pre-gate outputs.
+template <bool FAST>
+__device__ __forceinline__ void scan_step(float2 (&h)[2][8], const float2 xv, const float2 dv, const float* bc,
+                                          const float* A2_0, const float* sA2c, const float* Dv, bool head,
+                                          float (&R)[2], float2 (&P)[2][8], float* y) {
+  float Bv[16], Cv[16];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float4 b4 = *reinterpret_cast<const float4*>(bc + 4 * k);
+    const float4 c4 = *reinterpret_cast<const float4*>(bc + 16 + 4 * k);
+    Bv[4 * k] = b4.x; Bv[4 * k + 1] = b4.y; Bv[4 * k + 2] = b4.z; Bv[4 * k + 3] = b4.w;
+    Cv[4 * k] = c4.x; Cv[4 * k + 1] = c4.y; Cv[4 * k + 2] = c4.z; Cv[4 * k + 3] = c4.w;
+  }
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
-    A2_0[j] = sA2[(cl + j) * NS];
-    Dv[j] = valid ? __ldg(a.D + c + j) : 0.f;
+    const float xj = j ? xv.y : xv.x, dj = j ? dv.y : dv.x;
+    const float u = dj * xj;
+    float pw[16];
+    if constexpr (FAST) {
+      const float r = ex2(dj * A2_0[j]);
+      powers16(r, pw);
+      if (head) R[j] *= r;
+    } else {
+#pragma unroll
+      for (int n = 0; n < NS; ++n) pw[n] = ex2(dj * sA2c[j * NS + n]);
+    }
+    float2 y0 = make_float2(0.f, 0.f), y1 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int n2 = 0; n2 < 8; ++n2) {
+      const float2 a = make_float2(pw[2 * n2], pw[2 * n2 + 1]);
+      const float2 uB = fmul2(make_float2(u, u), make_float2(Bv[2 * n2], Bv[2 * n2 + 1]));
+      h[j][n2] = ffma2(a, h[j][n2], uB);
+      if (n2 & 1) y1 = ffma2(make_float2(Cv[2 * n2], Cv[2 * n2 + 1]), h[j][n2], y1);
+      else y0 = ffma2(make_float2(Cv[2 * n2], Cv[2 * n2 + 1]), h[j][n2], y0);
+      if constexpr (!FAST) {
+        if (head) P[j][n2] = fmul2(P[j][n2], a);
+      }
+    }
+    y[j] = (y0.x + y0.y) + (y1.x + y1.y) + Dv[j] * xj;
   }
+}
 
-  const bool known = (chunk == 0);   // the state entering chunk 0 is h0 (or zero)
+// Consumer warps: the stages of one pass over window [ts, te).  While `head`
+// the warp writes nothing and tracks the decay product; it leaves head mode
+// at the first stage end where that product is zero on all its channels.
+template <typename TX, typename TBC, bool FAST>
+__device__ __forceinline__ bool consumer_pass(uint8_t* smem, const ScanCtx& cx, const ScanArgs& a, int ts, int te,
+                                              int nsub, int g0, float2 (&h)[2][8], bool& head, int& t_head_end,
+                                              float (&R)[2], float2 (&P)[2][8], const float* A2_0,
+                                              const float* sA2c, const float* Dv, bool valid, int c) {
+  using Lyt = ScanLayout<TX, TBC, FAST>;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int cl = tid * 2;
+  const uint32_t full0 = smem_u32(smem + Lyt::OFF_BAR);
+  const uint32_t ready0 = full0 + 8 * SCAN_STAGES, empty0 = ready0 + 8 * SCAN_STAGES;
+  TX* yg = reinterpret_cast<TX*>(a.y);
+  for (int i = 0; i < nsub; ++i) {
+    const int g = g0 + i, slot = g % SCAN_STAGES;
+    if (!__all_sync(0xffffffffu, mbar_wait(ready0 + 8 * slot, (uint32_t)((g / SCAN_STAGES) & 1), a.err)))
+      return false;
+    const uint8_t* st = smem + slot * Lyt::STAGE;
+    const TX* sx = reinterpret_cast<const TX*>(st);
+    const TX* sz = reinterpret_cast<const TX*>(st + Lyt::OFF_Z);
+    const float* sdt = reinterpret_cast<const float*>(st + Lyt::OFF_DT);
+    const float* bcf = reinterpret_cast<const float*>(st + Lyt::OFF_BCF);
+    const int tb = ts + i * SCAN_Q;
+    const int nq = min(SCAN_Q, te - tb);
+    if (nq == SCAN_Q) {
+#pragma unroll
+      for (int q = 0; q < SCAN_Q; ++q) {
+        float y[2];
+        scan_step<FAST>(h, Pair<TX>::load(sx + q * SCAN_CH + cl), *reinterpret_cast<const float2*>(sdt + q * SCAN_CH + cl),
+                        bcf + q * 32, A2_0, sA2c, Dv, head, R, P, y);
+        if (!head && valid) {
+          const float2 zv = Pair<TX>::load(sz + q * SCAN_CH + cl);
+          Pair<TX>::store(yg + (cx.row0 + tb + q) * a.ld_y + c, y[0] * silu(zv.x), y[1] * silu(zv.y));
+        }
+      }
+    } else {
+      for (int q = 0; q < nq; ++q) {
+        float y[2];
+        scan_step<FAST>(h, Pair<TX>::load(sx + q * SCAN_CH + cl), *reinterpret_cast<const float2*>(sdt + q * SCAN_CH + cl),
+                        bcf + q * 32, A2_0, sA2c, Dv, head, R, P, y);
+        if (!head && valid) {
+          const float2 zv = Pair<TX>::load(sz + q * SCAN_CH + cl);
+          Pair<TX>::store(yg + (cx.row0 + tb + q) * a.ld_y + c, y[0] * silu(zv.x), y[1] * silu(zv.y));
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty0 + 8 * slot);
+    if (head) {
+      bool zero = !valid;
+      if (!zero) {
+        if constexpr (FAST) {
+          zero = R[0] == 0.f && R[1] == 0.f;
+        } else {
+          zero = true;
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int n2 = 0; n2 < 8; ++n2) zero = zero && P[j][n2].x == 0.f && P[j][n2].y == 0.f;
+        }
+      }
+      if (__all_sync(0xffffffffu, zero)) {
+        head = false;
+        t_head_end = min(te, tb + SCAN_Q);
+      }
+    }
+  }
+  return true;
+}
+
+template <typename TX, typename TBC, bool FAST>
+__global__ void __launch_bounds__(SCAN_THREADS, FAST ? 3 : 2)
+selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensorMap mz,
+                      const __grid_constant__ CUtensorMap mdt, const __grid_constant__ CUtensorMap mB,
+                      const __grid_constant__ CUtensorMap mC, const ScanArgs a) {
+  using Lyt = ScanLayout<TX, TBC, FAST>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  __shared__ int s_ticket, s_flag, s_head_end[4];
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const bool producer = warp == 4;
+  const uint32_t full0 = smem_u32(smem + Lyt::OFF_BAR);
+  const uint32_t ready0 = full0 + 8 * SCAN_STAGES, empty0 = ready0 + 8 * SCAN_STAGES;
+  if (tid == 0) {
+    s_ticket = atomicAdd(a.ticket + (FAST ? 0 : 1), 1);
+    for (int s = 0; s < SCAN_STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(ready0 + 8 * s, 32);
+      mbar_init(empty0 + 8 * s, 4);
+    }
+    mbar_fence_init();
+  }
+  __syncthreads();
+  ScanCtx cx;
+  const int groups_total = a.batch * a.cgroups;
+  cx.chunk = s_ticket / groups_total;
+  cx.grp = s_ticket - cx.chunk * groups_total;
+  cx.b = cx.grp / a.cgroups;
+  cx.cg = cx.grp - cx.b * a.cgroups;
+  cx.c_base = cx.cg * SCAN_CH;
+  cx.t0 = cx.chunk * a.chunk_len;
+  cx.t1 = min(a.L, cx.t0 + a.chunk_len);
+  cx.row0 = (long long)cx.b * a.L;
+
+  // which kernel owns this CTA: the power form needs A[c, n] == (n + 1) A[c, 0] on all its channels
+  const int cl = producer ? 0 : tid * 2;
+  const int c = cx.c_base + cl;
+  const bool valid = !producer && c < a.di;
+  float A2_0[2] = {0.f, 0.f}, Dv[2] = {0.f, 0.f};
+  bool ok = true;
+  float* sA2 = reinterpret_cast<float*>(smem + Lyt::OFF_A2);
+  if (valid) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const float* Ar = a.A + (long long)(c + j) * NS;
+      const float a0 = __ldg(Ar);
+      A2_0[j] = a0 * LOG2E;
+      Dv[j] = __ldg(a.D + c + j);
+#pragma unroll
+      for (int n = 0; n < NS; ++n) {
+        const float an = __ldg(Ar + n);
+        ok = ok && (an == (float)(n + 1) * a0);
+        if constexpr (!FAST) sA2[(cl + j) * NS + n] = an * LOG2E;
+      }
+    }
+  } else if constexpr (!FAST) {
+    if (!producer)
+      for (int n = 0; n < 2 * NS; ++n) sA2[cl * NS + n] = 0.f;
+  }
+  const bool structured = (__syncthreads_and(ok) != 0) && sizeof(TX) == 2;
+  if (structured != FAST) return;   // the other kernel of the pair owns these channels
+  const float* sA2c = FAST ? nullptr : sA2 + cl * NS;
+
+  const bool known = cx.chunk == 0;
   float2 h[2][8];
 #pragma unroll
   for (int j = 0; j < 2; ++j)
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
+      h[j][i] = make_float2(0.f, 0.f);
       if (known && a.h0 && valid) {
-        const float* src = a.h0 + ((long long)b * a.di + c + j) * NS + 2 * i;
+        const float* src = a.h0 + ((long long)cx.b * a.di + c + j) * NS + 2 * i;
         h[j][i] = make_float2(src[0], src[1]);
-      } else {
-        h[j][i] = make_float2(0.f, 0.f);
       }
     }
-  // decay product since t0 (only tracked while the warp still buffers)
   float R[2] = {1.f, 1.f};
   float2 P[2][8];
 #pragma unroll
   for (int j = 0; j < 2; ++j)
 #pragma unroll
     for (int i = 0; i < 8; ++i) P[j][i] = make_float2(1.f, 1.f);
-  bool buffering = !known;
-  int tA_end = t0;
+  bool head = !known;
+  int t_head_end = cx.t0;
 
-  const int nsub = (t1 - t0 + SCAN_Q - 1) / SCAN_Q;
-  auto issue = [&](int i) {
-    const int slot = i % SCAN_STAGES;
-    uint8_t* st = smem + slot * Lyt::STAGE;
-    const uint32_t bar = full0 + 8 * slot;
-    const int row = (int)(row0 + t0 + i * SCAN_Q);
-    mbar_arrive_tx(bar, Lyt::STAGE_TX);
-    tma_load_2d(smem_u32(st), mx, bar, c_base, row);
-    tma_load_2d(smem_u32(st + Lyt::OFF_Z), mz, bar, c_base, row);
-    tma_load_2d(smem_u32(st + Lyt::OFF_DT), mdt, bar, c_base, row);
-    tma_load_2d(smem_u32(st + Lyt::OFF_B), mB, bar, 0, row);
-    tma_load_2d(smem_u32(st + Lyt::OFF_C), mC, bar, 0, row);
-  };
-  if (tid == 0)
-    for (int i = 0; i < SCAN_STAGES - 1 && i < nsub; ++i) issue(i);
-
-  bool aborted = false;
-  for (int i = 0; i < nsub; ++i) {
-    const int slot = i % SCAN_STAGES;
-    const uint8_t* st = smem + slot * Lyt::STAGE;
-    const bool ok = mbar_wait(full0 + 8 * slot, (uint32_t)((i / SCAN_STAGES) & 1), a.err);
-    if (ok) {
-      // widen B|C of this stage to fp32, one element per thread
-      const int q = tid >> 5, k = tid & 31;
-      const TBC* src = reinterpret_cast<const TBC*>(st + (k < 16 ? Lyt::OFF_B : Lyt::OFF_C));
-      sBCf[(slot * SCAN_Q + q) * 32 + k] = to_f(src[q * NS + (k & 15)]);
-    }
-    if (__syncthreads_or(!ok)) { aborted = true; break; }
-    if (tid == 0 && i + SCAN_STAGES - 1 < nsub) issue(i + SCAN_STAGES - 1);
-
-    const TX* sx = reinterpret_cast<const TX*>(st);
-    const TX* sz = reinterpret_cast<const TX*>(st + Lyt::OFF_Z);
-    const float* sdt = reinterpret_cast<const float*>(st + Lyt::OFF_DT);
-#pragma unroll
-    for (int q = 0; q < SCAN_Q; ++q) {
-      const int t = t0 + i * SCAN_Q + q;
-      if (t >= t1) break;
-      const float2 xv = Pair<TX>::load(sx + q * SCAN_CH + cl);
-      const float2 dv = *reinterpret_cast<const float2*>(sdt + q * SCAN_CH + cl);
-      const float* bc = sBCf + (slot * SCAN_Q + q) * 32;
-      float y[2];
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const float xj = j ? xv.y : xv.x, dj = j ? dv.y : dv.x;
-        const float u = dj * xj;
-        float pw[16];
-        if constexpr (FAST) {
-          const float r = ex2(dj * A2_0[j]);
-          powers16(r, pw);
-          if (buffering) R[j] *= r;
-        } else {
-#pragma unroll
-          for (int n = 0; n < NS; ++n) pw[n] = ex2(dj * sA2[(cl + j) * NS + n]);
-        }
-        float2 ya = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int n2 = 0; n2 < 8; ++n2) {
-          const float2 Bn = *reinterpret_cast<const float2*>(bc + 2 * n2);
-          const float2 Cn = *reinterpret_cast<const float2*>(bc + 16 + 2 * n2);
-          const float2 uB = fmul2(make_float2(u, u), Bn);
-          h[j][n2] = ffma2(make_float2(pw[2 * n2], pw[2 * n2 + 1]), h[j][n2], uB);
-          ya = ffma2(Cn, h[j][n2], ya);
-          if constexpr (!FAST) {
-            if (buffering) P[j][n2] = fmul2(P[j][n2], make_float2(pw[2 * n2], pw[2 * n2 + 1]));
-          }
-        }
-        y[j] = ya.x + ya.y + Dv[j] * xj;
-      }
-      if (valid) {
-        const long long row = row0 + t;
-        if (buffering) {
-          *reinterpret_cast<float2*>(a.ylocal + row * a.di + c) = make_float2(y[0], y[1]);
-        } else {
-          const float2 zv = Pair<TX>::load(sz + q * SCAN_CH + cl);
-          Pair<TX>::store(reinterpret_cast<TX*>(a.y) + row * a.ld_y + c, y[0] * silu(zv.x), y[1] * silu(zv.y));
-        }
-      }
-    }
-    if (buffering) {
-      bool zero;
-      if constexpr (FAST) {
-        zero = (R[0] == 0.f && R[1] == 0.f) || !valid;
-      } else {
-        zero = true;
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-          for (int n2 = 0; n2 < 8; ++n2) zero = zero && P[j][n2].x == 0.f && P[j][n2].y == 0.f;
-        zero = zero || !valid;
-      }
-      if (__all_sync(0xffffffffu, zero)) {
-        buffering = false;
-        tA_end = min(t1, t0 + (i + 1) * SCAN_Q);
-      }
-    }
-  }
-  if (buffering) tA_end = t1;
-  if (__syncthreads_or(aborted)) return;
+  // ---------------------------------------------------------- pass 1
+  const int nsub1 = (cx.t1 - cx.t0 + SCAN_Q - 1) / SCAN_Q;
+  bool pass_ok;
+  if (producer)
+    pass_ok = producer_pass<TX, TBC, FAST>(&mx, &mz, &mdt, &mB, &mC, smem, cx, cx.t0, nsub1, 0, a.err);
+  else
+    pass_ok = consumer_pass<TX, TBC, FAST>(smem, cx, a, cx.t0, cx.t1, nsub1, 0, h, head, t_head_end, R, P, A2_0,
+                                           sA2c, Dv, valid, c);
+  if (!producer && head) t_head_end = cx.t1;
+  if (!producer && (tid & 31) == 0) s_head_end[warp] = t_head_end;
+  if (__syncthreads_or(!pass_ok)) return;
 
   // ---------------------------------------------------------- carry
-  const long long rbase = (long long)grp * a.n_chunks;
-  constexpr int REC = 3 * SCAN_CH * NS;
-  float* myrec = a.rec + (rbase + chunk) * REC;
-  int* myflag = a.flags + rbase + chunk;
-  const bool independent = __syncthreads_and(!buffering) != 0;  // end state does not depend on h_in
+  const long long rbase = (long long)cx.grp * a.n_chunks;
+  float* myrec = a.rec + (rbase + cx.chunk) * REC;
+  int* myflag = a.flags + rbase + cx.chunk;
+  const bool independent = __syncthreads_and(producer || !head) != 0;  // end state free of h_in
+  int t_head_max = cx.t0;
+  for (int w = 0; w < 4; ++w) t_head_max = max(t_head_max, s_head_end[w]);
   float Pend[2][16];
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
@@ -277,43 +402,34 @@ __device__ __forceinline__ void scan_chunk(const CUtensorMap* mx, const CUtensor
       for (int n2 = 0; n2 < 8; ++n2) { Pend[j][2 * n2] = P[j][n2].x; Pend[j][2 * n2 + 1] = P[j][n2].y; }
     }
   }
-  if (independent) {
-    // publish the true end state right away so later chunks need not wait
-#pragma unroll
-    for (int j = 0; j < 2; ++j)
-#pragma unroll
-      for (int n2 = 0; n2 < 8; ++n2)
-        *reinterpret_cast<float2*>(myrec + 2 * SCAN_CH * NS + (cl + j) * NS + 2 * n2) = h[j][n2];
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) st_release(myflag, 2);
-  } else {
-    // aggregate: decay product of the chunk (exactly zero for warps whose carry died out) and local end state
+  if (!producer) {
 #pragma unroll
     for (int j = 0; j < 2; ++j)
 #pragma unroll
       for (int n = 0; n < NS; n += 2) {
-        *reinterpret_cast<float2*>(myrec + (cl + j) * NS + n) = make_float2(Pend[j][n], Pend[j][n + 1]);
-        *reinterpret_cast<float2*>(myrec + SCAN_CH * NS + (cl + j) * NS + n) = h[j][n / 2];
+        float* o = myrec + (cl + j) * NS + n;
+        if (independent) {
+          *reinterpret_cast<float2*>(o + 2 * SCAN_CH * NS) = h[j][n / 2];
+        } else {
+          *reinterpret_cast<float2*>(o) = make_float2(Pend[j][n], Pend[j][n + 1]);
+          *reinterpret_cast<float2*>(o + SCAN_CH * NS) = h[j][n / 2];
+        }
       }
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) st_release(myflag, 1);
   }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) st_release(myflag, independent ? 2 : 1);
 
-  float hin[2][16];
   if (!known) {
-    // look back: h_in = h_{k-1} + P_{k-1} (h_{k-2} + P_{k-2} (... + incl_j))
-    float* sP = reinterpret_cast<float*>(smem);              // [256][16], the stage ring is free now
+    // look back: h_in = h_{k-1} + P_{k-1} (h_{k-2} + P_{k-2} (... + inclusive_j))
+    float* sP = reinterpret_cast<float*>(smem);   // the ring is idle between the passes
     float* sH = sP + SCAN_CH * NS;
-#pragma unroll
-    for (int j = 0; j < 2; ++j)
-#pragma unroll
-      for (int n = 0; n < NS; ++n) {
-        sP[(cl + j) * NS + n] = 1.f;
-        sH[(cl + j) * NS + n] = 0.f;
+    if (!producer)
+      for (int n = 0; n < 2 * NS; ++n) {
+        sP[cl * NS + n] = 1.f;
+        sH[cl * NS + n] = 0.f;
       }
-    int jc = chunk - 1;
+    int jc = cx.chunk - 1;
     bool done = false;
     while (!done) {
       if (tid == 0) {
@@ -332,15 +448,13 @@ __device__ __forceinline__ void scan_chunk(const CUtensorMap* mx, const CUtensor
       }
       __syncthreads();
       const int f = s_flag;
-      if (f < 0) return;   // uniform: every thread read the same s_flag
+      if (f < 0) return;   // every thread read the same value
       __threadfence();
       const float* rP = a.rec + (rbase + jc) * REC;
       bool allzero = true;
-#pragma unroll
-      for (int j = 0; j < 2; ++j)
-#pragma unroll
-        for (int n = 0; n < NS; ++n) {
-          const int o = (cl + j) * NS + n;
+      if (!producer) {
+        for (int n = 0; n < 2 * NS; ++n) {
+          const int o = cl * NS + n;
           if (f == 2) {
             sH[o] = fmaf(sP[o], __ldcg(rP + 2 * SCAN_CH * NS + o), sH[o]);
           } else {
@@ -349,6 +463,7 @@ __device__ __forceinline__ void scan_chunk(const CUtensorMap* mx, const CUtensor
             allzero = allzero && sP[o] == 0.f;
           }
         }
+      }
       if (f == 2) {
         done = true;
       } else {
@@ -357,132 +472,51 @@ __device__ __forceinline__ void scan_chunk(const CUtensorMap* mx, const CUtensor
       }
       __syncthreads();
     }
+    float2 hin[2][8];
 #pragma unroll
     for (int j = 0; j < 2; ++j)
 #pragma unroll
-      for (int n = 0; n < NS; ++n) hin[j][n] = sH[(cl + j) * NS + n];
-
+      for (int n2 = 0; n2 < 8; ++n2)
+        hin[j][n2] = producer ? make_float2(0.f, 0.f)
+                              : make_float2(sH[(cl + j) * NS + 2 * n2], sH[(cl + j) * NS + 2 * n2 + 1]);
+    __syncthreads();   // the ring is reused by pass 2
     if (!independent) {
       // true end state h + P_end * h_in, published as this chunk's inclusive record
+      if (!producer) {
 #pragma unroll
-      for (int j = 0; j < 2; ++j)
+        for (int j = 0; j < 2; ++j)
 #pragma unroll
-        for (int n2 = 0; n2 < 8; ++n2) {
-          h[j][n2].x = fmaf(Pend[j][2 * n2], hin[j][2 * n2], h[j][n2].x);
-          h[j][n2].y = fmaf(Pend[j][2 * n2 + 1], hin[j][2 * n2 + 1], h[j][n2].y);
-          *reinterpret_cast<float2*>(myrec + 2 * SCAN_CH * NS + (cl + j) * NS + 2 * n2) = h[j][n2];
-        }
+          for (int n2 = 0; n2 < 8; ++n2) {
+            h[j][n2].x = fmaf(Pend[j][2 * n2], hin[j][n2].x, h[j][n2].x);
+            h[j][n2].y = fmaf(Pend[j][2 * n2 + 1], hin[j][n2].y, h[j][n2].y);
+            *reinterpret_cast<float2*>(myrec + 2 * SCAN_CH * NS + (cl + j) * NS + 2 * n2) = h[j][n2];
+          }
+      }
       __threadfence();
       __syncthreads();
       if (tid == 0) st_release(myflag, 2);
     }
 
-    // finish the buffered steps of this warp: y = (y_local + C . (P_t * h_in)) * SiLU(z)
-    if (valid) {
-      const TX* zg = reinterpret_cast<const TX*>(a.z);
-      const TBC* Cg = reinterpret_cast<const TBC*>(a.C);
-      float Rf[2] = {1.f, 1.f};
-      float2 Pf[2][8];
-#pragma unroll
-      for (int j = 0; j < 2; ++j)
-#pragma unroll
-        for (int n2 = 0; n2 < 8; ++n2) Pf[j][n2] = make_float2(1.f, 1.f);
-#pragma unroll 2
-      for (int t = t0; t < tA_end; ++t) {
-        const long long row = row0 + t;
-        const float2 yl = __ldcg(reinterpret_cast<const float2*>(a.ylocal + row * a.di + c));
-        const float2 dv = __ldg(reinterpret_cast<const float2*>(a.dt + row * a.ld_dt + c));
-        const float2 zv = Pair<TX>::load(zg + row * a.ld_z + c);
-        float Cv[16];
-#pragma unroll
-        for (int n = 0; n < NS; ++n) Cv[n] = to_f(Cg[row * a.ld_c + n]);
-        float yo[2];
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const float dj = j ? dv.y : dv.x;
-          float corr;
-          if constexpr (FAST) {
-            Rf[j] *= ex2(dj * A2_0[j]);
-            float acc = Cv[15] * hin[j][15];
-#pragma unroll
-            for (int n = 14; n >= 0; --n) acc = fmaf(acc, Rf[j], Cv[n] * hin[j][n]);
-            corr = acc * Rf[j];
-          } else {
-            corr = 0.f;
-#pragma unroll
-            for (int n2 = 0; n2 < 8; ++n2) {
-              const float2 e = make_float2(ex2(dj * sA2[(cl + j) * NS + 2 * n2]),
-                                           ex2(dj * sA2[(cl + j) * NS + 2 * n2 + 1]));
-              Pf[j][n2] = fmul2(Pf[j][n2], e);
-              corr = fmaf(Cv[2 * n2] * hin[j][2 * n2], Pf[j][n2].x, corr);
-              corr = fmaf(Cv[2 * n2 + 1] * hin[j][2 * n2 + 1], Pf[j][n2].y, corr);
-            }
-          }
-          yo[j] = ((j ? yl.y : yl.x) + corr) * silu(j ? zv.y : zv.x);
-        }
-        Pair<TX>::store(reinterpret_cast<TX*>(a.y) + row * a.ld_y + c, yo[0], yo[1]);
-      }
+    // ---------------------------------------------------------- pass 2: replay the head from h_in
+    const int nsub2 = (t_head_max - cx.t0 + SCAN_Q - 1) / SCAN_Q;
+    if (producer) {
+      producer_pass<TX, TBC, FAST>(&mx, &mz, &mdt, &mB, &mC, smem, cx, cx.t0, nsub2, nsub1, a.err);
+    } else {
+      bool head2 = false;
+      int unused = 0;
+      consumer_pass<TX, TBC, FAST>(smem, cx, a, cx.t0, t_head_max, nsub2, nsub1, hin, head2, unused, R, P, A2_0,
+                                   sA2c, Dv, valid, c);
     }
   }
 
   // final state of the batch row
-  if (t1 == a.L && a.h_out && valid) {
+  if (cx.t1 == a.L && a.h_out && valid) {
 #pragma unroll
     for (int j = 0; j < 2; ++j)
 #pragma unroll
       for (int n2 = 0; n2 < 8; ++n2)
-        *reinterpret_cast<float2*>(a.h_out + ((long long)b * a.di + c + j) * NS + 2 * n2) = h[j][n2];
+        *reinterpret_cast<float2*>(a.h_out + ((long long)cx.b * a.di + c + j) * NS + 2 * n2) = h[j][n2];
   }
-}
-
-template <typename TX, typename TBC>
-__global__ void __launch_bounds__(SCAN_THREADS)
-selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensorMap mz,
-                      const __grid_constant__ CUtensorMap mdt, const __grid_constant__ CUtensorMap mB,
-                      const __grid_constant__ CUtensorMap mC, const ScanArgs a) {
-  using Lyt = ScanLayout<TX, TBC>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-  __shared__ int s_ticket;
-  const int tid = threadIdx.x;
-  if (tid == 0) {
-    s_ticket = atomicAdd(a.ticket, 1);
-    const uint32_t full0 = smem_u32(smem + Lyt::OFF_BAR);
-    for (int s = 0; s < SCAN_STAGES; ++s) mbar_init(full0 + 8 * s, 1);
-    mbar_fence_init();
-    tma_prefetch(&mx);
-    tma_prefetch(&mz);
-    tma_prefetch(&mdt);
-    tma_prefetch(&mB);
-    tma_prefetch(&mC);
-  }
-  __syncthreads();
-  const int groups_total = a.batch * a.cgroups;
-  const int ticket = s_ticket;
-  const int chunk = ticket / groups_total;
-  const int grp = ticket - chunk * groups_total;
-  const int b = grp / a.cgroups, cg = grp - b * a.cgroups;
-
-  // A * log2(e) of this CTA's channels, and whether A[c, n] == (n + 1) A[c, 0]
-  float* sA2 = reinterpret_cast<float*>(smem + Lyt::OFF_A2);
-  bool ok = true;
-#pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const int c = cg * SCAN_CH + tid * 2 + j;
-    const bool v = c < a.di;
-    const float a0 = v ? __ldg(a.A + (long long)c * NS) : 0.f;
-#pragma unroll
-    for (int n = 0; n < NS; ++n) {
-      const float an = v ? __ldg(a.A + (long long)c * NS + n) : 0.f;
-      ok = ok && (an == (float)(n + 1) * a0);
-      sA2[(tid * 2 + j) * NS + n] = an * LOG2E;
-    }
-  }
-  const bool fast = __syncthreads_and(ok) != 0;
-  if (fast)
-    scan_chunk<TX, TBC, true>(&mx, &mz, &mdt, &mB, &mC, a, smem, b, cg, chunk, grp);
-  else
-    scan_chunk<TX, TBC, false>(&mx, &mz, &mdt, &mB, &mC, a, smem, b, cg, chunk, grp);
 }
 
 // ------------------------------------------------------------ decode step
@@ -526,43 +560,83 @@ size_t scan_workspace_bytes(int batch, int L, int di, int chunk_len) {
   const int cgroups = (di + SCAN_CH - 1) / SCAN_CH;
   const int n_chunks = (L + chunk_len - 1) / chunk_len;
   const size_t recs = (size_t)batch * cgroups * n_chunks;
-  size_t bytes = 256;                                       // ticket
+  size_t bytes = 256;                                       // tickets
   bytes += (recs * sizeof(int) + 255) & ~size_t(255);       // flags
-  bytes += recs * 3 * SCAN_CH * NS * sizeof(float);         // records
-  bytes += (size_t)batch * L * di * sizeof(float);          // buffered pre-gate outputs
+  bytes += recs * REC * sizeof(float);                      // chunk records
   return bytes;
 }
 
-int scan_auto_chunk(int batch, int L, int di) {
+template <typename TX, typename TBC, bool FAST>
+static bool configure_scan() {
+  using Lyt = ScanLayout<TX, TBC, FAST>;
+  static bool done[64] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (!done[dev]) {
+    if (cudaFuncSetAttribute(selective_scan_kernel<TX, TBC, FAST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Lyt::BYTES) != cudaSuccess)
+      return false;
+    done[dev] = true;
+  }
+  return true;
+}
+
+template <typename TX, typename TBC, bool FAST>
+static int resident_ctas() {
+  using Lyt = ScanLayout<TX, TBC, FAST>;
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 2 * num_sms();
+  if (cache[dev] == 0) {
+    int per_sm = 0;
+    configure_scan<TX, TBC, FAST>();
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, selective_scan_kernel<TX, TBC, FAST>, SCAN_THREADS,
+                                                      Lyt::BYTES) != cudaSuccess || per_sm < 1)
+      per_sm = 1;
+    cache[dev] = per_sm * num_sms();
+  }
+  return cache[dev];
+}
+
+// Time chunk: every CTA of the launch resident at once (a CTA waiting on its
+// predecessor must never wait for a free SM slot), preferring chunks of at
+// least 8192 steps once half of the resident slots are filled, since each
+// chunk after the first replays its head.
+int scan_auto_chunk(int batch, int L, int di, int dtype, int bc_dtype) {
   const int cgroups = (di + SCAN_CH - 1) / SCAN_CH;
-  const int groups = batch * cgroups;
-  // aim for about two resident CTAs per SM
-  const int want = 2 * num_sms();
-  int n_chunks = (want + groups - 1) / groups;
+  const long long groups = (long long)batch * cgroups;
+  int cap;
+  if (dtype == JAMBA_BF16 && bc_dtype == JAMBA_BF16) cap = resident_ctas<bf16, bf16, true>();
+  else if (dtype == JAMBA_BF16) cap = resident_ctas<bf16, float, true>();
+  else cap = resident_ctas<float, float, false>();
+  long long full = cap / groups;
+  long long half = full / 2;
+  long long by_len = (L + 8191) / 8192;
+  long long n_chunks = by_len > half ? by_len : half;
+  if (n_chunks > full) n_chunks = full;
   if (n_chunks < 1) n_chunks = 1;
-  int chunk = (L + n_chunks - 1) / n_chunks;
+  int chunk = (int)((L + n_chunks - 1) / n_chunks);
   chunk = (chunk + 15) & ~15;
   if (chunk < 16) chunk = 16;
   return chunk;
 }
 
-
 template <typename TX, typename TBC>
 static jamba_status launch_scan(const ScanCall& s, cudaStream_t st) {
-  using Lyt = ScanLayout<TX, TBC>;
   const CUtensorMapDataType tx = sizeof(TX) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   const CUtensorMapDataType tb = sizeof(TBC) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   const uint64_t rows = (uint64_t)s.batch * s.L;
   CUtensorMap mx, mz, mdt, mB, mC;
   JB_TRY(make_map_2d(&mx, s.x, tx, sizeof(TX), s.di, rows, s.ld_x * sizeof(TX), SCAN_CH, SCAN_Q, CU_TENSOR_MAP_SWIZZLE_NONE));
   JB_TRY(make_map_2d(&mz, s.z, tx, sizeof(TX), s.di, rows, s.ld_z * sizeof(TX), SCAN_CH, SCAN_Q, CU_TENSOR_MAP_SWIZZLE_NONE));
-  JB_TRY(make_map_2d(&mdt, s.dt, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, s.di, rows, s.ld_dt * 4, SCAN_CH, SCAN_Q, CU_TENSOR_MAP_SWIZZLE_NONE));
+  JB_TRY(make_map_2d(&mdt, s.dt, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, s.di, rows, s.ld_dt * 4, SCAN_CH, SCAN_Q,
+                     CU_TENSOR_MAP_SWIZZLE_NONE));
   JB_TRY(make_map_2d(&mB, s.B, tb, sizeof(TBC), NS, rows, s.ld_b * sizeof(TBC), NS, SCAN_Q, CU_TENSOR_MAP_SWIZZLE_NONE));
   JB_TRY(make_map_2d(&mC, s.C, tb, sizeof(TBC), NS, rows, s.ld_c * sizeof(TBC), NS, SCAN_Q, CU_TENSOR_MAP_SWIZZLE_NONE));
 
   ScanArgs a;
-  a.ld_x = s.ld_x; a.ld_z = s.ld_z; a.ld_dt = s.ld_dt; a.ld_b = s.ld_b; a.ld_c = s.ld_c; a.ld_y = s.ld_y;
-  a.dt = s.dt; a.z = s.z; a.C = s.C; a.A = s.A; a.D = s.D; a.h0 = s.h0; a.y = s.y; a.h_out = s.h_out;
+  a.ld_y = s.ld_y;
+  a.A = s.A; a.D = s.D; a.h0 = s.h0; a.y = s.y; a.h_out = s.h_out;
   a.batch = s.batch; a.L = s.L; a.di = s.di;
   a.chunk_len = s.chunk;
   a.n_chunks = (s.L + s.chunk - 1) / s.chunk;
@@ -573,20 +647,19 @@ static jamba_status launch_scan(const ScanCall& s, cudaStream_t st) {
   a.flags = reinterpret_cast<int*>(w + 256);
   const size_t flags_bytes = (recs * sizeof(int) + 255) & ~size_t(255);
   a.rec = reinterpret_cast<float*>(w + 256 + flags_bytes);
-  a.ylocal = a.rec + recs * 3 * SCAN_CH * NS;
   a.err = device_error_word();
   if (!a.err) return fail(JAMBA_ERR_CUDA, "could not allocate the device status word");
   JB_CUDA(cudaMemsetAsync(w, 0, 256 + flags_bytes, st));
-
-  static bool configured[64] = {false};
-  int dev = 0;
-  JB_CUDA(cudaGetDevice(&dev));
-  if (dev < 64 && !configured[dev]) {
-    JB_CUDA(cudaFuncSetAttribute(selective_scan_kernel<TX, TBC>, cudaFuncAttributeMaxDynamicSharedMemorySize, Lyt::BYTES));
-    configured[dev] = true;
+  if (recs > 0x7fffffffull) return fail(JAMBA_ERR_UNSUPPORTED, "scan: too many chunks");
+  if (sizeof(TX) == 2) {
+    if (!configure_scan<TX, TBC, true>()) return fail(JAMBA_ERR_CUDA, "scan: kernel configuration failed");
+    selective_scan_kernel<TX, TBC, true>
+        <<<(unsigned)recs, SCAN_THREADS, ScanLayout<TX, TBC, true>::BYTES, st>>>(mx, mz, mdt, mB, mC, a);
+    JB_CUDA(cudaGetLastError());
   }
-  const long long grid = (long long)recs;
-  selective_scan_kernel<TX, TBC><<<(unsigned)grid, SCAN_THREADS, Lyt::BYTES, st>>>(mx, mz, mdt, mB, mC, a);
+  if (!configure_scan<TX, TBC, false>()) return fail(JAMBA_ERR_CUDA, "scan: kernel configuration failed");
+  selective_scan_kernel<TX, TBC, false>
+      <<<(unsigned)recs, SCAN_THREADS, ScanLayout<TX, TBC, false>::BYTES, st>>>(mx, mz, mdt, mB, mC, a);
   JB_CUDA(cudaGetLastError());
   return JAMBA_OK;
 }
@@ -599,12 +672,11 @@ jamba_status scan_run(const ScanCall& s, cudaStream_t st) {
   if (s.chunk <= 0 || s.chunk % 16) return fail(JAMBA_ERR_INVALID_ARG, "scan: chunk must be a positive multiple of 16");
   if (s.ld_x < s.di || s.ld_z < s.di || s.ld_dt < s.di || s.ld_y < s.di || s.ld_b < NS || s.ld_c < NS)
     return fail(JAMBA_ERR_INVALID_ARG, "scan: leading dimension below the row width");
-  if (s.ld_y % 2 || s.ld_z % 2 || s.ld_dt % 2)
-    return fail(JAMBA_ERR_INVALID_ARG, "scan: leading dimensions of y, z, dt must be even");
-  if (!aligned16(s.y) || !aligned16(s.z) || !aligned16(s.dt))
-    return fail(JAMBA_ERR_INVALID_ARG, "scan: y, z and dt must be 16-byte aligned");
+  if (s.ld_y % 2) return fail(JAMBA_ERR_INVALID_ARG, "scan: the leading dimension of y must be even");
+  if (!aligned16(s.y)) return fail(JAMBA_ERR_INVALID_ARG, "scan: y must be 16-byte aligned");
   if (s.ws_bytes < scan_workspace_bytes(s.batch, s.L, s.di, s.chunk) || !s.ws || !aligned16(s.ws))
     return fail(JAMBA_ERR_WORKSPACE, "scan: workspace too small");
+  if ((long long)s.batch * s.L > 0x7fffffffLL) return fail(JAMBA_ERR_UNSUPPORTED, "scan: too many tokens");
   if (s.dtype == JAMBA_BF16 && s.bc_dtype == JAMBA_BF16) return launch_scan<bf16, bf16>(s, st);
   if (s.dtype == JAMBA_BF16 && s.bc_dtype == JAMBA_F32) return launch_scan<bf16, float>(s, st);
   if (s.dtype == JAMBA_F32 && s.bc_dtype == JAMBA_F32) return launch_scan<float, float>(s, st);
