@@ -44,48 +44,55 @@ rmsnorm_kernel(const T* __restrict__ x, const float* __restrict__ w, T* __restri
 }
 
 // x_proj output: sum the split-K partials [splits][T][R + 2N], then the three
-// inner RMSNorms; dt_low goes out in the GEMM dtype, B | C in fp32.
+// inner RMSNorms; dt_low goes out in the GEMM dtype, B | C in fp32.  One block
+// per token, one thread per column.
 template <typename TD>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(512)
 xproj_norm_kernel(const float* __restrict__ part, int splits, long long split_stride, int T, int R, int N,
                   const float* __restrict__ w_dt, const float* __restrict__ w_B, const float* __restrict__ w_C,
                   int inner_norm, float eps, TD* __restrict__ dtlow, float* __restrict__ bc) {
-  const int warp = (blockIdx.x * 256 + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  if (warp >= T) return;
-  const int W = R + 2 * N;
-  constexpr int MAXPER = 16;  // up to 512 columns
-  float v[MAXPER];
-  float s_dt = 0.f, s_b = 0.f, s_c = 0.f;
+  const long long t = blockIdx.x;
+  const int col = threadIdx.x, W = R + 2 * N;
+  const int lane = col & 31, warp = col >> 5;
+  __shared__ float red[16][3];
+  __shared__ float inv[3];
+  float v = 0.f;
+  if (col < W) {
+    const float* p = part + t * W + col;
+    int s = 0;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    for (; s + 4 <= splits; s += 4) {
+      a0 += p[(s + 0) * split_stride];
+      a1 += p[(s + 1) * split_stride];
+      a2 += p[(s + 2) * split_stride];
+      a3 += p[(s + 3) * split_stride];
+    }
+    for (; s < splits; ++s) a0 += p[s * split_stride];
+    v = (a0 + a1) + (a2 + a3);
+  }
+  const int seg = col < R ? 0 : (col < R + N ? 1 : 2);
+  float sq[3] = {0.f, 0.f, 0.f};
+  if (col < W) sq[seg] = v * v;
 #pragma unroll
-  for (int k = 0; k < MAXPER; ++k) {
-    const int col = lane + 32 * k;
+  for (int k = 0; k < 3; ++k) {
+    sq[k] = warp_sum(sq[k]);
+    if (lane == 0) red[warp][k] = sq[k];
+  }
+  __syncthreads();
+  if (col < 3) {
     float acc = 0.f;
-    if (col < W) {
-      for (int s = 0; s < splits; ++s) acc += part[s * split_stride + (long long)warp * W + col];
-      if (col < R) s_dt = fmaf(acc, acc, s_dt);
-      else if (col < R + N) s_b = fmaf(acc, acc, s_b);
-      else s_c = fmaf(acc, acc, s_c);
-    }
-    v[k] = acc;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) acc += red[w][col];
+    const float n = col == 0 ? (float)R : (float)N;
+    inv[col] = inner_norm ? rsqrtf(acc / n + eps) : 1.f;
   }
-  float i_dt = 1.f, i_b = 1.f, i_c = 1.f;
-  if (inner_norm) {
-    i_dt = rsqrtf(warp_sum(s_dt) / (float)R + eps);
-    i_b = rsqrtf(warp_sum(s_b) / (float)N + eps);
-    i_c = rsqrtf(warp_sum(s_c) / (float)N + eps);
-  }
-#pragma unroll
-  for (int k = 0; k < MAXPER; ++k) {
-    const int col = lane + 32 * k;
-    if (col >= W) continue;
-    if (col < R) {
-      const float o = inner_norm ? v[k] * i_dt * w_dt[col] : v[k];
-      dtlow[(long long)warp * R + col] = from_f<TD>(o);
-    } else if (col < R + N) {
-      bc[(long long)warp * 2 * N + (col - R)] = inner_norm ? v[k] * i_b * w_B[col - R] : v[k];
-    } else {
-      bc[(long long)warp * 2 * N + (col - R)] = inner_norm ? v[k] * i_c * w_C[col - R - N] : v[k];
-    }
+  __syncthreads();
+  if (col >= W) return;
+  if (seg == 0) {
+    dtlow[t * R + col] = from_f<TD>(inner_norm ? v * inv[0] * w_dt[col] : v);
+  } else if (seg == 1) {
+    bc[t * 2 * N + (col - R)] = inner_norm ? v * inv[1] * w_B[col - R] : v;
+  } else {
+    bc[t * 2 * N + (col - R)] = inner_norm ? v * inv[2] * w_C[col - R - N] : v;
   }
 }
 
@@ -125,13 +132,13 @@ jamba_status xproj_norm(const float* part, int splits, long long split_stride, i
                         const float* w_dt, const float* w_B, const float* w_C, int inner_norm, float eps,
                         void* dtlow, float* bc, int dtype, cudaStream_t s) {
   if (R + 2 * N > 512) return fail(JAMBA_ERR_UNSUPPORTED, "x_proj width above 512");
-  const unsigned grid = (unsigned)(((long long)T * 32 + 255) / 256);
+  const int threads = ((R + 2 * N + 31) / 32) * 32;
   if (dtype == JAMBA_BF16)
-    xproj_norm_kernel<bf16><<<grid, 256, 0, s>>>(part, splits, split_stride, T, R, N, w_dt, w_B, w_C, inner_norm,
-                                                eps, reinterpret_cast<bf16*>(dtlow), bc);
+    xproj_norm_kernel<bf16><<<T, threads, 0, s>>>(part, splits, split_stride, T, R, N, w_dt, w_B, w_C, inner_norm,
+                                                  eps, reinterpret_cast<bf16*>(dtlow), bc);
   else
-    xproj_norm_kernel<float><<<grid, 256, 0, s>>>(part, splits, split_stride, T, R, N, w_dt, w_B, w_C, inner_norm,
-                                                 eps, reinterpret_cast<float*>(dtlow), bc);
+    xproj_norm_kernel<float><<<T, threads, 0, s>>>(part, splits, split_stride, T, R, N, w_dt, w_B, w_C, inner_norm,
+                                                   eps, reinterpret_cast<float*>(dtlow), bc);
   JB_CUDA(cudaGetLastError());
   return JAMBA_OK;
 }

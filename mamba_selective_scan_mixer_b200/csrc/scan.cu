@@ -520,39 +520,41 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
 }
 
 // ------------------------------------------------------------ decode step
-// One thread per (batch row, channel): advances the cached state by one token.
+// Advances the cached state of every (batch row, channel) by one token.  Four
+// threads share a channel, four states each, so state, A, B and C move as
+// float4 loads contiguous across the warp; y is summed over the four lanes.
 template <typename TX>
 __global__ void __launch_bounds__(256)
 ssm_step_kernel(const TX* __restrict__ xc, const TX* __restrict__ z, long long ld_z, const float* __restrict__ dt,
                 const float* __restrict__ bc, long long ld_bc, const float* __restrict__ A,
                 const float* __restrict__ D, float* __restrict__ state, TX* __restrict__ y, int batch, int di) {
-  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= (long long)batch * di) return;
-  const int b = (int)(i / di), c = (int)(i - (long long)b * di);
-  const float x = to_f(xc[i]);
-  const float d = dt[i];
-  const float* Bv = bc + (long long)b * ld_bc;
-  const float* Cv = Bv + NS;
-  float4* hs = reinterpret_cast<float4*>(state + i * NS);
-  const float4* Ar = reinterpret_cast<const float4*>(A + (long long)c * NS);
-  float acc = 0.f;
+  const long long i = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 2;   // flat (row, channel)
+  const int q = threadIdx.x & 3;
+  const bool live = i < (long long)batch * di;
+  const long long ii = live ? i : 0;
+  const int b = (int)(ii / di), c = (int)(ii - (long long)b * di);
+  const float x = to_f(xc[ii]);
+  const float d = dt[ii];
+  const float4 Bv = *reinterpret_cast<const float4*>(bc + (long long)b * ld_bc + 4 * q);
+  const float4 Cv = *reinterpret_cast<const float4*>(bc + (long long)b * ld_bc + NS + 4 * q);
+  const float4 av = __ldg(reinterpret_cast<const float4*>(A + (long long)c * NS + 4 * q));
+  float4* hs = reinterpret_cast<float4*>(state + ii * NS + 4 * q);
+  float4 h = *hs;
   const float u = d * x;
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    float4 h = hs[k];
-    const float4 av = __ldg(Ar + k);
-    h.x = fmaf(ex2(d * av.x * LOG2E), h.x, u * Bv[4 * k + 0]);
-    h.y = fmaf(ex2(d * av.y * LOG2E), h.y, u * Bv[4 * k + 1]);
-    h.z = fmaf(ex2(d * av.z * LOG2E), h.z, u * Bv[4 * k + 2]);
-    h.w = fmaf(ex2(d * av.w * LOG2E), h.w, u * Bv[4 * k + 3]);
-    acc = fmaf(Cv[4 * k + 0], h.x, acc);
-    acc = fmaf(Cv[4 * k + 1], h.y, acc);
-    acc = fmaf(Cv[4 * k + 2], h.z, acc);
-    acc = fmaf(Cv[4 * k + 3], h.w, acc);
-    hs[k] = h;
+  const float dl = d * LOG2E;
+  h.x = fmaf(ex2(dl * av.x), h.x, u * Bv.x);
+  h.y = fmaf(ex2(dl * av.y), h.y, u * Bv.y);
+  h.z = fmaf(ex2(dl * av.z), h.z, u * Bv.z);
+  h.w = fmaf(ex2(dl * av.w), h.w, u * Bv.w);
+  float part = Cv.x * h.x + Cv.y * h.y + Cv.z * h.z + Cv.w * h.w;
+  part += __shfl_xor_sync(0xffffffffu, part, 1);
+  part += __shfl_xor_sync(0xffffffffu, part, 2);
+  if (!live) return;
+  *hs = h;
+  if (q == 0) {
+    const float zv = to_f(z[(long long)b * ld_z + c]);
+    y[ii] = from_f<TX>((part + __ldg(D + c) * x) * silu(zv));
   }
-  const float zv = to_f(z[(long long)b * ld_z + c]);
-  y[i] = from_f<TX>((acc + __ldg(D + c) * x) * silu(zv));
 }
 
 // ------------------------------------------------------------ host side
@@ -686,7 +688,7 @@ jamba_status scan_run(const ScanCall& s, cudaStream_t st) {
 jamba_status ssm_step(const void* xc, const void* z, long long ld_z, const float* dt, const float* bc,
                       long long ld_bc, const float* A, const float* D, float* state, void* y, int batch, int di,
                       int dtype, cudaStream_t st) {
-  const long long n = (long long)batch * di;
+  const long long n = (long long)batch * di * 4;
   const unsigned grid = (unsigned)((n + 255) / 256);
   if (dtype == JAMBA_BF16)
     ssm_step_kernel<bf16><<<grid, 256, 0, st>>>(reinterpret_cast<const bf16*>(xc), reinterpret_cast<const bf16*>(z),
