@@ -157,6 +157,39 @@ jamba_status jamba_selective_scan(const void* x, int ld_x, const void* z, int ld
                                   int d_inner, int d_state, int dtype, int chunk, void* ws,
                                   size_t ws_bytes, jamba_stream_t stream);
 
+/* jamba_selective_scan without a workspace argument, for callers that must
+ * not allocate device memory.  Some callers cannot call cudaMalloc on their
+ * execution path: a kernel library plugged into another framework runs inside
+ * that framework's memory plan, whose allocator already owns the device
+ * memory, so an extra allocation may fail or stall everything else on the
+ * GPU.  This entry point allocates nothing: the scratch the scan needs (chunk
+ * records, flags, tickets) is a static device array of 32 MiB that every GPU
+ * loading the library holds until the process exits.  The caller still passes
+ * all inputs and outputs, exactly as for jamba_selective_scan.
+ *  - The paper has no counterpart to this entry point; it exists for the
+ *    callers described above.
+ *  - The first call on each device looks up the array's device address with
+ *    that device current (a host-side runtime query, no allocation); make
+ *    that first call before any stream capture.
+ *  - All calls on a device share the one array and it keeps the last call's
+ *    contents; each call clears the part that must start at zero.  Calls whose
+ *    execution overlaps on the GPU (different streams, no ordering between
+ *    them) race on the array and give undefined results: order them.
+ *  - Limit: batch * ceil(d_inner / 256) channel groups times the number of
+ *    time chunks must fit the array (48 KiB per chunk record); the time chunk
+ *    is lengthened until it fits, and JAMBA_ERR_UNSUPPORTED is returned when
+ *    even one chunk per group does not (more than about 680 groups, e.g.
+ *    batch 85 at d_inner 8192).
+ *  - status: a device int the kernel sets to JAMBA_ERR_TIMEOUT if one of its
+ *    bounded waits gives up (never cleared by the library), or NULL to use a
+ *    static word of the same array set.
+ * Other arguments, layouts and errors: as jamba_selective_scan. */
+jamba_status jamba_selective_scan_static(const void* x, int ld_x, const void* z, int ld_z, const float* dt,
+                                         int ld_dt, const void* B, int ld_b, const void* C, int ld_c,
+                                         int bc_dtype, const float* A, const float* D, const float* h0,
+                                         void* y, int ld_y, float* h_out, int batch, int seqlen, int d_inner,
+                                         int d_state, int dtype, int* status, jamba_stream_t stream);
+
 /* ------------------------------------------------------- building blocks */
 
 /* out = RMSNorm(x) * w over rows of `cols` elements (block norm of the layer pair).

@@ -84,6 +84,7 @@ struct ScanCall {
   float* h_out;
   int batch, L, di, dtype, chunk;
   void* ws; size_t ws_bytes;
+  int* err;   // device status word; null = the library's per-device word
 };
 jamba_status scan_run(const ScanCall& s, cudaStream_t st);
 size_t scan_workspace_bytes(int batch, int L, int di, int chunk_len);

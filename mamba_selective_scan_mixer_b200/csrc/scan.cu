@@ -649,7 +649,7 @@ static jamba_status launch_scan(const ScanCall& s, cudaStream_t st) {
   a.flags = reinterpret_cast<int*>(w + 256);
   const size_t flags_bytes = (recs * sizeof(int) + 255) & ~size_t(255);
   a.rec = reinterpret_cast<float*>(w + 256 + flags_bytes);
-  a.err = device_error_word();
+  a.err = s.err ? s.err : device_error_word();
   if (!a.err) return fail(JAMBA_ERR_CUDA, "could not allocate the device status word");
   JB_CUDA(cudaMemsetAsync(w, 0, 256 + flags_bytes, st));
   if (recs > 0x7fffffffull) return fail(JAMBA_ERR_UNSUPPORTED, "scan: too many chunks");

@@ -148,6 +148,25 @@ def selective_scan(x, z, dt, B, C, A, D, h0=None, chunk=0, want_state=True, y=No
     return y, h_out
 
 
+def selective_scan_static(x, z, dt, B, C, A, D, h0=None, want_state=True, y=None, status=None, stream=None):
+    """selective_scan() through the entry point that allocates nothing (its
+    scratch is a static device array inside libjamba.so).  Returns (y, h_out)."""
+    _cuda(x, z, dt, B, C, A, D, h0, status)
+    batch, L, di = x.shape
+    N = A.shape[1]
+    for t, n in ((x, "x"), (z, "z"), (dt, "dt"), (B, "B"), (C, "C")):
+        if t.stride(-1) != 1 or t.stride(0) != L * t.stride(1):
+            raise ValueError("%s: rows must be unit-stride and evenly spaced" % n)
+    if y is None:
+        y = torch.empty(batch, L, di, dtype=x.dtype, device=x.device)
+    h_out = torch.empty(batch, di, N, dtype=torch.float32, device=x.device) if want_state else None
+    check(lib().jamba_selective_scan_static(_p(x), x.stride(1), _p(z), z.stride(1), _p(dt), dt.stride(1), _p(B),
+                                            B.stride(1), _p(C), C.stride(1), _DT[B.dtype], _p(A), _p(D), _p(h0),
+                                            _p(y), y.stride(1), _p(h_out), batch, L, di, N, _DT[x.dtype],
+                                            _p(status), _stream(stream)))
+    return y, h_out
+
+
 def rmsnorm(x, w, eps=1e-6, out=None, stream=None):
     _cuda(x, w)
     _contig(x, "x")
