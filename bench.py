@@ -32,6 +32,10 @@ DECODE_B, DECODE_PREFILL, DECODE_STEPS = 64, 2048, 1024
 SCAN_L, SCAN_DI = 131072, 8192
 PAIR_B, PAIR_L = 4, 8192
 METRIC = "Mamba-layer tokens/s (prefill 128K, decode) at d_model=4096; scan HBM GB/s vs peak"
+# DRAM bytes (read + write) of one in_proj launch at 131072 tokens: ncu capture at 16384 tokens
+# (1.211 GB read + 0.515 GB written, see profiles/in_proj_gemm_traffic.md) scaled by 8, since
+# operand re-reads and the output all grow with the token count
+IN_PROJ_TRAFFIC_128K = 8 * (1.211251200e9 + 0.515489280e9)
 
 
 def parse():
@@ -41,7 +45,12 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="product", choices=["product", "reference"])
     ap.add_argument("--quick", action="store_true", help="skip the side measurements")
-    ap.add_argument("--seqlen", type=int, default=PREFILL_L)
+    ap.add_argument("--only", default="all",
+                    help="comma list of parts to run (prefill,gemm,scan,decode,pair,e2e,cpu); for profiling")
+    ap.add_argument("--seqlen", type=int, default=PREFILL_L, help="prefill tokens")
+    ap.add_argument("--scan-seqlen", type=int, default=SCAN_L)
+    ap.add_argument("--decode-steps", type=int, default=DECODE_STEPS)
+    ap.add_argument("--pair-seqlen", type=int, default=PAIR_L)
     return ap.parse_args()
 
 
@@ -74,7 +83,7 @@ class Clocks:
         os.close(fd)
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
-                                          "-lms", "200"] + self.sel, stdout=open(self.path, "w"),
+                                          "-lms", "20"] + self.sel, stdout=open(self.path, "w"),
                                          stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -209,42 +218,49 @@ def run_product(args):
     L = args.seqlen
     stream = torch.cuda.current_stream(dev)
 
+    parts = {"prefill", "gemm", "scan", "decode", "pair", "e2e", "cpu"} if args.only == "all" else \
+        set(args.only.split(","))
+    if args.quick:
+        parts &= {"prefill"}
     params = {k: v.to(dev) for k, v in mamba_params(sh, seed=0).items()}
     mixer = J.MambaMixer(params, sh)
-    u = mamba_input(sh, 1, L, seed=rank_seed(rank), device=dev)
-    out = torch.empty_like(u)
+    u = mamba_input(sh, 1, L, seed=rank_seed(rank), device=dev) if ({"prefill", "gemm", "e2e"} & parts) else None
+    out = torch.empty_like(u) if u is not None else None
     cs, ss = mixer.new_states(1)
     flush_buf = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     flush = lambda: flush_buf.zero_()
     step = lambda: mixer.prefill(u, out=out, conv_state_out=cs, ssm_state_out=ss)
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    J.device_status()
-    clocks = Clocks(dev)
-    barrier(world)
-    torch.cuda.synchronize()
-    clocks.start()
-    ms, per = event_time_ms(step, args.steps, stream, flush)
-    torch.cuda.synchronize()
-    barrier(world)
-    clk = clocks.stop()
-    J.device_status()
-    ms = max_over_ranks(ms, world)
-    value = aggregate_tokens_per_s(world, L, ms)
+    ms, clk, value = None, None, None
+    if "prefill" in parts:
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        J.device_status()
+        clocks = Clocks(dev)
+        barrier(world)
+        torch.cuda.synchronize()
+        clocks.start()
+        ms, per = event_time_ms(step, args.steps, stream, flush)
+        torch.cuda.synchronize()
+        barrier(world)
+        clk = clocks.stop()
+        J.device_status()
+        ms = max_over_ranks(ms, world)
+        value = aggregate_tokens_per_s(world, L, ms)
 
-    res = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-           "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+    res = {"metric": METRIC, "value": None if value is None else round(value, 1), "unit": "tokens/s",
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": None if ms is None else round(ms, 4), "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "bf16",
            "data": "synthetic: seeded N(0,1) input, N(0,0.02) weights, A=-(n+1), D=1, dt_bias log-uniform",
            "config": {"workload": "prefill_128k: Mamba mixer prefill, batch 1, L=%d, d_model 4096, d_inner 8192, "
                                   "d_state 16, dt_rank 256, inner RMSNorm, bf16 weights/activations, fp32 state" % L,
                       "global_batch": world, "seq_len": L, "parallelism": "replicas" if world > 1 else "single",
                       "l2": "512 MB buffer written before every timed step (outside the events)"},
-           "gpu_launches": 7 * args.steps, "clocks": clk}
+           "gpu_launches": None if ms is None else 8 * args.steps, "clocks": clk}
 
-    if rank == 0 and not args.quick:
+    if rank == 0 and "gemm" in parts:
         # dominant kernel: in_proj GEMM on the tensor cores, same shape as inside the step
         xz = torch.empty(L, 2 * sh.d_inner, dtype=torch.bfloat16, device=dev)
         a2 = u.view(L, sh.d_model)
@@ -256,73 +272,80 @@ def run_product(args):
         ach = flops / (gms / 1e3) / 1e12
         res["roofline"] = {"kernel": "in_proj gemm_bf16_tc_kernel<256,4> (%dx%dx%d)" % (L, 2 * sh.d_inner, sh.d_model),
                            "bound": "tensor", "achieved": round(ach, 1), "peak": pk["bf16"], "unit": "TFLOP/s",
-                           "frac": round(ach / pk["bf16"], 4), "traffic": None,
+                           "frac": round(ach / pk["bf16"], 4),
+                           "traffic": IN_PROJ_TRAFFIC_128K if L == PREFILL_L else None,
                            "peak_source": "%s bf16 burst (kernel timed alone)" % pk["src"],
                            "ms": round(gms, 3)}
         del xz
+    if rank == 0 and "scan" in parts:
         # selective scan alone at 128K context
-        s = {k: v.to(dev) for k, v in scan_inputs(1, SCAN_L, SCAN_DI, 16, seed=0, device=dev).items()}
+        SL = args.scan_seqlen
+        s = {k: v.to(dev) for k, v in scan_inputs(1, SL, SCAN_DI, 16, seed=0, device=dev).items()}
         y = torch.empty_like(s["x"])
         sc = lambda: J.selective_scan(s["x"], s["z"], s["dt"], s["B"], s["C"], s["A"], s["D"], y=y, ws=scan_ws,
                                       want_state=True)
         import ctypes
         nbytes = ctypes.c_size_t()
-        J.lib().jamba_selective_scan_workspace_size(1, SCAN_L, SCAN_DI, 16, 0, ctypes.byref(nbytes))
+        J.lib().jamba_selective_scan_workspace_size(1, SL, SCAN_DI, 16, 0, ctypes.byref(nbytes))
         scan_ws = torch.empty(nbytes.value, dtype=torch.uint8, device=dev)
         for _ in range(2):
             sc()
         sms, _ = event_time_ms(sc, 5, stream, flush)
-        sbytes = SCAN_L * (SCAN_DI * (2 + 2 + 4 + 2) + 16 * 2 * 2)
+        sbytes = SL * (SCAN_DI * (2 + 2 + 4 + 2) + 16 * 2 * 2)
         gbs = sbytes / (sms / 1e3) / 1e9
-        res["scan"] = {"workload": "scan_128k: selective scan + D + SiLU(z) gate alone, batch 1, L=131072, "
-                                   "d_inner 8192, bf16 x/z/B/C/y, fp32 dt",
+        res["scan"] = {"workload": "scan_128k: selective scan + D + SiLU(z) gate alone, batch 1, L=%d, "
+                                   "d_inner 8192, bf16 x/z/B/C/y, fp32 dt" % SL,
                        "ms": round(sms, 4), "GB/s": round(gbs, 1), "frac_of_measured_hbm": round(gbs / pk["hbm"], 4),
                        "frac_of_8TBs": round(gbs / 8000.0, 4), "algorithmic_bytes": sbytes,
-                       "tokens/s": round(SCAN_L / (sms / 1e3), 1)}
+                       "tokens/s": round(SL / (sms / 1e3), 1)}
         del s, y, scan_ws
+    if rank == 0 and "decode" in parts:
         # decode: batch 64, caches from a 2048-token prefill, steps in one CUDA graph
         B = DECODE_B
+        NST = args.decode_steps
         u0 = mamba_input(sh, B, DECODE_PREFILL, seed=1, device=dev)
         dcs, dss = mixer.new_states(B)
         mixer.prefill(u0, conv_state_out=dcs, ssm_state_out=dss)
-        steps_u = decode_inputs(sh, B, DECODE_STEPS, seed=1, device=dev)
+        steps_u = decode_inputs(sh, B, NST, seed=1, device=dev)
         dout = torch.empty(B, sh.d_model, dtype=torch.bfloat16, device=dev)
         mixer.step(steps_u[0], dcs, dss, out=dout)       # sizes the workspace before capture
         torch.cuda.synchronize()
         gs = torch.cuda.Stream(dev)
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, stream=gs):
-            for t in range(DECODE_STEPS):
+            for t in range(NST):
                 mixer.step(steps_u[t], dcs, dss, out=dout)
         graph.replay()
         torch.cuda.synchronize()
         dms, _ = event_time_ms(graph.replay, 3, stream, flush)
-        per_step_us = dms * 1e3 / DECODE_STEPS
+        per_step_us = dms * 1e3 / NST
         wbytes = sum(v.numel() * v.element_size() for v in params.values())
         step_bytes = wbytes + 2 * (B * sh.d_inner * 16 * 4 + B * sh.d_inner * 3 * 4) + 2 * B * sh.d_model * 2
-        res["decode"] = {"workload": "decode_b64: batch 64, one token per step, 1024 steps in one CUDA graph, "
-                                     "caches from a 2048-token prefill",
-                         "tokens/s": round(B * DECODE_STEPS / (dms / 1e3), 1), "us_per_step": round(per_step_us, 2),
+        res["decode"] = {"workload": "decode_b64: batch 64, one token per step, %d steps in one CUDA graph, "
+                                     "caches from a 2048-token prefill" % NST,
+                         "tokens/s": round(B * NST / (dms / 1e3), 1), "us_per_step": round(per_step_us, 2),
                          "GB/s": round(step_bytes / (per_step_us / 1e6) / 1e9, 1),
                          "frac_of_measured_hbm": round(step_bytes / (per_step_us / 1e6) / 1e9 / pk["hbm"], 4),
                          "algorithmic_bytes_per_step": step_bytes, "launches_per_step": 8}
         del graph, u0, steps_u
+    if rank == 0 and "pair" in parts:
         # layer pair: RMSNorm -> Mamba -> residual -> RMSNorm -> top-2-of-16 MoE -> residual
+        PL = args.pair_seqlen
         es = MoEShape()
         mp = moe_params(es, seed=0, device=dev)
         moe = J.MoE(mp, es)
         g1, g2 = block_norm_params(sh.d_model, device=dev)
-        xp = mamba_input(sh, PAIR_B, PAIR_L, seed=2, device=dev)
+        xp = mamba_input(sh, PAIR_B, PL, seed=2, device=dev)
         pair = lambda: J.layer_pair(mixer, moe, xp, g1, g2)
         pair()
         torch.cuda.synchronize()
         pms, _ = event_time_ms(pair, 3, stream, flush)
-        T = PAIR_B * PAIR_L
+        T = PAIR_B * PL
         pflops = T * (2.0 * (2 * sh.d_inner * sh.d_model + (sh.dt_rank + 32) * sh.d_inner +
                              sh.dt_rank * sh.d_inner + sh.d_model * sh.d_inner)
                       + 2 * 2.0 * (3 * es.d_model * es.d_ff) + 2.0 * 16 * es.d_model)
-        res["layer_pair"] = {"workload": "layer_pair: batch 4 x 8192 tokens, Mamba (as prefill) + 16-expert "
-                                         "top-2 SwiGLU MoE (d_ff 14336)",
+        res["layer_pair"] = {"workload": "layer_pair: batch 4 x %d tokens, Mamba (as prefill) + 16-expert "
+                                         "top-2 SwiGLU MoE (d_ff 14336)" % PL,
                              "tokens/s": round(T / (pms / 1e3), 1), "ms": round(pms, 3),
                              "TFLOP/s": round(pflops / (pms / 1e3) / 1e12, 1),
                              "frac_of_bf16_sustained": round(pflops / (pms / 1e3) / 1e12 / pk["bf16_sus"], 4)}
@@ -330,7 +353,7 @@ def run_product(args):
         J.device_status()
 
     # end to end through the public API with host buffers (pinned), copies inside the timed region
-    if not args.quick:
+    if "e2e" in parts:
         hu = u.cpu().pin_memory()
         hout = torch.empty_like(hu).pin_memory()
         du = torch.empty_like(u)
@@ -347,7 +370,7 @@ def run_product(args):
         res["e2e"] = {"value": round(aggregate_tokens_per_s(world, L, ems), 1), "unit": "tokens/s",
                       "h2d_bytes_per_step": hu.numel() * hu.element_size(),
                       "d2h_bytes_per_step": hout.numel() * hout.element_size()}
-    if rank == 0 and not args.quick:
+    if rank == 0 and "cpu" in parts:
         res["cpu_baseline"] = cpu_baseline()
     if rank == 0:
         print(json.dumps(res), flush=True)

@@ -144,7 +144,7 @@ jamba_status jamba_selective_scan_workspace_size(int batch, int seqlen, int d_in
  *   B, C   [batch, seqlen, *] bc_dtype, row strides ld_b / ld_c (>= d_state)
  *   A      [d_inner, d_state] fp32, D [d_inner] fp32
  *   h0     [batch, d_inner, d_state] fp32 or NULL (zeros)
- *   y      [batch, seqlen, *] dtype, row stride ld_y
+ *   y      [batch, seqlen, *] dtype, row stride ld_y (a multiple of 4)
  *   h_out  [batch, d_inner, d_state] fp32 or NULL: state after the last step
  *   chunk  time steps per chunk (multiple of 16), 0 = automatic
  * Time is split into chunks scanned concurrently; the state entering each

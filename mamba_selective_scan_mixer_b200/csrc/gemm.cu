@@ -7,21 +7,43 @@
 
 namespace jb {
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int EPI, bool TRANS>
 static jamba_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb2,
-                              const GemmParams& p, int grid, cudaStream_t s) {
-  using S = GemmSmem<BN, STAGES>;
+                              const CUtensorMap& mc, const GemmParams& p, int grid, cudaStream_t s) {
+  using S = GemmSmem<BN, STAGES, EPI == EPI_SOFTPLUS && !TRANS>;
   static bool configured[64] = {false};
   int dev = 0;
   JB_CUDA(cudaGetDevice(&dev));
   if (dev < 64 && !configured[dev]) {
-    JB_CUDA(cudaFuncSetAttribute(gemm_bf16_tc_kernel<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)S::BYTES));
+    JB_CUDA(cudaFuncSetAttribute(gemm_bf16_tc_kernel<BN, STAGES, EPI, TRANS>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::BYTES));
     configured[dev] = true;
   }
-  gemm_bf16_tc_kernel<BN, STAGES><<<grid, 192, S::BYTES, s>>>(ma, mb, mb2, p);
+  gemm_bf16_tc_kernel<BN, STAGES, EPI, TRANS><<<grid, GEMM_THREADS, S::BYTES, s>>>(ma, mb, mb2, mc, p);
   JB_CUDA(cudaGetLastError());
   return JAMBA_OK;
+}
+
+template <int EPI, bool TRANS>
+static jamba_status launch_bn(int bn, const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb2,
+                              const CUtensorMap& mc, const GemmParams& p, int grid, cudaStream_t s) {
+  if constexpr (TRANS) {
+    if (bn == 64) return launch_tc<64, 8, EPI, true>(ma, mb, mb2, mc, p, grid, s);
+  } else if constexpr (EPI == EPI_SOFTPLUS) {
+    // three stages: the ring and the TMA-store staging boxes share the 227 KB
+    if (bn == 256) return launch_tc<256, 3, EPI, false>(ma, mb, mb2, mc, p, grid, s);
+  } else if constexpr (EPI == EPI_SWIGLU) {
+    if (bn == 256) return launch_tc<256, 4, EPI, false>(ma, mb, mb2, mc, p, grid, s);
+  } else {
+    switch (bn) {
+      case 64: return launch_tc<64, 8, EPI, false>(ma, mb, mb2, mc, p, grid, s);
+      case 128: return launch_tc<128, 6, EPI, false>(ma, mb, mb2, mc, p, grid, s);
+      case 144: return launch_tc<144, 6, EPI, false>(ma, mb, mb2, mc, p, grid, s);
+      case 256: return launch_tc<256, 4, EPI, false>(ma, mb, mb2, mc, p, grid, s);
+      default: break;
+    }
+  }
+  return fail(JAMBA_ERR_UNSUPPORTED, "gemm: no kernel for tile width " + std::to_string(bn) + " with this epilogue");
 }
 
 jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
@@ -41,8 +63,8 @@ jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
 
   int bn = g.bn;
   if (bn == 0) {
-    if (g.epi == EPI_SWIGLU) bn = 256;
-    else if (g.N <= 64) bn = 64;
+    if (g.epi == EPI_SWIGLU || g.epi == EPI_SOFTPLUS) bn = g.transpose_out ? 64 : 256;
+    else if (g.transpose_out || g.N <= 64) bn = 64;
     else if (g.N <= 128) bn = 128;
     else if (g.N <= 144 || g.N == 288) bn = 144;
     else bn = 256;
@@ -70,6 +92,11 @@ jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
     }
   }
 
+  CUtensorMap mc = mb;
+  if (g.epi == EPI_SOFTPLUS && !g.transpose_out)
+    JB_TRY(make_map_2d(&mc, g.out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)g.N, (uint64_t)g.M,
+                       (uint64_t)g.ldo * 4, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B));
+
   GemmParams p;
   p.M = g.M;
   p.N = g.N;
@@ -83,8 +110,6 @@ jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
   p.grouped = g.grouped;
   p.offsets = g.offsets;
   p.num_groups = g.num_groups;
-  p.epi = g.epi;
-  p.transpose_out = g.transpose_out;
   p.out = g.out;
   p.ldo = g.ldo;
   p.split_stride = g.split_stride;
@@ -97,20 +122,30 @@ jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
   long long tiles = g.grouped ? (long long)(p.m_tiles + g.num_groups) * p.n_tiles
                               : (long long)p.m_tiles * p.n_tiles * p.splits;
   const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
-  switch (bn) {
-    case 64: return launch_tc<64, 8>(ma, mb, mb2, p, grid, s);
-    case 128: return launch_tc<128, 6>(ma, mb, mb2, p, grid, s);
-    case 144: return launch_tc<144, 6>(ma, mb, mb2, p, grid, s);
-    case 256: return launch_tc<256, 4>(ma, mb, mb2, p, grid, s);
-    default: return fail(JAMBA_ERR_UNSUPPORTED, "gemm: tile width " + std::to_string(bn));
+  if (g.transpose_out) {
+    switch (g.epi) {
+      case EPI_BF16: return launch_bn<EPI_BF16, true>(bn, ma, mb, mb2, mc, p, grid, s);
+      case EPI_F32: return launch_bn<EPI_F32, true>(bn, ma, mb, mb2, mc, p, grid, s);
+      case EPI_SOFTPLUS: return launch_bn<EPI_SOFTPLUS, true>(bn, ma, mb, mb2, mc, p, grid, s);
+      default: break;
+    }
+  } else {
+    switch (g.epi) {
+      case EPI_BF16: return launch_bn<EPI_BF16, false>(bn, ma, mb, mb2, mc, p, grid, s);
+      case EPI_F32: return launch_bn<EPI_F32, false>(bn, ma, mb, mb2, mc, p, grid, s);
+      case EPI_SOFTPLUS: return launch_bn<EPI_SOFTPLUS, false>(bn, ma, mb, mb2, mc, p, grid, s);
+      case EPI_SWIGLU: return launch_bn<EPI_SWIGLU, false>(bn, ma, mb, mb2, mc, p, grid, s);
+      default: break;
+    }
   }
+  return fail(JAMBA_ERR_UNSUPPORTED, "gemm: unknown epilogue");
 }
 
 // ---------------------------------------------------------------- fp32 path
 // 64 x 64 output tile per 256-thread block, 4 x 4 per thread, k-steps of 16.
 __global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__ A, long long lda,
                                                        const float* __restrict__ B, long long ldb, int M, int N,
-                                                       int K, GemmParams p) {
+                                                       int K, int epi, int trans, GemmParams p) {
   __shared__ float As[16][64 + 4];
   __shared__ float Bs[16][64 + 4];
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
@@ -149,8 +184,8 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__
       const int n = n0 + tx * 4 + j;
       if (n >= N) continue;
       float v = acc[i][j];
-      if (p.epi == EPI_SOFTPLUS) v = softplus(v + p.bias[p.transpose_out ? m : n]);
-      if (p.transpose_out) {
+      if (epi == EPI_SOFTPLUS) v = softplus(v + p.bias[trans ? m : n]);
+      if (trans) {
         out[(long long)n * p.ldo + m] = v;
       } else {
         if (res) v += res[(long long)m * p.ldr + n];
@@ -166,8 +201,6 @@ jamba_status gemm_f32(const GemmDesc& g, cudaStream_t s) {
   if (g.grouped || g.splits > 1 || (g.epi != EPI_F32 && g.epi != EPI_SOFTPLUS))
     return fail(JAMBA_ERR_UNSUPPORTED, "fp32 gemm: dense, unsplit, fp32 or softplus epilogue only");
   GemmParams p = {};
-  p.epi = g.epi;
-  p.transpose_out = g.transpose_out;
   p.out = g.out;
   p.ldo = g.ldo;
   p.residual = g.residual;
@@ -175,7 +208,8 @@ jamba_status gemm_f32(const GemmDesc& g, cudaStream_t s) {
   p.bias = g.bias;
   dim3 grid((g.N + 63) / 64, (g.M + 63) / 64);
   gemm_f32_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const float*>(g.a), g.lda,
-                                       reinterpret_cast<const float*>(g.b), g.ldb, g.M, g.N, g.K, p);
+                                       reinterpret_cast<const float*>(g.b), g.ldb, g.M, g.N, g.K, g.epi,
+                                       g.transpose_out, p);
   JB_CUDA(cudaGetLastError());
   return JAMBA_OK;
 }

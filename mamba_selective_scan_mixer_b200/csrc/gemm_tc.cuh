@@ -1,24 +1,30 @@
 // tcgen05 / TMEM GEMM for sm_100a: D[m, n] = sum_k A[m, k] * B[n, k], bf16
 // inputs, fp32 accumulation in tensor memory.
 //
-// One persistent CTA per SM, 6 warps:
+// One persistent CTA per SM, 10 warps:
 //   warp 0     TMA producer: 128 x 64 A tile and BN x 64 B tile per k-step
 //              (128-byte swizzle) into a STAGES-deep shared-memory ring;
 //   warp 1     allocates TMEM and issues tcgen05.mma (one thread), M = 128,
 //              N = BN, K = 16 per instruction, into one of two TMEM
 //              accumulators so the epilogue of tile i overlaps tile i + 1;
-//   warps 2-5  epilogue: tcgen05.ld of their 32-lane quarter, fused
-//              elementwise op, stores to global memory.
-// Used for in_proj, x_proj, dt_proj (+bias+softplus), out_proj (+residual),
-// the decode projections (swap-AB: weights as A so the 64-row token batch is
-// the N side, stored transposed) and the grouped MoE expert GEMMs (SwiGLU
-// epilogue).  Every wait is bounded (see common.cuh).
+//   warps 2-9  epilogue: two warps per 32-lane TMEM quarter, splitting the
+//              32-column chunks between them; tcgen05.ld, fused elementwise
+//              op, stores to global memory.
+// The epilogue kind is a template parameter, so each instantiation carries
+// only its own epilogue code.  Used for in_proj, x_proj, dt_proj
+// (+bias+softplus), out_proj (+residual), the decode projections (swap-AB:
+// weights as A so the 64-row token batch is the N side, stored transposed)
+// and the grouped MoE expert GEMMs (SwiGLU epilogue).  Every wait is bounded
+// (see common.cuh).
 #pragma once
 #include "common.cuh"
 
 namespace jb {
 
 enum EpiKind : int { EPI_BF16 = 0, EPI_F32 = 1, EPI_SOFTPLUS = 2, EPI_SWIGLU = 3 };
+
+constexpr int GEMM_THREADS = 320;
+constexpr int GEMM_EPI_WARPS = 8;
 
 struct GemmParams {
   int M, N, K;           // N counts output columns (SwiGLU: d_ff)
@@ -28,8 +34,6 @@ struct GemmParams {
   int grouped;           // A rows split by offsets[], B is [groups, rows, K]
   const int* offsets;
   int num_groups;
-  int epi;
-  int transpose_out;     // store out[n * ldo + m]
   void* out;
   long long ldo, split_stride;
   const void* residual;  // bf16, same layout as out (non-transposed only)
@@ -42,20 +46,18 @@ struct TileInfo {
   int m0, m_end, n0, kt0, kt1, group, split;
 };
 
-template <int BN>
 __device__ __forceinline__ int total_tiles(const GemmParams& p) {
   if (!p.grouped) return p.m_tiles * p.n_tiles * p.splits;
   int tot = 0;
   for (int g = 0; g < p.num_groups; ++g) {
-    int cnt = __ldg(p.offsets + g + 1) - __ldg(p.offsets + g);
+    const int cnt = __ldg(p.offsets + g + 1) - __ldg(p.offsets + g);
     tot += ((cnt + 127) >> 7) * p.n_tiles;
   }
   return tot;
 }
 
-template <int BN>
+template <int BN_OUT>
 __device__ __forceinline__ void decode_tile(const GemmParams& p, int t, TileInfo& ti) {
-  const int bn_out = (p.epi == EPI_SWIGLU) ? BN / 2 : BN;
   if (!p.grouped) {
     const int per_split = p.m_tiles * p.n_tiles;
     const int s = t / per_split;
@@ -71,7 +73,7 @@ __device__ __forceinline__ void decode_tile(const GemmParams& p, int t, TileInfo
     const int nb = rr / gsize;
     ti.m0 = mb * 128;
     ti.m_end = p.M;
-    ti.n0 = nb * bn_out;
+    ti.n0 = nb * BN_OUT;
     ti.kt0 = s * p.k_tiles_per_split;
     ti.kt1 = min(p.k_tiles, ti.kt0 + p.k_tiles_per_split);
     ti.group = 0;
@@ -85,7 +87,7 @@ __device__ __forceinline__ void decode_tile(const GemmParams& p, int t, TileInfo
         const int mb = t % mt, nb = t / mt;  // m fastest: neighbours share the weight tile
         ti.m0 = o0 + mb * 128;
         ti.m_end = o1;
-        ti.n0 = nb * bn_out;
+        ti.n0 = nb * BN_OUT;
         ti.kt0 = 0;
         ti.kt1 = p.k_tiles;
         ti.group = g;
@@ -106,22 +108,65 @@ __device__ __forceinline__ void store_bf16x8(bf16* dst, const float* v) {
   *reinterpret_cast<uint4*>(dst) = u;
 }
 
-// Epilogue for one 32-column chunk held by this thread (row m, columns n..n+31).
-__device__ __forceinline__ void epi_chunk(const GemmParams& p, const TileInfo& ti, int m, int n, float* v) {
+// softplus for the bf16 path: log(1 + e^v) from one ex2 and one lg2, with the
+// series e - e^2/2 + e^3/3 - e^4/4 where e^v < 1/64 (relative error < 2e-8
+// there, < 1e-5 elsewhere; far inside the bf16 tolerance).
+__device__ __forceinline__ float softplus_fast(float v) {
+  const float e = ex2(1.4426950408889634f * v);
+  float l;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(l) : "f"(1.0f + e));
+  const float big = 0.6931471805599453f * l;
+  const float small = e * (1.0f - e * (0.5f - e * (0.33333334f - e * 0.25f)));
+  const float r = e < 0.015625f ? small : big;
+  return v > 15.0f ? v : r;
+}
+
+__device__ __forceinline__ float log1p_small(float e) {
+  // log(1 + e) for 0 <= e < 1/8: Taylor series through e^7 (relative error < 1e-7)
+  return e * (1.0f - e * (0.5f - e * (0.33333334f - e * (0.25f - e * (0.2f - e * (0.16666667f - e * 0.14285715f))))));
+}
+
+// softplus of 32 values in place: one ex2 each, the series when every e^v of
+// the warp is below 1/8 (the common case for dt), otherwise one lg2 as well.
+__device__ __forceinline__ void softplus32(float* w) {
+  float e[32];
+  bool small = true;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    e[i] = ex2(1.4426950408889634f * w[i]);
+    small = small && e[i] < 0.125f;
+  }
+  if (__all_sync(0xffffffffu, small)) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) w[i] = log1p_small(e[i]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      float l;
+      asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(l) : "f"(1.0f + e[i]));
+      const float r = e[i] < 0.125f ? log1p_small(e[i]) : 0.6931471805599453f * l;
+      w[i] = w[i] > 15.0f ? w[i] : r;
+    }
+  }
+}
+
+// Epilogue of one 32-column chunk held by this thread (row m, columns n..n+NC-1).
+template <int EPI, bool TRANS, int NC>
+__device__ __forceinline__ void epi_chunk(const GemmParams& p, const TileInfo& ti, int m, int n, const float* v) {
   if (m >= ti.m_end) return;
-  if (!p.transpose_out) {
-    if (p.epi == EPI_BF16) {
+  if constexpr (!TRANS) {
+    if constexpr (EPI == EPI_BF16) {
       bf16* o = reinterpret_cast<bf16*>(p.out) + (long long)m * p.ldo;
       const bf16* r = p.residual ? reinterpret_cast<const bf16*>(p.residual) + (long long)m * p.ldr : nullptr;
 #pragma unroll
-      for (int c = 0; c < 32; c += 8) {
+      for (int c = 0; c < NC; c += 8) {
         const int nn = n + c;
-        if (nn + 8 <= p.N) {
-          float w[8];
+        float w[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) w[i] = v[c + i];
+        for (int i = 0; i < 8; ++i) w[i] = v[c + i];
+        if (nn + 8 <= p.N) {
           if (r) {
-            uint4 rv = *reinterpret_cast<const uint4*>(r + nn);
+            const uint4 rv = *reinterpret_cast<const uint4*>(r + nn);
             const bf16* rb = reinterpret_cast<const bf16*>(&rv);
 #pragma unroll
             for (int i = 0; i < 8; ++i) w[i] += __bfloat162float(rb[i]);
@@ -129,25 +174,28 @@ __device__ __forceinline__ void epi_chunk(const GemmParams& p, const TileInfo& t
           store_bf16x8(o + nn, w);
         } else {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            if (nn + i < p.N) {
-              const float w = v[c + i] + (r ? __bfloat162float(r[nn + i]) : 0.f);
-              o[nn + i] = __float2bfloat16_rn(w);
-            }
-          }
+          for (int i = 0; i < 8; ++i)
+            if (nn + i < p.N) o[nn + i] = __float2bfloat16_rn(w[i] + (r ? __bfloat162float(r[nn + i]) : 0.f));
         }
       }
     } else {  // EPI_F32 / EPI_SOFTPLUS
       float* o = reinterpret_cast<float*>(p.out) + (long long)ti.split * p.split_stride + (long long)m * p.ldo;
-      const bool sp = p.epi == EPI_SOFTPLUS;
 #pragma unroll
-      for (int c = 0; c < 32; c += 4) {
+      for (int c = 0; c < NC; c += 4) {
         const int nn = n + c;
         float w[4];
+        if (EPI == EPI_SOFTPLUS && nn + 4 <= p.N) {
+          const float4 b4 = __ldg(reinterpret_cast<const float4*>(p.bias + nn));
+          w[0] = softplus_fast(v[c] + b4.x);
+          w[1] = softplus_fast(v[c + 1] + b4.y);
+          w[2] = softplus_fast(v[c + 2] + b4.z);
+          w[3] = softplus_fast(v[c + 3] + b4.w);
+        } else {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          w[i] = v[c + i];
-          if (sp && nn + i < p.N) w[i] = softplus(w[i] + __ldg(p.bias + nn + i));
+          for (int i = 0; i < 4; ++i) {
+            w[i] = v[c + i];
+            if (EPI == EPI_SOFTPLUS && nn + i < p.N) w[i] = softplus_fast(w[i] + __ldg(p.bias + nn + i));
+          }
         }
         if (nn + 4 <= p.N) {
           *reinterpret_cast<float4*>(o + nn) = make_float4(w[0], w[1], w[2], w[3]);
@@ -160,19 +208,19 @@ __device__ __forceinline__ void epi_chunk(const GemmParams& p, const TileInfo& t
     }
   } else {
     // swap-AB: row m is an output feature, column n a token; lanes hold consecutive m
-    if (p.epi == EPI_BF16) {
+    if constexpr (EPI == EPI_BF16) {
       bf16* o = reinterpret_cast<bf16*>(p.out);
 #pragma unroll
-      for (int c = 0; c < 32; ++c)
+      for (int c = 0; c < NC; ++c)
         if (n + c < p.N) o[(long long)(n + c) * p.ldo + m] = __float2bfloat16_rn(v[c]);
     } else {
       float* o = reinterpret_cast<float*>(p.out) + (long long)ti.split * p.split_stride;
-      const float b = (p.epi == EPI_SOFTPLUS) ? __ldg(p.bias + m) : 0.f;
+      const float b = (EPI == EPI_SOFTPLUS) ? __ldg(p.bias + m) : 0.f;
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
+      for (int c = 0; c < NC; ++c) {
         if (n + c < p.N) {
           float w = v[c];
-          if (p.epi == EPI_SOFTPLUS) w = softplus(w + b);
+          if constexpr (EPI == EPI_SOFTPLUS) w = softplus_fast(w + b);
           o[(long long)(n + c) * p.ldo + m] = w;
         }
       }
@@ -180,23 +228,30 @@ __device__ __forceinline__ void epi_chunk(const GemmParams& p, const TileInfo& t
   }
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool STAGED = false>
 struct GemmSmem {
   static constexpr uint32_t A_BYTES = 128 * 128;
   static constexpr uint32_t B_BYTES = BN * 128;
-  static constexpr uint32_t BAR_OFF = STAGES * (A_BYTES + B_BYTES);
-  static constexpr uint32_t BYTES = BAR_OFF + 256 + 1024;  // + barriers + alignment slack
+  // STAGED: per epilogue warp two 32 x 32 fp32 boxes for TMA stores (1024-aligned)
+  static constexpr uint32_t STG_OFF = STAGES * (A_BYTES + B_BYTES);
+  static constexpr uint32_t STG_BYTES = STAGED ? GEMM_EPI_WARPS * 2 * 4096 : 0;
+  static constexpr uint32_t BAR_OFF = STG_OFF + STG_BYTES;
   // barrier slots: full[STAGES], empty[STAGES], tmem_full[2], tmem_empty[2], drain, tmem holder
+  static constexpr uint32_t BYTES = BAR_OFF + 256 + 1024;  // + barriers + alignment slack
   static constexpr uint32_t TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
                                         : (2 * BN <= 256) ? 256 : 512;
 };
 
-template <int BN, int STAGES>
-__global__ void __launch_bounds__(192, 1)
+template <int BN, int STAGES, int EPI, bool TRANS>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const __grid_constant__ CUtensorMap tmB2, const GemmParams p) {
-  using S = GemmSmem<BN, STAGES>;
+                    const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmC,
+                    const GemmParams p) {
+  // fp32 softplus outputs (dt) leave through shared memory and TMA stores
+  constexpr bool STAGED = EPI == EPI_SOFTPLUS && !TRANS;
+  using S = GemmSmem<BN, STAGES, STAGED>;
   static_assert(BN % 16 == 0 && BN >= 32 && BN <= 256, "UMMA N for M = 128");
+  constexpr int BN_OUT = EPI == EPI_SWIGLU ? BN / 2 : BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -215,19 +270,20 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(tfull0 + 8 * i, 1);
-      mbar_init(tempty0 + 8 * i, 4);
+      mbar_init(tempty0 + 8 * i, GEMM_EPI_WARPS);
     }
     mbar_init(drain, 1);
     mbar_fence_init();
     tma_prefetch(&tmA);
     tma_prefetch(&tmB);
-    if (p.epi == EPI_SWIGLU) tma_prefetch(&tmB2);
+    if (EPI == EPI_SWIGLU) tma_prefetch(&tmB2);
+    if (STAGED) tma_prefetch(&tmC);
   }
   if (warp == 1) tmem_alloc(smem_u32(tmem_holder), S::TMEM_COLS);
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_holder;
-  const int ntiles = total_tiles<BN>(p);
+  const int ntiles = total_tiles(p);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -236,7 +292,7 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
         TileInfo ti;
-        decode_tile<BN>(p, t, ti);
+        decode_tile<BN_OUT>(p, t, ti);
         for (int kt = ti.kt0; kt < ti.kt1; ++kt) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, p.err)) { ok = false; break; }
           const uint32_t fb = full0 + 8 * stage;
@@ -246,7 +302,7 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           tma_load_2d(a_dst, &tmA, fb, kt * 64, ti.m0);
           if (!p.grouped) {
             tma_load_2d(b_dst, &tmB, fb, kt * 64, ti.n0);
-          } else if (p.epi != EPI_SWIGLU) {
+          } else if (EPI != EPI_SWIGLU) {
             tma_load_3d(b_dst, &tmB, fb, kt * 64, ti.n0, ti.group);
           } else {
             tma_load_3d(b_dst, &tmB, fb, kt * 64, ti.n0, ti.group);
@@ -265,7 +321,7 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       int it = 0;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++it) {
         TileInfo ti;
-        decode_tile<BN>(p, t, ti);
+        decode_tile<BN_OUT>(p, t, ti);
         const int acc = it & 1;
         const uint32_t use = (uint32_t)(it >> 1);
         if (!mbar_wait(tempty0 + 8 * acc, (use & 1) ^ 1, p.err)) break;
@@ -290,41 +346,76 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       mbar_wait(drain, 0, p.err);
     }
   } else {
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int q = warp & 3;                 // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;       // which of the two warps of this quarter
     int it = 0;
+    int stg_count = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
       TileInfo ti;
-      decode_tile<BN>(p, t, ti);
+      decode_tile<BN_OUT>(p, t, ti);
       const int acc = it & 1;
       const uint32_t use = (uint32_t)(it >> 1);
       if (!mbar_wait(tfull0 + 8 * acc, use & 1, p.err)) break;
       tc_fence_after();
       const int m = ti.m0 + q * 32 + lane;
       const uint32_t tl = tbase + ((uint32_t)(q * 32) << 16) + acc * BN;
-      if (p.epi != EPI_SWIGLU) {
+      if constexpr (STAGED) {
+        static_assert(BN % 32 == 0, "staged epilogue works on whole 32-column chunks");
+        uint8_t* stg = smem + S::STG_OFF + (warp - 2) * 8192;
 #pragma unroll 1
-        for (int j = 0; j < BN / 32; ++j) {
+        for (int j = half; j < BN / 32; j += 2) {
           float v[32];
           tmem_ld32(tl + j * 32, v);
           tmem_wait_ld();
-          epi_chunk(p, ti, m, ti.n0 + j * 32, v);
+          const int n = ti.n0 + j * 32;
+#pragma unroll
+          for (int c = 0; c < 32; c += 4) {
+            if (n + c + 4 <= p.N) {
+              const float4 b4 = __ldg(reinterpret_cast<const float4*>(p.bias + n + c));
+              v[c] += b4.x; v[c + 1] += b4.y; v[c + 2] += b4.z; v[c + 3] += b4.w;
+            } else {
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                if (n + c + i < p.N) v[c + i] += __ldg(p.bias + n + c + i);
+            }
+          }
+          softplus32(v);
+          uint8_t* buf = stg + (stg_count & 1) * 4096;
+          if (lane == 0) bulk_wait_read<1>();   // this buffer's previous store has read it
+          __syncwarp();
+          // row `lane` of the 32 x 32 box, 16-byte chunks placed by the 128-byte swizzle
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            *reinterpret_cast<float4*>(buf + lane * 128 + ((k ^ (lane & 7)) << 4)) =
+                make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+          fence_async_shared();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmC, smem_u32(buf), n, ti.m0 + q * 32);
+            bulk_commit();
+          }
+          ++stg_count;
+        }
+      } else if constexpr (EPI != EPI_SWIGLU) {
+#pragma unroll 1
+        for (int j = half; j < BN / 32; j += 2) {
+          float v[32];
+          tmem_ld32(tl + j * 32, v);
+          tmem_wait_ld();
+          epi_chunk<EPI, TRANS, 32>(p, ti, m, ti.n0 + j * 32, v);
         }
         if constexpr (BN % 32 != 0) {
-          float v[16];
-          tmem_ld16(tl + (BN / 32) * 32, v);
-          tmem_wait_ld();
-          float w[32];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) { w[i] = v[i]; w[16 + i] = 0.f; }
-          // only 16 valid columns here: clamp N for this chunk
-          GemmParams q2 = p;
-          q2.N = min(p.N, ti.n0 + (BN / 32) * 32 + 16);
-          epi_chunk(q2, ti, m, ti.n0 + (BN / 32) * 32, w);
+          if (half == (BN / 32) % 2) {
+            float v[16];
+            tmem_ld16(tl + (BN / 32) * 32, v);
+            tmem_wait_ld();
+            epi_chunk<EPI, TRANS, 16>(p, ti, m, ti.n0 + (BN / 32) * 32, v);
+          }
         }
       } else {
         bf16* o = reinterpret_cast<bf16*>(p.out) + (long long)m * p.ldo;
 #pragma unroll 1
-        for (int j = 0; j < BN / 64; ++j) {
+        for (int j = half; j < BN / 64; j += 2) {
           float g[32], u[32];
           tmem_ld32(tl + j * 32, g);
           tmem_ld32(tl + BN / 2 + j * 32, u);
@@ -350,6 +441,10 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
+    }
+    if constexpr (STAGED) {
+      if (lane == 0) bulk_wait_all();   // shared memory must outlive the stores reading it
+      __syncwarp();
     }
   }
   __syncthreads();

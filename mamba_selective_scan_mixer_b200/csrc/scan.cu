@@ -38,14 +38,24 @@
 
 namespace jb {
 
-constexpr int SCAN_CONSUMERS = 128;                 // 4 warps x 32 threads x 2 channels
-constexpr int SCAN_THREADS = SCAN_CONSUMERS + 32;   // + producer warp
 constexpr int SCAN_CH = 256;                        // channels per CTA
 constexpr int SCAN_Q = 8;                           // time steps per stage
 constexpr int SCAN_STAGES = 3;
 constexpr int NS = 16;                              // d_state
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr int REC = 3 * SCAN_CH * NS;               // floats per chunk record: P, h, inclusive h
+
+// CTA shape: CPT channels per consumer thread, 256 / (32 CPT) consumer warps,
+// one producer warp; MINB resident CTAs per SM (sets the register cap).
+template <int CPT_, int MINB_>
+struct ScanShape {
+  static constexpr int CPT = CPT_;
+  static constexpr int NCW = SCAN_CH / (32 * CPT_);
+  static constexpr int CONSUMERS = 32 * NCW;
+  static constexpr int THREADS = CONSUMERS + 32;
+  static constexpr int MINB = MINB_;
+  static_assert(NCW * 32 * CPT == SCAN_CH, "a CTA owns 256 channels");
+};
 
 __host__ __device__ constexpr int al128(int v) { return (v + 127) & ~127; }
 
@@ -89,19 +99,55 @@ __device__ __forceinline__ void st_release(int* p, int v) {
   asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-template <typename T> struct Pair;
-template <> struct Pair<bf16> {
-  static __device__ __forceinline__ float2 load(const bf16* p) {
-    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+// CPT consecutive elements <-> floats
+template <typename T, int CPT> struct Vec;
+template <> struct Vec<bf16, 1> {
+  static __device__ __forceinline__ void load(const bf16* p, float* v) { v[0] = __bfloat162float(*p); }
+  static __device__ __forceinline__ void store(bf16* p, const float* v) { *p = __float2bfloat16_rn(v[0]); }
+};
+template <> struct Vec<bf16, 2> {
+  static __device__ __forceinline__ void load(const bf16* p, float* v) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+    v[0] = f.x; v[1] = f.y;
   }
-  static __device__ __forceinline__ void store(bf16* p, float a, float b) {
-    *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
+  static __device__ __forceinline__ void store(bf16* p, const float* v) {
+    *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(v[0], v[1]);
   }
 };
-template <> struct Pair<float> {
-  static __device__ __forceinline__ float2 load(const float* p) { return *reinterpret_cast<const float2*>(p); }
-  static __device__ __forceinline__ void store(float* p, float a, float b) {
-    *reinterpret_cast<float2*>(p) = make_float2(a, b);
+template <> struct Vec<bf16, 4> {
+  static __device__ __forceinline__ void load(const bf16* p, float* v) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+  }
+  static __device__ __forceinline__ void store(bf16* p, const float* v) {
+    uint2 u;
+    *reinterpret_cast<__nv_bfloat162*>(&u.x) = __floats2bfloat162_rn(v[0], v[1]);
+    *reinterpret_cast<__nv_bfloat162*>(&u.y) = __floats2bfloat162_rn(v[2], v[3]);
+    *reinterpret_cast<uint2*>(p) = u;
+  }
+};
+template <> struct Vec<float, 1> {
+  static __device__ __forceinline__ void load(const float* p, float* v) { v[0] = *p; }
+  static __device__ __forceinline__ void store(float* p, const float* v) { *p = v[0]; }
+};
+template <> struct Vec<float, 2> {
+  static __device__ __forceinline__ void load(const float* p, float* v) {
+    const float2 f = *reinterpret_cast<const float2*>(p);
+    v[0] = f.x; v[1] = f.y;
+  }
+  static __device__ __forceinline__ void store(float* p, const float* v) {
+    *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+  }
+};
+template <> struct Vec<float, 4> {
+  static __device__ __forceinline__ void load(const float* p, float* v) {
+    const float4 f = *reinterpret_cast<const float4*>(p);
+    v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+  }
+  static __device__ __forceinline__ void store(float* p, const float* v) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
   }
 };
 
@@ -175,12 +221,12 @@ __device__ __forceinline__ bool producer_pass(const CUtensorMap* mx, const CUten
   return ok;
 }
 
-// One time step for this thread's two channels: updates h (and, while `head`,
-// the decay trackers) and returns the two pre-gate outputs.
-template <bool FAST>
-__device__ __forceinline__ void scan_step(float2 (&h)[2][8], const float2 xv, const float2 dv, const float* bc,
+// One time step for this thread's CPT channels: updates h (and, while `head`,
+// the decay trackers) and returns the pre-gate outputs.
+template <bool FAST, int CPT>
+__device__ __forceinline__ void scan_step(float2 (&h)[CPT][8], const float* xv, const float* dv, const float* bc,
                                           const float* A2_0, const float* sA2c, const float* Dv, bool head,
-                                          float (&R)[2], float2 (&P)[2][8], float* y) {
+                                          float (&R)[CPT], float2 (&P)[CPT][8], float* y) {
   float Bv[16], Cv[16];
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
@@ -190,8 +236,8 @@ __device__ __forceinline__ void scan_step(float2 (&h)[2][8], const float2 xv, co
     Cv[4 * k] = c4.x; Cv[4 * k + 1] = c4.y; Cv[4 * k + 2] = c4.z; Cv[4 * k + 3] = c4.w;
   }
 #pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const float xj = j ? xv.y : xv.x, dj = j ? dv.y : dv.x;
+  for (int j = 0; j < CPT; ++j) {
+    const float xj = xv[j], dj = dv[j];
     const float u = dj * xj;
     float pw[16];
     if constexpr (FAST) {
@@ -221,14 +267,15 @@ __device__ __forceinline__ void scan_step(float2 (&h)[2][8], const float2 xv, co
 // Consumer warps: the stages of one pass over window [ts, te).  While `head`
 // the warp writes nothing and tracks the decay product; it leaves head mode
 // at the first stage end where that product is zero on all its channels.
-template <typename TX, typename TBC, bool FAST>
+template <typename TX, typename TBC, bool FAST, int CPT>
 __device__ __forceinline__ bool consumer_pass(uint8_t* smem, const ScanCtx& cx, const ScanArgs& a, int ts, int te,
-                                              int nsub, int g0, float2 (&h)[2][8], bool& head, int& t_head_end,
-                                              float (&R)[2], float2 (&P)[2][8], const float* A2_0,
+                                              int te_warp, int nsub, int g0, float2 (&h)[CPT][8], bool& head,
+                                              int& t_head_end,
+                                              float (&R)[CPT], float2 (&P)[CPT][8], const float* A2_0,
                                               const float* sA2c, const float* Dv, bool valid, int c) {
   using Lyt = ScanLayout<TX, TBC, FAST>;
   const int tid = threadIdx.x, lane = tid & 31;
-  const int cl = tid * 2;
+  const int cl = tid * CPT;
   const uint32_t full0 = smem_u32(smem + Lyt::OFF_BAR);
   const uint32_t ready0 = full0 + 8 * SCAN_STAGES, empty0 = ready0 + 8 * SCAN_STAGES;
   TX* yg = reinterpret_cast<TX*>(a.y);
@@ -243,39 +290,39 @@ __device__ __forceinline__ bool consumer_pass(uint8_t* smem, const ScanCtx& cx, 
     const float* bcf = reinterpret_cast<const float*>(st + Lyt::OFF_BCF);
     const int tb = ts + i * SCAN_Q;
     const int nq = min(SCAN_Q, te - tb);
-    if (nq == SCAN_Q) {
+    auto step = [&](int q) {
+      float xv[CPT], dv[CPT], y[CPT];
+      Vec<TX, CPT>::load(sx + q * SCAN_CH + cl, xv);
+      Vec<float, CPT>::load(sdt + q * SCAN_CH + cl, dv);
+      scan_step<FAST, CPT>(h, xv, dv, bcf + q * 32, A2_0, sA2c, Dv, head, R, P, y);
+      if (!head && valid) {
+        float zv[CPT];
+        Vec<TX, CPT>::load(sz + q * SCAN_CH + cl, zv);
 #pragma unroll
-      for (int q = 0; q < SCAN_Q; ++q) {
-        float y[2];
-        scan_step<FAST>(h, Pair<TX>::load(sx + q * SCAN_CH + cl), *reinterpret_cast<const float2*>(sdt + q * SCAN_CH + cl),
-                        bcf + q * 32, A2_0, sA2c, Dv, head, R, P, y);
-        if (!head && valid) {
-          const float2 zv = Pair<TX>::load(sz + q * SCAN_CH + cl);
-          Pair<TX>::store(yg + (cx.row0 + tb + q) * a.ld_y + c, y[0] * silu(zv.x), y[1] * silu(zv.y));
-        }
+        for (int j = 0; j < CPT; ++j) y[j] *= silu(zv[j]);
+        Vec<TX, CPT>::store(yg + (cx.row0 + tb + q) * a.ld_y + c, y);
       }
+    };
+    if (tb >= te_warp) {
+      // this warp's own head ended earlier: nothing of this stage is needed
+    } else if (nq == SCAN_Q) {
+#pragma unroll
+      for (int q = 0; q < SCAN_Q; ++q) step(q);
     } else {
-      for (int q = 0; q < nq; ++q) {
-        float y[2];
-        scan_step<FAST>(h, Pair<TX>::load(sx + q * SCAN_CH + cl), *reinterpret_cast<const float2*>(sdt + q * SCAN_CH + cl),
-                        bcf + q * 32, A2_0, sA2c, Dv, head, R, P, y);
-        if (!head && valid) {
-          const float2 zv = Pair<TX>::load(sz + q * SCAN_CH + cl);
-          Pair<TX>::store(yg + (cx.row0 + tb + q) * a.ld_y + c, y[0] * silu(zv.x), y[1] * silu(zv.y));
-        }
-      }
+      for (int q = 0; q < nq; ++q) step(q);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(empty0 + 8 * slot);
     if (head) {
       bool zero = !valid;
       if (!zero) {
+        zero = true;
         if constexpr (FAST) {
-          zero = R[0] == 0.f && R[1] == 0.f;
-        } else {
-          zero = true;
 #pragma unroll
-          for (int j = 0; j < 2; ++j)
+          for (int j = 0; j < CPT; ++j) zero = zero && R[j] == 0.f;
+        } else {
+#pragma unroll
+          for (int j = 0; j < CPT; ++j)
 #pragma unroll
             for (int n2 = 0; n2 < 8; ++n2) zero = zero && P[j][n2].x == 0.f && P[j][n2].y == 0.f;
         }
@@ -289,17 +336,19 @@ __device__ __forceinline__ bool consumer_pass(uint8_t* smem, const ScanCtx& cx, 
   return true;
 }
 
-template <typename TX, typename TBC, bool FAST>
-__global__ void __launch_bounds__(SCAN_THREADS, FAST ? 3 : 2)
+template <typename TX, typename TBC, bool FAST, int CPT, int MINB>
+__global__ void __launch_bounds__(ScanShape<CPT, MINB>::THREADS, MINB)
 selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensorMap mz,
                       const __grid_constant__ CUtensorMap mdt, const __grid_constant__ CUtensorMap mB,
                       const __grid_constant__ CUtensorMap mC, const ScanArgs a) {
   using Lyt = ScanLayout<TX, TBC, FAST>;
+  using Shp = ScanShape<CPT, MINB>;
+  constexpr int NCW = Shp::NCW;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-  __shared__ int s_ticket, s_flag, s_head_end[4];
+  __shared__ int s_ticket, s_flag, s_head_end[NCW];
   const int tid = threadIdx.x, warp = tid >> 5;
-  const bool producer = warp == 4;
+  const bool producer = warp == NCW;
   const uint32_t full0 = smem_u32(smem + Lyt::OFF_BAR);
   const uint32_t ready0 = full0 + 8 * SCAN_STAGES, empty0 = ready0 + 8 * SCAN_STAGES;
   if (tid == 0) {
@@ -307,7 +356,7 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
     for (int s = 0; s < SCAN_STAGES; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(ready0 + 8 * s, 32);
-      mbar_init(empty0 + 8 * s, 4);
+      mbar_init(empty0 + 8 * s, NCW);
     }
     mbar_fence_init();
   }
@@ -324,15 +373,17 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
   cx.row0 = (long long)cx.b * a.L;
 
   // which kernel owns this CTA: the power form needs A[c, n] == (n + 1) A[c, 0] on all its channels
-  const int cl = producer ? 0 : tid * 2;
+  const int cl = producer ? 0 : tid * CPT;
   const int c = cx.c_base + cl;
-  const bool valid = !producer && c < a.di;
-  float A2_0[2] = {0.f, 0.f}, Dv[2] = {0.f, 0.f};
+  const bool valid = !producer && c < a.di;   // d_inner % 8 == 0: all CPT channels valid or none
+  float A2_0[CPT], Dv[CPT];
   bool ok = true;
   float* sA2 = reinterpret_cast<float*>(smem + Lyt::OFF_A2);
-  if (valid) {
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
+  for (int j = 0; j < CPT; ++j) {
+    A2_0[j] = 0.f;
+    Dv[j] = 0.f;
+    if (valid) {
       const float* Ar = a.A + (long long)(c + j) * NS;
       const float a0 = __ldg(Ar);
       A2_0[j] = a0 * LOG2E;
@@ -343,19 +394,19 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
         ok = ok && (an == (float)(n + 1) * a0);
         if constexpr (!FAST) sA2[(cl + j) * NS + n] = an * LOG2E;
       }
+    } else if constexpr (!FAST) {
+      if (!producer)
+        for (int n = 0; n < NS; ++n) sA2[(cl + j) * NS + n] = 0.f;
     }
-  } else if constexpr (!FAST) {
-    if (!producer)
-      for (int n = 0; n < 2 * NS; ++n) sA2[cl * NS + n] = 0.f;
   }
   const bool structured = (__syncthreads_and(ok) != 0) && sizeof(TX) == 2;
   if (structured != FAST) return;   // the other kernel of the pair owns these channels
   const float* sA2c = FAST ? nullptr : sA2 + cl * NS;
 
   const bool known = cx.chunk == 0;
-  float2 h[2][8];
+  float2 h[CPT][8];
 #pragma unroll
-  for (int j = 0; j < 2; ++j)
+  for (int j = 0; j < CPT; ++j)
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       h[j][i] = make_float2(0.f, 0.f);
@@ -364,12 +415,14 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
         h[j][i] = make_float2(src[0], src[1]);
       }
     }
-  float R[2] = {1.f, 1.f};
-  float2 P[2][8];
+  float R[CPT];
+  float2 P[CPT][8];
 #pragma unroll
-  for (int j = 0; j < 2; ++j)
+  for (int j = 0; j < CPT; ++j) {
+    R[j] = 1.f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) P[j][i] = make_float2(1.f, 1.f);
+  }
   bool head = !known;
   int t_head_end = cx.t0;
 
@@ -379,8 +432,8 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
   if (producer)
     pass_ok = producer_pass<TX, TBC, FAST>(&mx, &mz, &mdt, &mB, &mC, smem, cx, cx.t0, nsub1, 0, a.err);
   else
-    pass_ok = consumer_pass<TX, TBC, FAST>(smem, cx, a, cx.t0, cx.t1, nsub1, 0, h, head, t_head_end, R, P, A2_0,
-                                           sA2c, Dv, valid, c);
+    pass_ok = consumer_pass<TX, TBC, FAST, CPT>(smem, cx, a, cx.t0, cx.t1, cx.t1, nsub1, 0, h, head, t_head_end, R,
+                                                P, A2_0, sA2c, Dv, valid, c);
   if (!producer && head) t_head_end = cx.t1;
   if (!producer && (tid & 31) == 0) s_head_end[warp] = t_head_end;
   if (__syncthreads_or(!pass_ok)) return;
@@ -391,10 +444,10 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
   int* myflag = a.flags + rbase + cx.chunk;
   const bool independent = __syncthreads_and(producer || !head) != 0;  // end state free of h_in
   int t_head_max = cx.t0;
-  for (int w = 0; w < 4; ++w) t_head_max = max(t_head_max, s_head_end[w]);
-  float Pend[2][16];
+  for (int w = 0; w < NCW; ++w) t_head_max = max(t_head_max, s_head_end[w]);
+  float Pend[CPT][16];
 #pragma unroll
-  for (int j = 0; j < 2; ++j) {
+  for (int j = 0; j < CPT; ++j) {
     if constexpr (FAST) {
       powers16(R[j], Pend[j]);
     } else {
@@ -404,7 +457,7 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
   }
   if (!producer) {
 #pragma unroll
-    for (int j = 0; j < 2; ++j)
+    for (int j = 0; j < CPT; ++j)
 #pragma unroll
       for (int n = 0; n < NS; n += 2) {
         float* o = myrec + (cl + j) * NS + n;
@@ -425,7 +478,7 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
     float* sP = reinterpret_cast<float*>(smem);   // the ring is idle between the passes
     float* sH = sP + SCAN_CH * NS;
     if (!producer)
-      for (int n = 0; n < 2 * NS; ++n) {
+      for (int n = 0; n < CPT * NS; ++n) {
         sP[cl * NS + n] = 1.f;
         sH[cl * NS + n] = 0.f;
       }
@@ -453,7 +506,7 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
       const float* rP = a.rec + (rbase + jc) * REC;
       bool allzero = true;
       if (!producer) {
-        for (int n = 0; n < 2 * NS; ++n) {
+        for (int n = 0; n < CPT * NS; ++n) {
           const int o = cl * NS + n;
           if (f == 2) {
             sH[o] = fmaf(sP[o], __ldcg(rP + 2 * SCAN_CH * NS + o), sH[o]);
@@ -472,9 +525,9 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
       }
       __syncthreads();
     }
-    float2 hin[2][8];
+    float2 hin[CPT][8];
 #pragma unroll
-    for (int j = 0; j < 2; ++j)
+    for (int j = 0; j < CPT; ++j)
 #pragma unroll
       for (int n2 = 0; n2 < 8; ++n2)
         hin[j][n2] = producer ? make_float2(0.f, 0.f)
@@ -484,7 +537,7 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
       // true end state h + P_end * h_in, published as this chunk's inclusive record
       if (!producer) {
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
+        for (int j = 0; j < CPT; ++j)
 #pragma unroll
           for (int n2 = 0; n2 < 8; ++n2) {
             h[j][n2].x = fmaf(Pend[j][2 * n2], hin[j][n2].x, h[j][n2].x);
@@ -504,15 +557,16 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
     } else {
       bool head2 = false;
       int unused = 0;
-      consumer_pass<TX, TBC, FAST>(smem, cx, a, cx.t0, t_head_max, nsub2, nsub1, hin, head2, unused, R, P, A2_0,
-                                   sA2c, Dv, valid, c);
+      // each warp replays only its own head; the stages after it are passed through
+      consumer_pass<TX, TBC, FAST, CPT>(smem, cx, a, cx.t0, t_head_max, s_head_end[warp], nsub2, nsub1, hin, head2,
+                                        unused, R, P, A2_0, sA2c, Dv, valid, c);
     }
   }
 
   // final state of the batch row
   if (cx.t1 == a.L && a.h_out && valid) {
 #pragma unroll
-    for (int j = 0; j < 2; ++j)
+    for (int j = 0; j < CPT; ++j)
 #pragma unroll
       for (int n2 = 0; n2 < 8; ++n2)
         *reinterpret_cast<float2*>(a.h_out + ((long long)cx.b * a.di + c + j) * NS + 2 * n2) = h[j][n2];
@@ -568,22 +622,26 @@ size_t scan_workspace_bytes(int batch, int L, int di, int chunk_len) {
   return bytes;
 }
 
-template <typename TX, typename TBC, bool FAST>
+// CTA shapes used by the library: power-form kernel and general kernel.
+using FastShape = ScanShape<2, 3>;
+using GenShape = ScanShape<2, 2>;
+
+template <typename TX, typename TBC, bool FAST, int CPT, int MINB>
 static bool configure_scan() {
   using Lyt = ScanLayout<TX, TBC, FAST>;
   static bool done[64] = {false};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
   if (!done[dev]) {
-    if (cudaFuncSetAttribute(selective_scan_kernel<TX, TBC, FAST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Lyt::BYTES) != cudaSuccess)
+    if (cudaFuncSetAttribute(selective_scan_kernel<TX, TBC, FAST, CPT, MINB>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, Lyt::BYTES) != cudaSuccess)
       return false;
     done[dev] = true;
   }
   return true;
 }
 
-template <typename TX, typename TBC, bool FAST>
+template <typename TX, typename TBC, bool FAST, int CPT, int MINB>
 static int resident_ctas() {
   using Lyt = ScanLayout<TX, TBC, FAST>;
   static int cache[64] = {0};
@@ -591,31 +649,39 @@ static int resident_ctas() {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 2 * num_sms();
   if (cache[dev] == 0) {
     int per_sm = 0;
-    configure_scan<TX, TBC, FAST>();
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, selective_scan_kernel<TX, TBC, FAST>, SCAN_THREADS,
-                                                      Lyt::BYTES) != cudaSuccess || per_sm < 1)
+    configure_scan<TX, TBC, FAST, CPT, MINB>();
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, selective_scan_kernel<TX, TBC, FAST, CPT, MINB>,
+                                                      ScanShape<CPT, MINB>::THREADS, Lyt::BYTES) != cudaSuccess ||
+        per_sm < 1)
       per_sm = 1;
     cache[dev] = per_sm * num_sms();
   }
   return cache[dev];
 }
 
-// Time chunk: every CTA of the launch resident at once (a CTA waiting on its
-// predecessor must never wait for a free SM slot), preferring chunks of at
-// least 8192 steps once half of the resident slots are filled, since each
-// chunk after the first replays its head.
+template <typename TX, typename TBC, bool FAST, int CPT, int MINB>
+static jamba_status launch_kernel(size_t recs, const CUtensorMap& mx, const CUtensorMap& mz, const CUtensorMap& mdt,
+                                  const CUtensorMap& mB, const CUtensorMap& mC, const ScanArgs& a, cudaStream_t st) {
+  if (!configure_scan<TX, TBC, FAST, CPT, MINB>()) return fail(JAMBA_ERR_CUDA, "scan: kernel configuration failed");
+  selective_scan_kernel<TX, TBC, FAST, CPT, MINB>
+      <<<(unsigned)recs, ScanShape<CPT, MINB>::THREADS, ScanLayout<TX, TBC, FAST>::BYTES, st>>>(mx, mz, mdt, mB,
+                                                                                                  mC, a);
+  JB_CUDA(cudaGetLastError());
+  return JAMBA_OK;
+}
+
+// Time chunk: as many chunks as keep every CTA of the launch resident at once
+// (a CTA waiting on its predecessor must never wait for a free SM slot).
+// Shorter chunks replay shorter heads and a CTA's step rate is bounded by its
+// own dependency chain, so full occupancy is the fastest choice measured.
 int scan_auto_chunk(int batch, int L, int di, int dtype, int bc_dtype) {
   const int cgroups = (di + SCAN_CH - 1) / SCAN_CH;
   const long long groups = (long long)batch * cgroups;
   int cap;
-  if (dtype == JAMBA_BF16 && bc_dtype == JAMBA_BF16) cap = resident_ctas<bf16, bf16, true>();
-  else if (dtype == JAMBA_BF16) cap = resident_ctas<bf16, float, true>();
-  else cap = resident_ctas<float, float, false>();
-  long long full = cap / groups;
-  long long half = full / 2;
-  long long by_len = (L + 8191) / 8192;
-  long long n_chunks = by_len > half ? by_len : half;
-  if (n_chunks > full) n_chunks = full;
+  if (dtype == JAMBA_BF16 && bc_dtype == JAMBA_BF16) cap = resident_ctas<bf16, bf16, true, FastShape::CPT, FastShape::MINB>();
+  else if (dtype == JAMBA_BF16) cap = resident_ctas<bf16, float, true, FastShape::CPT, FastShape::MINB>();
+  else cap = resident_ctas<float, float, false, GenShape::CPT, GenShape::MINB>();
+  long long n_chunks = cap / groups;
   if (n_chunks < 1) n_chunks = 1;
   int chunk = (int)((L + n_chunks - 1) / n_chunks);
   chunk = (chunk + 15) & ~15;
@@ -653,17 +719,9 @@ static jamba_status launch_scan(const ScanCall& s, cudaStream_t st) {
   if (!a.err) return fail(JAMBA_ERR_CUDA, "could not allocate the device status word");
   JB_CUDA(cudaMemsetAsync(w, 0, 256 + flags_bytes, st));
   if (recs > 0x7fffffffull) return fail(JAMBA_ERR_UNSUPPORTED, "scan: too many chunks");
-  if (sizeof(TX) == 2) {
-    if (!configure_scan<TX, TBC, true>()) return fail(JAMBA_ERR_CUDA, "scan: kernel configuration failed");
-    selective_scan_kernel<TX, TBC, true>
-        <<<(unsigned)recs, SCAN_THREADS, ScanLayout<TX, TBC, true>::BYTES, st>>>(mx, mz, mdt, mB, mC, a);
-    JB_CUDA(cudaGetLastError());
-  }
-  if (!configure_scan<TX, TBC, false>()) return fail(JAMBA_ERR_CUDA, "scan: kernel configuration failed");
-  selective_scan_kernel<TX, TBC, false>
-      <<<(unsigned)recs, SCAN_THREADS, ScanLayout<TX, TBC, false>::BYTES, st>>>(mx, mz, mdt, mB, mC, a);
-  JB_CUDA(cudaGetLastError());
-  return JAMBA_OK;
+  if (sizeof(TX) == 2)
+    JB_TRY((launch_kernel<TX, TBC, true, FastShape::CPT, FastShape::MINB>(recs, mx, mz, mdt, mB, mC, a, st)));
+  return launch_kernel<TX, TBC, false, GenShape::CPT, GenShape::MINB>(recs, mx, mz, mdt, mB, mC, a, st);
 }
 
 jamba_status scan_run(const ScanCall& s, cudaStream_t st) {
@@ -674,7 +732,7 @@ jamba_status scan_run(const ScanCall& s, cudaStream_t st) {
   if (s.chunk <= 0 || s.chunk % 16) return fail(JAMBA_ERR_INVALID_ARG, "scan: chunk must be a positive multiple of 16");
   if (s.ld_x < s.di || s.ld_z < s.di || s.ld_dt < s.di || s.ld_y < s.di || s.ld_b < NS || s.ld_c < NS)
     return fail(JAMBA_ERR_INVALID_ARG, "scan: leading dimension below the row width");
-  if (s.ld_y % 2) return fail(JAMBA_ERR_INVALID_ARG, "scan: the leading dimension of y must be even");
+  if (s.ld_y % 4) return fail(JAMBA_ERR_INVALID_ARG, "scan: the leading dimension of y must be a multiple of 4");
   if (!aligned16(s.y)) return fail(JAMBA_ERR_INVALID_ARG, "scan: y must be 16-byte aligned");
   if (s.ws_bytes < scan_workspace_bytes(s.batch, s.L, s.di, s.chunk) || !s.ws || !aligned16(s.ws))
     return fail(JAMBA_ERR_WORKSPACE, "scan: workspace too small");
