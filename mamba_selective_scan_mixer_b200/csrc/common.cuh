@@ -53,6 +53,12 @@ __device__ __forceinline__ float softplus(float v) {
   return v > 20.0f ? v : log1pf(__expf(v));
 }
 
+// Programmatic dependent launch: wait for the preceding grid in the stream to
+// complete (a no-op when the launch carried no programmatic dependency), and
+// let the next grid begin launching while this one runs.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- packed fp32
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
   float2 d;

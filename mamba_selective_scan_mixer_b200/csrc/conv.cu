@@ -55,6 +55,8 @@ conv_prefill_kernel(const T* __restrict__ x, long long ld_x, const T* __restrict
                     T* __restrict__ out, const float* __restrict__ st_in, float* __restrict__ st_out, int L,
                     int C) {
   constexpr int V = Vec16<T>::N;
+  griddep_wait();
+  griddep_launch();
   const int c0 = (blockIdx.x * CONV_THREADS + threadIdx.x) * V;
   if (c0 >= C) return;
   const int b = blockIdx.z;
@@ -111,6 +113,8 @@ template <typename T>
 __global__ void __launch_bounds__(256)
 conv_step_kernel(const T* __restrict__ x, long long ld_x, const T* __restrict__ w, const T* __restrict__ bias,
                  T* __restrict__ out, float* __restrict__ state, int batch, int C) {
+  griddep_wait();
+  griddep_launch();
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (long long)batch * C) return;
   const int b = (int)(i / C), c = (int)(i - (long long)b * C);
@@ -135,14 +139,13 @@ jamba_status conv_prefill(const void* x, long long ld_x, const void* w, const vo
     return fail(JAMBA_ERR_INVALID_ARG, "conv: channels and row stride must fill 16-byte vectors");
   dim3 grid((C / V + CONV_THREADS - 1) / CONV_THREADS, (L + CONV_TQ - 1) / CONV_TQ, batch);
   if (dtype == JAMBA_BF16)
-    conv_prefill_kernel<bf16><<<grid, CONV_THREADS, 0, s>>>(
-        reinterpret_cast<const bf16*>(x), ld_x, reinterpret_cast<const bf16*>(w), reinterpret_cast<const bf16*>(b),
-        reinterpret_cast<bf16*>(out), st_in, st_out, L, C);
+    JB_CUDA(launch_pdl(conv_prefill_kernel<bf16>, grid, dim3(CONV_THREADS), 0, s, reinterpret_cast<const bf16*>(x),
+                       ld_x, reinterpret_cast<const bf16*>(w), reinterpret_cast<const bf16*>(b),
+                       reinterpret_cast<bf16*>(out), st_in, st_out, L, C));
   else
-    conv_prefill_kernel<float><<<grid, CONV_THREADS, 0, s>>>(
-        reinterpret_cast<const float*>(x), ld_x, reinterpret_cast<const float*>(w),
-        reinterpret_cast<const float*>(b), reinterpret_cast<float*>(out), st_in, st_out, L, C);
-  JB_CUDA(cudaGetLastError());
+    JB_CUDA(launch_pdl(conv_prefill_kernel<float>, grid, dim3(CONV_THREADS), 0, s, reinterpret_cast<const float*>(x),
+                       ld_x, reinterpret_cast<const float*>(w), reinterpret_cast<const float*>(b),
+                       reinterpret_cast<float*>(out), st_in, st_out, L, C));
   return JAMBA_OK;
 }
 
@@ -151,14 +154,13 @@ jamba_status conv_step(const void* x, long long ld_x, const void* w, const void*
   const long long n = (long long)batch * C;
   const unsigned grid = (unsigned)((n + 255) / 256);
   if (dtype == JAMBA_BF16)
-    conv_step_kernel<bf16><<<grid, 256, 0, s>>>(reinterpret_cast<const bf16*>(x), ld_x,
-                                               reinterpret_cast<const bf16*>(w), reinterpret_cast<const bf16*>(b),
-                                               reinterpret_cast<bf16*>(out), state, batch, C);
+    JB_CUDA(launch_pdl(conv_step_kernel<bf16>, dim3(grid), dim3(256), 0, s, reinterpret_cast<const bf16*>(x), ld_x,
+                       reinterpret_cast<const bf16*>(w), reinterpret_cast<const bf16*>(b),
+                       reinterpret_cast<bf16*>(out), state, batch, C));
   else
-    conv_step_kernel<float><<<grid, 256, 0, s>>>(reinterpret_cast<const float*>(x), ld_x,
-                                                reinterpret_cast<const float*>(w), reinterpret_cast<const float*>(b),
-                                                reinterpret_cast<float*>(out), state, batch, C);
-  JB_CUDA(cudaGetLastError());
+    JB_CUDA(launch_pdl(conv_step_kernel<float>, dim3(grid), dim3(256), 0, s, reinterpret_cast<const float*>(x), ld_x,
+                       reinterpret_cast<const float*>(w), reinterpret_cast<const float*>(b),
+                       reinterpret_cast<float*>(out), state, batch, C));
   return JAMBA_OK;
 }
 

@@ -19,8 +19,8 @@ static jamba_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, cons
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::BYTES));
     configured[dev] = true;
   }
-  gemm_bf16_tc_kernel<BN, STAGES, EPI, TRANS><<<grid, GEMM_THREADS, S::BYTES, s>>>(ma, mb, mb2, mc, p);
-  JB_CUDA(cudaGetLastError());
+  JB_CUDA(launch_pdl(gemm_bf16_tc_kernel<BN, STAGES, EPI, TRANS>, dim3(grid), dim3(GEMM_THREADS), S::BYTES, s, ma, mb,
+                     mb2, mc, p));
   return JAMBA_OK;
 }
 
@@ -148,6 +148,8 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__
                                                        int K, int epi, int trans, GemmParams p) {
   __shared__ float As[16][64 + 4];
   __shared__ float Bs[16][64 + 4];
+  griddep_wait();
+  griddep_launch();
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
   float acc[4][4] = {};
@@ -207,10 +209,8 @@ jamba_status gemm_f32(const GemmDesc& g, cudaStream_t s) {
   p.ldr = g.ldr;
   p.bias = g.bias;
   dim3 grid((g.N + 63) / 64, (g.M + 63) / 64);
-  gemm_f32_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const float*>(g.a), g.lda,
-                                       reinterpret_cast<const float*>(g.b), g.ldb, g.M, g.N, g.K, g.epi,
-                                       g.transpose_out, p);
-  JB_CUDA(cudaGetLastError());
+  JB_CUDA(launch_pdl(gemm_f32_kernel, grid, dim3(256), 0, s, reinterpret_cast<const float*>(g.a), g.lda,
+                     reinterpret_cast<const float*>(g.b), g.ldb, g.M, g.N, g.K, g.epi, g.transpose_out, p));
   return JAMBA_OK;
 }
 

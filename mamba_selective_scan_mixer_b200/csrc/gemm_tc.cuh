@@ -283,23 +283,42 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_holder;
-  const int ntiles = total_tiles(p);
+  griddep_launch();   // the next kernel may begin its own prologue
 
   if (warp == 0) {
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      // Swap-AB (decode): A is a weight matrix, independent of the previous
+      // kernel, so the first ring stages of it stream in before the wait.
+      int pre = 0;
+      if constexpr (TRANS) {
+        if ((int)blockIdx.x < p.m_tiles * p.n_tiles * p.splits) {
+          TileInfo t0;
+          decode_tile<BN_OUT>(p, blockIdx.x, t0);
+          for (int kt = t0.kt0; kt < t0.kt1 && pre < STAGES; ++kt, ++pre) {
+            const uint32_t fb = full0 + 8 * pre;
+            mbar_arrive_tx(fb, S::A_BYTES + S::B_BYTES);
+            tma_load_2d(smem_u32(sA + pre * S::A_BYTES), &tmA, fb, kt * 64, t0.m0);
+          }
+        }
+      }
+      griddep_wait();
+      const int ntiles = total_tiles(p);
+      int issued = 0;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
         TileInfo ti;
         decode_tile<BN_OUT>(p, t, ti);
-        for (int kt = ti.kt0; kt < ti.kt1; ++kt) {
-          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, p.err)) { ok = false; break; }
+        for (int kt = ti.kt0; kt < ti.kt1; ++kt, ++issued) {
           const uint32_t fb = full0 + 8 * stage;
-          mbar_arrive_tx(fb, S::A_BYTES + S::B_BYTES);
           const uint32_t a_dst = smem_u32(sA + stage * S::A_BYTES);
           const uint32_t b_dst = smem_u32(sB + stage * S::B_BYTES);
-          tma_load_2d(a_dst, &tmA, fb, kt * 64, ti.m0);
+          if (issued >= pre) {
+            if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, p.err)) { ok = false; break; }
+            mbar_arrive_tx(fb, S::A_BYTES + S::B_BYTES);
+            tma_load_2d(a_dst, &tmA, fb, kt * 64, ti.m0);
+          }
           if (!p.grouped) {
             tma_load_2d(b_dst, &tmB, fb, kt * 64, ti.n0);
           } else if (EPI != EPI_SWIGLU) {
@@ -313,6 +332,8 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       }
     }
   } else if (warp == 1) {
+    griddep_wait();
+    const int ntiles = total_tiles(p);
     if (lane == 0) {
       constexpr uint32_t IDESC = idesc_bf16(128, BN);
       int stage = 0;
@@ -346,6 +367,8 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       mbar_wait(drain, 0, p.err);
     }
   } else {
+    griddep_wait();
+    const int ntiles = total_tiles(p);
     const int q = warp & 3;                 // TMEM lane quarter this warp may access
     const int half = (warp - 2) >> 2;       // which of the two warps of this quarter
     int it = 0;

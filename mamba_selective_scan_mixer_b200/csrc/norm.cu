@@ -21,6 +21,8 @@ __device__ __forceinline__ float warp_sum(float v) {
 template <typename T>
 __global__ void __launch_bounds__(256)
 rmsnorm_kernel(const T* __restrict__ x, const float* __restrict__ w, T* __restrict__ out, int cols, float eps) {
+  griddep_wait();
+  griddep_launch();
   const long long row = blockIdx.x;
   const T* xr = x + row * cols;
   T* orow = out + row * cols;
@@ -51,6 +53,8 @@ __global__ void __launch_bounds__(512)
 xproj_norm_kernel(const float* __restrict__ part, int splits, long long split_stride, int T, int R, int N,
                   const float* __restrict__ w_dt, const float* __restrict__ w_B, const float* __restrict__ w_C,
                   int inner_norm, float eps, TD* __restrict__ dtlow, float* __restrict__ bc) {
+  griddep_wait();
+  griddep_launch();
   const long long t = blockIdx.x;
   const int col = threadIdx.x, W = R + 2 * N;
   const int lane = col & 31, warp = col >> 5;
@@ -101,6 +105,8 @@ template <typename T>
 __global__ void __launch_bounds__(256)
 splitk_reduce_kernel(const float* __restrict__ part, int splits, long long split_stride, long long n,
                      const T* __restrict__ residual, T* __restrict__ out) {
+  griddep_wait();
+  griddep_launch();
   const long long i = ((long long)blockIdx.x * 256 + threadIdx.x) * 4;
   if (i >= n) return;
   float4 acc = *reinterpret_cast<const float4*>(part + i);
@@ -119,12 +125,11 @@ splitk_reduce_kernel(const float* __restrict__ part, int splits, long long split
 jamba_status rmsnorm(const void* x, const float* w, void* out, int rows, int cols, float eps, int dtype,
                      cudaStream_t s) {
   if (dtype == JAMBA_BF16)
-    rmsnorm_kernel<bf16><<<rows, 256, 0, s>>>(reinterpret_cast<const bf16*>(x), w, reinterpret_cast<bf16*>(out),
-                                             cols, eps);
+    JB_CUDA(launch_pdl(rmsnorm_kernel<bf16>, dim3(rows), dim3(256), 0, s, reinterpret_cast<const bf16*>(x), w,
+                       reinterpret_cast<bf16*>(out), cols, eps));
   else
-    rmsnorm_kernel<float><<<rows, 256, 0, s>>>(reinterpret_cast<const float*>(x), w, reinterpret_cast<float*>(out),
-                                              cols, eps);
-  JB_CUDA(cudaGetLastError());
+    JB_CUDA(launch_pdl(rmsnorm_kernel<float>, dim3(rows), dim3(256), 0, s, reinterpret_cast<const float*>(x), w,
+                       reinterpret_cast<float*>(out), cols, eps));
   return JAMBA_OK;
 }
 
@@ -134,12 +139,11 @@ jamba_status xproj_norm(const float* part, int splits, long long split_stride, i
   if (R + 2 * N > 512) return fail(JAMBA_ERR_UNSUPPORTED, "x_proj width above 512");
   const int threads = ((R + 2 * N + 31) / 32) * 32;
   if (dtype == JAMBA_BF16)
-    xproj_norm_kernel<bf16><<<T, threads, 0, s>>>(part, splits, split_stride, T, R, N, w_dt, w_B, w_C, inner_norm,
-                                                  eps, reinterpret_cast<bf16*>(dtlow), bc);
+    JB_CUDA(launch_pdl(xproj_norm_kernel<bf16>, dim3(T), dim3(threads), 0, s, part, splits, split_stride, T, R, N, w_dt,
+                       w_B, w_C, inner_norm, eps, reinterpret_cast<bf16*>(dtlow), bc));
   else
-    xproj_norm_kernel<float><<<T, threads, 0, s>>>(part, splits, split_stride, T, R, N, w_dt, w_B, w_C, inner_norm,
-                                                   eps, reinterpret_cast<float*>(dtlow), bc);
-  JB_CUDA(cudaGetLastError());
+    JB_CUDA(launch_pdl(xproj_norm_kernel<float>, dim3(T), dim3(threads), 0, s, part, splits, split_stride, T, R, N,
+                       w_dt, w_B, w_C, inner_norm, eps, reinterpret_cast<float*>(dtlow), bc));
   return JAMBA_OK;
 }
 
@@ -148,13 +152,11 @@ jamba_status splitk_reduce(const float* part, int splits, long long split_stride
   if (n % 4) return fail(JAMBA_ERR_INVALID_ARG, "split-K reduce: size must be a multiple of 4");
   const unsigned grid = (unsigned)((n / 4 + 255) / 256);
   if (dtype == JAMBA_BF16)
-    splitk_reduce_kernel<bf16><<<grid, 256, 0, s>>>(part, splits, split_stride, n,
-                                                   reinterpret_cast<const bf16*>(residual), reinterpret_cast<bf16*>(out));
+    JB_CUDA(launch_pdl(splitk_reduce_kernel<bf16>, dim3(grid), dim3(256), 0, s, part, splits, split_stride, n,
+                       reinterpret_cast<const bf16*>(residual), reinterpret_cast<bf16*>(out)));
   else
-    splitk_reduce_kernel<float><<<grid, 256, 0, s>>>(part, splits, split_stride, n,
-                                                    reinterpret_cast<const float*>(residual),
-                                                    reinterpret_cast<float*>(out));
-  JB_CUDA(cudaGetLastError());
+    JB_CUDA(launch_pdl(splitk_reduce_kernel<float>, dim3(grid), dim3(256), 0, s, part, splits, split_stride, n,
+                       reinterpret_cast<const float*>(residual), reinterpret_cast<float*>(out)));
   return JAMBA_OK;
 }
 

@@ -582,6 +582,8 @@ __global__ void __launch_bounds__(256)
 ssm_step_kernel(const TX* __restrict__ xc, const TX* __restrict__ z, long long ld_z, const float* __restrict__ dt,
                 const float* __restrict__ bc, long long ld_bc, const float* __restrict__ A,
                 const float* __restrict__ D, float* __restrict__ state, TX* __restrict__ y, int batch, int di) {
+  griddep_wait();
+  griddep_launch();
   const long long i = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 2;   // flat (row, channel)
   const int q = threadIdx.x & 3;
   const bool live = i < (long long)batch * di;
@@ -749,12 +751,13 @@ jamba_status ssm_step(const void* xc, const void* z, long long ld_z, const float
   const long long n = (long long)batch * di * 4;
   const unsigned grid = (unsigned)((n + 255) / 256);
   if (dtype == JAMBA_BF16)
-    ssm_step_kernel<bf16><<<grid, 256, 0, st>>>(reinterpret_cast<const bf16*>(xc), reinterpret_cast<const bf16*>(z),
-                                               ld_z, dt, bc, ld_bc, A, D, state, reinterpret_cast<bf16*>(y), batch, di);
+    JB_CUDA(launch_pdl(ssm_step_kernel<bf16>, dim3(grid), dim3(256), 0, st, reinterpret_cast<const bf16*>(xc),
+                       reinterpret_cast<const bf16*>(z), ld_z, dt, bc, ld_bc, A, D, state, reinterpret_cast<bf16*>(y),
+                       batch, di));
   else
-    ssm_step_kernel<float><<<grid, 256, 0, st>>>(reinterpret_cast<const float*>(xc), reinterpret_cast<const float*>(z),
-                                                ld_z, dt, bc, ld_bc, A, D, state, reinterpret_cast<float*>(y), batch, di);
-  JB_CUDA(cudaGetLastError());
+    JB_CUDA(launch_pdl(ssm_step_kernel<float>, dim3(grid), dim3(256), 0, st, reinterpret_cast<const float*>(xc),
+                       reinterpret_cast<const float*>(z), ld_z, dt, bc, ld_bc, A, D, state, reinterpret_cast<float*>(y),
+                       batch, di));
   return JAMBA_OK;
 }
 
