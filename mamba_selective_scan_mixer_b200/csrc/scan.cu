@@ -14,10 +14,13 @@
 //
 // Chunks of the same channels run concurrently.  Before the state entering a
 // chunk is known, its outputs depend on it through C_t . (P_t * h_in), P_t the
-// decay product since the chunk start.  P_t only shrinks, and once it is
-// exactly zero for every channel of a warp the warp's later outputs no longer
-// depend on h_in: the first pass therefore runs the chunk's head (the steps
-// before that point) in state-only mode and writes final outputs after it.
+// decay product since the chunk start.  P_t only shrinks (A < 0), and once it
+// is at most 2^-40 for every state of every channel of a warp, h_in's share of
+// the warp's later states is at most 2^-40 |h_in| -- 2^16 times below the fp32
+// rounding unit -- and is dropped: the first pass runs the chunk's head (the
+// steps before that point) in state-only mode and writes final outputs after
+// it.  (Waiting for P_t to underflow to exact zero instead would lengthen the
+// head about fourfold: ln(2^-149) / ln(2^-40).)
 // At the chunk end the CTA publishes (P, local end state) -- or its true end
 // state if every warp's P died -- and looks back over its predecessors'
 // records (decoupled look-back, (P2, h2) o (P1, h1) = (P2 P1, P2 h1 + h2)).
@@ -32,6 +35,7 @@
 // with one exponential per state.  Both kernels are launched; each CTA runs
 // only if its channels belong to its kind.
 #include <string>
+#include <type_traits>
 
 #include "common.cuh"
 #include "host.hpp"
@@ -44,6 +48,7 @@ constexpr int SCAN_STAGES = 3;
 constexpr int NS = 16;                              // d_state
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr int REC = 3 * SCAN_CH * NS;               // floats per chunk record: P, h, inclusive h
+constexpr float CARRY_DROP = 0x1p-40f;              // decay product below which h_in's share is dropped
 
 // CTA shape: CPT channels per consumer thread, 256 / (32 CPT) consumer warps,
 // one producer warp; MINB resident CTAs per SM (sets the register cap).
@@ -221,19 +226,22 @@ __device__ __forceinline__ bool producer_pass(const CUtensorMap* mx, const CUten
   return ok;
 }
 
-// One time step for this thread's CPT channels: updates h (and, while `head`,
-// the decay trackers) and returns the pre-gate outputs.
-template <bool FAST, int CPT>
+// One time step for this thread's CPT channels.  HEAD: state only, tracking
+// the decay product (no output is formed); otherwise the state and the
+// pre-gate outputs.
+template <bool FAST, int CPT, bool HEAD>
 __device__ __forceinline__ void scan_step(float2 (&h)[CPT][8], const float* xv, const float* dv, const float* bc,
-                                          const float* A2_0, const float* sA2c, const float* Dv, bool head,
+                                          const float* A2_0, const float* sA2c, const float* Dv,
                                           float (&R)[CPT], float2 (&P)[CPT][8], float* y) {
   float Bv[16], Cv[16];
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const float4 b4 = *reinterpret_cast<const float4*>(bc + 4 * k);
-    const float4 c4 = *reinterpret_cast<const float4*>(bc + 16 + 4 * k);
     Bv[4 * k] = b4.x; Bv[4 * k + 1] = b4.y; Bv[4 * k + 2] = b4.z; Bv[4 * k + 3] = b4.w;
-    Cv[4 * k] = c4.x; Cv[4 * k + 1] = c4.y; Cv[4 * k + 2] = c4.z; Cv[4 * k + 3] = c4.w;
+    if constexpr (!HEAD) {
+      const float4 c4 = *reinterpret_cast<const float4*>(bc + 16 + 4 * k);
+      Cv[4 * k] = c4.x; Cv[4 * k + 1] = c4.y; Cv[4 * k + 2] = c4.z; Cv[4 * k + 3] = c4.w;
+    }
   }
 #pragma unroll
   for (int j = 0; j < CPT; ++j) {
@@ -243,7 +251,7 @@ __device__ __forceinline__ void scan_step(float2 (&h)[CPT][8], const float* xv, 
     if constexpr (FAST) {
       const float r = ex2(dj * A2_0[j]);
       powers16(r, pw);
-      if (head) R[j] *= r;
+      if constexpr (HEAD) R[j] *= r;
     } else {
 #pragma unroll
       for (int n = 0; n < NS; ++n) pw[n] = ex2(dj * sA2c[j * NS + n]);
@@ -254,20 +262,53 @@ __device__ __forceinline__ void scan_step(float2 (&h)[CPT][8], const float* xv, 
       const float2 a = make_float2(pw[2 * n2], pw[2 * n2 + 1]);
       const float2 uB = fmul2(make_float2(u, u), make_float2(Bv[2 * n2], Bv[2 * n2 + 1]));
       h[j][n2] = ffma2(a, h[j][n2], uB);
-      if (n2 & 1) y1 = ffma2(make_float2(Cv[2 * n2], Cv[2 * n2 + 1]), h[j][n2], y1);
-      else y0 = ffma2(make_float2(Cv[2 * n2], Cv[2 * n2 + 1]), h[j][n2], y0);
-      if constexpr (!FAST) {
-        if (head) P[j][n2] = fmul2(P[j][n2], a);
+      if constexpr (HEAD) {
+        if constexpr (!FAST) P[j][n2] = fmul2(P[j][n2], a);
+      } else {
+        if (n2 & 1) y1 = ffma2(make_float2(Cv[2 * n2], Cv[2 * n2 + 1]), h[j][n2], y1);
+        else y0 = ffma2(make_float2(Cv[2 * n2], Cv[2 * n2 + 1]), h[j][n2], y0);
       }
     }
-    y[j] = (y0.x + y0.y) + (y1.x + y1.y) + Dv[j] * xj;
+    if constexpr (!HEAD) y[j] = (y0.x + y0.y) + (y1.x + y1.y) + Dv[j] * xj;
+  }
+}
+
+// One stage (up to SCAN_Q steps) of one warp, specialised on the warp-uniform
+// head mode; yrow points at this thread's first output of the stage.
+template <typename TX, bool FAST, int CPT, bool HEAD>
+__device__ __forceinline__ void scan_stage(const uint8_t* st, int off_z, int off_dt, int off_bcf, int nq, int cl,
+                                           float2 (&h)[CPT][8], const float* A2_0, const float* sA2c,
+                                           const float* Dv, float (&R)[CPT], float2 (&P)[CPT][8], bool valid,
+                                           TX* yrow, long long ld_y) {
+  const TX* sx = reinterpret_cast<const TX*>(st);
+  const TX* sz = reinterpret_cast<const TX*>(st + off_z);
+  const float* sdt = reinterpret_cast<const float*>(st + off_dt);
+  const float* bcf = reinterpret_cast<const float*>(st + off_bcf);
+#pragma unroll
+  for (int q = 0; q < SCAN_Q; ++q) {
+    if (q < nq) {
+      float xv[CPT], dv[CPT], y[CPT];
+      Vec<TX, CPT>::load(sx + q * SCAN_CH + cl, xv);
+      Vec<float, CPT>::load(sdt + q * SCAN_CH + cl, dv);
+      scan_step<FAST, CPT, HEAD>(h, xv, dv, bcf + q * 32, A2_0, sA2c, Dv, R, P, y);
+      if constexpr (!HEAD) {
+        if (valid) {
+          float zv[CPT];
+          Vec<TX, CPT>::load(sz + q * SCAN_CH + cl, zv);
+#pragma unroll
+          for (int j = 0; j < CPT; ++j) y[j] *= silu(zv[j]);
+          Vec<TX, CPT>::store(yrow + q * ld_y, y);
+        }
+      }
+    }
   }
 }
 
 // Consumer warps: the stages of one pass over window [ts, te).  While `head`
 // the warp writes nothing and tracks the decay product; it leaves head mode
-// at the first stage end where that product is zero on all its channels.
-template <typename TX, typename TBC, bool FAST, int CPT>
+// at the first stage end where that product is at most CARRY_DROP on all its
+// channels.
+template <typename TX, typename TBC, bool FAST, int CPT, bool MAY_HEAD>
 __device__ __forceinline__ bool consumer_pass(uint8_t* smem, const ScanCtx& cx, const ScanArgs& a, int ts, int te,
                                               int te_warp, int nsub, int g0, float2 (&h)[CPT][8], bool& head,
                                               int& t_head_end,
@@ -284,47 +325,32 @@ __device__ __forceinline__ bool consumer_pass(uint8_t* smem, const ScanCtx& cx, 
     if (!__all_sync(0xffffffffu, mbar_wait(ready0 + 8 * slot, (uint32_t)((g / SCAN_STAGES) & 1), a.err)))
       return false;
     const uint8_t* st = smem + slot * Lyt::STAGE;
-    const TX* sx = reinterpret_cast<const TX*>(st);
-    const TX* sz = reinterpret_cast<const TX*>(st + Lyt::OFF_Z);
-    const float* sdt = reinterpret_cast<const float*>(st + Lyt::OFF_DT);
-    const float* bcf = reinterpret_cast<const float*>(st + Lyt::OFF_BCF);
     const int tb = ts + i * SCAN_Q;
     const int nq = min(SCAN_Q, te - tb);
-    auto step = [&](int q) {
-      float xv[CPT], dv[CPT], y[CPT];
-      Vec<TX, CPT>::load(sx + q * SCAN_CH + cl, xv);
-      Vec<float, CPT>::load(sdt + q * SCAN_CH + cl, dv);
-      scan_step<FAST, CPT>(h, xv, dv, bcf + q * 32, A2_0, sA2c, Dv, head, R, P, y);
-      if (!head && valid) {
-        float zv[CPT];
-        Vec<TX, CPT>::load(sz + q * SCAN_CH + cl, zv);
-#pragma unroll
-        for (int j = 0; j < CPT; ++j) y[j] *= silu(zv[j]);
-        Vec<TX, CPT>::store(yg + (cx.row0 + tb + q) * a.ld_y + c, y);
-      }
-    };
     if (tb >= te_warp) {
       // this warp's own head ended earlier: nothing of this stage is needed
-    } else if (nq == SCAN_Q) {
-#pragma unroll
-      for (int q = 0; q < SCAN_Q; ++q) step(q);
+    } else if (MAY_HEAD && head) {
+      scan_stage<TX, FAST, CPT, MAY_HEAD>(st, Lyt::OFF_Z, Lyt::OFF_DT, Lyt::OFF_BCF, nq, cl, h, A2_0, sA2c, Dv, R, P,
+                                          valid, yg + (cx.row0 + tb) * a.ld_y + c, a.ld_y);
     } else {
-      for (int q = 0; q < nq; ++q) step(q);
+      scan_stage<TX, FAST, CPT, false>(st, Lyt::OFF_Z, Lyt::OFF_DT, Lyt::OFF_BCF, nq, cl, h, A2_0, sA2c, Dv, R, P,
+                                       valid, yg + (cx.row0 + tb) * a.ld_y + c, a.ld_y);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(empty0 + 8 * slot);
-    if (head) {
+    if (MAY_HEAD && head) {
       bool zero = !valid;
       if (!zero) {
         zero = true;
         if constexpr (FAST) {
 #pragma unroll
-          for (int j = 0; j < CPT; ++j) zero = zero && R[j] == 0.f;
+          for (int j = 0; j < CPT; ++j) zero = zero && R[j] <= CARRY_DROP;
         } else {
 #pragma unroll
           for (int j = 0; j < CPT; ++j)
 #pragma unroll
-            for (int n2 = 0; n2 < 8; ++n2) zero = zero && P[j][n2].x == 0.f && P[j][n2].y == 0.f;
+            for (int n2 = 0; n2 < 8; ++n2)
+              zero = zero && P[j][n2].x <= CARRY_DROP && P[j][n2].y <= CARRY_DROP;
         }
       }
       if (__all_sync(0xffffffffu, zero)) {
@@ -432,7 +458,7 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
   if (producer)
     pass_ok = producer_pass<TX, TBC, FAST>(&mx, &mz, &mdt, &mB, &mC, smem, cx, cx.t0, nsub1, 0, a.err);
   else
-    pass_ok = consumer_pass<TX, TBC, FAST, CPT>(smem, cx, a, cx.t0, cx.t1, cx.t1, nsub1, 0, h, head, t_head_end, R,
+    pass_ok = consumer_pass<TX, TBC, FAST, CPT, true>(smem, cx, a, cx.t0, cx.t1, cx.t1, nsub1, 0, h, head, t_head_end, R,
                                                 P, A2_0, sA2c, Dv, valid, c);
   if (!producer && head) t_head_end = cx.t1;
   if (!producer && (tid & 31) == 0) s_head_end[warp] = t_head_end;
@@ -513,7 +539,7 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
           } else {
             sH[o] = fmaf(sP[o], __ldcg(rP + SCAN_CH * NS + o), sH[o]);
             sP[o] *= __ldcg(rP + o);
-            allzero = allzero && sP[o] == 0.f;
+            allzero = allzero && sP[o] <= CARRY_DROP;
           }
         }
       }
@@ -532,7 +558,11 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
       for (int n2 = 0; n2 < 8; ++n2)
         hin[j][n2] = producer ? make_float2(0.f, 0.f)
                               : make_float2(sH[(cl + j) * NS + 2 * n2], sH[(cl + j) * NS + 2 * n2 + 1]);
-    __syncthreads();   // the ring is reused by pass 2
+    // The ring is reused by pass 2: TMA (the async proxy) will overwrite the
+    // scratch written above through ordinary stores, so those stores are
+    // ordered before it with a proxy fence ahead of the barrier.
+    fence_async_shared();
+    __syncthreads();
     if (!independent) {
       // true end state h + P_end * h_in, published as this chunk's inclusive record
       if (!producer) {
@@ -558,7 +588,7 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
       bool head2 = false;
       int unused = 0;
       // each warp replays only its own head; the stages after it are passed through
-      consumer_pass<TX, TBC, FAST, CPT>(smem, cx, a, cx.t0, t_head_max, s_head_end[warp], nsub2, nsub1, hin, head2,
+      consumer_pass<TX, TBC, FAST, CPT, false>(smem, cx, a, cx.t0, t_head_max, s_head_end[warp], nsub2, nsub1, hin, head2,
                                         unused, R, P, A2_0, sA2c, Dv, valid, c);
     }
   }

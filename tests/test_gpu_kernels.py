@@ -143,6 +143,40 @@ def test_scan_chunk_invariance(dev, chunk):
     assert rel_l2(y1, wy) < TOL_F32
 
 
+def _bf16_elementwise_bad(got, want):
+    """Elements further from the exact value than one bf16 step (2^-7
+    relative) plus an fp32-accumulation allowance: a correct fp32 scan
+    rounded to bf16 has none."""
+    scale = np.sqrt(np.mean(want ** 2))
+    return int((np.abs(got - want) > 2.0 ** -7 * np.abs(want) + 1e-5 * scale).sum())
+
+
+@pytest.mark.parametrize("dt_kind", ["iid", "per_channel"])
+@pytest.mark.parametrize("chunk", [0, 512, 2048])
+def test_scan_bf16_elementwise_many_chunks(dev, dt_kind, chunk):
+    """Every sampled output within one bf16 step of the exact scan, over many
+    chunks (several waves of CTAs at chunk 512) and both dt regimes: i.i.d.
+    per step (short carried-state heads) and fixed per channel, log-uniform
+    in [1e-3, 1e-1] as the dt_bias initialisation gives (heads as long as a
+    chunk)."""
+    import mamba_selective_scan_mixer_b200 as J
+    L, di = 32768, 2048
+    s = scan_inputs(1, L, di, 16, seed=31)
+    if dt_kind == "per_channel":
+        g = _gen(32)
+        dt0 = torch.exp(torch.empty(di).uniform_(np.log(1e-3), np.log(1e-1), generator=g))
+        s["dt"] = (dt0[None, None, :] * torch.exp(0.3 * torch.randn(1, L, di, generator=g))).float()
+    args = {k: v.to(dev) for k, v in s.items()}
+    y, h = J.selective_scan(args["x"], args["z"], args["dt"], args["B"], args["C"], args["A"], args["D"],
+                            chunk=chunk)
+    cols = np.arange(5, di, 37)   # a few channels of every warp of every CTA
+    n = lambda k: to_np(s[k])
+    wy, wh = om.selective_scan_c(n("x")[:, :, cols], n("dt")[:, :, cols], n("A")[cols], n("B"), n("C"),
+                                 n("D")[cols], n("z")[:, :, cols])
+    assert _bf16_elementwise_bad(to_np(y)[:, :, cols], wy) == 0
+    assert rel_l2(to_np(h)[:, cols], wh) < 1e-5
+
+
 def test_scan_repeated_calls_reuse_workspace(dev):
     import mamba_selective_scan_mixer_b200 as J
     s = {k: v.to(dev) for k, v in scan_inputs(1, 640, 256, 16, seed=21).items()}
