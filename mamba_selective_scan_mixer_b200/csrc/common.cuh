@@ -53,6 +53,36 @@ __device__ __forceinline__ float softplus(float v) {
   return v > 20.0f ? v : log1pf(__expf(v));
 }
 
+// softplus for the bf16 path: log(1 + e^v) from one ex2 and one lg2, with the
+// series e - e^2/2 + e^3/3 - e^4/4 where e^v < 1/64 (relative error < 2e-8
+// there, < 1e-5 elsewhere; far inside the bf16 tolerance).
+__device__ __forceinline__ float softplus_fast(float v) {
+  const float e = ex2(1.4426950408889634f * v);
+  float l;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(l) : "f"(1.0f + e));
+  const float big = 0.6931471805599453f * l;
+  const float small = e * (1.0f - e * (0.5f - e * (0.33333334f - e * 0.25f)));
+  const float r = e < 0.015625f ? small : big;
+  return v > 15.0f ? v : r;
+}
+
+// sum over the 32 lanes of a warp
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Acquire / release accesses of a flag in global memory (GPU scope).
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // Programmatic dependent launch: wait for the preceding grid in the stream to
 // complete (a no-op when the launch carried no programmatic dependency), and
 // let the next grid begin launching while this one runs.
@@ -78,6 +108,23 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
   return d;
 }
+
+// r^1 .. r^16
+__device__ __forceinline__ void powers16(float r, float* pw) {
+  pw[0] = r;
+  pw[1] = r * r;
+  const float2 p34 = fmul2(make_float2(pw[1], pw[1]), make_float2(pw[0], pw[1]));
+  pw[2] = p34.x; pw[3] = p34.y;
+  const float2 p56 = fmul2(make_float2(pw[3], pw[3]), make_float2(pw[0], pw[1]));
+  const float2 p78 = fmul2(make_float2(pw[3], pw[3]), make_float2(pw[2], pw[3]));
+  pw[4] = p56.x; pw[5] = p56.y; pw[6] = p78.x; pw[7] = p78.y;
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {
+    const float2 q = fmul2(make_float2(pw[7], pw[7]), make_float2(pw[i], pw[i + 1]));
+    pw[8 + i] = q.x; pw[9 + i] = q.y;
+  }
+}
+
 
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

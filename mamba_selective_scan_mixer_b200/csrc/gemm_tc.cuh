@@ -108,19 +108,6 @@ __device__ __forceinline__ void store_bf16x8(bf16* dst, const float* v) {
   *reinterpret_cast<uint4*>(dst) = u;
 }
 
-// softplus for the bf16 path: log(1 + e^v) from one ex2 and one lg2, with the
-// series e - e^2/2 + e^3/3 - e^4/4 where e^v < 1/64 (relative error < 2e-8
-// there, < 1e-5 elsewhere; far inside the bf16 tolerance).
-__device__ __forceinline__ float softplus_fast(float v) {
-  const float e = ex2(1.4426950408889634f * v);
-  float l;
-  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(l) : "f"(1.0f + e));
-  const float big = 0.6931471805599453f * l;
-  const float small = e * (1.0f - e * (0.5f - e * (0.33333334f - e * 0.25f)));
-  const float r = e < 0.015625f ? small : big;
-  return v > 15.0f ? v : r;
-}
-
 __device__ __forceinline__ float log1p_small(float e) {
   // log(1 + e) for 0 <= e < 1/8: Taylor series through e^7 (relative error < 1e-7)
   return e * (1.0f - e * (0.5f - e * (0.33333334f - e * (0.25f - e * (0.2f - e * (0.16666667f - e * 0.14285715f))))));

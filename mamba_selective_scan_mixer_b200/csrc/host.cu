@@ -83,7 +83,7 @@ jamba_status make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType d
 jamba_status make_map_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes,
                          uint64_t inner, uint64_t rows, uint64_t outer, uint64_t row_stride,
                          uint64_t outer_stride, uint32_t box_inner, uint32_t box_rows,
-                         CUtensorMapSwizzle sw) {
+                         CUtensorMapSwizzle sw, uint32_t box_outer) {
   auto enc = encoder();
   if (!enc) return fail(JAMBA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
   if (!aligned16(base) || (row_stride & 15u) || (outer_stride & 15u))
@@ -91,7 +91,7 @@ jamba_status make_map_3d(CUtensorMap* m, const void* base, CUtensorMapDataType d
   (void)elem_bytes;
   cuuint64_t dims[3] = {inner, rows, outer};
   cuuint64_t strides[2] = {row_stride, outer_stride};
-  cuuint32_t box[3] = {box_inner, box_rows, 1};
+  cuuint32_t box[3] = {box_inner, box_rows, box_outer};
   cuuint32_t es[3] = {1, 1, 1};
   CUresult r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);

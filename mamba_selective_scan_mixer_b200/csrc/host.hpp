@@ -59,7 +59,7 @@ jamba_status make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType d
 jamba_status make_map_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes,
                          uint64_t inner, uint64_t rows, uint64_t outer, uint64_t row_stride,
                          uint64_t outer_stride, uint32_t box_inner, uint32_t box_rows,
-                         CUtensorMapSwizzle sw);
+                         CUtensorMapSwizzle sw, uint32_t box_outer = 1);
 
 // ---------------------------------------------------------------- GEMM
 struct GemmDesc {

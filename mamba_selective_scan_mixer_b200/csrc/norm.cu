@@ -11,11 +11,6 @@
 
 namespace jb {
 
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
 
 // one 256-thread block per row
 template <typename T>

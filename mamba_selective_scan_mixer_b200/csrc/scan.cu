@@ -95,14 +95,6 @@ struct ScanArgs {
   int* err;
 };
 
-__device__ __forceinline__ int ld_acquire(const int* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release(int* p, int v) {
-  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
 
 // CPT consecutive elements <-> floats
 template <typename T, int CPT> struct Vec;
@@ -156,21 +148,6 @@ template <> struct Vec<float, 4> {
   }
 };
 
-// r^1 .. r^16
-__device__ __forceinline__ void powers16(float r, float* pw) {
-  pw[0] = r;
-  pw[1] = r * r;
-  const float2 p34 = fmul2(make_float2(pw[1], pw[1]), make_float2(pw[0], pw[1]));
-  pw[2] = p34.x; pw[3] = p34.y;
-  const float2 p56 = fmul2(make_float2(pw[3], pw[3]), make_float2(pw[0], pw[1]));
-  const float2 p78 = fmul2(make_float2(pw[3], pw[3]), make_float2(pw[2], pw[3]));
-  pw[4] = p56.x; pw[5] = p56.y; pw[6] = p78.x; pw[7] = p78.y;
-#pragma unroll
-  for (int i = 0; i < 8; i += 2) {
-    const float2 q = fmul2(make_float2(pw[7], pw[7]), make_float2(pw[i], pw[i + 1]));
-    pw[8 + i] = q.x; pw[9 + i] = q.y;
-  }
-}
 
 // Per-CTA context shared by the passes.
 struct ScanCtx {

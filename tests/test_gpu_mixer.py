@@ -99,6 +99,30 @@ def test_bf16_decode_steps_match_oracle_and_prefill(dev):
     assert rel_l2(np.stack(outs, 1), to_np(out_full)[:, L0:]) < TOL_BF16
 
 
+@pytest.mark.parametrize("dt_rank,batch,inner_norm,a_init", [
+    (64, 5, True, "structured"),
+    (64, 64, False, "random"),      # no inner norm, per-state decays
+    (64, 1, True, "random"),        # one row
+    (40, 5, True, "structured"),    # dt_rank not a multiple of 32
+    (64, 65, True, "structured"),   # odd batch above 64
+])
+def test_bf16_decode_shapes(dev, dt_rank, batch, inner_norm, a_init):
+    """decode steps against the oracle across batch sizes, dt ranks, norm and
+    A variants, caches included"""
+    sh = MambaShape(d_model=256, d_inner=1024, dt_rank=dt_rank, dtype="bf16", inner_norm=inner_norm)
+    mix, p64 = _mixer(sh, 6, dev, a_init=a_init, norm_init="random")
+    L0, S = 24, 6
+    u = mamba_input(sh, batch, L0, seed=6)
+    steps = decode_inputs(sh, batch, S, seed=6)
+    _, cs, ss = mix.prefill(u.to(dev))
+    outs = [to_np(mix.step(steps[t].to(dev), cs, ss)) for t in range(S)]
+    full = torch.cat([u, steps.transpose(0, 1)], dim=1)
+    ref = om.mamba_prefill(p64, to_np(full), sh)
+    assert rel_l2(np.stack(outs, 1), ref["out"][:, L0:]) < TOL_BF16
+    assert rel_l2(to_np(ss), ref["ssm_state"]) < TOL_BF16
+    assert rel_l2(to_np(cs), ref["conv_state"]) < TOL_BF16
+
+
 @pytest.mark.slow
 def test_prefill_4k_full_width(dev):
     """Jamba-width prefill of 4096 tokens with inner RMSNorm, whole output vs the oracle"""
