@@ -250,6 +250,18 @@ __device__ __forceinline__ void scan_step(float2 (&h)[CPT][8], const float* xv, 
   }
 }
 
+// Decay product of a channel over its chunk, per state: from R (the n = 0
+// factor; power form) or the tracked products P.
+template <bool FAST>
+__device__ __forceinline__ void chunk_decay(float R, const float2 (&P)[8], float* pe) {
+  if constexpr (FAST) {
+    powers16(R, pe);
+  } else {
+#pragma unroll
+    for (int n2 = 0; n2 < 8; ++n2) { pe[2 * n2] = P[n2].x; pe[2 * n2 + 1] = P[n2].y; }
+  }
+}
+
 // One stage (up to SCAN_Q steps) of one warp, specialised on the warp-uniform
 // head mode; yrow points at this thread's first output of the stage.
 template <typename TX, bool FAST, int CPT, bool HEAD>
@@ -448,29 +460,22 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
   const bool independent = __syncthreads_and(producer || !head) != 0;  // end state free of h_in
   int t_head_max = cx.t0;
   for (int w = 0; w < NCW; ++w) t_head_max = max(t_head_max, s_head_end[w]);
-  float Pend[CPT][16];
-#pragma unroll
-  for (int j = 0; j < CPT; ++j) {
-    if constexpr (FAST) {
-      powers16(R[j], Pend[j]);
-    } else {
-#pragma unroll
-      for (int n2 = 0; n2 < 8; ++n2) { Pend[j][2 * n2] = P[j][n2].x; Pend[j][2 * n2 + 1] = P[j][n2].y; }
-    }
-  }
   if (!producer) {
 #pragma unroll
-    for (int j = 0; j < CPT; ++j)
+    for (int j = 0; j < CPT; ++j) {
+      float pe[16];   // decay product over the chunk
+      chunk_decay<FAST>(R[j], P[j], pe);
 #pragma unroll
       for (int n = 0; n < NS; n += 2) {
         float* o = myrec + (cl + j) * NS + n;
         if (independent) {
           *reinterpret_cast<float2*>(o + 2 * SCAN_CH * NS) = h[j][n / 2];
         } else {
-          *reinterpret_cast<float2*>(o) = make_float2(Pend[j][n], Pend[j][n + 1]);
+          *reinterpret_cast<float2*>(o) = make_float2(pe[n], pe[n + 1]);
           *reinterpret_cast<float2*>(o + SCAN_CH * NS) = h[j][n / 2];
         }
       }
+    }
   }
   __threadfence();
   __syncthreads();
@@ -528,34 +533,35 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
       }
       __syncthreads();
     }
-    float2 hin[CPT][8];
+    // The true end state (h + P_end * h_in, published as this chunk's
+    // inclusive record unless already final) and the final state of the batch
+    // row; then h takes h_in, pass 2's starting state.
+    const bool last = cx.t1 == a.L && a.h_out && valid;
+    if (!producer) {
 #pragma unroll
-    for (int j = 0; j < CPT; ++j)
+      for (int j = 0; j < CPT; ++j) {
+        float pe[16];
+        chunk_decay<FAST>(R[j], P[j], pe);
 #pragma unroll
-      for (int n2 = 0; n2 < 8; ++n2)
-        hin[j][n2] = producer ? make_float2(0.f, 0.f)
-                              : make_float2(sH[(cl + j) * NS + 2 * n2], sH[(cl + j) * NS + 2 * n2 + 1]);
+        for (int n2 = 0; n2 < 8; ++n2) {
+          const float2 hi = make_float2(sH[(cl + j) * NS + 2 * n2], sH[(cl + j) * NS + 2 * n2 + 1]);
+          float2 he = h[j][n2];
+          if (!independent) {
+            he = make_float2(fmaf(pe[2 * n2], hi.x, he.x), fmaf(pe[2 * n2 + 1], hi.y, he.y));
+            *reinterpret_cast<float2*>(myrec + 2 * SCAN_CH * NS + (cl + j) * NS + 2 * n2) = he;
+          }
+          if (last) *reinterpret_cast<float2*>(a.h_out + ((long long)cx.b * a.di + c + j) * NS + 2 * n2) = he;
+          h[j][n2] = hi;
+        }
+      }
+    }
     // The ring is reused by pass 2: TMA (the async proxy) will overwrite the
-    // scratch written above through ordinary stores, so those stores are
-    // ordered before it with a proxy fence ahead of the barrier.
+    // scratch read above, so the accesses are ordered before it with a proxy
+    // fence ahead of the barrier; the inclusive record is published after it.
+    __threadfence();
     fence_async_shared();
     __syncthreads();
-    if (!independent) {
-      // true end state h + P_end * h_in, published as this chunk's inclusive record
-      if (!producer) {
-#pragma unroll
-        for (int j = 0; j < CPT; ++j)
-#pragma unroll
-          for (int n2 = 0; n2 < 8; ++n2) {
-            h[j][n2].x = fmaf(Pend[j][2 * n2], hin[j][n2].x, h[j][n2].x);
-            h[j][n2].y = fmaf(Pend[j][2 * n2 + 1], hin[j][n2].y, h[j][n2].y);
-            *reinterpret_cast<float2*>(myrec + 2 * SCAN_CH * NS + (cl + j) * NS + 2 * n2) = h[j][n2];
-          }
-      }
-      __threadfence();
-      __syncthreads();
-      if (tid == 0) st_release(myflag, 2);
-    }
+    if (!independent && tid == 0) st_release(myflag, 2);
 
     // ---------------------------------------------------------- pass 2: replay the head from h_in
     const int nsub2 = (t_head_max - cx.t0 + SCAN_Q - 1) / SCAN_Q;
@@ -565,13 +571,11 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
       bool head2 = false;
       int unused = 0;
       // each warp replays only its own head; the stages after it are passed through
-      consumer_pass<TX, TBC, FAST, CPT, false>(smem, cx, a, cx.t0, t_head_max, s_head_end[warp], nsub2, nsub1, hin, head2,
+      consumer_pass<TX, TBC, FAST, CPT, false>(smem, cx, a, cx.t0, t_head_max, s_head_end[warp], nsub2, nsub1, h, head2,
                                         unused, R, P, A2_0, sA2c, Dv, valid, c);
     }
-  }
-
-  // final state of the batch row
-  if (cx.t1 == a.L && a.h_out && valid) {
+  } else if (cx.t1 == a.L && a.h_out && valid) {
+    // the first chunk started from the known state: h is the final state of the batch row
 #pragma unroll
     for (int j = 0; j < CPT; ++j)
 #pragma unroll
