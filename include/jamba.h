@@ -123,6 +123,29 @@ jamba_status jamba_mamba_prefill(jamba_mamba_t h, const void* u, const void* res
                                  float* ssm_state_out, void* ws, size_t ws_bytes,
                                  jamba_stream_t stream);
 
+/* Prefill from and to HOST memory, pipelined: the sequence is cut into time
+ * chunks of `chunk` tokens (0 = 16384); the copy of chunk i+1 to the device,
+ * the prefill of chunk i (continuing the caches) and the copy of chunk i-1
+ * back overlap on two internal copy streams, so the transfers hide behind the
+ * compute.  The result equals jamba_mamba_prefill of the whole sequence up to
+ * rounding order at the chunk boundaries.
+ *   u_host / residual_host (or NULL) / out_host: [batch, seqlen, d_model] dtype in
+ *            page-locked host memory (cudaHostAlloc / cudaHostRegister);
+ *            out_host may alias residual_host, not u_host
+ *   conv_state_in / ssm_state_in: device, as in jamba_mamba_prefill (NULL = zeros)
+ *   conv_state_out / ssm_state_out: device, required (they carry the chunks);
+ *            may alias the inputs
+ *   ws / ws_bytes: device workspace of at least jamba_mamba_host_workspace_size
+ * The call is stream-ordered on `stream`: work queued on it afterwards sees the
+ * finished output in out_host.  Errors: INVALID_ARG (host buffers not
+ * page-locked, null states), WORKSPACE, CUDA. */
+jamba_status jamba_mamba_host_workspace_size(jamba_mamba_t h, int batch, int chunk, size_t* bytes);
+jamba_status jamba_mamba_prefill_host(jamba_mamba_t h, const void* u_host, const void* residual_host,
+                                      void* out_host, int batch, int seqlen, int chunk,
+                                      const float* conv_state_in, const float* ssm_state_in,
+                                      float* conv_state_out, float* ssm_state_out, void* ws,
+                                      size_t ws_bytes, jamba_stream_t stream);
+
 /* One-token decode step for every batch row, updating both caches in place.
  *   u [batch, d_model], residual [batch, d_model] or NULL, out [batch, d_model]
  *   conv_state [batch, d_inner, d_conv-1] fp32, ssm_state [batch, d_inner, d_state] fp32

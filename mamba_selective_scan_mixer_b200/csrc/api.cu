@@ -13,6 +13,10 @@ struct jamba_mamba {
   jamba_mamba_config cfg;
   jamba_mamba_weights w;
   int device;
+  // host-buffer prefill pipeline: two copy streams and the events that order
+  // the double-buffered chunks (created on first use)
+  cudaStream_t io_in = nullptr, io_out = nullptr;
+  cudaEvent_t ev_in[2] = {nullptr, nullptr}, ev_comp[2] = {nullptr, nullptr}, ev_out[2] = {nullptr, nullptr};
 };
 
 namespace {
@@ -180,6 +184,15 @@ jamba_status jamba_mamba_create(const jamba_mamba_config* cfg, const jamba_mamba
 }
 
 jamba_status jamba_mamba_destroy(jamba_mamba_t h) {
+  if (h) {
+    if (h->io_in) cudaStreamDestroy(h->io_in);
+    if (h->io_out) cudaStreamDestroy(h->io_out);
+    for (int i = 0; i < 2; ++i) {
+      if (h->ev_in[i]) cudaEventDestroy(h->ev_in[i]);
+      if (h->ev_comp[i]) cudaEventDestroy(h->ev_comp[i]);
+      if (h->ev_out[i]) cudaEventDestroy(h->ev_out[i]);
+    }
+  }
   delete h;
   return JAMBA_OK;
 }
@@ -327,6 +340,124 @@ jamba_status jamba_mamba_step(jamba_mamba_t h, const void* u, const void* residu
     g4.ldr = dm;
     JB_TRY(gemm_f32(g4, s));
   }
+  return JAMBA_OK;
+}
+
+// --------------------------------------------------------- prefill from host memory
+
+namespace {
+
+constexpr int kHostChunk = 16384;
+
+size_t host_chunk_bytes(const jamba_mamba_config& c, int batch, int chunk) {
+  return al((size_t)batch * chunk * c.d_model * esize(c.dtype));
+}
+
+jamba_status check_pinned(const void* p, const char* name, bool required) {
+  if (!p) return required ? fail(JAMBA_ERR_INVALID_ARG, std::string(name) + " is null") : JAMBA_OK;
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return fail(JAMBA_ERR_INVALID_ARG, std::string(name) + ": not page-locked host memory");
+  }
+  if (at.type != cudaMemoryTypeHost)
+    return fail(JAMBA_ERR_INVALID_ARG, std::string(name) + ": not page-locked host memory");
+  return JAMBA_OK;
+}
+
+jamba_status ensure_io(jamba_mamba* h) {
+  if (h->io_in) return JAMBA_OK;
+  JB_CUDA(cudaStreamCreateWithFlags(&h->io_in, cudaStreamNonBlocking));
+  JB_CUDA(cudaStreamCreateWithFlags(&h->io_out, cudaStreamNonBlocking));
+  for (int i = 0; i < 2; ++i) {
+    JB_CUDA(cudaEventCreateWithFlags(&h->ev_in[i], cudaEventDisableTiming));
+    JB_CUDA(cudaEventCreateWithFlags(&h->ev_comp[i], cudaEventDisableTiming));
+    JB_CUDA(cudaEventCreateWithFlags(&h->ev_out[i], cudaEventDisableTiming));
+  }
+  return JAMBA_OK;
+}
+
+// columns [t0, t0 + n) of every batch row of a [batch, L, d_model] host tensor
+cudaError_t copy_rows(void* dst, const void* src, size_t row_bytes, size_t src_pitch, size_t dst_pitch, int batch,
+                      cudaMemcpyKind kind, cudaStream_t s) {
+  return cudaMemcpy2DAsync(dst, dst_pitch, src, src_pitch, row_bytes, (size_t)batch, kind, s);
+}
+
+}  // namespace
+
+jamba_status jamba_mamba_host_workspace_size(jamba_mamba_t h, int batch, int chunk, size_t* bytes) {
+  if (!h || !bytes || batch <= 0 || chunk < 0) return fail(JAMBA_ERR_INVALID_ARG, "host workspace_size: bad argument");
+  if (chunk == 0) chunk = kHostChunk;
+  size_t pre = 0;
+  JB_TRY(jamba_mamba_workspace_size(h, batch, chunk, &pre));
+  // prefill workspace, then u, residual and out chunk buffers, two of each
+  *bytes = al(pre) + 6 * host_chunk_bytes(h->cfg, batch, chunk);
+  return JAMBA_OK;
+}
+
+jamba_status jamba_mamba_prefill_host(jamba_mamba_t h, const void* u_host, const void* residual_host, void* out_host,
+                                      int batch, int seqlen, int chunk, const float* conv_state_in,
+                                      const float* ssm_state_in, float* conv_state_out, float* ssm_state_out,
+                                      void* ws, size_t ws_bytes, jamba_stream_t stream) {
+  if (!h) return fail(JAMBA_ERR_INVALID_ARG, "prefill_host: null handle");
+  if (batch <= 0 || seqlen <= 0 || chunk < 0)
+    return fail(JAMBA_ERR_INVALID_ARG, "prefill_host: batch and seqlen must be positive, chunk >= 0");
+  JB_TRY(check_device(h));
+  JB_TRY(check_pinned(u_host, "u_host", true));
+  JB_TRY(check_pinned(out_host, "out_host", true));
+  JB_TRY(check_pinned(residual_host, "residual_host", false));
+  if (u_host == out_host) return fail(JAMBA_ERR_INVALID_ARG, "prefill_host: out_host may not alias u_host");
+  JB_TRY(check_ptr(conv_state_out, "conv_state_out"));
+  JB_TRY(check_ptr(ssm_state_out, "ssm_state_out"));
+  JB_TRY(check_ptr(ws, "workspace"));
+  if (chunk == 0) chunk = kHostChunk;
+  if (chunk > seqlen) chunk = seqlen;
+  size_t need = 0;
+  JB_TRY(jamba_mamba_host_workspace_size(h, batch, chunk, &need));
+  if (ws_bytes < need) return fail(JAMBA_ERR_WORKSPACE, "prefill_host: workspace too small");
+  JB_TRY(ensure_io(h));
+  const jamba_mamba_config& c = h->cfg;
+  const size_t es = (size_t)esize(c.dtype), tok = (size_t)c.d_model * es;   // bytes per token row
+  size_t pre = 0;
+  JB_TRY(jamba_mamba_workspace_size(h, batch, chunk, &pre));
+  uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+  const size_t cb = host_chunk_bytes(c, batch, chunk);
+  uint8_t* in_buf[2] = {base + al(pre), base + al(pre) + cb};
+  uint8_t* res_buf[2] = {base + al(pre) + 2 * cb, base + al(pre) + 3 * cb};
+  uint8_t* out_buf[2] = {base + al(pre) + 4 * cb, base + al(pre) + 5 * cb};
+  cudaStream_t s = cs(stream);
+  const size_t pitch = (size_t)seqlen * tok;   // host row pitch: one batch row of the whole sequence
+  const int n_chunks = (seqlen + chunk - 1) / chunk;
+  // the copy streams start after the work already queued on `stream`
+  JB_CUDA(cudaEventRecord(h->ev_comp[1], s));
+  JB_CUDA(cudaStreamWaitEvent(h->io_in, h->ev_comp[1], 0));
+  JB_CUDA(cudaStreamWaitEvent(h->io_out, h->ev_comp[1], 0));
+  for (int i = 0; i < n_chunks; ++i) {
+    const int k = i & 1, t0 = i * chunk, n = seqlen - t0 < chunk ? seqlen - t0 : chunk;
+    const size_t row = (size_t)n * tok;
+    // in: the buffer's previous chunk (i - 2) has been consumed by its prefill
+    if (i >= 2) JB_CUDA(cudaStreamWaitEvent(h->io_in, h->ev_comp[k], 0));
+    JB_CUDA(copy_rows(in_buf[k], reinterpret_cast<const uint8_t*>(u_host) + (size_t)t0 * tok, row, pitch, row, batch,
+                      cudaMemcpyHostToDevice, h->io_in));
+    if (residual_host)
+      JB_CUDA(copy_rows(res_buf[k], reinterpret_cast<const uint8_t*>(residual_host) + (size_t)t0 * tok, row, pitch,
+                        row, batch, cudaMemcpyHostToDevice, h->io_in));
+    JB_CUDA(cudaEventRecord(h->ev_in[k], h->io_in));
+    // compute: chunk i is in, and the out buffer's previous chunk is back on the host
+    JB_CUDA(cudaStreamWaitEvent(s, h->ev_in[k], 0));
+    if (i >= 2) JB_CUDA(cudaStreamWaitEvent(s, h->ev_out[k], 0));
+    JB_TRY(jamba_mamba_prefill(h, in_buf[k], residual_host ? res_buf[k] : nullptr, out_buf[k], batch, n,
+                               i == 0 ? conv_state_in : conv_state_out, i == 0 ? ssm_state_in : ssm_state_out,
+                               conv_state_out, ssm_state_out, ws, pre, stream));
+    JB_CUDA(cudaEventRecord(h->ev_comp[k], s));
+    // out
+    JB_CUDA(cudaStreamWaitEvent(h->io_out, h->ev_comp[k], 0));
+    JB_CUDA(copy_rows(reinterpret_cast<uint8_t*>(out_host) + (size_t)t0 * tok, out_buf[k], row, row, pitch, batch,
+                      cudaMemcpyDeviceToHost, h->io_out));
+    JB_CUDA(cudaEventRecord(h->ev_out[k], h->io_out));
+  }
+  // work queued on `stream` afterwards sees every chunk back on the host
+  for (int k = 0; k < 2 && k < n_chunks; ++k) JB_CUDA(cudaStreamWaitEvent(s, h->ev_out[k], 0));
   return JAMBA_OK;
 }
 

@@ -110,6 +110,32 @@ class MambaMixer:
                                         ws.numel(), _stream(stream)))
         return out, conv_state_out, ssm_state_out
 
+    def prefill_host(self, u_host, residual_host=None, out_host=None, chunk=0, conv_state_in=None,
+                     ssm_state_in=None, conv_state_out=None, ssm_state_out=None, stream=None):
+        """Prefill from and to pinned host tensors [B, L, d_model]; the library
+        pipelines the transfers with the compute in time chunks of `chunk`
+        tokens (0: its default).  Returns (out_host, conv_state_out, ssm_state_out);
+        the caches live on the device."""
+        for t, name in ((u_host, "u_host"), (residual_host, "residual_host"), (out_host, "out_host")):
+            if t is not None and (t.is_cuda or not t.is_pinned()):
+                raise ValueError(name + " must be a pinned host tensor")
+            _contig(t, name)
+        B, L, _ = u_host.shape
+        if out_host is None:
+            out_host = torch.empty(u_host.shape, dtype=u_host.dtype, pin_memory=True)
+        if conv_state_out is None or ssm_state_out is None:
+            cs, ss = self.new_states(B)
+            conv_state_out = cs if conv_state_out is None else conv_state_out
+            ssm_state_out = ss if ssm_state_out is None else ssm_state_out
+        _cuda(conv_state_in, ssm_state_in, conv_state_out, ssm_state_out)
+        n = ctypes.c_size_t()
+        check(lib().jamba_mamba_host_workspace_size(self.handle, B, int(chunk), ctypes.byref(n)))
+        ws = self.ws.get(n.value, self.device)
+        check(lib().jamba_mamba_prefill_host(self.handle, _p(u_host), _p(residual_host), _p(out_host), B, L,
+                                             int(chunk), _p(conv_state_in), _p(ssm_state_in), _p(conv_state_out),
+                                             _p(ssm_state_out), _p(ws), ws.numel(), _stream(stream)))
+        return out_host, conv_state_out, ssm_state_out
+
     def step(self, u, conv_state, ssm_state, residual=None, out=None, stream=None):
         """u [B, d_model]; updates both caches in place; returns out [B, d_model]."""
         _cuda(u, conv_state, ssm_state, residual)

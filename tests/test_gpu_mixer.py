@@ -123,6 +123,36 @@ def test_bf16_decode_shapes(dev, dt_rank, batch, inner_norm, a_init):
     assert rel_l2(to_np(cs), ref["conv_state"]) < TOL_BF16
 
 
+def test_prefill_from_host_memory_pipelined(dev):
+    """the host-buffer prefill (transfers overlapped with compute in time
+    chunks, ragged last chunk, residual aliasing the output) equals the device
+    prefill and the oracle"""
+    sh = MambaShape(d_model=256, d_inner=512, dt_rank=32, dtype="bf16")
+    mix, p64 = _mixer(sh, 7, dev, a_init="random")
+    B, L = 2, 200
+    u = mamba_input(sh, B, L, seed=8)
+    res = mamba_input(sh, B, L, seed=9)
+    cs0, ss0 = mix.new_states(B)
+    cs0.normal_()
+    ss0.normal_()
+    cs0 = cs0.to(torch.bfloat16).float()   # the cache holds bf16 values
+    want, wcs, wss = mix.prefill(u.to(dev), residual=res.to(dev), conv_state_in=cs0, ssm_state_in=ss0)
+    hu = u.clone().pin_memory()
+    hres = res.clone().pin_memory()
+    out, cs, ss = mix.prefill_host(hu, residual_host=hres, out_host=hres, chunk=48, conv_state_in=cs0,
+                                   ssm_state_in=ss0)
+    torch.cuda.synchronize()
+    assert out.data_ptr() == hres.data_ptr()
+    assert rel_l2(to_np(out), to_np(want)) < TOL_BF16
+    assert rel_l2(to_np(cs), to_np(wcs)) < 1e-6
+    assert rel_l2(to_np(ss), to_np(wss)) < 1e-4
+    ref = om.mamba_prefill(p64, to_np(u), sh, conv_state0=to_np(cs0), ssm_state0=to_np(ss0))
+    assert rel_l2(to_np(out), ref["out"] + to_np(res)) < TOL_BF16
+    # pageable host memory is refused
+    with pytest.raises(ValueError):
+        mix.prefill_host(u.clone())
+
+
 @pytest.mark.slow
 def test_prefill_4k_full_width(dev):
     """Jamba-width prefill of 4096 tokens with inner RMSNorm, whole output vs the oracle"""
