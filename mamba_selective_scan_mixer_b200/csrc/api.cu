@@ -3,6 +3,7 @@
 // blocks and the MoE.  See include/jamba.h for the contract of each call.
 #include <new>
 #include <string>
+#include <vector>
 
 #include "gemm_tc.cuh"
 #include "host.hpp"
@@ -427,13 +428,31 @@ jamba_status jamba_mamba_prefill_host(jamba_mamba_t h, const void* u_host, const
   uint8_t* out_buf[2] = {base + al(pre) + 4 * cb, base + al(pre) + 5 * cb};
   cudaStream_t s = cs(stream);
   const size_t pitch = (size_t)seqlen * tok;   // host row pitch: one batch row of the whole sequence
-  const int n_chunks = (seqlen + chunk - 1) / chunk;
+  // chunk lengths: the first and last chunks ramp (chunk/4, chunk/2) so that
+  // the copy-in before the first prefill and the copy-out after the last one,
+  // which nothing overlaps, stay short
+  std::vector<int> lens;
+  if (seqlen >= 4 * chunk && chunk >= 64) {
+    const int q = chunk / 4, hlf = chunk / 2;
+    lens.push_back(q);
+    lens.push_back(hlf);
+    int rem = seqlen - 2 * (q + hlf);
+    while (rem > 0) {
+      lens.push_back(rem < chunk ? rem : chunk);
+      rem -= lens.back();
+    }
+    lens.push_back(hlf);
+    lens.push_back(q);
+  } else {
+    for (int t = 0; t < seqlen; t += chunk) lens.push_back(seqlen - t < chunk ? seqlen - t : chunk);
+  }
+  const int n_chunks = (int)lens.size();
   // the copy streams start after the work already queued on `stream`
   JB_CUDA(cudaEventRecord(h->ev_comp[1], s));
   JB_CUDA(cudaStreamWaitEvent(h->io_in, h->ev_comp[1], 0));
   JB_CUDA(cudaStreamWaitEvent(h->io_out, h->ev_comp[1], 0));
-  for (int i = 0; i < n_chunks; ++i) {
-    const int k = i & 1, t0 = i * chunk, n = seqlen - t0 < chunk ? seqlen - t0 : chunk;
+  for (int i = 0, t0 = 0; i < n_chunks; t0 += lens[i], ++i) {
+    const int k = i & 1, n = lens[i];
     const size_t row = (size_t)n * tok;
     // in: the buffer's previous chunk (i - 2) has been consumed by its prefill
     if (i >= 2) JB_CUDA(cudaStreamWaitEvent(h->io_in, h->ev_comp[k], 0));

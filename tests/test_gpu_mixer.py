@@ -123,13 +123,14 @@ def test_bf16_decode_shapes(dev, dt_rank, batch, inner_norm, a_init):
     assert rel_l2(to_np(cs), ref["conv_state"]) < TOL_BF16
 
 
-def test_prefill_from_host_memory_pipelined(dev):
+@pytest.mark.parametrize("L,chunk", [(200, 48), (300, 64)])
+def test_prefill_from_host_memory_pipelined(dev, L, chunk):
     """the host-buffer prefill (transfers overlapped with compute in time
-    chunks, ragged last chunk, residual aliasing the output) equals the device
-    prefill and the oracle"""
+    chunks: uniform with a ragged tail, or ramped at both ends; residual
+    aliasing the output) equals the device prefill and the oracle"""
     sh = MambaShape(d_model=256, d_inner=512, dt_rank=32, dtype="bf16")
     mix, p64 = _mixer(sh, 7, dev, a_init="random")
-    B, L = 2, 200
+    B = 2
     u = mamba_input(sh, B, L, seed=8)
     res = mamba_input(sh, B, L, seed=9)
     cs0, ss0 = mix.new_states(B)
@@ -139,7 +140,7 @@ def test_prefill_from_host_memory_pipelined(dev):
     want, wcs, wss = mix.prefill(u.to(dev), residual=res.to(dev), conv_state_in=cs0, ssm_state_in=ss0)
     hu = u.clone().pin_memory()
     hres = res.clone().pin_memory()
-    out, cs, ss = mix.prefill_host(hu, residual_host=hres, out_host=hres, chunk=48, conv_state_in=cs0,
+    out, cs, ss = mix.prefill_host(hu, residual_host=hres, out_host=hres, chunk=chunk, conv_state_in=cs0,
                                    ssm_state_in=ss0)
     torch.cuda.synchronize()
     assert out.data_ptr() == hres.data_ptr()
