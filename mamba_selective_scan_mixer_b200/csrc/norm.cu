@@ -57,17 +57,19 @@ xproj_norm_kernel(const float* __restrict__ part, int splits, long long split_st
   __shared__ float inv[3];
   float v = 0.f;
   if (col < W) {
+    // up to 32 partials in flight per round: the sum is one memory round trip
+    // for the split counts used (at most 32 at decode sizes)
     const float* p = part + t * W + col;
-    int s = 0;
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-    for (; s + 4 <= splits; s += 4) {
-      a0 += p[(s + 0) * split_stride];
-      a1 += p[(s + 1) * split_stride];
-      a2 += p[(s + 2) * split_stride];
-      a3 += p[(s + 3) * split_stride];
+    for (int s0 = 0; s0 < splits; s0 += 32) {
+      float a[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) a[i] = s0 + i < splits ? p[(long long)(s0 + i) * split_stride] : 0.f;
+#pragma unroll
+      for (int w = 16; w; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) a[i] += a[i + w];
+      v += a[0];
     }
-    for (; s < splits; ++s) a0 += p[s * split_stride];
-    v = (a0 + a1) + (a2 + a3);
   }
   const int seg = col < R ? 0 : (col < R + N ? 1 : 2);
   float sq[3] = {0.f, 0.f, 0.f};
