@@ -60,15 +60,19 @@ xproj_norm_kernel(const float* __restrict__ part, int splits, long long split_st
     // up to 32 partials in flight per round: the sum is one memory round trip
     // for the split counts used (at most 32 at decode sizes)
     const float* p = part + t * W + col;
-    for (int s0 = 0; s0 < splits; s0 += 32) {
-      float a[32];
+    if (splits == 1) {
+      v = *p;
+    } else {
+      for (int s0 = 0; s0 < splits; s0 += 32) {
+        float a[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) a[i] = s0 + i < splits ? p[(long long)(s0 + i) * split_stride] : 0.f;
+        for (int i = 0; i < 32; ++i) a[i] = s0 + i < splits ? p[(long long)(s0 + i) * split_stride] : 0.f;
 #pragma unroll
-      for (int w = 16; w; w >>= 1)
+        for (int w = 16; w; w >>= 1)
 #pragma unroll
-        for (int i = 0; i < w; ++i) a[i] += a[i + w];
-      v += a[0];
+          for (int i = 0; i < w; ++i) a[i] += a[i + w];
+        v += a[0];
+      }
     }
   }
   const int seg = col < R ? 0 : (col < R + N ? 1 : 2);
