@@ -13,15 +13,30 @@ computes down(SiLU(gate v) * (up v)); routed rows are ordered by (expert,
 token, slot).  The layer pair is pre-norm residual: h = x + Mamba(RMSNorm(x)),
 out = h + MoE(RMSNorm(h)).
 
+ExpertsInt8 ("Jamba-1.5" article, section on ExpertsInt8; "Jamba-1.5"
+abstract): only the expert (MoE/MLP) weights are stored as INT8 and are
+dequantised inside the MoE kernel at run time; activations stay BF16; no
+calibration data is used.  The pages do not give the scheme.  Reading: each
+output row of each expert matrix (a row of w_gate / w_up over d_model, a row
+of w_down over d_ff) gets one symmetric scale s = max|w| / 127, taken in
+fp32; q = round-half-even(w / s) in fp32, an integer in [-127, 127]; an
+all-zero row has s = 0 and q = 0.  The dequantised weight is q * s, formed
+here in fp64, so the int8 MoE is the MoE above on the weights q * s.
+
 Parity pins (tests/test_oracle_pins.py): top-K vs a brute-force sort with
 Python's sorted(); forced ties; constructed winning rows; the permutation
 invariants (a permutation, sorted by (expert, token, slot), counts sum to
 T*K, inverse composes to identity); identical experts give
 (w_0 + w_1) * expert(v); SwiGLU vs a pure-Python loop on a tiny case.
+Int8: hand-worked rows with exact halves (ties to even); the error bound
+|q s - w| <= s / 2; the row maximum maps to +-127; per-row independence;
+power-of-two scaling of a row scales s alone; weights that are already
+q * s with s a power of two quantise losslessly, so the int8 MoE equals the
+plain MoE exactly.
 """
 import numpy as np
 
-from .mamba import linear, rmsnorm, silu, mamba_prefill
+from .mamba import linear, rmsnorm, silu, mamba_prefill, to64
 
 
 def router(v, W_r, top_k):
@@ -57,6 +72,44 @@ def permute(idx, n_experts):
 
 def swiglu_expert(v, w_gate, w_up, w_down):
     return linear(silu(linear(v, w_gate)) * linear(v, w_up), w_down)
+
+
+def quantize_int8_rows(w):
+    """Per-row symmetric INT8 codes of w [..., k] (any float array).
+
+    Returns (q int8 [..., k], s float32 [...]).  Every decision is taken in
+    fp32: s = fp32(max|w|) / 127, q = rint(fp32(w) / s) (numpy rounds halves
+    to even); rows of zeros give s = 0, q = 0.
+    """
+    w32 = to64(w).astype(np.float32)   # bf16 and fp32 inputs are exact in both
+    amax = np.max(np.abs(w32), axis=-1)
+    s = (amax / np.float32(127.0)).astype(np.float32)
+    safe = np.where(s > 0, s, np.float32(1.0)).astype(np.float32)
+    q = np.rint(w32 / safe[..., None])
+    q = np.where(s[..., None] > 0, q, 0.0)
+    assert np.abs(q).max(initial=0) <= 127
+    return q.astype(np.int8), s
+
+
+def dequantize_int8_rows(q, s):
+    """fp64 weights q * s (s broadcast over the last axis)."""
+    return np.asarray(q, dtype=np.float64) * np.asarray(s, dtype=np.float64)[..., None]
+
+
+def experts_int8(p):
+    """INT8 codes and scales of the expert matrices of a MoE parameter dict."""
+    out = dict(router=to64(p["router"]))
+    for k in ("w_gate", "w_up", "w_down"):
+        out["q_" + k[2:]], out["s_" + k[2:]] = quantize_int8_rows(p[k])
+    return out
+
+
+def dequantized(pq):
+    """fp64 MoE parameter dict from the output of experts_int8."""
+    out = dict(router=np.asarray(pq["router"], dtype=np.float64))
+    for k in ("gate", "up", "down"):
+        out["w_" + k] = dequantize_int8_rows(pq["q_" + k], pq["s_" + k])
+    return out
 
 
 def moe_forward(p, v, top_k, tokens=None):

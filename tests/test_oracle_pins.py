@@ -411,3 +411,77 @@ def test_moe_single_expert_routing_by_hand():
     f = lambda e: omoe.swiglu_expert(v, p["w_gate"][e], p["w_up"][e], p["w_down"][e])
     want = r["w"][:, :1] * f(0) + r["w"][:, 1:] * f(1)
     np.testing.assert_allclose(r["out"], want, rtol=1e-13)
+
+
+# ------------------------------------------------------------------ ExpertsInt8 pins
+
+def test_int8_rows_by_hand():
+    """Rows whose maxima make s a power of two, so every w / s is exact.
+
+    Row 0: max 127 -> s = 1; -63.5 and 2.5, 0.5, -1.5 are halves that round
+    to the even neighbour.  Row 1: max 254 -> s = 2.  Row 2: all zero.
+    """
+    w = np.array([[127.0, -63.5, 2.5, 0.5, -1.5, 0.0, 1e-3],
+                  [-254.0, -3.0, 5.0, 1.0, 7.0, 253.0, 3.0],
+                  [0.0] * 7])
+    q, s = omoe.quantize_int8_rows(w)
+    assert q.dtype == np.int8 and s.dtype == np.float32
+    assert s.tolist() == [1.0, 2.0, 0.0]
+    assert q.tolist() == [[127, -64, 2, 0, -2, 0, 0],
+                          [-127, -2, 2, 0, 4, 126, 2],
+                          [0] * 7]
+
+
+def test_int8_error_bound_and_extremes():
+    rng = np.random.default_rng(19)
+    w = (rng.standard_normal((3, 40, 33)) * 0.02).astype(np.float32)
+    w[1, 5] *= 1000.0                              # one row far larger than the rest
+    q, s = omoe.quantize_int8_rows(w)
+    assert q.shape == w.shape and s.shape == w.shape[:2]
+    deq = omoe.dequantize_int8_rows(q, s)
+    err = np.abs(deq - w.astype(np.float64))
+    # rint leaves at most half a step; the fp32 division adds one rounding of w / s
+    assert (err <= s[..., None].astype(np.float64) * (0.5 + 2.0 ** -17)).all()
+    # the row maximum is +-127, no code exceeds it, signs agree where q != 0
+    amax_pos = np.abs(w).argmax(-1)
+    np.testing.assert_array_equal(np.abs(np.take_along_axis(q, amax_pos[..., None], -1))[..., 0], 127)
+    assert np.abs(q.astype(np.int32)).max() <= 127
+    nz = q != 0
+    assert (np.sign(q[nz]) == np.sign(w[nz])).all()
+    # per-row: the large row does not change its neighbours' codes
+    w2 = w.copy()
+    w2[1, 5] = w[1, 5] / 1000.0
+    q2, _ = omoe.quantize_int8_rows(w2)
+    np.testing.assert_array_equal(np.delete(q2[1], 5, 0), np.delete(q[1], 5, 0))
+
+
+def test_int8_power_of_two_scaling():
+    rng = np.random.default_rng(20)
+    w = (rng.standard_normal((8, 64)) * 0.02).astype(np.float32)
+    q, s = omoe.quantize_int8_rows(w)
+    for k in (-3, 1, 5):
+        qk, sk = omoe.quantize_int8_rows(w * np.float32(2.0 ** k))
+        np.testing.assert_array_equal(qk, q)
+        np.testing.assert_array_equal(sk, s * np.float32(2.0 ** k))
+
+
+def test_int8_moe_lossless_on_representable_weights():
+    """Weights q * 2^-e with the row maximum at |q| = 127 come back exactly,
+    so the MoE on the int8 codes equals the MoE on the original weights."""
+    rng = np.random.default_rng(21)
+    E, dm, dff = 16, 8, 6
+
+    def grid(shape):
+        q = rng.integers(-127, 128, size=shape)
+        q[..., 0] = 127 * np.where(rng.random(shape[:-1]) < 0.5, -1, 1)
+        e = rng.integers(5, 9, size=shape[:-1])[..., None]
+        return q * 2.0 ** (-e)
+
+    p = dict(router=rng.standard_normal((E, dm)), w_gate=grid((E, dff, dm)),
+             w_up=grid((E, dff, dm)), w_down=grid((E, dm, dff)))
+    pq = omoe.experts_int8(p)
+    back = omoe.dequantized(pq)
+    for k in ("w_gate", "w_up", "w_down"):
+        np.testing.assert_array_equal(back[k], p[k])
+    v = rng.standard_normal((13, dm))
+    np.testing.assert_array_equal(omoe.moe_forward(back, v, 2)["out"], omoe.moe_forward(p, v, 2)["out"])
