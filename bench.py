@@ -46,7 +46,7 @@ def parse():
     ap.add_argument("--impl", default="product", choices=["product", "reference"])
     ap.add_argument("--quick", action="store_true", help="skip the side measurements")
     ap.add_argument("--only", default="all",
-                    help="comma list of parts to run (prefill,gemm,scan,decode,pair,e2e,cpu); for profiling")
+                    help="comma list of parts to run (prefill,gemm,scan,decode,pair,moe8,e2e,cpu); for profiling")
     ap.add_argument("--seqlen", type=int, default=PREFILL_L, help="prefill tokens")
     ap.add_argument("--scan-seqlen", type=int, default=SCAN_L)
     ap.add_argument("--decode-steps", type=int, default=DECODE_STEPS)
@@ -208,8 +208,8 @@ def cpu_baseline(sample_tokens=1024):
 # ------------------------------------------------------------------ product arm
 def run_product(args):
     import mamba_selective_scan_mixer_b200 as J
-    from synthetic import MoEShape, block_norm_params, decode_inputs, mamba_input, mamba_params, moe_params, \
-        scan_inputs, workload
+    from synthetic import MoEShape, block_norm_params, decode_inputs, mamba_input, mamba_params, moe_input, \
+        moe_params, scan_inputs, workload
 
     world, rank, local = dist_setup(args)
     dev = torch.device("cuda", local)
@@ -218,7 +218,7 @@ def run_product(args):
     L = args.seqlen
     stream = torch.cuda.current_stream(dev)
 
-    parts = {"prefill", "gemm", "scan", "decode", "pair", "e2e", "cpu"} if args.only == "all" else \
+    parts = {"prefill", "gemm", "scan", "decode", "pair", "moe8", "e2e", "cpu"} if args.only == "all" else \
         set(args.only.split(","))
     if args.quick:
         parts &= {"prefill"}
@@ -356,6 +356,39 @@ def run_product(args):
                              "tokens/s": round(T / (pms / 1e3), 1), "ms": round(pms, 3),
                              "TFLOP/s": round(pflops / (pms / 1e3) / 1e12, 1),
                              "frac_of_bf16_sustained": round(pflops / (pms / 1e3) / 1e12 / pk["bf16_sus"], 4)}
+        if "moe8" in parts:
+            # ExpertsInt8: the same MoE with int8 expert codes, at the layer pair's token count
+            # (tensor-bound) and at a decode batch of 64 tokens (bound by the expert weight bytes)
+            pq = J.quantize_experts_int8(mp)
+            moe8 = J.MoE(pq, es)
+            pair8 = lambda: J.layer_pair(mixer, moe8, xp, g1, g2)
+            pair8()
+            torch.cuda.synchronize()
+            p8ms, _ = event_time_ms(pair8, 3, stream, flush)
+            wb16 = sum(mp[k].numel() * mp[k].element_size() for k in ("w_gate", "w_up", "w_down"))
+            wb8 = sum(pq[k].numel() * pq[k].element_size() for k in ("w_gate", "w_up", "w_down",
+                                                                      "s_gate", "s_up", "s_down"))
+            moe_t = {}
+            for name, m in (("bf16", moe), ("int8", moe8)):
+                for tok in (T, 64):
+                    v = moe_input(es, tok, seed=3, device=dev)
+                    f = (lambda m=m, v=v: m.forward(v))
+                    f()
+                    torch.cuda.synchronize()
+                    moe_t[(name, tok)] = event_time_ms(f, 5, stream, flush)[0]
+            eflops = T * 2 * 2.0 * (3 * es.d_model * es.d_ff)
+            res["moe_int8"] = {
+                "workload": "ExpertsInt8: 16-expert top-2 SwiGLU MoE (d_model 4096, d_ff 14336) with int8 "
+                            "expert codes and per-row fp32 scales, bf16 activations",
+                "expert_weight_bytes": {"bf16": wb16, "int8": wb8},
+                "layer_pair_ms": round(p8ms, 3), "layer_pair_tokens/s": round(T / (p8ms / 1e3), 1),
+                "moe_%d_tokens_ms" % T: {"bf16": round(moe_t[("bf16", T)], 3), "int8": round(moe_t[("int8", T)], 3)},
+                "moe_%d_tokens_TFLOP/s_int8" % T: round(eflops / (moe_t[("int8", T)] / 1e3) / 1e12, 1),
+                "moe_64_tokens_us": {"bf16": round(1e3 * moe_t[("bf16", 64)], 1),
+                                     "int8": round(1e3 * moe_t[("int8", 64)], 1)},
+                "moe_64_tokens_weight_GB/s": {"bf16": round(wb16 / (moe_t[("bf16", 64)] / 1e3) / 1e9, 1),
+                                              "int8": round(wb8 / (moe_t[("int8", 64)] / 1e3) / 1e9, 1)}}
+            del pq, moe8
         del mp, moe, xp
         J.device_status()
 

@@ -52,7 +52,7 @@ typedef enum jamba_status {
   JAMBA_ERR_OOM = 6          /* host allocation failed                            */
 } jamba_status;
 
-typedef enum jamba_dtype { JAMBA_F32 = 0, JAMBA_BF16 = 1 } jamba_dtype;
+typedef enum jamba_dtype { JAMBA_F32 = 0, JAMBA_BF16 = 1, JAMBA_INT8 = 2 } jamba_dtype;
 
 typedef struct CUstream_st* jamba_stream_t; /* same type as cudaStream_t */
 
@@ -238,19 +238,43 @@ jamba_status jamba_gemm(const void* a, const void* b, void* out, int ld_out, con
 /* -------------------------------------------------------------------- MoE */
 
 typedef struct jamba_moe_config {
-  int d_model;   /* 4096 */
-  int d_ff;      /* expert hidden width (14336), multiple of 128 */
-  int n_experts; /* n (16 in Jamba section 3.1), at most 64 */
-  int top_k;     /* K (2 in Jamba section 3.1), 1 or 2 */
-  int dtype;     /* JAMBA_BF16 */
+  int d_model;      /* 4096 */
+  int d_ff;         /* expert hidden width (14336), multiple of 128 */
+  int n_experts;    /* n (16 in Jamba section 3.1), at most 64 */
+  int top_k;        /* K (2 in Jamba section 3.1), 1 or 2 */
+  int dtype;        /* JAMBA_BF16: activations and router */
+  int expert_dtype; /* JAMBA_BF16: w_gate / w_up / w_down in bf16;
+                       JAMBA_INT8: ExpertsInt8 (Jamba-1.5 article, section on
+                       ExpertsInt8): the three expert matrices hold int8 codes
+                       q with one fp32 scale per output row (see
+                       jamba_quantize_int8_rows); the weight is q * scale and
+                       is widened to bf16 inside the expert GEMM kernels, the
+                       scale applied to the fp32 accumulator.  Activations and
+                       the router stay bf16. */
 } jamba_moe_config;
 
 typedef struct jamba_moe_weights {
-  const void* router; /* [n_experts, d_model] */
-  const void* w_gate; /* [n_experts, d_ff, d_model] */
-  const void* w_up;   /* [n_experts, d_ff, d_model] */
-  const void* w_down; /* [n_experts, d_model, d_ff] */
+  const void* router; /* [n_experts, d_model] dtype */
+  const void* w_gate; /* [n_experts, d_ff, d_model] expert_dtype */
+  const void* w_up;   /* [n_experts, d_ff, d_model] expert_dtype */
+  const void* w_down; /* [n_experts, d_model, d_ff] expert_dtype */
+  const float* s_gate; /* JAMBA_INT8 only: [n_experts, d_ff] row scales of w_gate (else NULL) */
+  const float* s_up;   /* JAMBA_INT8 only: [n_experts, d_ff] row scales of w_up */
+  const float* s_down; /* JAMBA_INT8 only: [n_experts, d_model] row scales of w_down */
 } jamba_moe_weights;
+
+/* Per-row symmetric INT8 quantisation, the ExpertsInt8 weight format (no
+ * calibration data: every row is quantised from its own values).
+ *   w     [rows, cols] dtype (JAMBA_BF16 or JAMBA_F32), row-major, contiguous
+ *   q     [rows, cols] int8 out
+ *   scale [rows] fp32 out
+ * For each row, in fp32 with IEEE division: scale = max|w| / 127 and
+ * q = round-half-even(w / scale), an integer in [-127, 127]; an all-zero row
+ * gives scale = 0 and q = 0.  cols must be a multiple of 8 and every pointer
+ * 16-byte aligned; JAMBA_ERR_INVALID_ARG otherwise.  Deterministic: the
+ * output depends only on w. */
+jamba_status jamba_quantize_int8_rows(const void* w, int dtype, long long rows, int cols, int8_t* q,
+                                      float* scale, jamba_stream_t stream);
 
 jamba_status jamba_moe_workspace_size(const jamba_moe_config* cfg, int tokens, size_t* bytes);
 

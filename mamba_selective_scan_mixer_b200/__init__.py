@@ -6,4 +6,5 @@ built or the tensors are not on a CUDA device.
 """
 from ._abi import JambaError, LIB_PATH, SIGNATURES, lib  # noqa: F401
 from .ops import (MambaMixer, MoE, causal_conv1d, device_status, gemm, layer_pair,  # noqa: F401
-                  rmsnorm, selective_scan, selective_scan_static)
+                  quantize_experts_int8, quantize_int8_rows, rmsnorm, selective_scan,
+                  selective_scan_static)

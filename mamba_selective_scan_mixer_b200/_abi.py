@@ -16,6 +16,7 @@ STATUS_NAMES = {0: "JAMBA_OK", 1: "JAMBA_ERR_INVALID_ARG", 2: "JAMBA_ERR_UNSUPPO
                 6: "JAMBA_ERR_OOM"}
 JAMBA_F32 = 0
 JAMBA_BF16 = 1
+JAMBA_INT8 = 2
 
 
 class JambaError(RuntimeError):
@@ -38,11 +39,12 @@ class MambaWeights(ctypes.Structure):
 
 class MoeConfig(ctypes.Structure):
     _fields_ = [("d_model", ctypes.c_int), ("d_ff", ctypes.c_int), ("n_experts", ctypes.c_int),
-                ("top_k", ctypes.c_int), ("dtype", ctypes.c_int)]
+                ("top_k", ctypes.c_int), ("dtype", ctypes.c_int), ("expert_dtype", ctypes.c_int)]
 
 
 class MoeWeights(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in ("router", "w_gate", "w_up", "w_down")]
+    _fields_ = [(n, ctypes.c_void_p) for n in ("router", "w_gate", "w_up", "w_down",
+                                               "s_gate", "s_up", "s_down")]
 
 
 P = ctypes.c_void_p
@@ -66,6 +68,7 @@ SIGNATURES = {
     "jamba_rmsnorm": [P, P, P, I, I, F, I, P],
     "jamba_causal_conv1d": [P, I, P, P, P, P, P, I, I, I, I, P],
     "jamba_gemm": [P, P, P, I, P, I, I, I, I, I, P],
+    "jamba_quantize_int8_rows": [P, I, ctypes.c_longlong, I, P, P, P],
     "jamba_moe_workspace_size": [ctypes.POINTER(MoeConfig), I, ctypes.POINTER(SZ)],
     "jamba_moe_forward": [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), P, P, P, I, P, P, P, P,
                           P, SZ, P],

@@ -594,9 +594,21 @@ jamba_status check_moe_cfg(const jamba_moe_config* c) {
   if (c->top_k < 1 || c->top_k > 2 || c->top_k > c->n_experts) return fail(JAMBA_ERR_UNSUPPORTED, "moe: top_k must be 1 or 2");
   if (c->d_model <= 0 || c->d_model % 256) return fail(JAMBA_ERR_UNSUPPORTED, "moe: d_model must be a multiple of 256");
   if (c->d_ff <= 0 || c->d_ff % 128) return fail(JAMBA_ERR_UNSUPPORTED, "moe: d_ff must be a multiple of 128");
+  if (c->expert_dtype != JAMBA_BF16 && c->expert_dtype != JAMBA_INT8)
+    return fail(JAMBA_ERR_UNSUPPORTED, "moe: expert_dtype must be JAMBA_BF16 or JAMBA_INT8");
   return JAMBA_OK;
 }
 }  // namespace
+
+jamba_status jamba_quantize_int8_rows(const void* w, int dtype, long long rows, int cols, int8_t* q, float* scale,
+                                      jamba_stream_t stream) {
+  JB_TRY(check_dtype(dtype));
+  if (rows <= 0 || cols <= 0 || cols % 8) return fail(JAMBA_ERR_INVALID_ARG, "quantize: rows > 0, cols a positive multiple of 8");
+  JB_TRY(check_ptr(w, "w"));
+  JB_TRY(check_ptr(q, "q"));
+  JB_TRY(check_ptr(scale, "scale"));
+  return quantize_int8_rows(w, dtype, rows, cols, q, scale, cs(stream));
+}
 
 jamba_status jamba_moe_workspace_size(const jamba_moe_config* cfg, int tokens, size_t* bytes) {
   JB_TRY(check_moe_cfg(cfg));
@@ -615,6 +627,10 @@ jamba_status jamba_moe_forward(const jamba_moe_config* cfg, const jamba_moe_weig
   JB_TRY(check_ptr(w->w_gate, "w_gate"));
   JB_TRY(check_ptr(w->w_up, "w_up"));
   JB_TRY(check_ptr(w->w_down, "w_down"));
+  const bool q8 = cfg->expert_dtype == JAMBA_INT8;
+  JB_TRY(check_ptr(w->s_gate, "s_gate", q8));
+  JB_TRY(check_ptr(w->s_up, "s_up", q8));
+  JB_TRY(check_ptr(w->s_down, "s_down", q8));
   JB_TRY(check_ptr(x, "x"));
   JB_TRY(check_ptr(y, "y"));
   JB_TRY(check_ptr(residual, "residual", false));
@@ -638,6 +654,11 @@ jamba_status jamba_moe_forward(const jamba_moe_config* cfg, const jamba_moe_weig
   g1.offsets = expert_offsets;
   g1.num_groups = E;
   g1.b_rows = dff;
+  if (q8) {
+    g1.b_int8 = 1;
+    g1.scale_b = w->s_gate;
+    g1.scale_b2 = w->s_up;
+  }
   JB_TRY(gemm_bf16(g1, s));
   // down: Y = act W_d^T, fp32 rows in routed order
   GemmDesc g2 = gdesc(m.act, dff, w->w_down, dff, rows, dm, dff, EPI_F32, m.Y, dm);
@@ -645,6 +666,10 @@ jamba_status jamba_moe_forward(const jamba_moe_config* cfg, const jamba_moe_weig
   g2.offsets = expert_offsets;
   g2.num_groups = E;
   g2.b_rows = dm;
+  if (q8) {
+    g2.b_int8 = 1;
+    g2.scale_b = w->s_down;
+  }
   JB_TRY(gemm_bf16(g2, s));
   JB_TRY(moe_combine(m.Y, m.inv, topk_w, tokens, K, dm, residual, y, s));
   return JAMBA_OK;

@@ -7,26 +7,34 @@
 
 namespace jb {
 
-template <int BN, int STAGES, int EPI, bool TRANS>
+template <int BN, int STAGES, int EPI, bool TRANS, bool QB = false>
 static jamba_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb2,
                               const CUtensorMap& mc, const GemmParams& p, int grid, cudaStream_t s) {
-  using S = GemmSmem<BN, STAGES, EPI == EPI_SOFTPLUS && !TRANS>;
+  using S = GemmSmem<BN, STAGES, EPI == EPI_SOFTPLUS && !TRANS, QB>;
   static bool configured[64] = {false};
   int dev = 0;
   JB_CUDA(cudaGetDevice(&dev));
   if (dev < 64 && !configured[dev]) {
-    JB_CUDA(cudaFuncSetAttribute(gemm_bf16_tc_kernel<BN, STAGES, EPI, TRANS>,
+    JB_CUDA(cudaFuncSetAttribute(gemm_bf16_tc_kernel<BN, STAGES, EPI, TRANS, QB>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::BYTES));
     configured[dev] = true;
   }
-  JB_CUDA(launch_pdl(gemm_bf16_tc_kernel<BN, STAGES, EPI, TRANS>, dim3(grid), dim3(GEMM_THREADS), S::BYTES, s, ma, mb,
-                     mb2, mc, p));
+  JB_CUDA(launch_pdl(gemm_bf16_tc_kernel<BN, STAGES, EPI, TRANS, QB>, dim3(grid), dim3(gemm_threads(QB)), S::BYTES,
+                     s, ma, mb, mb2, mc, p));
   return JAMBA_OK;
 }
 
 template <int EPI, bool TRANS>
-static jamba_status launch_bn(int bn, const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb2,
+static jamba_status launch_bn(int bn, bool qb, const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb2,
                               const CUtensorMap& mc, const GemmParams& p, int grid, cudaStream_t s) {
+  if constexpr (!TRANS && (EPI == EPI_SWIGLU || EPI == EPI_F32)) {
+    // INT8 B: three stages of A, widened B and codes (3 x 64 KB at BN = 256)
+    if (qb) {
+      if (bn == 256) return launch_tc<256, 3, EPI, false, true>(ma, mb, mb2, mc, p, grid, s);
+      return fail(JAMBA_ERR_UNSUPPORTED, "gemm: INT8 weights need tile width 256");
+    }
+  }
+  if (qb) return fail(JAMBA_ERR_UNSUPPORTED, "gemm: INT8 weights only with the grouped SwiGLU / fp32 epilogues");
   if constexpr (TRANS) {
     if (bn == 64) return launch_tc<64, 8, EPI, true>(ma, mb, mb2, mc, p, grid, s);
   } else if constexpr (EPI == EPI_SOFTPLUS) {
@@ -60,6 +68,15 @@ jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
     return fail(JAMBA_ERR_INVALID_ARG, "gemm: split-K writes fp32 partials only");
   if (g.epi == EPI_SWIGLU && (!g.grouped || !g.b2))
     return fail(JAMBA_ERR_INVALID_ARG, "gemm: SwiGLU needs grouped gate and up weights");
+  const bool qb = g.b_int8 != 0;
+  if (qb) {
+    if (!g.grouped || g.transpose_out || g.splits > 1 || (g.epi != EPI_SWIGLU && g.epi != EPI_F32))
+      return fail(JAMBA_ERR_UNSUPPORTED, "gemm: INT8 weights only in the grouped SwiGLU / fp32 expert GEMMs");
+    if (!g.scale_b || (g.epi == EPI_SWIGLU && !g.scale_b2) || !aligned16(g.scale_b) ||
+        (g.scale_b2 && !aligned16(g.scale_b2)) || g.N % 4 || g.ldb % 16 || g.K % 16)
+      return fail(JAMBA_ERR_INVALID_ARG,
+                  "gemm: INT8 weights need 16-byte aligned scales, N a multiple of 4, K and ldb of 16");
+  }
 
   int bn = g.bn;
   if (bn == 0) {
@@ -80,6 +97,15 @@ jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
     JB_TRY(make_map_2d(&mb, g.b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)g.K, (uint64_t)g.N,
                        (uint64_t)g.ldb * 2, 64, (uint32_t)b_box, CU_TENSOR_MAP_SWIZZLE_128B));
     mb2 = mb;
+  } else if (qb) {
+    // codes: 64 x b_box boxes of bytes, unswizzled (the dequantisers re-lay them out)
+    const uint64_t rs = (uint64_t)g.ldb, os = rs * (uint64_t)g.b_rows;
+    JB_TRY(make_map_3d(&mb, g.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)g.K, (uint64_t)g.b_rows,
+                       (uint64_t)g.num_groups, rs, os, 64, (uint32_t)b_box, CU_TENSOR_MAP_SWIZZLE_NONE));
+    mb2 = mb;
+    if (g.b2)
+      JB_TRY(make_map_3d(&mb2, g.b2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)g.K, (uint64_t)g.b_rows,
+                         (uint64_t)g.num_groups, rs, os, 64, (uint32_t)b_box, CU_TENSOR_MAP_SWIZZLE_NONE));
   } else {
     const uint64_t rs = (uint64_t)g.ldb * 2, os = rs * (uint64_t)g.b_rows;
     JB_TRY(make_map_3d(&mb, g.b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)g.K, (uint64_t)g.b_rows,
@@ -116,6 +142,8 @@ jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
   p.residual = g.residual;
   p.ldr = g.ldr;
   p.bias = g.bias;
+  p.scale_b = g.scale_b;
+  p.scale_b2 = g.scale_b2;
   p.err = device_error_word();
   if (!p.err) return fail(JAMBA_ERR_CUDA, "could not allocate the device status word");
 
@@ -124,17 +152,17 @@ jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
   const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
   if (g.transpose_out) {
     switch (g.epi) {
-      case EPI_BF16: return launch_bn<EPI_BF16, true>(bn, ma, mb, mb2, mc, p, grid, s);
-      case EPI_F32: return launch_bn<EPI_F32, true>(bn, ma, mb, mb2, mc, p, grid, s);
-      case EPI_SOFTPLUS: return launch_bn<EPI_SOFTPLUS, true>(bn, ma, mb, mb2, mc, p, grid, s);
+      case EPI_BF16: return launch_bn<EPI_BF16, true>(bn, qb, ma, mb, mb2, mc, p, grid, s);
+      case EPI_F32: return launch_bn<EPI_F32, true>(bn, qb, ma, mb, mb2, mc, p, grid, s);
+      case EPI_SOFTPLUS: return launch_bn<EPI_SOFTPLUS, true>(bn, qb, ma, mb, mb2, mc, p, grid, s);
       default: break;
     }
   } else {
     switch (g.epi) {
-      case EPI_BF16: return launch_bn<EPI_BF16, false>(bn, ma, mb, mb2, mc, p, grid, s);
-      case EPI_F32: return launch_bn<EPI_F32, false>(bn, ma, mb, mb2, mc, p, grid, s);
-      case EPI_SOFTPLUS: return launch_bn<EPI_SOFTPLUS, false>(bn, ma, mb, mb2, mc, p, grid, s);
-      case EPI_SWIGLU: return launch_bn<EPI_SWIGLU, false>(bn, ma, mb, mb2, mc, p, grid, s);
+      case EPI_BF16: return launch_bn<EPI_BF16, false>(bn, qb, ma, mb, mb2, mc, p, grid, s);
+      case EPI_F32: return launch_bn<EPI_F32, false>(bn, qb, ma, mb, mb2, mc, p, grid, s);
+      case EPI_SOFTPLUS: return launch_bn<EPI_SOFTPLUS, false>(bn, qb, ma, mb, mb2, mc, p, grid, s);
+      case EPI_SWIGLU: return launch_bn<EPI_SWIGLU, false>(bn, qb, ma, mb, mb2, mc, p, grid, s);
       default: break;
     }
   }

@@ -82,6 +82,9 @@ struct GemmDesc {
   const float* bias;
   int splits;      // >= 1; more than one only with fp32 partial outputs
   int bn;          // 0 = automatic
+  int b_int8;      // grouped expert GEMMs: b / b2 hold INT8 codes (row stride ldb bytes)
+  const float* scale_b;   // with b_int8: per-row scales [groups, b_rows] of b
+  const float* scale_b2;  // ... and of b2
 };
 jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s);
 jamba_status gemm_f32(const GemmDesc& g, cudaStream_t s);
@@ -129,6 +132,8 @@ jamba_status splitk_reduce(const float* part, int splits, long long split_stride
 jamba_status moe_route(const void* x, const void* W, int T, int dm, int E, int K, int* idx, float* w, int* counts,
                        int* offsets, int* perm, int* inv, cudaStream_t s);
 jamba_status moe_gather(const void* x, const int* perm, int rows, int K, int dm, void* out, cudaStream_t s);
+jamba_status quantize_int8_rows(const void* w, int dtype, long long rows, int cols, int8_t* q, float* scale,
+                                cudaStream_t s);
 jamba_status moe_combine(const float* Y, const int* inv, const float* w, int T, int K, int dm, const void* residual,
                          void* out, cudaStream_t s);
 

@@ -170,6 +170,76 @@ combine_kernel(const float* __restrict__ Y, const int* __restrict__ inv, const f
   }
 }
 
+// ExpertsInt8 weight format: one warp per row, absolute maximum, then the
+// codes.  Both passes read the row; the second finds it in L1/L2.
+template <typename T>
+__device__ __forceinline__ void load8(const T* p, float* f);
+template <>
+__device__ __forceinline__ void load8<bf16>(const bf16* p, float* f) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 v = __bfloat1622float2(h[i]);
+    f[2 * i] = v.x;
+    f[2 * i + 1] = v.y;
+  }
+}
+template <>
+__device__ __forceinline__ void load8<float>(const float* p, float* f) {
+  const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+quantize_rows_kernel(const T* __restrict__ w, long long rows, int cols, int8_t* __restrict__ q,
+                     float* __restrict__ scale) {
+  const int lane = threadIdx.x & 31;
+  const long long warps = (long long)gridDim.x * 8;
+  for (long long r = blockIdx.x * 8ll + (threadIdx.x >> 5); r < rows; r += warps) {
+    const T* wr = w + r * cols;
+    float amax = 0.f;
+    for (int c = lane * 8; c < cols; c += 256) {
+      float f[8];
+      load8(wr + c, f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float s = __fdiv_rn(amax, 127.0f);
+    if (lane == 0) scale[r] = s;
+    int8_t* qr = q + r * cols;
+    for (int c = lane * 8; c < cols; c += 256) {
+      float f[8];
+      load8(wr + c, f);
+      uint32_t pk[2] = {0u, 0u};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        // round half to even of the correctly rounded quotient; |w| <= amax keeps it within 127
+        const int v = s > 0.f ? max(-127, min(127, __float2int_rn(__fdiv_rn(f[i], s)))) : 0;
+        pk[i >> 2] |= (uint32_t)(v & 0xff) << (8 * (i & 3));
+      }
+      *reinterpret_cast<uint2*>(qr + c) = make_uint2(pk[0], pk[1]);
+    }
+  }
+}
+
+jamba_status quantize_int8_rows(const void* w, int dtype, long long rows, int cols, int8_t* q, float* scale,
+                                cudaStream_t s) {
+  long long blocks = (rows + 7) / 8;
+  const long long cap = 16ll * num_sms();
+  if (blocks > cap) blocks = cap;
+  if (dtype == JAMBA_BF16)
+    quantize_rows_kernel<bf16><<<(int)blocks, 256, 0, s>>>(reinterpret_cast<const bf16*>(w), rows, cols, q, scale);
+  else
+    quantize_rows_kernel<float><<<(int)blocks, 256, 0, s>>>(reinterpret_cast<const float*>(w), rows, cols, q, scale);
+  JB_CUDA(cudaGetLastError());
+  return JAMBA_OK;
+}
+
 jamba_status moe_route(const void* x, const void* W, int T, int dm, int E, int K, int* idx, float* w, int* counts,
                        int* offsets, int* perm, int* inv, cudaStream_t s) {
   JB_CUDA(cudaMemsetAsync(counts, 0, sizeof(int) * E, s));

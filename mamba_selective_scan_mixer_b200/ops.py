@@ -230,16 +230,45 @@ def gemm(a, b, residual=None, out_dtype=None, out=None, stream=None):
     return out
 
 
+def quantize_int8_rows(w, stream=None):
+    """ExpertsInt8 codes of w [..., cols] (bf16 or fp32, CUDA): (q int8 like w, scale fp32 [...])."""
+    _cuda(w)
+    _contig(w, "w")
+    cols = w.shape[-1]
+    rows = w.numel() // cols
+    q = torch.empty(w.shape, dtype=torch.int8, device=w.device)
+    s = torch.empty(w.shape[:-1], dtype=torch.float32, device=w.device)
+    check(lib().jamba_quantize_int8_rows(_p(w), _DT[w.dtype], rows, cols, _p(q), _p(s), _stream(stream)))
+    return q, s
+
+
+def quantize_experts_int8(params, stream=None):
+    """MoE parameters with the expert matrices replaced by ExpertsInt8 codes
+    (w_gate -> int8 codes + s_gate, ...); the router is kept as it is."""
+    out = {"router": params["router"]}
+    for k in ("gate", "up", "down"):
+        out["w_" + k], out["s_" + k] = quantize_int8_rows(params["w_" + k].contiguous(), stream)
+    return out
+
+
 class MoE:
-    """Top-K SwiGLU mixture of experts over borrowed weights (router, w_gate, w_up, w_down)."""
+    """Top-K SwiGLU mixture of experts over borrowed weights.
+
+    params: router, w_gate, w_up, w_down (bf16); with int8 expert matrices
+    (ExpertsInt8, see quantize_experts_int8) also s_gate, s_up, s_down.
+    """
 
     def __init__(self, params, shape):
         self.shape = shape
         self.params = {k: v.contiguous() for k, v in params.items()}
         _cuda(*self.params.values())
-        self.cfg = _abi.MoeConfig(shape.d_model, shape.d_ff, shape.n_experts, shape.top_k, _abi.JAMBA_BF16)
-        self.w = _abi.MoeWeights(*[ctypes.c_void_p(self.params[k].data_ptr())
-                                   for k in ("router", "w_gate", "w_up", "w_down")])
+        int8 = self.params["w_gate"].dtype == torch.int8
+        if int8 and not all(("s_" + k) in self.params for k in ("gate", "up", "down")):
+            raise ValueError("int8 expert weights need s_gate, s_up and s_down")
+        self.cfg = _abi.MoeConfig(shape.d_model, shape.d_ff, shape.n_experts, shape.top_k, _abi.JAMBA_BF16,
+                                  _abi.JAMBA_INT8 if int8 else _abi.JAMBA_BF16)
+        self.w = _abi.MoeWeights(*[_p(self.params.get(k)) for k in
+                                   ("router", "w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down")])
         self.ws = _Workspace()
 
     def workspace_size(self, tokens):

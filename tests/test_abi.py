@@ -71,14 +71,28 @@ def test_scan_and_moe_reject_bad_shapes_without_gpu(lib):
     st = lib.jamba_selective_scan(p, 64, p, 64, p, 64, p, 16, p, 16, 1, p, p, None, p, 64, None,
                                   1, 64, 64, 8, 1, 0, p, 1 << 20, None)
     assert st == 2
-    cfg = _abi.MoeConfig(4096, 14336, 16, 3, _abi.JAMBA_BF16)      # top_k 3
+    BF, I8 = _abi.JAMBA_BF16, _abi.JAMBA_INT8
+    cfg = _abi.MoeConfig(4096, 14336, 16, 3, BF, BF)      # top_k 3
     assert lib.jamba_moe_workspace_size(ctypes.byref(cfg), 128, ctypes.byref(n)) == 2
-    cfg = _abi.MoeConfig(4096, 14336, 16, 2, _abi.JAMBA_F32)       # fp32 MoE
+    cfg = _abi.MoeConfig(4096, 14336, 16, 2, _abi.JAMBA_F32, BF)       # fp32 MoE
     assert lib.jamba_moe_workspace_size(ctypes.byref(cfg), 128, ctypes.byref(n)) == 2
-    cfg = _abi.MoeConfig(4096, 14336, 16, 2, _abi.JAMBA_BF16)
+    cfg = _abi.MoeConfig(4096, 14336, 16, 2, BF, _abi.JAMBA_F32)       # fp32 expert weights
+    assert lib.jamba_moe_workspace_size(ctypes.byref(cfg), 128, ctypes.byref(n)) == 2
+    cfg = _abi.MoeConfig(4096, 14336, 16, 2, BF, I8)                   # ExpertsInt8
+    assert lib.jamba_moe_workspace_size(ctypes.byref(cfg), 128, ctypes.byref(n)) == 0
+    cfg = _abi.MoeConfig(4096, 14336, 16, 2, BF, BF)
     assert lib.jamba_moe_workspace_size(ctypes.byref(cfg), 32768, ctypes.byref(n)) == 0
     # routed rows 65536: gathered input, SwiGLU activations and fp32 expert outputs dominate
     assert n.value >= 65536 * (4096 * 2 + 14336 * 2 + 4096 * 4)
+    # int8 MoE without scales, and the quantiser's argument checks, fail before any launch
+    w = _abi.MoeWeights(p, p, p, p, None, None, None)
+    cfg = _abi.MoeConfig(4096, 14336, 16, 2, BF, I8)
+    st = lib.jamba_moe_forward(ctypes.byref(cfg), ctypes.byref(w), p, None, p, 64, p, p, p, p, p, 1 << 30, None)
+    assert st == 1
+    assert lib.jamba_quantize_int8_rows(p, BF, 16, 12, p, p, None) == 1     # cols not a multiple of 8
+    assert lib.jamba_quantize_int8_rows(p, BF, 0, 16, p, p, None) == 1      # no rows
+    assert lib.jamba_quantize_int8_rows(p, I8, 16, 16, p, p, None) == 2     # int8 input
+    assert lib.jamba_quantize_int8_rows(ctypes.c_void_p(4100), BF, 16, 16, p, p, None) == 1  # misaligned
 
 
 def test_product_path_fails_loudly_without_library(tmp_path):

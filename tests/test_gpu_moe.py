@@ -107,3 +107,95 @@ def test_layer_pair_small(dev):
     gap_ok = np.setdiff1d(np.arange(B * L), _near_ties(want["logits"], K, rel=2e-2))
     agree = (r["idx"].cpu().numpy()[gap_ok] == want["idx"][gap_ok]).all(axis=1).mean()
     assert agree == 1.0
+
+
+# ------------------------------------------------------------------ ExpertsInt8
+
+def _codes_equal(J_pq, o_pq):
+    for k in ("gate", "up", "down"):
+        np.testing.assert_array_equal(J_pq["w_" + k].cpu().numpy(), o_pq["q_" + k])
+        np.testing.assert_array_equal(J_pq["s_" + k].cpu().numpy(), o_pq["s_" + k])
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_quantize_int8_rows_bit_exact(dev, dtype):
+    import mamba_selective_scan_mixer_b200 as J
+    g = torch.Generator().manual_seed(3)
+    w = torch.randn(5, 37, 520, generator=g) * 0.02
+    w[1, 3] = 0.0                                                   # zero row: s = 0, q = 0
+    w[2, 4] = 0.0
+    w[2, 4, :8] = torch.tensor([127.0, -63.5, 2.5, 0.5, -1.5, 0.0, 1.0, 3.0])   # s = 1: halves tie to even
+    w[3, 7] *= 1e4                                                  # one row far above the rest
+    w = w.to(dtype)
+    q, s = J.quantize_int8_rows(w.to(dev))
+    qo, so = omoe.quantize_int8_rows(to_np(w))
+    np.testing.assert_array_equal(q.cpu().numpy(), qo)
+    np.testing.assert_array_equal(s.cpu().numpy(), so)
+    assert q[2, 4, :8].tolist() == [127, -64, 2, 0, -2, 0, 1, 3] and s[1, 3].item() == 0.0
+    # long rows (the d_ff width) with a ragged row count
+    w2 = (torch.randn(67, 14336, generator=g) * 0.02).to(dtype)
+    q2, s2 = J.quantize_int8_rows(w2.to(dev))
+    qo2, so2 = omoe.quantize_int8_rows(to_np(w2))
+    np.testing.assert_array_equal(q2.cpu().numpy(), qo2)
+    np.testing.assert_array_equal(s2.cpu().numpy(), so2)
+
+
+@pytest.mark.parametrize("T,dm,dff,residual,top_k", [(1000, 512, 384, False, 2), (333, 256, 640, True, 2),
+                                                     (1024, 4096, 1024, True, 2), (5, 256, 128, False, 2),
+                                                     (257, 512, 256, True, 1)])
+def test_moe_int8_forward(dev, T, dm, dff, residual, top_k):
+    """ExpertsInt8 MoE vs the oracle MoE on the dequantised weights q * s;
+    the codes and scales themselves bit-exact.  T = 5 leaves most experts
+    without rows; expert 0's gate and one down row are all zero (s = 0)."""
+    import mamba_selective_scan_mixer_b200 as J
+    shape = MoEShape(d_model=dm, d_ff=dff, n_experts=E, top_k=top_k)
+    seed = 100 + T + dff
+    p = moe_params(shape, seed=seed)
+    p["w_gate"][0] = 0.0
+    p["w_down"][1, 5] = 0.0
+    x = moe_input(shape, T, seed=seed)
+    res = moe_input(shape, T, seed=seed + 1) if residual else None
+    pq = J.quantize_experts_int8({k: v.to(dev) for k, v in p.items()})
+    oq = omoe.experts_int8({k: to_np(v) for k, v in p.items()})
+    _codes_equal(pq, oq)
+    r = J.MoE(pq, shape).forward(x.to(dev), residual=None if res is None else res.to(dev))
+    want = omoe.moe_forward(omoe.dequantized(oq), to_np(x), top_k)
+    if res is not None:
+        want["out"] = want["out"] + to_np(res)
+    np.testing.assert_array_equal(r["idx"].cpu().numpy(), want["idx"])
+    np.testing.assert_array_equal(r["offsets"].cpu().numpy(), want["offsets"])
+    assert rel_l2(to_np(r["out"]), want["out"]) < TOL_BF16
+
+
+def test_moe_int8_full_size_sampled(dev):
+    """d_model 4096, d_ff 14336, 16 experts, top-2, 32768 tokens (the layer
+    pair's MoE) with INT8 experts: every router decision and the codes of
+    the sampled tokens' experts bit-exact, 48 sampled tokens' outputs within
+    the bf16 bar (the oracle dequantises one expert at a time)."""
+    import mamba_selective_scan_mixer_b200 as J
+    shape = MoEShape()
+    T = 32768
+    p = moe_params(shape, seed=11, device=dev)
+    x = moe_input(shape, T, seed=11, device=dev)
+    pq = J.quantize_experts_int8(p)
+    moe = J.MoE(pq, shape)
+    r = moe.forward(x)
+    torch.cuda.synchronize()
+    xs = to_np(x)
+    idx, w, logits = omoe.router(xs, to_np(p["router"]), shape.top_k)
+    assert len(_near_ties(logits, shape.top_k)) == 0
+    np.testing.assert_array_equal(r["idx"].cpu().numpy(), idx)
+    rng = np.random.default_rng(12)
+    tok = np.sort(rng.choice(T, 48, replace=False))
+    got = to_np(r["out"][torch.as_tensor(tok, device=dev)])
+    want = np.zeros((len(tok), shape.d_model))
+    for e in np.unique(idx[tok]):
+        oq = omoe.experts_int8({"router": np.zeros(1), **{k: to_np(p[k][e]) for k in ("w_gate", "w_up", "w_down")}})
+        _codes_equal({k: pq[k][e] for k in pq if k != "router"}, oq)
+        d = omoe.dequantized(oq)
+        rows, slots = np.nonzero(idx[tok] == e)
+        ye = omoe.swiglu_expert(xs[tok[rows]], d["w_gate"], d["w_up"], d["w_down"])
+        for k in range(shape.top_k):
+            m = slots == k
+            want[rows[m]] += w[tok[rows[m]], k][:, None] * ye[m]
+    assert rel_l2(got, want) < TOL_BF16
