@@ -109,40 +109,6 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
   return d;
 }
 
-__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
-  float2 d;
-  asm("{.reg .b64 ra, rb, rd;\n\t"
-      "mov.b64 ra, {%2,%3};\n\tmov.b64 rb, {%4,%5};\n\t"
-      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0,%1}, rd;}"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  return d;
-}
-
-// Sixteen signed 8-bit integers (little-endian in v) to sixteen bf16 values,
-// exactly.  Each code x is biased to x + 128 (flip the sign bit of the byte),
-// placed in the low mantissa byte of the fp32 number 2^23 (which has a unit
-// step there), so the float equals 2^23 + 128 + x; subtracting 2^23 + 128
-// leaves x, and |x| <= 128 fits in bf16's 8 significant bits.
-__device__ __forceinline__ void i8x16_to_bf16(uint4 v, uint4& lo, uint4& hi) {
-  const uint32_t w[4] = {v.x ^ 0x80808080u, v.y ^ 0x80808080u, v.z ^ 0x80808080u, v.w ^ 0x80808080u};
-  const float2 bias = make_float2(-8388736.0f, -8388736.0f);
-  uint32_t o[8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const float2 f = fadd2(make_float2(__uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7540u | (2 * j))),
-                                         __uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7540u | (2 * j + 1)))),
-                             bias);
-      const __nv_bfloat162 h = __floats2bfloat162_rn(f.x, f.y);   // .x -> the lower address
-      o[2 * i + j] = *reinterpret_cast<const uint32_t*>(&h);
-    }
-  }
-  lo = make_uint4(o[0], o[1], o[2], o[3]);
-  hi = make_uint4(o[4], o[5], o[6], o[7]);
-}
-
 // r^1 .. r^16
 __device__ __forceinline__ void powers16(float r, float* pw) {
   pw[0] = r;

@@ -1,40 +1,66 @@
-// GEMM launchers: the tcgen05 kernel for bf16 and a CUDA-core kernel for the
-// fp32 path (fp32 inputs must keep ~1e-5 accuracy, which TF32 would not).
+// GEMM launchers: the tcgen05 kernel for bf16, the INT8-weight grouped expert
+// kernel, and a CUDA-core kernel for the fp32 path (fp32 inputs must keep ~1e-5
+// accuracy, which TF32 would not).
 #include <string>
 
+#include "gemm_i8w.cuh"
 #include "gemm_tc.cuh"
 #include "host.hpp"
 
 namespace jb {
 
-template <int BN, int STAGES, int EPI, bool TRANS, bool QB = false>
+template <int BN, int STAGES, int EPI, bool TRANS>
 static jamba_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb2,
                               const CUtensorMap& mc, const GemmParams& p, int grid, cudaStream_t s) {
-  using S = GemmSmem<BN, STAGES, EPI == EPI_SOFTPLUS && !TRANS, QB>;
+  using S = GemmSmem<BN, STAGES, EPI == EPI_SOFTPLUS && !TRANS>;
   static bool configured[64] = {false};
   int dev = 0;
   JB_CUDA(cudaGetDevice(&dev));
   if (dev < 64 && !configured[dev]) {
-    JB_CUDA(cudaFuncSetAttribute(gemm_bf16_tc_kernel<BN, STAGES, EPI, TRANS, QB>,
+    JB_CUDA(cudaFuncSetAttribute(gemm_bf16_tc_kernel<BN, STAGES, EPI, TRANS>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::BYTES));
     configured[dev] = true;
   }
-  JB_CUDA(launch_pdl(gemm_bf16_tc_kernel<BN, STAGES, EPI, TRANS, QB>, dim3(grid), dim3(gemm_threads(QB)), S::BYTES,
-                     s, ma, mb, mb2, mc, p));
+  JB_CUDA(launch_pdl(gemm_bf16_tc_kernel<BN, STAGES, EPI, TRANS>, dim3(grid), dim3(GEMM_THREADS), S::BYTES, s, ma, mb,
+                     mb2, mc, p));
+  return JAMBA_OK;
+}
+
+template <int EPI, int MT>
+static jamba_status launch_i8w(const CUtensorMap& ma, const CUtensorMap& mq, const CUtensorMap& mq2,
+                               const GemmParams& p, int grid, cudaStream_t s) {
+  using S = I8wSmem<MT>;
+  static bool configured[64] = {false};
+  int dev = 0;
+  JB_CUDA(cudaGetDevice(&dev));
+  if (dev < 64 && !configured[dev]) {
+    JB_CUDA(cudaFuncSetAttribute(gemm_i8w_kernel<EPI, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)S::BYTES));
+    configured[dev] = true;
+  }
+  JB_CUDA(launch_pdl(gemm_i8w_kernel<EPI, MT>, dim3(grid), dim3(I8W_THREADS), S::BYTES, s, ma, mq, mq2, p));
+  return JAMBA_OK;
+}
+
+template <int EPI>
+static jamba_status launch_i8t(const CUtensorMap& ma, const CUtensorMap& mq, const CUtensorMap& mq2,
+                               const GemmParams& p, int grid, cudaStream_t s) {
+  using S = I8tSmem<EPI>;
+  static bool configured[64] = {false};
+  int dev = 0;
+  JB_CUDA(cudaGetDevice(&dev));
+  if (dev < 64 && !configured[dev]) {
+    JB_CUDA(cudaFuncSetAttribute(gemm_i8w_tok_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)S::BYTES));
+    configured[dev] = true;
+  }
+  JB_CUDA(launch_pdl(gemm_i8w_tok_kernel<EPI>, dim3(grid), dim3(I8W_THREADS), S::BYTES, s, ma, mq, mq2, p));
   return JAMBA_OK;
 }
 
 template <int EPI, bool TRANS>
-static jamba_status launch_bn(int bn, bool qb, const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb2,
+static jamba_status launch_bn(int bn, const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb2,
                               const CUtensorMap& mc, const GemmParams& p, int grid, cudaStream_t s) {
-  if constexpr (!TRANS && (EPI == EPI_SWIGLU || EPI == EPI_F32)) {
-    // INT8 B: three stages of A, widened B and codes (3 x 64 KB at BN = 256)
-    if (qb) {
-      if (bn == 256) return launch_tc<256, 3, EPI, false, true>(ma, mb, mb2, mc, p, grid, s);
-      return fail(JAMBA_ERR_UNSUPPORTED, "gemm: INT8 weights need tile width 256");
-    }
-  }
-  if (qb) return fail(JAMBA_ERR_UNSUPPORTED, "gemm: INT8 weights only with the grouped SwiGLU / fp32 epilogues");
   if constexpr (TRANS) {
     if (bn == 64) return launch_tc<64, 8, EPI, true>(ma, mb, mb2, mc, p, grid, s);
   } else if constexpr (EPI == EPI_SOFTPLUS) {
@@ -54,6 +80,69 @@ static jamba_status launch_bn(int bn, bool qb, const CUtensorMap& ma, const CUte
   return fail(JAMBA_ERR_UNSUPPORTED, "gemm: no kernel for tile width " + std::to_string(bn) + " with this epilogue");
 }
 
+// Grouped expert GEMMs with INT8 weights (see gemm_i8w.cuh), by the average
+// number of routed rows per expert: up to 32, the weights take the M side
+// (decode batches: bound by streaming the codes); up to 255, 128-row tiles
+// with double-buffered accumulators; from 256, two 128-row halves share one
+// widened weight tile.
+static jamba_status gemm_i8w(const GemmDesc& g, cudaStream_t s) {
+  if (!g.grouped || g.transpose_out || g.splits > 1 || g.residual || (g.epi != EPI_SWIGLU && g.epi != EPI_F32))
+    return fail(JAMBA_ERR_UNSUPPORTED, "gemm: INT8 weights only in the grouped SwiGLU / fp32 expert GEMMs");
+  if (!g.scale_b || (g.epi == EPI_SWIGLU && (!g.scale_b2 || !g.b2)) || !aligned16(g.scale_b) ||
+      (g.scale_b2 && !aligned16(g.scale_b2)) || g.N % 4 || g.ldb % 16 || g.K % 16 || !aligned16(g.b) ||
+      (g.b2 && !aligned16(g.b2)))
+    return fail(JAMBA_ERR_INVALID_ARG,
+                "gemm: INT8 weights need 16-byte aligned codes and scales, N a multiple of 4, K and ldb of 16");
+  const int avg_rows = g.M / g.num_groups;
+  const bool tok = avg_rows <= I8T_BNT;
+  const int bn_out = tok ? 128 : g.epi == EPI_SWIGLU ? I8W_BN / 2 : I8W_BN;
+  const uint32_t q_box = (uint32_t)(tok ? 128 : bn_out);
+  const uint32_t q_inner = tok ? 128 : 64;   // codes per row per load
+  const CUtensorMapSwizzle q_sw = tok ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
+  CUtensorMap ma, mq, mq2;
+  JB_TRY(make_map_2d(&ma, g.a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)g.K, (uint64_t)g.M,
+                     (uint64_t)g.lda * 2, 64, tok ? I8T_BNT : 128, CU_TENSOR_MAP_SWIZZLE_128B));
+  const uint64_t rs = (uint64_t)g.ldb, os = rs * (uint64_t)g.b_rows;
+  JB_TRY(make_map_3d(&mq, g.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)g.K, (uint64_t)g.b_rows,
+                     (uint64_t)g.num_groups, rs, os, q_inner, q_box, q_sw));
+  mq2 = mq;
+  if (g.b2)
+    JB_TRY(make_map_3d(&mq2, g.b2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)g.K, (uint64_t)g.b_rows,
+                       (uint64_t)g.num_groups, rs, os, q_inner, q_box, q_sw));
+  GemmParams p = {};
+  p.M = g.M;
+  p.N = g.N;
+  p.K = g.K;
+  p.k_tiles = (g.K + 63) / 64;
+  p.splits = 1;
+  p.k_tiles_per_split = p.k_tiles;
+  p.n_tiles = (g.N + bn_out - 1) / bn_out;
+  p.grouped = 1;
+  p.offsets = g.offsets;
+  p.num_groups = g.num_groups;
+  p.out = g.out;
+  p.ldo = g.ldo;
+  p.scale_b = g.scale_b;
+  p.scale_b2 = g.scale_b2;
+  p.err = device_error_word();
+  if (!p.err) return fail(JAMBA_ERR_CUDA, "could not allocate the device status word");
+  if (tok) {
+    if (g.N % 128 || g.K % 128)
+      return fail(JAMBA_ERR_INVALID_ARG, "gemm: INT8 weights with few rows need N and K multiples of 128");
+    const long long tiles = (long long)((g.M + I8T_BNT - 1) / I8T_BNT + g.num_groups) * p.n_tiles;
+    const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
+    return g.epi == EPI_SWIGLU ? launch_i8t<EPI_SWIGLU>(ma, mq, mq2, p, grid, s)
+                               : launch_i8t<EPI_F32>(ma, mq, mq2, p, grid, s);
+  }
+  const bool pairs = avg_rows >= 256;
+  const int mh = pairs ? 256 : 128;
+  const long long tiles = (long long)((g.M + mh - 1) / mh + g.num_groups) * p.n_tiles;
+  const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
+  if (g.epi == EPI_SWIGLU)
+    return pairs ? launch_i8w<EPI_SWIGLU, 2>(ma, mq, mq2, p, grid, s) : launch_i8w<EPI_SWIGLU, 1>(ma, mq, mq2, p, grid, s);
+  return pairs ? launch_i8w<EPI_F32, 2>(ma, mq, mq2, p, grid, s) : launch_i8w<EPI_F32, 1>(ma, mq, mq2, p, grid, s);
+}
+
 jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
   if (g.M <= 0 || g.N <= 0 || g.K <= 0) return fail(JAMBA_ERR_INVALID_ARG, "gemm: sizes must be positive");
   if (!g.a || !g.b || !g.out) return fail(JAMBA_ERR_INVALID_ARG, "gemm: null operand");
@@ -68,16 +157,7 @@ jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
     return fail(JAMBA_ERR_INVALID_ARG, "gemm: split-K writes fp32 partials only");
   if (g.epi == EPI_SWIGLU && (!g.grouped || !g.b2))
     return fail(JAMBA_ERR_INVALID_ARG, "gemm: SwiGLU needs grouped gate and up weights");
-  const bool qb = g.b_int8 != 0;
-  if (qb) {
-    if (!g.grouped || g.transpose_out || g.splits > 1 || (g.epi != EPI_SWIGLU && g.epi != EPI_F32))
-      return fail(JAMBA_ERR_UNSUPPORTED, "gemm: INT8 weights only in the grouped SwiGLU / fp32 expert GEMMs");
-    if (!g.scale_b || (g.epi == EPI_SWIGLU && !g.scale_b2) || !aligned16(g.scale_b) ||
-        (g.scale_b2 && !aligned16(g.scale_b2)) || g.N % 4 || g.ldb % 16 || g.K % 16)
-      return fail(JAMBA_ERR_INVALID_ARG,
-                  "gemm: INT8 weights need 16-byte aligned scales, N a multiple of 4, K and ldb of 16");
-  }
-
+  if (g.b_int8) return gemm_i8w(g, s);
   int bn = g.bn;
   if (bn == 0) {
     if (g.epi == EPI_SWIGLU || g.epi == EPI_SOFTPLUS) bn = g.transpose_out ? 64 : 256;
@@ -97,15 +177,6 @@ jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
     JB_TRY(make_map_2d(&mb, g.b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)g.K, (uint64_t)g.N,
                        (uint64_t)g.ldb * 2, 64, (uint32_t)b_box, CU_TENSOR_MAP_SWIZZLE_128B));
     mb2 = mb;
-  } else if (qb) {
-    // codes: 64 x b_box boxes of bytes, unswizzled (the dequantisers re-lay them out)
-    const uint64_t rs = (uint64_t)g.ldb, os = rs * (uint64_t)g.b_rows;
-    JB_TRY(make_map_3d(&mb, g.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)g.K, (uint64_t)g.b_rows,
-                       (uint64_t)g.num_groups, rs, os, 64, (uint32_t)b_box, CU_TENSOR_MAP_SWIZZLE_NONE));
-    mb2 = mb;
-    if (g.b2)
-      JB_TRY(make_map_3d(&mb2, g.b2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)g.K, (uint64_t)g.b_rows,
-                         (uint64_t)g.num_groups, rs, os, 64, (uint32_t)b_box, CU_TENSOR_MAP_SWIZZLE_NONE));
   } else {
     const uint64_t rs = (uint64_t)g.ldb * 2, os = rs * (uint64_t)g.b_rows;
     JB_TRY(make_map_3d(&mb, g.b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)g.K, (uint64_t)g.b_rows,
@@ -142,8 +213,6 @@ jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
   p.residual = g.residual;
   p.ldr = g.ldr;
   p.bias = g.bias;
-  p.scale_b = g.scale_b;
-  p.scale_b2 = g.scale_b2;
   p.err = device_error_word();
   if (!p.err) return fail(JAMBA_ERR_CUDA, "could not allocate the device status word");
 
@@ -152,17 +221,17 @@ jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
   const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
   if (g.transpose_out) {
     switch (g.epi) {
-      case EPI_BF16: return launch_bn<EPI_BF16, true>(bn, qb, ma, mb, mb2, mc, p, grid, s);
-      case EPI_F32: return launch_bn<EPI_F32, true>(bn, qb, ma, mb, mb2, mc, p, grid, s);
-      case EPI_SOFTPLUS: return launch_bn<EPI_SOFTPLUS, true>(bn, qb, ma, mb, mb2, mc, p, grid, s);
+      case EPI_BF16: return launch_bn<EPI_BF16, true>(bn, ma, mb, mb2, mc, p, grid, s);
+      case EPI_F32: return launch_bn<EPI_F32, true>(bn, ma, mb, mb2, mc, p, grid, s);
+      case EPI_SOFTPLUS: return launch_bn<EPI_SOFTPLUS, true>(bn, ma, mb, mb2, mc, p, grid, s);
       default: break;
     }
   } else {
     switch (g.epi) {
-      case EPI_BF16: return launch_bn<EPI_BF16, false>(bn, qb, ma, mb, mb2, mc, p, grid, s);
-      case EPI_F32: return launch_bn<EPI_F32, false>(bn, qb, ma, mb, mb2, mc, p, grid, s);
-      case EPI_SOFTPLUS: return launch_bn<EPI_SOFTPLUS, false>(bn, qb, ma, mb, mb2, mc, p, grid, s);
-      case EPI_SWIGLU: return launch_bn<EPI_SWIGLU, false>(bn, qb, ma, mb, mb2, mc, p, grid, s);
+      case EPI_BF16: return launch_bn<EPI_BF16, false>(bn, ma, mb, mb2, mc, p, grid, s);
+      case EPI_F32: return launch_bn<EPI_F32, false>(bn, ma, mb, mb2, mc, p, grid, s);
+      case EPI_SOFTPLUS: return launch_bn<EPI_SOFTPLUS, false>(bn, ma, mb, mb2, mc, p, grid, s);
+      case EPI_SWIGLU: return launch_bn<EPI_SWIGLU, false>(bn, ma, mb, mb2, mc, p, grid, s);
       default: break;
     }
   }

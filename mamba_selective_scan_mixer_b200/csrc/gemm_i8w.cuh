@@ -1,0 +1,604 @@
+// Grouped expert GEMM with INT8 weights (ExpertsInt8: the expert matrices are
+// stored as 8-bit codes with one fp32 scale per output row and are widened
+// inside this kernel; activations stay bf16).
+//
+//   D[m, n] = scale[g, n] * sum_k A[m, k] * q[g, n, k]     (rows m of group g)
+//
+// A: the gathered activations [rows, K] bf16; q: [groups, N_rows, K] int8.
+// The widened weights are exact (|q| <= 127 fits bf16), so the only rounding
+// is the fp32 accumulation and the scale product, as in the bf16 path.
+//
+// One persistent CTA per SM, 14 warps:
+//   warp 0      TMA producer: per k-step MT activation tiles (128 x 64 bf16,
+//               128-byte swizzle) and the 256 x 64 code tile (unswizzled
+//               bytes) into a TSTAGES-deep ring;
+//   warp 1      TMEM owner and MMA issuer: M = 128, N = 256, K = 16 per
+//               instruction, MT accumulators per tile (MT = 2: both halves of
+//               a 256-row tile share one widened weight tile);
+//   warps 2-9   epilogue: scales, SwiGLU or fp32 stores;
+//   warps 10-13 dequantisers: code tile -> bf16 weight tile in the 128-byte
+//               swizzled K-major layout, into a separate BSTAGES-deep ring,
+//               so widening k-step i + 1 overlaps the MMAs of k-step i.
+// Widening one code: the low 7 bits l go under the bf16 exponent of 128
+// (value 128 + l) and the sign bit under the same exponent (value 128 or
+// 256); their bf16 difference is the code exactly.  Two codes per
+// instruction: 2 LOP3 + 4 PRMT + 2 HSUB2 per 4 codes.
+// Every wait is bounded (see common.cuh).
+#pragma once
+#include "gemm_tc.cuh"
+
+namespace jb {
+
+constexpr int I8W_THREADS = 448;
+constexpr int I8W_BN = 256;          // MMA N: SwiGLU 128 gate + 128 up rows, or 256 down rows
+constexpr int I8W_TSTAGES = 3;
+constexpr int I8W_BSTAGES = 2;
+constexpr int I8W_DQ_WARPS = 4;
+
+template <int MT>
+struct I8wSmem {
+  static constexpr uint32_t A_BYTES = 128 * 128;              // one 128 x 64 bf16 activation tile
+  static constexpr uint32_t Q_BYTES = I8W_BN * 64;            // 256 x 64 codes
+  static constexpr uint32_t B_BYTES = I8W_BN * 128;           // 256 x 64 bf16 widened weights
+  static constexpr uint32_t T_STAGE = MT * A_BYTES + Q_BYTES;
+  static constexpr uint32_t B_OFF = I8W_TSTAGES * T_STAGE;
+  static constexpr uint32_t BAR_OFF = B_OFF + I8W_BSTAGES * B_BYTES;
+  static constexpr uint32_t BYTES = BAR_OFF + 256 + 1024;
+};
+
+// bf16x2 a - b (exact here: both operands and the result are small integers)
+__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// 16 int8 codes (little-endian) -> 16 bf16 values, exactly
+__device__ __forceinline__ void widen16(uint4 v, uint4& lo, uint4& hi) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t l = w[i] & 0x7F7F7F7Fu, s = w[i] & 0x80808080u;
+    // bytes {l0, 0x43, l1, 0x43}: bf16 128 + l; {s0, 0x43, s1, 0x43}: bf16 128 or 256
+    o[2 * i] = bf16x2_sub(__byte_perm(l, 0x43434343u, 0x5140u), __byte_perm(s, 0x43434343u, 0x5140u));
+    o[2 * i + 1] = bf16x2_sub(__byte_perm(l, 0x43434343u, 0x5342u), __byte_perm(s, 0x43434343u, 0x5342u));
+  }
+  lo = make_uint4(o[0], o[1], o[2], o[3]);
+  hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+// ROWS x 64 codes (row-major, 64-byte rows) -> ROWS x 64 bf16 in the 128-byte
+// swizzled K-major layout, by the I8W_DQ_WARPS dequantiser warps (thread ct).
+// 16 codes per load become two 16-byte chunks of the same row; a quarter-warp
+// covers two rows and stores to eight distinct chunks (no bank conflicts).
+template <int ROWS>
+__device__ __forceinline__ void widen_tile(const uint8_t* qs, uint8_t* bdst, int ct) {
+  constexpr int PER = 32 * I8W_DQ_WARPS;
+  static_assert((ROWS * 4) % PER == 0, "whole iterations");
+#pragma unroll
+  for (int i = 0; i < ROWS * 4 / PER; ++i) {
+    const int idx = ct + PER * i;
+    const int row = idx >> 2, g = idx & 3;
+    uint4 lo, hi;
+    widen16(*reinterpret_cast<const uint4*>(qs + idx * 16), lo, hi);
+    *reinterpret_cast<uint4*>(bdst + row * 128 + (((2 * g) ^ (row & 7)) << 4)) = lo;
+    *reinterpret_cast<uint4*>(bdst + row * 128 + (((2 * g + 1) ^ (row & 7)) << 4)) = hi;
+  }
+}
+
+template <int MH>
+__device__ __forceinline__ int total_tiles_grouped(const GemmParams& p) {
+  int tot = 0;
+  for (int g = 0; g < p.num_groups; ++g) {
+    const int cnt = __ldg(p.offsets + g + 1) - __ldg(p.offsets + g);
+    tot += ((cnt + MH - 1) / MH) * p.n_tiles;
+  }
+  return tot;
+}
+
+// grouped tile t -> (group, rows m0..m0+MH-1 clipped at m_end, output columns n0..)
+template <int MH, int BN_OUT>
+__device__ __forceinline__ void decode_tile_grouped(const GemmParams& p, int t, TileInfo& ti) {
+  for (int g = 0; g < p.num_groups; ++g) {
+    const int o0 = __ldg(p.offsets + g), o1 = __ldg(p.offsets + g + 1);
+    const int mt = (o1 - o0 + MH - 1) / MH;
+    const int tg = mt * p.n_tiles;
+    if (t < tg) {
+      const int mb = t % mt, nb = t / mt;   // m fastest: neighbouring CTAs share the code tile in L2
+      ti.m0 = o0 + mb * MH;
+      ti.m_end = o1;
+      ti.n0 = nb * BN_OUT;
+      ti.kt0 = 0;
+      ti.kt1 = p.k_tiles;
+      ti.group = g;
+      ti.split = 0;
+      return;
+    }
+    t -= tg;
+  }
+  ti.m0 = ti.m_end = ti.n0 = ti.kt0 = ti.kt1 = ti.group = ti.split = 0;
+}
+
+template <int EPI, int MT>
+__global__ void __launch_bounds__(I8W_THREADS, 1)
+gemm_i8w_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmQ,
+                const __grid_constant__ CUtensorMap tmQ2, const GemmParams p) {
+  static_assert(EPI == EPI_SWIGLU || EPI == EPI_F32, "expert GEMMs only");
+  static_assert(MT == 1 || MT == 2, "one or two 128-row halves per tile");
+  using S = I8wSmem<MT>;
+  constexpr int BN = I8W_BN;
+  constexpr int BN_OUT = EPI == EPI_SWIGLU ? BN / 2 : BN;
+  constexpr int MH = 128 * MT;
+  constexpr int NBUF = 2 / MT;             // accumulator sets in TMEM (512 columns in all)
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sB = smem + S::B_OFF;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::BAR_OFF);
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + I8W_TSTAGES);
+  const uint32_t bfull0 = smem_u32(bars + 2 * I8W_TSTAGES);
+  const uint32_t bempty0 = smem_u32(bars + 2 * I8W_TSTAGES + I8W_BSTAGES);
+  const uint32_t tfull0 = smem_u32(bars + 2 * I8W_TSTAGES + 2 * I8W_BSTAGES);
+  const uint32_t tempty0 = tfull0 + 16;
+  const uint32_t drain = tfull0 + 32;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * I8W_TSTAGES + 2 * I8W_BSTAGES + 5);
+  static_assert(8 * (2 * I8W_TSTAGES + 2 * I8W_BSTAGES + 6) <= 256, "barrier slots");
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < I8W_TSTAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int s = 0; s < I8W_BSTAGES; ++s) {
+      mbar_init(bfull0 + 8 * s, I8W_DQ_WARPS);
+      mbar_init(bempty0 + 8 * s, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(tfull0 + 8 * i, 1);
+      mbar_init(tempty0 + 8 * i, GEMM_EPI_WARPS);
+    }
+    mbar_init(drain, 1);
+    mbar_fence_init();
+    tma_prefetch(&tmA);
+    tma_prefetch(&tmQ);
+    if (EPI == EPI_SWIGLU) tma_prefetch(&tmQ2);
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_holder), 512);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_holder;
+  griddep_launch();
+  griddep_wait();   // offsets and activations come from the previous kernels
+  const int ntiles = total_tiles_grouped<MH>(p);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        TileInfo ti;
+        decode_tile_grouped<MH, BN_OUT>(p, t, ti);
+        const bool two = MT == 2 && ti.m0 + 128 < ti.m_end;
+        for (int kt = ti.kt0; kt < ti.kt1; ++kt) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, p.err)) { ok = false; break; }
+          const uint32_t fb = full0 + 8 * stage;
+          uint8_t* st = smem + stage * S::T_STAGE;
+          mbar_arrive_tx(fb, (two ? 2 : 1) * S::A_BYTES + S::Q_BYTES);
+          tma_load_2d(smem_u32(st), &tmA, fb, kt * 64, ti.m0);
+          if (two) tma_load_2d(smem_u32(st + S::A_BYTES), &tmA, fb, kt * 64, ti.m0 + 128);
+          const uint32_t q_dst = smem_u32(st + MT * S::A_BYTES);
+          if constexpr (EPI == EPI_SWIGLU) {
+            tma_load_3d(q_dst, &tmQ, fb, kt * 64, ti.n0, ti.group);
+            tma_load_3d(q_dst + (BN / 2) * 64, &tmQ2, fb, kt * 64, ti.n0, ti.group);
+          } else {
+            tma_load_3d(q_dst, &tmQ, fb, kt * 64, ti.n0, ti.group);
+          }
+          if (++stage == I8W_TSTAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_bf16(128, BN);
+      int ts = 0, bs = 0;
+      uint32_t tph = 0, bph = 0;
+      bool ok = true;
+      int it = 0;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++it) {
+        TileInfo ti;
+        decode_tile_grouped<MH, BN_OUT>(p, t, ti);
+        const bool two = MT == 2 && ti.m0 + 128 < ti.m_end;
+        const int buf = it % NBUF;
+        const uint32_t use = (uint32_t)(it / NBUF);
+        if (!mbar_wait(tempty0 + 8 * buf, (use & 1) ^ 1, p.err)) break;
+        tc_fence_after();
+        const uint32_t d0 = tbase + buf * BN;   // MT = 2: buf is 0, the halves use columns 0 and 256
+        for (int kt = ti.kt0; kt < ti.kt1; ++kt) {
+          if (!mbar_wait(full0 + 8 * ts, tph, p.err)) { ok = false; break; }
+          if (!mbar_wait(bfull0 + 8 * bs, bph, p.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint8_t* st = smem + ts * S::T_STAGE;
+          const uint64_t bd = sw128_desc(smem_u32(sB + bs * S::B_BYTES));
+          const uint64_t ad0 = sw128_desc(smem_u32(st));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(d0, ad0 + 2 * kk, bd + 2 * kk, IDESC, (kt > ti.kt0 || kk > 0) ? 1u : 0u);
+          if (two) {
+            const uint64_t ad1 = sw128_desc(smem_u32(st + S::A_BYTES));
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16(d0 + BN, ad1 + 2 * kk, bd + 2 * kk, IDESC, (kt > ti.kt0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(empty0 + 8 * ts);
+          umma_commit(bempty0 + 8 * bs);
+          if (++ts == I8W_TSTAGES) { ts = 0; tph ^= 1; }
+          if (++bs == I8W_BSTAGES) { bs = 0; bph ^= 1; }
+        }
+        if (!ok) break;
+        umma_commit(tfull0 + 8 * buf);
+      }
+      umma_commit(drain);
+      mbar_wait(drain, 0, p.err);
+    }
+  } else if (warp >= 2 + GEMM_EPI_WARPS) {
+    const int ct = threadIdx.x - 32 * (2 + GEMM_EPI_WARPS);
+    int ts = 0, bs = 0;
+    uint32_t tph = 0, bph = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+      TileInfo ti;
+      decode_tile_grouped<MH, BN_OUT>(p, t, ti);
+      for (int kt = ti.kt0; kt < ti.kt1; ++kt) {
+        if (!mbar_wait(full0 + 8 * ts, tph, p.err)) { ok = false; break; }
+        if (!mbar_wait(bempty0 + 8 * bs, bph ^ 1, p.err)) { ok = false; break; }
+        widen_tile<BN>(smem + ts * S::T_STAGE + MT * S::A_BYTES, sB + bs * S::B_BYTES, ct);
+        fence_async_shared();   // the tensor core reads these stores through the async proxy
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bfull0 + 8 * bs);
+        if (++ts == I8W_TSTAGES) { ts = 0; tph ^= 1; }
+        if (++bs == I8W_BSTAGES) { bs = 0; bph ^= 1; }
+      }
+    }
+  } else {
+    const int q = warp & 3;                 // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;       // which of the two warps of this quarter
+    int it = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
+      TileInfo ti;
+      decode_tile_grouped<MH, BN_OUT>(p, t, ti);
+      const bool two = MT == 2 && ti.m0 + 128 < ti.m_end;
+      const int buf = it % NBUF;
+      const uint32_t use = (uint32_t)(it / NBUF);
+      if (!mbar_wait(tfull0 + 8 * buf, use & 1, p.err)) break;
+      tc_fence_after();
+      const float* sc = p.scale_b + (long long)ti.group * p.N;
+      for (int h = 0; h < (two ? 2 : 1); ++h) {
+        const int m = ti.m0 + h * 128 + q * 32 + lane;
+        const uint32_t tl = tbase + ((uint32_t)(q * 32) << 16) + buf * BN + h * BN;
+        if constexpr (EPI == EPI_F32) {
+#pragma unroll 1
+          for (int j = half; j < BN / 32; j += 2) {
+            float v[32];
+            tmem_ld32(tl + j * 32, v);
+            tmem_wait_ld();
+            scale32(v, sc, ti.n0 + j * 32, p.N);
+            epi_chunk<EPI_F32, false, 32>(p, ti, m, ti.n0 + j * 32, v);
+          }
+        } else {
+          const float* sc2 = p.scale_b2 + (long long)ti.group * p.N;
+          bf16* o = reinterpret_cast<bf16*>(p.out) + (long long)m * p.ldo;
+#pragma unroll 1
+          for (int j = half; j < BN / 64; j += 2) {
+            float g[32], u[32];
+            tmem_ld32(tl + j * 32, g);
+            tmem_ld32(tl + BN / 2 + j * 32, u);
+            tmem_wait_ld();
+            if (m < ti.m_end) {
+              const int n = ti.n0 + j * 32;
+              scale32(g, sc, n, p.N);
+              scale32(u, sc2, n, p.N);
+#pragma unroll
+              for (int c = 0; c < 32; c += 8) {
+                float w[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) w[i] = silu(g[c + i]) * u[c + i];
+                if (n + c + 8 <= p.N) {
+                  store_bf16x8(o + n + c, w);
+                } else {
+#pragma unroll
+                  for (int i = 0; i < 8; ++i)
+                    if (n + c + i < p.N) o[n + c + i] = __float2bfloat16_rn(w[i]);
+                }
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty0 + 8 * buf);
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Few routed rows per expert (decode batches): weights on the M side.
+//
+//   D[f, m] = sum_k w[g, f, k] * A[m, k]  for 128 weight rows f and BNT rows m
+//
+// The widened weight tile is the MMA's A operand and a BNT-row activation tile
+// its B operand (M = 128, N = BNT), so the tensor core does no work for empty
+// rows and the shared memory goes to a deep ring of code tiles: this mode is
+// bound by streaming the codes from HBM.  Code tiles are 128 codes deep
+// (128-byte rows, 128-byte swizzle): TMA moves whole 128-byte lines, and each
+// ring stage feeds two 64-deep MMA steps.  The epilogue writes the transpose
+// (consecutive lanes are consecutive weight rows, so stores stay coalesced).
+// SwiGLU holds the gate and up rows f in two accumulators.
+constexpr int I8T_BNT = 32;
+constexpr int I8T_EPI_WARPS = 4;   // one per TMEM lane quarter: a 32-token tile is one chunk
+constexpr int I8T_DQ_WARPS = 8;    // two per SM sub-partition, to hide the widening's latency
+static_assert(2 + I8T_EPI_WARPS + I8T_DQ_WARPS == I8W_THREADS / 32, "warp roles");
+
+template <int EPI>
+struct I8tSmem {
+  static constexpr int QROWS = EPI == EPI_SWIGLU ? 256 : 128;     // gate + up, or down rows
+  static constexpr uint32_t X_SUB = I8T_BNT * 128;                  // BNT x 64 bf16 activations
+  static constexpr uint32_t X_BYTES = 2 * X_SUB;                    // two 64-deep steps per stage
+  static constexpr uint32_t Q_BYTES = QROWS * 128;                  // QROWS x 128 codes
+  static constexpr uint32_t T_STAGE = X_BYTES + Q_BYTES;            // a multiple of 1024
+  static constexpr int TSTAGES = EPI == EPI_SWIGLU ? 4 : 6;
+  static constexpr int BSTAGES = 2;
+  static constexpr uint32_t B_BYTES = QROWS * 128;                  // QROWS x 64 bf16 widened
+  static constexpr uint32_t B_OFF = TSTAGES * T_STAGE;
+  static constexpr uint32_t BAR_OFF = B_OFF + BSTAGES * B_BYTES;
+  static constexpr uint32_t BYTES = BAR_OFF + 256 + 1024;
+  static constexpr int ACC = EPI == EPI_SWIGLU ? 2 * I8T_BNT : I8T_BNT;   // TMEM columns per buffer
+  static constexpr uint32_t TMEM_COLS = 2 * ACC <= 32 ? 32 : 2 * ACC <= 64 ? 64 : 128;
+};
+
+// Codes h*64 .. h*64+63 of ROWS rows stored as 128-byte rows under the
+// 128-byte swizzle -> ROWS x 64 bf16 (swizzled K-major).  A quarter-warp
+// takes the rows pi and pi ^ 5 of an 8-row group (pi < 4): their loads fall
+// in opposite halves of the swizzled row and their stores in chunks of
+// opposite parity, so neither side has bank conflicts.
+template <int ROWS, int DQ_WARPS>
+__device__ __forceinline__ void widen_tile_sw(const uint8_t* qs, int h, uint8_t* bdst, int ct) {
+  constexpr int PER = 32 * DQ_WARPS;
+  static_assert((ROWS * 4) % PER == 0, "whole iterations");
+#pragma unroll
+  for (int i = 0; i < ROWS * 4 / PER; ++i) {
+    const int idx = ct + PER * i;
+    const int g = idx & 3, sel = (idx >> 2) & 1, pi = (idx >> 3) & 3;
+    const int row = (idx >> 5) * 8 + (sel ? (pi ^ 5) : pi);
+    uint4 lo, hi;
+    widen16(*reinterpret_cast<const uint4*>(qs + row * 128 + (((4 * h + g) ^ (row & 7)) << 4)), lo, hi);
+    *reinterpret_cast<uint4*>(bdst + row * 128 + (((2 * g) ^ (row & 7)) << 4)) = lo;
+    *reinterpret_cast<uint4*>(bdst + row * 128 + (((2 * g + 1) ^ (row & 7)) << 4)) = hi;
+  }
+}
+
+// tile t -> (group, token rows m0.. clipped at m_end, weight rows n0..n0+127)
+__device__ __forceinline__ int total_tiles_tok(const GemmParams& p) {
+  int tot = 0;
+  for (int g = 0; g < p.num_groups; ++g) {
+    const int cnt = __ldg(p.offsets + g + 1) - __ldg(p.offsets + g);
+    tot += ((cnt + I8T_BNT - 1) / I8T_BNT) * p.n_tiles;
+  }
+  return tot;
+}
+__device__ __forceinline__ void decode_tile_tok(const GemmParams& p, int t, TileInfo& ti) {
+  for (int g = 0; g < p.num_groups; ++g) {
+    const int o0 = __ldg(p.offsets + g), o1 = __ldg(p.offsets + g + 1);
+    const int nt = (o1 - o0 + I8T_BNT - 1) / I8T_BNT;
+    const int tg = nt * p.n_tiles;
+    if (t < tg) {
+      const int tb = t % nt, wb = t / nt;   // token tiles of one weight tile are neighbours
+      ti.m0 = o0 + tb * I8T_BNT;
+      ti.m_end = o1;
+      ti.n0 = wb * 128;
+      ti.kt0 = 0;
+      ti.kt1 = p.k_tiles;                   // 64-deep steps, an even number here
+      ti.group = g;
+      ti.split = 0;
+      return;
+    }
+    t -= tg;
+  }
+  ti.m0 = ti.m_end = ti.n0 = ti.kt0 = ti.kt1 = ti.group = ti.split = 0;
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(I8W_THREADS, 1)
+gemm_i8w_tok_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmQ,
+                    const __grid_constant__ CUtensorMap tmQ2, const GemmParams p) {
+  static_assert(EPI == EPI_SWIGLU || EPI == EPI_F32, "expert GEMMs only");
+  using S = I8tSmem<EPI>;
+  constexpr int BNT = I8T_BNT;
+  constexpr int TST = S::TSTAGES;
+  constexpr int BST = S::BSTAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sB = smem + S::B_OFF;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::BAR_OFF);
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + TST);
+  const uint32_t bfull0 = smem_u32(bars + 2 * TST);
+  const uint32_t bempty0 = smem_u32(bars + 2 * TST + BST);
+  const uint32_t tfull0 = smem_u32(bars + 2 * TST + 2 * BST);
+  const uint32_t tempty0 = tfull0 + 16;
+  const uint32_t drain = tfull0 + 32;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * TST + 2 * BST + 5);
+  static_assert(8 * (2 * TST + 2 * BST + 6) <= 256, "barrier slots");
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < TST; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int s = 0; s < BST; ++s) {
+      mbar_init(bfull0 + 8 * s, I8T_DQ_WARPS);
+      mbar_init(bempty0 + 8 * s, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(tfull0 + 8 * i, 1);
+      mbar_init(tempty0 + 8 * i, I8T_EPI_WARPS);
+    }
+    mbar_init(drain, 1);
+    mbar_fence_init();
+    tma_prefetch(&tmA);
+    tma_prefetch(&tmQ);
+    if (EPI == EPI_SWIGLU) tma_prefetch(&tmQ2);
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_holder), S::TMEM_COLS);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_holder;
+  griddep_launch();
+  griddep_wait();
+  const int ntiles = total_tiles_tok(p);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        TileInfo ti;
+        decode_tile_tok(p, t, ti);
+        for (int kt = ti.kt0; kt < ti.kt1; kt += 2) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, p.err)) { ok = false; break; }
+          const uint32_t fb = full0 + 8 * stage;
+          const uint32_t st = smem_u32(smem + stage * S::T_STAGE);
+          mbar_arrive_tx(fb, S::T_STAGE);
+          tma_load_2d(st, &tmA, fb, kt * 64, ti.m0);
+          tma_load_2d(st + S::X_SUB, &tmA, fb, kt * 64 + 64, ti.m0);
+          tma_load_3d(st + S::X_BYTES, &tmQ, fb, kt * 64, ti.n0, ti.group);
+          if constexpr (EPI == EPI_SWIGLU)
+            tma_load_3d(st + S::X_BYTES + 128 * 128, &tmQ2, fb, kt * 64, ti.n0, ti.group);
+          if (++stage == TST) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_bf16(128, BNT);
+      int ts = 0, bs = 0;
+      uint32_t tph = 0, bph = 0;
+      bool ok = true;
+      int it = 0;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++it) {
+        TileInfo ti;
+        decode_tile_tok(p, t, ti);
+        const int buf = it & 1;
+        const uint32_t use = (uint32_t)(it >> 1);
+        if (!mbar_wait(tempty0 + 8 * buf, (use & 1) ^ 1, p.err)) break;
+        tc_fence_after();
+        const uint32_t d0 = tbase + buf * S::ACC;
+        for (int kt = ti.kt0; kt < ti.kt1 && ok; kt += 2) {
+          if (!mbar_wait(full0 + 8 * ts, tph, p.err)) { ok = false; break; }
+          for (int h = 0; h < 2; ++h) {
+            if (!mbar_wait(bfull0 + 8 * bs, bph, p.err)) { ok = false; break; }
+            tc_fence_after();
+            const uint64_t xd = sw128_desc(smem_u32(smem + ts * S::T_STAGE + h * S::X_SUB));
+            const uint64_t wd = sw128_desc(smem_u32(sB + bs * S::B_BYTES));
+            const uint32_t acc0 = (kt > ti.kt0 || h > 0) ? 1u : 0u;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) umma_bf16(d0, wd + 2 * kk, xd + 2 * kk, IDESC, (acc0 || kk > 0) ? 1u : 0u);
+            if constexpr (EPI == EPI_SWIGLU) {
+              const uint64_t ud = sw128_desc(smem_u32(sB + bs * S::B_BYTES + 128 * 128));
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                umma_bf16(d0 + BNT, ud + 2 * kk, xd + 2 * kk, IDESC, (acc0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(bempty0 + 8 * bs);
+            if (++bs == BST) { bs = 0; bph ^= 1; }
+          }
+          if (!ok) break;
+          umma_commit(empty0 + 8 * ts);
+          if (++ts == TST) { ts = 0; tph ^= 1; }
+        }
+        if (!ok) break;
+        umma_commit(tfull0 + 8 * buf);
+      }
+      umma_commit(drain);
+      mbar_wait(drain, 0, p.err);
+    }
+  } else if (warp >= 2 + I8T_EPI_WARPS) {
+    const int ct = threadIdx.x - 32 * (2 + I8T_EPI_WARPS);
+    int ts = 0, bs = 0;
+    uint32_t tph = 0, bph = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+      TileInfo ti;
+      decode_tile_tok(p, t, ti);
+      for (int kt = ti.kt0; kt < ti.kt1 && ok; kt += 2) {
+        if (!mbar_wait(full0 + 8 * ts, tph, p.err)) { ok = false; break; }
+        for (int h = 0; h < 2; ++h) {
+          if (!mbar_wait(bempty0 + 8 * bs, bph ^ 1, p.err)) { ok = false; break; }
+          widen_tile_sw<S::QROWS, I8T_DQ_WARPS>(smem + ts * S::T_STAGE + S::X_BYTES, h, sB + bs * S::B_BYTES, ct);
+          fence_async_shared();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bfull0 + 8 * bs);
+          if (++bs == BST) { bs = 0; bph ^= 1; }
+        }
+        if (++ts == TST) { ts = 0; tph ^= 1; }
+      }
+    }
+  } else {
+    const int q = warp & 3;                // warps 2-5: TMEM lane quarters 2, 3, 0, 1
+    int it = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
+      TileInfo ti;
+      decode_tile_tok(p, t, ti);
+      const int buf = it & 1;
+      const uint32_t use = (uint32_t)(it >> 1);
+      if (!mbar_wait(tfull0 + 8 * buf, use & 1, p.err)) break;
+      tc_fence_after();
+      const int f = ti.n0 + q * 32 + lane;   // weight row (output column); N is a multiple of 128
+      const uint32_t tl = tbase + ((uint32_t)(q * 32) << 16) + buf * S::ACC;
+      const float s1 = __ldg(p.scale_b + (long long)ti.group * p.N + f);
+#pragma unroll 1
+      for (int j = 0; j < BNT / 32; ++j) {
+        float v[32];
+        tmem_ld32(tl + j * 32, v);
+        if constexpr (EPI == EPI_SWIGLU) {
+          float u[32];
+          tmem_ld32(tl + BNT + j * 32, u);
+          tmem_wait_ld();
+          const float s2 = __ldg(p.scale_b2 + (long long)ti.group * p.N + f);
+          bf16* o = reinterpret_cast<bf16*>(p.out) + f;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const int m = ti.m0 + j * 32 + c;
+            if (m < ti.m_end) o[(long long)m * p.ldo] = __float2bfloat16_rn(silu(v[c] * s1) * (u[c] * s2));
+          }
+        } else {
+          tmem_wait_ld();
+          float* o = reinterpret_cast<float*>(p.out) + f;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const int m = ti.m0 + j * 32 + c;
+            if (m < ti.m_end) o[(long long)m * p.ldo] = v[c] * s1;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty0 + 8 * buf);
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, S::TMEM_COLS);
+  }
+}
+
+}  // namespace jb

@@ -10,12 +10,6 @@
 //   warps 2-9  epilogue: two warps per 32-lane TMEM quarter, splitting the
 //              32-column chunks between them; tcgen05.ld, fused elementwise
 //              op, stores to global memory.
-//   warps 10-13 (INT8 weights only) dequantisers: the producer lands the
-//              BN x 64 tile of 8-bit codes in its own ring slot; these warps
-//              widen it to bf16 in the 128-byte-swizzled layout the MMA reads
-//              and signal a third barrier.  The per-row scales of the codes
-//              are applied to the fp32 accumulators in the epilogue, so the
-//              product is exact up to fp32 accumulation order.
 // The epilogue kind is a template parameter, so each instantiation carries
 // only its own epilogue code.  Used for in_proj, x_proj, dt_proj
 // (+bias+softplus), out_proj (+residual), the decode projections (swap-AB:
@@ -31,8 +25,6 @@ enum EpiKind : int { EPI_BF16 = 0, EPI_F32 = 1, EPI_SOFTPLUS = 2, EPI_SWIGLU = 3
 
 constexpr int GEMM_THREADS = 320;
 constexpr int GEMM_EPI_WARPS = 8;
-constexpr int GEMM_DQ_WARPS = 4;   // INT8-weight dequantisers
-__host__ __device__ constexpr int gemm_threads(bool qb) { return GEMM_THREADS + (qb ? 32 * GEMM_DQ_WARPS : 0); }
 
 struct GemmParams {
   int M, N, K;           // N counts output columns (SwiGLU: d_ff)
@@ -47,8 +39,8 @@ struct GemmParams {
   const void* residual;  // bf16, same layout as out (non-transposed only)
   long long ldr;
   const float* bias;     // indexed by n (or by m when transposed)
-  const float* scale_b;  // INT8 B: per-row scales [groups, N] (SwiGLU: of the gate rows)
-  const float* scale_b2; // INT8 B, SwiGLU: scales of the up rows
+  const float* scale_b;  // INT8 weights: per-row scales [groups, N] (SwiGLU: of the gate rows)
+  const float* scale_b2; // INT8 weights, SwiGLU: scales of the up rows
   int* err;
 };
 
@@ -240,48 +232,41 @@ __device__ __forceinline__ void epi_chunk(const GemmParams& p, const TileInfo& t
   }
 }
 
-template <int BN, int STAGES, bool STAGED = false, bool QB = false>
+template <int BN, int STAGES, bool STAGED = false>
 struct GemmSmem {
   static constexpr uint32_t A_BYTES = 128 * 128;
   static constexpr uint32_t B_BYTES = BN * 128;
-  static constexpr uint32_t Q_BYTES = QB ? BN * 64 : 0;   // INT8 codes of the B tile
   // STAGED: per epilogue warp two 32 x 32 fp32 boxes for TMA stores (1024-aligned)
-  static constexpr uint32_t STG_OFF = STAGES * (A_BYTES + B_BYTES + Q_BYTES);
+  static constexpr uint32_t STG_OFF = STAGES * (A_BYTES + B_BYTES);
   static constexpr uint32_t STG_BYTES = STAGED ? GEMM_EPI_WARPS * 2 * 4096 : 0;
   static constexpr uint32_t BAR_OFF = STG_OFF + STG_BYTES;
-  // barrier slots: full[STAGES], empty[STAGES], tmem_full[2], tmem_empty[2], drain, tmem holder,
-  // INT8 B: b_ready[STAGES]
-  static_assert(8 * (3 * STAGES + 6) <= 256, "barrier slots");
+  // barrier slots: full[STAGES], empty[STAGES], tmem_full[2], tmem_empty[2], drain, tmem holder
+  static_assert(8 * (2 * STAGES + 6) <= 256, "barrier slots");
   static constexpr uint32_t BYTES = BAR_OFF + 256 + 1024;  // + barriers + alignment slack
   static constexpr uint32_t TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
                                         : (2 * BN <= 256) ? 256 : 512;
 };
 
-template <int BN, int STAGES, int EPI, bool TRANS, bool QB = false>
-__global__ void __launch_bounds__(gemm_threads(QB), 1)
+template <int BN, int STAGES, int EPI, bool TRANS>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmC,
                     const GemmParams p) {
   // fp32 softplus outputs (dt) leave through shared memory and TMA stores
   constexpr bool STAGED = EPI == EPI_SOFTPLUS && !TRANS;
-  using S = GemmSmem<BN, STAGES, STAGED, QB>;
+  using S = GemmSmem<BN, STAGES, STAGED>;
   static_assert(BN % 16 == 0 && BN >= 32 && BN <= 256, "UMMA N for M = 128");
-  static_assert(!QB || (!TRANS && !STAGED && (EPI == EPI_SWIGLU || EPI == EPI_F32) && BN % 32 == 0),
-                "INT8 B: grouped expert GEMMs only");
   constexpr int BN_OUT = EPI == EPI_SWIGLU ? BN / 2 : BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * S::A_BYTES;
-  uint8_t* sQ = sB + STAGES * S::B_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::BAR_OFF);
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES);
   const uint32_t tfull0 = smem_u32(bars + 2 * STAGES), tempty0 = smem_u32(bars + 2 * STAGES + 2);
   const uint32_t drain = smem_u32(bars + 2 * STAGES + 4);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
-  const uint32_t bready0 = smem_u32(bars + 2 * STAGES + 6);
-  // bytes the producer's TMA loads land per stage
-  constexpr uint32_t STAGE_TX = S::A_BYTES + (QB ? S::Q_BYTES : S::B_BYTES);
+  constexpr uint32_t STAGE_TX = S::A_BYTES + S::B_BYTES;   // bytes the TMA loads land per stage
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp == 0 && lane == 0) {
@@ -294,8 +279,6 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       mbar_init(tempty0 + 8 * i, GEMM_EPI_WARPS);
     }
     mbar_init(drain, 1);
-    if (QB)
-      for (int st = 0; st < STAGES; ++st) mbar_init(bready0 + 8 * st, GEMM_DQ_WARPS);
     mbar_fence_init();
     tma_prefetch(&tmA);
     tma_prefetch(&tmB);
@@ -342,15 +325,7 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             mbar_arrive_tx(fb, STAGE_TX);
             tma_load_2d(a_dst, &tmA, fb, kt * 64, ti.m0);
           }
-          if constexpr (QB) {
-            const uint32_t q_dst = smem_u32(sQ + stage * S::Q_BYTES);
-            if constexpr (EPI == EPI_SWIGLU) {
-              tma_load_3d(q_dst, &tmB, fb, kt * 64, ti.n0, ti.group);
-              tma_load_3d(q_dst + (BN / 2) * 64, &tmB2, fb, kt * 64, ti.n0, ti.group);
-            } else {
-              tma_load_3d(q_dst, &tmB, fb, kt * 64, ti.n0, ti.group);
-            }
-          } else if (!p.grouped) {
+          if (!p.grouped) {
             tma_load_2d(b_dst, &tmB, fb, kt * 64, ti.n0);
           } else if (EPI != EPI_SWIGLU) {
             tma_load_3d(b_dst, &tmB, fb, kt * 64, ti.n0, ti.group);
@@ -381,7 +356,6 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         const uint32_t d_tmem = tbase + acc * BN;
         for (int kt = ti.kt0; kt < ti.kt1; ++kt) {
           if (!mbar_wait(full0 + 8 * stage, phase, p.err)) { ok = false; break; }
-          if (QB && !mbar_wait(bready0 + 8 * stage, phase, p.err)) { ok = false; break; }
           tc_fence_after();
           const uint64_t ad = sw128_desc(smem_u32(sA + stage * S::A_BYTES));
           const uint64_t bd = sw128_desc(smem_u32(sB + stage * S::B_BYTES));
@@ -397,39 +371,6 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       // drain: no MMA may still be writing TMEM when the CTA frees it
       umma_commit(drain);
       mbar_wait(drain, 0, p.err);
-    }
-  } else if (QB && warp >= 2 + GEMM_EPI_WARPS) {
-    // INT8 dequantisers: ring slot `stage` holds the BN x 64 codes, row-major
-    // with 64-byte rows; 16 codes (one 16-byte load) become two 16-byte bf16
-    // chunks of the same row, placed by the 128-byte swizzle.  A quarter-warp
-    // covers two rows, so its eight stores hit eight distinct chunks.
-    griddep_wait();
-    const int ntiles = total_tiles(p);
-    const int ct = threadIdx.x - 32 * (2 + GEMM_EPI_WARPS);
-    int stage = 0;
-    uint32_t phase = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-      TileInfo ti;
-      decode_tile<BN_OUT>(p, t, ti);
-      for (int kt = ti.kt0; kt < ti.kt1; ++kt) {
-        if (!mbar_wait(full0 + 8 * stage, phase, p.err)) { ok = false; break; }
-        const uint8_t* qs = sQ + stage * S::Q_BYTES;
-        uint8_t* bs = sB + stage * S::B_BYTES;
-#pragma unroll
-        for (int i = 0; i < BN / 32; ++i) {
-          const int idx = ct + 32 * GEMM_DQ_WARPS * i;
-          const int row = idx >> 2, g = idx & 3;
-          uint4 lo, hi;
-          i8x16_to_bf16(*reinterpret_cast<const uint4*>(qs + idx * 16), lo, hi);
-          *reinterpret_cast<uint4*>(bs + row * 128 + (((2 * g) ^ (row & 7)) << 4)) = lo;
-          *reinterpret_cast<uint4*>(bs + row * 128 + (((2 * g + 1) ^ (row & 7)) << 4)) = hi;
-        }
-        fence_async_shared();   // the tensor core reads these stores through the async proxy
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bready0 + 8 * stage);
-        if (++stage == STAGES) { stage = 0; phase ^= 1; }
-      }
     }
   } else {
     griddep_wait();
@@ -490,7 +431,6 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           float v[32];
           tmem_ld32(tl + j * 32, v);
           tmem_wait_ld();
-          if constexpr (QB) scale32(v, p.scale_b + (long long)ti.group * p.N, ti.n0 + j * 32, p.N);
           epi_chunk<EPI, TRANS, 32>(p, ti, m, ti.n0 + j * 32, v);
         }
         if constexpr (BN % 32 != 0) {
@@ -511,10 +451,6 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           tmem_wait_ld();
           if (m < ti.m_end) {
             const int n = ti.n0 + j * 32;
-            if constexpr (QB) {
-              scale32(g, p.scale_b + (long long)ti.group * p.N, n, p.N);
-              scale32(u, p.scale_b2 + (long long)ti.group * p.N, n, p.N);
-            }
 #pragma unroll
             for (int c = 0; c < 32; c += 8) {
               float w[8];

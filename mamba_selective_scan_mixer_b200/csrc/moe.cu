@@ -15,6 +15,28 @@ namespace jb {
 
 constexpr int ROUTER_EG = 16;  // experts per register group
 
+// softmax over the E logits of token t and its top K (descending logit, ties
+// to the lower index), probabilities not renormalised
+__device__ __forceinline__ void route_token(const double* logit, int E, int K, int t, int* __restrict__ idx_out,
+                                            float* __restrict__ w_out, int* __restrict__ counts) {
+  double mx = logit[0];
+  for (int e = 1; e < E; ++e) mx = logit[e] > mx ? logit[e] : mx;
+  double den = 0.0;
+  for (int e = 0; e < E; ++e) den += exp(logit[e] - mx);
+  unsigned long long taken = 0ull;
+  for (int k = 0; k < K; ++k) {
+    int best = -1;
+    for (int e = 0; e < E; ++e) {
+      if (taken >> e & 1ull) continue;
+      if (best < 0 || logit[e] > logit[best]) best = e;  // strict: ties keep the lower index
+    }
+    taken |= 1ull << best;
+    idx_out[(long long)t * K + k] = best;
+    w_out[(long long)t * K + k] = (float)(exp(logit[best] - mx) / den);
+    atomicAdd(counts + best, 1);
+  }
+}
+
 // one warp per token
 __global__ void __launch_bounds__(256)
 router_kernel(const bf16* __restrict__ x, const bf16* __restrict__ W, int T, int dm, int E, int K,
@@ -59,24 +81,65 @@ router_kernel(const bf16* __restrict__ x, const bf16* __restrict__ W, int T, int
         if (e0 + e < E) logit[e0 + e] = v;
       }
     }
-    if (lane == 0) {
-      double mx = logit[0];
-      for (int e = 1; e < E; ++e) mx = logit[e] > mx ? logit[e] : mx;
-      double den = 0.0;
-      for (int e = 0; e < E; ++e) den += exp(logit[e] - mx);
-      unsigned long long taken = 0ull;
-      for (int k = 0; k < K; ++k) {
-        int best = -1;
-        for (int e = 0; e < E; ++e) {
-          if (taken >> e & 1ull) continue;
-          if (best < 0 || logit[e] > logit[best]) best = e;  // strict: ties keep the lower index
+    if (lane == 0) route_token(logit, E, K, t, idx_out, w_out, counts);
+  }
+}
+
+// Few tokens: one block per token, the d_model sum split over 8 warps (each
+// its own slice, partials added in warp order), so the logits of a decode
+// batch take a few microseconds instead of one warp's serial fp64 chain.
+__global__ void __launch_bounds__(256)
+router_split_kernel(const bf16* __restrict__ x, const bf16* __restrict__ W, int dm, int E, int K,
+                    int* __restrict__ idx_out, float* __restrict__ w_out, int* __restrict__ counts) {
+  __shared__ double part[8][64];
+  __shared__ double logit[64];
+  const int t = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int slice = dm / 8;   // a multiple of 32
+  const bf16* xr = x + (long long)t * dm;
+  for (int e0 = 0; e0 < E; e0 += ROUTER_EG) {
+    double acc[ROUTER_EG];
+#pragma unroll
+    for (int e = 0; e < ROUTER_EG; ++e) acc[e] = 0.0;
+    for (int k0 = warp * slice + lane * 8; k0 < (warp + 1) * slice; k0 += 256) {
+      const uint4 xv = *reinterpret_cast<const uint4*>(xr + k0);
+      const __nv_bfloat162* xh = reinterpret_cast<const __nv_bfloat162*>(&xv);
+      float xf[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(xh[i]);
+        xf[2 * i] = f.x;
+        xf[2 * i + 1] = f.y;
+      }
+#pragma unroll
+      for (int e = 0; e < ROUTER_EG; ++e) {
+        if (e0 + e >= E) break;
+        const uint4 wv = __ldg(reinterpret_cast<const uint4*>(W + (long long)(e0 + e) * dm + k0));
+        const __nv_bfloat162* wh = reinterpret_cast<const __nv_bfloat162*>(&wv);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __bfloat1622float2(wh[i]);
+          acc[e] += (double)(xf[2 * i] * f.x);      // exact product of two bf16 values
+          acc[e] += (double)(xf[2 * i + 1] * f.y);
         }
-        taken |= 1ull << best;
-        idx_out[(long long)t * K + k] = best;
-        w_out[(long long)t * K + k] = (float)(exp(logit[best] - mx) / den);
-        atomicAdd(counts + best, 1);
       }
     }
+#pragma unroll
+    for (int e = 0; e < ROUTER_EG; ++e) {
+      double v = acc[e];
+#pragma unroll
+      for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0 && e0 + e < E) part[warp][e0 + e] = v;
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    for (int e = lane; e < E; e += 32) {
+      double v = part[0][e];
+      for (int w = 1; w < 8; ++w) v += part[w][e];
+      logit[e] = v;
+    }
+    __syncwarp();
+    if (lane == 0) route_token(logit, E, K, t, idx_out, w_out, counts);
   }
 }
 
@@ -243,11 +306,16 @@ jamba_status quantize_int8_rows(const void* w, int dtype, long long rows, int co
 jamba_status moe_route(const void* x, const void* W, int T, int dm, int E, int K, int* idx, float* w, int* counts,
                        int* offsets, int* perm, int* inv, cudaStream_t s) {
   JB_CUDA(cudaMemsetAsync(counts, 0, sizeof(int) * E, s));
-  int blocks = (T + 7) / 8;
-  const int cap = 8 * num_sms();
-  if (blocks > cap) blocks = cap;
-  router_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const bf16*>(x), reinterpret_cast<const bf16*>(W), T, dm, E,
-                                       K, idx, w, counts);
+  if (T <= 4096) {
+    router_split_kernel<<<T, 256, 0, s>>>(reinterpret_cast<const bf16*>(x), reinterpret_cast<const bf16*>(W), dm, E,
+                                          K, idx, w, counts);
+  } else {
+    int blocks = (T + 7) / 8;
+    const int cap = 8 * num_sms();
+    if (blocks > cap) blocks = cap;
+    router_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const bf16*>(x), reinterpret_cast<const bf16*>(W), T, dm,
+                                         E, K, idx, w, counts);
+  }
   JB_CUDA(cudaGetLastError());
   permute_kernel<<<E, 1024, 0, s>>>(idx, T * K, E, counts, offsets, perm, inv);
   JB_CUDA(cudaGetLastError());

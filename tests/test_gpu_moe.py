@@ -142,11 +142,17 @@ def test_quantize_int8_rows_bit_exact(dev, dtype):
 
 @pytest.mark.parametrize("T,dm,dff,residual,top_k", [(1000, 512, 384, False, 2), (333, 256, 640, True, 2),
                                                      (1024, 4096, 1024, True, 2), (5, 256, 128, False, 2),
-                                                     (257, 512, 256, True, 1)])
+                                                     (257, 512, 256, True, 1), (256, 512, 384, True, 2),
+                                                     (3000, 512, 384, True, 2), (4100, 256, 256, False, 1)])
 def test_moe_int8_forward(dev, T, dm, dff, residual, top_k):
     """ExpertsInt8 MoE vs the oracle MoE on the dequantised weights q * s;
     the codes and scales themselves bit-exact.  T = 5 leaves most experts
-    without rows; expert 0's gate and one down row are all zero (s = 0)."""
+    without rows; expert 0's gate and one down row are all zero (s = 0).
+    Up to 32 routed rows per expert on average (T = 5, 257 with K = 1, 256)
+    the weights take the M side, with experts spilling into a second
+    32-row token tile at T = 256; from 256 rows per expert (T = 3000, 4100)
+    the kernel pairs 128-row halves on one widened weight tile, with ragged
+    second halves and tiles whose second half is empty."""
     import mamba_selective_scan_mixer_b200 as J
     shape = MoEShape(d_model=dm, d_ff=dff, n_experts=E, top_k=top_k)
     seed = 100 + T + dff
@@ -167,16 +173,15 @@ def test_moe_int8_forward(dev, T, dm, dff, residual, top_k):
     assert rel_l2(to_np(r["out"]), want["out"]) < TOL_BF16
 
 
-def test_moe_int8_full_size_sampled(dev):
-    """d_model 4096, d_ff 14336, 16 experts, top-2, 32768 tokens (the layer
-    pair's MoE) with INT8 experts: every router decision and the codes of
-    the sampled tokens' experts bit-exact, 48 sampled tokens' outputs within
-    the bf16 bar (the oracle dequantises one expert at a time)."""
+def _int8_full_width_check(dev, T, n_sample, seed):
+    """MoE at d_model 4096, d_ff 14336, 16 experts, top-2 with INT8 experts:
+    every router decision and the codes of the sampled tokens' experts
+    bit-exact, the sampled tokens' outputs within the bf16 bar (the oracle
+    dequantises one expert at a time)."""
     import mamba_selective_scan_mixer_b200 as J
     shape = MoEShape()
-    T = 32768
-    p = moe_params(shape, seed=11, device=dev)
-    x = moe_input(shape, T, seed=11, device=dev)
+    p = moe_params(shape, seed=seed, device=dev)
+    x = moe_input(shape, T, seed=seed, device=dev)
     pq = J.quantize_experts_int8(p)
     moe = J.MoE(pq, shape)
     r = moe.forward(x)
@@ -185,8 +190,8 @@ def test_moe_int8_full_size_sampled(dev):
     idx, w, logits = omoe.router(xs, to_np(p["router"]), shape.top_k)
     assert len(_near_ties(logits, shape.top_k)) == 0
     np.testing.assert_array_equal(r["idx"].cpu().numpy(), idx)
-    rng = np.random.default_rng(12)
-    tok = np.sort(rng.choice(T, 48, replace=False))
+    rng = np.random.default_rng(seed + 1)
+    tok = np.sort(rng.choice(T, n_sample, replace=False))
     got = to_np(r["out"][torch.as_tensor(tok, device=dev)])
     want = np.zeros((len(tok), shape.d_model))
     for e in np.unique(idx[tok]):
@@ -199,3 +204,13 @@ def test_moe_int8_full_size_sampled(dev):
             m = slots == k
             want[rows[m]] += w[tok[rows[m]], k][:, None] * ye[m]
     assert rel_l2(got, want) < TOL_BF16
+
+
+def test_moe_int8_full_size_sampled(dev):
+    """The layer pair's MoE (32768 tokens, paired 128-row halves): 48 sampled tokens."""
+    _int8_full_width_check(dev, 32768, 48, seed=11)
+
+
+def test_moe_int8_decode_batch_full_width(dev):
+    """A 64-token decode batch at full width (weights on the M side): every token."""
+    _int8_full_width_check(dev, 64, 64, seed=13)
