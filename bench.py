@@ -46,7 +46,8 @@ def parse():
     ap.add_argument("--impl", default="product", choices=["product", "reference"])
     ap.add_argument("--quick", action="store_true", help="skip the side measurements")
     ap.add_argument("--only", default="all",
-                    help="comma list of parts to run (prefill,gemm,scan,decode,pair,moe8,e2e,cpu); for profiling")
+                    help="comma list of parts to run (prefill,gemm,scan,decode,pair,moe8,moe8dec,e2e,cpu); "
+                         "for profiling")
     ap.add_argument("--seqlen", type=int, default=PREFILL_L, help="prefill tokens")
     ap.add_argument("--scan-seqlen", type=int, default=SCAN_L)
     ap.add_argument("--decode-steps", type=int, default=DECODE_STEPS)
@@ -387,9 +388,34 @@ def run_product(args):
                 "moe_64_tokens_us": {"bf16": round(1e3 * moe_t[("bf16", 64)], 1),
                                      "int8": round(1e3 * moe_t[("int8", 64)], 1)},
                 "moe_64_tokens_weight_GB/s": {"bf16": round(wb16 / (moe_t[("bf16", 64)] / 1e3) / 1e9, 1),
-                                              "int8": round(wb8 / (moe_t[("int8", 64)] / 1e3) / 1e9, 1)}}
+                                              "int8": round(wb8 / (moe_t[("int8", 64)] / 1e3) / 1e9, 1)},
+                "moe_64_tokens_int8_frac_of_measured_hbm": round(wb8 / (moe_t[("int8", 64)] / 1e3) / 1e9 / pk["hbm"], 4)}
             del pq, moe8
         del mp, moe, xp
+        J.device_status()
+
+    if rank == 0 and "moe8dec" in parts:
+        # ExpertsInt8 decode batch alone, with only the int8 experts resident (a few GB): the
+        # small case the expert-kernel profiles are taken on
+        es = MoEShape()
+        mp = moe_params(es, seed=0, device=dev)
+        pq = J.quantize_experts_int8(mp)
+        del mp
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        moe8 = J.MoE(pq, es)
+        v = moe_input(es, 64, seed=3, device=dev)
+        f = lambda: moe8.forward(v)
+        for _ in range(args.warmup):
+            f()
+        torch.cuda.synchronize()
+        dms, _ = event_time_ms(f, args.steps, stream, flush)
+        wb8 = sum(pq[k].numel() * pq[k].element_size() for k in ("w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down"))
+        res["moe_int8_decode"] = {"workload": "ExpertsInt8 MoE, 64 tokens, 16 experts top-2, d_model 4096, d_ff 14336",
+                                  "us": round(1e3 * dms, 1),
+                                  "weight_GB/s": round(wb8 / (dms / 1e3) / 1e9, 1),
+                                  "frac_of_measured_hbm": round(wb8 / (dms / 1e3) / 1e9 / pk["hbm"], 4)}
+        del pq, moe8
         J.device_status()
 
     # end to end through the public API with host buffers (pinned), copies inside the timed region

@@ -69,23 +69,42 @@ __device__ __forceinline__ void widen16(uint4 v, uint4& lo, uint4& hi) {
 }
 
 // ROWS x 64 codes (row-major, 64-byte rows) -> ROWS x 64 bf16 in the 128-byte
-// swizzled K-major layout, by the I8W_DQ_WARPS dequantiser warps (thread ct).
-// 16 codes per load become two 16-byte chunks of the same row; a quarter-warp
-// covers two rows and stores to eight distinct chunks (no bank conflicts).
+// swizzled K-major layout, by the I8W_DQ_WARPS dequantiser warps.  16 codes
+// per load become two 16-byte chunks of the same row; a quarter-warp covers
+// two rows and stores to eight distinct chunks (no bank conflicts).  The
+// offsets are the same for every stage and are worked out once.
 template <int ROWS>
-__device__ __forceinline__ void widen_tile(const uint8_t* qs, uint8_t* bdst, int ct) {
-  constexpr int PER = 32 * I8W_DQ_WARPS;
-  static_assert((ROWS * 4) % PER == 0, "whole iterations");
+struct WidenPlanLinear {
+  static constexpr int PER = 32 * I8W_DQ_WARPS;
+  static constexpr int IT = ROWS * 4 / PER;
+  static_assert(IT * PER == ROWS * 4, "whole iterations");
+  uint32_t dlo[IT], dhi[IT];
+  uint32_t src0;
+  __device__ __forceinline__ explicit WidenPlanLinear(int ct) {
+    src0 = ct * 16;
 #pragma unroll
-  for (int i = 0; i < ROWS * 4 / PER; ++i) {
-    const int idx = ct + PER * i;
-    const int row = idx >> 2, g = idx & 3;
-    uint4 lo, hi;
-    widen16(*reinterpret_cast<const uint4*>(qs + idx * 16), lo, hi);
-    *reinterpret_cast<uint4*>(bdst + row * 128 + (((2 * g) ^ (row & 7)) << 4)) = lo;
-    *reinterpret_cast<uint4*>(bdst + row * 128 + (((2 * g + 1) ^ (row & 7)) << 4)) = hi;
+    for (int i = 0; i < IT; ++i) {
+      const int idx = ct + PER * i;
+      const int row = idx >> 2, g = idx & 3;
+      dlo[i] = row * 128 + (((2 * g) ^ (row & 7)) << 4);
+      dhi[i] = row * 128 + (((2 * g + 1) ^ (row & 7)) << 4);
+    }
   }
-}
+  // q, b: shared-memory addresses of the code tile and the widened tile
+  __device__ __forceinline__ void run(uint32_t q, uint32_t b) const {
+#pragma unroll
+    for (int i = 0; i < IT; ++i) {
+      uint4 v, lo, hi;
+      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(q + src0 + PER * 16 * i));
+      widen16(v, lo, hi);
+      asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(b + dlo[i]), "r"(lo.x), "r"(lo.y), "r"(lo.z),
+                   "r"(lo.w) : "memory");
+      asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(b + dhi[i]), "r"(hi.x), "r"(hi.y), "r"(hi.z),
+                   "r"(hi.w) : "memory");
+    }
+  }
+};
 
 template <int MH>
 __device__ __forceinline__ int total_tiles_grouped(const GemmParams& p) {
@@ -243,7 +262,8 @@ gemm_i8w_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       mbar_wait(drain, 0, p.err);
     }
   } else if (warp >= 2 + GEMM_EPI_WARPS) {
-    const int ct = threadIdx.x - 32 * (2 + GEMM_EPI_WARPS);
+    const WidenPlanLinear<BN> plan(threadIdx.x - 32 * (2 + GEMM_EPI_WARPS));
+    const uint32_t qbase = smem_u32(smem + MT * S::A_BYTES), bbase = smem_u32(sB);
     int ts = 0, bs = 0;
     uint32_t tph = 0, bph = 0;
     bool ok = true;
@@ -253,7 +273,7 @@ gemm_i8w_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       for (int kt = ti.kt0; kt < ti.kt1; ++kt) {
         if (!mbar_wait(full0 + 8 * ts, tph, p.err)) { ok = false; break; }
         if (!mbar_wait(bempty0 + 8 * bs, bph ^ 1, p.err)) { ok = false; break; }
-        widen_tile<BN>(smem + ts * S::T_STAGE + MT * S::A_BYTES, sB + bs * S::B_BYTES, ct);
+        plan.run(qbase + ts * S::T_STAGE, bbase + bs * S::B_BYTES);
         fence_async_shared();   // the tensor core reads these stores through the async proxy
         __syncwarp();
         if (lane == 0) mbar_arrive(bfull0 + 8 * bs);
@@ -343,8 +363,8 @@ gemm_i8w_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 // SwiGLU holds the gate and up rows f in two accumulators.
 constexpr int I8T_BNT = 32;
 constexpr int I8T_EPI_WARPS = 4;   // one per TMEM lane quarter: a 32-token tile is one chunk
-constexpr int I8T_DQ_WARPS = 8;    // two per SM sub-partition, to hide the widening's latency
-static_assert(2 + I8T_EPI_WARPS + I8T_DQ_WARPS == I8W_THREADS / 32, "warp roles");
+constexpr int I8T_DQ_WARPS = 8;    // two per SM sub-partition
+constexpr int I8T_THREADS = 32 * (2 + I8T_EPI_WARPS + I8T_DQ_WARPS);
 
 template <int EPI>
 struct I8tSmem {
@@ -367,22 +387,41 @@ struct I8tSmem {
 // 128-byte swizzle -> ROWS x 64 bf16 (swizzled K-major).  A quarter-warp
 // takes the rows pi and pi ^ 5 of an 8-row group (pi < 4): their loads fall
 // in opposite halves of the swizzled row and their stores in chunks of
-// opposite parity, so neither side has bank conflicts.
+// opposite parity, so neither side has bank conflicts.  The byte offsets of a
+// thread's loads and stores are the same for every stage, so they are worked
+// out once (the second half's loads differ from the first's in bit 6 only).
 template <int ROWS, int DQ_WARPS>
-__device__ __forceinline__ void widen_tile_sw(const uint8_t* qs, int h, uint8_t* bdst, int ct) {
-  constexpr int PER = 32 * DQ_WARPS;
-  static_assert((ROWS * 4) % PER == 0, "whole iterations");
+struct WidenPlan {
+  static constexpr int IT = ROWS * 4 / (32 * DQ_WARPS);
+  static_assert(IT * 32 * DQ_WARPS == ROWS * 4, "whole iterations");
+  uint32_t src[IT], dlo[IT], dhi[IT];
+  __device__ __forceinline__ explicit WidenPlan(int ct) {
 #pragma unroll
-  for (int i = 0; i < ROWS * 4 / PER; ++i) {
-    const int idx = ct + PER * i;
-    const int g = idx & 3, sel = (idx >> 2) & 1, pi = (idx >> 3) & 3;
-    const int row = (idx >> 5) * 8 + (sel ? (pi ^ 5) : pi);
-    uint4 lo, hi;
-    widen16(*reinterpret_cast<const uint4*>(qs + row * 128 + (((4 * h + g) ^ (row & 7)) << 4)), lo, hi);
-    *reinterpret_cast<uint4*>(bdst + row * 128 + (((2 * g) ^ (row & 7)) << 4)) = lo;
-    *reinterpret_cast<uint4*>(bdst + row * 128 + (((2 * g + 1) ^ (row & 7)) << 4)) = hi;
+    for (int i = 0; i < IT; ++i) {
+      const int idx = ct + 32 * DQ_WARPS * i;
+      const int g = idx & 3, sel = (idx >> 2) & 1, pi = (idx >> 3) & 3;
+      const int row = (idx >> 5) * 8 + (sel ? (pi ^ 5) : pi);
+      src[i] = row * 128 + ((g ^ (row & 7)) << 4);
+      dlo[i] = row * 128 + (((2 * g) ^ (row & 7)) << 4);
+      dhi[i] = row * 128 + (((2 * g + 1) ^ (row & 7)) << 4);
+    }
   }
-}
+  // q, b: shared-memory addresses of the code tile and the widened tile
+  __device__ __forceinline__ void run(uint32_t q, int h, uint32_t b) const {
+    const uint32_t hx = (uint32_t)h << 6;
+#pragma unroll
+    for (int i = 0; i < IT; ++i) {
+      uint4 v, lo, hi;
+      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(q + (src[i] ^ hx)));
+      widen16(v, lo, hi);
+      asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(b + dlo[i]), "r"(lo.x), "r"(lo.y), "r"(lo.z),
+                   "r"(lo.w) : "memory");
+      asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(b + dhi[i]), "r"(hi.x), "r"(hi.y), "r"(hi.z),
+                   "r"(hi.w) : "memory");
+    }
+  }
+};
 
 // tile t -> (group, token rows m0.. clipped at m_end, weight rows n0..n0+127)
 __device__ __forceinline__ int total_tiles_tok(const GemmParams& p) {
@@ -415,7 +454,7 @@ __device__ __forceinline__ void decode_tile_tok(const GemmParams& p, int t, Tile
 }
 
 template <int EPI>
-__global__ void __launch_bounds__(I8W_THREADS, 1)
+__global__ void __launch_bounds__(I8T_THREADS, 1)
 gemm_i8w_tok_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmQ,
                     const __grid_constant__ CUtensorMap tmQ2, const GemmParams p) {
   static_assert(EPI == EPI_SWIGLU || EPI == EPI_F32, "expert GEMMs only");
@@ -531,7 +570,8 @@ gemm_i8w_tok_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       mbar_wait(drain, 0, p.err);
     }
   } else if (warp >= 2 + I8T_EPI_WARPS) {
-    const int ct = threadIdx.x - 32 * (2 + I8T_EPI_WARPS);
+    const WidenPlan<S::QROWS, I8T_DQ_WARPS> plan(threadIdx.x - 32 * (2 + I8T_EPI_WARPS));
+    const uint32_t qbase = smem_u32(smem + S::X_BYTES), bbase = smem_u32(sB);
     int ts = 0, bs = 0;
     uint32_t tph = 0, bph = 0;
     bool ok = true;
@@ -542,7 +582,7 @@ gemm_i8w_tok_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         if (!mbar_wait(full0 + 8 * ts, tph, p.err)) { ok = false; break; }
         for (int h = 0; h < 2; ++h) {
           if (!mbar_wait(bempty0 + 8 * bs, bph ^ 1, p.err)) { ok = false; break; }
-          widen_tile_sw<S::QROWS, I8T_DQ_WARPS>(smem + ts * S::T_STAGE + S::X_BYTES, h, sB + bs * S::B_BYTES, ct);
+          plan.run(qbase + ts * S::T_STAGE, h, bbase + bs * S::B_BYTES);
           fence_async_shared();
           __syncwarp();
           if (lane == 0) mbar_arrive(bfull0 + 8 * bs);
