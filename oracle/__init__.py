@@ -25,4 +25,4 @@ Sources (titles and sections of the pages the method is taken from):
 
 Parity status per function is listed in each module header.
 """
-from . import mamba, moe  # noqa: F401
+from . import attention, mamba, moe  # noqa: F401

@@ -17,6 +17,9 @@ workload stores bf16):
   fp32; A[c, n] = -(n + 1); D = 1.
 * MoE: router [E, d_model], gate and up [E, d_ff, d_model], down
   [E, d_model, d_ff], all N(0, 0.02); input ~ N(0, 1).
+* Attention: wq [n_heads*head_dim, d_model], wk and wv
+  [n_kv_heads*head_dim, d_model], wo [d_model, n_heads*head_dim], all
+  N(0, 0.02); input ~ N(0, 1).
 
 dt_bias and the softplus of the scan-only dt are part of the input recipe
 (how the benchmark initialises its tensors), not a step of the method.
@@ -135,6 +138,23 @@ def moe_params(shape, seed=0, device="cpu"):
 def moe_input(shape, tokens, seed=0, device="cpu"):
     g = _gen(seed + 65537, device)
     return _store(_normal(g, (tokens, shape.d_model), device=device), shape.dtype)
+
+
+def attn_params(shape, seed=0, device="cpu"):
+    g = _gen(seed + 271828, device)
+    H, G, D, dm = shape.n_heads, shape.n_kv_heads, shape.head_dim, shape.d_model
+    dt = shape.dtype
+    return dict(
+        wq=_store(_normal(g, (H * D, dm), STD, device=device), dt),
+        wk=_store(_normal(g, (G * D, dm), STD, device=device), dt),
+        wv=_store(_normal(g, (G * D, dm), STD, device=device), dt),
+        wo=_store(_normal(g, (dm, H * D), STD, device=device), dt),
+    )
+
+
+def attn_input(shape, batch, seqlen, seed=0, device="cpu"):
+    g = _gen(seed + 314159, device)
+    return _store(_normal(g, (batch, seqlen, shape.d_model), device=device), shape.dtype)
 
 
 def block_norm_params(d_model, seed=0, device="cpu", init="ones"):

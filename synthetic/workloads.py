@@ -37,6 +37,18 @@ class MoEShape:
         return replace(self, **kw)
 
 
+@dataclass(frozen=True)
+class AttnShape:
+    d_model: int = 4096
+    n_heads: int = 32
+    n_kv_heads: int = 8
+    head_dim: int = 128
+    dtype: str = "bf16"
+
+    def with_(self, **kw):
+        return replace(self, **kw)
+
+
 JAMBA_MAMBA = MambaShape(d_model=4096, d_inner=8192, d_state=16, d_conv=4,
                          dt_rank=256, dtype="bf16", inner_norm=True)
 
@@ -55,6 +67,8 @@ WORKLOADS = {
     "decode_b64": dict(mamba=JAMBA_MAMBA, batch=64, prefill=2048, steps=1024),
     # RMSNorm -> Mamba -> residual -> RMSNorm -> top-2-of-16 MoE -> residual
     "layer_pair": dict(mamba=JAMBA_MAMBA, moe=MoEShape(), batch=4, seqlen=8192),
+    # the block's GQA attention layer: prefill of 32768 tokens (batch 1)
+    "attn_32k": dict(attn=AttnShape(), batch=1, seqlen=32768),
 }
 
 

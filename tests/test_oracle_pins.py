@@ -485,3 +485,107 @@ def test_int8_moe_lossless_on_representable_weights():
         np.testing.assert_array_equal(back[k], p[k])
     v = rng.standard_normal((13, dm))
     np.testing.assert_array_equal(omoe.moe_forward(back, v, 2)["out"], omoe.moe_forward(p, v, 2)["out"])
+
+
+# ------------------------------------------------------------------ attention pins
+
+from oracle import attention as oatt  # noqa: E402
+from synthetic import AttnShape  # noqa: E402
+
+
+def _attn_rand(rng, shape, B, L):
+    H, G, D, dm = shape.n_heads, shape.n_kv_heads, shape.head_dim, shape.d_model
+    p = dict(wq=rng.standard_normal((H * D, dm)) * 0.5, wk=rng.standard_normal((G * D, dm)) * 0.5,
+             wv=rng.standard_normal((G * D, dm)), wo=rng.standard_normal((dm, H * D)))
+    return p, rng.standard_normal((B, L, dm))
+
+
+def test_attention_vs_python_loop():
+    sh = AttnShape(d_model=5, n_heads=4, n_kv_heads=2, head_dim=3)
+    rng = np.random.default_rng(30)
+    p, x = _attn_rand(rng, sh, 2, 4)
+    H, G, D = 4, 2, 3
+    want = np.zeros((2, 4, 5))
+    for b in range(2):
+        for t in range(4):
+            o = []
+            for h in range(H):
+                g = h // (H // G)
+                q = [sum(p["wq"][h * D + d, i] * x[b, t, i] for i in range(5)) for d in range(D)]
+                ks = [[sum(p["wk"][g * D + d, i] * x[b, j, i] for i in range(5)) for d in range(D)] for j in range(t + 1)]
+                vs = [[sum(p["wv"][g * D + d, i] * x[b, j, i] for i in range(5)) for d in range(D)] for j in range(t + 1)]
+                sc = [sum(q[d] * ks[j][d] for d in range(D)) / math.sqrt(D) for j in range(t + 1)]
+                mx = max(sc)
+                e = [math.exp(v - mx) for v in sc]
+                z = sum(e)
+                o += [sum(e[j] / z * vs[j][d] for j in range(t + 1)) for d in range(D)]
+            for i in range(5):
+                want[b, t, i] = sum(p["wo"][i, c] * o[c] for c in range(H * D))
+    np.testing.assert_allclose(oatt.attention_prefill(p, x, sh)["out"], want, rtol=1e-12, atol=1e-12)
+
+
+def test_attention_zero_query_is_running_mean():
+    sh = AttnShape(d_model=6, n_heads=2, n_kv_heads=1, head_dim=4)
+    rng = np.random.default_rng(31)
+    p, x = _attn_rand(rng, sh, 1, 7)
+    p["wq"][:] = 0.0
+    r = oatt.attention_prefill(p, x, sh)
+    v = r["v"][0, :, 0]                                     # [L, D]
+    want = np.cumsum(v, axis=0) / np.arange(1, 8)[:, None]
+    for h in range(2):
+        np.testing.assert_allclose(r["o"][0, :, h], want, rtol=1e-13)
+    # the first token sees only itself
+    np.testing.assert_allclose(r["o"][0, 0, 0], v[0], rtol=1e-14)
+
+
+def test_attention_gqa_equals_repeated_mha():
+    sh = AttnShape(d_model=8, n_heads=6, n_kv_heads=2, head_dim=3)
+    rng = np.random.default_rng(32)
+    p, x = _attn_rand(rng, sh, 2, 5)
+    rep = dict(p)
+    for k in ("wk", "wv"):
+        w = p[k].reshape(2, 3, 8)
+        rep[k] = np.repeat(w, 3, axis=0).reshape(18, 8)      # KV head g serves query heads 3g..3g+2
+    mha = AttnShape(d_model=8, n_heads=6, n_kv_heads=6, head_dim=3)
+    np.testing.assert_allclose(oatt.attention_prefill(p, x, sh)["out"],
+                               oatt.attention_prefill(rep, x, mha)["out"], rtol=1e-13, atol=1e-13)
+
+
+def test_attention_key_shift_and_causality():
+    sh = AttnShape(d_model=6, n_heads=4, n_kv_heads=2, head_dim=4)
+    rng = np.random.default_rng(33)
+    p, x = _attn_rand(rng, sh, 1, 9)
+    q, k, v = oatt.project(p, x, sh)
+    o = oatt.attend(q, k, v)
+    # a vector common to every key adds the same amount to a query's logits
+    o2 = oatt.attend(q, k + rng.standard_normal((1, 1, 2, 4)), v)
+    np.testing.assert_allclose(o2, o, rtol=1e-12, atol=1e-12)
+    # changing token 5 leaves tokens 0..4 unchanged and moves token 5
+    x2 = x.copy()
+    x2[0, 5] += 1.0
+    a = oatt.attention_prefill(p, x, sh)["out"]
+    b = oatt.attention_prefill(p, x2, sh)["out"]
+    np.testing.assert_array_equal(a[0, :5], b[0, :5])
+    assert np.abs(a[0, 5:] - b[0, 5:]).min() > 0
+
+
+def test_attention_two_keys_closed_form():
+    """Query (s, 0) against one-hot keys e0, e1: weights e^{s/sqrt(2)} : 1."""
+    q = np.zeros((1, 1, 1, 2))
+    q[0, 0, 0, 0] = 3.0
+    k = np.array([[[[1.0, 0.0]], [[0.0, 1.0]]]])            # [1, 2, 1, 2]
+    v = np.array([[[[10.0, 0.0]], [[0.0, 20.0]]]])
+    o = oatt.attend(q, k, v, q_pos0=1)
+    w0 = math.exp(3.0 / math.sqrt(2)) / (math.exp(3.0 / math.sqrt(2)) + 1.0)
+    np.testing.assert_allclose(o[0, 0, 0], [10.0 * w0, 20.0 * (1 - w0)], rtol=1e-14)
+
+
+def test_attention_step_equals_prefill_last_row():
+    sh = AttnShape(d_model=8, n_heads=4, n_kv_heads=2, head_dim=4)
+    rng = np.random.default_rng(34)
+    p, x = _attn_rand(rng, sh, 3, 7)
+    full = oatt.attention_prefill(p, x, sh)
+    pre = oatt.attention_prefill(p, x[:, :6], sh)
+    st = oatt.attention_step(p, x[:, 6], pre["k"], pre["v"], 6, sh)
+    np.testing.assert_allclose(st["out"], full["out"][:, 6], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(st["k_new"], full["k"][:, 6], rtol=1e-13)
