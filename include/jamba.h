@@ -294,6 +294,56 @@ jamba_status jamba_moe_forward(const jamba_moe_config* cfg, const jamba_moe_weig
                                int32_t* topk_idx, float* topk_w, int32_t* expert_offsets,
                                int32_t* perm, void* ws, size_t ws_bytes, jamba_stream_t stream);
 
+/* ------------------------------------------------------------- attention */
+
+/* The Jamba block's attention layer ("Jamba: A Hybrid Transformer-Mamba
+ * Language Model", section 2: one layer in eight; standard details including
+ * grouped-query attention; no explicit positional information, so no
+ * positional embedding or RoPE).  Query head h reads KV head
+ * h / (n_heads / n_kv_heads); causal softmax of q . k / sqrt(head_dim);
+ * projections without bias. */
+typedef struct jamba_attn_config {
+  int d_model;    /* 4096 */
+  int n_heads;    /* query heads (32 at Jamba width) */
+  int n_kv_heads; /* key/value heads, divides n_heads (8 at Jamba width) */
+  int head_dim;   /* 128 (the only width supported) */
+  int dtype;      /* JAMBA_BF16 */
+} jamba_attn_config;
+
+typedef struct jamba_attn_weights {
+  const void* w_qkv; /* [(n_heads + 2 n_kv_heads) * head_dim, d_model]: W_q rows, then W_k, then W_v */
+  const void* w_o;   /* [d_model, n_heads * head_dim] */
+} jamba_attn_weights;
+
+jamba_status jamba_attn_prefill_workspace_size(const jamba_attn_config* cfg, int batch, int seqlen, size_t* bytes);
+
+/* Causal attention over `seqlen` tokens of each of `batch` sequences.
+ *   x        [batch, seqlen, d_model] dtype (already block-normed)
+ *   residual [batch, seqlen, d_model] or NULL, added to the output
+ *   out      [batch, seqlen, d_model] (may not alias x)
+ *   k_cache, v_cache  NULL, or [batch, n_kv_heads, max_len, head_dim] dtype:
+ *            positions 0..seqlen-1 are written (max_len >= seqlen)
+ * The workspace holds the fused q|k|v rows, V transposed and the attention
+ * output before out_proj.  seqlen >= 1; no other limit than the workspace. */
+jamba_status jamba_attn_prefill(const jamba_attn_config* cfg, const jamba_attn_weights* w, const void* x,
+                                const void* residual, void* out, int batch, int seqlen, void* k_cache,
+                                void* v_cache, int max_len, void* ws, size_t ws_bytes, jamba_stream_t stream);
+
+jamba_status jamba_attn_step_workspace_size(const jamba_attn_config* cfg, int batch, int max_len, size_t* bytes);
+
+/* One decode token per sequence.
+ *   x [batch, d_model]; residual [batch, d_model] or NULL; out [batch, d_model]
+ *   k_cache, v_cache [batch, n_kv_heads, max_len, head_dim]
+ *   lengths [batch] int32 device array: tokens already cached per sequence.
+ *            The new token's k and v are written at position lengths[b], the
+ *            token attends to positions 0..lengths[b], and lengths[b] is then
+ *            incremented (so a captured CUDA graph can be replayed step after
+ *            step).  A sequence whose length is outside [0, max_len) is left
+ *            untouched by the cache append; the caller keeps lengths < max_len. */
+jamba_status jamba_attn_step(const jamba_attn_config* cfg, const jamba_attn_weights* w, const void* x,
+                             const void* residual, void* out, int batch, void* k_cache, void* v_cache,
+                             int max_len, int32_t* lengths, void* ws, size_t ws_bytes, jamba_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -47,6 +47,15 @@ class MoeWeights(ctypes.Structure):
                                                "s_gate", "s_up", "s_down")]
 
 
+class AttnConfig(ctypes.Structure):
+    _fields_ = [("d_model", ctypes.c_int), ("n_heads", ctypes.c_int), ("n_kv_heads", ctypes.c_int),
+                ("head_dim", ctypes.c_int), ("dtype", ctypes.c_int)]
+
+
+class AttnWeights(ctypes.Structure):
+    _fields_ = [("w_qkv", ctypes.c_void_p), ("w_o", ctypes.c_void_p)]
+
+
 P = ctypes.c_void_p
 I = ctypes.c_int
 SZ = ctypes.c_size_t
@@ -72,6 +81,12 @@ SIGNATURES = {
     "jamba_moe_workspace_size": [ctypes.POINTER(MoeConfig), I, ctypes.POINTER(SZ)],
     "jamba_moe_forward": [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), P, P, P, I, P, P, P, P,
                           P, SZ, P],
+    "jamba_attn_prefill_workspace_size": [ctypes.POINTER(AttnConfig), I, I, ctypes.POINTER(SZ)],
+    "jamba_attn_prefill": [ctypes.POINTER(AttnConfig), ctypes.POINTER(AttnWeights), P, P, P, I, I, P, P, I,
+                           P, SZ, P],
+    "jamba_attn_step_workspace_size": [ctypes.POINTER(AttnConfig), I, I, ctypes.POINTER(SZ)],
+    "jamba_attn_step": [ctypes.POINTER(AttnConfig), ctypes.POINTER(AttnWeights), P, P, P, I, P, P, I, P,
+                        P, SZ, P],
 }
 
 _lib = None

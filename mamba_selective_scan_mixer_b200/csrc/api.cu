@@ -676,3 +676,141 @@ jamba_status jamba_moe_forward(const jamba_moe_config* cfg, const jamba_moe_weig
 }
 
 }  // extern "C"
+
+// -------------------------------------------------------------- attention
+
+namespace {
+struct AttnPrefillWs {
+  void* qkv; void* vt; void* o;
+  long long ldv;
+  size_t total;
+};
+AttnPrefillWs carve_attn_prefill(const jamba_attn_config& c, int B, int L, void* ws) {
+  AttnPrefillWs a;
+  const long long T = (long long)B * L;
+  const int W = (c.n_heads + 2 * c.n_kv_heads) * c.head_dim;
+  a.ldv = (L + 7) / 8 * 8;
+  Carver cv(ws);
+  a.qkv = cv.take((size_t)T * W * 2);
+  a.vt = cv.take((size_t)B * c.n_kv_heads * c.head_dim * a.ldv * 2);
+  a.o = cv.take((size_t)T * c.n_heads * c.head_dim * 2);
+  a.total = cv.off;
+  return a;
+}
+struct AttnStepWs {
+  void* qkv; float* part; void* o; float* opart;
+  int splits, o_splits;
+  size_t total;
+};
+AttnStepWs carve_attn_step(const jamba_attn_config& c, int B, int max_len, void* ws) {
+  AttnStepWs a;
+  const int W = (c.n_heads + 2 * c.n_kv_heads) * c.head_dim, HD = c.n_heads * c.head_dim;
+  a.splits = attn_decode_splits(B, c.n_kv_heads, max_len);
+  a.o_splits = choose_splits(c.d_model, B, HD, 64, 8);
+  Carver cv(ws);
+  a.qkv = cv.take((size_t)B * W * 2);
+  a.part = cv.take<float>((size_t)B * c.n_heads * a.splits * (c.head_dim + 2) * 4);
+  a.o = cv.take((size_t)B * HD * 2);
+  a.opart = cv.take<float>((size_t)a.o_splits * B * c.d_model * 4);
+  a.total = cv.off;
+  return a;
+}
+jamba_status check_attn_cfg(const jamba_attn_config* c) {
+  if (!c) return fail(JAMBA_ERR_INVALID_ARG, "attention: null config");
+  if (c->dtype != JAMBA_BF16) return fail(JAMBA_ERR_UNSUPPORTED, "attention: bf16 only");
+  if (c->head_dim != 128) return fail(JAMBA_ERR_UNSUPPORTED, "attention: head_dim must be 128");
+  if (c->n_heads <= 0 || c->n_kv_heads <= 0 || c->n_heads % c->n_kv_heads)
+    return fail(JAMBA_ERR_INVALID_ARG, "attention: n_kv_heads must divide n_heads");
+  if (c->d_model <= 0 || c->d_model % 64) return fail(JAMBA_ERR_UNSUPPORTED, "attention: d_model must be a multiple of 64");
+  return JAMBA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+jamba_status jamba_attn_prefill_workspace_size(const jamba_attn_config* cfg, int batch, int seqlen, size_t* bytes) {
+  JB_TRY(check_attn_cfg(cfg));
+  if (!bytes || batch <= 0 || seqlen <= 0) return fail(JAMBA_ERR_INVALID_ARG, "attention workspace: bad argument");
+  *bytes = carve_attn_prefill(*cfg, batch, seqlen, nullptr).total;
+  return JAMBA_OK;
+}
+
+jamba_status jamba_attn_prefill(const jamba_attn_config* cfg, const jamba_attn_weights* w, const void* x,
+                                const void* residual, void* out, int batch, int seqlen, void* k_cache,
+                                void* v_cache, int max_len, void* ws, size_t ws_bytes, jamba_stream_t stream) {
+  JB_TRY(check_attn_cfg(cfg));
+  if (!w || batch <= 0 || seqlen <= 0) return fail(JAMBA_ERR_INVALID_ARG, "attention prefill: bad argument");
+  JB_TRY(check_ptr(w->w_qkv, "w_qkv"));
+  JB_TRY(check_ptr(w->w_o, "w_o"));
+  JB_TRY(check_ptr(x, "x"));
+  JB_TRY(check_ptr(out, "out"));
+  JB_TRY(check_ptr(residual, "residual", false));
+  JB_TRY(check_ptr(k_cache, "k_cache", false));
+  JB_TRY(check_ptr(v_cache, "v_cache", false));
+  JB_TRY(check_ptr(ws, "workspace"));
+  if (x == out) return fail(JAMBA_ERR_INVALID_ARG, "attention prefill: out may not alias x");
+  if ((k_cache == nullptr) != (v_cache == nullptr))
+    return fail(JAMBA_ERR_INVALID_ARG, "attention prefill: give both caches or neither");
+  if (k_cache && max_len < seqlen) return fail(JAMBA_ERR_INVALID_ARG, "attention prefill: max_len < seqlen");
+  const jamba_attn_config& c = *cfg;
+  AttnPrefillWs a = carve_attn_prefill(c, batch, seqlen, ws);
+  if (ws_bytes < a.total) return fail(JAMBA_ERR_WORKSPACE, "attention prefill: workspace too small");
+  cudaStream_t s = cs(stream);
+  const int T = batch * seqlen, dm = c.d_model, HD = c.n_heads * c.head_dim;
+  const int W = (c.n_heads + 2 * c.n_kv_heads) * c.head_dim;
+  JB_TRY(gemm_bf16(gdesc(x, dm, w->w_qkv, dm, T, W, dm, EPI_BF16, a.qkv, W), s));
+  JB_TRY(attn_prefill_core(a.qkv, a.vt, a.ldv, a.o, k_cache, v_cache, max_len, batch, seqlen, c.n_heads,
+                           c.n_kv_heads, s));
+  GemmDesc go = gdesc(a.o, HD, w->w_o, HD, T, dm, HD, EPI_BF16, out, dm);
+  go.residual = residual;
+  go.ldr = dm;
+  JB_TRY(gemm_bf16(go, s));
+  return JAMBA_OK;
+}
+
+jamba_status jamba_attn_step_workspace_size(const jamba_attn_config* cfg, int batch, int max_len, size_t* bytes) {
+  JB_TRY(check_attn_cfg(cfg));
+  if (!bytes || batch <= 0 || max_len <= 0) return fail(JAMBA_ERR_INVALID_ARG, "attention workspace: bad argument");
+  *bytes = carve_attn_step(*cfg, batch, max_len, nullptr).total;
+  return JAMBA_OK;
+}
+
+jamba_status jamba_attn_step(const jamba_attn_config* cfg, const jamba_attn_weights* w, const void* x,
+                             const void* residual, void* out, int batch, void* k_cache, void* v_cache,
+                             int max_len, int32_t* lengths, void* ws, size_t ws_bytes, jamba_stream_t stream) {
+  JB_TRY(check_attn_cfg(cfg));
+  if (!w || batch <= 0 || max_len <= 0) return fail(JAMBA_ERR_INVALID_ARG, "attention step: bad argument");
+  JB_TRY(check_ptr(w->w_qkv, "w_qkv"));
+  JB_TRY(check_ptr(w->w_o, "w_o"));
+  JB_TRY(check_ptr(x, "x"));
+  JB_TRY(check_ptr(out, "out"));
+  JB_TRY(check_ptr(residual, "residual", false));
+  JB_TRY(check_ptr(k_cache, "k_cache"));
+  JB_TRY(check_ptr(v_cache, "v_cache"));
+  JB_TRY(check_ptr(ws, "workspace"));
+  if (!lengths) return fail(JAMBA_ERR_INVALID_ARG, "attention step: lengths is null");
+  if (x == out) return fail(JAMBA_ERR_INVALID_ARG, "attention step: out may not alias x");
+  const jamba_attn_config& c = *cfg;
+  AttnStepWs a = carve_attn_step(c, batch, max_len, ws);
+  if (ws_bytes < a.total) return fail(JAMBA_ERR_WORKSPACE, "attention step: workspace too small");
+  cudaStream_t s = cs(stream);
+  const int dm = c.d_model, HD = c.n_heads * c.head_dim;
+  const int W = (c.n_heads + 2 * c.n_kv_heads) * c.head_dim;
+  // weights stream through the tensor cores as the 128-row side; the token batch is the N side
+  GemmDesc g1 = gdesc(w->w_qkv, dm, x, dm, W, batch, dm, EPI_BF16, a.qkv, W);
+  g1.transpose_out = 1;
+  g1.bn = 64;
+  JB_TRY(gemm_bf16(g1, s));
+  JB_TRY(attn_decode_core(a.qkv, k_cache, v_cache, max_len, lengths, a.part, a.splits, a.o, batch, c.n_heads,
+                          c.n_kv_heads, s));
+  GemmDesc g2 = gdesc(w->w_o, HD, a.o, HD, dm, batch, HD, EPI_F32, a.opart, dm);
+  g2.transpose_out = 1;
+  g2.bn = 64;
+  g2.splits = a.o_splits;
+  g2.split_stride = (long long)batch * dm;
+  JB_TRY(gemm_bf16(g2, s));
+  JB_TRY(splitk_reduce(a.opart, a.o_splits, (long long)batch * dm, (long long)batch * dm, residual, out, JAMBA_BF16, s));
+  return JAMBA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,530 @@
+// Grouped-query attention layer of the Jamba block.
+//
+// "Jamba: A Hybrid Transformer-Mamba Language Model" (summary page),
+// section 2: one layer in eight is attention, of the standard kind with
+// grouped-query attention; no explicit positional information is used (no
+// positional embedding, no RoPE).  Query head h reads KV head h / (H / G);
+// causal softmax of q . k / sqrt(head_dim).
+//
+// Prefill: the fused q|k|v projection is one tcgen05 GEMM ([T, (H + 2G) D]
+// rows); the attention kernel reads its Q and K tiles in place from that
+// buffer with TMA.  V is written transposed ([B*G*D, L]) by kv_prep_kernel so
+// that P.V is a K-major product like every other operand here; the same
+// kernel fills the KV cache.  flash_attn_kernel: one CTA per (sequence,
+// query head, 128-query block), heavy (late) blocks first; per 128-key block
+// S = Q K^T (tcgen05, fp32 in TMEM, double-buffered), an online softmax by
+// four warps (thread = query row; the running maximum is raised lazily, only
+// when a row's maximum grows by more than 2^8, and O is then rescaled in
+// TMEM), P in bf16 through swizzled shared memory, O += P V (tcgen05, fp32
+// in TMEM).  Every wait is bounded (see common.cuh).
+//
+// Decode: the new token's k and v are appended to the cache at the
+// sequence's current length, then attn_decode_kernel splits the cached
+// positions of each (sequence, KV head) over CTAs (all query heads of the
+// group read each key and value once) and attn_combine_kernel merges the
+// partial softmaxes and advances the lengths.  Bound by reading the cache.
+#include "common.cuh"
+#include "host.hpp"
+
+namespace jb {
+
+constexpr int ATT_D = 128;       // head width (the only one supported)
+constexpr int ATT_BQ = 128;      // query rows per CTA
+constexpr int ATT_BK = 128;      // keys per block
+constexpr int ATT_KVST = 2;      // K / V^T ring stages
+constexpr int ATT_THREADS = 192; // producer, MMA, four softmax warps
+
+struct AttnSmem {
+  static constexpr uint32_t SUB = 128 * 128;                 // 128 rows x 64 bf16, swizzled
+  static constexpr uint32_t Q_OFF = 0;                       // Q: dims 0-63 | 64-127
+  static constexpr uint32_t KV_OFF = 2 * SUB;                // per stage: K (dims) x2, V^T (keys) x2
+  static constexpr uint32_t KV_STAGE = 4 * SUB;
+  static constexpr uint32_t P_OFF = KV_OFF + ATT_KVST * KV_STAGE;   // P: keys 0-63 | 64-127
+  static constexpr uint32_t BAR_OFF = P_OFF + 2 * SUB;
+  static constexpr uint32_t BYTES = BAR_OFF + 256 + 1024;
+};
+
+struct AttnParams {
+  int B, L, H, G, rep, nq;
+  bf16* o;
+  long long ldo;
+  float sl2;   // log2(e) / sqrt(head_dim)
+  int* err;
+};
+
+__global__ void __launch_bounds__(ATT_THREADS, 1)
+flash_attn_kernel(const __grid_constant__ CUtensorMap tmQK, const __grid_constant__ CUtensorMap tmVt,
+                  const AttnParams p) {
+  using S = AttnSmem;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::BAR_OFF);
+  const uint32_t q_full = smem_u32(bars);
+  const uint32_t kv_full0 = smem_u32(bars + 1), kv_empty0 = smem_u32(bars + 3);
+  const uint32_t s_full0 = smem_u32(bars + 5), s_free0 = smem_u32(bars + 7);
+  const uint32_t p_full = smem_u32(bars + 9), pv_done = smem_u32(bars + 10), drain = smem_u32(bars + 11);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 12);
+
+  const int bh = blockIdx.x % (p.B * p.H);
+  const int qi = p.nq - 1 - (int)(blockIdx.x / (p.B * p.H));   // late query blocks (more keys) first
+  const int b = bh / p.H, h = bh % p.H, g = h / p.rep;
+  const int nkv = qi + 1;
+  const int row0 = b * p.L + qi * ATT_BQ;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (warp == 0 && lane == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(kv_full0 + 8 * i, 1);
+      mbar_init(kv_empty0 + 8 * i, 1);
+      mbar_init(s_full0 + 8 * i, 1);
+      mbar_init(s_free0 + 8 * i, 4);
+    }
+    mbar_init(p_full, 4);
+    mbar_init(pv_done, 1);
+    mbar_init(drain, 1);
+    mbar_fence_init();
+    tma_prefetch(&tmQK);
+    tma_prefetch(&tmVt);
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_holder), 512);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_holder;
+  const uint32_t tS = tbase, tO = tbase + 256;   // S buffers at columns 0 and 128, O at 256
+  griddep_launch();
+  griddep_wait();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_tx(q_full, 2 * S::SUB);
+      tma_load_2d(smem_u32(smem + S::Q_OFF), &tmQK, q_full, h * ATT_D, row0);
+      tma_load_2d(smem_u32(smem + S::Q_OFF + S::SUB), &tmQK, q_full, h * ATT_D + 64, row0);
+      for (int j = 0; j < nkv; ++j) {
+        const int st = j & 1;
+        if (!mbar_wait(kv_empty0 + 8 * st, ((j >> 1) & 1) ^ 1, p.err)) break;
+        const uint32_t fb = kv_full0 + 8 * st;
+        const uint32_t base = smem_u32(smem + S::KV_OFF + st * S::KV_STAGE);
+        mbar_arrive_tx(fb, 4 * S::SUB);
+        const int krow = b * p.L + j * ATT_BK, kcol = (p.H + g) * ATT_D, vrow = (b * p.G + g) * ATT_D;
+        tma_load_2d(base, &tmQK, fb, kcol, krow);
+        tma_load_2d(base + S::SUB, &tmQK, fb, kcol + 64, krow);
+        tma_load_2d(base + 2 * S::SUB, &tmVt, fb, j * ATT_BK, vrow);
+        tma_load_2d(base + 3 * S::SUB, &tmVt, fb, j * ATT_BK + 64, vrow);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_bf16(128, 128);
+      const uint64_t qd[2] = {sw128_desc(smem_u32(smem + S::Q_OFF)), sw128_desc(smem_u32(smem + S::Q_OFF + S::SUB))};
+      const uint64_t pd[2] = {sw128_desc(smem_u32(smem + S::P_OFF)), sw128_desc(smem_u32(smem + S::P_OFF + S::SUB))};
+      // S = Q K^T over the head width: k-steps 0-3 in the first 64 dims, 4-7 in the second
+      auto issue_s = [&](uint32_t d, int st) {
+        const uint32_t base = smem_u32(smem + S::KV_OFF + st * S::KV_STAGE);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_bf16(d, qd[kk >> 2] + 2 * (kk & 3), sw128_desc(base + (kk >> 2) * S::SUB) + 2 * (kk & 3), IDESC,
+                    kk > 0 ? 1u : 0u);
+      };
+      bool ok = mbar_wait(q_full, 0, p.err) && mbar_wait(kv_full0, 0, p.err);
+      if (ok) {
+        tc_fence_after();
+        issue_s(tS, 0);
+        umma_commit(s_full0);
+      }
+      for (int j = 0; j < nkv && ok; ++j) {
+        if (j + 1 < nkv) {
+          const int nb = (j + 1) & 1;
+          if (!mbar_wait(s_free0 + 8 * nb, (((j + 1) >> 1) & 1) ^ 1, p.err)) break;
+          if (!mbar_wait(kv_full0 + 8 * nb, ((j + 1) >> 1) & 1, p.err)) break;
+          tc_fence_after();
+          issue_s(tS + nb * 128, nb);
+          umma_commit(s_full0 + 8 * nb);
+        }
+        if (!mbar_wait(p_full, j & 1, p.err)) break;
+        tc_fence_after();
+        // O += P V: keys 0-63 in the first P / V^T sub-tiles, 64-127 in the second
+        const uint32_t vbase = smem_u32(smem + S::KV_OFF + (j & 1) * S::KV_STAGE + 2 * S::SUB);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_bf16(tO, pd[kk >> 2] + 2 * (kk & 3), sw128_desc(vbase + (kk >> 2) * S::SUB) + 2 * (kk & 3), IDESC,
+                    (j > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(kv_empty0 + 8 * (j & 1));
+        umma_commit(pv_done);
+      }
+      umma_commit(drain);
+      mbar_wait(drain, 0, p.err);
+    }
+  } else {
+    // softmax: thread = query row r of this warp's TMEM lane quarter
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    float m = 0.f, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nkv; ++j) {
+      const int buf = j & 1;
+      if (!mbar_wait(s_full0 + 8 * buf, (j >> 1) & 1, p.err)) { ok = false; break; }
+      tc_fence_after();
+      float s[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + lane_off + buf * 128 + 32 * c, s + 32 * c);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free0 + 8 * buf);
+      if (j == qi) {   // diagonal block: key c is visible to row r when c <= r
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c > r) s[c] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+      const float mnew = mx * p.sl2;
+      float corr = 1.f;
+      if (j == 0) {
+        m = mnew;
+      } else if (mnew > m + 8.f) {   // raise the reference only when the terms would exceed 2^8
+        corr = ex2(m - mnew);
+        m = mnew;
+      }
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) {
+        s[c] = ex2(fmaf(s[c], p.sl2, -m));
+        sum += s[c];
+      }
+      l = l * corr + sum;
+      if (j > 0) {
+        // P_{j-1} and the O it fed are done: P may be overwritten and O rescaled
+        if (!mbar_wait(pv_done, (j - 1) & 1, p.err)) { ok = false; break; }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, corr != 1.f)) {
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            float o[32];
+            tmem_ld32(tO + lane_off + 32 * c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= corr;
+            tmem_st32(tO + lane_off + 32 * c, o);
+          }
+          tmem_wait_st();
+        }
+      }
+      // P row r (bf16) into the two swizzled sub-tiles: 16-byte chunk k of row r at (k ^ (r & 7))
+      uint8_t* prow = smem + S::P_OFF + r * 128;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        uint4 u;
+        __nv_bfloat162* hh = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) hh[i] = __floats2bfloat162_rn(s[8 * k + 2 * i], s[8 * k + 2 * i + 1]);
+        *reinterpret_cast<uint4*>(prow + (k >> 3) * S::SUB + (((k & 7) ^ (r & 7)) << 4)) = u;
+      }
+      fence_async_shared();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    if (ok && mbar_wait(pv_done, (nkv - 1) & 1, p.err)) {
+      tc_fence_after();
+      const float inv = 1.f / l;
+      const int row = qi * ATT_BQ + r;
+      bf16* dst = p.o + (long long)(b * p.L + row) * p.ldo + h * ATT_D;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float o[32];
+        tmem_ld32(tO + lane_off + 32 * c, o);
+        tmem_wait_ld();
+        if (row < p.L) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            float w[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) w[i] = o[8 * k + i] * inv;
+            uint4 u;
+            __nv_bfloat162* hh = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) hh[i] = __floats2bfloat162_rn(w[2 * i], w[2 * i + 1]);
+            *reinterpret_cast<uint4*>(dst + 32 * c + 8 * k) = u;
+          }
+        }
+      }
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// qkv [B*L, W] (W = (H + 2G) D): V transposed into vt [B*G*D, ldv] (row
+// (b, g, d), column = position) and, when given, K and V into the caches
+// [B, G, max_len, D].  Block: one (sequence, KV head, 64 positions).
+__global__ void __launch_bounds__(256)
+kv_prep_kernel(const bf16* __restrict__ qkv, int L, int H, int G, bf16* __restrict__ vt, long long ldv,
+               bf16* __restrict__ kc, bf16* __restrict__ vc, int max_len) {
+  __shared__ bf16 tile[64][ATT_D + 8];
+  griddep_wait();
+  griddep_launch();
+  const int bg = blockIdx.y, b = bg / G, g = bg % G;
+  const int pos0 = blockIdx.x * 64;
+  const long long W = (long long)(H + 2 * G) * ATT_D;
+  // rows: 64 positions x 16 chunks of 8 values
+  for (int i = threadIdx.x; i < 64 * 16; i += 256) {
+    const int pr = i >> 4, ch = i & 15, pos = pos0 + pr;
+    uint4 vv = make_uint4(0, 0, 0, 0);
+    if (pos < L) {
+      const bf16* row = qkv + (long long)(b * L + pos) * W;
+      vv = *reinterpret_cast<const uint4*>(row + (long long)(H + G + g) * ATT_D + ch * 8);
+      if (kc) {
+        const uint4 kv = *reinterpret_cast<const uint4*>(row + (long long)(H + g) * ATT_D + ch * 8);
+        const long long o = (((long long)b * G + g) * max_len + pos) * ATT_D + ch * 8;
+        *reinterpret_cast<uint4*>(kc + o) = kv;
+        *reinterpret_cast<uint4*>(vc + o) = vv;
+      }
+    }
+    *reinterpret_cast<uint4*>(&tile[pr][ch * 8]) = vv;
+  }
+  __syncthreads();
+  // columns: 128 dims x 64 positions, two positions per thread-step
+  for (int i = threadIdx.x; i < ATT_D * 32; i += 256) {
+    const int d = i >> 5, pp = (i & 31) * 2, pos = pos0 + pp;
+    if (pos < L) {
+      bf16* dst = vt + ((long long)bg * ATT_D + d) * ldv + pos;
+      dst[0] = tile[pp][d];
+      if (pos + 1 < L) dst[1] = tile[pp + 1][d];
+    }
+  }
+}
+
+jamba_status attn_prefill_core(const void* qkv, void* vt, long long ldv, void* o, void* k_cache, void* v_cache,
+                               int max_len, int B, int L, int H, int G, cudaStream_t s) {
+  const int W = (H + 2 * G) * ATT_D;
+  JB_CUDA(launch_pdl(kv_prep_kernel, dim3((L + 63) / 64, B * G), dim3(256), 0, s,
+                     reinterpret_cast<const bf16*>(qkv), L, H, G, reinterpret_cast<bf16*>(vt), ldv,
+                     reinterpret_cast<bf16*>(k_cache), reinterpret_cast<bf16*>(v_cache), max_len));
+  CUtensorMap mqk, mvt;
+  JB_TRY(make_map_2d(&mqk, qkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)W, (uint64_t)B * L, (uint64_t)W * 2,
+                     64, 128, CU_TENSOR_MAP_SWIZZLE_128B));
+  JB_TRY(make_map_2d(&mvt, vt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)L, (uint64_t)B * G * ATT_D,
+                     (uint64_t)ldv * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B));
+  AttnParams p;
+  p.B = B;
+  p.L = L;
+  p.H = H;
+  p.G = G;
+  p.rep = H / G;
+  p.nq = (L + ATT_BQ - 1) / ATT_BQ;
+  p.o = reinterpret_cast<bf16*>(o);
+  p.ldo = (long long)H * ATT_D;
+  p.sl2 = 1.4426950408889634f / sqrtf((float)ATT_D);
+  p.err = device_error_word();
+  if (!p.err) return fail(JAMBA_ERR_CUDA, "could not allocate the device status word");
+  static bool configured[64] = {false};
+  int dev = 0;
+  JB_CUDA(cudaGetDevice(&dev));
+  if (dev < 64 && !configured[dev]) {
+    JB_CUDA(cudaFuncSetAttribute(flash_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)AttnSmem::BYTES));
+    configured[dev] = true;
+  }
+  JB_CUDA(launch_pdl(flash_attn_kernel, dim3((unsigned)(B * H * p.nq)), dim3(ATT_THREADS), AttnSmem::BYTES, s, mqk,
+                     mvt, p));
+  return JAMBA_OK;
+}
+
+// ---------------------------------------------------------------- decode
+
+// qkv [B, W]: k and v of the new token into the caches at position lengths[b]
+__global__ void __launch_bounds__(256)
+kv_append_kernel(const bf16* __restrict__ qkv, int H, int G, const int* __restrict__ lengths, bf16* __restrict__ kc,
+                 bf16* __restrict__ vc, int max_len) {
+  griddep_wait();
+  griddep_launch();
+  const int b = blockIdx.x;
+  const int pos = lengths[b];
+  if (pos < 0 || pos >= max_len) return;   // rejected on the host side for the lengths it can see
+  const long long W = (long long)(H + 2 * G) * ATT_D;
+  for (int i = threadIdx.x; i < G * 16; i += 256) {
+    const int g = i >> 4, ch = i & 15;
+    const bf16* row = qkv + b * W;
+    const long long o = (((long long)b * G + g) * max_len + pos) * ATT_D + ch * 8;
+    *reinterpret_cast<uint4*>(kc + o) = *reinterpret_cast<const uint4*>(row + (long long)(H + g) * ATT_D + ch * 8);
+    *reinterpret_cast<uint4*>(vc + o) =
+        *reinterpret_cast<const uint4*>(row + (long long)(H + G + g) * ATT_D + ch * 8);
+  }
+}
+
+constexpr int DEC_REP_MAX = 8;   // query heads per KV head handled by one CTA
+
+// One CTA per (sequence, KV head, split of the positions 0..lengths[b]): for
+// each query head of the group, the partial softmax (max, sum, weighted sum of
+// values) over its positions.  Warp w takes 32 positions at a time: scores
+// with lanes over positions, then values with lanes over the head width.
+__global__ void __launch_bounds__(128)
+attn_decode_kernel(const bf16* __restrict__ qkv, int H, int G, const int* __restrict__ lengths,
+                   const bf16* __restrict__ kc, const bf16* __restrict__ vc, int max_len, int splits, float sl2,
+                   float* __restrict__ part) {
+  __shared__ float q_s[DEC_REP_MAX][ATT_D];
+  __shared__ float w_m[4][DEC_REP_MAX], w_l[4][DEC_REP_MAX];
+  __shared__ float w_o[4][DEC_REP_MAX][ATT_D];
+  griddep_wait();
+  griddep_launch();
+  const int bg = blockIdx.x, b = bg / G, g = bg % G, split = blockIdx.y;
+  const int rep = H / G;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n = max(0, min(lengths[b] + 1, max_len));   // the appended token included; never past the cache
+  const int per = (n + splits - 1) / splits;
+  const int p0 = split * per, p1 = min(n, p0 + per);
+  const long long W = (long long)(H + 2 * G) * ATT_D;
+  for (int i = threadIdx.x; i < rep * ATT_D; i += 128)
+    q_s[i / ATT_D][i % ATT_D] = __bfloat162float(qkv[b * W + (long long)(g * rep) * ATT_D + i]);
+  __syncthreads();
+  const bf16* kbase = kc + ((long long)b * G + g) * max_len * ATT_D;
+  const bf16* vbase = vc + ((long long)b * G + g) * max_len * ATT_D;
+  float m[DEC_REP_MAX], l[DEC_REP_MAX], acc[DEC_REP_MAX][4];
+#pragma unroll
+  for (int h = 0; h < DEC_REP_MAX; ++h) {
+    m[h] = -INFINITY;
+    l[h] = 0.f;
+    acc[h][0] = acc[h][1] = acc[h][2] = acc[h][3] = 0.f;
+  }
+  for (int c0 = p0 + warp * 32; c0 < p1; c0 += 128) {
+    const int pos = c0 + lane;
+    float sc[DEC_REP_MAX];
+#pragma unroll
+    for (int h = 0; h < DEC_REP_MAX; ++h) sc[h] = 0.f;
+    if (pos < p1) {
+      const uint4* kr = reinterpret_cast<const uint4*>(kbase + (long long)pos * ATT_D);
+#pragma unroll 4
+      for (int ch = 0; ch < 16; ++ch) {
+        const uint4 u = kr[ch];
+        const __nv_bfloat162* kh = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 kf = __bfloat1622float2(kh[i]);
+#pragma unroll
+          for (int h = 0; h < DEC_REP_MAX; ++h)
+            if (h < rep) sc[h] = fmaf(q_s[h][ch * 8 + 2 * i + 1], kf.y, fmaf(q_s[h][ch * 8 + 2 * i], kf.x, sc[h]));
+        }
+      }
+    }
+    float pr[DEC_REP_MAX];
+#pragma unroll
+    for (int h = 0; h < DEC_REP_MAX; ++h) {
+      if (h >= rep) continue;
+      const float s = pos < p1 ? sc[h] * sl2 : -INFINITY;   // log2 units
+      float mx = s;
+#pragma unroll
+      for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      const float mn = fmaxf(m[h], mx);
+      const float corr = ex2(m[h] - mn);   // 0 when m was -inf
+      pr[h] = ex2(s - mn);
+      float sum = pr[h];
+#pragma unroll
+      for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      l[h] = l[h] * corr + sum;
+      m[h] = mn;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[h][i] *= corr;
+    }
+    // values: lane owns dims 4*lane .. 4*lane+3
+    const int cnt = min(32, p1 - c0);
+    for (int k = 0; k < cnt; ++k) {
+      const uint2 u = *reinterpret_cast<const uint2*>(vbase + (long long)(c0 + k) * ATT_D + 4 * lane);
+      const __nv_bfloat162* vh = reinterpret_cast<const __nv_bfloat162*>(&u);
+      const float2 v01 = __bfloat1622float2(vh[0]), v23 = __bfloat1622float2(vh[1]);
+#pragma unroll
+      for (int h = 0; h < DEC_REP_MAX; ++h) {
+        if (h >= rep) continue;
+        const float pk = __shfl_sync(0xffffffffu, pr[h], k);
+        acc[h][0] = fmaf(pk, v01.x, acc[h][0]);
+        acc[h][1] = fmaf(pk, v01.y, acc[h][1]);
+        acc[h][2] = fmaf(pk, v23.x, acc[h][2]);
+        acc[h][3] = fmaf(pk, v23.y, acc[h][3]);
+      }
+    }
+  }
+  // merge the four warps, then write this split's partial per query head
+#pragma unroll
+  for (int h = 0; h < DEC_REP_MAX; ++h) {
+    if (h >= rep) continue;
+    if (lane == 0) {
+      w_m[warp][h] = m[h];
+      w_l[warp][h] = l[h];
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w_o[warp][h][4 * lane + i] = acc[h][i];
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < rep * ATT_D; i += 128) {
+    const int h = i / ATT_D, d = i % ATT_D;
+    float mm = -INFINITY;
+    for (int w = 0; w < 4; ++w) mm = fmaxf(mm, w_m[w][h]);
+    float ls = 0.f, os = 0.f;
+    for (int w = 0; w < 4; ++w) {
+      const float f = w_m[w][h] == -INFINITY ? 0.f : ex2(w_m[w][h] - mm);
+      ls += w_l[w][h] * f;
+      os += w_o[w][h][d] * f;
+    }
+    // part layout: [B*H][splits][D + 2]: o (unnormalised), then max (log2 units), sum
+    float* dst = part + ((long long)(b * H + g * rep + h) * splits + split) * (ATT_D + 2);
+    dst[d] = os;
+    if (d == 0) {
+      dst[ATT_D] = mm;
+      dst[ATT_D + 1] = ls;
+    }
+  }
+}
+
+// o[b, h*D + d] = sum over splits, normalised; then lengths[b] += 1
+__global__ void __launch_bounds__(128)
+attn_combine_kernel(const float* __restrict__ part, int H, int splits, bf16* __restrict__ o, int* __restrict__ lengths) {
+  griddep_wait();
+  griddep_launch();
+  const int bh = blockIdx.x, d = threadIdx.x;
+  const float* src = part + (long long)bh * splits * (ATT_D + 2);
+  float mm = -INFINITY;
+  for (int s = 0; s < splits; ++s) mm = fmaxf(mm, src[s * (ATT_D + 2) + ATT_D]);
+  float ls = 0.f, os = 0.f;
+  for (int s = 0; s < splits; ++s) {
+    const float ms = src[s * (ATT_D + 2) + ATT_D];
+    const float f = ms == -INFINITY ? 0.f : ex2(ms - mm);
+    ls += src[s * (ATT_D + 2) + ATT_D + 1] * f;
+    os += src[s * (ATT_D + 2) + d] * f;
+  }
+  o[(long long)bh * ATT_D + d] = __float2bfloat16_rn(os / ls);
+  __syncthreads();
+  if (d == 0 && bh % H == 0) lengths[bh / H] += 1;
+}
+
+int attn_decode_splits(int B, int G, int max_len) {
+  const int ctas = B * G;
+  int s = (4 * num_sms() + ctas - 1) / ctas;
+  const int cap = (max_len + 255) / 256;   // at least 256 positions per split
+  if (s > cap) s = cap;
+  if (s < 1) s = 1;
+  return s;
+}
+
+jamba_status attn_decode_core(const void* qkv, void* k_cache, void* v_cache, int max_len, int* lengths, float* part,
+                              int splits, void* o, int B, int H, int G, cudaStream_t s) {
+  if (H / G > DEC_REP_MAX) return fail(JAMBA_ERR_UNSUPPORTED, "attention step: at most 8 query heads per KV head");
+  JB_CUDA(launch_pdl(kv_append_kernel, dim3(B), dim3(256), 0, s, reinterpret_cast<const bf16*>(qkv), H, G,
+                     (const int*)lengths, reinterpret_cast<bf16*>(k_cache), reinterpret_cast<bf16*>(v_cache),
+                     max_len));
+  const float sl2 = 1.4426950408889634f / sqrtf((float)ATT_D);
+  JB_CUDA(launch_pdl(attn_decode_kernel, dim3(B * G, splits), dim3(128), 0, s, reinterpret_cast<const bf16*>(qkv),
+                     H, G, (const int*)lengths, reinterpret_cast<const bf16*>(k_cache),
+                     reinterpret_cast<const bf16*>(v_cache), max_len, splits, sl2, part));
+  JB_CUDA(launch_pdl(attn_combine_kernel, dim3(B * H), dim3(ATT_D), 0, s, (const float*)part, H, splits,
+                     reinterpret_cast<bf16*>(o), lengths));
+  return JAMBA_OK;
+}
+
+}  // namespace jb

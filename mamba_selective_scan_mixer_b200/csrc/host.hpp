@@ -137,4 +137,11 @@ jamba_status quantize_int8_rows(const void* w, int dtype, long long rows, int co
 jamba_status moe_combine(const float* Y, const int* inv, const float* w, int T, int K, int dm, const void* residual,
                          void* out, cudaStream_t s);
 
+// ---------------------------------------------------------------- attention
+jamba_status attn_prefill_core(const void* qkv, void* vt, long long ldv, void* o, void* k_cache, void* v_cache,
+                               int max_len, int B, int L, int H, int G, cudaStream_t s);
+int attn_decode_splits(int B, int G, int max_len);
+jamba_status attn_decode_core(const void* qkv, void* k_cache, void* v_cache, int max_len, int* lengths, float* part,
+                              int splits, void* o, int B, int H, int G, cudaStream_t s);
+
 }  // namespace jb

@@ -295,6 +295,64 @@ class MoE:
         return dict(out=out, idx=idx, w=w, offsets=offs, perm=perm)
 
 
+class Attention:
+    """GQA attention layer (prefill and one-token decode) over borrowed weights.
+
+    params: wq [n_heads*head_dim, d_model], wk and wv [n_kv_heads*head_dim,
+    d_model], wo [d_model, n_heads*head_dim]; the q|k|v rows are stacked once
+    into the fused w_qkv the library takes.
+    """
+
+    def __init__(self, params, shape):
+        self.shape = shape
+        _cuda(*params.values())
+        self.w_qkv = torch.cat([params["wq"], params["wk"], params["wv"]], dim=0).contiguous()
+        self.w_o = params["wo"].contiguous()
+        self.cfg = _abi.AttnConfig(shape.d_model, shape.n_heads, shape.n_kv_heads, shape.head_dim,
+                                   _DT[self.w_o.dtype])
+        self.w = _abi.AttnWeights(_p(self.w_qkv), _p(self.w_o))
+        self.ws = _Workspace()
+
+    def new_cache(self, batch, max_len, device=None):
+        """Zeroed K and V caches [batch, n_kv_heads, max_len, head_dim] and int32 lengths [batch]."""
+        dev = device if device is not None else self.w_o.device
+        sh = (batch, self.shape.n_kv_heads, max_len, self.shape.head_dim)
+        return (torch.zeros(sh, dtype=self.w_o.dtype, device=dev), torch.zeros(sh, dtype=self.w_o.dtype, device=dev),
+                torch.zeros(batch, dtype=torch.int32, device=dev))
+
+    def prefill(self, x, residual=None, out=None, k_cache=None, v_cache=None, stream=None):
+        """x [B, L, d_model] -> out; k_cache / v_cache (optional) receive positions 0..L-1."""
+        _cuda(x, residual, out, k_cache, v_cache)
+        _contig(x, "x")
+        B, L, _ = x.shape
+        out = torch.empty_like(x) if out is None else out
+        max_len = k_cache.shape[2] if k_cache is not None else 0
+        n = ctypes.c_size_t()
+        check(lib().jamba_attn_prefill_workspace_size(ctypes.byref(self.cfg), B, L, ctypes.byref(n)))
+        ws = self.ws.get(n.value, x.device)
+        check(lib().jamba_attn_prefill(ctypes.byref(self.cfg), ctypes.byref(self.w), _p(x), _p(residual), _p(out),
+                                       B, L, _p(k_cache), _p(v_cache), max_len, _p(ws), ws.numel(),
+                                       _stream(stream)))
+        return out
+
+    def step(self, x, k_cache, v_cache, lengths, residual=None, out=None, stream=None):
+        """x [B, d_model] at position lengths[b]; appends to the caches and advances lengths."""
+        _cuda(x, k_cache, v_cache, lengths, residual, out)
+        _contig(x, "x")
+        if lengths.dtype != torch.int32:
+            raise ValueError("lengths must be int32")
+        B = x.shape[0]
+        out = torch.empty_like(x) if out is None else out
+        max_len = k_cache.shape[2]
+        n = ctypes.c_size_t()
+        check(lib().jamba_attn_step_workspace_size(ctypes.byref(self.cfg), B, max_len, ctypes.byref(n)))
+        ws = self.ws.get(n.value, x.device)
+        check(lib().jamba_attn_step(ctypes.byref(self.cfg), ctypes.byref(self.w), _p(x), _p(residual), _p(out), B,
+                                    _p(k_cache), _p(v_cache), max_len, _p(lengths), _p(ws), ws.numel(),
+                                    _stream(stream)))
+        return out
+
+
 def layer_pair(mixer, moe, x, g1, g2, eps=1e-6, stream=None):
     """RMSNorm -> Mamba -> residual -> RMSNorm -> MoE -> residual on x [B, L, d_model]."""
     B, L, dm = x.shape
