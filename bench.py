@@ -31,6 +31,7 @@ PREFILL_L = 131072
 DECODE_B, DECODE_PREFILL, DECODE_STEPS = 64, 2048, 1024
 SCAN_L, SCAN_DI = 131072, 8192
 PAIR_B, PAIR_L = 4, 8192
+ATTN_L = 32768
 METRIC = "Mamba-layer tokens/s (prefill 128K, decode) at d_model=4096; scan HBM GB/s vs peak"
 # DRAM bytes (read + write) of one in_proj launch at 131072 tokens: ncu capture at 16384 tokens
 # (1.209 GB read + 0.514 GB written, see profiles/in_proj_gemm_traffic.md) scaled by 8, since
@@ -46,12 +47,13 @@ def parse():
     ap.add_argument("--impl", default="product", choices=["product", "reference"])
     ap.add_argument("--quick", action="store_true", help="skip the side measurements")
     ap.add_argument("--only", default="all",
-                    help="comma list of parts to run (prefill,gemm,scan,decode,pair,moe8,moe8dec,e2e,cpu); "
+                    help="comma list of parts to run (prefill,gemm,scan,decode,pair,moe8,moe8dec,attn,e2e,cpu); "
                          "for profiling")
     ap.add_argument("--seqlen", type=int, default=PREFILL_L, help="prefill tokens")
     ap.add_argument("--scan-seqlen", type=int, default=SCAN_L)
     ap.add_argument("--decode-steps", type=int, default=DECODE_STEPS)
     ap.add_argument("--pair-seqlen", type=int, default=PAIR_L)
+    ap.add_argument("--attn-seqlen", type=int, default=ATTN_L)
     return ap.parse_args()
 
 
@@ -209,8 +211,8 @@ def cpu_baseline(sample_tokens=1024):
 # ------------------------------------------------------------------ product arm
 def run_product(args):
     import mamba_selective_scan_mixer_b200 as J
-    from synthetic import MoEShape, block_norm_params, decode_inputs, mamba_input, mamba_params, moe_input, \
-        moe_params, scan_inputs, workload
+    from synthetic import AttnShape, MoEShape, attn_input, attn_params, block_norm_params, decode_inputs, \
+        mamba_input, mamba_params, moe_input, moe_params, scan_inputs, workload
 
     world, rank, local = dist_setup(args)
     dev = torch.device("cuda", local)
@@ -219,7 +221,7 @@ def run_product(args):
     L = args.seqlen
     stream = torch.cuda.current_stream(dev)
 
-    parts = {"prefill", "gemm", "scan", "decode", "pair", "moe8", "e2e", "cpu"} if args.only == "all" else \
+    parts = {"prefill", "gemm", "scan", "decode", "pair", "moe8", "attn", "e2e", "cpu"} if args.only == "all" else \
         set(args.only.split(","))
     if args.quick:
         parts &= {"prefill"}
@@ -394,6 +396,56 @@ def run_product(args):
         del mp, moe, xp
         J.device_status()
 
+    if rank == 0 and "attn" in parts:
+        # the block's GQA attention layer: prefill of 32768 tokens, and a batch-64 decode step
+        # over 2048-token caches
+        ash = AttnShape()
+        AL = args.attn_seqlen
+        att = J.Attention(attn_params(ash, seed=0, device=dev), ash)
+        xa = attn_input(ash, 1, AL, seed=5, device=dev)
+        outa = torch.empty_like(xa)
+        fa = lambda: att.prefill(xa, out=outa)
+        fa()
+        torch.cuda.synchronize()
+        ams, _ = event_time_ms(fa, 3, stream, flush)
+        H, G, D, dm = ash.n_heads, ash.n_kv_heads, ash.head_dim, ash.d_model
+        core = 2.0 * AL * AL * H * D                   # causal: QK^T and PV over the lower triangle
+        proj = 2.0 * AL * dm * (H + 2 * G) * D + 2.0 * AL * H * D * dm
+        del xa, outa
+        DB, DL, DS = 64, 2048, 32
+        kc, vc, lens = att.new_cache(DB, DL + DS)
+        kc.normal_()
+        vc.normal_()
+        xd = attn_input(ash, DB, 1, seed=6, device=dev)[:, 0].contiguous()
+        od = torch.empty_like(xd)
+
+        def dec():
+            for _ in range(DS):
+                att.step(xd, kc, vc, lens, out=od)
+
+        lens.fill_(DL)
+        dec()
+        torch.cuda.synchronize()
+        dts = []
+        for _ in range(3):
+            lens.fill_(DL)
+            dts.append(event_time_ms(dec, 1, stream, flush)[0])
+        dus = 1e3 * min(dts) / DS
+        kv_bytes = 2.0 * DB * G * (DL + DS / 2 + 1) * D * 2
+        w_bytes = 2.0 * ((H + 2 * G) * D * dm + dm * H * D)
+        res["attention"] = {
+            "workload": "attn_32k: GQA attention layer (32 query heads over 8 KV heads of 128, d_model 4096, no "
+                        "positional encoding), causal prefill of %d tokens; decode: batch 64 over %d-token caches" %
+                        (AL, DL),
+            "prefill_ms": round(ams, 3), "prefill_tokens/s": round(AL / (ams / 1e3), 1),
+            "prefill_TFLOP/s": round((core + proj) / (ams / 1e3) / 1e12, 1),
+            "prefill_frac_of_bf16_sustained": round((core + proj) / (ams / 1e3) / 1e12 / pk["bf16_sus"], 4),
+            "prefill_flops": {"attention_core": core, "projections": proj},
+            "decode_us_per_step": round(dus, 2),
+            "decode_GB/s": round((kv_bytes + w_bytes) / (dus / 1e6) / 1e9, 1),
+            "decode_frac_of_measured_hbm": round((kv_bytes + w_bytes) / (dus / 1e6) / 1e9 / pk["hbm"], 4)}
+        del att, kc, vc
+        J.device_status()
     if rank == 0 and "moe8dec" in parts:
         # ExpertsInt8 decode batch alone, with only the int8 experts resident (a few GB): the
         # small case the expert-kernel profiles are taken on

@@ -360,89 +360,116 @@ kv_append_kernel(const bf16* __restrict__ qkv, int H, int G, const int* __restri
   }
 }
 
-constexpr int DEC_REP_MAX = 8;   // query heads per KV head handled by one CTA
+constexpr int DEC_REP = 4;   // query heads per KV head in the decode kernel (8 KV heads under 32 query heads)
 
 // One CTA per (sequence, KV head, split of the positions 0..lengths[b]): for
-// each query head of the group, the partial softmax (max, sum, weighted sum of
-// values) over its positions.  Warp w takes 32 positions at a time: scores
-// with lanes over positions, then values with lanes over the head width.
+// each of the group's query heads, the partial softmax (max, sum, weighted
+// sum of values) over its positions.  A warp takes 16 consecutive positions
+// at a time, their value rows requested together with the keys.  Scores:
+// each load instruction covers two whole key rows (lanes 0-15 one row, 16-31
+// the next, 8 dims per lane), the query slice stays in registers, and each
+// row's dot product is reduced across its 16 lanes.  Values: lanes over the
+// head width (4 dims each), the weight of each row broadcast from the lane
+// holding it.
 __global__ void __launch_bounds__(128)
 attn_decode_kernel(const bf16* __restrict__ qkv, int H, int G, const int* __restrict__ lengths,
                    const bf16* __restrict__ kc, const bf16* __restrict__ vc, int max_len, int splits, float sl2,
                    float* __restrict__ part) {
-  __shared__ float q_s[DEC_REP_MAX][ATT_D];
-  __shared__ float w_m[4][DEC_REP_MAX], w_l[4][DEC_REP_MAX];
-  __shared__ float w_o[4][DEC_REP_MAX][ATT_D];
+  __shared__ float w_m[4][DEC_REP], w_l[4][DEC_REP];
+  __shared__ float w_o[4][DEC_REP][ATT_D];
   griddep_wait();
   griddep_launch();
   const int bg = blockIdx.x, b = bg / G, g = bg % G, split = blockIdx.y;
-  const int rep = H / G;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int half = lane >> 4, hl = lane & 15;
   const int n = max(0, min(lengths[b] + 1, max_len));   // the appended token included; never past the cache
   const int per = (n + splits - 1) / splits;
   const int p0 = split * per, p1 = min(n, p0 + per);
   const long long W = (long long)(H + 2 * G) * ATT_D;
-  for (int i = threadIdx.x; i < rep * ATT_D; i += 128)
-    q_s[i / ATT_D][i % ATT_D] = __bfloat162float(qkv[b * W + (long long)(g * rep) * ATT_D + i]);
-  __syncthreads();
+  // this lane's 8 dims of each query head, pre-scaled to log2 units
+  float q[DEC_REP][8];
+#pragma unroll
+  for (int h = 0; h < DEC_REP; ++h) {
+    const uint4 u = *reinterpret_cast<const uint4*>(qkv + b * W + (long long)(g * DEC_REP + h) * ATT_D + hl * 8);
+    const __nv_bfloat162* qh = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(qh[i]);
+      q[h][2 * i] = f.x * sl2;
+      q[h][2 * i + 1] = f.y * sl2;
+    }
+  }
   const bf16* kbase = kc + ((long long)b * G + g) * max_len * ATT_D;
   const bf16* vbase = vc + ((long long)b * G + g) * max_len * ATT_D;
-  float m[DEC_REP_MAX], l[DEC_REP_MAX], acc[DEC_REP_MAX][4];
+  float m[DEC_REP], l[DEC_REP], acc[DEC_REP][4];
 #pragma unroll
-  for (int h = 0; h < DEC_REP_MAX; ++h) {
+  for (int h = 0; h < DEC_REP; ++h) {
     m[h] = -INFINITY;
     l[h] = 0.f;
     acc[h][0] = acc[h][1] = acc[h][2] = acc[h][3] = 0.f;
   }
-  for (int c0 = p0 + warp * 32; c0 < p1; c0 += 128) {
-    const int pos = c0 + lane;
-    float sc[DEC_REP_MAX];
+  constexpr int RW = 16;   // rows per warp and step: 4 KB of keys and 4 KB of values
+  for (int c0 = p0 + warp * RW; c0 < p1; c0 += 4 * RW) {
+    // this lane's 4 dims of the step's value rows, requested before the scores so the loads overlap
+    uint2 vr[RW];
 #pragma unroll
-    for (int h = 0; h < DEC_REP_MAX; ++h) sc[h] = 0.f;
-    if (pos < p1) {
-      const uint4* kr = reinterpret_cast<const uint4*>(kbase + (long long)pos * ATT_D);
-#pragma unroll 4
-      for (int ch = 0; ch < 16; ++ch) {
-        const uint4 u = kr[ch];
-        const __nv_bfloat162* kh = reinterpret_cast<const __nv_bfloat162*>(&u);
+    for (int k = 0; k < RW; ++k)
+      vr[k] = c0 + k < p1 ? *reinterpret_cast<const uint2*>(vbase + (long long)(c0 + k) * ATT_D + 4 * lane)
+                          : make_uint2(0, 0);
+    // scores of rows c0 + 2i + half, every lane of a half holding its row's value
+    float sc[RW / 2][DEC_REP];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 kf = __bfloat1622float2(kh[i]);
+    for (int i = 0; i < RW / 2; ++i) {
+      const int pos = c0 + 2 * i + half;
+      uint4 u = make_uint4(0, 0, 0, 0);
+      if (pos < p1) u = *reinterpret_cast<const uint4*>(kbase + (long long)pos * ATT_D + hl * 8);
+      const __nv_bfloat162* kh = reinterpret_cast<const __nv_bfloat162*>(&u);
+      float kf[8];
 #pragma unroll
-          for (int h = 0; h < DEC_REP_MAX; ++h)
-            if (h < rep) sc[h] = fmaf(q_s[h][ch * 8 + 2 * i + 1], kf.y, fmaf(q_s[h][ch * 8 + 2 * i], kf.x, sc[h]));
-        }
+      for (int t = 0; t < 4; ++t) {
+        const float2 f = __bfloat1622float2(kh[t]);
+        kf[2 * t] = f.x;
+        kf[2 * t + 1] = f.y;
+      }
+#pragma unroll
+      for (int h = 0; h < DEC_REP; ++h) {
+        float d = 0.f;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) d = fmaf(q[h][t], kf[t], d);
+#pragma unroll
+        for (int o = 8; o; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+        sc[i][h] = pos < p1 ? d : -INFINITY;
       }
     }
-    float pr[DEC_REP_MAX];
+    // online softmax; the scores become the weights in place
 #pragma unroll
-    for (int h = 0; h < DEC_REP_MAX; ++h) {
-      if (h >= rep) continue;
-      const float s = pos < p1 ? sc[h] * sl2 : -INFINITY;   // log2 units
-      float mx = s;
+    for (int h = 0; h < DEC_REP; ++h) {
+      float mx = sc[0][h];
 #pragma unroll
-      for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      const float mn = fmaxf(m[h], mx);
-      const float corr = ex2(m[h] - mn);   // 0 when m was -inf
-      pr[h] = ex2(s - mn);
-      float sum = pr[h];
+      for (int i = 1; i < RW / 2; ++i) mx = fmaxf(mx, sc[i][h]);
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      const float mn = fmaxf(m[h], mx);                   // finite: row c0 is valid
+      const float corr = ex2(m[h] - mn);                  // 0 when m was -inf
+      float sum = 0.f;
 #pragma unroll
-      for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      for (int i = 0; i < RW / 2; ++i) {
+        sc[i][h] = ex2(sc[i][h] - mn);
+        sum += sc[i][h];
+      }
+      sum += __shfl_xor_sync(0xffffffffu, sum, 16);
       l[h] = l[h] * corr + sum;
       m[h] = mn;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc[h][i] *= corr;
+      for (int t = 0; t < 4; ++t) acc[h][t] *= corr;
     }
-    // values: lane owns dims 4*lane .. 4*lane+3
-    const int cnt = min(32, p1 - c0);
-    for (int k = 0; k < cnt; ++k) {
-      const uint2 u = *reinterpret_cast<const uint2*>(vbase + (long long)(c0 + k) * ATT_D + 4 * lane);
-      const __nv_bfloat162* vh = reinterpret_cast<const __nv_bfloat162*>(&u);
+    // values: row c0 + k, weight sc[k / 2] from a lane of half k % 2 (rows past the end carry 0)
+#pragma unroll
+    for (int k = 0; k < RW; ++k) {
+      const __nv_bfloat162* vh = reinterpret_cast<const __nv_bfloat162*>(&vr[k]);
       const float2 v01 = __bfloat1622float2(vh[0]), v23 = __bfloat1622float2(vh[1]);
 #pragma unroll
-      for (int h = 0; h < DEC_REP_MAX; ++h) {
-        if (h >= rep) continue;
-        const float pk = __shfl_sync(0xffffffffu, pr[h], k);
+      for (int h = 0; h < DEC_REP; ++h) {
+        const float pk = __shfl_sync(0xffffffffu, sc[k >> 1][h], (k & 1) * 16);
         acc[h][0] = fmaf(pk, v01.x, acc[h][0]);
         acc[h][1] = fmaf(pk, v01.y, acc[h][1]);
         acc[h][2] = fmaf(pk, v23.x, acc[h][2]);
@@ -452,17 +479,16 @@ attn_decode_kernel(const bf16* __restrict__ qkv, int H, int G, const int* __rest
   }
   // merge the four warps, then write this split's partial per query head
 #pragma unroll
-  for (int h = 0; h < DEC_REP_MAX; ++h) {
-    if (h >= rep) continue;
+  for (int h = 0; h < DEC_REP; ++h) {
     if (lane == 0) {
       w_m[warp][h] = m[h];
       w_l[warp][h] = l[h];
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) w_o[warp][h][4 * lane + i] = acc[h][i];
+    for (int t = 0; t < 4; ++t) w_o[warp][h][4 * lane + t] = acc[h][t];
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < rep * ATT_D; i += 128) {
+  for (int i = threadIdx.x; i < DEC_REP * ATT_D; i += 128) {
     const int h = i / ATT_D, d = i % ATT_D;
     float mm = -INFINITY;
     for (int w = 0; w < 4; ++w) mm = fmaxf(mm, w_m[w][h]);
@@ -473,7 +499,7 @@ attn_decode_kernel(const bf16* __restrict__ qkv, int H, int G, const int* __rest
       os += w_o[w][h][d] * f;
     }
     // part layout: [B*H][splits][D + 2]: o (unnormalised), then max (log2 units), sum
-    float* dst = part + ((long long)(b * H + g * rep + h) * splits + split) * (ATT_D + 2);
+    float* dst = part + ((long long)(b * H + g * DEC_REP + h) * splits + split) * (ATT_D + 2);
     dst[d] = os;
     if (d == 0) {
       dst[ATT_D] = mm;
@@ -504,8 +530,10 @@ attn_combine_kernel(const float* __restrict__ part, int H, int splits, bf16* __r
 }
 
 int attn_decode_splits(int B, int G, int max_len) {
+  // enough CTAs for ~16 per SM over the run (three are resident at a time),
+  // so the last wave is a small part of the whole
   const int ctas = B * G;
-  int s = (4 * num_sms() + ctas - 1) / ctas;
+  int s = (16 * num_sms() + ctas - 1) / ctas;
   const int cap = (max_len + 255) / 256;   // at least 256 positions per split
   if (s > cap) s = cap;
   if (s < 1) s = 1;
@@ -514,7 +542,7 @@ int attn_decode_splits(int B, int G, int max_len) {
 
 jamba_status attn_decode_core(const void* qkv, void* k_cache, void* v_cache, int max_len, int* lengths, float* part,
                               int splits, void* o, int B, int H, int G, cudaStream_t s) {
-  if (H / G > DEC_REP_MAX) return fail(JAMBA_ERR_UNSUPPORTED, "attention step: at most 8 query heads per KV head");
+  if (H / G != DEC_REP) return fail(JAMBA_ERR_UNSUPPORTED, "attention step: 4 query heads per KV head");
   JB_CUDA(launch_pdl(kv_append_kernel, dim3(B), dim3(256), 0, s, reinterpret_cast<const bf16*>(qkv), H, G,
                      (const int*)lengths, reinterpret_cast<bf16*>(k_cache), reinterpret_cast<bf16*>(v_cache),
                      max_len));
