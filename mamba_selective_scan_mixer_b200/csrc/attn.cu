@@ -13,7 +13,8 @@
 // kernel fills the KV cache.  flash_attn_kernel: one CTA per (sequence,
 // query head, 128-query block), heavy (late) blocks first; per 128-key block
 // S = Q K^T (tcgen05, fp32 in TMEM, double-buffered), an online softmax by
-// four warps (thread = query row; the running maximum is raised lazily, only
+// eight warps (two threads per query row, 64 keys each, meeting in shared
+// memory for the row maximum; the running maximum is raised lazily, only
 // when a row's maximum grows by more than 2^8, and O is then rescaled in
 // TMEM), P in bf16 through swizzled shared memory, O += P V (tcgen05, fp32
 // in TMEM).  Every wait is bounded (see common.cuh).
@@ -32,7 +33,8 @@ constexpr int ATT_D = 128;       // head width (the only one supported)
 constexpr int ATT_BQ = 128;      // query rows per CTA
 constexpr int ATT_BK = 128;      // keys per block
 constexpr int ATT_KVST = 2;      // K / V^T ring stages
-constexpr int ATT_THREADS = 192; // producer, MMA, four softmax warps
+constexpr int ATT_SM_WARPS = 8;  // softmax: two warps per TMEM lane quarter, 64 keys each
+constexpr int ATT_THREADS = 32 * (2 + ATT_SM_WARPS);
 
 struct AttnSmem {
   static constexpr uint32_t SUB = 128 * 128;                 // 128 rows x 64 bf16, swizzled
@@ -40,9 +42,15 @@ struct AttnSmem {
   static constexpr uint32_t KV_OFF = 2 * SUB;                // per stage: K (dims) x2, V^T (keys) x2
   static constexpr uint32_t KV_STAGE = 4 * SUB;
   static constexpr uint32_t P_OFF = KV_OFF + ATT_KVST * KV_STAGE;   // P: keys 0-63 | 64-127
-  static constexpr uint32_t BAR_OFF = P_OFF + 2 * SUB;
+  static constexpr uint32_t RED_OFF = P_OFF + 2 * SUB;        // row maxima / sums exchanged by the two halves
+  static constexpr uint32_t BAR_OFF = RED_OFF + 2 * 2 * 128 * 4;
   static constexpr uint32_t BYTES = BAR_OFF + 256 + 1024;
 };
+
+// named barrier over the softmax warps only
+__device__ __forceinline__ void softmax_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(32 * ATT_SM_WARPS) : "memory");
+}
 
 struct AttnParams {
   int B, L, H, G, rep, nq;
@@ -78,9 +86,9 @@ flash_attn_kernel(const __grid_constant__ CUtensorMap tmQK, const __grid_constan
       mbar_init(kv_full0 + 8 * i, 1);
       mbar_init(kv_empty0 + 8 * i, 1);
       mbar_init(s_full0 + 8 * i, 1);
-      mbar_init(s_free0 + 8 * i, 4);
+      mbar_init(s_free0 + 8 * i, ATT_SM_WARPS);
     }
-    mbar_init(p_full, 4);
+    mbar_init(p_full, ATT_SM_WARPS);
     mbar_init(pv_done, 1);
     mbar_init(drain, 1);
     mbar_fence_init();
@@ -156,31 +164,42 @@ flash_attn_kernel(const __grid_constant__ CUtensorMap tmQK, const __grid_constan
       mbar_wait(drain, 0, p.err);
     }
   } else {
-    // softmax: thread = query row r of this warp's TMEM lane quarter
-    const int q4 = warp & 3;
+    // softmax: query row r of this warp's TMEM lane quarter, keys half*64 .. half*64+63 of
+    // each block (and the same 64 columns of O); the two halves of a row meet in shared memory
+    const int q4 = warp & 3, half = (warp - 2) >> 2;
     const int r = q4 * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    float* red = reinterpret_cast<float*>(smem + S::RED_OFF);   // [2 parities][2 halves][128 rows]
     float m = 0.f, l = 0.f;
     bool ok = true;
+    // After a failed wait the loop still runs to its end (on whatever the buffers hold), so
+    // that every softmax warp reaches every named barrier; the error is already latched.
     for (int j = 0; j < nkv; ++j) {
       const int buf = j & 1;
-      if (!mbar_wait(s_full0 + 8 * buf, (j >> 1) & 1, p.err)) { ok = false; break; }
+      ok = mbar_wait(s_full0 + 8 * buf, (j >> 1) & 1, p.err) && ok;
       tc_fence_after();
-      float s[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + lane_off + buf * 128 + 32 * c, s + 32 * c);
+      float s[64];
+      tmem_ld32(tS + lane_off + buf * 128 + half * 64, s);
+      tmem_ld32(tS + lane_off + buf * 128 + half * 64 + 32, s + 32);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(s_free0 + 8 * buf);
       if (j == qi) {   // diagonal block: key c is visible to row r when c <= r
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c > r) s[c] = -INFINITY;
+        for (int c = 0; c < 64; ++c)
+          if (half * 64 + c > r) s[c] = -INFINITY;
       }
-      float mx = s[0];
+      float mx8[8];
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+      for (int t = 0; t < 8; ++t) mx8[t] = s[t];
+#pragma unroll
+      for (int c = 8; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      red[(buf * 2 + half) * 128 + r] = mx;
+      softmax_sync();
+      mx = fmaxf(mx, red[(buf * 2 + (half ^ 1)) * 128 + r]);   // finite: key 0 of the block is visible
       const float mnew = mx * p.sl2;
       float corr = 1.f;
       if (j == 0) {
@@ -189,65 +208,69 @@ flash_attn_kernel(const __grid_constant__ CUtensorMap tmQK, const __grid_constan
         corr = ex2(m - mnew);
         m = mnew;
       }
-      float sum = 0.f;
+      float sm8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
+      for (int c = 0; c < 64; ++c) {
         s[c] = ex2(fmaf(s[c], p.sl2, -m));
-        sum += s[c];
+        sm8[c & 7] += s[c];
       }
-      l = l * corr + sum;
+      l = l * corr + (((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7])));
       if (j > 0) {
         // P_{j-1} and the O it fed are done: P may be overwritten and O rescaled
-        if (!mbar_wait(pv_done, (j - 1) & 1, p.err)) { ok = false; break; }
+        ok = mbar_wait(pv_done, (j - 1) & 1, p.err) && ok;
         tc_fence_after();
         if (__any_sync(0xffffffffu, corr != 1.f)) {
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
+          for (int c = 0; c < 2; ++c) {
             float o[32];
-            tmem_ld32(tO + lane_off + 32 * c, o);
+            tmem_ld32(tO + lane_off + half * 64 + 32 * c, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= corr;
-            tmem_st32(tO + lane_off + 32 * c, o);
+            for (int t = 0; t < 32; ++t) o[t] *= corr;
+            tmem_st32(tO + lane_off + half * 64 + 32 * c, o);
           }
           tmem_wait_st();
         }
       }
-      // P row r (bf16) into the two swizzled sub-tiles: 16-byte chunk k of row r at (k ^ (r & 7))
-      uint8_t* prow = smem + S::P_OFF + r * 128;
+      // P row r, keys half*64.. (bf16): sub-tile `half`, 16-byte chunk k of row r at (k ^ (r & 7))
+      uint8_t* prow = smem + S::P_OFF + half * S::SUB + r * 128;
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
+      for (int k = 0; k < 8; ++k) {
         uint4 u;
         __nv_bfloat162* hh = reinterpret_cast<__nv_bfloat162*>(&u);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) hh[i] = __floats2bfloat162_rn(s[8 * k + 2 * i], s[8 * k + 2 * i + 1]);
-        *reinterpret_cast<uint4*>(prow + (k >> 3) * S::SUB + (((k & 7) ^ (r & 7)) << 4)) = u;
+        for (int t = 0; t < 4; ++t) hh[t] = __floats2bfloat162_rn(s[8 * k + 2 * t], s[8 * k + 2 * t + 1]);
+        *reinterpret_cast<uint4*>(prow + ((k ^ (r & 7)) << 4)) = u;
       }
       fence_async_shared();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
     }
+    // the row sum is split over the two halves (same reference m, same corrections); the
+    // parity slot the last block did not use is free (its reads came before the last sync)
+    const float lpart = l;
+    const int fb = nkv & 1;
+    red[(fb * 2 + half) * 128 + r] = lpart;
+    softmax_sync();
+    l = lpart + red[(fb * 2 + (half ^ 1)) * 128 + r];
     if (ok && mbar_wait(pv_done, (nkv - 1) & 1, p.err)) {
       tc_fence_after();
       const float inv = 1.f / l;
       const int row = qi * ATT_BQ + r;
-      bf16* dst = p.o + (long long)(b * p.L + row) * p.ldo + h * ATT_D;
+      bf16* dst = p.o + (long long)(b * p.L + row) * p.ldo + h * ATT_D + half * 64;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         float o[32];
-        tmem_ld32(tO + lane_off + 32 * c, o);
+        tmem_ld32(tO + lane_off + half * 64 + 32 * c, o);
         tmem_wait_ld();
         if (row < p.L) {
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            float w[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) w[i] = o[8 * k + i] * inv;
             uint4 u;
             __nv_bfloat162* hh = reinterpret_cast<__nv_bfloat162*>(&u);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) hh[i] = __floats2bfloat162_rn(w[2 * i], w[2 * i + 1]);
+            for (int t = 0; t < 4; ++t) hh[t] = __floats2bfloat162_rn(o[8 * k + 2 * t] * inv, o[8 * k + 2 * t + 1] * inv);
             *reinterpret_cast<uint4*>(dst + 32 * c + 8 * k) = u;
           }
         }
