@@ -176,7 +176,7 @@ flash_attn_kernel(const __grid_constant__ CUtensorMap tmQK, const __grid_constan
     // that every softmax warp reaches every named barrier; the error is already latched.
     for (int j = 0; j < nkv; ++j) {
       const int buf = j & 1;
-      ok = mbar_wait(s_full0 + 8 * buf, (j >> 1) & 1, p.err) && ok;
+      ok = mbar_wait_warp(s_full0 + 8 * buf, (j >> 1) & 1, p.err) && ok;
       tc_fence_after();
       float s[64];
       tmem_ld32(tS + lane_off + buf * 128 + half * 64, s);
@@ -217,7 +217,7 @@ flash_attn_kernel(const __grid_constant__ CUtensorMap tmQK, const __grid_constan
       l = l * corr + (((sm8[0] + sm8[1]) + (sm8[2] + sm8[3])) + ((sm8[4] + sm8[5]) + (sm8[6] + sm8[7])));
       if (j > 0) {
         // P_{j-1} and the O it fed are done: P may be overwritten and O rescaled
-        ok = mbar_wait(pv_done, (j - 1) & 1, p.err) && ok;
+        ok = mbar_wait_warp(pv_done, (j - 1) & 1, p.err) && ok;
         tc_fence_after();
         if (__any_sync(0xffffffffu, corr != 1.f)) {
 #pragma unroll 1
@@ -254,7 +254,7 @@ flash_attn_kernel(const __grid_constant__ CUtensorMap tmQK, const __grid_constan
     red[(fb * 2 + half) * 128 + r] = lpart;
     softmax_sync();
     l = lpart + red[(fb * 2 + (half ^ 1)) * 128 + r];
-    if (ok && mbar_wait(pv_done, (nkv - 1) & 1, p.err)) {
+    if (ok && mbar_wait_warp(pv_done, (nkv - 1) & 1, p.err)) {
       tc_fence_after();
       const float inv = 1.f / l;
       const int row = qi * ATT_BQ + r;
@@ -284,6 +284,295 @@ flash_attn_kernel(const __grid_constant__ CUtensorMap tmQK, const __grid_constan
     tmem_dealloc(tbase, 512);
   }
 }
+
+// Two query heads of one KV group per CTA (used when the group size is even):
+// tiles A and B share every K and V^T tile, and the tensor core alternates
+// between them so that one tile's softmax runs while the other's products
+// do.  MMA order per key block j: O_A += P_A V_j, S_A(j+1) = Q_A K_{j+1}^T,
+// O_B += P_B V_j, S_B(j+1).  K_j and V^T_j are separate 32 KB items of a
+// three-slot ring (K_0, V_0, K_1, V_1, ...).  Softmax: four warps per tile,
+// thread = query row, the running maximum raised lazily as above.
+constexpr int ATT2_THREADS = 320;   // producer, MMA, 4 + 4 softmax warps
+
+struct Attn2Smem {
+  static constexpr uint32_t SUB = 128 * 128;
+  static constexpr uint32_t Q_OFF = 0;            // Q_A (2 sub-tiles), Q_B (2)
+  static constexpr uint32_t P_OFF = 4 * SUB;      // P_A (2), P_B (2)
+  static constexpr uint32_t KV_OFF = 8 * SUB;     // 3 slots x 2 sub-tiles
+  static constexpr int SLOTS = 3;
+  static constexpr uint32_t BAR_OFF = KV_OFF + SLOTS * 2 * SUB;
+  static constexpr uint32_t BYTES = BAR_OFF + 256 + 1024;
+};
+
+__global__ void __launch_bounds__(ATT2_THREADS, 1)
+flash_attn2_kernel(const __grid_constant__ CUtensorMap tmQK, const __grid_constant__ CUtensorMap tmVt,
+                   const AttnParams p) {
+  using S = Attn2Smem;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::BAR_OFF);
+  const uint32_t q_full = smem_u32(bars);
+  const uint32_t kv_full0 = smem_u32(bars + 1), kv_empty0 = smem_u32(bars + 4);
+  // per tile t: s_full, s_free, p_full, pv_done at slots 7 + 4t ..
+  const uint32_t tb0 = smem_u32(bars + 7);
+  const uint32_t drain = smem_u32(bars + 15);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 16);
+#define S_FULL(t) (tb0 + 32 * (t))
+#define S_FREE(t) (tb0 + 32 * (t) + 8)
+#define P_FULL(t) (tb0 + 32 * (t) + 16)
+#define PV_DONE(t) (tb0 + 32 * (t) + 24)
+
+  const int HP = p.H / 2;
+  const int bp = blockIdx.x % (p.B * HP);
+  const int qi = p.nq - 1 - (int)(blockIdx.x / (p.B * HP));
+  const int b = bp / HP, h0 = 2 * (bp % HP), g = h0 / p.rep;
+  const int nkv = qi + 1;
+  const int row0 = b * p.L + qi * ATT_BQ;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (warp == 0 && lane == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < S::SLOTS; ++i) {
+      mbar_init(kv_full0 + 8 * i, 1);
+      mbar_init(kv_empty0 + 8 * i, 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(S_FULL(t), 1);
+      mbar_init(S_FREE(t), 4);
+      mbar_init(P_FULL(t), 4);
+      mbar_init(PV_DONE(t), 1);
+    }
+    mbar_init(drain, 1);
+    mbar_fence_init();
+    tma_prefetch(&tmQK);
+    tma_prefetch(&tmVt);
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_holder), 512);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_holder;   // tile t: S at 256 t, O at 256 t + 128
+  griddep_launch();
+  griddep_wait();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_tx(q_full, 4 * S::SUB);
+      for (int t = 0; t < 2; ++t)
+        for (int k = 0; k < 2; ++k)
+          tma_load_2d(smem_u32(smem + S::Q_OFF + (2 * t + k) * S::SUB), &tmQK, q_full, (h0 + t) * ATT_D + 64 * k,
+                      row0);
+      const int kcol = (p.H + g) * ATT_D, vrow = (b * p.G + g) * ATT_D;
+      for (int item = 0; item < 2 * nkv; ++item) {
+        const int slot = item % S::SLOTS, j = item >> 1;
+        if (!mbar_wait(kv_empty0 + 8 * slot, ((item / S::SLOTS) & 1) ^ 1, p.err)) break;
+        const uint32_t fb = kv_full0 + 8 * slot;
+        const uint32_t dst = smem_u32(smem + S::KV_OFF + slot * 2 * S::SUB);
+        mbar_arrive_tx(fb, 2 * S::SUB);
+        if ((item & 1) == 0) {   // K_j: keys 128j.., dims 0-63 | 64-127
+          tma_load_2d(dst, &tmQK, fb, kcol, b * p.L + j * ATT_BK);
+          tma_load_2d(dst + S::SUB, &tmQK, fb, kcol + 64, b * p.L + j * ATT_BK);
+        } else {                 // V^T_j: dims 0-127, keys 128j.. | +64
+          tma_load_2d(dst, &tmVt, fb, j * ATT_BK, vrow);
+          tma_load_2d(dst + S::SUB, &tmVt, fb, j * ATT_BK + 64, vrow);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_bf16(128, 128);
+      auto slot_of = [](int item) { return item % S::SLOTS; };
+      auto ph_of = [](int item) { return (uint32_t)((item / S::SLOTS) & 1); };
+      auto issue_s = [&](int t, int j) {
+        const uint32_t kb = smem_u32(smem + S::KV_OFF + slot_of(2 * j) * 2 * S::SUB);
+        const uint32_t qb = smem_u32(smem + S::Q_OFF + 2 * t * S::SUB);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_bf16(tbase + 256 * t, sw128_desc(qb + (kk >> 2) * S::SUB) + 2 * (kk & 3),
+                    sw128_desc(kb + (kk >> 2) * S::SUB) + 2 * (kk & 3), IDESC, kk > 0 ? 1u : 0u);
+        umma_commit(S_FULL(t));
+      };
+      auto issue_pv = [&](int t, int j) {
+        const uint32_t vb = smem_u32(smem + S::KV_OFF + slot_of(2 * j + 1) * 2 * S::SUB);
+        const uint32_t pb = smem_u32(smem + S::P_OFF + 2 * t * S::SUB);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_bf16(tbase + 256 * t + 128, sw128_desc(pb + (kk >> 2) * S::SUB) + 2 * (kk & 3),
+                    sw128_desc(vb + (kk >> 2) * S::SUB) + 2 * (kk & 3), IDESC, (j > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(PV_DONE(t));
+      };
+      bool ok = mbar_wait(q_full, 0, p.err) && mbar_wait(kv_full0 + 8 * slot_of(0), ph_of(0), p.err);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+        umma_commit(kv_empty0 + 8 * slot_of(0));
+      }
+      for (int j = 0; j < nkv && ok; ++j) {
+        const uint32_t par = j & 1;
+        const bool more = j + 1 < nkv;
+        if (!mbar_wait(P_FULL(0), par, p.err) || !mbar_wait(kv_full0 + 8 * slot_of(2 * j + 1), ph_of(2 * j + 1), p.err)) break;
+        tc_fence_after();
+        issue_pv(0, j);
+        if (more) {
+          if (!mbar_wait(kv_full0 + 8 * slot_of(2 * j + 2), ph_of(2 * j + 2), p.err) ||
+              !mbar_wait(S_FREE(0), par, p.err)) break;
+          tc_fence_after();
+          issue_s(0, j + 1);
+        }
+        if (!mbar_wait(P_FULL(1), par, p.err)) break;
+        tc_fence_after();
+        issue_pv(1, j);
+        umma_commit(kv_empty0 + 8 * slot_of(2 * j + 1));
+        if (more) {
+          if (!mbar_wait(S_FREE(1), par, p.err)) break;
+          tc_fence_after();
+          issue_s(1, j + 1);
+          umma_commit(kv_empty0 + 8 * slot_of(2 * j + 2));
+        }
+      }
+      umma_commit(drain);
+      mbar_wait(drain, 0, p.err);
+    }
+  } else {
+    // softmax of tile t (warps 2-5: head h0, warps 6-9: head h0 + 1); thread = query row r
+    const int t = (warp - 2) >> 2;
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const uint32_t tS = tbase + 256 * t, tO = tS + 128;
+    // One read of S per block in the common case: the terms are formed against the running
+    // reference m while the block maximum is tracked; only when that maximum exceeds m by more
+    // than 8 (log2 units; always for the first block) is the block read again with the new m.
+    // The tensor core runs O += P V of the previous block before this block's S, so by the
+    // time S is complete the shared P tile is free and P goes straight to it.
+    float m = 0.f, l = 0.f;
+    bool ok = true;
+    uint8_t* prow = smem + S::P_OFF + 2 * t * S::SUB + r * 128;
+    for (int j = 0; j < nkv; ++j) {
+      ok = mbar_wait_warp(S_FULL(t), j & 1, p.err) && ok;
+      if (j > 0) ok = mbar_wait_warp(PV_DONE(t), (j - 1) & 1, p.err) && ok;
+      tc_fence_after();
+      const bool diag = j == qi;   // key c visible to row r when c <= r
+      float sum = 0.f;
+      // form the terms against reference `ref` into the P tile; returns the block maximum
+      auto pass = [&](float ref) {
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        float sm4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2) {
+          float sv[64];
+          tmem_ld32(tS + lane_off + 64 * c2, sv);
+          tmem_ld32(tS + lane_off + 64 * c2 + 32, sv + 32);
+          tmem_wait_ld();
+          if (diag) {
+#pragma unroll
+            for (int k2 = 0; k2 < 64; ++k2)
+              if (64 * c2 + k2 > r) sv[k2] = -INFINITY;
+          }
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {   // 16-byte chunk kc = 8 c2 + q: keys 8kc .. 8kc+7
+            uint32_t w[4];
+#pragma unroll
+            for (int i2 = 0; i2 < 4; ++i2) {
+              const float a = sv[8 * q + 2 * i2] * p.sl2, bb = sv[8 * q + 2 * i2 + 1] * p.sl2;
+              mx4[i2] = fmaxf(mx4[i2], fmaxf(a, bb));
+              const float ea = ex2(a - ref), eb = ex2(bb - ref);
+              sm4[i2] += ea + eb;
+              __nv_bfloat162 hh = __floats2bfloat162_rn(ea, eb);
+              w[i2] = *reinterpret_cast<uint32_t*>(&hh);
+            }
+            *reinterpret_cast<uint4*>(prow + c2 * S::SUB + ((q ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+        sum = (sm4[0] + sm4[1]) + (sm4[2] + sm4[3]);
+        return fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      };
+      float corr = 1.f;
+      if (j == 0) {
+        // first block: find the maximum, then form the terms against it
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float sv[32];
+          tmem_ld32(tS + lane_off + 32 * c, sv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k2 = 0; k2 < 32; ++k2) {
+            const float v = (diag && 32 * c + k2 > r) ? -INFINITY : sv[k2];
+            mx4[k2 & 3] = fmaxf(mx4[k2 & 3], v);
+          }
+        }
+        m = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * p.sl2;
+        pass(m);
+      } else {
+        const float mx = pass(m);
+        const bool raise = mx > m + 8.f;
+        // rare: raise the reference and form the block again.  The TMEM loads in pass() are
+        // warp-collective, so the whole warp repeats it; rows that keep their reference
+        // recompute the same terms.
+        if (__any_sync(0xffffffffu, raise)) {
+          if (raise) {
+            corr = ex2(m - mx);
+            m = mx;
+          }
+          pass(m);
+        }
+      }
+      l = l * corr + sum;
+      if (j > 0 && __any_sync(0xffffffffu, corr != 1.f)) {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float o[32];
+          tmem_ld32(tO + lane_off + 32 * c, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k2 = 0; k2 < 32; ++k2) o[k2] *= corr;
+          tmem_st32(tO + lane_off + 32 * c, o);
+        }
+        tmem_wait_st();
+      }
+      fence_async_shared();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(S_FREE(t));   // S may be overwritten
+        mbar_arrive(P_FULL(t));
+      }
+    }
+    if (ok && mbar_wait_warp(PV_DONE(t), (nkv - 1) & 1, p.err)) {
+      tc_fence_after();
+      const float inv = 1.f / l;
+      const int row = qi * ATT_BQ + r;
+      bf16* dst = p.o + (long long)(b * p.L + row) * p.ldo + (h0 + t) * ATT_D;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float o[32];
+        tmem_ld32(tO + lane_off + 32 * c, o);
+        tmem_wait_ld();
+        if (row < p.L) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            uint4 u;
+            __nv_bfloat162* hh = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) hh[i] = __floats2bfloat162_rn(o[8 * k + 2 * i] * inv, o[8 * k + 2 * i + 1] * inv);
+            *reinterpret_cast<uint4*>(dst + 32 * c + 8 * k) = u;
+          }
+        }
+      }
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+#undef S_FULL
+#undef S_FREE
+#undef P_FULL
+#undef PV_DONE
 
 // qkv [B*L, W] (W = (H + 2G) D): V transposed into vt [B*G*D, ldv] (row
 // (b, g, d), column = position) and, when given, K and V into the caches
@@ -354,10 +643,17 @@ jamba_status attn_prefill_core(const void* qkv, void* vt, long long ldv, void* o
   if (dev < 64 && !configured[dev]) {
     JB_CUDA(cudaFuncSetAttribute(flash_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)AttnSmem::BYTES));
+    JB_CUDA(cudaFuncSetAttribute(flash_attn2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)Attn2Smem::BYTES));
     configured[dev] = true;
   }
-  JB_CUDA(launch_pdl(flash_attn_kernel, dim3((unsigned)(B * H * p.nq)), dim3(ATT_THREADS), AttnSmem::BYTES, s, mqk,
-                     mvt, p));
+  if (p.rep % 2 == 0) {   // pairs of query heads stay inside one KV group
+    JB_CUDA(launch_pdl(flash_attn2_kernel, dim3((unsigned)(B * (H / 2) * p.nq)), dim3(ATT2_THREADS),
+                       Attn2Smem::BYTES, s, mqk, mvt, p));
+  } else {
+    JB_CUDA(launch_pdl(flash_attn_kernel, dim3((unsigned)(B * H * p.nq)), dim3(ATT_THREADS), AttnSmem::BYTES, s,
+                       mqk, mvt, p));
+  }
   return JAMBA_OK;
 }
 

@@ -169,6 +169,14 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* er
   }
 }
 
+// The same wait taken by every lane of a warp, with one answer for all of
+// them (a lane whose own wait gave up makes the whole warp give up), so that
+// warp-collective instructions after it (tcgen05.ld / st, shuffles,
+// __syncwarp) are always reached by the full warp.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, int* err) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, err));
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(m) : "memory");

@@ -271,8 +271,8 @@ gemm_i8w_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       TileInfo ti;
       decode_tile_grouped<MH, BN_OUT>(p, t, ti);
       for (int kt = ti.kt0; kt < ti.kt1; ++kt) {
-        if (!mbar_wait(full0 + 8 * ts, tph, p.err)) { ok = false; break; }
-        if (!mbar_wait(bempty0 + 8 * bs, bph ^ 1, p.err)) { ok = false; break; }
+        if (!mbar_wait_warp(full0 + 8 * ts, tph, p.err)) { ok = false; break; }
+        if (!mbar_wait_warp(bempty0 + 8 * bs, bph ^ 1, p.err)) { ok = false; break; }
         plan.run(qbase + ts * S::T_STAGE, bbase + bs * S::B_BYTES);
         fence_async_shared();   // the tensor core reads these stores through the async proxy
         __syncwarp();
@@ -291,7 +291,7 @@ gemm_i8w_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       const bool two = MT == 2 && ti.m0 + 128 < ti.m_end;
       const int buf = it % NBUF;
       const uint32_t use = (uint32_t)(it / NBUF);
-      if (!mbar_wait(tfull0 + 8 * buf, use & 1, p.err)) break;
+      if (!mbar_wait_warp(tfull0 + 8 * buf, use & 1, p.err)) break;
       tc_fence_after();
       const float* sc = p.scale_b + (long long)ti.group * p.N;
       for (int h = 0; h < (two ? 2 : 1); ++h) {
@@ -579,9 +579,9 @@ gemm_i8w_tok_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       TileInfo ti;
       decode_tile_tok(p, t, ti);
       for (int kt = ti.kt0; kt < ti.kt1 && ok; kt += 2) {
-        if (!mbar_wait(full0 + 8 * ts, tph, p.err)) { ok = false; break; }
+        if (!mbar_wait_warp(full0 + 8 * ts, tph, p.err)) { ok = false; break; }
         for (int h = 0; h < 2; ++h) {
-          if (!mbar_wait(bempty0 + 8 * bs, bph ^ 1, p.err)) { ok = false; break; }
+          if (!mbar_wait_warp(bempty0 + 8 * bs, bph ^ 1, p.err)) { ok = false; break; }
           plan.run(qbase + ts * S::T_STAGE, h, bbase + bs * S::B_BYTES);
           fence_async_shared();
           __syncwarp();
@@ -599,7 +599,7 @@ gemm_i8w_tok_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       decode_tile_tok(p, t, ti);
       const int buf = it & 1;
       const uint32_t use = (uint32_t)(it >> 1);
-      if (!mbar_wait(tfull0 + 8 * buf, use & 1, p.err)) break;
+      if (!mbar_wait_warp(tfull0 + 8 * buf, use & 1, p.err)) break;
       tc_fence_after();
       const int f = ti.n0 + q * 32 + lane;   // weight row (output column); N is a multiple of 128
       const uint32_t tl = tbase + ((uint32_t)(q * 32) << 16) + buf * S::ACC;

@@ -384,7 +384,7 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       decode_tile<BN_OUT>(p, t, ti);
       const int acc = it & 1;
       const uint32_t use = (uint32_t)(it >> 1);
-      if (!mbar_wait(tfull0 + 8 * acc, use & 1, p.err)) break;
+      if (!mbar_wait_warp(tfull0 + 8 * acc, use & 1, p.err)) break;
       tc_fence_after();
       const int m = ti.m0 + q * 32 + lane;
       const uint32_t tl = tbase + ((uint32_t)(q * 32) << 16) + acc * BN;
