@@ -54,6 +54,7 @@ def parse():
     ap.add_argument("--decode-steps", type=int, default=DECODE_STEPS)
     ap.add_argument("--pair-seqlen", type=int, default=PAIR_L)
     ap.add_argument("--attn-seqlen", type=int, default=ATTN_L)
+    ap.add_argument("--moe8-tokens", type=int, default=64, help="tokens of the moe8dec part")
     return ap.parse_args()
 
 
@@ -456,14 +457,15 @@ def run_product(args):
         torch.cuda.synchronize()
         torch.cuda.empty_cache()
         moe8 = J.MoE(pq, es)
-        v = moe_input(es, 64, seed=3, device=dev)
+        v = moe_input(es, args.moe8_tokens, seed=3, device=dev)
         f = lambda: moe8.forward(v)
         for _ in range(args.warmup):
             f()
         torch.cuda.synchronize()
         dms, _ = event_time_ms(f, args.steps, stream, flush)
         wb8 = sum(pq[k].numel() * pq[k].element_size() for k in ("w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down"))
-        res["moe_int8_decode"] = {"workload": "ExpertsInt8 MoE, 64 tokens, 16 experts top-2, d_model 4096, d_ff 14336",
+        res["moe_int8_decode"] = {"workload": "ExpertsInt8 MoE, %d tokens, 16 experts top-2, d_model 4096, d_ff 14336"
+                                              % args.moe8_tokens,
                                   "us": round(1e3 * dms, 1),
                                   "weight_GB/s": round(wb8 / (dms / 1e3) / 1e9, 1),
                                   "frac_of_measured_hbm": round(wb8 / (dms / 1e3) / 1e9 / pk["hbm"], 4)}

@@ -681,130 +681,187 @@ kv_append_kernel(const bf16* __restrict__ qkv, int H, int G, const int* __restri
 
 constexpr int DEC_REP = 4;   // query heads per KV head in the decode kernel (8 KV heads under 32 query heads)
 
-// One CTA per (sequence, KV head, split of the positions 0..lengths[b]): for
-// each of the group's query heads, the partial softmax (max, sum, weighted
-// sum of values) over its positions.  A warp takes 16 consecutive positions
-// at a time, their value rows requested together with the keys.  Scores:
-// each load instruction covers two whole key rows (lanes 0-15 one row, 16-31
-// the next, 8 dims per lane), the query slice stays in registers, and each
-// row's dot product is reduced across its 16 lanes.  Values: lanes over the
-// head width (4 dims each), the weight of each row broadcast from the lane
-// holding it.
+// One CTA of four warps per (sequence, KV head, split of the positions
+// 0..lengths[b]): for each of the group's four query heads, the partial
+// softmax (max, sum, weighted sum of values) over its positions.  A warp takes
+// 16 positions at a time: their key and value rows are copied into shared
+// memory (cp.async, 16 bytes per copy, two buffers so the next rows stream in
+// while these are used; rows padded to 272 bytes so ldmatrix reads hit 32
+// distinct banks), then two tensor-core products per 16 positions
+// (mma.sync m16n8k16, bf16 in, fp32 out):
+//   S^T = K Q^T   positions on M, the 4 query heads (padded to 8) on N, head width as K;
+//   O^T += V^T P^T   head width on M (8 tiles of 16), heads on N, positions as K
+//                    (V^T through ldmatrix .trans).
+// In the S^T layout lane (g, t) holds positions g and g + 8 of heads 2t and
+// 2t + 1, which is also where O^T keeps those heads, so the running maximum,
+// sum and rescaling of a head stay in its lanes; the softmax reduces over
+// positions with three shuffles.  P^T's fragment is gathered with eight.
+constexpr int DEC_PITCH = 272;                     // bytes per staged row (256 + 16)
+constexpr int DEC_TILE = 16 * DEC_PITCH;           // 16 rows
+constexpr uint32_t DEC_SMEM = 4 * 2 * 2 * DEC_TILE;   // warps x buffers x (K, V)
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+// 16 bytes global -> shared; src_bytes 0 writes zeros (the source is not read)
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 __global__ void __launch_bounds__(128)
 attn_decode_kernel(const bf16* __restrict__ qkv, int H, int G, const int* __restrict__ lengths,
                    const bf16* __restrict__ kc, const bf16* __restrict__ vc, int max_len, int splits, float sl2,
                    float* __restrict__ part) {
+  extern __shared__ uint8_t dsm[];
   __shared__ float w_m[4][DEC_REP], w_l[4][DEC_REP];
   __shared__ float w_o[4][DEC_REP][ATT_D];
   griddep_wait();
   griddep_launch();
   const int bg = blockIdx.x, b = bg / G, g = bg % G, split = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int half = lane >> 4, hl = lane & 15;
+  const int gq = lane >> 2, tq = lane & 3;   // mma fragment coordinates
   const int n = max(0, min(lengths[b] + 1, max_len));   // the appended token included; never past the cache
   const int per = (n + splits - 1) / splits;
   const int p0 = split * per, p1 = min(n, p0 + per);
   const long long W = (long long)(H + 2 * G) * ATT_D;
-  // this lane's 8 dims of each query head, pre-scaled to log2 units
-  float q[DEC_REP][8];
+  // B fragments of Q^T (k = head dims, n = head gq; heads 4-7 are zero padding)
+  uint32_t qb[8][2];
+  {
+    const bf16* qrow = qkv + b * W + (long long)(g * DEC_REP + (gq & 3)) * ATT_D;
 #pragma unroll
-  for (int h = 0; h < DEC_REP; ++h) {
-    const uint4 u = *reinterpret_cast<const uint4*>(qkv + b * W + (long long)(g * DEC_REP + h) * ATT_D + hl * 8);
-    const __nv_bfloat162* qh = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 f = __bfloat1622float2(qh[i]);
-      q[h][2 * i] = f.x * sl2;
-      q[h][2 * i + 1] = f.y * sl2;
+    for (int kk = 0; kk < 8; ++kk) {
+      uint32_t lo = 0, hi = 0;
+      if (gq < DEC_REP) {
+        lo = *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * tq);
+        hi = *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * tq + 8);
+      }
+      qb[kk][0] = lo;
+      qb[kk][1] = hi;
     }
   }
   const bf16* kbase = kc + ((long long)b * G + g) * max_len * ATT_D;
   const bf16* vbase = vc + ((long long)b * G + g) * max_len * ATT_D;
-  float m[DEC_REP], l[DEC_REP], acc[DEC_REP][4];
+  const uint32_t wbase = smem_u32(dsm) + warp * 2 * 2 * DEC_TILE;   // [buffer][K, V]
+  // stage 16 rows of K and V at positions c0.. into buffer `buf` (zeros past p1)
+  auto stage = [&](int c0, int buf) {
+    const uint32_t kd = wbase + buf * 2 * DEC_TILE, vd = kd + DEC_TILE;
 #pragma unroll
-  for (int h = 0; h < DEC_REP; ++h) {
-    m[h] = -INFINITY;
-    l[h] = 0.f;
-    acc[h][0] = acc[h][1] = acc[h][2] = acc[h][3] = 0.f;
-  }
-  constexpr int RW = 16;   // rows per warp and step: 4 KB of keys and 4 KB of values
-  for (int c0 = p0 + warp * RW; c0 < p1; c0 += 4 * RW) {
-    // this lane's 4 dims of the step's value rows, requested before the scores so the loads overlap
-    uint2 vr[RW];
+    for (int i = 0; i < 8; ++i) {
+      const int idx = lane + 32 * i;          // 16 rows x 16 pieces of 16 bytes
+      const int row = idx >> 4, piece = idx & 15;
+      const int pos = c0 + row;
+      const bool in = pos < p1;
+      const long long off = (long long)(in ? pos : 0) * ATT_D + piece * 8;
+      cp_async16(kd + row * DEC_PITCH + piece * 16, kbase + off, in ? 16 : 0);
+      cp_async16(vd + row * DEC_PITCH + piece * 16, vbase + off, in ? 16 : 0);
+    }
+    cp_async_commit();
+  };
+  float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};   // heads 2tq, 2tq + 1
+  float acc[8][4];
 #pragma unroll
-    for (int k = 0; k < RW; ++k)
-      vr[k] = c0 + k < p1 ? *reinterpret_cast<const uint2*>(vbase + (long long)(c0 + k) * ATT_D + 4 * lane)
-                          : make_uint2(0, 0);
-    // scores of rows c0 + 2i + half, every lane of a half holding its row's value
-    float sc[RW / 2][DEC_REP];
+  for (int mm = 0; mm < 8; ++mm) acc[mm][0] = acc[mm][1] = acc[mm][2] = acc[mm][3] = 0.f;
+  const int mi = lane >> 3, rr = lane & 7;   // ldmatrix: matrix and row this lane addresses
+  int c0 = p0 + warp * 16, buf = 0;
+  if (c0 < p1) stage(c0, 0);
+  for (; c0 < p1; c0 += 64, buf ^= 1) {
+    if (c0 + 64 < p1) {
+      stage(c0 + 64, buf ^ 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncwarp();
+    const uint32_t kt = wbase + buf * 2 * DEC_TILE, vt = kt + DEC_TILE;
+    // S^T = K Q^T: [16 positions x 8 heads]
+    float sc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int i = 0; i < RW / 2; ++i) {
-      const int pos = c0 + 2 * i + half;
-      uint4 u = make_uint4(0, 0, 0, 0);
-      if (pos < p1) u = *reinterpret_cast<const uint4*>(kbase + (long long)pos * ATT_D + hl * 8);
-      const __nv_bfloat162* kh = reinterpret_cast<const __nv_bfloat162*>(&u);
-      float kf[8];
+    for (int kk = 0; kk < 8; ++kk) {
+      uint32_t a[4];
+      ldsm_x4(a, kt + (rr + 8 * (mi & 1)) * DEC_PITCH + (16 * kk + 8 * (mi >> 1)) * 2);
+      mma_bf16_16816(sc, a, qb[kk][0], qb[kk][1]);
+    }
+    // online softmax per head (lane-local heads 2tq, 2tq + 1; positions gq and gq + 8)
+    const bool in0 = c0 + gq < p1, in8 = c0 + gq + 8 < p1;
+    float pr[4];
 #pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const float2 f = __bfloat1622float2(kh[t]);
-        kf[2 * t] = f.x;
-        kf[2 * t + 1] = f.y;
-      }
+    for (int e = 0; e < 2; ++e) {
+      const float s0 = in0 ? sc[e] * sl2 : -INFINITY, s8 = in8 ? sc[2 + e] * sl2 : -INFINITY;
+      float mx = fmaxf(s0, s8);
 #pragma unroll
-      for (int h = 0; h < DEC_REP; ++h) {
-        float d = 0.f;
+      for (int o = 4; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      const float mn = fmaxf(m[e], mx);                  // finite: position c0 is valid
+      const float corr = ex2(m[e] - mn);                 // 0 when m was -inf
+      pr[e] = ex2(s0 - mn);
+      pr[2 + e] = ex2(s8 - mn);
+      float sum = pr[e] + pr[2 + e];
 #pragma unroll
-        for (int t = 0; t < 8; ++t) d = fmaf(q[h][t], kf[t], d);
+      for (int o = 4; o < 32; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      l[e] = l[e] * corr + sum;
+      m[e] = mn;
 #pragma unroll
-        for (int o = 8; o; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-        sc[i][h] = pos < p1 ? d : -INFINITY;
+      for (int mm = 0; mm < 8; ++mm) {
+        acc[mm][e] *= corr;
+        acc[mm][2 + e] *= corr;
       }
     }
-    // online softmax; the scores become the weights in place
-#pragma unroll
-    for (int h = 0; h < DEC_REP; ++h) {
-      float mx = sc[0][h];
-#pragma unroll
-      for (int i = 1; i < RW / 2; ++i) mx = fmaxf(mx, sc[i][h]);
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-      const float mn = fmaxf(m[h], mx);                   // finite: row c0 is valid
-      const float corr = ex2(m[h] - mn);                  // 0 when m was -inf
-      float sum = 0.f;
-#pragma unroll
-      for (int i = 0; i < RW / 2; ++i) {
-        sc[i][h] = ex2(sc[i][h] - mn);
-        sum += sc[i][h];
-      }
-      sum += __shfl_xor_sync(0xffffffffu, sum, 16);
-      l[h] = l[h] * corr + sum;
-      m[h] = mn;
-#pragma unroll
-      for (int t = 0; t < 4; ++t) acc[h][t] *= corr;
+    // P^T fragment: (positions 2tq, 2tq+1 | 2tq+8, 2tq+9; head gq) from the lanes holding them
+    uint32_t pb0, pb1;
+    {
+      const int srcA = (2 * tq) * 4 + (gq >> 1), srcB = (2 * tq + 1) * 4 + (gq >> 1);
+      const bool odd = gq & 1;
+      float v[4];
+      const float a0 = __shfl_sync(0xffffffffu, pr[0], srcA), a1 = __shfl_sync(0xffffffffu, pr[1], srcA);
+      const float b0 = __shfl_sync(0xffffffffu, pr[0], srcB), b1 = __shfl_sync(0xffffffffu, pr[1], srcB);
+      const float a2 = __shfl_sync(0xffffffffu, pr[2], srcA), a3 = __shfl_sync(0xffffffffu, pr[3], srcA);
+      const float b2 = __shfl_sync(0xffffffffu, pr[2], srcB), b3 = __shfl_sync(0xffffffffu, pr[3], srcB);
+      v[0] = odd ? a1 : a0;   // position 2tq
+      v[1] = odd ? b1 : b0;   // position 2tq + 1
+      v[2] = odd ? a3 : a2;   // position 2tq + 8
+      v[3] = odd ? b3 : b2;   // position 2tq + 9
+      __nv_bfloat162 h01 = __floats2bfloat162_rn(v[0], v[1]), h23 = __floats2bfloat162_rn(v[2], v[3]);
+      pb0 = *reinterpret_cast<uint32_t*>(&h01);
+      pb1 = *reinterpret_cast<uint32_t*>(&h23);
     }
-    // values: row c0 + k, weight sc[k / 2] from a lane of half k % 2 (rows past the end carry 0)
+    // O^T += V^T P^T: 8 tiles of 16 head dims
 #pragma unroll
-    for (int k = 0; k < RW; ++k) {
-      const __nv_bfloat162* vh = reinterpret_cast<const __nv_bfloat162*>(&vr[k]);
-      const float2 v01 = __bfloat1622float2(vh[0]), v23 = __bfloat1622float2(vh[1]);
-#pragma unroll
-      for (int h = 0; h < DEC_REP; ++h) {
-        const float pk = __shfl_sync(0xffffffffu, sc[k >> 1][h], (k & 1) * 16);
-        acc[h][0] = fmaf(pk, v01.x, acc[h][0]);
-        acc[h][1] = fmaf(pk, v01.y, acc[h][1]);
-        acc[h][2] = fmaf(pk, v23.x, acc[h][2]);
-        acc[h][3] = fmaf(pk, v23.y, acc[h][3]);
-      }
+    for (int mm = 0; mm < 8; ++mm) {
+      uint32_t a[4];
+      ldsm_x4_t(a, vt + (rr + 8 * (mi >> 1)) * DEC_PITCH + (16 * mm + 8 * (mi & 1)) * 2);
+      mma_bf16_16816(acc[mm], a, pb0, pb1);
     }
+    __syncwarp();   // this buffer is refilled two groups later
   }
   // merge the four warps, then write this split's partial per query head
 #pragma unroll
-  for (int h = 0; h < DEC_REP; ++h) {
-    if (lane == 0) {
-      w_m[warp][h] = m[h];
-      w_l[warp][h] = l[h];
-    }
+  for (int e = 0; e < 2; ++e) {
+    const int hq = 2 * tq + e;
+    if (hq < DEC_REP) {
+      if (gq == 0) {
+        w_m[warp][hq] = m[e];
+        w_l[warp][hq] = l[e];
+      }
 #pragma unroll
-    for (int t = 0; t < 4; ++t) w_o[warp][h][4 * lane + t] = acc[h][t];
+      for (int mm = 0; mm < 8; ++mm) {
+        w_o[warp][hq][16 * mm + gq] = acc[mm][e];
+        w_o[warp][hq][16 * mm + gq + 8] = acc[mm][2 + e];
+      }
+    }
   }
   __syncthreads();
   for (int i = threadIdx.x; i < DEC_REP * ATT_D; i += 128) {
@@ -866,7 +923,14 @@ jamba_status attn_decode_core(const void* qkv, void* k_cache, void* v_cache, int
                      (const int*)lengths, reinterpret_cast<bf16*>(k_cache), reinterpret_cast<bf16*>(v_cache),
                      max_len));
   const float sl2 = 1.4426950408889634f / sqrtf((float)ATT_D);
-  JB_CUDA(launch_pdl(attn_decode_kernel, dim3(B * G, splits), dim3(128), 0, s, reinterpret_cast<const bf16*>(qkv),
+  static bool configured[64] = {false};
+  int dev = 0;
+  JB_CUDA(cudaGetDevice(&dev));
+  if (dev < 64 && !configured[dev]) {
+    JB_CUDA(cudaFuncSetAttribute(attn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DEC_SMEM));
+    configured[dev] = true;
+  }
+  JB_CUDA(launch_pdl(attn_decode_kernel, dim3(B * G, splits), dim3(128), DEC_SMEM, s, reinterpret_cast<const bf16*>(qkv),
                      H, G, (const int*)lengths, reinterpret_cast<const bf16*>(k_cache),
                      reinterpret_cast<const bf16*>(v_cache), max_len, splits, sl2, part));
   JB_CUDA(launch_pdl(attn_combine_kernel, dim3(B * H), dim3(ATT_D), 0, s, (const float*)part, H, splits,
