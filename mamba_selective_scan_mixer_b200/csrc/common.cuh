@@ -282,6 +282,20 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// d += a b on the tensor cores through the warp-synchronous path: m16n8k16,
+// bf16 inputs, fp32 accumulators (fragment layouts as the PTX ISA gives them
+// for mma.m16n8k16: lane (g, t) = (lane / 4, lane % 4) holds A rows g, g + 8 at
+// columns 2t, 2t + 1 and 2t + 8, 2t + 9; B column g at rows 2t, 2t + 1 and
+// 2t + 8, 2t + 9; D rows g, g + 8 at columns 2t, 2t + 1).  For decode-sized
+// products, where the operands arrive in registers.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 // Shared-memory matrix descriptor of a K-major bf16 tile written by TMA with
 // 128-byte swizzle: rows of 64 elements (128 B), 8-row groups 1024 B apart.
 // Bits: start address >> 4 [0,14), leading offset >> 4 [16,30) (unused for
