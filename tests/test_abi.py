@@ -109,3 +109,38 @@ def test_no_product_module_imports_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".hpp", ".h")):
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
+
+
+def test_attention_entry_points_validate_without_gpu(lib):
+    """Config and argument checks of the attention entry points (no launch reached)."""
+    from mamba_selective_scan_mixer_b200 import _abi
+    n = ctypes.c_size_t()
+    BF = _abi.JAMBA_BF16
+    good = _abi.AttnConfig(4096, 32, 8, 128, BF)
+    assert lib.jamba_attn_prefill_workspace_size(ctypes.byref(good), 1, 32768, ctypes.byref(n)) == 0
+    # q|k|v rows (6144 wide) + V transposed + attention output, bf16
+    assert n.value >= 32768 * (6144 + 1024 + 4096) * 2
+    assert lib.jamba_attn_step_workspace_size(ctypes.byref(good), 64, 2048, ctypes.byref(n)) == 0
+    for bad, code in ((_abi.AttnConfig(4096, 32, 8, 64, BF), 2),        # head_dim 64
+                      (_abi.AttnConfig(4096, 32, 7, 128, BF), 1),       # 7 does not divide 32
+                      (_abi.AttnConfig(4096, 32, 8, 128, _abi.JAMBA_F32), 2),
+                      (_abi.AttnConfig(4000, 32, 8, 128, BF), 2)):      # d_model not a multiple of 64
+        assert lib.jamba_attn_prefill_workspace_size(ctypes.byref(bad), 1, 128, ctypes.byref(n)) == code
+    assert lib.jamba_attn_prefill_workspace_size(ctypes.byref(good), 1, 0, ctypes.byref(n)) == 1
+    p = ctypes.c_void_p(4096)
+    w = _abi.AttnWeights(p, p)
+    ws = ctypes.c_void_p(8192)
+    # out aliasing x, one cache without the other, max_len below seqlen, null lengths: rejected up front
+    assert lib.jamba_attn_prefill(ctypes.byref(good), ctypes.byref(w), p, None, p, 1, 128, None, None, 0,
+                                  ws, 1 << 30, None) == 1
+    q = ctypes.c_void_p(1 << 20)
+    assert lib.jamba_attn_prefill(ctypes.byref(good), ctypes.byref(w), p, None, q, 1, 128, p, None, 256,
+                                  ws, 1 << 30, None) == 1
+    assert lib.jamba_attn_prefill(ctypes.byref(good), ctypes.byref(w), p, None, q, 1, 128, p, p, 64,
+                                  ws, 1 << 30, None) == 1
+    assert lib.jamba_attn_prefill(ctypes.byref(good), ctypes.byref(w), p, None, q, 1, 128, None, None, 0,
+                                  ws, 16, None) == 3                      # workspace too small
+    assert lib.jamba_attn_step(ctypes.byref(good), ctypes.byref(w), p, None, q, 4, p, p, 256, None,
+                               ws, 1 << 30, None) == 1
+    assert lib.jamba_attn_step(ctypes.byref(good), ctypes.byref(w), ctypes.c_void_p(4100), None, q, 4, p, p,
+                               256, p, ws, 1 << 30, None) == 1            # misaligned x
