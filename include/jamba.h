@@ -331,7 +331,7 @@ jamba_status jamba_attn_prefill(const jamba_attn_config* cfg, const jamba_attn_w
 
 jamba_status jamba_attn_step_workspace_size(const jamba_attn_config* cfg, int batch, int max_len, size_t* bytes);
 
-/* One decode token per sequence (n_heads = 4 n_kv_heads, the Jamba grouping;
+/* One decode token per sequence (at most 8 query heads per KV head;
  * JAMBA_ERR_UNSUPPORTED otherwise).
  *   x [batch, d_model]; residual [batch, d_model] or NULL; out [batch, d_model]
  *   k_cache, v_cache [batch, n_kv_heads, max_len, head_dim]

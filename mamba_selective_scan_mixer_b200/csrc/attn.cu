@@ -679,17 +679,18 @@ kv_append_kernel(const bf16* __restrict__ qkv, int H, int G, const int* __restri
   }
 }
 
-constexpr int DEC_REP = 4;   // query heads per KV head in the decode kernel (8 KV heads under 32 query heads)
+constexpr int DEC_REP = 8;   // query heads per KV head the decode kernel takes at most (the padded N of its tiles)
 
 // One CTA of four warps per (sequence, KV head, split of the positions
-// 0..lengths[b]): for each of the group's four query heads, the partial
+// 0..lengths[b]): for each of the group's query heads, the partial
 // softmax (max, sum, weighted sum of values) over its positions.  A warp takes
 // 16 positions at a time: their key and value rows are copied into shared
 // memory (cp.async, 16 bytes per copy, two buffers so the next rows stream in
 // while these are used; rows padded to 272 bytes so ldmatrix reads hit 32
 // distinct banks), then two tensor-core products per 16 positions
 // (mma.sync m16n8k16, bf16 in, fp32 out):
-//   S^T = K Q^T   positions on M, the 4 query heads (padded to 8) on N, head width as K;
+//   S^T = K Q^T   positions on M, the group's query heads (up to 8; padded to 8) on N,
+//                 head width as K;
 //   O^T += V^T P^T   head width on M (8 tiles of 16), heads on N, positions as K
 //                    (V^T through ldmatrix .trans).
 // In the S^T layout lane (g, t) holds positions g and g + 8 of heads 2t and
@@ -723,6 +724,7 @@ attn_decode_kernel(const bf16* __restrict__ qkv, int H, int G, const int* __rest
   extern __shared__ uint8_t dsm[];
   __shared__ float w_m[4][DEC_REP], w_l[4][DEC_REP];
   __shared__ float w_o[4][DEC_REP][ATT_D];
+  const int rep = H / G;   // query heads of the group: 1 .. DEC_REP
   griddep_wait();
   griddep_launch();
   const int bg = blockIdx.x, b = bg / G, g = bg % G, split = blockIdx.y;
@@ -735,11 +737,11 @@ attn_decode_kernel(const bf16* __restrict__ qkv, int H, int G, const int* __rest
   // B fragments of Q^T (k = head dims, n = head gq; heads 4-7 are zero padding)
   uint32_t qb[8][2];
   {
-    const bf16* qrow = qkv + b * W + (long long)(g * DEC_REP + (gq & 3)) * ATT_D;
+    const bf16* qrow = qkv + b * W + (long long)(g * rep + (gq < rep ? gq : 0)) * ATT_D;
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
       uint32_t lo = 0, hi = 0;
-      if (gq < DEC_REP) {
+      if (gq < rep) {
         lo = *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * tq);
         hi = *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * tq + 8);
       }
@@ -844,7 +846,7 @@ attn_decode_kernel(const bf16* __restrict__ qkv, int H, int G, const int* __rest
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
     const int hq = 2 * tq + e;
-    if (hq < DEC_REP) {
+    if (hq < rep) {
       if (gq == 0) {
         w_m[warp][hq] = m[e];
         w_l[warp][hq] = l[e];
@@ -857,7 +859,7 @@ attn_decode_kernel(const bf16* __restrict__ qkv, int H, int G, const int* __rest
     }
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < DEC_REP * ATT_D; i += 128) {
+  for (int i = threadIdx.x; i < rep * ATT_D; i += 128) {
     const int h = i / ATT_D, d = i % ATT_D;
     float mm = -INFINITY;
     for (int w = 0; w < 4; ++w) mm = fmaxf(mm, w_m[w][h]);
@@ -868,7 +870,7 @@ attn_decode_kernel(const bf16* __restrict__ qkv, int H, int G, const int* __rest
       os += w_o[w][h][d] * f;
     }
     // part layout: [B*H][splits][D + 2]: o (unnormalised), then max (log2 units), sum
-    float* dst = part + ((long long)(b * H + g * DEC_REP + h) * splits + split) * (ATT_D + 2);
+    float* dst = part + ((long long)(b * H + g * rep + h) * splits + split) * (ATT_D + 2);
     dst[d] = os;
     if (d == 0) {
       dst[ATT_D] = mm;
@@ -911,7 +913,7 @@ int attn_decode_splits(int B, int G, int max_len) {
 
 jamba_status attn_decode_core(const void* qkv, void* k_cache, void* v_cache, int max_len, int* lengths, float* part,
                               int splits, void* o, int B, int H, int G, cudaStream_t s) {
-  if (H / G != DEC_REP) return fail(JAMBA_ERR_UNSUPPORTED, "attention step: 4 query heads per KV head");
+  if (H / G > DEC_REP) return fail(JAMBA_ERR_UNSUPPORTED, "attention step: at most 8 query heads per KV head");
   JB_CUDA(launch_pdl(kv_append_kernel, dim3(B), dim3(256), 0, s, reinterpret_cast<const bf16*>(qkv), H, G,
                      (const int*)lengths, reinterpret_cast<bf16*>(k_cache), reinterpret_cast<bf16*>(v_cache),
                      max_len));
