@@ -47,15 +47,17 @@ def test_attention_prefill(dev, B, L, H, G, dm, residual):
     assert not kc_h[:, :, L:].any() and not vc_h[:, :, L:].any()
 
 
-def test_attention_prefill_concentrated_softmax(dev):
+@pytest.mark.parametrize("G", [2, 4])
+def test_attention_prefill_concentrated_softmax(dev, G):
     """Logits that grow block after block (up to about 300), with q, k and v
     exact in bf16 so that only P and O are rounded: token t is the one-hot
     vector e_(t mod 256) scaled by 2^(t // 128 - 2), weights N(0, 2).  The
     running maximum of most rows rises by more than 8 (log2 units) from one
     128-key block to a later one, so O is rescaled in TMEM, up to four times
-    in a row."""
+    in a row.  G = 2 runs the two-heads-per-CTA kernel, G = 4 (one query head
+    per KV head) the one-head kernel."""
     import mamba_selective_scan_mixer_b200 as J
-    sh = AttnShape(d_model=256, n_heads=4, n_kv_heads=2, head_dim=128)
+    sh = AttnShape(d_model=256, n_heads=4, n_kv_heads=G, head_dim=128)
     p = attn_params(sh, seed=41)
     for k in ("wq", "wk", "wv"):
         p[k] = (p[k].float() * 100).to(torch.bfloat16)
