@@ -617,6 +617,7 @@ kv_prep_kernel(const bf16* __restrict__ qkv, int L, int H, int G, bf16* __restri
 jamba_status attn_prefill_core(const void* qkv, void* vt, long long ldv, void* o, void* k_cache, void* v_cache,
                                int max_len, int B, int L, int H, int G, cudaStream_t s) {
   const int W = (H + 2 * G) * ATT_D;
+  if ((long long)B * G > 65535) return fail(JAMBA_ERR_UNSUPPORTED, "attention prefill: batch * n_kv_heads above 65535");
   JB_CUDA(launch_pdl(kv_prep_kernel, dim3((L + 63) / 64, B * G), dim3(256), 0, s,
                      reinterpret_cast<const bf16*>(qkv), L, H, G, reinterpret_cast<bf16*>(vt), ldv,
                      reinterpret_cast<bf16*>(k_cache), reinterpret_cast<bf16*>(v_cache), max_len));
@@ -913,6 +914,7 @@ int attn_decode_splits(int B, int G, int max_len) {
 
 jamba_status attn_decode_core(const void* qkv, void* k_cache, void* v_cache, int max_len, int* lengths, float* part,
                               int splits, void* o, int B, int H, int G, cudaStream_t s) {
+  if (splits > 65535) return fail(JAMBA_ERR_UNSUPPORTED, "attention step: too many position splits");
   if (H / G > DEC_REP) return fail(JAMBA_ERR_UNSUPPORTED, "attention step: at most 8 query heads per KV head");
   JB_CUDA(launch_pdl(kv_append_kernel, dim3(B), dim3(256), 0, s, reinterpret_cast<const bf16*>(qkv), H, G,
                      (const int*)lengths, reinterpret_cast<bf16*>(k_cache), reinterpret_cast<bf16*>(v_cache),
