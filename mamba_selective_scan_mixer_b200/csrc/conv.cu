@@ -8,7 +8,8 @@
 // Prefill: each thread owns 16 bytes of channels (8 bf16 or 4 fp32) over a run
 // of 64 time steps, keeping the three previous inputs in registers, so every
 // input row is read once (plus a 3-row halo per run) with 16-byte loads that
-// are contiguous across the warp.
+// are contiguous across the warp; eight rows are requested at a time so that
+// enough bytes are in flight to stream at HBM speed.
 #include "common.cuh"
 #include "host.hpp"
 
@@ -16,6 +17,7 @@ namespace jb {
 
 constexpr int CONV_TQ = 64;
 constexpr int CONV_THREADS = 128;
+constexpr int CONV_BATCH = 8;   // input rows a thread has in flight
 
 template <typename T> struct Vec16;
 template <> struct Vec16<bf16> {
@@ -83,22 +85,32 @@ conv_prefill_kernel(const T* __restrict__ x, long long ld_x, const T* __restrict
     }
   }
   T* ob = out + (long long)b * L * C;
-  for (int t = t0; t < t1; ++t) {
-    float cur[V], o[V];
-    Vec16<T>::load(xb + (long long)t * ld_x + c0, cur);
+  // eight input rows requested together (kept as raw 16-byte words), then consumed in order
+  for (int tb = t0; tb < t1; tb += CONV_BATCH) {
+    const int nb = min(CONV_BATCH, t1 - tb);
+    uint4 raw[CONV_BATCH];
 #pragma unroll
-    for (int i = 0; i < V; ++i) {
-      float acc = bv[i];
-      acc = fmaf(wk[0][i], win[0][i], acc);
-      acc = fmaf(wk[1][i], win[1][i], acc);
-      acc = fmaf(wk[2][i], win[2][i], acc);
-      acc = fmaf(wk[3][i], cur[i], acc);
-      o[i] = silu(acc);
-      win[0][i] = win[1][i];
-      win[1][i] = win[2][i];
-      win[2][i] = cur[i];
+    for (int j = 0; j < CONV_BATCH; ++j)
+      if (j < nb) raw[j] = *reinterpret_cast<const uint4*>(xb + (long long)(tb + j) * ld_x + c0);
+#pragma unroll
+    for (int j = 0; j < CONV_BATCH; ++j) {
+      if (j >= nb) break;
+      float cur[V], o[V];
+      Vec16<T>::load(reinterpret_cast<const T*>(&raw[j]), cur);
+#pragma unroll
+      for (int i = 0; i < V; ++i) {
+        float acc = bv[i];
+        acc = fmaf(wk[0][i], win[0][i], acc);
+        acc = fmaf(wk[1][i], win[1][i], acc);
+        acc = fmaf(wk[2][i], win[2][i], acc);
+        acc = fmaf(wk[3][i], cur[i], acc);
+        o[i] = silu(acc);
+        win[0][i] = win[1][i];
+        win[1][i] = win[2][i];
+        win[2][i] = cur[i];
+      }
+      Vec16<T>::store(ob + (long long)(tb + j) * C + c0, o);
     }
-    Vec16<T>::store(ob + (long long)t * C + c0, o);
   }
   if (st_out && t1 == L) {
 #pragma unroll
