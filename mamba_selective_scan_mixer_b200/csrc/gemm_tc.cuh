@@ -239,7 +239,11 @@ struct GemmSmem {
   // STAGED: per epilogue warp two 32 x 32 fp32 boxes for TMA stores (1024-aligned)
   static constexpr uint32_t STG_OFF = STAGES * (A_BYTES + B_BYTES);
   static constexpr uint32_t STG_BYTES = STAGED ? GEMM_EPI_WARPS * 2 * 4096 : 0;
-  static constexpr uint32_t BAR_OFF = STG_OFF + STG_BYTES;
+  // STAGED: per epilogue warp the bias of its 32-column chunks of the tile
+  static constexpr int SB_CHUNKS = (BN / 32 + 1) / 2;
+  static constexpr uint32_t SB_OFF = STG_OFF + STG_BYTES;
+  static constexpr uint32_t SB_BYTES = STAGED ? GEMM_EPI_WARPS * SB_CHUNKS * 128 : 0;
+  static constexpr uint32_t BAR_OFF = SB_OFF + SB_BYTES;
   // barrier slots: full[STAGES], empty[STAGES], tmem_full[2], tmem_empty[2], drain, tmem holder
   static_assert(8 * (2 * STAGES + 6) <= 256, "barrier slots");
   static constexpr uint32_t BYTES = BAR_OFF + 256 + 1024;  // + barriers + alignment slack
@@ -384,6 +388,16 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       decode_tile<BN_OUT>(p, t, ti);
       const int acc = it & 1;
       const uint32_t use = (uint32_t)(it >> 1);
+      // staged epilogue: the bias of this warp's chunks (lane = column within
+      // a chunk) is fetched while the accumulator is still being computed
+      float bl[S::SB_CHUNKS];
+      if constexpr (STAGED) {
+#pragma unroll
+        for (int jj = 0; jj < S::SB_CHUNKS; ++jj) {
+          const int col = ti.n0 + (half + 2 * jj) * 32 + lane;
+          bl[jj] = (half + 2 * jj < BN / 32 && col < p.N) ? __ldg(p.bias + col) : 0.f;
+        }
+      }
       if (!mbar_wait_warp(tfull0 + 8 * acc, use & 1, p.err)) break;
       tc_fence_after();
       const int m = ti.m0 + q * 32 + lane;
@@ -391,22 +405,31 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       if constexpr (STAGED) {
         static_assert(BN % 32 == 0, "staged epilogue works on whole 32-column chunks");
         uint8_t* stg = smem + S::STG_OFF + (warp - 2) * 8192;
-#pragma unroll 1
-        for (int j = half; j < BN / 32; j += 2) {
-          float v[32];
-          tmem_ld32(tl + j * 32, v);
-          tmem_wait_ld();
+        float* sb = reinterpret_cast<float*>(smem + S::SB_OFF) + (warp - 2) * S::SB_CHUNKS * 32;
+        __syncwarp();                    // every lane is done with the last tile's bias
+#pragma unroll
+        for (int jj = 0; jj < S::SB_CHUNKS; ++jj) sb[jj * 32 + lane] = bl[jj];
+        __syncwarp();
+        // this warp's chunks j = half, half + 2, ...; the TMEM load of the
+        // next one is in flight while the current one is processed
+        constexpr int NCH = BN / 32;
+        const int cnt = (NCH - half + 1) / 2;
+        float vb[2][32];
+        if (cnt > 0) tmem_ld32(tl + half * 32, vb[0]);
+#pragma unroll
+        for (int jj = 0; jj < (NCH + 1) / 2; ++jj) {
+          if (jj >= cnt) break;
+          const int j = half + 2 * jj;
+          float* v = vb[jj & 1];
+          tmem_wait_ld32(v);
+          if (jj + 1 < cnt) tmem_ld32(tl + (j + 2) * 32, vb[(jj + 1) & 1]);
           const int n = ti.n0 + j * 32;
+          // the same 32 bias values for every lane: broadcast reads (zero past N,
+          // where the TMA store clips the columns anyway)
 #pragma unroll
           for (int c = 0; c < 32; c += 4) {
-            if (n + c + 4 <= p.N) {
-              const float4 b4 = __ldg(reinterpret_cast<const float4*>(p.bias + n + c));
-              v[c] += b4.x; v[c + 1] += b4.y; v[c + 2] += b4.z; v[c + 3] += b4.w;
-            } else {
-#pragma unroll
-              for (int i = 0; i < 4; ++i)
-                if (n + c + i < p.N) v[c + i] += __ldg(p.bias + n + c + i);
-            }
+            const float4 b4 = *reinterpret_cast<const float4*>(sb + jj * 32 + c);
+            v[c] += b4.x; v[c + 1] += b4.y; v[c + 2] += b4.z; v[c + 3] += b4.w;
           }
           softplus32(v);
           uint8_t* buf = stg + (stg_count & 1) * 4096;
