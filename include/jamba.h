@@ -339,8 +339,10 @@ jamba_status jamba_attn_step_workspace_size(const jamba_attn_config* cfg, int ba
  *            The new token's k and v are written at position lengths[b], the
  *            token attends to positions 0..lengths[b], and lengths[b] is then
  *            incremented (so a captured CUDA graph can be replayed step after
- *            step).  A sequence whose length is outside [0, max_len) is left
- *            untouched by the cache append; the caller keeps lengths < max_len. */
+ *            step).  Lengths are device data, so the host cannot check them:
+ *            for a sequence whose length is outside [0, max_len) nothing is
+ *            appended, no cache position at or past max_len is read, and its
+ *            output row is unspecified; the caller keeps lengths < max_len. */
 jamba_status jamba_attn_step(const jamba_attn_config* cfg, const jamba_attn_weights* w, const void* x,
                              const void* residual, void* out, int batch, void* k_cache, void* v_cache,
                              int max_len, int32_t* lengths, void* ws, size_t ws_bytes, jamba_stream_t stream);

@@ -668,7 +668,7 @@ kv_append_kernel(const bf16* __restrict__ qkv, int H, int G, const int* __restri
   griddep_launch();
   const int b = blockIdx.x;
   const int pos = lengths[b];
-  if (pos < 0 || pos >= max_len) return;   // rejected on the host side for the lengths it can see
+  if (pos < 0 || pos >= max_len) return;   // out-of-range lengths append nothing
   const long long W = (long long)(H + 2 * G) * ATT_D;
   for (int i = threadIdx.x; i < G * 16; i += 256) {
     const int g = i >> 4, ch = i & 15;
