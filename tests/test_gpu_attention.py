@@ -85,11 +85,12 @@ def test_attention_prefill_concentrated_softmax(dev, G):
 
 
 @pytest.mark.parametrize("B,H,G,dm", [(3, 8, 2, 256), (2, 32, 8, 512), (2, 4, 4, 256), (3, 8, 1, 256),
-                                     (1, 6, 3, 128)])
+                                     (1, 6, 3, 128), (2, 16, 4, 2048)])
 def test_attention_decode_steps(dev, B, H, G, dm):
     """Prefill 200 tokens, cut sequence lengths to 200, 137, 1 (different per
     sequence), then 4 decode steps each checked against the oracle step;
-    group sizes 4 (Jamba), 1 (MHA), 8 and 2 (odd head counts, 6 over 3)."""
+    group sizes 4 (Jamba), 1 (MHA), 8 and 2 (odd head counts, 6 over 3);
+    d_model 2048 with 16 heads over 4."""
     import mamba_selective_scan_mixer_b200 as J
     sh = AttnShape(d_model=dm, n_heads=H, n_kv_heads=G, head_dim=128)
     p = attn_params(sh, seed=50 + H)

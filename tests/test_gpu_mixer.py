@@ -123,6 +123,22 @@ def test_bf16_decode_shapes(dev, dt_rank, batch, inner_norm, a_init):
     assert rel_l2(to_np(cs), ref["conv_state"]) < TOL_BF16
 
 
+def test_bf16_decode_mid_width(dev):
+    """d_model 1024 / d_inner 2048, batch 8: the decode GEMMs at a width
+    between the small cases and Jamba's"""
+    sh = MambaShape(d_model=1024, d_inner=2048, dt_rank=64, dtype="bf16", inner_norm=True)
+    mix, p64 = _mixer(sh, 10, dev, a_init="structured", norm_init="random")
+    L0, S, batch = 16, 4, 8
+    u = mamba_input(sh, batch, L0, seed=10)
+    steps = decode_inputs(sh, batch, S, seed=10)
+    _, cs, ss = mix.prefill(u.to(dev))
+    outs = [to_np(mix.step(steps[t].to(dev), cs, ss)) for t in range(S)]
+    full = torch.cat([u, steps.transpose(0, 1)], dim=1)
+    ref = om.mamba_prefill(p64, to_np(full), sh)
+    assert rel_l2(np.stack(outs, 1), ref["out"][:, L0:]) < TOL_BF16
+    assert rel_l2(to_np(ss), ref["ssm_state"]) < TOL_BF16
+
+
 def test_bf16_decode_ragged_width(dev):
     """d_inner 136 (not a multiple of 64) at batch 3: 408 (row, channel) pairs,
     so the last block of the state update is partly empty"""
