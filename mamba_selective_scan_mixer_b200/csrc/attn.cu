@@ -638,7 +638,7 @@ jamba_status attn_prefill_core(const void* qkv, void* vt, long long ldv, void* o
   p.sl2 = 1.4426950408889634f / sqrtf((float)ATT_D);
   p.err = device_error_word();
   if (!p.err) return fail(JAMBA_ERR_CUDA, "could not allocate the device status word");
-  static bool configured[64] = {false};
+  static std::atomic<bool> configured[64];
   int dev = 0;
   JB_CUDA(cudaGetDevice(&dev));
   if (dev < 64 && !configured[dev]) {
@@ -920,7 +920,7 @@ jamba_status attn_decode_core(const void* qkv, void* k_cache, void* v_cache, int
                      (const int*)lengths, reinterpret_cast<bf16*>(k_cache), reinterpret_cast<bf16*>(v_cache),
                      max_len));
   const float sl2 = 1.4426950408889634f / sqrtf((float)ATT_D);
-  static bool configured[64] = {false};
+  static std::atomic<bool> configured[64];
   int dev = 0;
   JB_CUDA(cudaGetDevice(&dev));
   if (dev < 64 && !configured[dev]) {

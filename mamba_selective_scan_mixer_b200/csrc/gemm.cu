@@ -13,7 +13,7 @@ template <int BN, int STAGES, int EPI, bool TRANS>
 static jamba_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb2,
                               const CUtensorMap& mc, const GemmParams& p, int grid, cudaStream_t s) {
   using S = GemmSmem<BN, STAGES, EPI == EPI_SOFTPLUS && !TRANS>;
-  static bool configured[64] = {false};
+  static std::atomic<bool> configured[64];
   int dev = 0;
   JB_CUDA(cudaGetDevice(&dev));
   if (dev < 64 && !configured[dev]) {
@@ -30,7 +30,7 @@ template <int EPI, int MT>
 static jamba_status launch_i8w(const CUtensorMap& ma, const CUtensorMap& mq, const CUtensorMap& mq2,
                                const GemmParams& p, int grid, cudaStream_t s) {
   using S = I8wSmem<MT>;
-  static bool configured[64] = {false};
+  static std::atomic<bool> configured[64];
   int dev = 0;
   JB_CUDA(cudaGetDevice(&dev));
   if (dev < 64 && !configured[dev]) {
@@ -46,7 +46,7 @@ template <int EPI>
 static jamba_status launch_i8t(const CUtensorMap& ma, const CUtensorMap& mq, const CUtensorMap& mq2,
                                const GemmParams& p, int grid, cudaStream_t s) {
   using S = I8tSmem<EPI>;
-  static bool configured[64] = {false};
+  static std::atomic<bool> configured[64];
   int dev = 0;
   JB_CUDA(cudaGetDevice(&dev));
   if (dev < 64 && !configured[dev]) {

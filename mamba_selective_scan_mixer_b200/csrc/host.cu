@@ -23,7 +23,7 @@ jamba_status cuda_fail(cudaError_t e, const char* what) {
 static constexpr int kMaxDevices = 64;
 
 int num_sms() {
-  static int cache[kMaxDevices] = {0};
+  static std::atomic<int> cache[kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
   if (cache[dev] == 0) {

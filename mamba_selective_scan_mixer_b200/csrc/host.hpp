@@ -1,6 +1,7 @@
 // Host-side internals shared by the launchers: error reporting, device
 // properties, TMA tensor-map encoding, per-device error word.
 #pragma once
+#include <atomic>
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>

@@ -642,7 +642,7 @@ using GenShape = ScanShape<2, 2>;
 template <typename TX, typename TBC, bool FAST, int CPT, int MINB>
 static bool configure_scan() {
   using Lyt = ScanLayout<TX, TBC, FAST>;
-  static bool done[64] = {false};
+  static std::atomic<bool> done[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
   if (!done[dev]) {
@@ -657,7 +657,7 @@ static bool configure_scan() {
 template <typename TX, typename TBC, bool FAST, int CPT, int MINB>
 static int resident_ctas() {
   using Lyt = ScanLayout<TX, TBC, FAST>;
-  static int cache[64] = {0};
+  static std::atomic<int> cache[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 2 * num_sms();
   if (cache[dev] == 0) {
