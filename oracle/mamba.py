@@ -28,9 +28,11 @@ brute-force unrolled sum for L <= 5, constant-input geometric series, C = 0,
 linearity in x, a hand-worked three-step example (tests/golden), the chunked
 associative form for several chunk sizes, conv delta kernels and
 torch.nn.functional.conv1d, linear vs a pure-Python triple loop, RMSNorm and
-softplus / SiLU identities, and decode step == prefill of L + 1.
-End-to-end outputs of the full layer have no printed reference values on the
-pages: beyond the pins above, parity of the full composition is unpinned.
+softplus / SiLU identities, and decode step == prefill of L + 1.  The whole
+composition is pinned by a three-token mixer example worked out by hand
+(tests/golden/mixer_hand_example.json: every intermediate from the x|z split
+to both caches, in closed form) and, inside the layer pair, by the same
+layer written with scalar Python loops.
 """
 import numpy as np
 

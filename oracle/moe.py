@@ -33,6 +33,10 @@ Int8: hand-worked rows with exact halves (ties to even); the error bound
 power-of-two scaling of a row scales s alone; weights that are already
 q * s with s a power of two quantise losslessly, so the int8 MoE equals the
 plain MoE exactly.
+Layer pair: the whole pair against the same pair written with scalar Python
+loops on a tiny case (router indices equal, outputs to 1e-12), and two
+closed forms: out_proj = 0 gives h = x exactly, and identical experts give
+out = h + (p_1 + p_2) f(RMSNorm(h)).
 """
 import numpy as np
 

@@ -308,6 +308,201 @@ def test_prefill_step_order_by_hand():
     np.testing.assert_allclose(got, want.numpy(), rtol=1e-12, atol=1e-13)
 
 
+def _hand_value(expr):
+    """Evaluates one hand-derived value of a golden file: numbers, ln2, ln3, + - * / and parentheses."""
+    import ast
+    names = {"ln2": math.log(2.0), "ln3": math.log(3.0)}
+    ops = {ast.Add: lambda a, b: a + b, ast.Sub: lambda a, b: a - b,
+           ast.Mult: lambda a, b: a * b, ast.Div: lambda a, b: a / b}
+
+    def ev(n):
+        if isinstance(n, ast.Expression):
+            return ev(n.body)
+        if isinstance(n, ast.Constant) and isinstance(n.value, (int, float)):
+            return float(n.value)
+        if isinstance(n, ast.Name) and n.id in names:
+            return names[n.id]
+        if isinstance(n, ast.UnaryOp) and isinstance(n.op, ast.USub):
+            return -ev(n.operand)
+        if isinstance(n, ast.BinOp) and type(n.op) in ops:
+            return ops[type(n.op)](ev(n.left), ev(n.right))
+        raise ValueError("not a hand value: " + expr)
+
+    return ev(ast.parse(expr, mode="eval"))
+
+
+def _hand_array(v):
+    return np.vectorize(_hand_value, otypes=[np.float64])(np.array(v, dtype=object))
+
+
+def test_mixer_hand_example():
+    """The whole mixer on a worked example derived by hand step by step (tests/golden).
+
+    Pins the wiring of the composition: which half of xz is x and which is z,
+    the conv orientation and bias, SiLU after the conv, the [dt_low | B | C]
+    split with a norm on each piece, dt_proj + dt_bias + softplus, the scan,
+    D on the post-conv x, the SiLU(z) gate and out_proj, plus both caches.
+    """
+    g = _golden("mixer_hand_example.json")
+    p = {k: _hand_array(v) for k, v in g["params"].items()}
+    u = _hand_array(g["u"])[None]
+    sh = MambaShape(d_model=2, d_inner=1, d_state=2, d_conv=4, dt_rank=2, dtype="f32",
+                    inner_norm=True, eps=0.0)
+    r = om.mamba_prefill(p, u, sh, keep=True)
+    e = {k: _hand_array(v) for k, v in g["expect"].items()}
+    close = dict(rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(r["xz"][0, :, 0], e["x"], **close)
+    np.testing.assert_allclose(r["xz"][0, :, 1], e["z"], **close)
+    np.testing.assert_allclose(r["xc"][0, :, 0], e["xc"], **close)
+    np.testing.assert_allclose(r["dt_low"][0], e["dt_low"], **close)
+    np.testing.assert_allclose(r["B"][0], e["B"], **close)
+    np.testing.assert_allclose(r["C"][0], e["C"], **close)
+    np.testing.assert_allclose(r["dt"][0, :, 0], e["dt"], **close)
+    np.testing.assert_allclose(r["y"][0, :, 0], e["y"], **close)
+    np.testing.assert_allclose(r["out"][0], e["out"], **close)
+    np.testing.assert_allclose(r["conv_state"][0, 0], e["conv_state"], **close)
+    np.testing.assert_allclose(r["ssm_state"][0, 0], e["ssm_state"], **close)
+    # the sequential C loop reaches the same scan
+    r_c = om.mamba_prefill(p, u, sh, scan="c")
+    np.testing.assert_allclose(r_c["out"][0], e["out"], **close)
+    # and decoding the three tokens one at a time from empty caches does too
+    cs, ss = np.zeros((1, 1, 3)), np.zeros((1, 1, 2))
+    for t in range(3):
+        o, cs, ss = om.mamba_step(p, u[:, t], sh, cs, ss)
+        np.testing.assert_allclose(o[0], e["out"][t], **close)
+    np.testing.assert_allclose(ss[0, 0], e["ssm_state"], **close)
+
+
+# ------------------------------------------------------------- layer-pair pins
+
+def _py_layer_pair(mp, moe_p, x, R, N, K_top, g1, g2, eps):
+    """Jamba layer pair with scalar Python loops only (no numpy arithmetic).
+
+    RMSNorm -> Mamba mixer -> residual -> RMSNorm -> top-K softmax MoE of
+    SwiGLU experts -> residual (summary page, section 2: pre-norm "standard"
+    layers; RMSNorm on dt_low, B and C inside the mixer).  x: list of L
+    token vectors; weights as nested lists.
+    """
+    dm = len(x[0])
+    di = len(mp["conv_b"])
+    K = len(mp["conv_w"][0])
+    sig = lambda v: 1.0 / (1.0 + math.exp(-v))
+
+    def norm(v, w):
+        r = math.sqrt(sum(a * a for a in v) / len(v) + eps)
+        return [a / r * b for a, b in zip(v, w)]
+
+    def mv(W, v):
+        return [sum(W[i][j] * v[j] for j in range(len(v))) for i in range(len(W))]
+
+    L = len(x)
+    us = [norm(x[t], g1) for t in range(L)]
+    xs, zs = [], []
+    for t in range(L):
+        xz = mv(mp["in_proj"], us[t])
+        xs.append(xz[:di])
+        zs.append(xz[di:])
+    h = [[0.0] * N for _ in range(di)]
+    hs = []
+    for t in range(L):
+        xc = []
+        for c in range(di):
+            acc = mp["conv_b"][c]
+            for k in range(K):
+                s = t - (K - 1) + k
+                if s >= 0:
+                    acc += mp["conv_w"][c][k] * xs[s][c]
+            xc.append(acc * sig(acc))
+        pr = mv(mp["x_proj"], xc)
+        dtl = norm(pr[:R], mp["norm_dt"])
+        Bv = norm(pr[R:R + N], mp["norm_B"])
+        Cv = norm(pr[R + N:], mp["norm_C"])
+        y = []
+        for c in range(di):
+            v = mp["dt_bias"][c] + sum(mp["dt_proj"][c][j] * dtl[j] for j in range(R))
+            dt = math.log1p(math.exp(v))
+            acc = mp["D"][c] * xc[c]
+            for n in range(N):
+                h[c][n] = math.exp(dt * mp["A"][c][n]) * h[c][n] + dt * Bv[n] * xc[c]
+                acc += Cv[n] * h[c][n]
+            y.append(acc * zs[t][c] * sig(zs[t][c]))
+        mo = mv(mp["out_proj"], y)
+        hs.append([x[t][i] + mo[i] for i in range(dm)])
+    E = len(moe_p["router"])
+    outs, idxs = [], []
+    for t in range(L):
+        v = norm(hs[t], g2)
+        logits = mv(moe_p["router"], v)
+        m = max(logits)
+        ex = [math.exp(a - m) for a in logits]
+        tot = sum(ex)
+        order = sorted(range(E), key=lambda e: (-logits[e], e))[:K_top]
+        o = list(hs[t])
+        for e in order:
+            gt = mv(moe_p["w_gate"][e], v)
+            up = mv(moe_p["w_up"][e], v)
+            act = [a * sig(a) * b for a, b in zip(gt, up)]
+            dn = mv(moe_p["w_down"][e], act)
+            o = [o[i] + ex[e] / tot * dn[i] for i in range(dm)]
+        outs.append(o)
+        idxs.append(order)
+    return outs, hs, idxs
+
+
+def test_layer_pair_vs_python_loops():
+    """oracle.moe.layer_pair against the pair written with scalar loops (tiny case)."""
+    sh = MambaShape(d_model=6, d_inner=8, d_state=3, d_conv=4, dt_rank=2, dtype="f32",
+                    inner_norm=True)
+    mp = om.params64(mamba_params(sh, seed=21, a_init="random", norm_init="random",
+                                  d_init="random"))
+    rng = np.random.default_rng(21)
+    # larger weights than the init so every term moves the result
+    for k in ("in_proj", "x_proj", "dt_proj", "out_proj", "conv_w", "conv_b"):
+        mp[k] = mp[k] * 20.0
+    E, dff = 16, 3
+    moe_p = dict(router=rng.standard_normal((E, 6)), w_gate=rng.standard_normal((E, dff, 6)),
+                 w_up=rng.standard_normal((E, dff, 6)), w_down=rng.standard_normal((E, 6, dff)))
+    x = rng.standard_normal((1, 7, 6))
+    g1 = 1.0 + 0.3 * rng.standard_normal(6)
+    g2 = 1.0 + 0.3 * rng.standard_normal(6)
+    r = omoe.layer_pair(mp, moe_p, x, sh, 2, g1, g2)
+    tl = lambda a: np.asarray(a).tolist()
+    outs, hs, idxs = _py_layer_pair({k: tl(v) for k, v in mp.items()},
+                                    {k: tl(v) for k, v in moe_p.items()},
+                                    tl(x[0]), sh.dt_rank, sh.d_state, 2, tl(g1), tl(g2), sh.eps)
+    np.testing.assert_allclose(r["h"], np.array(hs), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(r["out"], np.array(outs), rtol=1e-12, atol=1e-13)
+    assert (r["idx"] == np.array(idxs)).all()
+    # the Mamba half moved h away from x, and the MoE half moved out away from h
+    assert np.abs(r["h"] - x[0]).max() > 1e-2 and np.abs(r["out"] - r["h"]).max() > 1e-2
+
+
+def test_layer_pair_identical_experts_and_zero_mixer():
+    """Closed forms of the pair: out_proj = 0 gives h = x; identical experts give
+    out = h + (p_1 + p_2) f(RMSNorm(h)) with the two softmax weights of the router."""
+    sh = MambaShape(d_model=6, d_inner=8, d_state=3, d_conv=4, dt_rank=2, dtype="f32")
+    mp = om.params64(mamba_params(sh, seed=22))
+    rng = np.random.default_rng(22)
+    E, dff = 16, 5
+    gt, up, dn = rng.standard_normal((dff, 6)), rng.standard_normal((dff, 6)), rng.standard_normal((6, dff))
+    moe_p = dict(router=rng.standard_normal((E, 6)), w_gate=np.stack([gt] * E),
+                 w_up=np.stack([up] * E), w_down=np.stack([dn] * E))
+    x = rng.standard_normal((2, 5, 6))
+    g1 = np.abs(rng.standard_normal(6)) + 0.5
+    g2 = np.abs(rng.standard_normal(6)) + 0.5
+    mp0 = dict(mp, out_proj=np.zeros_like(mp["out_proj"]))
+    r = omoe.layer_pair(mp0, moe_p, x, sh, 2, g1, g2)
+    xf = x.reshape(10, 6)
+    np.testing.assert_allclose(r["h"], xf, rtol=0, atol=0)
+    v = xf / np.sqrt((xf ** 2).mean(1, keepdims=True) + 1e-6) * g2
+    f = (v @ gt.T) / (1 + np.exp(-(v @ gt.T))) * (v @ up.T) @ dn.T
+    lg = v @ moe_p["router"].T
+    pr = np.exp(lg - lg.max(1, keepdims=True))
+    pr /= pr.sum(1, keepdims=True)
+    top2 = np.sort(pr, axis=1)[:, -2:].sum(1)
+    np.testing.assert_allclose(r["out"], xf + top2[:, None] * f, rtol=1e-12, atol=1e-13)
+
+
 # ------------------------------------------------------------------ MoE pins
 
 def test_router_vs_bruteforce_sort():
