@@ -61,7 +61,10 @@ const char* jamba_last_error(void);
 
 /* Synchronizes `stream`, then returns and clears the device error word of the
  * current device: JAMBA_OK, JAMBA_ERR_TIMEOUT, or JAMBA_ERR_CUDA when the
- * stream itself reports an error. */
+ * stream itself reports an error.  The word latches: once a wait has given
+ * up, later kernels that share the word stop early (writing nothing) until
+ * this call clears it.  It also reads and clears the word that
+ * jamba_selective_scan_static uses when called with status == NULL. */
 jamba_status jamba_device_status(jamba_stream_t stream);
 
 /* ------------------------------------------------------------------ Mamba */
@@ -199,19 +202,38 @@ jamba_status jamba_selective_scan(const void* x, int ld_x, const void* z, int ld
  *    execution overlaps on the GPU (different streams, no ordering between
  *    them) race on the array and give undefined results: order them.
  *  - Limit: batch * ceil(d_inner / 256) channel groups times the number of
- *    time chunks must fit the array (48 KiB per chunk record); the time chunk
- *    is lengthened until it fits, and JAMBA_ERR_UNSUPPORTED is returned when
- *    even one chunk per group does not (more than about 680 groups, e.g.
- *    batch 85 at d_inner 8192).
+ *    time chunks must fit the array (48 KiB per chunk record).  The automatic
+ *    time chunk gives at most one record per CTA resident on the GPU, which
+ *    always fits; beyond that the call takes one chunk per group, and
+ *    JAMBA_ERR_UNSUPPORTED is returned (nothing launched) when even that
+ *    does not fit: more than 682 groups, e.g. batch 22 at d_inner 8192
+ *    (batch 21 is accepted).
  *  - status: a device int the kernel sets to JAMBA_ERR_TIMEOUT if one of its
- *    bounded waits gives up (never cleared by the library), or NULL to use a
- *    static word of the same array set.
+ *    bounded waits gives up (never cleared by the library; while it is set,
+ *    later calls given the same word stop early), or NULL to use a static
+ *    word of the library that jamba_device_status() reads and clears.
  * Other arguments, layouts and errors: as jamba_selective_scan. */
 jamba_status jamba_selective_scan_static(const void* x, int ld_x, const void* z, int ld_z, const float* dt,
                                          int ld_dt, const void* B, int ld_b, const void* C, int ld_c,
                                          int bc_dtype, const float* A, const float* D, const float* h0,
                                          void* y, int ld_y, float* h_out, int batch, int seqlen, int d_inner,
                                          int d_state, int dtype, int* status, jamba_stream_t stream);
+
+/* Test support for the bounded device waits (failure detection without a GPU
+ * fault).  Runs jamba_selective_scan (same arguments, chunk > 0 and at least
+ * two chunks) but launches no CTA for the first time chunk, so the flags of
+ * chunk 0 are never published: every CTA whose look-back reaches chunk 0
+ * gives up after wait_ns nanoseconds, latches JAMBA_ERR_TIMEOUT in the device
+ * error word (read and cleared by jamba_device_status) and returns.  Every
+ * load and store stays inside the caller's tensors and the workspace; y and
+ * h_out hold unspecified values afterwards.  Not part of the method. */
+jamba_status jamba_test_scan_missing_predecessor(const void* x, int ld_x, const void* z, int ld_z,
+                                                 const float* dt, int ld_dt, const void* B, int ld_b,
+                                                 const void* C, int ld_c, int bc_dtype, const float* A,
+                                                 const float* D, void* y, int ld_y, float* h_out, int batch,
+                                                 int seqlen, int d_inner, int d_state, int dtype, int chunk,
+                                                 unsigned long long wait_ns, void* ws, size_t ws_bytes,
+                                                 jamba_stream_t stream);
 
 /* ------------------------------------------------------- building blocks */
 

@@ -14,6 +14,7 @@ struct jamba_mamba {
   jamba_mamba_config cfg;
   jamba_mamba_weights w;
   int device;
+  int a_form;   // ScanAForm of A, read once at create: picks the one scan kernel to launch
   // host-buffer prefill pipeline: two copy streams and the events that order
   // the double-buffered chunks (created on first use)
   cudaStream_t io_in = nullptr, io_out = nullptr;
@@ -137,10 +138,11 @@ jamba_status jamba_device_status(jamba_stream_t stream) {
   if (!w) return fail(JAMBA_ERR_CUDA, "could not allocate the device status word");
   int v = 0;
   JB_CUDA(cudaMemcpy(&v, w, sizeof(int), cudaMemcpyDeviceToHost));
-  if (v != 0) {
-    JB_CUDA(cudaMemset(w, 0, sizeof(int)));
-    return fail((jamba_status)v, "a device-side wait gave up");
-  }
+  if (v != 0) JB_CUDA(cudaMemset(w, 0, sizeof(int)));
+  int vs = 0;   // the word of jamba_selective_scan_static calls made without a status argument
+  JB_TRY(jb::static_scan_status_take(&vs));
+  if (v == 0) v = vs;
+  if (v != 0) return fail((jamba_status)v, "a device-side wait gave up");
   return JAMBA_OK;
 }
 
@@ -179,6 +181,21 @@ jamba_status jamba_mamba_create(const jamba_mamba_config* cfg, const jamba_mamba
   if (cudaGetDevice(&h->device) != cudaSuccess) {
     delete h;
     return fail(JAMBA_ERR_CUDA, "create: no CUDA device");
+  }
+  // A decides which scan kernel owns the channels: the power form when
+  // A[c, n] == (n + 1) A[c, 0] for every channel (bf16 only), else the general one
+  h->a_form = jb::SCAN_A_GENERAL;
+  if (c.dtype == JAMBA_BF16) {
+    std::vector<float> A((size_t)c.d_inner * c.d_state);
+    if (cudaMemcpy(A.data(), w->A, A.size() * sizeof(float), cudaMemcpyDeviceToHost) != cudaSuccess) {
+      delete h;
+      return fail(JAMBA_ERR_CUDA, "create: could not read A");
+    }
+    bool power = true;
+    for (int ch = 0; ch < c.d_inner && power; ++ch)
+      for (int n = 0; n < c.d_state; ++n)
+        power = power && A[(size_t)ch * c.d_state + n] == (float)(n + 1) * A[(size_t)ch * c.d_state];
+    h->a_form = power ? jb::SCAN_A_POWER : jb::SCAN_A_GENERAL;
   }
   *out = h;
   return JAMBA_OK;
@@ -269,6 +286,7 @@ jamba_status jamba_mamba_prefill(jamba_mamba_t h, const void* u, const void* res
   sc.h_out = ssm_state_out;
   sc.batch = batch; sc.L = seqlen; sc.di = di; sc.dtype = c.dtype; sc.chunk = p.chunk;
   sc.ws = p.scan; sc.ws_bytes = p.scan_bytes;
+  sc.a_form = h->a_form;
   JB_TRY(scan_run(sc, s));
   // out_proj (+ residual)
   GemmDesc go = gdesc(p.y, di, w.out_proj, di, T, dm, di, c.dtype == JAMBA_BF16 ? EPI_BF16 : EPI_F32, out, dm);
@@ -525,6 +543,37 @@ jamba_status jamba_selective_scan(const void* x, int ld_x, const void* z, int ld
   sc.A = A; sc.D = D; sc.h0 = h0; sc.y = y; sc.ld_y = ld_y; sc.h_out = h_out;
   sc.batch = batch; sc.L = seqlen; sc.di = d_inner; sc.dtype = dtype; sc.chunk = chunk;
   sc.ws = ws; sc.ws_bytes = ws_bytes;
+  return scan_run(sc, cs(stream));
+}
+
+jamba_status jamba_test_scan_missing_predecessor(const void* x, int ld_x, const void* z, int ld_z, const float* dt,
+                                                 int ld_dt, const void* B, int ld_b, const void* C, int ld_c,
+                                                 int bc_dtype, const float* A, const float* D, void* y, int ld_y,
+                                                 float* h_out, int batch, int seqlen, int d_inner, int d_state,
+                                                 int dtype, int chunk, unsigned long long wait_ns, void* ws,
+                                                 size_t ws_bytes, jamba_stream_t stream) {
+  JB_TRY(check_dtype(dtype));
+  JB_TRY(check_dtype(bc_dtype));
+  if (d_state != 16) return fail(JAMBA_ERR_UNSUPPORTED, "d_state must be 16");
+  if (batch <= 0 || seqlen <= 0 || d_inner <= 0 || chunk <= 0 || wait_ns == 0)
+    return fail(JAMBA_ERR_INVALID_ARG, "scan test: sizes, chunk and wait must be positive");
+  JB_TRY(check_ptr(x, "x"));
+  JB_TRY(check_ptr(z, "z"));
+  JB_TRY(check_ptr(dt, "dt"));
+  JB_TRY(check_ptr(B, "B"));
+  JB_TRY(check_ptr(C, "C"));
+  JB_TRY(check_ptr(A, "A"));
+  JB_TRY(check_ptr(D, "D"));
+  JB_TRY(check_ptr(y, "y"));
+  JB_TRY(check_ptr(h_out, "h_out", false));
+  ScanCall sc = {};
+  sc.x = x; sc.ld_x = ld_x; sc.z = z; sc.ld_z = ld_z; sc.dt = dt; sc.ld_dt = ld_dt;
+  sc.B = B; sc.ld_b = ld_b; sc.C = C; sc.ld_c = ld_c; sc.bc_dtype = bc_dtype;
+  sc.A = A; sc.D = D; sc.h0 = nullptr; sc.y = y; sc.ld_y = ld_y; sc.h_out = h_out;
+  sc.batch = batch; sc.L = seqlen; sc.di = d_inner; sc.dtype = dtype; sc.chunk = chunk;
+  sc.ws = ws; sc.ws_bytes = ws_bytes;
+  sc.wait_ns = wait_ns;
+  sc.skip_first_chunk = 1;
   return scan_run(sc, cs(stream));
 }
 

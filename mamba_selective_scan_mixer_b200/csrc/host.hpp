@@ -108,10 +108,15 @@ struct ScanCall {
   int batch, L, di, dtype, chunk;
   void* ws; size_t ws_bytes;
   int* err;   // device status word; null = the library's per-device word
+  int a_form;                    // SCAN_A_*: which kernel owns the channels, when the caller knows
+  unsigned long long wait_ns;    // look-back wait limit; 0 = the library default
+  int skip_first_chunk;          // test only: launch no CTA for chunk 0 (its flags stay unset)
 };
+enum ScanAForm { SCAN_A_UNKNOWN = 0, SCAN_A_POWER = 1, SCAN_A_GENERAL = 2 };
 jamba_status scan_run(const ScanCall& s, cudaStream_t st);
 size_t scan_workspace_bytes(int batch, int L, int di, int chunk_len);
 int scan_auto_chunk(int batch, int L, int di, int dtype, int bc_dtype);
+jamba_status static_scan_status_take(int* value);   // static scan's own status word (read and cleared)
 jamba_status ssm_step(const void* xc, const void* z, long long ld_z, const float* dt, const float* bc,
                       long long ld_bc, const float* A, const float* D, float* state, void* y, int batch, int di,
                       int dtype, cudaStream_t st);

@@ -93,6 +93,9 @@ struct ScanArgs {
   int* flags;            // [batch * cgroups * n_chunks]
   float* rec;            // per record: P[256][16], h[256][16], inclusive h[256][16]
   int* err;
+  unsigned long long wait_ns;   // limit of the look-back waits on a predecessor's flag
+  int ticket_base;              // first ticket handed out (> 0 only in the missing-predecessor test)
+  int single_kind;              // only one of the two kernels was launched
 };
 
 
@@ -148,6 +151,26 @@ template <> struct Vec<float, 4> {
   }
 };
 
+
+// Thread 0 waits until *flag is non-zero and returns it; -1 once the wait has
+// taken longer than limit_ns (JAMBA_ERR_TIMEOUT is latched in err) or another
+// thread has raised an error.
+__device__ __forceinline__ int wait_flag(const int* flag, int* err, unsigned long long limit_ns) {
+  int f = ld_acquire(flag);
+  if (f != 0) return f;
+  const uint64_t start = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    f = ld_acquire(flag);
+    if (f != 0) return f;
+    if ((it & 255) == 0) {
+      if (error_raised(err)) return -1;
+      if (globaltimer() - start > limit_ns) {
+        set_error(err, JAMBA_ERR_TIMEOUT);
+        return -1;
+      }
+    }
+  }
+}
 
 // Per-CTA context shared by the passes.
 struct ScanCtx {
@@ -367,7 +390,7 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
   const uint32_t full0 = smem_u32(smem + Lyt::OFF_BAR);
   const uint32_t ready0 = full0 + 8 * SCAN_STAGES, empty0 = ready0 + 8 * SCAN_STAGES;
   if (tid == 0) {
-    s_ticket = atomicAdd(a.ticket + (FAST ? 0 : 1), 1);
+    s_ticket = atomicAdd(a.ticket + (FAST ? 0 : 1), 1) + a.ticket_base;
     for (int s = 0; s < SCAN_STAGES; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(ready0 + 8 * s, 32);
@@ -415,7 +438,12 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
     }
   }
   const bool structured = (__syncthreads_and(ok) != 0) && sizeof(TX) == 2;
-  if (structured != FAST) return;   // the other kernel of the pair owns these channels
+  if (structured != FAST) {
+    // the other kernel of the pair owns these channels; when it was not
+    // launched (A changed form after the caller read it) say so
+    if (a.single_kind && tid == 0) set_error(a.err, JAMBA_ERR_INVALID_ARG);
+    return;
+  }
   const float* sA2c = FAST ? nullptr : sA2 + cl * NS;
 
   const bool known = cx.chunk == 0;
@@ -491,22 +519,10 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
         sH[cl * NS + n] = 0.f;
       }
     int jc = cx.chunk - 1;
-    bool done = false;
+    bool done = false, seen0 = false;
     while (!done) {
-      if (tid == 0) {
-        int f = ld_acquire(a.flags + rbase + jc);
-        if (f == 0) {
-          const uint64_t start = globaltimer();
-          for (uint32_t it = 1; f == 0; ++it) {
-            f = ld_acquire(a.flags + rbase + jc);
-            if (f == 0 && (it & 255) == 0) {
-              if (error_raised(a.err)) { f = -1; break; }
-              if (globaltimer() - start > kWaitLimitNs) { set_error(a.err, JAMBA_ERR_TIMEOUT); f = -1; break; }
-            }
-          }
-        }
-        s_flag = f;
-      }
+      seen0 = jc == 0;
+      if (tid == 0) s_flag = wait_flag(a.flags + rbase + jc, a.err, a.wait_ns);
       __syncthreads();
       const int f = s_flag;
       if (f < 0) return;   // every thread read the same value
@@ -532,6 +548,15 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
         if (__syncthreads_and(allzero)) done = true;
       }
       __syncthreads();
+    }
+    // When the final state overwrites the initial one (h_out == h0, a prefill
+    // continuing in place), chunk 0 must have read h0 before the last chunk
+    // writes: a look-back that stopped early never saw chunk 0's flag, which
+    // chunk 0 publishes after its first pass, long after reading h0.
+    if (cx.t1 == a.L && a.h_out && a.h_out == a.h0 && !seen0) {
+      if (tid == 0) s_flag = wait_flag(a.flags + rbase, a.err, a.wait_ns);
+      __syncthreads();
+      if (s_flag < 0) return;
     }
     // The true end state (h + P_end * h_in, published as this chunk's
     // inclusive record unless already final) and the final state of the batch
@@ -730,11 +755,29 @@ static jamba_status launch_scan(const ScanCall& s, cudaStream_t st) {
   a.rec = reinterpret_cast<float*>(w + 256 + flags_bytes);
   a.err = s.err ? s.err : device_error_word();
   if (!a.err) return fail(JAMBA_ERR_CUDA, "could not allocate the device status word");
+  a.wait_ns = s.wait_ns ? s.wait_ns : kWaitLimitNs;
+  a.ticket_base = 0;
+  size_t grid = recs;
+  if (s.skip_first_chunk) {
+    // test of the bounded waits: the CTAs of chunk 0 are never launched, so
+    // every flag of chunk 0 stays unpublished and the look-backs give up
+    a.ticket_base = s.batch * a.cgroups;
+    if (a.n_chunks < 2) return fail(JAMBA_ERR_INVALID_ARG, "scan: the missing-predecessor test needs two chunks");
+    grid = recs - (size_t)a.ticket_base;
+  }
   JB_CUDA(cudaMemsetAsync(w, 0, 256 + flags_bytes, st));
   if (recs > 0x7fffffffull) return fail(JAMBA_ERR_UNSUPPORTED, "scan: too many chunks");
-  if (sizeof(TX) == 2)
-    JB_TRY((launch_kernel<TX, TBC, true, FastShape::CPT, FastShape::MINB>(recs, mx, mz, mdt, mB, mC, a, st)));
-  return launch_kernel<TX, TBC, false, GenShape::CPT, GenShape::MINB>(recs, mx, mz, mdt, mB, mC, a, st);
+  // A's form picks the kernel: the power form (bf16 only) when A[c, n] = (n + 1) A[c, 0]
+  // everywhere, the general one otherwise; unknown form: both launch and each
+  // CTA runs in the kernel its channels belong to
+  const bool fast_ok = sizeof(TX) == 2 && s.a_form != SCAN_A_GENERAL;
+  const bool gen_ok = sizeof(TX) != 2 || s.a_form != SCAN_A_POWER;
+  a.single_kind = sizeof(TX) == 2 && s.a_form != SCAN_A_UNKNOWN;
+  if (fast_ok)
+    JB_TRY((launch_kernel<TX, TBC, true, FastShape::CPT, FastShape::MINB>(grid, mx, mz, mdt, mB, mC, a, st)));
+  if (gen_ok)
+    JB_TRY((launch_kernel<TX, TBC, false, GenShape::CPT, GenShape::MINB>(grid, mx, mz, mdt, mB, mC, a, st)));
+  return JAMBA_OK;
 }
 
 jamba_status scan_run(const ScanCall& s, cudaStream_t st) {

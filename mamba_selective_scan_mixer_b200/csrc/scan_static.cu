@@ -30,13 +30,15 @@ struct StaticAddrs {
 
 constexpr int kMaxDev = 64;
 
+StaticAddrs g_cache[kMaxDev];
+std::mutex g_mu;
+
 jamba_status static_addrs(StaticAddrs* out) {
-  static StaticAddrs cache[kMaxDev];
-  static std::mutex mu;
   int dev = -1;
   JB_CUDA(cudaGetDevice(&dev));
   if (dev < 0 || dev >= kMaxDev) return fail(JAMBA_ERR_UNSUPPORTED, "static scan: device index out of range");
-  std::lock_guard<std::mutex> lock(mu);
+  std::lock_guard<std::mutex> lock(g_mu);
+  StaticAddrs* cache = g_cache;
   if (!cache[dev].scratch) {
     void* p = nullptr;
     void* q = nullptr;
@@ -50,6 +52,26 @@ jamba_status static_addrs(StaticAddrs* out) {
 }
 
 }  // namespace
+
+// Reads and clears the static status word of the current device: the word
+// the static scan latches a timeout in when its caller passes no status.
+// Nothing to read (JAMBA_OK) until a static call has run on this device.
+jamba_status static_scan_status_take(int* value) {
+  *value = 0;
+  int dev = -1;
+  JB_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDev) return JAMBA_OK;
+  int* w = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    w = g_cache[dev].status;
+  }
+  if (!w) return JAMBA_OK;
+  JB_CUDA(cudaMemcpy(value, w, sizeof(int), cudaMemcpyDeviceToHost));
+  if (*value != 0) JB_CUDA(cudaMemset(w, 0, sizeof(int)));
+  return JAMBA_OK;
+}
+
 }  // namespace jb
 
 using namespace jb;
@@ -70,14 +92,15 @@ extern "C" jamba_status jamba_selective_scan_static(const void* x, int ld_x, con
   if ((h0 && !aligned16(h0)) || (h_out && !aligned16(h_out)))
     return fail(JAMBA_ERR_INVALID_ARG, "static scan: misaligned state");
 
-  // the automatic chunk, lengthened until the chunk records fit the array
+  // The automatic chunk gives at most one record per resident CTA (a few
+  // hundred records, well inside the array); should it not fit, one chunk per
+  // channel group is the smallest layout there is.
   int chunk = scan_auto_chunk(batch, seqlen, d_inner, dtype, bc_dtype);
-  while (scan_workspace_bytes(batch, seqlen, d_inner, chunk) > kStaticScratchBytes && chunk < seqlen)
-    chunk = chunk * 2 < seqlen ? chunk * 2 : ((seqlen + 15) & ~15);
+  if (scan_workspace_bytes(batch, seqlen, d_inner, chunk) > kStaticScratchBytes) chunk = (seqlen + 15) & ~15;
   if (scan_workspace_bytes(batch, seqlen, d_inner, chunk) > kStaticScratchBytes)
     return fail(JAMBA_ERR_UNSUPPORTED,
                 "static scan: batch * ceil(d_inner / 256) = " + std::to_string((long long)batch * ((d_inner + 255) / 256)) +
-                    " channel groups need more than the 32 MiB static scratch (at most 680 groups)");
+                    " channel groups need more than the 32 MiB static scratch (at most 682 groups)");
 
   StaticAddrs sa;
   JB_TRY(static_addrs(&sa));

@@ -64,14 +64,42 @@ def test_static_scratch_scan_matches_workspace_scan(J, dtype, a_init, batch, L, 
     assert int(status.item()) == 0
 
 
-def test_static_scratch_scan_rejects_sizes_beyond_the_array(J):
+def test_static_scratch_scan_without_status_word(J):
+    """status = NULL: the library's own word, read and cleared by jamba_device_status."""
+    dev = torch.device("cuda:0")
+    s = {k: v.to(dev) for k, v in scan_inputs(1, 2000, 512, 16, seed=5, dtype="bf16").items()}
+    ref_y, ref_h = J.selective_scan(s["x"], s["z"], s["dt"], s["B"], s["C"], s["A"], s["D"])
+    for _ in range(2):
+        y, h = _static_call(J, s, None, None)
+        torch.cuda.synchronize()
+        assert rel_l2(to_np(y), to_np(ref_y)) < TOL_BF16
+        assert rel_l2(to_np(h), to_np(ref_h)) < TOL_BF16
+    J.device_status()   # raises on a latched timeout
+
+
+def test_static_scratch_scan_at_the_group_limit(J):
+    """682 channel groups fit the array: batch 21 at d_inner 8192 (672 groups) runs
+    with one time chunk per group and matches the workspace scan."""
+    dev = torch.device("cuda:0")
+    s = {k: v.to(dev) for k, v in scan_inputs(21, 48, 8192, 16, seed=21, dtype="bf16").items()}
+    ref_y, ref_h = J.selective_scan(s["x"], s["z"], s["dt"], s["B"], s["C"], s["A"], s["D"])
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    y, h = _static_call(J, s, None, status)
+    torch.cuda.synchronize()
+    assert rel_l2(to_np(y), to_np(ref_y)) < TOL_BF16
+    assert rel_l2(to_np(h), to_np(ref_h)) < TOL_BF16
+    assert int(status.item()) == 0
+
+
+@pytest.mark.parametrize("batch", [22, 86])
+def test_static_scratch_scan_rejects_sizes_beyond_the_array(J, batch):
     from mamba_selective_scan_mixer_b200 import _abi
     dev = torch.device("cuda:0")
     t = torch.zeros(16, device=dev)
     p = ctypes.c_void_p(t.data_ptr())
-    # batch 86 at d_inner 8192: 2752 channel groups, 48 KiB of records each even with one chunk
+    # batch 22 at d_inner 8192: 704 channel groups, 48 KiB of records each even with one chunk
     st = _abi.lib().jamba_selective_scan_static(p, 8192, p, 8192, p, 8192, p, 16, p, 16, _abi.JAMBA_BF16, p, p,
-                                                None, p, 8192, None, 86, 64, 8192, 16, _abi.JAMBA_BF16, None,
+                                                None, p, 8192, None, batch, 64, 8192, 16, _abi.JAMBA_BF16, None,
                                                 ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == 2   # JAMBA_ERR_UNSUPPORTED, nothing launched
     assert b"static scratch" in _abi.lib().jamba_last_error()
