@@ -438,9 +438,12 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
     }
   }
   const bool structured = (__syncthreads_and(ok) != 0) && sizeof(TX) == 2;
-  if (structured != FAST) {
-    // the other kernel of the pair owns these channels; when it was not
-    // launched (A changed form after the caller read it) say so
+  // Both kernels launched: each CTA runs in the kernel of its channels' form.
+  // One launched: the general kernel takes every CTA; the power form cannot
+  // take channels outside its form (A changed after the caller read it), which
+  // is reported instead of computed.
+  const bool mine = a.single_kind ? (!FAST || structured) : structured == FAST;
+  if (!mine) {
     if (a.single_kind && tid == 0) set_error(a.err, JAMBA_ERR_INVALID_ARG);
     return;
   }
