@@ -157,6 +157,70 @@ jamba_status jamba_mamba_step(jamba_mamba_t h, const void* u, const void* residu
                               int batch, float* conv_state, float* ssm_state, void* ws,
                               size_t ws_bytes, jamba_stream_t stream);
 
+/* ------------------------------------------- context-parallel prefill */
+
+/* Prefill of sequences split over ranks by time (context parallelism): rank r
+ * holds tokens [t_r, t_r+1) of every batch row.  The Jamba summary page
+ * names sequence parallelism among its training-infrastructure parallelisms
+ * (appendix on training infrastructure) and the news article names MoE
+ * parallelism and a faster Mamba as future speed-ups; the pages give no
+ * scheme.  Here the split follows the scan's associativity: the state after
+ * a slice is P (.) h_in + h_loc, with P the product of the slice's decays
+ * exp(dt A) and h_loc the slice's end state from zero, so each rank scans
+ * its slice once without the state entering it and once with it, and only
+ * these [batch, d_inner, d_state] carries (plus a 3-token conv halo) cross
+ * between ranks.  The exchanges are the caller's (two small collectives):
+ *   1. before begin: the d_conv - 1 = 3 input rows preceding the slice (the
+ *      last 3 rows of rank r-1's u) reach rank r as u_halo;
+ *   2. between begin and finish: every rank's (carry_p, carry_h) gathered in
+ *      rank order.
+ *
+ * Bytes of workspace the two calls need (the same workspace must be passed,
+ * unchanged, to both: it carries the slice's activations between them). */
+jamba_status jamba_mamba_cp_workspace_size(jamba_mamba_t h, int batch, int seqlen, size_t* bytes);
+
+/* in_proj, causal conv + SiLU, x_proj, inner RMSNorms and dt_proj of the
+ * slice, then a state-only scan of it from zero:
+ *   u       [batch, seqlen, d_model] dtype, this rank's tokens
+ *   u_halo  [batch, 3, d_model] dtype: the 3 input rows before the slice
+ *           (ranks > 0), or NULL
+ *   conv_state_in  [batch, d_inner, 3] fp32 or NULL: the conv cache before
+ *           the first slice (rank 0; NULL = zeros).  At most one of u_halo
+ *           and conv_state_in.
+ *   ssm_state_in   [batch, d_inner, 16] fp32 or NULL: the state before the
+ *           first slice (rank 0 only; it seeds rank 0's carry_h, so the
+ *           other ranks never need it)
+ *   conv_state_out [batch, d_inner, 3] fp32: the slice's last 3 pre-conv
+ *           inputs (the global conv cache on the last rank)
+ *   carry_p [batch, d_inner, 16] fp32 out: the slice's decay product per state
+ *   carry_h [batch, d_inner, 16] fp32 out: the slice's end state from zero
+ *           (rank 0: from ssm_state_in)
+ * Errors: INVALID_ARG (null / misaligned, both halo sources), WORKSPACE,
+ * UNSUPPORTED (too many tokens), CUDA. */
+jamba_status jamba_mamba_prefill_cp_begin(jamba_mamba_t h, const void* u, const void* u_halo, int batch,
+                                          int seqlen, const float* conv_state_in, const float* ssm_state_in,
+                                          float* conv_state_out, float* carry_p, float* carry_h, void* ws,
+                                          size_t ws_bytes, jamba_stream_t stream);
+
+/* The state entering the slice, h_in = fold over j < rank of
+ * P_j (.) h + h_j starting from zero (rank 0: h_in = ssm_state_in), then the
+ * selective scan of the slice from h_in with D skip and SiLU(z) gate, and
+ * out_proj.
+ *   carries_p, carries_h [world][batch][d_inner][16] fp32: every rank's
+ *           carry_p / carry_h in rank order (entries 0 .. rank-1 are read;
+ *           may be NULL on rank 0)
+ *   ssm_state_in  [batch, d_inner, 16] fp32 or NULL: rank 0 only, as in begin
+ *           (INVALID_ARG on other ranks)
+ *   ssm_state_out [batch, d_inner, 16] fp32: state after this rank's slice
+ *           (the global final state on the last rank)
+ *   out [batch, seqlen, d_model] dtype; residual as in jamba_mamba_prefill
+ * Errors: INVALID_ARG, WORKSPACE, CUDA. */
+jamba_status jamba_mamba_prefill_cp_finish(jamba_mamba_t h, const void* residual, void* out, int batch,
+                                           int seqlen, int rank, const float* carries_p,
+                                           const float* carries_h, const float* ssm_state_in,
+                                           float* ssm_state_out, void* ws, size_t ws_bytes,
+                                           jamba_stream_t stream);
+
 /* ------------------------------------------------------- selective scan */
 
 /* Bytes of workspace jamba_selective_scan needs (chunk 0 = automatic). */

@@ -46,10 +46,13 @@ struct PrefillWs {
   void* xz; void* xc; float* xpart; void* dtlow; float* bc; float* dt; void* y; float* conv_tmp; void* scan;
   size_t scan_bytes;
   int splits, chunk;
+  // context-parallel prefill only: in_proj rows of the 3 input tokens before
+  // the slice, the conv cache they make, and the state entering the slice
+  void* xz_halo; float* conv_halo; float* h_in;
   size_t total;
 };
 
-PrefillWs carve_prefill(const jamba_mamba_config& c, int batch, int L, void* ws) {
+PrefillWs carve_prefill(const jamba_mamba_config& c, int batch, int L, void* ws, bool cp = false) {
   PrefillWs p;
   const size_t T = (size_t)batch * L;
   const int es = esize(c.dtype);
@@ -67,9 +70,16 @@ PrefillWs carve_prefill(const jamba_mamba_config& c, int batch, int L, void* ws)
   p.conv_tmp = cv.take<float>((size_t)batch * c.d_inner * (c.d_conv - 1) * 4);
   p.scan_bytes = scan_workspace_bytes(batch, L, c.d_inner, p.chunk);
   p.scan = cv.take(p.scan_bytes);
+  p.xz_halo = p.conv_halo = p.h_in = nullptr;
+  if (cp) {
+    p.xz_halo = cv.take((size_t)batch * (c.d_conv - 1) * 2 * c.d_inner * es);
+    p.conv_halo = cv.take<float>((size_t)batch * c.d_inner * (c.d_conv - 1) * 4);
+    p.h_in = cv.take<float>((size_t)batch * c.d_inner * c.d_state * 4);
+  }
   p.total = cv.off;
   return p;
 }
+
 
 struct StepWs {
   void* xz; void* xc; float* xpart; void* dtlow; float* bc; float* dt; void* y; float* opart;
@@ -124,6 +134,72 @@ jamba_status check_device(const jamba_mamba* h) {
   JB_CUDA(cudaGetDevice(&dev));
   if (dev != h->device) return fail(JAMBA_ERR_INVALID_ARG, "handle was created on another device");
   return JAMBA_OK;
+}
+
+// The prefill up to the scan's inputs: in_proj, conv + SiLU (cache in -> out),
+// x_proj, inner RMSNorms, dt_proj + softplus.
+jamba_status prefill_front(const jamba_mamba& h, const PrefillWs& p, const void* u, int batch, int seqlen,
+                           const float* conv_state_in, float* conv_state_out, cudaStream_t s) {
+  const jamba_mamba_config& c = h.cfg;
+  const jamba_mamba_weights& w = h.w;
+  const int T = batch * seqlen, di = c.d_inner, dm = c.d_model, R = c.dt_rank, N = c.d_state;
+  const int W = R + 2 * N;
+  // in_proj: xz = u W_in^T
+  JB_TRY(gemm_any(c.dtype, gdesc(u, dm, w.in_proj, dm, T, 2 * di, dm, c.dtype == JAMBA_BF16 ? EPI_BF16 : EPI_F32,
+                                 p.xz, 2 * di), s));
+  // conv + SiLU (cache in -> out; an aliased cache is copied first)
+  const float* cin = conv_state_in;
+  if (cin && cin == conv_state_out) {
+    JB_CUDA(cudaMemcpyAsync(p.conv_tmp, cin, sizeof(float) * (size_t)batch * di * 3, cudaMemcpyDeviceToDevice, s));
+    cin = p.conv_tmp;
+  }
+  JB_TRY(conv_prefill(p.xz, 2 * di, w.conv_w, w.conv_b, p.xc, cin, conv_state_out, batch, seqlen, di, c.dtype, s));
+  // x_proj (split-K partials) -> sum + inner RMSNorms
+  GemmDesc gx = gdesc(p.xc, di, w.x_proj, di, T, W, di, EPI_F32, p.xpart, W);
+  gx.splits = p.splits;
+  gx.split_stride = (long long)T * W;
+  if (c.dtype == JAMBA_BF16) gx.bn = 144;
+  JB_TRY(gemm_any(c.dtype, gx, s));
+  JB_TRY(xproj_norm(p.xpart, p.splits, (long long)T * W, T, R, N, w.norm_dt, w.norm_B, w.norm_C, c.inner_rmsnorm,
+                    c.eps, p.dtlow, p.bc, c.dtype, s));
+  // dt = softplus(dt_low W_dt^T + dt_bias)
+  GemmDesc gd = gdesc(p.dtlow, R, w.dt_proj, R, T, di, R, EPI_SOFTPLUS, p.dt, di);
+  gd.bias = w.dt_bias;
+  return gemm_any(c.dtype, gd, s);
+}
+
+// The scan's arguments over the front's outputs.
+ScanCall scan_call(const jamba_mamba& h, const PrefillWs& p, int batch, int seqlen) {
+  const jamba_mamba_config& c = h.cfg;
+  const int di = c.d_inner, N = c.d_state;
+  ScanCall sc = {};
+  sc.x = p.xc; sc.ld_x = di;
+  sc.z = reinterpret_cast<const uint8_t*>(p.xz) + (size_t)di * esize(c.dtype); sc.ld_z = 2 * di;
+  sc.dt = p.dt; sc.ld_dt = di;
+  sc.B = p.bc; sc.ld_b = 2 * N;
+  sc.C = p.bc + N; sc.ld_c = 2 * N;
+  sc.bc_dtype = JAMBA_F32;
+  sc.A = h.w.A; sc.D = h.w.D;
+  sc.y = p.y; sc.ld_y = di;
+  sc.batch = batch; sc.L = seqlen; sc.di = di; sc.dtype = c.dtype; sc.chunk = p.chunk;
+  sc.ws = p.scan; sc.ws_bytes = p.scan_bytes;
+  sc.a_form = h.a_form;
+  return sc;
+}
+
+// The prefill from the scan on: selective scan + D skip + SiLU(z) gate, out_proj (+ residual).
+jamba_status prefill_back(const jamba_mamba& h, const PrefillWs& p, int batch, int seqlen, const float* ssm_state_in,
+                          float* ssm_state_out, const void* residual, void* out, cudaStream_t s) {
+  const jamba_mamba_config& c = h.cfg;
+  const int T = batch * seqlen, di = c.d_inner, dm = c.d_model;
+  ScanCall sc = scan_call(h, p, batch, seqlen);
+  sc.h0 = ssm_state_in;
+  sc.h_out = ssm_state_out;
+  JB_TRY(scan_run(sc, s));
+  GemmDesc go = gdesc(p.y, di, h.w.out_proj, di, T, dm, di, c.dtype == JAMBA_BF16 ? EPI_BF16 : EPI_F32, out, dm);
+  go.residual = residual;
+  go.ldr = dm;
+  return gemm_any(c.dtype, go, s);
 }
 
 }  // namespace
@@ -243,57 +319,90 @@ jamba_status jamba_mamba_prefill(jamba_mamba_t h, const void* u, const void* res
   JB_TRY(check_ptr(ws, "workspace"));
   if (u == out) return fail(JAMBA_ERR_INVALID_ARG, "prefill: out may not alias u");
   const jamba_mamba_config& c = h->cfg;
-  const jamba_mamba_weights& w = h->w;
   if ((long long)batch * seqlen > (1LL << 31) / 2) return fail(JAMBA_ERR_UNSUPPORTED, "prefill: too many tokens");
   PrefillWs p = carve_prefill(c, batch, seqlen, ws);
   if (ws_bytes < p.total) return fail(JAMBA_ERR_WORKSPACE, "prefill: workspace too small");
   cudaStream_t s = cs(stream);
-  const int T = batch * seqlen, di = c.d_inner, dm = c.d_model, R = c.dt_rank, N = c.d_state;
-  const int W = R + 2 * N;
+  JB_TRY(prefill_front(*h, p, u, batch, seqlen, conv_state_in, conv_state_out, s));
+  return prefill_back(*h, p, batch, seqlen, ssm_state_in, ssm_state_out, residual, out, s);
+}
 
-  // in_proj: xz = u W_in^T
-  JB_TRY(gemm_any(c.dtype, gdesc(u, dm, w.in_proj, dm, T, 2 * di, dm, c.dtype == JAMBA_BF16 ? EPI_BF16 : EPI_F32,
-                                 p.xz, 2 * di), s));
-  // conv + SiLU (cache in -> out; an aliased cache is copied first)
-  const float* cin = conv_state_in;
-  if (cin && cin == conv_state_out) {
-    JB_CUDA(cudaMemcpyAsync(p.conv_tmp, cin, sizeof(float) * (size_t)batch * di * 3, cudaMemcpyDeviceToDevice, s));
-    cin = p.conv_tmp;
-  }
-  JB_TRY(conv_prefill(p.xz, 2 * di, w.conv_w, w.conv_b, p.xc, cin, conv_state_out, batch, seqlen, di, c.dtype, s));
-  // x_proj (split-K partials) -> sum + inner RMSNorms
-  GemmDesc gx = gdesc(p.xc, di, w.x_proj, di, T, W, di, EPI_F32, p.xpart, W);
-  gx.splits = p.splits;
-  gx.split_stride = (long long)T * W;
-  if (c.dtype == JAMBA_BF16) gx.bn = 144;
-  JB_TRY(gemm_any(c.dtype, gx, s));
-  JB_TRY(xproj_norm(p.xpart, p.splits, (long long)T * W, T, R, N, w.norm_dt, w.norm_B, w.norm_C, c.inner_rmsnorm,
-                    c.eps, p.dtlow, p.bc, c.dtype, s));
-  // dt = softplus(dt_low W_dt^T + dt_bias)
-  GemmDesc gd = gdesc(p.dtlow, R, w.dt_proj, R, T, di, R, EPI_SOFTPLUS, p.dt, di);
-  gd.bias = w.dt_bias;
-  JB_TRY(gemm_any(c.dtype, gd, s));
-  // selective scan + D skip + SiLU(z) gate
-  ScanCall sc = {};
-  sc.x = p.xc; sc.ld_x = di;
-  sc.z = reinterpret_cast<const uint8_t*>(p.xz) + (size_t)di * esize(c.dtype); sc.ld_z = 2 * di;
-  sc.dt = p.dt; sc.ld_dt = di;
-  sc.B = p.bc; sc.ld_b = 2 * N;
-  sc.C = p.bc + N; sc.ld_c = 2 * N;
-  sc.bc_dtype = JAMBA_F32;
-  sc.A = w.A; sc.D = w.D; sc.h0 = ssm_state_in;
-  sc.y = p.y; sc.ld_y = di;
-  sc.h_out = ssm_state_out;
-  sc.batch = batch; sc.L = seqlen; sc.di = di; sc.dtype = c.dtype; sc.chunk = p.chunk;
-  sc.ws = p.scan; sc.ws_bytes = p.scan_bytes;
-  sc.a_form = h->a_form;
-  JB_TRY(scan_run(sc, s));
-  // out_proj (+ residual)
-  GemmDesc go = gdesc(p.y, di, w.out_proj, di, T, dm, di, c.dtype == JAMBA_BF16 ? EPI_BF16 : EPI_F32, out, dm);
-  go.residual = residual;
-  go.ldr = dm;
-  JB_TRY(gemm_any(c.dtype, go, s));
+// ------------------------------------------------- context-parallel prefill
+
+jamba_status jamba_mamba_cp_workspace_size(jamba_mamba_t h, int batch, int seqlen, size_t* bytes) {
+  if (!h || !bytes || batch <= 0 || seqlen <= 0) return fail(JAMBA_ERR_INVALID_ARG, "cp workspace_size: bad argument");
+  *bytes = carve_prefill(h->cfg, batch, seqlen, nullptr, true).total;
   return JAMBA_OK;
+}
+
+jamba_status jamba_mamba_prefill_cp_begin(jamba_mamba_t h, const void* u, const void* u_halo, int batch, int seqlen,
+                                          const float* conv_state_in, const float* ssm_state_in,
+                                          float* conv_state_out, float* carry_p, float* carry_h, void* ws,
+                                          size_t ws_bytes, jamba_stream_t stream) {
+  if (!h) return fail(JAMBA_ERR_INVALID_ARG, "cp begin: null handle");
+  if (batch <= 0 || seqlen <= 0) return fail(JAMBA_ERR_INVALID_ARG, "cp begin: batch and seqlen must be positive");
+  JB_TRY(check_device(h));
+  JB_TRY(check_ptr(u, "u"));
+  JB_TRY(check_ptr(u_halo, "u_halo", false));
+  JB_TRY(check_ptr(conv_state_in, "conv_state_in", false));
+  JB_TRY(check_ptr(ssm_state_in, "ssm_state_in", false));
+  JB_TRY(check_ptr(conv_state_out, "conv_state_out"));
+  JB_TRY(check_ptr(carry_p, "carry_p"));
+  JB_TRY(check_ptr(carry_h, "carry_h"));
+  JB_TRY(check_ptr(ws, "workspace"));
+  if (u_halo && conv_state_in) return fail(JAMBA_ERR_INVALID_ARG, "cp begin: pass u_halo or conv_state_in, not both");
+  if (conv_state_in && conv_state_in == conv_state_out)
+    return fail(JAMBA_ERR_INVALID_ARG, "cp begin: conv_state_out may not alias conv_state_in");
+  if (ssm_state_in && (ssm_state_in == carry_h || ssm_state_in == carry_p))
+    return fail(JAMBA_ERR_INVALID_ARG, "cp begin: the carries may not alias ssm_state_in");
+  const jamba_mamba_config& c = h->cfg;
+  if ((long long)batch * seqlen > (1LL << 31) / 2) return fail(JAMBA_ERR_UNSUPPORTED, "cp begin: too many tokens");
+  PrefillWs p = carve_prefill(c, batch, seqlen, ws, true);
+  if (ws_bytes < p.total) return fail(JAMBA_ERR_WORKSPACE, "cp begin: workspace too small");
+  cudaStream_t s = cs(stream);
+  const int di = c.d_inner, dm = c.d_model, K1 = c.d_conv - 1;
+  const float* cin = conv_state_in;
+  if (u_halo) {
+    // the conv cache entering the slice: in_proj of the d_conv - 1 input rows before it
+    JB_TRY(gemm_any(c.dtype, gdesc(u_halo, dm, h->w.in_proj, dm, batch * K1, 2 * di, dm,
+                                   c.dtype == JAMBA_BF16 ? EPI_BF16 : EPI_F32, p.xz_halo, 2 * di), s));
+    JB_TRY(conv_halo_state(p.xz_halo, 2 * di, p.conv_halo, batch, di, c.dtype, s));
+    cin = p.conv_halo;
+  }
+  JB_TRY(prefill_front(*h, p, u, batch, seqlen, cin, conv_state_out, s));
+  // the slice's summary: its end state from ssm_state_in (or zero) and its decay product
+  ScanCall sc = scan_call(*h, p, batch, seqlen);
+  sc.h0 = ssm_state_in;
+  sc.z = nullptr;
+  sc.y = nullptr;
+  sc.summary = 1;
+  sc.h_out = carry_h;
+  sc.p_out = carry_p;
+  return scan_run(sc, s);
+}
+
+jamba_status jamba_mamba_prefill_cp_finish(jamba_mamba_t h, const void* residual, void* out, int batch, int seqlen,
+                                           int rank, const float* carries_p, const float* carries_h,
+                                           const float* ssm_state_in, float* ssm_state_out, void* ws, size_t ws_bytes,
+                                           jamba_stream_t stream) {
+  if (!h) return fail(JAMBA_ERR_INVALID_ARG, "cp finish: null handle");
+  if (batch <= 0 || seqlen <= 0 || rank < 0) return fail(JAMBA_ERR_INVALID_ARG, "cp finish: bad sizes or rank");
+  JB_TRY(check_device(h));
+  JB_TRY(check_ptr(out, "out"));
+  JB_TRY(check_ptr(residual, "residual", false));
+  JB_TRY(check_ptr(ssm_state_in, "ssm_state_in", false));
+  JB_TRY(check_ptr(ssm_state_out, "ssm_state_out"));
+  JB_TRY(check_ptr(carries_p, "carries_p", rank > 0));
+  JB_TRY(check_ptr(carries_h, "carries_h", rank > 0));
+  JB_TRY(check_ptr(ws, "workspace"));
+  const jamba_mamba_config& c = h->cfg;
+  PrefillWs p = carve_prefill(c, batch, seqlen, ws, true);
+  if (ws_bytes < p.total) return fail(JAMBA_ERR_WORKSPACE, "cp finish: workspace too small");
+  cudaStream_t s = cs(stream);
+  if (rank == 0) return prefill_back(*h, p, batch, seqlen, ssm_state_in, ssm_state_out, residual, out, s);
+  if (ssm_state_in) return fail(JAMBA_ERR_INVALID_ARG, "cp finish: ssm_state_in is rank 0's (it is in its carry)");
+  JB_TRY(carry_combine(carries_p, carries_h, rank, nullptr, p.h_in, (long long)batch * c.d_inner * c.d_state, s));
+  return prefill_back(*h, p, batch, seqlen, p.h_in, ssm_state_out, residual, out, s);
 }
 
 jamba_status jamba_mamba_step(jamba_mamba_t h, const void* u, const void* residual, void* out, int batch,

@@ -144,6 +144,31 @@ conv_step_kernel(const T* __restrict__ x, long long ld_x, const T* __restrict__ 
   s[2] = xv;
 }
 
+// conv cache [batch, C, 3] (fp32, oldest first) from the in_proj rows of the
+// three tokens before a sequence slice: xz [batch * 3, *], x in the first C columns
+template <typename T>
+__global__ void __launch_bounds__(256)
+conv_halo_kernel(const T* __restrict__ xz, long long ld, float* __restrict__ state, int batch, int C) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;   // flat (row, channel, tap)
+  if (i >= (long long)batch * C * 3) return;
+  const int k = (int)(i % 3);
+  const long long bc = i / 3;
+  const int b = (int)(bc / C), c = (int)(bc - (long long)b * C);
+  state[i] = to_f(xz[((long long)b * 3 + k) * ld + c]);
+}
+
+jamba_status conv_halo_state(const void* xz, long long ld, float* state, int batch, int C, int dtype,
+                             cudaStream_t s) {
+  const long long n = (long long)batch * C * 3;
+  const unsigned grid = (unsigned)((n + 255) / 256);
+  if (dtype == JAMBA_BF16)
+    conv_halo_kernel<bf16><<<grid, 256, 0, s>>>(reinterpret_cast<const bf16*>(xz), ld, state, batch, C);
+  else
+    conv_halo_kernel<float><<<grid, 256, 0, s>>>(reinterpret_cast<const float*>(xz), ld, state, batch, C);
+  JB_CUDA(cudaGetLastError());
+  return JAMBA_OK;
+}
+
 jamba_status conv_prefill(const void* x, long long ld_x, const void* w, const void* b, void* out,
                           const float* st_in, float* st_out, int batch, int L, int C, int dtype, cudaStream_t s) {
   const int V = dtype == JAMBA_BF16 ? 8 : 4;

@@ -111,12 +111,17 @@ struct ScanCall {
   int a_form;                    // SCAN_A_*: which kernel owns the channels, when the caller knows
   unsigned long long wait_ns;    // look-back wait limit; 0 = the library default
   int skip_first_chunk;          // test only: launch no CTA for chunk 0 (its flags stay unset)
+  int summary;                   // state-only: no y / z; h_out (required) and p_out (decay product) out
+  float* p_out;
 };
 enum ScanAForm { SCAN_A_UNKNOWN = 0, SCAN_A_POWER = 1, SCAN_A_GENERAL = 2 };
 jamba_status scan_run(const ScanCall& s, cudaStream_t st);
 size_t scan_workspace_bytes(int batch, int L, int di, int chunk_len);
 int scan_auto_chunk(int batch, int L, int di, int dtype, int bc_dtype);
 jamba_status static_scan_status_take(int* value);   // static scan's own status word (read and cleared)
+// context-parallel prefill: the state entering slice `rank` from the slices' carries
+jamba_status carry_combine(const float* P, const float* H, int rank, const float* h_init, float* h_in, long long n,
+                           cudaStream_t st);
 jamba_status ssm_step(const void* xc, const void* z, long long ld_z, const float* dt, const float* bc,
                       long long ld_bc, const float* A, const float* D, float* state, void* y, int batch, int di,
                       int dtype, cudaStream_t st);
@@ -126,6 +131,8 @@ jamba_status conv_prefill(const void* x, long long ld_x, const void* w, const vo
                           const float* st_in, float* st_out, int batch, int L, int C, int dtype, cudaStream_t s);
 jamba_status conv_step(const void* x, long long ld_x, const void* w, const void* b, void* out, float* state,
                        int batch, int C, int dtype, cudaStream_t s);
+jamba_status conv_halo_state(const void* xz, long long ld, float* state, int batch, int C, int dtype,
+                             cudaStream_t s);
 jamba_status rmsnorm(const void* x, const float* w, void* out, int rows, int cols, float eps, int dtype,
                      cudaStream_t s);
 jamba_status xproj_norm(const float* part, int splits, long long split_stride, int T, int R, int N,

@@ -96,6 +96,11 @@ struct ScanArgs {
   unsigned long long wait_ns;   // limit of the look-back waits on a predecessor's flag
   int ticket_base;              // first ticket handed out (> 0 only in the missing-predecessor test)
   int single_kind;              // only one of the two kernels was launched
+  // Summary mode: no outputs; every chunk runs state-only and the last one
+  // writes h_out (the end state from h0, or from zero) and p_out, the decay
+  // product over the whole sequence [batch, di, 16].
+  int summary;
+  float* p_out;
 };
 
 
@@ -186,7 +191,8 @@ struct ScanCtx {
 template <typename TX, typename TBC, bool FAST>
 __device__ __forceinline__ bool producer_pass(const CUtensorMap* mx, const CUtensorMap* mz, const CUtensorMap* mdt,
                                               const CUtensorMap* mB, const CUtensorMap* mC, uint8_t* smem,
-                                              const ScanCtx& cx, int ts, int nsub, int g0, int* err) {
+                                              const ScanCtx& cx, int ts, int nsub, int g0, int* err,
+                                              bool load_z) {
   using Lyt = ScanLayout<TX, TBC, FAST>;
   const int lane = threadIdx.x & 31;
   const uint32_t full0 = smem_u32(smem + Lyt::OFF_BAR);
@@ -198,9 +204,9 @@ __device__ __forceinline__ bool producer_pass(const CUtensorMap* mx, const CUten
     uint8_t* st = smem + slot * Lyt::STAGE;
     const uint32_t bar = full0 + 8 * slot;
     const int row = (int)(cx.row0 + ts + (g - g0) * SCAN_Q);
-    mbar_arrive_tx(bar, Lyt::STAGE_TX);
+    mbar_arrive_tx(bar, Lyt::STAGE_TX - (load_z ? 0 : Lyt::X));
     tma_load_2d(smem_u32(st), mx, bar, cx.c_base, row);
-    tma_load_2d(smem_u32(st + Lyt::OFF_Z), mz, bar, cx.c_base, row);
+    if (load_z) tma_load_2d(smem_u32(st + Lyt::OFF_Z), mz, bar, cx.c_base, row);
     tma_load_2d(smem_u32(st + Lyt::OFF_DT), mdt, bar, cx.c_base, row);
     tma_load_2d(smem_u32(st + Lyt::OFF_B), mB, bar, 0, row);
     tma_load_2d(smem_u32(st + Lyt::OFF_C), mC, bar, 0, row);
@@ -350,7 +356,7 @@ __device__ __forceinline__ bool consumer_pass(uint8_t* smem, const ScanCtx& cx, 
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(empty0 + 8 * slot);
-    if (MAY_HEAD && head) {
+    if (MAY_HEAD && head && !a.summary) {
       bool zero = !valid;
       if (!zero) {
         zero = true;
@@ -469,14 +475,14 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
 #pragma unroll
     for (int i = 0; i < 8; ++i) P[j][i] = make_float2(1.f, 1.f);
   }
-  bool head = !known;
+  bool head = !known || a.summary;   // summary mode: state-only from the first step
   int t_head_end = cx.t0;
 
   // ---------------------------------------------------------- pass 1
   const int nsub1 = (cx.t1 - cx.t0 + SCAN_Q - 1) / SCAN_Q;
   bool pass_ok;
   if (producer)
-    pass_ok = producer_pass<TX, TBC, FAST>(&mx, &mz, &mdt, &mB, &mC, smem, cx, cx.t0, nsub1, 0, a.err);
+    pass_ok = producer_pass<TX, TBC, FAST>(&mx, &mz, &mdt, &mB, &mC, smem, cx, cx.t0, nsub1, 0, a.err, !a.summary);
   else
     pass_ok = consumer_pass<TX, TBC, FAST, CPT, true>(smem, cx, a, cx.t0, cx.t1, cx.t1, nsub1, 0, h, head, t_head_end, R,
                                                 P, A2_0, sA2c, Dv, valid, c);
@@ -488,7 +494,8 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
   const long long rbase = (long long)cx.grp * a.n_chunks;
   float* myrec = a.rec + (rbase + cx.chunk) * REC;
   int* myflag = a.flags + rbase + cx.chunk;
-  const bool independent = __syncthreads_and(producer || !head) != 0;  // end state free of h_in
+  // end state free of h_in: the first chunk (its start state is known), or every warp's head ended
+  const bool independent = (__syncthreads_and(producer || !head) != 0) || known;
   int t_head_max = cx.t0;
   for (int w = 0; w < NCW; ++w) t_head_max = max(t_head_max, s_head_end[w]);
   if (!producer) {
@@ -501,6 +508,7 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
         float* o = myrec + (cl + j) * NS + n;
         if (independent) {
           *reinterpret_cast<float2*>(o + 2 * SCAN_CH * NS) = h[j][n / 2];
+          if (a.summary) *reinterpret_cast<float2*>(o) = make_float2(pe[n], pe[n + 1]);
         } else {
           *reinterpret_cast<float2*>(o) = make_float2(pe[n], pe[n + 1]);
           *reinterpret_cast<float2*>(o + SCAN_CH * NS) = h[j][n / 2];
@@ -511,6 +519,8 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
   __threadfence();
   __syncthreads();
   if (tid == 0) st_release(myflag, independent ? 2 : 1);
+  // summary mode: only the last chunk goes on (to combine the records)
+  if (a.summary && cx.t1 != a.L) return;
 
   if (!known) {
     // look back: h_in = h_{k-1} + P_{k-1} (h_{k-2} + P_{k-2} (... + inclusive_j))
@@ -537,6 +547,7 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
           const int o = cl * NS + n;
           if (f == 2) {
             sH[o] = fmaf(sP[o], __ldcg(rP + 2 * SCAN_CH * NS + o), sH[o]);
+            if (a.summary) sP[o] *= __ldcg(rP + o);   // the first chunk's decay, published beside its state
           } else {
             sH[o] = fmaf(sP[o], __ldcg(rP + SCAN_CH * NS + o), sH[o]);
             sP[o] *= __ldcg(rP + o);
@@ -548,7 +559,8 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
         done = true;
       } else {
         --jc;
-        if (__syncthreads_and(allzero)) done = true;
+        // summary mode walks back to the first chunk: p_out is the whole product
+        if (__syncthreads_and(allzero) && !a.summary) done = true;
       }
       __syncthreads();
     }
@@ -579,6 +591,11 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
             *reinterpret_cast<float2*>(myrec + 2 * SCAN_CH * NS + (cl + j) * NS + 2 * n2) = he;
           }
           if (last) *reinterpret_cast<float2*>(a.h_out + ((long long)cx.b * a.di + c + j) * NS + 2 * n2) = he;
+          if (a.summary && valid) {
+            const float2 pin = make_float2(sP[(cl + j) * NS + 2 * n2], sP[(cl + j) * NS + 2 * n2 + 1]);
+            *reinterpret_cast<float2*>(a.p_out + ((long long)cx.b * a.di + c + j) * NS + 2 * n2) =
+                make_float2(pe[2 * n2] * pin.x, pe[2 * n2 + 1] * pin.y);
+          }
           h[j][n2] = hi;
         }
       }
@@ -590,11 +607,12 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
     fence_async_shared();
     __syncthreads();
     if (!independent && tid == 0) st_release(myflag, 2);
+    if (a.summary) return;
 
     // ---------------------------------------------------------- pass 2: replay the head from h_in
     const int nsub2 = (t_head_max - cx.t0 + SCAN_Q - 1) / SCAN_Q;
     if (producer) {
-      producer_pass<TX, TBC, FAST>(&mx, &mz, &mdt, &mB, &mC, smem, cx, cx.t0, nsub2, nsub1, a.err);
+      producer_pass<TX, TBC, FAST>(&mx, &mz, &mdt, &mB, &mC, smem, cx, cx.t0, nsub2, nsub1, a.err, true);
     } else {
       bool head2 = false;
       int unused = 0;
@@ -602,13 +620,19 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
       consumer_pass<TX, TBC, FAST, CPT, false>(smem, cx, a, cx.t0, t_head_max, s_head_end[warp], nsub2, nsub1, h, head2,
                                         unused, R, P, A2_0, sA2c, Dv, valid, c);
     }
-  } else if (cx.t1 == a.L && a.h_out && valid) {
+  } else if (cx.t1 == a.L && valid) {
     // the first chunk started from the known state: h is the final state of the batch row
 #pragma unroll
-    for (int j = 0; j < CPT; ++j)
+    for (int j = 0; j < CPT; ++j) {
+      float pe[16];
+      chunk_decay<FAST>(R[j], P[j], pe);
 #pragma unroll
-      for (int n2 = 0; n2 < 8; ++n2)
-        *reinterpret_cast<float2*>(a.h_out + ((long long)cx.b * a.di + c + j) * NS + 2 * n2) = h[j][n2];
+      for (int n2 = 0; n2 < 8; ++n2) {
+        const long long o = ((long long)cx.b * a.di + c + j) * NS + 2 * n2;
+        if (a.h_out) *reinterpret_cast<float2*>(a.h_out + o) = h[j][n2];
+        if (a.summary) *reinterpret_cast<float2*>(a.p_out + o) = make_float2(pe[2 * n2], pe[2 * n2 + 1]);
+      }
+    }
   }
 }
 
@@ -650,6 +674,27 @@ ssm_step_kernel(const TX* __restrict__ xc, const TX* __restrict__ z, long long l
     const float zv = to_f(z[(long long)b * ld_z + c]);
     y[ii] = from_f<TX>((part + __ldg(D + c) * x) * silu(zv));
   }
+}
+
+// ------------------------------------------------------------ carries across ranks
+// State entering slice `rank` of a sequence split by time: fold the slices
+// before it, h = P_j * h + h_j for j = 0 .. rank-1, from h_init (or zero).
+__global__ void __launch_bounds__(256)
+carry_combine_kernel(const float* __restrict__ P, const float* __restrict__ H, int rank,
+                     const float* __restrict__ h_init, float* __restrict__ h_in, long long n) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  float h = h_init ? h_init[i] : 0.f;
+  for (int j = 0; j < rank; ++j) h = fmaf(P[(long long)j * n + i], h, H[(long long)j * n + i]);
+  h_in[i] = h;
+}
+
+jamba_status carry_combine(const float* P, const float* H, int rank, const float* h_init, float* h_in, long long n,
+                           cudaStream_t st) {
+  const unsigned grid = (unsigned)((n + 255) / 256);
+  carry_combine_kernel<<<grid, 256, 0, st>>>(P, H, rank, h_init, h_in, n);
+  JB_CUDA(cudaGetLastError());
+  return JAMBA_OK;
 }
 
 // ------------------------------------------------------------ host side
@@ -737,7 +782,10 @@ static jamba_status launch_scan(const ScanCall& s, cudaStream_t st) {
   const uint64_t rows = (uint64_t)s.batch * s.L;
   CUtensorMap mx, mz, mdt, mB, mC;
   JB_TRY(make_map_2d(&mx, s.x, tx, sizeof(TX), s.di, rows, s.ld_x * sizeof(TX), SCAN_CH, SCAN_Q, CU_TENSOR_MAP_SWIZZLE_NONE));
-  JB_TRY(make_map_2d(&mz, s.z, tx, sizeof(TX), s.di, rows, s.ld_z * sizeof(TX), SCAN_CH, SCAN_Q, CU_TENSOR_MAP_SWIZZLE_NONE));
+  // summary mode reads no z: its map is never used, so it may describe x
+  const void* zp = s.z ? s.z : s.x;
+  const long long ldz = s.z ? s.ld_z : s.ld_x;
+  JB_TRY(make_map_2d(&mz, zp, tx, sizeof(TX), s.di, rows, ldz * sizeof(TX), SCAN_CH, SCAN_Q, CU_TENSOR_MAP_SWIZZLE_NONE));
   JB_TRY(make_map_2d(&mdt, s.dt, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, s.di, rows, s.ld_dt * 4, SCAN_CH, SCAN_Q,
                      CU_TENSOR_MAP_SWIZZLE_NONE));
   JB_TRY(make_map_2d(&mB, s.B, tb, sizeof(TBC), NS, rows, s.ld_b * sizeof(TBC), NS, SCAN_Q, CU_TENSOR_MAP_SWIZZLE_NONE));
@@ -759,6 +807,8 @@ static jamba_status launch_scan(const ScanCall& s, cudaStream_t st) {
   a.err = s.err ? s.err : device_error_word();
   if (!a.err) return fail(JAMBA_ERR_CUDA, "could not allocate the device status word");
   a.wait_ns = s.wait_ns ? s.wait_ns : kWaitLimitNs;
+  a.summary = s.summary;
+  a.p_out = s.p_out;
   a.ticket_base = 0;
   size_t grid = recs;
   if (s.skip_first_chunk) {
@@ -786,13 +836,17 @@ static jamba_status launch_scan(const ScanCall& s, cudaStream_t st) {
 jamba_status scan_run(const ScanCall& s, cudaStream_t st) {
   if (s.batch <= 0 || s.L <= 0 || s.di <= 0) return fail(JAMBA_ERR_INVALID_ARG, "scan: sizes must be positive");
   if (s.di % 8) return fail(JAMBA_ERR_UNSUPPORTED, "scan: d_inner must be a multiple of 8");
-  if (!s.x || !s.z || !s.dt || !s.B || !s.C || !s.A || !s.D || !s.y)
+  if (!s.x || !s.dt || !s.B || !s.C || !s.A || !s.D)
+    return fail(JAMBA_ERR_INVALID_ARG, "scan: null tensor");
+  if (s.summary ? (!s.h_out || !s.p_out || !aligned16(s.h_out) || !aligned16(s.p_out)) : (!s.z || !s.y))
     return fail(JAMBA_ERR_INVALID_ARG, "scan: null tensor");
   if (s.chunk <= 0 || s.chunk % 16) return fail(JAMBA_ERR_INVALID_ARG, "scan: chunk must be a positive multiple of 16");
-  if (s.ld_x < s.di || s.ld_z < s.di || s.ld_dt < s.di || s.ld_y < s.di || s.ld_b < NS || s.ld_c < NS)
+  if (s.ld_x < s.di || s.ld_dt < s.di || s.ld_b < NS || s.ld_c < NS ||
+      (!s.summary && (s.ld_z < s.di || s.ld_y < s.di)))
     return fail(JAMBA_ERR_INVALID_ARG, "scan: leading dimension below the row width");
-  if (s.ld_y % 4) return fail(JAMBA_ERR_INVALID_ARG, "scan: the leading dimension of y must be a multiple of 4");
-  if (!aligned16(s.y)) return fail(JAMBA_ERR_INVALID_ARG, "scan: y must be 16-byte aligned");
+  if (!s.summary && s.ld_y % 4)
+    return fail(JAMBA_ERR_INVALID_ARG, "scan: the leading dimension of y must be a multiple of 4");
+  if (!s.summary && !aligned16(s.y)) return fail(JAMBA_ERR_INVALID_ARG, "scan: y must be 16-byte aligned");
   if (s.ws_bytes < scan_workspace_bytes(s.batch, s.L, s.di, s.chunk) || !s.ws || !aligned16(s.ws))
     return fail(JAMBA_ERR_WORKSPACE, "scan: workspace too small");
   if ((long long)s.batch * s.L > 0x7fffffffLL) return fail(JAMBA_ERR_UNSUPPORTED, "scan: too many tokens");

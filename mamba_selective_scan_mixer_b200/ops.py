@@ -110,6 +110,49 @@ class MambaMixer:
                                         ws.numel(), _stream(stream)))
         return out, conv_state_out, ssm_state_out
 
+    def cp_workspace_size(self, batch, seqlen):
+        n = ctypes.c_size_t()
+        check(lib().jamba_mamba_cp_workspace_size(self.handle, batch, seqlen, ctypes.byref(n)))
+        return n.value
+
+    def prefill_cp_begin(self, u, u_halo=None, conv_state_in=None, ssm_state_in=None, stream=None):
+        """First half of a context-parallel prefill on this rank's slice u
+        [B, L, d_model]: returns (conv_state_out, carry_p, carry_h).  The
+        slice's activations stay in this mixer's workspace for
+        prefill_cp_finish."""
+        _cuda(u, u_halo, conv_state_in, ssm_state_in)
+        _contig(u, "u")
+        _contig(u_halo, "u_halo")
+        B, L, _ = u.shape
+        sh = self.shape
+        conv_out = torch.empty(B, sh.d_inner, sh.d_conv - 1, device=u.device)
+        carry_p = torch.empty(B, sh.d_inner, sh.d_state, device=u.device)
+        carry_h = torch.empty_like(carry_p)
+        ws = self.ws.get(self.cp_workspace_size(B, L), u.device)
+        check(lib().jamba_mamba_prefill_cp_begin(self.handle, _p(u), _p(u_halo), B, L, _p(conv_state_in),
+                                                 _p(ssm_state_in), _p(conv_out), _p(carry_p), _p(carry_h),
+                                                 _p(ws), ws.numel(), _stream(stream)))
+        self._cp = (B, L)
+        return conv_out, carry_p, carry_h
+
+    def prefill_cp_finish(self, rank, carries_p, carries_h, ssm_state_in=None, residual=None, out=None,
+                          stream=None):
+        """Second half: carries_* [world, B, d_inner, 16] of every rank in rank
+        order.  Returns (out, ssm_state_out)."""
+        B, L = self._cp
+        _cuda(carries_p, carries_h, ssm_state_in, residual, out)
+        _contig(carries_p, "carries_p")
+        _contig(carries_h, "carries_h")
+        _contig(residual, "residual")
+        sh = self.shape
+        out = torch.empty(B, L, sh.d_model, dtype=self.dtype, device=self.device) if out is None else out
+        ss = torch.empty(B, sh.d_inner, sh.d_state, device=self.device)
+        ws = self.ws.get(self.cp_workspace_size(B, L), self.device)
+        check(lib().jamba_mamba_prefill_cp_finish(self.handle, _p(residual), _p(out), B, L, int(rank),
+                                                  _p(carries_p), _p(carries_h), _p(ssm_state_in), _p(ss), _p(ws),
+                                                  ws.numel(), _stream(stream)))
+        return out, ss
+
     def prefill_host(self, u_host, residual_host=None, out_host=None, chunk=0, conv_state_in=None,
                      ssm_state_in=None, conv_state_out=None, ssm_state_out=None, stream=None):
         """Prefill from and to pinned host tensors [B, L, d_model]; the library
