@@ -55,6 +55,8 @@ def parse():
     ap.add_argument("--pair-seqlen", type=int, default=PAIR_L)
     ap.add_argument("--attn-seqlen", type=int, default=ATTN_L)
     ap.add_argument("--moe8-tokens", type=int, default=64, help="tokens of the moe8dec part")
+    ap.add_argument("--cpu-table", action="store_true",
+                    help="time the fp64 oracle of every workload on this host (single thread and all cores)")
     return ap.parse_args()
 
 
@@ -497,6 +499,88 @@ def run_product(args):
         dist.destroy_process_group()
 
 
+def _host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_table(args):
+    """The fp64 oracle timed on this host for every workload, single-threaded and
+    on all cores, each on a bounded sample of the workload (batch rows, tokens
+    and channels are independent, so per-unit rates carry over; time
+    recurrences are never cut).  One JSON line."""
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+    from oracle import mamba as om
+    from oracle import moe as omoe
+    from synthetic import MoEShape, block_norm_params, mamba_input, mamba_params, moe_params, scan_inputs, \
+        workload
+
+    class _Lazy:   # expert weights widened to fp64 one expert at a time
+        def __init__(self, t):
+            self.t = t
+
+        def __getitem__(self, e):
+            return om.to64(self.t[e])
+
+    def timed(fn):
+        t0 = time.perf_counter()
+        fn()
+        return time.perf_counter() - t0
+
+    tiny = workload("tiny_fp32")
+    jam = workload("prefill_4k")["mamba"]
+    pt = om.params64(mamba_params(tiny["mamba"], seed=0))
+    ut = om.to64(mamba_input(tiny["mamba"], 1, tiny["seqlen"] + tiny["steps"], seed=0))
+
+    def run_tiny():
+        r = om.mamba_prefill(pt, ut[:, :tiny["seqlen"]], tiny["mamba"])
+        cs, ss = r["conv_state"], r["ssm_state"]
+        for t in range(tiny["steps"]):
+            _, cs, ss = om.mamba_step(pt, ut[:, tiny["seqlen"] + t], tiny["mamba"], cs, ss)
+
+    pj = om.params64(mamba_params(jam, seed=0))
+    up = om.to64(mamba_input(jam, 1, 512, seed=0))
+    sc = {k: om.to64(v) for k, v in scan_inputs(1, SCAN_L, 256, 16, seed=0).items()}
+    ud = om.to64(mamba_input(jam, DECODE_B, 4, seed=1))
+    cs0 = np.zeros((DECODE_B, jam.d_inner, 3))
+    ss0 = np.zeros((DECODE_B, jam.d_inner, 16))
+    es = MoEShape()
+    mp = moe_params(es, seed=0)
+    ep = {"router": om.to64(mp["router"]), **{k: _Lazy(mp[k]) for k in ("w_gate", "w_up", "w_down")}}
+    g1, g2 = (om.to64(g) for g in block_norm_params(jam.d_model))
+    xp = om.to64(mamba_input(jam, 1, 256, seed=2))
+
+    def run_decode():
+        cs, ss = cs0, ss0
+        for t in range(4):
+            _, cs, ss = om.mamba_step(pj, ud[:, t], jam, cs, ss)
+
+    cases = [
+        ("tiny_fp32", "prefill of 256 tokens + 16 decode steps (whole workload)", tiny["seqlen"] + tiny["steps"],
+         run_tiny),
+        ("prefill_4k / prefill_128k", "prefill of 512 tokens at Jamba width (the per-token cost of both)", 512,
+         lambda: om.mamba_prefill(pj, up, jam, scan="c")),
+        ("scan_128k", "C scan of 256 of the 8192 channels over all 131072 steps, counted at 8192 channels",
+         SCAN_L * 256 / SCAN_DI,
+         lambda: om.selective_scan_c(sc["x"], sc["dt"], sc["A"], sc["B"], sc["C"], sc["D"], sc["z"])),
+        ("decode_b64", "4 decode steps of all 64 rows at Jamba width", 4 * DECODE_B, run_decode),
+        ("layer_pair", "layer pair on 256 tokens (Mamba + 16-expert top-2 MoE, d_ff 14336)", 256,
+         lambda: omoe.layer_pair(pj, ep, xp, jam, es.top_k, g1, g2, scan="c")),
+    ]
+    rows = {}
+    for name, sample, units, fn in cases:
+        with threadpool_limits(1):
+            t1 = timed(fn)
+        tn = timed(fn)
+        rows[name] = {"sample": sample, "unit": "tokens/s", "single_thread": round(units / t1, 3),
+                      "all_cores": round(units / tn, 3), "seconds": [round(t1, 2), round(tn, 2)]}
+    print(json.dumps({"cpu_table": rows, "cores": _host_cores(), "kind": "oracle",
+                      "note": "the C scan loop is single-threaded; numpy's BLAS uses the cores"}), flush=True)
+
+
 def run_reference(args):
     """The oracle as it stands, on this host's cores, same metric and workload (bounded sample)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -525,7 +609,9 @@ def run_reference(args):
 
 if __name__ == "__main__":
     a = parse()
-    if a.impl == "reference":
+    if a.cpu_table:
+        cpu_table(a)
+    elif a.impl == "reference":
         run_reference(a)
     else:
         run_product(a)
