@@ -47,7 +47,7 @@ def parse():
     ap.add_argument("--impl", default="product", choices=["product", "reference"])
     ap.add_argument("--quick", action="store_true", help="skip the side measurements")
     ap.add_argument("--only", default="all",
-                    help="comma list of parts to run (prefill,gemm,scan,decode,pair,moe8,moe8dec,attn,e2e,cpu); "
+                    help="comma list of parts to run (prefill,gemm,scan,decode,pair,moe8,moe8dec,moe,attn,e2e,cpu); "
                          "for profiling")
     ap.add_argument("--seqlen", type=int, default=PREFILL_L, help="prefill tokens")
     ap.add_argument("--scan-seqlen", type=int, default=SCAN_L)
@@ -55,6 +55,10 @@ def parse():
     ap.add_argument("--pair-seqlen", type=int, default=PAIR_L)
     ap.add_argument("--attn-seqlen", type=int, default=ATTN_L)
     ap.add_argument("--moe8-tokens", type=int, default=64, help="tokens of the moe8dec part")
+    ap.add_argument("--moe-tokens", type=int, default=4096, help="tokens of the moe part (bf16 experts alone)")
+    ap.add_argument("--decode-prefill", type=int, default=DECODE_PREFILL,
+                    help="prefill tokens that fill the decode caches (profiling: a short one keeps the "
+                         "device footprint small; the caches have their full size either way)")
     ap.add_argument("--cpu-table", action="store_true",
                     help="time the fp64 oracle of every workload on this host (single thread and all cores)")
     return ap.parse_args()
@@ -316,7 +320,7 @@ def run_product(args):
         # decode: batch 64, caches from a 2048-token prefill, steps in one CUDA graph
         B = DECODE_B
         NST = args.decode_steps
-        u0 = mamba_input(sh, B, DECODE_PREFILL, seed=1, device=dev)
+        u0 = mamba_input(sh, B, args.decode_prefill, seed=1, device=dev)
         dcs, dss = mixer.new_states(B)
         mixer.prefill(u0, conv_state_out=dcs, ssm_state_out=dss)
         steps_u = decode_inputs(sh, B, NST, seed=1, device=dev)
@@ -335,7 +339,7 @@ def run_product(args):
         wbytes = sum(v.numel() * v.element_size() for v in params.values())
         step_bytes = wbytes + 2 * (B * sh.d_inner * 16 * 4 + B * sh.d_inner * 3 * 4) + 2 * B * sh.d_model * 2
         res["decode"] = {"workload": "decode_b64: batch 64, one token per step, %d steps in one CUDA graph, "
-                                     "caches from a 2048-token prefill" % NST,
+                                     "caches from a %d-token prefill" % (NST, args.decode_prefill),
                          "tokens/s": round(B * NST / (dms / 1e3), 1), "us_per_step": round(per_step_us, 2),
                          "GB/s": round(step_bytes / (per_step_us / 1e6) / 1e9, 1),
                          "frac_of_measured_hbm": round(step_bytes / (per_step_us / 1e6) / 1e9 / pk["hbm"], 4),
@@ -448,6 +452,23 @@ def run_product(args):
             "decode_GB/s": round((kv_bytes + w_bytes) / (dus / 1e6) / 1e9, 1),
             "decode_frac_of_measured_hbm": round((kv_bytes + w_bytes) / (dus / 1e6) / 1e9 / pk["hbm"], 4)}
         del att, kc, vc
+        J.device_status()
+    if rank == 0 and "moe" in parts:
+        # bf16 experts alone (16 experts, d_ff 14336, a few GB resident): the small case the
+        # grouped expert GEMM profiles are taken on
+        es = MoEShape()
+        moe = J.MoE(moe_params(es, seed=0, device=dev), es)
+        v = moe_input(es, args.moe_tokens, seed=3, device=dev)
+        f = lambda: moe.forward(v)
+        for _ in range(args.warmup):
+            f()
+        torch.cuda.synchronize()
+        mms, _ = event_time_ms(f, args.steps, stream, flush)
+        eflops = args.moe_tokens * 2 * 2.0 * (3 * es.d_model * es.d_ff)
+        res["moe_bf16"] = {"workload": "top-2-of-16 SwiGLU MoE, bf16 experts, %d tokens, d_model 4096, d_ff 14336"
+                                       % args.moe_tokens,
+                           "ms": round(mms, 3), "TFLOP/s": round(eflops / (mms / 1e3) / 1e12, 1)}
+        del moe, v
         J.device_status()
     if rank == 0 and "moe8dec" in parts:
         # ExpertsInt8 decode batch alone, with only the int8 experts resident (a few GB): the
