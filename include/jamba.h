@@ -98,10 +98,19 @@ typedef struct jamba_mamba_weights {
 typedef struct jamba_mamba* jamba_mamba_t;
 
 /* Creates a mixer handle on the current CUDA device.  The weight pointers are
- * borrowed: they must stay valid and unchanged until destroy.  The handle owns
- * only host-side descriptors (TMA tensor maps of the weights).
+ * borrowed: they must stay valid and unchanged until destroy.
+ * bf16 mixers (d_inner up to 16384) also keep, in device memory the handle
+ * owns, a copy of the channel-indexed weights with the channels reordered by
+ * how long they carry state (softplus(dt_bias) * min |A| of each channel,
+ * slowest first) for the prefill: the selective scan's groups of 256
+ * channels then hold channels of like speed and each group gets its own
+ * number of time chunks.  The reordering is internal: inputs, outputs and
+ * both caches keep the caller's channel order, and decode steps use the
+ * caller's weights.  create is synchronous for bf16 (it reads dt_bias and A
+ * back and builds the copy).
  * Errors: INVALID_ARG (null pointers, misalignment), UNSUPPORTED (d_state != 16,
- * d_conv != 4, widths not multiples of 8). */
+ * d_conv != 4, widths not multiples of 8), OOM (no device memory for the
+ * copy), CUDA. */
 jamba_status jamba_mamba_create(const jamba_mamba_config* cfg, const jamba_mamba_weights* w,
                                 jamba_mamba_t* out);
 jamba_status jamba_mamba_destroy(jamba_mamba_t h);

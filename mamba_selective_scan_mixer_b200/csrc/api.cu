@@ -1,7 +1,10 @@
 // C ABI: argument checks, workspace layout and the launch sequences of the
 // Mamba mixer (prefill, decode step), the selective scan alone, the building
 // blocks and the MoE.  See include/jamba.h for the contract of each call.
+#include <algorithm>
+#include <cmath>
 #include <new>
+#include <numeric>
 #include <string>
 #include <vector>
 
@@ -15,6 +18,16 @@ struct jamba_mamba {
   jamba_mamba_weights w;
   int device;
   int a_form;   // ScanAForm of A, read once at create: picks the one scan kernel to launch
+  // bf16 mixers, prefill only: the channels reordered by how long they carry
+  // state (slowest decay first) so that the scan's channel groups hold
+  // channels of like speed.  wp holds the reordered weights (in `own`), perm
+  // maps a reordered channel to its cache row (the caller's channel), head[g]
+  // is the number of steps after which group g's slowest channel has lost the
+  // carried state.  Decode steps use the caller's weights and order.
+  jamba_mamba_weights wp;
+  void* own = nullptr;
+  int* perm = nullptr;
+  std::vector<float> head;
   // host-buffer prefill pipeline: two copy streams and the events that order
   // the double-buffered chunks (created on first use)
   cudaStream_t io_in = nullptr, io_out = nullptr;
@@ -54,10 +67,22 @@ struct PrefillWs {
   // context-parallel prefill only: in_proj rows of the 3 input tokens before
   // the slice, the conv cache they make, and the state entering the slice
   void* xz_halo; float* conv_halo; float* h_in;
+  ScanSchedule sched;   // the scan's per-group time chunks (n == 0: uniform chunks of `chunk`)
   size_t total;
 };
 
-PrefillWs carve_prefill(const jamba_mamba_config& c, int batch, int L, void* ws, bool cp = false) {
+// The scan's time chunks for one prefill call: per channel group when the
+// handle has reordered its channels, else uniform.
+void plan_scan(const jamba_mamba* h, int batch, int L, ScanSchedule* out) {
+  out->n = 0;
+  if (h->perm) {
+    const int groups = (int)h->head.size();
+    scan_plan(batch, L, groups, h->head.data(), scan_slots(h->cfg.dtype, JAMBA_F32), out);
+  }
+}
+
+PrefillWs carve_prefill(const jamba_mamba* h, int batch, int L, void* ws, bool cp = false) {
+  const jamba_mamba_config& c = h->cfg;
   PrefillWs p;
   const size_t T = (size_t)batch * L;
   const int es = esize(c.dtype);
@@ -73,7 +98,16 @@ PrefillWs carve_prefill(const jamba_mamba_config& c, int batch, int L, void* ws,
   p.dt = cv.take<float>(T * c.d_inner * 4);
   p.y = cv.take(T * c.d_inner * es);
   p.conv_tmp = cv.take<float>((size_t)batch * c.d_inner * (c.d_conv - 1) * 4);
-  p.scan_bytes = scan_workspace_bytes(batch, L, c.d_inner, p.chunk);
+  plan_scan(h, batch, L, &p.sched);
+  if (h->perm) {
+    // a per-group plan never exceeds the resident CTAs; sized for that bound
+    // so that shorter calls (the host pipeline's ramp chunks) always fit
+    const size_t uni = scan_records(batch, L, c.d_inner, p.chunk, nullptr);
+    const size_t cap = (size_t)scan_slots(c.dtype, JAMBA_F32);
+    p.scan_bytes = scan_records_bytes(uni > cap ? uni : cap);
+  } else {
+    p.scan_bytes = scan_workspace_bytes(batch, L, c.d_inner, p.chunk);
+  }
   p.scan = cv.take(p.scan_bytes);
   p.xz_halo = p.conv_halo = p.h_in = nullptr;
   if (cp) {
@@ -141,12 +175,98 @@ jamba_status check_device(const jamba_mamba* h) {
   return JAMBA_OK;
 }
 
+// Sort the channels by their slowest decay, softplus(dt_bias[c]) *
+// min_n |A[c, n]| (the decay rate when dt sits at its bias), slowest first,
+// and keep a copy of every channel-indexed weight in that order for the
+// prefill: in_proj rows (x and z halves), conv weight and bias, x_proj
+// columns, dt_proj rows and bias, A, D and out_proj columns (the norm weights
+// are not channel-indexed).  Caches stay in the caller's channel order (the
+// prefill kernels index them through perm).  Synchronous: it reads dt_bias
+// and A back to the host.
+jamba_status reorder_channels(jamba_mamba* h) {
+  const jamba_mamba_config& c = h->cfg;
+  const jamba_mamba_weights w = h->w;
+  const int di = c.d_inner, dm = c.d_model, R = c.dt_rank, N = c.d_state, W = R + 2 * N;
+  const size_t es = 2;   // bf16 weights
+  std::vector<float> bias(di), A((size_t)di * N);
+  JB_CUDA(cudaMemcpy(bias.data(), w.dt_bias, sizeof(float) * di, cudaMemcpyDeviceToHost));
+  JB_CUDA(cudaMemcpy(A.data(), w.A, sizeof(float) * A.size(), cudaMemcpyDeviceToHost));
+  std::vector<double> rate(di);
+  for (int ch = 0; ch < di; ++ch) {
+    const double b = bias[ch];
+    const double dt = b > 30.0 ? b : std::log1p(std::exp(b));
+    double amin = INFINITY;
+    for (int n = 0; n < N; ++n) amin = std::min(amin, std::fabs((double)A[(size_t)ch * N + n]));
+    rate[ch] = std::isfinite(dt * amin) ? dt * amin : 0.0;
+  }
+  std::vector<int> perm(di);
+  std::iota(perm.begin(), perm.end(), 0);
+  std::stable_sort(perm.begin(), perm.end(), [&](int a, int b) { return rate[a] < rate[b]; });
+  // steps until a group's slowest channel has decayed the carried state below 2^-40
+  const int groups = (di + SCAN_GROUP_CHANNELS - 1) / SCAN_GROUP_CHANNELS;
+  h->head.assign(groups, 0.f);
+  for (int g = 0; g < groups; ++g) {
+    const double r = rate[perm[(size_t)g * SCAN_GROUP_CHANNELS]];
+    h->head[g] = r > 0.0 ? (float)std::min(40.0 * std::log(2.0) / r, 1e9) : 1e9f;
+  }
+
+  Carver cv(nullptr);
+  const size_t o_in = (size_t)cv.off; cv.take((size_t)2 * di * dm * es);
+  const size_t o_cw = cv.off; cv.take((size_t)di * 4 * es);
+  const size_t o_cb = cv.off; cv.take((size_t)di * es);
+  const size_t o_x = cv.off; cv.take((size_t)W * di * es);
+  const size_t o_dtp = cv.off; cv.take((size_t)di * R * es);
+  const size_t o_dtb = cv.off; cv.take((size_t)di * 4);
+  const size_t o_A = cv.off; cv.take((size_t)di * N * 4);
+  const size_t o_D = cv.off; cv.take((size_t)di * 4);
+  const size_t o_out = cv.off; cv.take((size_t)dm * di * es);
+  const size_t o_p = cv.off; cv.take((size_t)di * 4);
+  void* buf = nullptr;
+  if (cudaMalloc(&buf, cv.off) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(JAMBA_ERR_OOM, "create: no device memory for the reordered weights");
+  }
+  h->own = buf;
+  uint8_t* base = reinterpret_cast<uint8_t*>(buf);
+  int* dperm = reinterpret_cast<int*>(base + o_p);
+  JB_CUDA(cudaMemcpy(dperm, perm.data(), sizeof(int) * di, cudaMemcpyHostToDevice));
+  cudaStream_t s = 0;
+  const uint8_t* in = reinterpret_cast<const uint8_t*>(w.in_proj);
+  JB_TRY(gather_rows(in, base + o_in, dperm, di, (int)(dm * es), s));
+  JB_TRY(gather_rows(in + (size_t)di * dm * es, base + o_in + (size_t)di * dm * es, dperm, di, (int)(dm * es), s));
+  JB_TRY(gather_rows(w.conv_w, base + o_cw, dperm, di, (int)(4 * es), s));
+  JB_TRY(gather_rows(w.conv_b, base + o_cb, dperm, di, (int)es, s));
+  JB_TRY(gather_cols(w.x_proj, base + o_x, dperm, W, di, (int)es, s));
+  JB_TRY(gather_rows(w.dt_proj, base + o_dtp, dperm, di, (int)(R * es), s));
+  JB_TRY(gather_rows(w.dt_bias, base + o_dtb, dperm, di, 4, s));
+  JB_TRY(gather_rows(w.A, base + o_A, dperm, di, N * 4, s));
+  JB_TRY(gather_rows(w.D, base + o_D, dperm, di, 4, s));
+  JB_TRY(gather_cols(w.out_proj, base + o_out, dperm, dm, di, (int)es, s));
+  JB_CUDA(cudaStreamSynchronize(s));
+  jamba_mamba_weights& o = h->wp;
+  o = h->w;
+  o.in_proj = base + o_in;
+  o.conv_w = base + o_cw;
+  o.conv_b = base + o_cb;
+  o.x_proj = base + o_x;
+  o.dt_proj = base + o_dtp;
+  o.dt_bias = reinterpret_cast<const float*>(base + o_dtb);
+  o.A = reinterpret_cast<const float*>(base + o_A);
+  o.D = reinterpret_cast<const float*>(base + o_D);
+  o.out_proj = base + o_out;
+  h->perm = dperm;
+  return JAMBA_OK;
+}
+
+// The weights the prefill runs on: the reordered copy when the handle has one.
+const jamba_mamba_weights& prefill_weights(const jamba_mamba& h) { return h.perm ? h.wp : h.w; }
+
 // The prefill up to the scan's inputs: in_proj, conv + SiLU (cache in -> out),
 // x_proj, inner RMSNorms, dt_proj + softplus.
 jamba_status prefill_front(const jamba_mamba& h, const PrefillWs& p, const void* u, int batch, int seqlen,
                            const float* conv_state_in, float* conv_state_out, cudaStream_t s) {
   const jamba_mamba_config& c = h.cfg;
-  const jamba_mamba_weights& w = h.w;
+  const jamba_mamba_weights& w = prefill_weights(h);
   const int T = batch * seqlen, di = c.d_inner, dm = c.d_model, R = c.dt_rank, N = c.d_state;
   const int W = R + 2 * N;
   // in_proj: xz = u W_in^T
@@ -158,7 +278,8 @@ jamba_status prefill_front(const jamba_mamba& h, const PrefillWs& p, const void*
     JB_CUDA(cudaMemcpyAsync(p.conv_tmp, cin, sizeof(float) * (size_t)batch * di * 3, cudaMemcpyDeviceToDevice, s));
     cin = p.conv_tmp;
   }
-  JB_TRY(conv_prefill(p.xz, 2 * di, w.conv_w, w.conv_b, p.xc, cin, conv_state_out, batch, seqlen, di, c.dtype, s));
+  JB_TRY(conv_prefill(p.xz, 2 * di, w.conv_w, w.conv_b, p.xc, cin, conv_state_out, batch, seqlen, di, c.dtype,
+                      h.perm, s));
   // x_proj (split-K partials) -> sum + inner RMSNorms
   GemmDesc gx = gdesc(p.xc, di, w.x_proj, di, T, W, di, EPI_F32, p.xpart, W);
   gx.splits = p.splits;
@@ -184,11 +305,13 @@ ScanCall scan_call(const jamba_mamba& h, const PrefillWs& p, int batch, int seql
   sc.B = p.bc; sc.ld_b = 2 * N;
   sc.C = p.bc + N; sc.ld_c = 2 * N;
   sc.bc_dtype = JAMBA_F32;
-  sc.A = h.w.A; sc.D = h.w.D;
+  sc.A = prefill_weights(h).A; sc.D = prefill_weights(h).D;
   sc.y = p.y; sc.ld_y = di;
   sc.batch = batch; sc.L = seqlen; sc.di = di; sc.dtype = c.dtype; sc.chunk = p.chunk;
   sc.ws = p.scan; sc.ws_bytes = p.scan_bytes;
   sc.a_form = h.a_form;
+  sc.sched = &p.sched;
+  sc.perm = h.perm;
   return sc;
 }
 
@@ -201,7 +324,7 @@ jamba_status prefill_back(const jamba_mamba& h, const PrefillWs& p, int batch, i
   sc.h0 = ssm_state_in;
   sc.h_out = ssm_state_out;
   JB_TRY(scan_run(sc, s));
-  GemmDesc go = gdesc(p.y, di, h.w.out_proj, di, T, dm, di, c.dtype == JAMBA_BF16 ? EPI_BF16 : EPI_F32, out, dm);
+  GemmDesc go = gdesc(p.y, di, prefill_weights(h).out_proj, di, T, dm, di, c.dtype == JAMBA_BF16 ? EPI_BF16 : EPI_F32, out, dm);
   go.residual = residual;
   go.ldr = dm;
   return gemm_any(c.dtype, go, s);
@@ -284,6 +407,13 @@ jamba_status jamba_mamba_create(const jamba_mamba_config* cfg, const jamba_mamba
       return fail(JAMBA_ERR_CUDA, "create: could not create the decode prefetch stream");
     }
   }
+  if (c.dtype == JAMBA_BF16 && (c.d_inner + SCAN_GROUP_CHANNELS - 1) / SCAN_GROUP_CHANNELS <= SCAN_MAX_GROUPS) {
+    const jamba_status st = reorder_channels(h);
+    if (st != JAMBA_OK) {
+      jamba_mamba_destroy(h);
+      return st;
+    }
+  }
   *out = h;
   return JAMBA_OK;
 }
@@ -293,6 +423,7 @@ jamba_status jamba_mamba_destroy(jamba_mamba_t h) {
     if (h->pf) cudaStreamDestroy(h->pf);
     if (h->ev_fork) cudaEventDestroy(h->ev_fork);
     if (h->ev_join) cudaEventDestroy(h->ev_join);
+    if (h->own) cudaFree(h->own);
     if (h->io_in) cudaStreamDestroy(h->io_in);
     if (h->io_out) cudaStreamDestroy(h->io_out);
     for (int i = 0; i < 2; ++i) {
@@ -307,7 +438,7 @@ jamba_status jamba_mamba_destroy(jamba_mamba_t h) {
 
 jamba_status jamba_mamba_workspace_size(jamba_mamba_t h, int batch, int seqlen, size_t* bytes) {
   if (!h || !bytes || batch <= 0 || seqlen <= 0) return fail(JAMBA_ERR_INVALID_ARG, "workspace_size: bad argument");
-  size_t a = carve_prefill(h->cfg, batch, seqlen, nullptr).total;
+  size_t a = carve_prefill(h, batch, seqlen, nullptr).total;
   if (seqlen == 1) {
     const size_t b = carve_step(h->cfg, batch, nullptr).total;
     a = a > b ? a : b;
@@ -334,7 +465,7 @@ jamba_status jamba_mamba_prefill(jamba_mamba_t h, const void* u, const void* res
   if (u == out) return fail(JAMBA_ERR_INVALID_ARG, "prefill: out may not alias u");
   const jamba_mamba_config& c = h->cfg;
   if ((long long)batch * seqlen > (1LL << 31) / 2) return fail(JAMBA_ERR_UNSUPPORTED, "prefill: too many tokens");
-  PrefillWs p = carve_prefill(c, batch, seqlen, ws);
+  PrefillWs p = carve_prefill(h, batch, seqlen, ws);
   if (ws_bytes < p.total) return fail(JAMBA_ERR_WORKSPACE, "prefill: workspace too small");
   cudaStream_t s = cs(stream);
   JB_TRY(prefill_front(*h, p, u, batch, seqlen, conv_state_in, conv_state_out, s));
@@ -345,7 +476,7 @@ jamba_status jamba_mamba_prefill(jamba_mamba_t h, const void* u, const void* res
 
 jamba_status jamba_mamba_cp_workspace_size(jamba_mamba_t h, int batch, int seqlen, size_t* bytes) {
   if (!h || !bytes || batch <= 0 || seqlen <= 0) return fail(JAMBA_ERR_INVALID_ARG, "cp workspace_size: bad argument");
-  *bytes = carve_prefill(h->cfg, batch, seqlen, nullptr, true).total;
+  *bytes = carve_prefill(h, batch, seqlen, nullptr, true).total;
   return JAMBA_OK;
 }
 
@@ -371,7 +502,7 @@ jamba_status jamba_mamba_prefill_cp_begin(jamba_mamba_t h, const void* u, const 
     return fail(JAMBA_ERR_INVALID_ARG, "cp begin: the carries may not alias ssm_state_in");
   const jamba_mamba_config& c = h->cfg;
   if ((long long)batch * seqlen > (1LL << 31) / 2) return fail(JAMBA_ERR_UNSUPPORTED, "cp begin: too many tokens");
-  PrefillWs p = carve_prefill(c, batch, seqlen, ws, true);
+  PrefillWs p = carve_prefill(h, batch, seqlen, ws, true);
   if (ws_bytes < p.total) return fail(JAMBA_ERR_WORKSPACE, "cp begin: workspace too small");
   cudaStream_t s = cs(stream);
   const int di = c.d_inner, dm = c.d_model, K1 = c.d_conv - 1;
@@ -410,7 +541,7 @@ jamba_status jamba_mamba_prefill_cp_finish(jamba_mamba_t h, const void* residual
   JB_TRY(check_ptr(carries_h, "carries_h", rank > 0));
   JB_TRY(check_ptr(ws, "workspace"));
   const jamba_mamba_config& c = h->cfg;
-  PrefillWs p = carve_prefill(c, batch, seqlen, ws, true);
+  PrefillWs p = carve_prefill(h, batch, seqlen, ws, true);
   if (ws_bytes < p.total) return fail(JAMBA_ERR_WORKSPACE, "cp finish: workspace too small");
   cudaStream_t s = cs(stream);
   if (rank == 0) return prefill_back(*h, p, batch, seqlen, ssm_state_in, ssm_state_out, residual, out, s);
@@ -731,7 +862,7 @@ jamba_status jamba_causal_conv1d(const void* x, int ld_x, const void* w, const v
   JB_TRY(check_ptr(out, "out"));
   if (state_in && state_in == state_out)
     return fail(JAMBA_ERR_INVALID_ARG, "conv: state_in and state_out may not alias here");
-  return conv_prefill(x, ld_x, w, b, out, state_in, state_out, batch, seqlen, channels, dtype, cs(stream));
+  return conv_prefill(x, ld_x, w, b, out, state_in, state_out, batch, seqlen, channels, dtype, nullptr, cs(stream));
 }
 
 jamba_status jamba_gemm(const void* a, const void* b, void* out, int ld_out, const void* residual, int m, int n,

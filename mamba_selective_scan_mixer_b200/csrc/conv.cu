@@ -55,7 +55,7 @@ template <typename T>
 __global__ void __launch_bounds__(CONV_THREADS)
 conv_prefill_kernel(const T* __restrict__ x, long long ld_x, const T* __restrict__ w, const T* __restrict__ bias,
                     T* __restrict__ out, const float* __restrict__ st_in, float* __restrict__ st_out, int L,
-                    int C) {
+                    int C, const int* __restrict__ perm) {
   constexpr int V = Vec16<T>::N;
   griddep_wait();
   griddep_launch();
@@ -80,8 +80,10 @@ conv_prefill_kernel(const T* __restrict__ x, long long ld_x, const T* __restrict
       Vec16<T>::load(xb + (long long)t * ld_x + c0, win[k]);
     } else {
 #pragma unroll
-      for (int i = 0; i < V; ++i)
-        win[k][i] = st_in ? st_in[((long long)b * C + c0 + i) * 3 + (3 + t)] : 0.f;
+      for (int i = 0; i < V; ++i) {
+        const int cn = perm ? __ldg(perm + c0 + i) : c0 + i;   // cache row of this channel
+        win[k][i] = st_in ? st_in[((long long)b * C + cn) * 3 + (3 + t)] : 0.f;
+      }
     }
   }
   T* ob = out + (long long)b * L * C;
@@ -114,9 +116,11 @@ conv_prefill_kernel(const T* __restrict__ x, long long ld_x, const T* __restrict
   }
   if (st_out && t1 == L) {
 #pragma unroll
-    for (int i = 0; i < V; ++i)
+    for (int i = 0; i < V; ++i) {
+      const int cn = perm ? __ldg(perm + c0 + i) : c0 + i;
 #pragma unroll
-      for (int k = 0; k < 3; ++k) st_out[((long long)b * C + c0 + i) * 3 + k] = win[k][i];
+      for (int k = 0; k < 3; ++k) st_out[((long long)b * C + cn) * 3 + k] = win[k][i];
+    }
   }
 }
 
@@ -170,7 +174,8 @@ jamba_status conv_halo_state(const void* xz, long long ld, float* state, int bat
 }
 
 jamba_status conv_prefill(const void* x, long long ld_x, const void* w, const void* b, void* out,
-                          const float* st_in, float* st_out, int batch, int L, int C, int dtype, cudaStream_t s) {
+                          const float* st_in, float* st_out, int batch, int L, int C, int dtype, const int* perm,
+                          cudaStream_t s) {
   const int V = dtype == JAMBA_BF16 ? 8 : 4;
   if (C % V || ld_x % V || !aligned16(x) || !aligned16(out))
     return fail(JAMBA_ERR_INVALID_ARG, "conv: channels and row stride must fill 16-byte vectors");
@@ -178,11 +183,11 @@ jamba_status conv_prefill(const void* x, long long ld_x, const void* w, const vo
   if (dtype == JAMBA_BF16)
     JB_CUDA(launch_pdl(conv_prefill_kernel<bf16>, grid, dim3(CONV_THREADS), 0, s, reinterpret_cast<const bf16*>(x),
                        ld_x, reinterpret_cast<const bf16*>(w), reinterpret_cast<const bf16*>(b),
-                       reinterpret_cast<bf16*>(out), st_in, st_out, L, C));
+                       reinterpret_cast<bf16*>(out), st_in, st_out, L, C, perm));
   else
     JB_CUDA(launch_pdl(conv_prefill_kernel<float>, grid, dim3(CONV_THREADS), 0, s, reinterpret_cast<const float*>(x),
                        ld_x, reinterpret_cast<const float*>(w), reinterpret_cast<const float*>(b),
-                       reinterpret_cast<float*>(out), st_in, st_out, L, C));
+                       reinterpret_cast<float*>(out), st_in, st_out, L, C, perm));
   return JAMBA_OK;
 }
 
@@ -198,6 +203,65 @@ jamba_status conv_step(const void* x, long long ld_x, const void* w, const void*
     JB_CUDA(launch_pdl(conv_step_kernel<float>, dim3(grid), dim3(256), 0, s, reinterpret_cast<const float*>(x), ld_x,
                        reinterpret_cast<const float*>(w), reinterpret_cast<const float*>(b),
                        reinterpret_cast<float*>(out), state, batch, C));
+  return JAMBA_OK;
+}
+
+// ------------------------------------------------------------ weight reordering
+// dst row r = src row perm[r]; 16-byte words when rows and pointers allow it,
+// else 2-byte elements (row_bytes is even for every weight reordered here).
+__global__ void __launch_bounds__(256)
+gather_rows_kernel(const uint8_t* __restrict__ src, uint8_t* __restrict__ dst, const int* __restrict__ perm,
+                   int rows, int row_bytes, int word) {
+  const int per_row = row_bytes / word;
+  const long long n = (long long)rows * per_row;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const int r = (int)(i / per_row), e = (int)(i - (long long)r * per_row);
+    const long long so = (long long)__ldg(perm + r) * row_bytes + (long long)e * word;
+    const long long d = (long long)r * row_bytes + (long long)e * word;
+    if (word == 16) *reinterpret_cast<uint4*>(dst + d) = *reinterpret_cast<const uint4*>(src + so);
+    else if (word == 4) *reinterpret_cast<uint32_t*>(dst + d) = *reinterpret_cast<const uint32_t*>(src + so);
+    else *reinterpret_cast<uint16_t*>(dst + d) = *reinterpret_cast<const uint16_t*>(src + so);
+  }
+}
+
+// dst[i, j] = src[i, perm[j]] for a [rows, cols] matrix of 2- or 4-byte elements
+__global__ void __launch_bounds__(256)
+gather_cols_kernel(const uint8_t* __restrict__ src, uint8_t* __restrict__ dst, const int* __restrict__ perm, int rows,
+                   int cols, int esize) {
+  const long long n = (long long)rows * cols;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const int r = (int)(i / cols), j = (int)(i - (long long)r * cols);
+    const long long so = ((long long)r * cols + __ldg(perm + j)) * esize;
+    if (esize == 4) *reinterpret_cast<uint32_t*>(dst + i * 4) = *reinterpret_cast<const uint32_t*>(src + so);
+    else *reinterpret_cast<uint16_t*>(dst + i * 2) = *reinterpret_cast<const uint16_t*>(src + so);
+  }
+}
+
+static unsigned gather_grid(long long n) {
+  const long long b = (n + 255) / 256;
+  const long long cap = 32LL * num_sms();
+  return (unsigned)(b < 1 ? 1 : b < cap ? b : cap);
+}
+
+jamba_status gather_rows(const void* src, void* dst, const int* perm, int rows, int row_bytes, cudaStream_t s) {
+  if (!src || !dst || !perm || rows <= 0 || row_bytes <= 0 || row_bytes % 2)
+    return fail(JAMBA_ERR_INVALID_ARG, "gather_rows: bad argument");
+  const bool a16 = aligned16(src) && aligned16(dst) && row_bytes % 16 == 0;
+  const bool a4 = (reinterpret_cast<uintptr_t>(src) % 4 == 0) && (reinterpret_cast<uintptr_t>(dst) % 4 == 0) &&
+                  row_bytes % 4 == 0;
+  const int word = a16 ? 16 : a4 ? 4 : 2;
+  gather_rows_kernel<<<gather_grid((long long)rows * (row_bytes / word)), 256, 0, s>>>(
+      reinterpret_cast<const uint8_t*>(src), reinterpret_cast<uint8_t*>(dst), perm, rows, row_bytes, word);
+  JB_CUDA(cudaGetLastError());
+  return JAMBA_OK;
+}
+
+jamba_status gather_cols(const void* src, void* dst, const int* perm, int rows, int cols, int esize, cudaStream_t s) {
+  if (!src || !dst || !perm || rows <= 0 || cols <= 0 || (esize != 2 && esize != 4))
+    return fail(JAMBA_ERR_INVALID_ARG, "gather_cols: bad argument");
+  gather_cols_kernel<<<gather_grid((long long)rows * cols), 256, 0, s>>>(
+      reinterpret_cast<const uint8_t*>(src), reinterpret_cast<uint8_t*>(dst), perm, rows, cols, esize);
+  JB_CUDA(cudaGetLastError());
   return JAMBA_OK;
 }
 

@@ -96,6 +96,23 @@ jamba_status gemm_f32(const GemmDesc& g, cudaStream_t s);
 int choose_splits(int M, int N, int K, int bn, int min_k_tiles);
 
 // ---------------------------------------------------------------- scan
+// Time chunks per channel group of 256 (groups = d_inner / 256 rounded up).
+// n == 0: every group takes the uniform chunk length of the call.
+constexpr int SCAN_MAX_GROUPS = 64;
+constexpr int SCAN_GROUP_CHANNELS = 256;   // channels of one scan CTA
+struct ScanSchedule {
+  int n;                           // channel groups covered (0 = uniform)
+  int chunks[SCAN_MAX_GROUPS];     // time chunks of each group
+  int len[SCAN_MAX_GROUPS];        // their length in steps (a multiple of 16)
+};
+// Per-group chunks for `batch` rows of L steps when the channels of group g
+// lose the carried state after about head[g] steps (groups sorted so that
+// later ones are no slower): the largest CTA cost (chunk + replayed head) is
+// minimised with at most `slots` CTAs in the launch.  Returns n = 0 when
+// batch rows alone fill the slots.
+void scan_plan(int batch, int L, int groups, const float* head, int slots, ScanSchedule* out);
+int scan_slots(int dtype, int bc_dtype);   // CTAs of the scan resident at once on this device
+
 struct ScanCall {
   const void* x; long long ld_x;
   const void* z; long long ld_z;
@@ -107,6 +124,8 @@ struct ScanCall {
   void* y; long long ld_y;
   float* h_out;
   int batch, L, di, dtype, chunk;
+  const ScanSchedule* sched;   // null or n == 0: uniform chunks of `chunk` steps
+  const int* perm;             // null, or [di]: the cache row of internal channel c is perm[c]
   void* ws; size_t ws_bytes;
   int* err;   // device status word; null = the library's per-device word
   int a_form;                    // SCAN_A_*: which kernel owns the channels, when the caller knows
@@ -117,7 +136,9 @@ struct ScanCall {
 };
 enum ScanAForm { SCAN_A_UNKNOWN = 0, SCAN_A_POWER = 1, SCAN_A_GENERAL = 2 };
 jamba_status scan_run(const ScanCall& s, cudaStream_t st);
-size_t scan_workspace_bytes(int batch, int L, int di, int chunk_len);
+size_t scan_workspace_bytes(int batch, int L, int di, int chunk_len, const ScanSchedule* sched = nullptr);
+size_t scan_records(int batch, int L, int di, int chunk_len, const ScanSchedule* sched);   // CTAs of a launch
+size_t scan_records_bytes(size_t recs);                                                   // workspace they use
 int scan_auto_chunk(int batch, int L, int di, int dtype, int bc_dtype);
 jamba_status static_scan_status_take(int* value);   // static scan's own status word (read and cleared)
 // context-parallel prefill: the state entering slice `rank` from the slices' carries
@@ -128,12 +149,20 @@ jamba_status ssm_step(const void* xc, const void* z, long long ld_z, const float
                       int dtype, cudaStream_t st);
 
 // ---------------------------------------------------------------- conv / norms
+// perm (prefill): null, or [C]: the cache row of internal channel c is perm[c]
 jamba_status conv_prefill(const void* x, long long ld_x, const void* w, const void* b, void* out,
-                          const float* st_in, float* st_out, int batch, int L, int C, int dtype, cudaStream_t s);
+                          const float* st_in, float* st_out, int batch, int L, int C, int dtype, const int* perm,
+                          cudaStream_t s);
 jamba_status conv_step(const void* x, long long ld_x, const void* w, const void* b, void* out, float* state,
                        int batch, int C, int dtype, cudaStream_t s);
 jamba_status conv_halo_state(const void* xz, long long ld, float* state, int batch, int C, int dtype,
                              cudaStream_t s);
+// Row and column gathers for reordering channel-indexed weights:
+// dst[r, :] = src[perm[r], :] over rows of row_bytes bytes, and, for a
+// [rows, cols] matrix of `esize`-byte elements, dst[:, j] = src[:, perm[j]].
+jamba_status gather_rows(const void* src, void* dst, const int* perm, int rows, int row_bytes, cudaStream_t s);
+jamba_status gather_cols(const void* src, void* dst, const int* perm, int rows, int cols, int esize,
+                         cudaStream_t s);
 jamba_status rmsnorm(const void* x, const float* w, void* out, int rows, int cols, float eps, int dtype,
                      cudaStream_t s);
 jamba_status xproj_norm(const float* part, int splits, long long split_stride, int T, int R, int N,

@@ -42,7 +42,7 @@
 
 namespace jb {
 
-constexpr int SCAN_CH = 256;                        // channels per CTA
+constexpr int SCAN_CH = SCAN_GROUP_CHANNELS;        // channels per CTA
 constexpr int SCAN_Q = 8;                           // time steps per stage
 constexpr int SCAN_STAGES = 3;
 constexpr int NS = 16;                              // d_state
@@ -89,8 +89,14 @@ struct ScanArgs {
   float* h_out;
   int batch, L, di;
   int chunk_len, n_chunks, cgroups;
+  // per-group schedule (sched_n == 0: uniform chunks of chunk_len): group g
+  // has g_chunks[g] chunks of g_len[g] steps, its records start at
+  // g_rec[g] within a batch row, which holds recs_row records
+  int sched_n, recs_row;
+  int g_chunks[SCAN_MAX_GROUPS], g_len[SCAN_MAX_GROUPS], g_rec[SCAN_MAX_GROUPS];
+  const int* perm;       // null, or [di]: the cache row (h0, h_out) of internal channel c
   int* ticket;           // [2]: one counter per kernel kind
-  int* flags;            // [batch * cgroups * n_chunks]
+  int* flags;            // one per record
   float* rec;            // per record: P[256][16], h[256][16], inclusive h[256][16]
   int* err;
   unsigned long long wait_ns;   // limit of the look-back waits on a predecessor's flag
@@ -182,6 +188,7 @@ struct ScanCtx {
   int b, cg, chunk, grp;
   int t0, t1;
   long long row0;
+  long long rbase;   // record of chunk 0 of this (batch row, channel group)
   int c_base;
 };
 
@@ -406,14 +413,39 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
   }
   __syncthreads();
   ScanCtx cx;
-  const int groups_total = a.batch * a.cgroups;
-  cx.chunk = s_ticket / groups_total;
-  cx.grp = s_ticket - cx.chunk * groups_total;
-  cx.b = cx.grp / a.cgroups;
-  cx.cg = cx.grp - cx.b * a.cgroups;
+  if (a.sched_n == 0) {
+    const int groups_total = a.batch * a.cgroups;
+    cx.chunk = s_ticket / groups_total;
+    cx.grp = s_ticket - cx.chunk * groups_total;
+    cx.b = cx.grp / a.cgroups;
+    cx.cg = cx.grp - cx.b * a.cgroups;
+    cx.t0 = cx.chunk * a.chunk_len;
+    cx.t1 = min(a.L, cx.t0 + a.chunk_len);
+    cx.rbase = (long long)cx.grp * a.n_chunks;
+  } else {
+    // tickets by chunk index, then batch row, then channel group among the
+    // groups that have a chunk of that index: a chunk's predecessors always
+    // hold smaller tickets, so they are already running
+    int t = s_ticket, k = 0, m = 0;
+    for (;; ++k) {
+      m = 0;
+      for (int g = 0; g < a.cgroups; ++g) m += a.g_chunks[g] > k ? 1 : 0;
+      if (m == 0) return;                    // past the schedule (the grid never is)
+      if (t < a.batch * m) break;
+      t -= a.batch * m;
+    }
+    cx.chunk = k;
+    cx.b = t / m;
+    int r = t - cx.b * m, g = 0;
+    for (; g < a.cgroups; ++g)
+      if (a.g_chunks[g] > k && r-- == 0) break;
+    cx.cg = g;
+    cx.grp = cx.b * a.cgroups + g;
+    cx.t0 = k * a.g_len[g];
+    cx.t1 = min(a.L, cx.t0 + a.g_len[g]);
+    cx.rbase = (long long)cx.b * a.recs_row + a.g_rec[g];
+  }
   cx.c_base = cx.cg * SCAN_CH;
-  cx.t0 = cx.chunk * a.chunk_len;
-  cx.t1 = min(a.L, cx.t0 + a.chunk_len);
   cx.row0 = (long long)cx.b * a.L;
 
   // which kernel owns this CTA: the power form needs A[c, n] == (n + 1) A[c, 0] on all its channels
@@ -463,7 +495,8 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
     for (int i = 0; i < 8; ++i) {
       h[j][i] = make_float2(0.f, 0.f);
       if (known && a.h0 && valid) {
-        const float* src = a.h0 + ((long long)cx.b * a.di + c + j) * NS + 2 * i;
+        const int cn = a.perm ? __ldg(a.perm + c + j) : c + j;
+        const float* src = a.h0 + ((long long)cx.b * a.di + cn) * NS + 2 * i;
         h[j][i] = make_float2(src[0], src[1]);
       }
     }
@@ -491,7 +524,7 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
   if (__syncthreads_or(!pass_ok)) return;
 
   // ---------------------------------------------------------- carry
-  const long long rbase = (long long)cx.grp * a.n_chunks;
+  const long long rbase = cx.rbase;
   float* myrec = a.rec + (rbase + cx.chunk) * REC;
   int* myflag = a.flags + rbase + cx.chunk;
   // end state free of h_in: the first chunk (its start state is known), or every warp's head ended
@@ -590,10 +623,14 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
             he = make_float2(fmaf(pe[2 * n2], hi.x, he.x), fmaf(pe[2 * n2 + 1], hi.y, he.y));
             *reinterpret_cast<float2*>(myrec + 2 * SCAN_CH * NS + (cl + j) * NS + 2 * n2) = he;
           }
-          if (last) *reinterpret_cast<float2*>(a.h_out + ((long long)cx.b * a.di + c + j) * NS + 2 * n2) = he;
+          if (last) {
+            const int cn = a.perm ? __ldg(a.perm + c + j) : c + j;
+            *reinterpret_cast<float2*>(a.h_out + ((long long)cx.b * a.di + cn) * NS + 2 * n2) = he;
+          }
           if (a.summary && valid) {
+            const int cn = a.perm ? __ldg(a.perm + c + j) : c + j;
             const float2 pin = make_float2(sP[(cl + j) * NS + 2 * n2], sP[(cl + j) * NS + 2 * n2 + 1]);
-            *reinterpret_cast<float2*>(a.p_out + ((long long)cx.b * a.di + c + j) * NS + 2 * n2) =
+            *reinterpret_cast<float2*>(a.p_out + ((long long)cx.b * a.di + cn) * NS + 2 * n2) =
                 make_float2(pe[2 * n2] * pin.x, pe[2 * n2 + 1] * pin.y);
           }
           h[j][n2] = hi;
@@ -624,11 +661,12 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
     // the first chunk started from the known state: h is the final state of the batch row
 #pragma unroll
     for (int j = 0; j < CPT; ++j) {
+      const int cn = a.perm ? __ldg(a.perm + c + j) : c + j;
       float pe[16];
       chunk_decay<FAST>(R[j], P[j], pe);
 #pragma unroll
       for (int n2 = 0; n2 < 8; ++n2) {
-        const long long o = ((long long)cx.b * a.di + c + j) * NS + 2 * n2;
+        const long long o = ((long long)cx.b * a.di + cn) * NS + 2 * n2;
         if (a.h_out) *reinterpret_cast<float2*>(a.h_out + o) = h[j][n2];
         if (a.summary) *reinterpret_cast<float2*>(a.p_out + o) = make_float2(pe[2 * n2], pe[2 * n2 + 1]);
       }
@@ -698,10 +736,23 @@ jamba_status carry_combine(const float* P, const float* H, int rank, const float
 }
 
 // ------------------------------------------------------------ host side
-size_t scan_workspace_bytes(int batch, int L, int di, int chunk_len) {
+// records (one per CTA) of a launch: batch rows x chunks of every channel group
+size_t scan_records(int batch, int L, int di, int chunk_len, const ScanSchedule* sched) {
   const int cgroups = (di + SCAN_CH - 1) / SCAN_CH;
+  if (sched && sched->n > 0) {
+    size_t row = 0;
+    for (int g = 0; g < cgroups; ++g) row += (size_t)sched->chunks[g];
+    return (size_t)batch * row;
+  }
   const int n_chunks = (L + chunk_len - 1) / chunk_len;
-  const size_t recs = (size_t)batch * cgroups * n_chunks;
+  return (size_t)batch * cgroups * n_chunks;
+}
+
+size_t scan_workspace_bytes(int batch, int L, int di, int chunk_len, const ScanSchedule* sched) {
+  return scan_records_bytes(scan_records(batch, L, di, chunk_len, sched));
+}
+
+size_t scan_records_bytes(size_t recs) {
   size_t bytes = 256;                                       // tickets
   bytes += (recs * sizeof(int) + 255) & ~size_t(255);       // flags
   bytes += recs * REC * sizeof(float);                      // chunk records
@@ -760,19 +811,69 @@ static jamba_status launch_kernel(size_t recs, const CUtensorMap& mx, const CUte
 // (a CTA waiting on its predecessor must never wait for a free SM slot).
 // Shorter chunks replay shorter heads and a CTA's step rate is bounded by its
 // own dependency chain, so full occupancy is the fastest choice measured.
+int scan_slots(int dtype, int bc_dtype) {
+  if (dtype == JAMBA_BF16 && bc_dtype == JAMBA_BF16) return resident_ctas<bf16, bf16, true, FastShape::CPT, FastShape::MINB>();
+  if (dtype == JAMBA_BF16) return resident_ctas<bf16, float, true, FastShape::CPT, FastShape::MINB>();
+  return resident_ctas<float, float, false, GenShape::CPT, GenShape::MINB>();
+}
+
 int scan_auto_chunk(int batch, int L, int di, int dtype, int bc_dtype) {
   const int cgroups = (di + SCAN_CH - 1) / SCAN_CH;
   const long long groups = (long long)batch * cgroups;
-  int cap;
-  if (dtype == JAMBA_BF16 && bc_dtype == JAMBA_BF16) cap = resident_ctas<bf16, bf16, true, FastShape::CPT, FastShape::MINB>();
-  else if (dtype == JAMBA_BF16) cap = resident_ctas<bf16, float, true, FastShape::CPT, FastShape::MINB>();
-  else cap = resident_ctas<float, float, false, GenShape::CPT, GenShape::MINB>();
+  const int cap = scan_slots(dtype, bc_dtype);
   long long n_chunks = cap / groups;
   if (n_chunks < 1) n_chunks = 1;
   int chunk = (int)((L + n_chunks - 1) / n_chunks);
   chunk = (chunk + 15) & ~15;
   if (chunk < 16) chunk = 16;
   return chunk;
+}
+
+// Cost of a CTA in steps: its chunk, plus the head it replays (the steps
+// until its slowest channel has lost the incoming state, at most the chunk).
+static double chunk_cost(int len, float head) { return len + (head < len ? (double)head : (double)len); }
+
+static int chunk_len_for(int L, int n) {
+  const int len = (L + n - 1) / n;
+  return (len + 15) & ~15;
+}
+
+void scan_plan(int batch, int L, int groups, const float* head, int slots, ScanSchedule* out) {
+  out->n = 0;
+  if (groups <= 0 || groups > SCAN_MAX_GROUPS || batch <= 0 || L <= 16) return;
+  if ((long long)batch * groups * 2 > slots) return;   // batch rows and groups already fill the GPU
+  const int max_n = (L + 15) / 16;
+  // fewest chunks of group g with a CTA cost of at most C (0 if none)
+  auto need = [&](int g, double C) {
+    int lo = 1, hi = max_n;
+    if (chunk_cost(chunk_len_for(L, hi), head[g]) > C) return 0;
+    while (lo < hi) {   // cost falls as n grows (chunk_len_for is non-increasing in n)
+      const int mid = (lo + hi) / 2;
+      if (chunk_cost(chunk_len_for(L, mid), head[g]) <= C) hi = mid; else lo = mid + 1;
+    }
+    return lo;
+  };
+  auto fits = [&](double C) {
+    long long total = 0;
+    for (int g = 0; g < groups; ++g) {
+      const int n = need(g, C);
+      if (n == 0) return false;
+      total += n;
+    }
+    return total * batch <= slots;
+  };
+  double lo = 32.0, hi = 2.0 * L + 32.0;
+  if (!fits(hi)) return;
+  for (int it = 0; it < 48 && hi - lo > 1.0; ++it) {
+    const double mid = 0.5 * (lo + hi);
+    if (fits(mid)) hi = mid; else lo = mid;
+  }
+  for (int g = 0; g < groups; ++g) {
+    const int len = chunk_len_for(L, need(g, hi));
+    out->len[g] = len;
+    out->chunks[g] = (L + len - 1) / len;
+  }
+  out->n = groups;
 }
 
 template <typename TX, typename TBC>
@@ -798,7 +899,19 @@ static jamba_status launch_scan(const ScanCall& s, cudaStream_t st) {
   a.chunk_len = s.chunk;
   a.n_chunks = (s.L + s.chunk - 1) / s.chunk;
   a.cgroups = (s.di + SCAN_CH - 1) / SCAN_CH;
-  const size_t recs = (size_t)s.batch * a.cgroups * a.n_chunks;
+  a.perm = s.perm;
+  a.sched_n = 0;
+  a.recs_row = 0;
+  if (s.sched && s.sched->n > 0) {
+    a.sched_n = s.sched->n;
+    for (int g = 0; g < a.cgroups; ++g) {
+      a.g_chunks[g] = s.sched->chunks[g];
+      a.g_len[g] = s.sched->len[g];
+      a.g_rec[g] = a.recs_row;
+      a.recs_row += s.sched->chunks[g];
+    }
+  }
+  const size_t recs = scan_records(s.batch, s.L, s.di, s.chunk, s.sched);
   uint8_t* w = reinterpret_cast<uint8_t*>(s.ws);
   a.ticket = reinterpret_cast<int*>(w);
   a.flags = reinterpret_cast<int*>(w + 256);
@@ -847,7 +960,17 @@ jamba_status scan_run(const ScanCall& s, cudaStream_t st) {
   if (!s.summary && s.ld_y % 4)
     return fail(JAMBA_ERR_INVALID_ARG, "scan: the leading dimension of y must be a multiple of 4");
   if (!s.summary && !aligned16(s.y)) return fail(JAMBA_ERR_INVALID_ARG, "scan: y must be 16-byte aligned");
-  if (s.ws_bytes < scan_workspace_bytes(s.batch, s.L, s.di, s.chunk) || !s.ws || !aligned16(s.ws))
+  if (s.sched && s.sched->n > 0) {
+    const int cgroups = (s.di + SCAN_CH - 1) / SCAN_CH;
+    if (s.sched->n != cgroups || cgroups > SCAN_MAX_GROUPS)
+      return fail(JAMBA_ERR_INVALID_ARG, "scan: the schedule does not cover the channel groups");
+    for (int g = 0; g < cgroups; ++g) {
+      const long long n = s.sched->chunks[g], len = s.sched->len[g];
+      if (n < 1 || len < 16 || len % 16 || n * len < s.L || (n - 1) * len >= s.L)
+        return fail(JAMBA_ERR_INVALID_ARG, "scan: a group's chunks do not tile the sequence");
+    }
+  }
+  if (s.ws_bytes < scan_workspace_bytes(s.batch, s.L, s.di, s.chunk, s.sched) || !s.ws || !aligned16(s.ws))
     return fail(JAMBA_ERR_WORKSPACE, "scan: workspace too small");
   if ((long long)s.batch * s.L > 0x7fffffffLL) return fail(JAMBA_ERR_UNSUPPORTED, "scan: too many tokens");
   if (s.dtype == JAMBA_BF16 && s.bc_dtype == JAMBA_BF16) return launch_scan<bf16, bf16>(s, st);

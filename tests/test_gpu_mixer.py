@@ -82,6 +82,23 @@ def test_bf16_prefill_residual_and_continuation(dev):
     assert rel_l2(to_np(ss3), to_np(ss2)) < 1e-6
 
 
+def test_bf16_prefill_reordered_channel_groups(dev):
+    """d_inner 2048: eight scan groups of 256 channels after the bf16 handle
+    reorders its channels by decay speed, each group with its own number of
+    time chunks; 1200 tokens in two calls (the second from the first's
+    caches), outputs and both caches in the caller's channel order"""
+    sh = MambaShape(d_model=512, d_inner=2048, dt_rank=64, dtype="bf16", inner_norm=True)
+    mix, p64 = _mixer(sh, 12, dev, a_init="structured", norm_init="random")
+    u = mamba_input(sh, 2, 1200, seed=12)
+    ud = u.to(dev)
+    out1, cs, ss = mix.prefill(ud[:, :700].contiguous())
+    out2, cs2, ss2 = mix.prefill(ud[:, 700:].contiguous(), conv_state_in=cs, ssm_state_in=ss)
+    ref = om.mamba_prefill(p64, to_np(u), sh)
+    assert rel_l2(np.concatenate([to_np(out1), to_np(out2)], axis=1), ref["out"]) < TOL_BF16
+    assert rel_l2(to_np(ss2), ref["ssm_state"]) < TOL_BF16
+    assert rel_l2(to_np(cs2), ref["conv_state"]) < TOL_BF16
+
+
 def test_bf16_decode_steps_match_oracle_and_prefill(dev):
     sh = MambaShape(d_model=512, d_inner=1024, dt_rank=64, dtype="bf16")
     mix, p64 = _mixer(sh, 4, dev)
