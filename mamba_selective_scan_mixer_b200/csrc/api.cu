@@ -570,9 +570,15 @@ jamba_status jamba_mamba_step(jamba_mamba_t h, const void* u, const void* residu
   const int di = c.d_inner, dm = c.d_model, R = c.dt_rank, N = c.d_state, W = R + 2 * N;
   if (c.dtype == JAMBA_BF16) {
     // weights stream through the tensor cores as the 128-row side; the token batch is the N side
-    GemmDesc g1 = gdesc(w.in_proj, dm, u, dm, 2 * di, batch, dm, EPI_BF16, p.xz, 2 * di);
+    // in_proj with the conv step in its epilogue: x rows -> conv cache shift + SiLU -> xc, z rows -> xz
+    GemmDesc g1 = gdesc(w.in_proj, dm, u, dm, 2 * di, batch, dm, EPI_CONV, p.xz, 2 * di);
     g1.transpose_out = 1;
     g1.bn = 64;
+    g1.conv_w = w.conv_w;
+    g1.conv_b = w.conv_b;
+    g1.conv_state = conv_state;
+    g1.xc_out = p.xc;
+    g1.conv_c = di;
     JB_TRY(gemm_bf16(g1, s));
     // once in_proj's weight stream is done, out_proj's weights (d_model x d_inner bf16, which fit
     // L2 beside the caches) are prefetched on the side stream while the small kernels below run
@@ -580,7 +586,6 @@ jamba_status jamba_mamba_step(jamba_mamba_t h, const void* u, const void* residu
     JB_CUDA(cudaStreamWaitEvent(h->pf, h->ev_fork, 0));
     JB_TRY(l2_prefetch(w.out_proj, (size_t)dm * di * 2, h->pf));
     JB_CUDA(cudaEventRecord(h->ev_join, h->pf));
-    JB_TRY(conv_step(p.xz, 2 * di, w.conv_w, w.conv_b, p.xc, conv_state, batch, di, c.dtype, s));
     GemmDesc g2 = gdesc(w.x_proj, di, p.xc, di, W, batch, di, EPI_F32, p.xpart, W);
     g2.transpose_out = 1;
     g2.bn = 64;

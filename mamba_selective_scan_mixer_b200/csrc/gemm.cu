@@ -178,6 +178,10 @@ jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
     return fail(JAMBA_ERR_INVALID_ARG, "gemm: split-K writes fp32 partials only");
   if (g.epi == EPI_SWIGLU && (!g.grouped || !g.b2))
     return fail(JAMBA_ERR_INVALID_ARG, "gemm: SwiGLU needs grouped gate and up weights");
+  if (g.epi == EPI_CONV && (!g.transpose_out || g.splits > 1 || !g.conv_w || !g.conv_b || !g.conv_state ||
+                            !g.xc_out || g.conv_c <= 0 || g.conv_c > g.M ||
+                            (reinterpret_cast<uintptr_t>(g.conv_w) & 7)))
+    return fail(JAMBA_ERR_INVALID_ARG, "gemm: the conv epilogue needs a swap-AB GEMM and its conv operands");
   if (g.b_int8) return gemm_i8w(g, s);
   int bn = g.bn;
   if (bn == 0) {
@@ -234,6 +238,11 @@ jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
   p.residual = g.residual;
   p.ldr = g.ldr;
   p.bias = g.bias;
+  p.conv_w = reinterpret_cast<const bf16*>(g.conv_w);
+  p.conv_b = reinterpret_cast<const bf16*>(g.conv_b);
+  p.conv_state = g.conv_state;
+  p.xc_out = reinterpret_cast<bf16*>(g.xc_out);
+  p.conv_c = g.conv_c;
   p.err = device_error_word();
   if (!p.err) return fail(JAMBA_ERR_CUDA, "could not allocate the device status word");
 
@@ -245,6 +254,7 @@ jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
       case EPI_BF16: return launch_bn<EPI_BF16, true>(bn, ma, mb, mb2, mc, p, grid, s);
       case EPI_F32: return launch_bn<EPI_F32, true>(bn, ma, mb, mb2, mc, p, grid, s);
       case EPI_SOFTPLUS: return launch_bn<EPI_SOFTPLUS, true>(bn, ma, mb, mb2, mc, p, grid, s);
+      case EPI_CONV: return launch_bn<EPI_CONV, true>(bn, ma, mb, mb2, mc, p, grid, s);
       default: break;
     }
   } else {

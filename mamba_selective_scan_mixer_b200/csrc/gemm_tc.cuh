@@ -21,7 +21,7 @@
 
 namespace jb {
 
-enum EpiKind : int { EPI_BF16 = 0, EPI_F32 = 1, EPI_SOFTPLUS = 2, EPI_SWIGLU = 3 };
+enum EpiKind : int { EPI_BF16 = 0, EPI_F32 = 1, EPI_SOFTPLUS = 2, EPI_SWIGLU = 3, EPI_CONV = 4 };
 
 constexpr int GEMM_THREADS = 320;
 constexpr int GEMM_EPI_WARPS = 8;
@@ -41,6 +41,15 @@ struct GemmParams {
   const float* bias;     // indexed by n (or by m when transposed)
   const float* scale_b;  // INT8 weights: per-row scales [groups, N] (SwiGLU: of the gate rows)
   const float* scale_b2; // INT8 weights, SwiGLU: scales of the up rows
+  // EPI_CONV (decode in_proj, swap-AB): output rows m < conv_c are the conv's
+  // input x: the causal conv over [cache, x] + SiLU goes to xc_out [N, conv_c]
+  // and the cache [N, conv_c, 3] shifts in place; rows >= conv_c are stored
+  // as in EPI_BF16
+  const bf16* conv_w;    // [conv_c, 4]
+  const bf16* conv_b;    // [conv_c]
+  float* conv_state;
+  bf16* xc_out;
+  int conv_c;
   int* err;
 };
 
@@ -212,7 +221,39 @@ __device__ __forceinline__ void epi_chunk(const GemmParams& p, const TileInfo& t
     }
   } else {
     // swap-AB: row m is an output feature, column n a token; lanes hold consecutive m
-    if constexpr (EPI == EPI_BF16) {
+    if constexpr (EPI == EPI_CONV) {
+      if (m < p.conv_c) {
+        // decode conv step of channel m for tokens n..n+NC-1: window [cache (oldest first), x]
+        const uint2 wr = *reinterpret_cast<const uint2*>(p.conv_w + (long long)m * 4);
+        const bf16* wb = reinterpret_cast<const bf16*>(&wr);
+        const float w0 = __bfloat162float(wb[0]), w1 = __bfloat162float(wb[1]);
+        const float w2 = __bfloat162float(wb[2]), w3 = __bfloat162float(wb[3]);
+        const float bias = __bfloat162float(p.conv_b[m]);
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+          if (n + c < p.N) {
+            const long long bc = (long long)(n + c) * p.conv_c + m;
+            float* st = p.conv_state + bc * 3;
+            const float s0 = st[0], s1 = st[1], s2 = st[2];
+            const float xv = __bfloat162float(__float2bfloat16_rn(v[c]));   // x as the bf16 activation
+            float acc = bias;
+            acc = fmaf(w0, s0, acc);
+            acc = fmaf(w1, s1, acc);
+            acc = fmaf(w2, s2, acc);
+            acc = fmaf(w3, xv, acc);
+            p.xc_out[bc] = __float2bfloat16_rn(silu(acc));
+            st[0] = s1;
+            st[1] = s2;
+            st[2] = xv;
+          }
+        }
+      } else {
+        bf16* o = reinterpret_cast<bf16*>(p.out);
+#pragma unroll
+        for (int c = 0; c < NC; ++c)
+          if (n + c < p.N) o[(long long)(n + c) * p.ldo + m] = __float2bfloat16_rn(v[c]);
+      }
+    } else if constexpr (EPI == EPI_BF16) {
       bf16* o = reinterpret_cast<bf16*>(p.out);
 #pragma unroll
       for (int c = 0; c < NC; ++c)

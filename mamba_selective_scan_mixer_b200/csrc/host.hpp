@@ -86,6 +86,8 @@ struct GemmDesc {
   int b_int8;      // grouped expert GEMMs: b / b2 hold INT8 codes (row stride ldb bytes)
   const float* scale_b;   // with b_int8: per-row scales [groups, b_rows] of b
   const float* scale_b2;  // ... and of b2
+  // EPI_CONV (swap-AB only): decode conv fused into in_proj's epilogue
+  const void* conv_w; const void* conv_b; float* conv_state; void* xc_out; int conv_c;
 };
 jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s);
 jamba_status l2_prefetch(const void* p, size_t bytes, cudaStream_t s);   // bulk L2 prefetch, fire and forget
