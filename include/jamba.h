@@ -166,6 +166,38 @@ jamba_status jamba_mamba_step(jamba_mamba_t h, const void* u, const void* residu
                               int batch, float* conv_state, float* ssm_state, void* ws,
                               size_t ws_bytes, jamba_stream_t stream);
 
+/* -------------------------------------------- tensor-parallel prefill */
+
+/* Prefill with the mixer's d_inner channels split over ranks (tensor
+ * parallelism; the summary page lists tensor parallelism among its training
+ * parallelisms, appendix on training infrastructure, without a scheme).
+ * Each rank creates its handle with d_inner = its channel count and its share
+ * of the channel-indexed weights: in_proj rows of its x channels followed by
+ * the rows of its z channels, conv weight and bias, x_proj columns, dt_proj
+ * rows, dt_bias, A, D and out_proj columns of its channels (norm weights
+ * whole).  Conv, the norms' inputs aside, dt_proj and the scan are per
+ * channel; the two contractions over d_inner (x_proj and out_proj) give
+ * per-rank partial sums that the caller all-reduces (sum) between the calls:
+ *   begin  -> xproj_part [batch*seqlen, dt_rank + 2*d_state] fp32
+ *   (all-reduce: xproj_sum)
+ *   finish -> out_part [batch*seqlen, d_model] fp32
+ *   (all-reduce: out_sum)
+ *   end    -> out = out_sum (+ residual), in the model dtype
+ * begin and finish take the same workspace (jamba_mamba_workspace_size of
+ * the handle), unchanged in between: it carries the slice's activations.
+ * Caches are this rank's channels: conv [batch, d_inner_r, 3], ssm
+ * [batch, d_inner_r, 16], as in jamba_mamba_prefill.  Errors: INVALID_ARG,
+ * WORKSPACE, UNSUPPORTED, CUDA. */
+jamba_status jamba_mamba_prefill_tp_begin(jamba_mamba_t h, const void* u, int batch, int seqlen,
+                                          const float* conv_state_in, float* conv_state_out,
+                                          float* xproj_part, void* ws, size_t ws_bytes,
+                                          jamba_stream_t stream);
+jamba_status jamba_mamba_prefill_tp_finish(jamba_mamba_t h, const float* xproj_sum, int batch, int seqlen,
+                                           const float* ssm_state_in, float* ssm_state_out, float* out_part,
+                                           void* ws, size_t ws_bytes, jamba_stream_t stream);
+jamba_status jamba_mamba_prefill_tp_end(jamba_mamba_t h, const float* out_sum, const void* residual,
+                                        void* out, int batch, int seqlen, jamba_stream_t stream);
+
 /* ------------------------------------------- context-parallel prefill */
 
 /* Prefill of sequences split over ranks by time (context parallelism): rank r

@@ -71,6 +71,9 @@ SIGNATURES = {
     "jamba_mamba_step": [P, P, P, P, I, P, P, P, SZ, P],
     "jamba_mamba_host_workspace_size": [P, I, I, ctypes.POINTER(SZ)],
     "jamba_mamba_prefill_host": [P, P, P, P, I, I, I, P, P, P, P, P, SZ, P],
+    "jamba_mamba_prefill_tp_begin": [P, P, I, I, P, P, P, P, SZ, P],
+    "jamba_mamba_prefill_tp_finish": [P, P, I, I, P, P, P, P, SZ, P],
+    "jamba_mamba_prefill_tp_end": [P, P, P, P, I, I, P],
     "jamba_mamba_cp_workspace_size": [P, I, I, ctypes.POINTER(SZ)],
     "jamba_mamba_prefill_cp_begin": [P, P, P, I, I, P, P, P, P, P, P, SZ, P],
     "jamba_mamba_prefill_cp_finish": [P, P, P, I, I, I, P, P, P, P, P, SZ, P],

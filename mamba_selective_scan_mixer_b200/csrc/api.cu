@@ -261,10 +261,10 @@ jamba_status reorder_channels(jamba_mamba* h) {
 // The weights the prefill runs on: the reordered copy when the handle has one.
 const jamba_mamba_weights& prefill_weights(const jamba_mamba& h) { return h.perm ? h.wp : h.w; }
 
-// The prefill up to the scan's inputs: in_proj, conv + SiLU (cache in -> out),
-// x_proj, inner RMSNorms, dt_proj + softplus.
-jamba_status prefill_front(const jamba_mamba& h, const PrefillWs& p, const void* u, int batch, int seqlen,
-                           const float* conv_state_in, float* conv_state_out, cudaStream_t s) {
+// The prefill's first steps: in_proj, conv + SiLU (cache in -> out), x_proj
+// into split-K partials (p.xpart, p.splits of them).
+jamba_status prefill_front_a(const jamba_mamba& h, const PrefillWs& p, const void* u, int batch, int seqlen,
+                             const float* conv_state_in, float* conv_state_out, cudaStream_t s) {
   const jamba_mamba_config& c = h.cfg;
   const jamba_mamba_weights& w = prefill_weights(h);
   const int T = batch * seqlen, di = c.d_inner, dm = c.d_model, R = c.dt_rank, N = c.d_state;
@@ -285,13 +285,30 @@ jamba_status prefill_front(const jamba_mamba& h, const PrefillWs& p, const void*
   gx.splits = p.splits;
   gx.split_stride = (long long)T * W;
   if (c.dtype == JAMBA_BF16) gx.bn = 144;
-  JB_TRY(gemm_any(c.dtype, gx, s));
-  JB_TRY(xproj_norm(p.xpart, p.splits, (long long)T * W, T, R, N, w.norm_dt, w.norm_B, w.norm_C, c.inner_rmsnorm,
-                    c.eps, p.dtlow, p.bc, c.dtype, s));
-  // dt = softplus(dt_low W_dt^T + dt_bias)
+  return gemm_any(c.dtype, gx, s);
+}
+
+// Then: the x_proj sum (`splits` fp32 partials of [T, R + 2N] at `part`) through
+// the inner RMSNorms into dt_low and B|C, and dt = softplus(dt_low W_dt^T + dt_bias).
+jamba_status prefill_front_b(const jamba_mamba& h, const PrefillWs& p, const float* part, int splits, int batch,
+                             int seqlen, cudaStream_t s) {
+  const jamba_mamba_config& c = h.cfg;
+  const jamba_mamba_weights& w = prefill_weights(h);
+  const int T = batch * seqlen, di = c.d_inner, R = c.dt_rank, N = c.d_state;
+  const int W = R + 2 * N;
+  JB_TRY(xproj_norm(part, splits, (long long)T * W, T, R, N, w.norm_dt, w.norm_B, w.norm_C, c.inner_rmsnorm, c.eps,
+                    p.dtlow, p.bc, c.dtype, s));
   GemmDesc gd = gdesc(p.dtlow, R, w.dt_proj, R, T, di, R, EPI_SOFTPLUS, p.dt, di);
   gd.bias = w.dt_bias;
   return gemm_any(c.dtype, gd, s);
+}
+
+// The prefill up to the scan's inputs: in_proj, conv + SiLU (cache in -> out),
+// x_proj, inner RMSNorms, dt_proj + softplus.
+jamba_status prefill_front(const jamba_mamba& h, const PrefillWs& p, const void* u, int batch, int seqlen,
+                           const float* conv_state_in, float* conv_state_out, cudaStream_t s) {
+  JB_TRY(prefill_front_a(h, p, u, batch, seqlen, conv_state_in, conv_state_out, s));
+  return prefill_front_b(h, p, p.xpart, p.splits, batch, seqlen, s);
 }
 
 // The scan's arguments over the front's outputs.
@@ -470,6 +487,68 @@ jamba_status jamba_mamba_prefill(jamba_mamba_t h, const void* u, const void* res
   cudaStream_t s = cs(stream);
   JB_TRY(prefill_front(*h, p, u, batch, seqlen, conv_state_in, conv_state_out, s));
   return prefill_back(*h, p, batch, seqlen, ssm_state_in, ssm_state_out, residual, out, s);
+}
+
+// ------------------------------------------------- tensor-parallel prefill
+
+jamba_status jamba_mamba_prefill_tp_begin(jamba_mamba_t h, const void* u, int batch, int seqlen,
+                                          const float* conv_state_in, float* conv_state_out, float* xproj_part,
+                                          void* ws, size_t ws_bytes, jamba_stream_t stream) {
+  if (!h) return fail(JAMBA_ERR_INVALID_ARG, "tp begin: null handle");
+  if (batch <= 0 || seqlen <= 0) return fail(JAMBA_ERR_INVALID_ARG, "tp begin: batch and seqlen must be positive");
+  JB_TRY(check_device(h));
+  JB_TRY(check_ptr(u, "u"));
+  JB_TRY(check_ptr(conv_state_in, "conv_state_in", false));
+  JB_TRY(check_ptr(conv_state_out, "conv_state_out", false));
+  JB_TRY(check_ptr(xproj_part, "xproj_part"));
+  JB_TRY(check_ptr(ws, "workspace"));
+  const jamba_mamba_config& c = h->cfg;
+  if ((long long)batch * seqlen > (1LL << 31) / 2) return fail(JAMBA_ERR_UNSUPPORTED, "tp begin: too many tokens");
+  PrefillWs p = carve_prefill(h, batch, seqlen, ws);
+  if (ws_bytes < p.total) return fail(JAMBA_ERR_WORKSPACE, "tp begin: workspace too small");
+  cudaStream_t s = cs(stream);
+  const long long T = (long long)batch * seqlen, W = c.dt_rank + 2 * c.d_state;
+  JB_TRY(prefill_front_a(*h, p, u, batch, seqlen, conv_state_in, conv_state_out, s));
+  // this rank's share of x_proj: its split-K partials summed (fp32)
+  return splitk_reduce(p.xpart, p.splits, T * W, T * W, nullptr, xproj_part, JAMBA_F32, s);
+}
+
+jamba_status jamba_mamba_prefill_tp_finish(jamba_mamba_t h, const float* xproj_sum, int batch, int seqlen,
+                                           const float* ssm_state_in, float* ssm_state_out, float* out_part,
+                                           void* ws, size_t ws_bytes, jamba_stream_t stream) {
+  if (!h) return fail(JAMBA_ERR_INVALID_ARG, "tp finish: null handle");
+  if (batch <= 0 || seqlen <= 0) return fail(JAMBA_ERR_INVALID_ARG, "tp finish: batch and seqlen must be positive");
+  JB_TRY(check_device(h));
+  JB_TRY(check_ptr(xproj_sum, "xproj_sum"));
+  JB_TRY(check_ptr(ssm_state_in, "ssm_state_in", false));
+  JB_TRY(check_ptr(ssm_state_out, "ssm_state_out", false));
+  JB_TRY(check_ptr(out_part, "out_part"));
+  JB_TRY(check_ptr(ws, "workspace"));
+  const jamba_mamba_config& c = h->cfg;
+  PrefillWs p = carve_prefill(h, batch, seqlen, ws);
+  if (ws_bytes < p.total) return fail(JAMBA_ERR_WORKSPACE, "tp finish: workspace too small");
+  cudaStream_t s = cs(stream);
+  const int T = batch * seqlen, di = c.d_inner, dm = c.d_model;
+  JB_TRY(prefill_front_b(*h, p, xproj_sum, 1, batch, seqlen, s));
+  ScanCall sc = scan_call(*h, p, batch, seqlen);
+  sc.h0 = ssm_state_in;
+  sc.h_out = ssm_state_out;
+  JB_TRY(scan_run(sc, s));
+  // this rank's share of out_proj (its d_inner columns), fp32
+  GemmDesc go = gdesc(p.y, di, prefill_weights(*h).out_proj, di, T, dm, di, EPI_F32, out_part, dm);
+  return gemm_any(c.dtype, go, s);
+}
+
+jamba_status jamba_mamba_prefill_tp_end(jamba_mamba_t h, const float* out_sum, const void* residual, void* out,
+                                        int batch, int seqlen, jamba_stream_t stream) {
+  if (!h) return fail(JAMBA_ERR_INVALID_ARG, "tp end: null handle");
+  if (batch <= 0 || seqlen <= 0) return fail(JAMBA_ERR_INVALID_ARG, "tp end: batch and seqlen must be positive");
+  JB_TRY(check_device(h));
+  JB_TRY(check_ptr(out_sum, "out_sum"));
+  JB_TRY(check_ptr(residual, "residual", false));
+  JB_TRY(check_ptr(out, "out"));
+  const long long n = (long long)batch * seqlen * h->cfg.d_model;
+  return splitk_reduce(out_sum, 1, n, n, residual, out, h->cfg.dtype, cs(stream));
 }
 
 // ------------------------------------------------- context-parallel prefill

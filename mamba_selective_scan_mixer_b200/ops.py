@@ -110,6 +110,46 @@ class MambaMixer:
                                         ws.numel(), _stream(stream)))
         return out, conv_state_out, ssm_state_out
 
+    def prefill_tp_begin(self, u, conv_state_in=None, stream=None):
+        """Tensor-parallel prefill, first part, on this rank's channel shard:
+        returns (xproj_part [B*L, R+2N] fp32, conv_state_out)."""
+        _cuda(u, conv_state_in)
+        _contig(u, "u")
+        B, L, _ = u.shape
+        sh = self.shape
+        part = torch.empty(B * L, sh.dt_rank + 2 * sh.d_state, device=u.device)
+        cs = torch.empty(B, sh.d_inner, sh.d_conv - 1, device=u.device)
+        ws = self.ws.get(self.workspace_size(B, L), u.device)
+        check(lib().jamba_mamba_prefill_tp_begin(self.handle, _p(u), B, L, _p(conv_state_in), _p(cs), _p(part),
+                                                 _p(ws), ws.numel(), _stream(stream)))
+        self._tp = (B, L)
+        return part, cs
+
+    def prefill_tp_finish(self, xproj_sum, ssm_state_in=None, stream=None):
+        """Second part from the all-reduced x_proj sum: returns (out_part [B*L,
+        d_model] fp32, ssm_state_out)."""
+        B, L = self._tp
+        _cuda(xproj_sum, ssm_state_in)
+        _contig(xproj_sum, "xproj_sum")
+        sh = self.shape
+        out = torch.empty(B * L, sh.d_model, device=self.device)
+        ss = torch.empty(B, sh.d_inner, sh.d_state, device=self.device)
+        ws = self.ws.get(self.workspace_size(B, L), self.device)
+        check(lib().jamba_mamba_prefill_tp_finish(self.handle, _p(xproj_sum), B, L, _p(ssm_state_in), _p(ss),
+                                                  _p(out), _p(ws), ws.numel(), _stream(stream)))
+        return out, ss
+
+    def prefill_tp_end(self, out_sum, residual=None, out=None, stream=None):
+        """out = out_sum (+ residual) in the model dtype, [B, L, d_model]."""
+        B, L = self._tp
+        _cuda(out_sum, residual, out)
+        _contig(out_sum, "out_sum")
+        _contig(residual, "residual")
+        out = torch.empty(B, L, self.shape.d_model, dtype=self.dtype, device=self.device) if out is None else out
+        check(lib().jamba_mamba_prefill_tp_end(self.handle, _p(out_sum), _p(residual), _p(out), B, L,
+                                               _stream(stream)))
+        return out
+
     def cp_workspace_size(self, batch, seqlen):
         n = ctypes.c_size_t()
         check(lib().jamba_mamba_cp_workspace_size(self.handle, batch, seqlen, ctypes.byref(n)))

@@ -79,3 +79,53 @@ def test_context_parallel_exchange(world):
         assert res[r][1] == res[r - 1][3]
     for r in range(world):
         assert res[r][2] == [float(j) for j in range(world)]
+
+
+def _tp_reduce_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    import datetime
+    import torch
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    from mamba_selective_scan_mixer_b200 import tensor_parallel as tp
+    t = torch.full((3, 5), float(rank + 1))
+    tp._all_reduce(t)
+    q.put((rank, t.tolist()))
+    dist.destroy_process_group()
+
+
+def test_tensor_parallel_all_reduce_sums_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    world = 3
+    procs = [ctx.Process(target=_tp_reduce_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for _, t in res:
+        assert t == [[6.0] * 5] * 3
+
+
+def test_tensor_parallel_shards_cover_the_channels():
+    """The shards of every channel-indexed weight put back together are the
+    original weights (in_proj: x rows, then z rows, of each shard)."""
+    import torch
+    from mamba_selective_scan_mixer_b200 import tensor_parallel as tp
+    from synthetic import MambaShape, mamba_params
+    sh = MambaShape(d_model=32, d_inner=64, dt_rank=8, dtype="f32")
+    p = mamba_params(sh, seed=1, a_init="random", norm_init="random", d_init="random")
+    world, k = 4, 16
+    sh_ = [tp.shard_params(p, r, world) for r in range(world)]
+    x = torch.cat([s["in_proj"][:k] for s in sh_])
+    z = torch.cat([s["in_proj"][k:] for s in sh_])
+    assert torch.equal(torch.cat([x, z]), p["in_proj"])
+    for n in ("conv_w", "conv_b", "dt_proj", "dt_bias", "A", "D"):
+        assert torch.equal(torch.cat([s[n] for s in sh_]), p[n])
+    for n in ("x_proj", "out_proj"):
+        assert torch.equal(torch.cat([s[n] for s in sh_], dim=1), p[n])
+    for n in ("norm_dt", "norm_B", "norm_C"):
+        assert all(torch.equal(s[n], p[n]) for s in sh_)
