@@ -32,11 +32,6 @@ struct jamba_mamba {
   // the double-buffered chunks (created on first use)
   cudaStream_t io_in = nullptr, io_out = nullptr;
   cudaEvent_t ev_in[2] = {nullptr, nullptr}, ev_comp[2] = {nullptr, nullptr}, ev_out[2] = {nullptr, nullptr};
-  // bf16 decode: a side stream that pulls out_proj's weights into L2 while the
-  // step's small kernels run (created with the handle, so a first step inside
-  // a stream capture needs no stream creation)
-  cudaStream_t pf = nullptr;
-  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
 };
 
 namespace {
@@ -417,12 +412,6 @@ jamba_status jamba_mamba_create(const jamba_mamba_config* cfg, const jamba_mamba
       for (int n = 0; n < c.d_state; ++n)
         power = power && A[(size_t)ch * c.d_state + n] == (float)(n + 1) * A[(size_t)ch * c.d_state];
     h->a_form = power ? jb::SCAN_A_POWER : jb::SCAN_A_GENERAL;
-    if (cudaStreamCreateWithFlags(&h->pf, cudaStreamNonBlocking) != cudaSuccess ||
-        cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming) != cudaSuccess) {
-      jamba_mamba_destroy(h);
-      return fail(JAMBA_ERR_CUDA, "create: could not create the decode prefetch stream");
-    }
   }
   if (c.dtype == JAMBA_BF16 && (c.d_inner + SCAN_GROUP_CHANNELS - 1) / SCAN_GROUP_CHANNELS <= SCAN_MAX_GROUPS) {
     const jamba_status st = reorder_channels(h);
@@ -437,9 +426,6 @@ jamba_status jamba_mamba_create(const jamba_mamba_config* cfg, const jamba_mamba
 
 jamba_status jamba_mamba_destroy(jamba_mamba_t h) {
   if (h) {
-    if (h->pf) cudaStreamDestroy(h->pf);
-    if (h->ev_fork) cudaEventDestroy(h->ev_fork);
-    if (h->ev_join) cudaEventDestroy(h->ev_join);
     if (h->own) cudaFree(h->own);
     if (h->io_in) cudaStreamDestroy(h->io_in);
     if (h->io_out) cudaStreamDestroy(h->io_out);
@@ -659,12 +645,6 @@ jamba_status jamba_mamba_step(jamba_mamba_t h, const void* u, const void* residu
     g1.xc_out = p.xc;
     g1.conv_c = di;
     JB_TRY(gemm_bf16(g1, s));
-    // once in_proj's weight stream is done, out_proj's weights (d_model x d_inner bf16, which fit
-    // L2 beside the caches) are prefetched on the side stream while the small kernels below run
-    JB_CUDA(cudaEventRecord(h->ev_fork, s));
-    JB_CUDA(cudaStreamWaitEvent(h->pf, h->ev_fork, 0));
-    JB_TRY(l2_prefetch(w.out_proj, (size_t)dm * di * 2, h->pf));
-    JB_CUDA(cudaEventRecord(h->ev_join, h->pf));
     GemmDesc g2 = gdesc(w.x_proj, di, p.xc, di, W, batch, di, EPI_F32, p.xpart, W);
     g2.transpose_out = 1;
     g2.bn = 64;
@@ -680,7 +660,6 @@ jamba_status jamba_mamba_step(jamba_mamba_t h, const void* u, const void* residu
     JB_TRY(gemm_bf16(g3, s));
     JB_TRY(ssm_step(p.xc, reinterpret_cast<const uint8_t*>(p.xz) + (size_t)di * 2, 2 * di, p.dt, p.bc, 2 * N, w.A,
                     w.D, ssm_state, p.y, batch, di, c.dtype, s));
-    JB_CUDA(cudaStreamWaitEvent(s, h->ev_join, 0));
     GemmDesc g4 = gdesc(w.out_proj, di, p.y, di, dm, batch, di, EPI_F32, p.opart, dm);
     g4.transpose_out = 1;
     g4.bn = 64;

@@ -143,27 +143,6 @@ static jamba_status gemm_i8w(const GemmDesc& g, cudaStream_t s) {
   return pairs ? launch_i8w<EPI_F32, 2>(ma, mq, mq2, p, grid, s) : launch_i8w<EPI_F32, 1>(ma, mq, mq2, p, grid, s);
 }
 
-// Pulls `bytes` at p into L2 (bulk prefetches of 64 KB, no completion to wait
-// for): weights a later kernel of the same step will stream, fetched while the
-// kernels in between leave HBM idle.
-__global__ void __launch_bounds__(128) l2_prefetch_kernel(const uint8_t* __restrict__ p, size_t bytes) {
-  constexpr size_t kChunk = 65536;
-  const size_t stride = (size_t)gridDim.x * blockDim.x * kChunk;
-  for (size_t off = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * kChunk; off < bytes; off += stride) {
-    const uint32_t n = (uint32_t)(bytes - off < kChunk ? bytes - off : kChunk);
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p + off), "r"(n) : "memory");
-  }
-}
-
-jamba_status l2_prefetch(const void* p, size_t bytes, cudaStream_t s) {
-  if (!aligned16(p) || bytes % 16) return fail(JAMBA_ERR_INVALID_ARG, "l2 prefetch: 16-byte aligned sizes only");
-  const size_t chunks = (bytes + 65535) / 65536;
-  const unsigned grid = (unsigned)((chunks + 127) / 128);
-  l2_prefetch_kernel<<<grid > 0 ? grid : 1, 128, 0, s>>>(reinterpret_cast<const uint8_t*>(p), bytes);
-  JB_CUDA(cudaGetLastError());
-  return JAMBA_OK;
-}
-
 jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
   if (g.M <= 0 || g.N <= 0 || g.K <= 0) return fail(JAMBA_ERR_INVALID_ARG, "gemm: sizes must be positive");
   if (!g.a || !g.b || !g.out) return fail(JAMBA_ERR_INVALID_ARG, "gemm: null operand");

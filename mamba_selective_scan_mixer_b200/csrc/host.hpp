@@ -90,7 +90,6 @@ struct GemmDesc {
   const void* conv_w; const void* conv_b; float* conv_state; void* xc_out; int conv_c;
 };
 jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s);
-jamba_status l2_prefetch(const void* p, size_t bytes, cudaStream_t s);   // bulk L2 prefetch, fire and forget
 jamba_status gemm_f32(const GemmDesc& g, cudaStream_t s);
 
 // Splits so that m_tiles * n_tiles * splits fills the SMs, each split keeping
