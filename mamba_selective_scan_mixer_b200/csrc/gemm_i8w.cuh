@@ -366,6 +366,10 @@ constexpr int I8T_EPI_WARPS = 4;   // one per TMEM lane quarter: a 32-token tile
 constexpr int I8T_DQ_WARPS = 8;    // two per SM sub-partition
 constexpr int I8T_THREADS = 32 * (2 + I8T_EPI_WARPS + I8T_DQ_WARPS);
 
+// The widened weights never touch shared memory: the dequantiser warps write
+// them into tensor memory (tcgen05.st, one weight row per TMEM lane) and the
+// MMA takes its A operand from there, so shared memory carries only the codes
+// (1 byte per weight) and the activations.
 template <int EPI>
 struct I8tSmem {
   static constexpr int QROWS = EPI == EPI_SWIGLU ? 256 : 128;     // gate + up, or down rows
@@ -373,14 +377,16 @@ struct I8tSmem {
   static constexpr uint32_t X_BYTES = 2 * X_SUB;                    // two 64-deep steps per stage
   static constexpr uint32_t Q_BYTES = QROWS * 128;                  // QROWS x 128 codes
   static constexpr uint32_t T_STAGE = X_BYTES + Q_BYTES;            // a multiple of 1024
-  static constexpr int TSTAGES = EPI == EPI_SWIGLU ? 4 : 6;
-  static constexpr int BSTAGES = 2;
-  static constexpr uint32_t B_BYTES = QROWS * 128;                  // QROWS x 64 bf16 widened
-  static constexpr uint32_t B_OFF = TSTAGES * T_STAGE;
-  static constexpr uint32_t BAR_OFF = B_OFF + BSTAGES * B_BYTES;
+  static constexpr int TSTAGES = EPI == EPI_SWIGLU ? 5 : 8;
+  static constexpr int BSTAGES = 4;                                 // widened 64-deep steps in TMEM
+  static constexpr uint32_t BAR_OFF = TSTAGES * T_STAGE;
   static constexpr uint32_t BYTES = BAR_OFF + 256 + 1024;
-  static constexpr int ACC = EPI == EPI_SWIGLU ? 2 * I8T_BNT : I8T_BNT;   // TMEM columns per buffer
-  static constexpr uint32_t TMEM_COLS = 2 * ACC <= 32 ? 32 : 2 * ACC <= 64 ? 64 : 128;
+  static constexpr int ACC = EPI == EPI_SWIGLU ? 2 * I8T_BNT : I8T_BNT;   // TMEM columns per accumulator
+  static constexpr int A_COLS = (QROWS / 128) * 32;                 // widened 128 x 64 tiles, 32 columns each
+  static constexpr int A_OFF = 2 * ACC;                             // after the two accumulators
+  static constexpr int USED = A_OFF + BSTAGES * A_COLS;
+  static constexpr uint32_t TMEM_COLS = USED <= 32 ? 32 : USED <= 64 ? 64 : USED <= 128 ? 128 : USED <= 256 ? 256 : 512;
+  static_assert(USED <= 512, "tensor memory");
 };
 
 // Codes h*64 .. h*64+63 of ROWS rows stored as 128-byte rows under the
@@ -464,7 +470,6 @@ gemm_i8w_tok_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   constexpr int BST = S::BSTAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sB = smem + S::B_OFF;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::BAR_OFF);
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + TST);
   const uint32_t bfull0 = smem_u32(bars + 2 * TST);
@@ -546,15 +551,14 @@ gemm_i8w_tok_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             if (!mbar_wait(bfull0 + 8 * bs, bph, p.err)) { ok = false; break; }
             tc_fence_after();
             const uint64_t xd = sw128_desc(smem_u32(smem + ts * S::T_STAGE + h * S::X_SUB));
-            const uint64_t wd = sw128_desc(smem_u32(sB + bs * S::B_BYTES));
+            const uint32_t wa = tbase + S::A_OFF + bs * S::A_COLS;   // widened weights in TMEM
             const uint32_t acc0 = (kt > ti.kt0 || h > 0) ? 1u : 0u;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) umma_bf16(d0, wd + 2 * kk, xd + 2 * kk, IDESC, (acc0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk) umma_bf16_ta(d0, wa + 8 * kk, xd + 2 * kk, IDESC, (acc0 || kk > 0) ? 1u : 0u);
             if constexpr (EPI == EPI_SWIGLU) {
-              const uint64_t ud = sw128_desc(smem_u32(sB + bs * S::B_BYTES + 128 * 128));
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
-                umma_bf16(d0 + BNT, ud + 2 * kk, xd + 2 * kk, IDESC, (acc0 || kk > 0) ? 1u : 0u);
+                umma_bf16_ta(d0 + BNT, wa + 32 + 8 * kk, xd + 2 * kk, IDESC, (acc0 || kk > 0) ? 1u : 0u);
             }
             umma_commit(bempty0 + 8 * bs);
             if (++bs == BST) { bs = 0; bph ^= 1; }
@@ -570,8 +574,19 @@ gemm_i8w_tok_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       mbar_wait(drain, 0, p.err);
     }
   } else if (warp >= 2 + I8T_EPI_WARPS) {
-    const WidenPlan<S::QROWS, I8T_DQ_WARPS> plan(threadIdx.x - 32 * (2 + I8T_EPI_WARPS));
-    const uint32_t qbase = smem_u32(smem + S::X_BYTES), bbase = smem_u32(sB);
+    // Dequantiser warps, two per TMEM lane quarter q: thread `lane` widens row
+    // 32 q + lane of a 128-row weight tile.  SwiGLU: the warp pair splits the
+    // gate and up tiles; down: it splits the 64-deep step into two halves.
+    // Codes sit in 128-byte rows under the 128-byte swizzle (16-byte chunk c of
+    // row r at r * 128 + ((c ^ (r & 7)) << 4)): eight consecutive rows read
+    // eight distinct chunk positions, so a quarter-warp's loads are conflict-free.
+    const int q = warp & 3;
+    const int pi = (warp - 2 - I8T_EPI_WARPS) >> 2;   // which warp of the quarter's pair
+    const int r = q * 32 + lane;
+    constexpr bool SW = EPI == EPI_SWIGLU;
+    const uint32_t row_off = (uint32_t)((SW ? pi * 128 : 0) + r) * 128;
+    const uint32_t qbase = smem_u32(smem + S::X_BYTES) + row_off;
+    const uint32_t tl = tbase + ((uint32_t)(q * 32) << 16) + S::A_OFF + (SW ? pi * 32 : pi * 16);
     int ts = 0, bs = 0;
     uint32_t tph = 0, bph = 0;
     bool ok = true;
@@ -580,10 +595,26 @@ gemm_i8w_tok_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       decode_tile_tok(p, t, ti);
       for (int kt = ti.kt0; kt < ti.kt1 && ok; kt += 2) {
         if (!mbar_wait_warp(full0 + 8 * ts, tph, p.err)) { ok = false; break; }
+        const uint32_t qs = qbase + ts * S::T_STAGE;
         for (int h = 0; h < 2; ++h) {
           if (!mbar_wait_warp(bempty0 + 8 * bs, bph ^ 1, p.err)) { ok = false; break; }
-          plan.run(qbase + ts * S::T_STAGE, h, bbase + bs * S::B_BYTES);
-          fence_async_shared();
+          tc_fence_after();
+          constexpr int NCH = SW ? 4 : 2;        // 16-byte code chunks this thread widens
+          uint32_t wv[2 * 4 * NCH];
+#pragma unroll
+          for (int i = 0; i < NCH; ++i) {
+            const int c = 4 * h + (SW ? 0 : 2 * pi) + i;
+            uint4 v, lo, hi;
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(qs + ((c ^ (r & 7)) << 4)));
+            widen16(v, lo, hi);
+            wv[8 * i] = lo.x; wv[8 * i + 1] = lo.y; wv[8 * i + 2] = lo.z; wv[8 * i + 3] = lo.w;
+            wv[8 * i + 4] = hi.x; wv[8 * i + 5] = hi.y; wv[8 * i + 6] = hi.z; wv[8 * i + 7] = hi.w;
+          }
+          if constexpr (SW) tmem_st32u(tl + bs * S::A_COLS, wv);
+          else tmem_st16u(tl + bs * S::A_COLS, wv);
+          tmem_wait_st();
+          tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(bfull0 + 8 * bs);
           if (++bs == BST) { bs = 0; bph ^= 1; }
