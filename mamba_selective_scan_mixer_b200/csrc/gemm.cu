@@ -9,20 +9,20 @@
 
 namespace jb {
 
-template <int BN, int STAGES, int EPI, bool TRANS>
+template <int BN, int STAGES, int EPI, bool TRANS, int EW = GEMM_EPI_WARPS>
 static jamba_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb2,
                               const CUtensorMap& mc, const GemmParams& p, int grid, cudaStream_t s) {
-  using S = GemmSmem<BN, STAGES, EPI == EPI_SOFTPLUS && !TRANS>;
+  using S = GemmSmem<BN, STAGES, EPI == EPI_SOFTPLUS && !TRANS, EW, gemm_nstg<EW>()>;
   static std::atomic<bool> configured[64];
   int dev = 0;
   JB_CUDA(cudaGetDevice(&dev));
   if (dev < 64 && !configured[dev]) {
-    JB_CUDA(cudaFuncSetAttribute(gemm_bf16_tc_kernel<BN, STAGES, EPI, TRANS>,
+    JB_CUDA(cudaFuncSetAttribute(gemm_bf16_tc_kernel<BN, STAGES, EPI, TRANS, EW>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::BYTES));
     configured[dev] = true;
   }
-  JB_CUDA(launch_pdl(gemm_bf16_tc_kernel<BN, STAGES, EPI, TRANS>, dim3(grid), dim3(GEMM_THREADS), S::BYTES, s, ma, mb,
-                     mb2, mc, p));
+  JB_CUDA(launch_pdl(gemm_bf16_tc_kernel<BN, STAGES, EPI, TRANS, EW>, dim3(grid), dim3(64 + 32 * EW), S::BYTES, s,
+                     ma, mb, mb2, mc, p));
   return JAMBA_OK;
 }
 
@@ -64,8 +64,11 @@ static jamba_status launch_bn(int bn, const CUtensorMap& ma, const CUtensorMap& 
   if constexpr (TRANS) {
     if (bn == 64) return launch_tc<64, 8, EPI, true>(ma, mb, mb2, mc, p, grid, s);
   } else if constexpr (EPI == EPI_SOFTPLUS) {
-    // three stages: the ring and the TMA-store staging boxes share the 227 KB
-    if (bn == 256) return launch_tc<256, 3, EPI, false>(ma, mb, mb2, mc, p, grid, s);
+    // bias + softplus of every output element: sixteen epilogue warps (four per
+    // scheduler) keep the epilogue, which bounds this GEMM (K = dt_rank is
+    // short), fed; three ring stages and one TMA-store box per epilogue warp
+    // share the 227 KB
+    if (bn == 256) return launch_tc<256, 3, EPI, false, 16>(ma, mb, mb2, mc, p, grid, s);
   } else if constexpr (EPI == EPI_SWIGLU) {
     if (bn == 256) return launch_tc<256, 4, EPI, false>(ma, mb, mb2, mc, p, grid, s);
   } else {

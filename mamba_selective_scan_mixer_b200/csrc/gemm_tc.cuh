@@ -273,17 +273,19 @@ __device__ __forceinline__ void epi_chunk(const GemmParams& p, const TileInfo& t
   }
 }
 
-template <int BN, int STAGES, bool STAGED = false>
+// EW epilogue warps, EW / 4 per TMEM lane quarter; NSTG staging boxes per
+// epilogue warp in the staged (TMA-store) epilogue.
+template <int BN, int STAGES, bool STAGED = false, int EW = GEMM_EPI_WARPS, int NSTG = 2>
 struct GemmSmem {
   static constexpr uint32_t A_BYTES = 128 * 128;
   static constexpr uint32_t B_BYTES = BN * 128;
-  // STAGED: per epilogue warp two 32 x 32 fp32 boxes for TMA stores (1024-aligned)
+  // STAGED: per epilogue warp NSTG 32 x 32 fp32 boxes for TMA stores (1024-aligned)
   static constexpr uint32_t STG_OFF = STAGES * (A_BYTES + B_BYTES);
-  static constexpr uint32_t STG_BYTES = STAGED ? GEMM_EPI_WARPS * 2 * 4096 : 0;
+  static constexpr uint32_t STG_BYTES = STAGED ? EW * NSTG * 4096 : 0;
   // STAGED: per epilogue warp the bias of its 32-column chunks of the tile
-  static constexpr int SB_CHUNKS = (BN / 32 + 1) / 2;
+  static constexpr int SB_CHUNKS = (BN / 32 + EW / 4 - 1) / (EW / 4);
   static constexpr uint32_t SB_OFF = STG_OFF + STG_BYTES;
-  static constexpr uint32_t SB_BYTES = STAGED ? GEMM_EPI_WARPS * SB_CHUNKS * 128 : 0;
+  static constexpr uint32_t SB_BYTES = STAGED ? EW * SB_CHUNKS * 128 : 0;
   static constexpr uint32_t BAR_OFF = SB_OFF + SB_BYTES;
   // barrier slots: full[STAGES], empty[STAGES], tmem_full[2], tmem_empty[2], drain, tmem holder
   static_assert(8 * (2 * STAGES + 6) <= 256, "barrier slots");
@@ -292,14 +294,21 @@ struct GemmSmem {
                                         : (2 * BN <= 256) ? 256 : 512;
 };
 
-template <int BN, int STAGES, int EPI, bool TRANS>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
+// Staging boxes per epilogue warp: two with the default eight epilogue warps,
+// one with more (shared memory is the limit).
+template <int EW> constexpr int gemm_nstg() { return EW > GEMM_EPI_WARPS ? 1 : 2; }
+
+template <int BN, int STAGES, int EPI, bool TRANS, int EW = GEMM_EPI_WARPS>
+__global__ void __launch_bounds__(64 + 32 * EW, 1)
 gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmC,
                     const GemmParams p) {
   // fp32 softplus outputs (dt) leave through shared memory and TMA stores
   constexpr bool STAGED = EPI == EPI_SOFTPLUS && !TRANS;
-  using S = GemmSmem<BN, STAGES, STAGED>;
+  constexpr int NSTG = gemm_nstg<EW>();
+  constexpr int WPQ = EW / 4;                 // epilogue warps per TMEM lane quarter
+  static_assert(EW % 4 == 0 && EW >= 4, "whole lane quarters");
+  using S = GemmSmem<BN, STAGES, STAGED, EW, NSTG>;
   static_assert(BN % 16 == 0 && BN >= 32 && BN <= 256, "UMMA N for M = 128");
   constexpr int BN_OUT = EPI == EPI_SWIGLU ? BN / 2 : BN;
   extern __shared__ uint8_t smem_raw[];
@@ -321,7 +330,7 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(tfull0 + 8 * i, 1);
-      mbar_init(tempty0 + 8 * i, GEMM_EPI_WARPS);
+      mbar_init(tempty0 + 8 * i, EW);
     }
     mbar_init(drain, 1);
     mbar_fence_init();
@@ -421,7 +430,7 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     griddep_wait();
     const int ntiles = total_tiles(p);
     const int q = warp & 3;                 // TMEM lane quarter this warp may access
-    const int half = (warp - 2) >> 2;       // which of the two warps of this quarter
+    const int half = (warp - 2) >> 2;       // which of the WPQ warps of this quarter
     int it = 0;
     int stg_count = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
@@ -435,8 +444,8 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       if constexpr (STAGED) {
 #pragma unroll
         for (int jj = 0; jj < S::SB_CHUNKS; ++jj) {
-          const int col = ti.n0 + (half + 2 * jj) * 32 + lane;
-          bl[jj] = (half + 2 * jj < BN / 32 && col < p.N) ? __ldg(p.bias + col) : 0.f;
+          const int col = ti.n0 + (half + WPQ * jj) * 32 + lane;
+          bl[jj] = (half + WPQ * jj < BN / 32 && col < p.N) ? __ldg(p.bias + col) : 0.f;
         }
       }
       if (!mbar_wait_warp(tfull0 + 8 * acc, use & 1, p.err)) break;
@@ -445,25 +454,28 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       const uint32_t tl = tbase + ((uint32_t)(q * 32) << 16) + acc * BN;
       if constexpr (STAGED) {
         static_assert(BN % 32 == 0, "staged epilogue works on whole 32-column chunks");
-        uint8_t* stg = smem + S::STG_OFF + (warp - 2) * 8192;
+        uint8_t* stg = smem + S::STG_OFF + (warp - 2) * (NSTG * 4096);
         float* sb = reinterpret_cast<float*>(smem + S::SB_OFF) + (warp - 2) * S::SB_CHUNKS * 32;
         __syncwarp();                    // every lane is done with the last tile's bias
 #pragma unroll
         for (int jj = 0; jj < S::SB_CHUNKS; ++jj) sb[jj * 32 + lane] = bl[jj];
         __syncwarp();
-        // this warp's chunks j = half, half + 2, ...; the TMEM load of the
+        // this warp's chunks j = half, half + WPQ, ...; the TMEM load of the
         // next one is in flight while the current one is processed
+        // (with more than two warps per quarter the others hide the load latency,
+        // and a single buffer keeps the registers within the budget)
         constexpr int NCH = BN / 32;
-        const int cnt = (NCH - half + 1) / 2;
-        float vb[2][32];
+        constexpr int NVB = WPQ > 2 ? 1 : 2;
+        const int cnt = (NCH - half + WPQ - 1) / WPQ;
+        float vb[NVB][32];
         if (cnt > 0) tmem_ld32(tl + half * 32, vb[0]);
 #pragma unroll
-        for (int jj = 0; jj < (NCH + 1) / 2; ++jj) {
+        for (int jj = 0; jj < (NCH + WPQ - 1) / WPQ; ++jj) {
           if (jj >= cnt) break;
-          const int j = half + 2 * jj;
-          float* v = vb[jj & 1];
+          const int j = half + WPQ * jj;
+          float* v = vb[jj % NVB];
           tmem_wait_ld32(v);
-          if (jj + 1 < cnt) tmem_ld32(tl + (j + 2) * 32, vb[(jj + 1) & 1]);
+          if (NVB == 2 && jj + 1 < cnt) tmem_ld32(tl + (j + WPQ) * 32, vb[(jj + 1) % NVB]);
           const int n = ti.n0 + j * 32;
           // the same 32 bias values for every lane: broadcast reads (zero past N,
           // where the TMA store clips the columns anyway)
@@ -473,8 +485,8 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             v[c] += b4.x; v[c + 1] += b4.y; v[c + 2] += b4.z; v[c + 3] += b4.w;
           }
           softplus32(v);
-          uint8_t* buf = stg + (stg_count & 1) * 4096;
-          if (lane == 0) bulk_wait_read<1>();   // this buffer's previous store has read it
+          uint8_t* buf = stg + (stg_count % NSTG) * 4096;
+          if (lane == 0) bulk_wait_read<NSTG - 1>();   // this buffer's previous store has read it
           __syncwarp();
           // row `lane` of the 32 x 32 box, 16-byte chunks placed by the 128-byte swizzle
 #pragma unroll
@@ -488,17 +500,18 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             bulk_commit();
           }
           ++stg_count;
+          if (NVB == 1 && jj + 1 < cnt) tmem_ld32(tl + (j + WPQ) * 32, vb[0]);
         }
       } else if constexpr (EPI != EPI_SWIGLU) {
 #pragma unroll 1
-        for (int j = half; j < BN / 32; j += 2) {
+        for (int j = half; j < BN / 32; j += WPQ) {
           float v[32];
           tmem_ld32(tl + j * 32, v);
           tmem_wait_ld();
           epi_chunk<EPI, TRANS, 32>(p, ti, m, ti.n0 + j * 32, v);
         }
         if constexpr (BN % 32 != 0) {
-          if (half == (BN / 32) % 2) {
+          if (half == (BN / 32) % WPQ) {
             float v[16];
             tmem_ld16(tl + (BN / 32) * 32, v);
             tmem_wait_ld();
@@ -508,7 +521,7 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       } else {
         bf16* o = reinterpret_cast<bf16*>(p.out) + (long long)m * p.ldo;
 #pragma unroll 1
-        for (int j = half; j < BN / 64; j += 2) {
+        for (int j = half; j < BN / 64; j += WPQ) {
           float g[32], u[32];
           tmem_ld32(tl + j * 32, g);
           tmem_ld32(tl + BN / 2 + j * 32, u);
