@@ -421,6 +421,47 @@ jamba_status jamba_moe_forward(const jamba_moe_config* cfg, const jamba_moe_weig
                                int32_t* topk_idx, float* topk_w, int32_t* expert_offsets,
                                int32_t* perm, void* ws, size_t ws_bytes, jamba_stream_t stream);
 
+/* ------------------------------------------------- expert-parallel MoE */
+
+/* The top-K MoE with its experts split over ranks (expert parallelism; the
+ * news article names MoE parallelism as a future speed-up, the summary page
+ * expert parallelism among its training parallelisms; no scheme is given).
+ * Each rank routes its own tokens, sends every routed row to the rank that
+ * owns its expert, runs its share of the experts on what it receives, and
+ * gets the results back; the caller does the two all-to-alls (and one of the
+ * per-expert row counts) between the calls.  Rank r owns experts
+ * [r E / world, (r + 1) E / world); a rank's routed rows are already in
+ * (expert, token, slot) order, so the rows for rank r are one contiguous
+ * range: expert_offsets[r E / world] .. expert_offsets[(r + 1) E / world].
+ *
+ * dispatch (cfg: the whole MoE, n_experts = E; router [E, d_model]):
+ *   routing as in jamba_moe_forward, and send_rows [tokens * top_k, d_model]
+ *   dtype, the routed rows in that order.  ws: jamba_moe_workspace_size(cfg,
+ *   tokens); it keeps the inverse permutation for combine: pass it unchanged.
+ * experts (cfg: this rank's share, n_experts = E / world; w: its w_gate /
+ *   w_up / w_down [and scales]; router unused):
+ *   rows_in [rows, d_model] dtype: the rows received, grouped by source rank
+ *   and, within one source, by local expert; group_counts [world * E_local]
+ *   int32 on the device: rows of (source s, local expert e) at s * E_local + e.
+ *   rows_out [rows, d_model] fp32: the expert outputs, same order.
+ *   ws: jamba_moe_ep_experts_workspace_size(cfg, rows, world).
+ * combine (cfg: the whole MoE): rows_back [tokens * top_k, d_model] fp32, the
+ *   expert outputs of this rank's routed rows in routed order; y = the
+ *   top-K weighted sum (+ residual), as jamba_moe_forward.
+ * Errors: INVALID_ARG, UNSUPPORTED (as jamba_moe_forward), WORKSPACE, CUDA. */
+jamba_status jamba_moe_ep_dispatch(const jamba_moe_config* cfg, const void* router, const void* x, int tokens,
+                                   int32_t* topk_idx, float* topk_w, int32_t* expert_offsets, int32_t* perm,
+                                   void* send_rows, void* ws, size_t ws_bytes, jamba_stream_t stream);
+jamba_status jamba_moe_ep_experts_workspace_size(const jamba_moe_config* cfg, int rows, int world,
+                                                 size_t* bytes);
+jamba_status jamba_moe_ep_experts(const jamba_moe_config* cfg, const jamba_moe_weights* w, const void* rows_in,
+                                  int rows, const int32_t* group_counts, int world, float* rows_out, void* ws,
+                                  size_t ws_bytes, jamba_stream_t stream);
+jamba_status jamba_moe_ep_combine(const jamba_moe_config* cfg, const float* rows_back, const float* topk_w,
+                                  int tokens, const void* residual, void* y, void* ws, size_t ws_bytes,
+                                  jamba_stream_t stream);
+
+
 /* ------------------------------------------------------------- attention */
 
 /* The Jamba block's attention layer ("Jamba: A Hybrid Transformer-Mamba

@@ -89,6 +89,10 @@ SIGNATURES = {
     "jamba_moe_workspace_size": [ctypes.POINTER(MoeConfig), I, ctypes.POINTER(SZ)],
     "jamba_moe_forward": [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), P, P, P, I, P, P, P, P,
                           P, SZ, P],
+    "jamba_moe_ep_dispatch": [ctypes.POINTER(MoeConfig), P, P, I, P, P, P, P, P, P, SZ, P],
+    "jamba_moe_ep_experts_workspace_size": [ctypes.POINTER(MoeConfig), I, I, ctypes.POINTER(SZ)],
+    "jamba_moe_ep_experts": [ctypes.POINTER(MoeConfig), ctypes.POINTER(MoeWeights), P, I, P, I, P, P, SZ, P],
+    "jamba_moe_ep_combine": [ctypes.POINTER(MoeConfig), P, P, I, P, P, P, SZ, P],
     "jamba_attn_prefill_workspace_size": [ctypes.POINTER(AttnConfig), I, I, ctypes.POINTER(SZ)],
     "jamba_attn_prefill": [ctypes.POINTER(AttnConfig), ctypes.POINTER(AttnWeights), P, P, P, I, I, P, P, I,
                            P, SZ, P],

@@ -1048,6 +1048,108 @@ jamba_status jamba_moe_forward(const jamba_moe_config* cfg, const jamba_moe_weig
   return JAMBA_OK;
 }
 
+// ------------------------------------------------------ expert-parallel MoE
+
+jamba_status jamba_moe_ep_dispatch(const jamba_moe_config* cfg, const void* router, const void* x, int tokens,
+                                   int32_t* topk_idx, float* topk_w, int32_t* expert_offsets, int32_t* perm,
+                                   void* send_rows, void* ws, size_t ws_bytes, jamba_stream_t stream) {
+  JB_TRY(check_moe_cfg(cfg));
+  if (tokens <= 0) return fail(JAMBA_ERR_INVALID_ARG, "moe ep dispatch: tokens must be positive");
+  JB_TRY(check_ptr(router, "router"));
+  JB_TRY(check_ptr(x, "x"));
+  JB_TRY(check_ptr(topk_idx, "topk_idx"));
+  JB_TRY(check_ptr(topk_w, "topk_w"));
+  JB_TRY(check_ptr(expert_offsets, "expert_offsets"));
+  JB_TRY(check_ptr(perm, "perm"));
+  JB_TRY(check_ptr(send_rows, "send_rows"));
+  JB_TRY(check_ptr(ws, "workspace"));
+  const jamba_moe_config& c = *cfg;
+  MoeWs m = carve_moe(c, tokens, ws);
+  if (ws_bytes < m.total) return fail(JAMBA_ERR_WORKSPACE, "moe ep dispatch: workspace too small");
+  cudaStream_t s = cs(stream);
+  JB_TRY(moe_route(x, router, tokens, c.d_model, c.n_experts, c.top_k, topk_idx, topk_w, m.counts, expert_offsets,
+                   perm, m.inv, s));
+  return moe_gather(x, perm, tokens * c.top_k, c.top_k, c.d_model, send_rows, s);
+}
+
+jamba_status jamba_moe_ep_experts_workspace_size(const jamba_moe_config* cfg, int rows, int world, size_t* bytes) {
+  JB_TRY(check_moe_cfg(cfg));
+  if (!bytes || rows < 0 || world <= 0) return fail(JAMBA_ERR_INVALID_ARG, "moe ep workspace: bad argument");
+  *bytes = al(sizeof(int) * ((size_t)world * cfg->n_experts + 1)) + al((size_t)(rows > 0 ? rows : 1) * cfg->d_ff * 2);
+  return JAMBA_OK;
+}
+
+jamba_status jamba_moe_ep_experts(const jamba_moe_config* cfg, const jamba_moe_weights* w, const void* rows_in,
+                                  int rows, const int32_t* group_counts, int world, float* rows_out, void* ws,
+                                  size_t ws_bytes, jamba_stream_t stream) {
+  JB_TRY(check_moe_cfg(cfg));
+  if (!w || rows < 0 || world <= 0 || world * cfg->n_experts > 4096)
+    return fail(JAMBA_ERR_INVALID_ARG, "moe ep experts: bad argument");
+  if (rows == 0) return JAMBA_OK;
+  JB_TRY(check_ptr(w->w_gate, "w_gate"));
+  JB_TRY(check_ptr(w->w_up, "w_up"));
+  JB_TRY(check_ptr(w->w_down, "w_down"));
+  const bool q8 = cfg->expert_dtype == JAMBA_INT8;
+  JB_TRY(check_ptr(w->s_gate, "s_gate", q8));
+  JB_TRY(check_ptr(w->s_up, "s_up", q8));
+  JB_TRY(check_ptr(w->s_down, "s_down", q8));
+  JB_TRY(check_ptr(rows_in, "rows_in"));
+  JB_TRY(check_ptr(group_counts, "group_counts"));
+  JB_TRY(check_ptr(rows_out, "rows_out"));
+  JB_TRY(check_ptr(ws, "workspace"));
+  size_t need = 0;
+  JB_TRY(jamba_moe_ep_experts_workspace_size(cfg, rows, world, &need));
+  if (ws_bytes < need) return fail(JAMBA_ERR_WORKSPACE, "moe ep experts: workspace too small");
+  const jamba_moe_config& c = *cfg;
+  const int E = c.n_experts, G = world * E, dm = c.d_model, dff = c.d_ff;
+  Carver cv(ws);
+  int* offsets = cv.take<int>(sizeof(int) * ((size_t)G + 1));
+  void* act = cv.take((size_t)rows * dff * 2);
+  cudaStream_t s = cs(stream);
+  // groups in received order: (source rank, local expert); group g uses local expert g % E
+  JB_TRY(group_offsets(group_counts, G, offsets, s));
+  GemmDesc g1 = gdesc(rows_in, dm, w->w_gate, dm, rows, dff, dm, EPI_SWIGLU, act, dff);
+  g1.b2 = w->w_up;
+  g1.grouped = 1;
+  g1.offsets = offsets;
+  g1.num_groups = G;
+  g1.group_mod = E;
+  g1.b_rows = dff;
+  if (q8) {
+    g1.b_int8 = 1;
+    g1.scale_b = w->s_gate;
+    g1.scale_b2 = w->s_up;
+  }
+  JB_TRY(gemm_bf16(g1, s));
+  GemmDesc g2 = gdesc(act, dff, w->w_down, dff, rows, dm, dff, EPI_F32, rows_out, dm);
+  g2.grouped = 1;
+  g2.offsets = offsets;
+  g2.num_groups = G;
+  g2.group_mod = E;
+  g2.b_rows = dm;
+  if (q8) {
+    g2.b_int8 = 1;
+    g2.scale_b = w->s_down;
+  }
+  return gemm_bf16(g2, s);
+}
+
+jamba_status jamba_moe_ep_combine(const jamba_moe_config* cfg, const float* rows_back, const float* topk_w,
+                                  int tokens, const void* residual, void* y, void* ws, size_t ws_bytes,
+                                  jamba_stream_t stream) {
+  JB_TRY(check_moe_cfg(cfg));
+  if (tokens <= 0) return fail(JAMBA_ERR_INVALID_ARG, "moe ep combine: tokens must be positive");
+  JB_TRY(check_ptr(rows_back, "rows_back"));
+  JB_TRY(check_ptr(topk_w, "topk_w"));
+  JB_TRY(check_ptr(residual, "residual", false));
+  JB_TRY(check_ptr(y, "y"));
+  JB_TRY(check_ptr(ws, "workspace"));
+  const jamba_moe_config& c = *cfg;
+  MoeWs m = carve_moe(c, tokens, ws);
+  if (ws_bytes < m.total) return fail(JAMBA_ERR_WORKSPACE, "moe ep combine: workspace too small");
+  return moe_combine(rows_back, m.inv, topk_w, tokens, c.top_k, c.d_model, residual, y, cs(stream));
+}
+
 }  // extern "C"
 
 // -------------------------------------------------------------- attention

@@ -107,11 +107,11 @@ static jamba_status gemm_i8w(const GemmDesc& g, cudaStream_t s) {
                      (uint64_t)g.lda * 2, 64, tok ? I8T_BNT : 128, CU_TENSOR_MAP_SWIZZLE_128B));
   const uint64_t rs = (uint64_t)g.ldb, os = rs * (uint64_t)g.b_rows;
   JB_TRY(make_map_3d(&mq, g.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)g.K, (uint64_t)g.b_rows,
-                     (uint64_t)g.num_groups, rs, os, q_inner, q_box, q_sw));
+                     (uint64_t)(g.group_mod > 0 ? g.group_mod : g.num_groups), rs, os, q_inner, q_box, q_sw));
   mq2 = mq;
   if (g.b2)
     JB_TRY(make_map_3d(&mq2, g.b2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)g.K, (uint64_t)g.b_rows,
-                       (uint64_t)g.num_groups, rs, os, q_inner, q_box, q_sw));
+                       (uint64_t)(g.group_mod > 0 ? g.group_mod : g.num_groups), rs, os, q_inner, q_box, q_sw));
   GemmParams p = {};
   p.M = g.M;
   p.N = g.N;
@@ -123,6 +123,7 @@ static jamba_status gemm_i8w(const GemmDesc& g, cudaStream_t s) {
   p.grouped = 1;
   p.offsets = g.offsets;
   p.num_groups = g.num_groups;
+  p.group_mod = g.group_mod;
   p.out = g.out;
   p.ldo = g.ldo;
   p.scale_b = g.scale_b;
@@ -187,10 +188,10 @@ jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
   } else {
     const uint64_t rs = (uint64_t)g.ldb * 2, os = rs * (uint64_t)g.b_rows;
     JB_TRY(make_map_3d(&mb, g.b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)g.K, (uint64_t)g.b_rows,
-                       (uint64_t)g.num_groups, rs, os, 64, (uint32_t)b_box, CU_TENSOR_MAP_SWIZZLE_128B));
+                       (uint64_t)(g.group_mod > 0 ? g.group_mod : g.num_groups), rs, os, 64, (uint32_t)b_box, CU_TENSOR_MAP_SWIZZLE_128B));
     if (g.b2) {
       JB_TRY(make_map_3d(&mb2, g.b2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)g.K, (uint64_t)g.b_rows,
-                         (uint64_t)g.num_groups, rs, os, 64, (uint32_t)b_box, CU_TENSOR_MAP_SWIZZLE_128B));
+                         (uint64_t)(g.group_mod > 0 ? g.group_mod : g.num_groups), rs, os, 64, (uint32_t)b_box, CU_TENSOR_MAP_SWIZZLE_128B));
     } else {
       mb2 = mb;
     }
@@ -201,7 +202,7 @@ jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
     JB_TRY(make_map_2d(&mc, g.out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)g.N, (uint64_t)g.M,
                        (uint64_t)g.ldo * 4, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B));
 
-  GemmParams p;
+  GemmParams p = {};
   p.M = g.M;
   p.N = g.N;
   p.K = g.K;
@@ -214,6 +215,7 @@ jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
   p.grouped = g.grouped;
   p.offsets = g.offsets;
   p.num_groups = g.num_groups;
+  p.group_mod = g.group_mod;
   p.out = g.out;
   p.ldo = g.ldo;
   p.split_stride = g.split_stride;

@@ -130,7 +130,7 @@ __device__ __forceinline__ void decode_tile_grouped(const GemmParams& p, int t, 
       ti.n0 = nb * BN_OUT;
       ti.kt0 = 0;
       ti.kt1 = p.k_tiles;
-      ti.group = g;
+      ti.group = p.group_mod > 0 ? g % p.group_mod : g;
       ti.split = 0;
       return;
     }
@@ -450,7 +450,7 @@ __device__ __forceinline__ void decode_tile_tok(const GemmParams& p, int t, Tile
       ti.n0 = wb * 128;
       ti.kt0 = 0;
       ti.kt1 = p.k_tiles;                   // 64-deep steps, an even number here
-      ti.group = g;
+      ti.group = p.group_mod > 0 ? g % p.group_mod : g;
       ti.split = 0;
       return;
     }

@@ -34,6 +34,7 @@ struct GemmParams {
   int grouped;           // A rows split by offsets[], B is [groups, rows, K]
   const int* offsets;
   int num_groups;
+  int group_mod;         // > 0: group g uses weight set g % group_mod (groups of rows from several ranks)
   void* out;
   long long ldo, split_stride;
   const void* residual;  // bf16, same layout as out (non-transposed only)
@@ -101,7 +102,7 @@ __device__ __forceinline__ void decode_tile(const GemmParams& p, int t, TileInfo
         ti.n0 = nb * BN_OUT;
         ti.kt0 = 0;
         ti.kt1 = p.k_tiles;
-        ti.group = g;
+        ti.group = p.group_mod > 0 ? g % p.group_mod : g;
         ti.split = 0;
         return;
       }

@@ -74,6 +74,7 @@ struct GemmDesc {
   int grouped;
   const int* offsets;
   int num_groups;
+  int group_mod;   // grouped: > 0 maps group g to weight set g % group_mod
   int epi;         // EpiKind
   int transpose_out;
   void* out;
@@ -176,6 +177,7 @@ jamba_status splitk_reduce(const float* part, int splits, long long split_stride
 jamba_status moe_route(const void* x, const void* W, int T, int dm, int E, int K, int* idx, float* w, int* counts,
                        int* offsets, int* perm, int* inv, cudaStream_t s);
 jamba_status moe_gather(const void* x, const int* perm, int rows, int K, int dm, void* out, cudaStream_t s);
+jamba_status group_offsets(const int* counts, int n, int* offsets, cudaStream_t s);   // exclusive prefix sum
 jamba_status quantize_int8_rows(const void* w, int dtype, long long rows, int cols, int8_t* q, float* scale,
                                 cudaStream_t s);
 jamba_status moe_combine(const float* Y, const int* inv, const float* w, int T, int K, int dm, const void* residual,

@@ -322,6 +322,24 @@ jamba_status moe_route(const void* x, const void* W, int T, int dm, int E, int K
   return JAMBA_OK;
 }
 
+// offsets[0] = 0, offsets[g + 1] = offsets[g] + counts[g] (one thread; n is small)
+__global__ void group_offsets_kernel(const int* __restrict__ counts, int n, int* __restrict__ offsets) {
+  if (threadIdx.x == 0 && blockIdx.x == 0) {
+    int acc = 0;
+    offsets[0] = 0;
+    for (int g = 0; g < n; ++g) {
+      acc += counts[g];
+      offsets[g + 1] = acc;
+    }
+  }
+}
+
+jamba_status group_offsets(const int* counts, int n, int* offsets, cudaStream_t s) {
+  group_offsets_kernel<<<1, 32, 0, s>>>(counts, n, offsets);
+  JB_CUDA(cudaGetLastError());
+  return JAMBA_OK;
+}
+
 jamba_status moe_gather(const void* x, const int* perm, int rows, int K, int dm, void* out, cudaStream_t s) {
   gather_rows_kernel<<<rows, 256, 0, s>>>(reinterpret_cast<const bf16*>(x), perm, K, dm, reinterpret_cast<bf16*>(out));
   JB_CUDA(cudaGetLastError());

@@ -129,3 +129,14 @@ def test_tensor_parallel_shards_cover_the_channels():
         assert torch.equal(torch.cat([s[n] for s in sh_], dim=1), p[n])
     for n in ("norm_dt", "norm_B", "norm_C"):
         assert all(torch.equal(s[n], p[n]) for s in sh_)
+
+
+def test_expert_parallel_shards_cover_the_experts():
+    import torch
+    from mamba_selective_scan_mixer_b200 import expert_parallel as ep
+    from synthetic import MoEShape, moe_params
+    p = moe_params(MoEShape(d_model=16, d_ff=8, n_experts=16, top_k=2), seed=0)
+    sh = [ep.shard_experts(p, r, 4) for r in range(4)]
+    for n in ("w_gate", "w_up", "w_down"):
+        assert torch.equal(torch.cat([s[n] for s in sh]), p[n])
+    assert all(torch.equal(s["router"], p["router"]) for s in sh)
