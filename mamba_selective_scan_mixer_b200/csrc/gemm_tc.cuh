@@ -230,22 +230,36 @@ __device__ __forceinline__ void epi_chunk(const GemmParams& p, const TileInfo& t
         const float w0 = __bfloat162float(wb[0]), w1 = __bfloat162float(wb[1]);
         const float w2 = __bfloat162float(wb[2]), w3 = __bfloat162float(wb[3]);
         const float bias = __bfloat162float(p.conv_b[m]);
+        // eight tokens at a time: their cache loads are all issued before any
+        // of the stores (which the compiler may not move the next loads past)
 #pragma unroll
-        for (int c = 0; c < NC; ++c) {
-          if (n + c < p.N) {
-            const long long bc = (long long)(n + c) * p.conv_c + m;
-            float* st = p.conv_state + bc * 3;
-            const float s0 = st[0], s1 = st[1], s2 = st[2];
-            const float xv = __bfloat162float(__float2bfloat16_rn(v[c]));   // x as the bf16 activation
-            float acc = bias;
-            acc = fmaf(w0, s0, acc);
-            acc = fmaf(w1, s1, acc);
-            acc = fmaf(w2, s2, acc);
-            acc = fmaf(w3, xv, acc);
-            p.xc_out[bc] = __float2bfloat16_rn(silu(acc));
-            st[0] = s1;
-            st[1] = s2;
-            st[2] = xv;
+        for (int c0 = 0; c0 < NC; c0 += 8) {
+          float sv[8][3];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            if (n + c0 + c < p.N) {
+              const float* st = p.conv_state + ((long long)(n + c0 + c) * p.conv_c + m) * 3;
+              sv[c][0] = st[0];
+              sv[c][1] = st[1];
+              sv[c][2] = st[2];
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            if (n + c0 + c < p.N) {
+              const long long bc = (long long)(n + c0 + c) * p.conv_c + m;
+              float* st = p.conv_state + bc * 3;
+              const float xv = __bfloat162float(__float2bfloat16_rn(v[c0 + c]));   // x as the bf16 activation
+              float acc = bias;
+              acc = fmaf(w0, sv[c][0], acc);
+              acc = fmaf(w1, sv[c][1], acc);
+              acc = fmaf(w2, sv[c][2], acc);
+              acc = fmaf(w3, xv, acc);
+              p.xc_out[bc] = __float2bfloat16_rn(silu(acc));
+              st[0] = sv[c][1];
+              st[1] = sv[c][2];
+              st[2] = xv;
+            }
           }
         }
       } else {
