@@ -683,20 +683,24 @@ __global__ void __launch_bounds__(256)
 ssm_step_kernel(const TX* __restrict__ xc, const TX* __restrict__ z, long long ld_z, const float* __restrict__ dt,
                 const float* __restrict__ bc, long long ld_bc, const float* __restrict__ A,
                 const float* __restrict__ D, float* __restrict__ state, TX* __restrict__ y, int batch, int di) {
-  griddep_wait();
-  griddep_launch();
   const long long i = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 2;   // flat (row, channel)
   const int q = threadIdx.x & 3;
   const bool live = i < (long long)batch * di;
   const long long ii = live ? i : 0;
   const int b = (int)(ii / di), c = (int)(ii - (long long)b * di);
+  // The cached state and A are not written by the kernels this one overlaps
+  // (the previous step's state update completed before the x_proj sum and
+  // norm of this step released its dependents), so their loads go out before
+  // the wait for dt, B, C and x.
+  const float4 av = __ldg(reinterpret_cast<const float4*>(A + (long long)c * NS + 4 * q));
+  float4* hs = reinterpret_cast<float4*>(state + ii * NS + 4 * q);
+  float4 h = *hs;
+  griddep_wait();
+  griddep_launch();
   const float x = to_f(xc[ii]);
   const float d = dt[ii];
   const float4 Bv = *reinterpret_cast<const float4*>(bc + (long long)b * ld_bc + 4 * q);
   const float4 Cv = *reinterpret_cast<const float4*>(bc + (long long)b * ld_bc + NS + 4 * q);
-  const float4 av = __ldg(reinterpret_cast<const float4*>(A + (long long)c * NS + 4 * q));
-  float4* hs = reinterpret_cast<float4*>(state + ii * NS + 4 * q);
-  float4 h = *hs;
   const float u = d * x;
   const float dl = d * LOG2E;
   h.x = fmaf(ex2(dl * av.x), h.x, u * Bv.x);
