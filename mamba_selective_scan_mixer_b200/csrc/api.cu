@@ -197,12 +197,12 @@ jamba_status reorder_channels(jamba_mamba* h) {
   std::vector<int> perm(di);
   std::iota(perm.begin(), perm.end(), 0);
   std::stable_sort(perm.begin(), perm.end(), [&](int a, int b) { return rate[a] < rate[b]; });
-  // steps until a group's slowest channel has decayed the carried state below 2^-40
+  // steps until a group's slowest channel has decayed the carried state below the scan's drop threshold (2^-32)
   const int groups = (di + SCAN_GROUP_CHANNELS - 1) / SCAN_GROUP_CHANNELS;
   h->head.assign(groups, 0.f);
   for (int g = 0; g < groups; ++g) {
     const double r = rate[perm[(size_t)g * SCAN_GROUP_CHANNELS]];
-    h->head[g] = r > 0.0 ? (float)std::min(40.0 * std::log(2.0) / r, 1e9) : 1e9f;
+    h->head[g] = r > 0.0 ? (float)std::min(32.0 * std::log(2.0) / r, 1e9) : 1e9f;
   }
 
   Carver cv(nullptr);

@@ -54,7 +54,7 @@ static jamba_status launch_i8t(const CUtensorMap& ma, const CUtensorMap& mq, con
                                  (int)S::BYTES));
     configured[dev] = true;
   }
-  JB_CUDA(launch_pdl(gemm_i8w_tok_kernel<EPI>, dim3(grid), dim3(I8T_THREADS), S::BYTES, s, ma, mq, mq2, p));
+  JB_CUDA(launch_pdl(gemm_i8w_tok_kernel<EPI>, dim3(grid), dim3(i8t_threads<EPI>()), S::BYTES, s, ma, mq, mq2, p));
   return JAMBA_OK;
 }
 

@@ -363,8 +363,11 @@ gemm_i8w_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 // SwiGLU holds the gate and up rows f in two accumulators.
 constexpr int I8T_BNT = 32;
 constexpr int I8T_EPI_WARPS = 4;   // one per TMEM lane quarter: a 32-token tile is one chunk
-constexpr int I8T_DQ_WARPS = 8;    // two per SM sub-partition
-constexpr int I8T_THREADS = 32 * (2 + I8T_EPI_WARPS + I8T_DQ_WARPS);
+// Dequantiser warps: two groups that widen alternate 64-deep halves of the
+// code stages, each group one warp per TMEM lane quarter per 128-row tile
+// (gate and up: two tiles).
+template <int EPI> constexpr int i8t_dq_warps() { return EPI == EPI_SWIGLU ? 16 : 8; }
+template <int EPI> constexpr int i8t_threads() { return 32 * (2 + I8T_EPI_WARPS + i8t_dq_warps<EPI>()); }
 
 // The widened weights never touch shared memory: the dequantiser warps write
 // them into tensor memory (tcgen05.st, one weight row per TMEM lane) and the
@@ -460,7 +463,7 @@ __device__ __forceinline__ void decode_tile_tok(const GemmParams& p, int t, Tile
 }
 
 template <int EPI>
-__global__ void __launch_bounds__(I8T_THREADS, 1)
+__global__ void __launch_bounds__(i8t_threads<EPI>(), 1)
 gemm_i8w_tok_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmQ,
                     const __grid_constant__ CUtensorMap tmQ2, const GemmParams p) {
   static_assert(EPI == EPI_SWIGLU || EPI == EPI_F32, "expert GEMMs only");
@@ -487,7 +490,7 @@ gemm_i8w_tok_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       mbar_init(empty0 + 8 * s, 1);
     }
     for (int s = 0; s < BST; ++s) {
-      mbar_init(bfull0 + 8 * s, I8T_DQ_WARPS);
+      mbar_init(bfull0 + 8 * s, i8t_dq_warps<EPI>() / 2);   // one group widens each half-stage
       mbar_init(bempty0 + 8 * s, 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -574,51 +577,55 @@ gemm_i8w_tok_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       mbar_wait(drain, 0, p.err);
     }
   } else if (warp >= 2 + I8T_EPI_WARPS) {
-    // Dequantiser warps, two per TMEM lane quarter q: thread `lane` widens row
-    // 32 q + lane of a 128-row weight tile.  SwiGLU: the warp pair splits the
-    // gate and up tiles; down: it splits the 64-deep step into two halves.
-    // Codes sit in 128-byte rows under the 128-byte swizzle (16-byte chunk c of
-    // row r at r * 128 + ((c ^ (r & 7)) << 4)): eight consecutive rows read
-    // eight distinct chunk positions, so a quarter-warp's loads are conflict-free.
-    const int q = warp & 3;
-    const int pi = (warp - 2 - I8T_EPI_WARPS) >> 2;   // which warp of the quarter's pair
-    const int r = q * 32 + lane;
+    // Dequantiser warps in two groups: group h widens the h-th 64-deep half of
+    // every code stage, so consecutive halves are widened concurrently.
+    // Within a group, warp w takes TMEM lane quarter q = w & 3 (thread `lane`
+    // widens row 32 q + lane of a 128-row weight tile; gate and up: the
+    // group's two warps of a quarter take one tile each) and stores the row's
+    // 64 widened codes with one tcgen05.st into its lane.  Codes sit in
+    // 128-byte rows under the 128-byte swizzle (16-byte chunk c of row r at
+    // r * 128 + ((c ^ (r & 7)) << 4)): eight consecutive rows read eight
+    // distinct chunk positions, so a quarter-warp's loads are conflict-free.
+    constexpr int DQ = i8t_dq_warps<EPI>();
     constexpr bool SW = EPI == EPI_SWIGLU;
-    const uint32_t row_off = (uint32_t)((SW ? pi * 128 : 0) + r) * 128;
+    const int d = warp - 2 - I8T_EPI_WARPS;           // 0 .. DQ-1
+    const int h = d / (DQ / 2);                         // which half this warp's group widens
+    const int tile = SW ? (d % (DQ / 2)) >> 2 : 0;      // gate (0) or up (1) tile
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const uint32_t row_off = (uint32_t)(tile * 128 + r) * 128;
     const uint32_t qbase = smem_u32(smem + S::X_BYTES) + row_off;
-    const uint32_t tl = tbase + ((uint32_t)(q * 32) << 16) + S::A_OFF + (SW ? pi * 32 : pi * 16);
-    int ts = 0, bs = 0;
-    uint32_t tph = 0, bph = 0;
+    const uint32_t tl = tbase + ((uint32_t)(q * 32) << 16) + S::A_OFF + tile * 32;
+    int ts = 0, k = h;                                  // k: this group's half-stages, 2 j + h
+    uint32_t tph = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
       TileInfo ti;
       decode_tile_tok(p, t, ti);
       for (int kt = ti.kt0; kt < ti.kt1 && ok; kt += 2) {
         if (!mbar_wait_warp(full0 + 8 * ts, tph, p.err)) { ok = false; break; }
+        const int bs = k % BST;
+        const uint32_t bph = (uint32_t)(k / BST) & 1u;
+        if (!mbar_wait_warp(bempty0 + 8 * bs, bph ^ 1, p.err)) { ok = false; break; }
+        tc_fence_after();
         const uint32_t qs = qbase + ts * S::T_STAGE;
-        for (int h = 0; h < 2; ++h) {
-          if (!mbar_wait_warp(bempty0 + 8 * bs, bph ^ 1, p.err)) { ok = false; break; }
-          tc_fence_after();
-          constexpr int NCH = SW ? 4 : 2;        // 16-byte code chunks this thread widens
-          uint32_t wv[2 * 4 * NCH];
+        uint32_t wv[32];
 #pragma unroll
-          for (int i = 0; i < NCH; ++i) {
-            const int c = 4 * h + (SW ? 0 : 2 * pi) + i;
-            uint4 v, lo, hi;
-            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(qs + ((c ^ (r & 7)) << 4)));
-            widen16(v, lo, hi);
-            wv[8 * i] = lo.x; wv[8 * i + 1] = lo.y; wv[8 * i + 2] = lo.z; wv[8 * i + 3] = lo.w;
-            wv[8 * i + 4] = hi.x; wv[8 * i + 5] = hi.y; wv[8 * i + 6] = hi.z; wv[8 * i + 7] = hi.w;
-          }
-          if constexpr (SW) tmem_st32u(tl + bs * S::A_COLS, wv);
-          else tmem_st16u(tl + bs * S::A_COLS, wv);
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bfull0 + 8 * bs);
-          if (++bs == BST) { bs = 0; bph ^= 1; }
+        for (int i = 0; i < 4; ++i) {
+          const int c = 4 * h + i;
+          uint4 v, lo, hi;
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(qs + ((c ^ (r & 7)) << 4)));
+          widen16(v, lo, hi);
+          wv[8 * i] = lo.x; wv[8 * i + 1] = lo.y; wv[8 * i + 2] = lo.z; wv[8 * i + 3] = lo.w;
+          wv[8 * i + 4] = hi.x; wv[8 * i + 5] = hi.y; wv[8 * i + 6] = hi.z; wv[8 * i + 7] = hi.w;
         }
+        tmem_st32u(tl + bs * S::A_COLS, wv);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bfull0 + 8 * bs);
+        k += 2;
         if (++ts == TST) { ts = 0; tph ^= 1; }
       }
     }

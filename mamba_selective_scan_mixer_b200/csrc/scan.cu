@@ -15,12 +15,12 @@
 // Chunks of the same channels run concurrently.  Before the state entering a
 // chunk is known, its outputs depend on it through C_t . (P_t * h_in), P_t the
 // decay product since the chunk start.  P_t only shrinks (A < 0), and once it
-// is at most 2^-40 for every state of every channel of a warp, h_in's share of
-// the warp's later states is at most 2^-40 |h_in| -- 2^16 times below the fp32
+// is at most 2^-32 for every state of every channel of a warp, h_in's share of
+// the warp's later states is at most 2^-32 |h_in| -- 2^8 times below the fp32
 // rounding unit -- and is dropped: the first pass runs the chunk's head (the
 // steps before that point) in state-only mode and writes final outputs after
 // it.  (Waiting for P_t to underflow to exact zero instead would lengthen the
-// head about fourfold: ln(2^-149) / ln(2^-40).)
+// head more than fourfold: ln(2^-149) / ln(2^-32).)
 // At the chunk end the CTA publishes (P, local end state) -- or its true end
 // state if every warp's P died -- and looks back over its predecessors'
 // records (decoupled look-back, (P2, h2) o (P1, h1) = (P2 P1, P2 h1 + h2)).
@@ -48,7 +48,7 @@ constexpr int SCAN_STAGES = 3;
 constexpr int NS = 16;                              // d_state
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr int REC = 3 * SCAN_CH * NS;               // floats per chunk record: P, h, inclusive h
-constexpr float CARRY_DROP = 0x1p-40f;              // decay product below which h_in's share is dropped
+constexpr float CARRY_DROP = 0x1p-32f;              // decay product below which h_in's share is dropped
 
 // CTA shape: CPT channels per consumer thread, 256 / (32 CPT) consumer warps,
 // one producer warp; MINB resident CTAs per SM (sets the register cap).
