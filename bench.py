@@ -268,7 +268,8 @@ def run_product(args):
                                   "d_state 16, dt_rank 256, inner RMSNorm, bf16 weights/activations, fp32 state" % L,
                       "global_batch": world, "seq_len": L, "parallelism": "replicas" if world > 1 else "single",
                       "l2": "512 MB buffer written before every timed step (outside the events)"},
-           "gpu_launches": None if ms is None else 8 * args.steps, "clocks": clk}
+           # per prefill step: in_proj, conv, x_proj, x_proj sum + norms, dt_proj, scan, out_proj
+           "gpu_launches": None if ms is None else 7 * args.steps, "clocks": clk}
 
     if rank == 0 and "gemm" in parts:
         # dominant kernel: in_proj GEMM on the tensor cores, same shape as inside the step
@@ -343,7 +344,9 @@ def run_product(args):
                          "tokens/s": round(B * NST / (dms / 1e3), 1), "us_per_step": round(per_step_us, 2),
                          "GB/s": round(step_bytes / (per_step_us / 1e6) / 1e9, 1),
                          "frac_of_measured_hbm": round(step_bytes / (per_step_us / 1e6) / 1e9 / pk["hbm"], 4),
-                         "algorithmic_bytes_per_step": step_bytes, "launches_per_step": 8}
+                         # in_proj (conv in its epilogue), x_proj, x_proj sum + norms, dt_proj, state update,
+                         # out_proj, split-K sum
+                         "algorithmic_bytes_per_step": step_bytes, "launches_per_step": 7}
         del graph, u0, steps_u
     if rank == 0 and "pair" in parts:
         # layer pair: RMSNorm -> Mamba -> residual -> RMSNorm -> top-2-of-16 MoE -> residual
