@@ -301,13 +301,18 @@ def run_product(args):
         scan_ws = torch.empty(nbytes.value, dtype=torch.uint8, device=dev)
         for _ in range(2):
             sc()
-        sms, _ = event_time_ms(sc, 5, stream, flush)
+        torch.cuda.synchronize()
+        sclocks = Clocks(dev)
+        sclocks.start()
+        sms, _ = event_time_ms(sc, 20, stream, flush)
+        torch.cuda.synchronize()
+        sclk = sclocks.stop()
         sbytes = SL * (SCAN_DI * (2 + 2 + 4 + 2) + 16 * 2 * 2)
         gbs = sbytes / (sms / 1e3) / 1e9
         # the arithmetic bound: 64 fp32 lane-ops per (token, channel) in the power
         # form (16 decay powers, 16 dt*x*B, 16 state FMAs, 16 C.h FMAs) against
-        # 128 fp32 lanes per SM per clock, at the clock seen in the prefill run
-        mhz = (clk or {}).get("sm_mhz") or 1965.0
+        # 128 fp32 lanes per SM per clock, at the clock seen while the scan ran
+        mhz = (sclk or clk or {}).get("sm_mhz") or 1965.0
         alu_ms = 1e3 * SL * SCAN_DI * 64 / (128 * torch.cuda.get_device_properties(dev).multi_processor_count
                                             * mhz * 1e6)
         res["scan"] = {"workload": "scan_128k: selective scan + D + SiLU(z) gate alone, batch 1, L=%d, "
@@ -315,7 +320,7 @@ def run_product(args):
                        "ms": round(sms, 4), "GB/s": round(gbs, 1), "frac_of_measured_hbm": round(gbs / pk["hbm"], 4),
                        "frac_of_8TBs": round(gbs / 8000.0, 4), "algorithmic_bytes": sbytes,
                        "alu_floor_ms": round(alu_ms, 4), "frac_of_fp32_pipe": round(alu_ms / sms, 4),
-                       "alu_clock_mhz": mhz, "tokens/s": round(SL / (sms / 1e3), 1)}
+                       "alu_clock_mhz": mhz, "clocks": sclk, "tokens/s": round(SL / (sms / 1e3), 1)}
         del s, y, scan_ws
     if rank == 0 and "decode" in parts:
         # decode: batch 64, caches from a 2048-token prefill, steps in one CUDA graph
