@@ -49,7 +49,9 @@ typedef enum jamba_status {
   JAMBA_ERR_WORKSPACE = 3,   /* workspace missing or smaller than *_workspace_size */
   JAMBA_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed                 */
   JAMBA_ERR_TIMEOUT = 5,     /* a device-side bounded wait gave up                */
-  JAMBA_ERR_OOM = 6          /* host allocation failed                            */
+  JAMBA_ERR_OOM = 6,         /* host allocation failed                            */
+  JAMBA_ERR_BOUNDS = 7       /* checked build: an index read from device data was
+                                out of range (the access was skipped)             */
 } jamba_status;
 
 typedef enum jamba_dtype { JAMBA_F32 = 0, JAMBA_BF16 = 1, JAMBA_INT8 = 2 } jamba_dtype;
@@ -59,9 +61,19 @@ typedef struct CUstream_st* jamba_stream_t; /* same type as cudaStream_t */
 /* Last error message of the calling thread (static storage, never NULL). */
 const char* jamba_last_error(void);
 
+/* 1 in the checked build of the library (libjamba_checked.so, compiled with
+ * -DJAMBA_CHECKS), 0 otherwise.  The checked build tests on the device every
+ * index that kernels read from device data before using it: routed-row
+ * positions (permutation and its inverse), expert group offsets, channel
+ * permutations of the reordered caches, cache lengths of the attention step.
+ * A failed test latches JAMBA_ERR_BOUNDS in the device error word and skips
+ * the access; nothing traps.  Group offsets are clamped into range in both
+ * builds. */
+int jamba_checked_build(void);
+
 /* Synchronizes `stream`, then returns and clears the device error word of the
- * current device: JAMBA_OK, JAMBA_ERR_TIMEOUT, or JAMBA_ERR_CUDA when the
- * stream itself reports an error.  The word latches: once a wait has given
+ * current device: JAMBA_OK, JAMBA_ERR_TIMEOUT, JAMBA_ERR_BOUNDS (checked build
+ * only), or JAMBA_ERR_CUDA when the stream itself reports an error.  The word latches: once a wait has given
  * up, later kernels that share the word stop early (writing nothing) until
  * this call clears it.  It also reads and clears the word that
  * jamba_selective_scan_static uses when called with status == NULL. */
@@ -128,7 +140,8 @@ jamba_status jamba_mamba_workspace_size(jamba_mamba_t h, int batch, int seqlen, 
  *   conv_state_out / ssm_state_out: same shapes, fp32 or NULL: the caches after
  *            the last token (conv: the last d_conv-1 pre-conv inputs, oldest first)
  *   ws / ws_bytes: device workspace of at least jamba_mamba_workspace_size bytes
- * The states may alias (in == out) for in-place continuation. */
+ * The states may alias (in == out) for in-place continuation; an aliased
+ * ssm state is copied to the workspace before the scan reads it. */
 jamba_status jamba_mamba_prefill(jamba_mamba_t h, const void* u, const void* residual, void* out,
                                  int batch, int seqlen, const float* conv_state_in,
                                  const float* ssm_state_in, float* conv_state_out,
@@ -276,11 +289,16 @@ jamba_status jamba_selective_scan_workspace_size(int batch, int seqlen, int d_in
  *   A      [d_inner, d_state] fp32, D [d_inner] fp32
  *   h0     [batch, d_inner, d_state] fp32 or NULL (zeros)
  *   y      [batch, seqlen, *] dtype, row stride ld_y (a multiple of 4)
- *   h_out  [batch, d_inner, d_state] fp32 or NULL: state after the last step
+ *   h_out  [batch, d_inner, d_state] fp32 or NULL: state after the last step;
+ *          may not overlap h0 (the first chunk's reads of h0 and the last
+ *          chunk's writes of h_out are not ordered)
  *   chunk  time steps per chunk (multiple of 16), 0 = automatic
  * Time is split into chunks scanned concurrently; the state entering each
- * chunk is passed between chunks with a decoupled look-back.  Errors:
- * UNSUPPORTED for d_state != 16, INVALID_ARG for strides/alignment. */
+ * chunk is passed between chunks with a decoupled look-back, which folds the
+ * carries in the order they become available: repeated calls agree up to
+ * that rounding order (last bits), not bit for bit.  Errors:
+ * UNSUPPORTED for d_state != 16, INVALID_ARG for strides/alignment or h_out
+ * overlapping h0. */
 jamba_status jamba_selective_scan(const void* x, int ld_x, const void* z, int ld_z, const float* dt,
                                   int ld_dt, const void* B, int ld_b, const void* C, int ld_c,
                                   int bc_dtype, const float* A, const float* D, const float* h0,

@@ -2,18 +2,22 @@
 
 Argument marshalling only: every step of the computation runs in the CUDA
 library.  Importing this module does not load the library; the first call
-does, and raises if libjamba.so has not been built.
+does, and raises if libjamba.so has not been built.  With JAMBA_CHECKED=1 in
+the environment the checked build (libjamba_checked.so: device-side index
+checks that report JAMBA_ERR_BOUNDS) is loaded instead.
 """
 import ctypes
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libjamba.so")
+CHECKED = os.environ.get("JAMBA_CHECKED", "0") == "1"
+LIB_PATH = os.path.join(HERE, "libjamba_checked.so" if CHECKED else "libjamba.so")
 
 JAMBA_OK = 0
 STATUS_NAMES = {0: "JAMBA_OK", 1: "JAMBA_ERR_INVALID_ARG", 2: "JAMBA_ERR_UNSUPPORTED",
                 3: "JAMBA_ERR_WORKSPACE", 4: "JAMBA_ERR_CUDA", 5: "JAMBA_ERR_TIMEOUT",
-                6: "JAMBA_ERR_OOM"}
+                6: "JAMBA_ERR_OOM", 7: "JAMBA_ERR_BOUNDS"}
+JAMBA_ERR_BOUNDS = 7
 JAMBA_F32 = 0
 JAMBA_BF16 = 1
 JAMBA_INT8 = 2
@@ -109,10 +113,13 @@ def lib():
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise ImportError("libjamba.so is not built (python -m mamba_selective_scan_mixer_b200.build)")
+            raise ImportError("%s is not built (python -m mamba_selective_scan_mixer_b200.build%s)"
+                              % (os.path.basename(LIB_PATH), " --checked" if CHECKED else ""))
         L = ctypes.CDLL(LIB_PATH)
         L.jamba_last_error.restype = ctypes.c_char_p
         L.jamba_last_error.argtypes = []
+        L.jamba_checked_build.restype = ctypes.c_int
+        L.jamba_checked_build.argtypes = []
         for name, args in SIGNATURES.items():
             f = getattr(L, name)
             f.restype = ctypes.c_int

@@ -62,6 +62,7 @@ struct PrefillWs {
   // context-parallel prefill only: in_proj rows of the 3 input tokens before
   // the slice, the conv cache they make, and the state entering the slice
   void* xz_halo; float* conv_halo; float* h_in;
+  float* h_tmp;         // the state entering the scan, when the caller's in and out states are one buffer
   ScanSchedule sched;   // the scan's per-group time chunks (n == 0: uniform chunks of `chunk`)
   size_t total;
 };
@@ -93,6 +94,7 @@ PrefillWs carve_prefill(const jamba_mamba* h, int batch, int L, void* ws, bool c
   p.dt = cv.take<float>(T * c.d_inner * 4);
   p.y = cv.take(T * c.d_inner * es);
   p.conv_tmp = cv.take<float>((size_t)batch * c.d_inner * (c.d_conv - 1) * 4);
+  p.h_tmp = cv.take<float>((size_t)batch * c.d_inner * c.d_state * 4);
   plan_scan(h, batch, L, &p.sched);
   if (h->perm) {
     // a per-group plan never exceeds the resident CTAs; sized for that bound
@@ -264,10 +266,13 @@ jamba_status prefill_front_a(const jamba_mamba& h, const PrefillWs& p, const voi
   const jamba_mamba_weights& w = prefill_weights(h);
   const int T = batch * seqlen, di = c.d_inner, dm = c.d_model, R = c.dt_rank, N = c.d_state;
   const int W = R + 2 * N;
+  NvtxSteps nv;
   // in_proj: xz = u W_in^T
+  nv.next("in_proj");
   JB_TRY(gemm_any(c.dtype, gdesc(u, dm, w.in_proj, dm, T, 2 * di, dm, c.dtype == JAMBA_BF16 ? EPI_BF16 : EPI_F32,
                                  p.xz, 2 * di), s));
   // conv + SiLU (cache in -> out; an aliased cache is copied first)
+  nv.next("conv1d");
   const float* cin = conv_state_in;
   if (cin && cin == conv_state_out) {
     JB_CUDA(cudaMemcpyAsync(p.conv_tmp, cin, sizeof(float) * (size_t)batch * di * 3, cudaMemcpyDeviceToDevice, s));
@@ -276,6 +281,7 @@ jamba_status prefill_front_a(const jamba_mamba& h, const PrefillWs& p, const voi
   JB_TRY(conv_prefill(p.xz, 2 * di, w.conv_w, w.conv_b, p.xc, cin, conv_state_out, batch, seqlen, di, c.dtype,
                       h.perm, s));
   // x_proj (split-K partials) -> sum + inner RMSNorms
+  nv.next("x_proj");
   GemmDesc gx = gdesc(p.xc, di, w.x_proj, di, T, W, di, EPI_F32, p.xpart, W);
   gx.splits = p.splits;
   gx.split_stride = (long long)T * W;
@@ -291,8 +297,11 @@ jamba_status prefill_front_b(const jamba_mamba& h, const PrefillWs& p, const flo
   const jamba_mamba_weights& w = prefill_weights(h);
   const int T = batch * seqlen, di = c.d_inner, R = c.dt_rank, N = c.d_state;
   const int W = R + 2 * N;
+  NvtxSteps nv;
+  nv.next("x_proj_sum_norms");
   JB_TRY(xproj_norm(part, splits, (long long)T * W, T, R, N, w.norm_dt, w.norm_B, w.norm_C, c.inner_rmsnorm, c.eps,
                     p.dtlow, p.bc, c.dtype, s));
+  nv.next("dt_proj_softplus");
   GemmDesc gd = gdesc(p.dtlow, R, w.dt_proj, R, T, di, R, EPI_SOFTPLUS, p.dt, di);
   gd.bias = w.dt_bias;
   return gemm_any(c.dtype, gd, s);
@@ -327,15 +336,34 @@ ScanCall scan_call(const jamba_mamba& h, const PrefillWs& p, int batch, int seql
   return sc;
 }
 
+// The state the scan starts from: the caller's, or a copy of it in the
+// workspace when it shares memory with the state the scan writes (in-place
+// continuation: the scan's first chunk reads the state while its last chunk
+// may already write it).
+jamba_status scan_state_in(const jamba_mamba& h, const PrefillWs& p, int batch, const float* in, const float* out,
+                           cudaStream_t s, const float** use) {
+  *use = in;
+  const size_t n = sizeof(float) * (size_t)batch * h.cfg.d_inner * h.cfg.d_state;
+  const uint8_t *a = reinterpret_cast<const uint8_t*>(in), *b = reinterpret_cast<const uint8_t*>(out);
+  if (a && b && a < b + n && b < a + n) {
+    JB_CUDA(cudaMemcpyAsync(p.h_tmp, in, n, cudaMemcpyDeviceToDevice, s));
+    *use = p.h_tmp;
+  }
+  return JAMBA_OK;
+}
+
 // The prefill from the scan on: selective scan + D skip + SiLU(z) gate, out_proj (+ residual).
 jamba_status prefill_back(const jamba_mamba& h, const PrefillWs& p, int batch, int seqlen, const float* ssm_state_in,
                           float* ssm_state_out, const void* residual, void* out, cudaStream_t s) {
   const jamba_mamba_config& c = h.cfg;
   const int T = batch * seqlen, di = c.d_inner, dm = c.d_model;
+  NvtxSteps nv;
+  nv.next("selective_scan");
   ScanCall sc = scan_call(h, p, batch, seqlen);
-  sc.h0 = ssm_state_in;
+  JB_TRY(scan_state_in(h, p, batch, ssm_state_in, ssm_state_out, s, &sc.h0));
   sc.h_out = ssm_state_out;
   JB_TRY(scan_run(sc, s));
+  nv.next("out_proj");
   GemmDesc go = gdesc(p.y, di, prefill_weights(h).out_proj, di, T, dm, di, c.dtype == JAMBA_BF16 ? EPI_BF16 : EPI_F32, out, dm);
   go.residual = residual;
   go.ldr = dm;
@@ -347,6 +375,14 @@ jamba_status prefill_back(const jamba_mamba& h, const PrefillWs& p, int batch, i
 extern "C" {
 
 const char* jamba_last_error(void) { return jb::last_error(); }
+
+int jamba_checked_build(void) {
+#ifdef JAMBA_CHECKS
+  return 1;
+#else
+  return 0;
+#endif
+}
 
 jamba_status jamba_device_status(jamba_stream_t stream) {
   JB_CUDA(cudaStreamSynchronize(cs(stream)));
@@ -365,6 +401,7 @@ jamba_status jamba_device_status(jamba_stream_t stream) {
 // ------------------------------------------------------------------ Mamba
 
 jamba_status jamba_mamba_create(const jamba_mamba_config* cfg, const jamba_mamba_weights* w, jamba_mamba_t* out) {
+  JB_RANGE("jamba_mamba_create");
   if (!cfg || !w || !out) return fail(JAMBA_ERR_INVALID_ARG, "create: null argument");
   *out = nullptr;
   const jamba_mamba_config& c = *cfg;
@@ -454,6 +491,7 @@ jamba_status jamba_mamba_prefill(jamba_mamba_t h, const void* u, const void* res
                                  int seqlen, const float* conv_state_in, const float* ssm_state_in,
                                  float* conv_state_out, float* ssm_state_out, void* ws, size_t ws_bytes,
                                  jamba_stream_t stream) {
+  JB_RANGE("jamba_mamba_prefill");
   if (!h) return fail(JAMBA_ERR_INVALID_ARG, "prefill: null handle");
   if (batch <= 0 || seqlen <= 0) return fail(JAMBA_ERR_INVALID_ARG, "prefill: batch and seqlen must be positive");
   JB_TRY(check_device(h));
@@ -480,6 +518,7 @@ jamba_status jamba_mamba_prefill(jamba_mamba_t h, const void* u, const void* res
 jamba_status jamba_mamba_prefill_tp_begin(jamba_mamba_t h, const void* u, int batch, int seqlen,
                                           const float* conv_state_in, float* conv_state_out, float* xproj_part,
                                           void* ws, size_t ws_bytes, jamba_stream_t stream) {
+  JB_RANGE("jamba_mamba_prefill_tp_begin");
   if (!h) return fail(JAMBA_ERR_INVALID_ARG, "tp begin: null handle");
   if (batch <= 0 || seqlen <= 0) return fail(JAMBA_ERR_INVALID_ARG, "tp begin: batch and seqlen must be positive");
   JB_TRY(check_device(h));
@@ -502,6 +541,7 @@ jamba_status jamba_mamba_prefill_tp_begin(jamba_mamba_t h, const void* u, int ba
 jamba_status jamba_mamba_prefill_tp_finish(jamba_mamba_t h, const float* xproj_sum, int batch, int seqlen,
                                            const float* ssm_state_in, float* ssm_state_out, float* out_part,
                                            void* ws, size_t ws_bytes, jamba_stream_t stream) {
+  JB_RANGE("jamba_mamba_prefill_tp_finish");
   if (!h) return fail(JAMBA_ERR_INVALID_ARG, "tp finish: null handle");
   if (batch <= 0 || seqlen <= 0) return fail(JAMBA_ERR_INVALID_ARG, "tp finish: batch and seqlen must be positive");
   JB_TRY(check_device(h));
@@ -517,7 +557,7 @@ jamba_status jamba_mamba_prefill_tp_finish(jamba_mamba_t h, const float* xproj_s
   const int T = batch * seqlen, di = c.d_inner, dm = c.d_model;
   JB_TRY(prefill_front_b(*h, p, xproj_sum, 1, batch, seqlen, s));
   ScanCall sc = scan_call(*h, p, batch, seqlen);
-  sc.h0 = ssm_state_in;
+  JB_TRY(scan_state_in(*h, p, batch, ssm_state_in, ssm_state_out, s, &sc.h0));
   sc.h_out = ssm_state_out;
   JB_TRY(scan_run(sc, s));
   // this rank's share of out_proj (its d_inner columns), fp32
@@ -527,6 +567,7 @@ jamba_status jamba_mamba_prefill_tp_finish(jamba_mamba_t h, const float* xproj_s
 
 jamba_status jamba_mamba_prefill_tp_end(jamba_mamba_t h, const float* out_sum, const void* residual, void* out,
                                         int batch, int seqlen, jamba_stream_t stream) {
+  JB_RANGE("jamba_mamba_prefill_tp_end");
   if (!h) return fail(JAMBA_ERR_INVALID_ARG, "tp end: null handle");
   if (batch <= 0 || seqlen <= 0) return fail(JAMBA_ERR_INVALID_ARG, "tp end: batch and seqlen must be positive");
   JB_TRY(check_device(h));
@@ -549,6 +590,7 @@ jamba_status jamba_mamba_prefill_cp_begin(jamba_mamba_t h, const void* u, const 
                                           const float* conv_state_in, const float* ssm_state_in,
                                           float* conv_state_out, float* carry_p, float* carry_h, void* ws,
                                           size_t ws_bytes, jamba_stream_t stream) {
+  JB_RANGE("jamba_mamba_prefill_cp_begin");
   if (!h) return fail(JAMBA_ERR_INVALID_ARG, "cp begin: null handle");
   if (batch <= 0 || seqlen <= 0) return fail(JAMBA_ERR_INVALID_ARG, "cp begin: batch and seqlen must be positive");
   JB_TRY(check_device(h));
@@ -595,6 +637,7 @@ jamba_status jamba_mamba_prefill_cp_finish(jamba_mamba_t h, const void* residual
                                            int rank, const float* carries_p, const float* carries_h,
                                            const float* ssm_state_in, float* ssm_state_out, void* ws, size_t ws_bytes,
                                            jamba_stream_t stream) {
+  JB_RANGE("jamba_mamba_prefill_cp_finish");
   if (!h) return fail(JAMBA_ERR_INVALID_ARG, "cp finish: null handle");
   if (batch <= 0 || seqlen <= 0 || rank < 0) return fail(JAMBA_ERR_INVALID_ARG, "cp finish: bad sizes or rank");
   JB_TRY(check_device(h));
@@ -617,6 +660,7 @@ jamba_status jamba_mamba_prefill_cp_finish(jamba_mamba_t h, const void* residual
 
 jamba_status jamba_mamba_step(jamba_mamba_t h, const void* u, const void* residual, void* out, int batch,
                               float* conv_state, float* ssm_state, void* ws, size_t ws_bytes, jamba_stream_t stream) {
+  JB_RANGE("jamba_mamba_step");
   if (!h) return fail(JAMBA_ERR_INVALID_ARG, "step: null handle");
   if (batch <= 0) return fail(JAMBA_ERR_INVALID_ARG, "step: batch must be positive");
   JB_TRY(check_device(h));
@@ -633,9 +677,11 @@ jamba_status jamba_mamba_step(jamba_mamba_t h, const void* u, const void* residu
   if (ws_bytes < p.total) return fail(JAMBA_ERR_WORKSPACE, "step: workspace too small");
   cudaStream_t s = cs(stream);
   const int di = c.d_inner, dm = c.d_model, R = c.dt_rank, N = c.d_state, W = R + 2 * N;
+  NvtxSteps nv;
   if (c.dtype == JAMBA_BF16) {
     // weights stream through the tensor cores as the 128-row side; the token batch is the N side
     // in_proj with the conv step in its epilogue: x rows -> conv cache shift + SiLU -> xc, z rows -> xz
+    nv.next("in_proj_conv");
     GemmDesc g1 = gdesc(w.in_proj, dm, u, dm, 2 * di, batch, dm, EPI_CONV, p.xz, 2 * di);
     g1.transpose_out = 1;
     g1.bn = 64;
@@ -645,21 +691,26 @@ jamba_status jamba_mamba_step(jamba_mamba_t h, const void* u, const void* residu
     g1.xc_out = p.xc;
     g1.conv_c = di;
     JB_TRY(gemm_bf16(g1, s));
+    nv.next("x_proj");
     GemmDesc g2 = gdesc(w.x_proj, di, p.xc, di, W, batch, di, EPI_F32, p.xpart, W);
     g2.transpose_out = 1;
     g2.bn = 64;
     g2.splits = p.x_splits;
     g2.split_stride = (long long)batch * W;
     JB_TRY(gemm_bf16(g2, s));
+    nv.next("x_proj_sum_norms");
     JB_TRY(xproj_norm(p.xpart, p.x_splits, (long long)batch * W, batch, R, N, w.norm_dt, w.norm_B, w.norm_C,
                       c.inner_rmsnorm, c.eps, p.dtlow, p.bc, c.dtype, s));
+    nv.next("dt_proj_softplus");
     GemmDesc g3 = gdesc(w.dt_proj, R, p.dtlow, R, di, batch, R, EPI_SOFTPLUS, p.dt, di);
     g3.transpose_out = 1;
     g3.bn = 64;
     g3.bias = w.dt_bias;
     JB_TRY(gemm_bf16(g3, s));
+    nv.next("state_update");
     JB_TRY(ssm_step(p.xc, reinterpret_cast<const uint8_t*>(p.xz) + (size_t)di * 2, 2 * di, p.dt, p.bc, 2 * N, w.A,
                     w.D, ssm_state, p.y, batch, di, c.dtype, s));
+    nv.next("out_proj");
     GemmDesc g4 = gdesc(w.out_proj, di, p.y, di, dm, batch, di, EPI_F32, p.opart, dm);
     g4.transpose_out = 1;
     g4.bn = 64;
@@ -742,6 +793,7 @@ jamba_status jamba_mamba_prefill_host(jamba_mamba_t h, const void* u_host, const
                                       int batch, int seqlen, int chunk, const float* conv_state_in,
                                       const float* ssm_state_in, float* conv_state_out, float* ssm_state_out,
                                       void* ws, size_t ws_bytes, jamba_stream_t stream) {
+  JB_RANGE("jamba_mamba_prefill_host");
   if (!h) return fail(JAMBA_ERR_INVALID_ARG, "prefill_host: null handle");
   if (batch <= 0 || seqlen <= 0 || chunk < 0)
     return fail(JAMBA_ERR_INVALID_ARG, "prefill_host: batch and seqlen must be positive, chunk >= 0");
@@ -846,6 +898,7 @@ jamba_status jamba_selective_scan(const void* x, int ld_x, const void* z, int ld
                                   const float* D, const float* h0, void* y, int ld_y, float* h_out, int batch,
                                   int seqlen, int d_inner, int d_state, int dtype, int chunk, void* ws,
                                   size_t ws_bytes, jamba_stream_t stream) {
+  JB_RANGE("jamba_selective_scan");
   JB_TRY(check_dtype(dtype));
   JB_TRY(check_dtype(bc_dtype));
   if (d_state != 16) return fail(JAMBA_ERR_UNSUPPORTED, "d_state must be 16");
@@ -876,6 +929,7 @@ jamba_status jamba_test_scan_missing_predecessor(const void* x, int ld_x, const 
                                                  float* h_out, int batch, int seqlen, int d_inner, int d_state,
                                                  int dtype, int chunk, unsigned long long wait_ns, void* ws,
                                                  size_t ws_bytes, jamba_stream_t stream) {
+  JB_RANGE("jamba_test_scan_missing_predecessor");
   JB_TRY(check_dtype(dtype));
   JB_TRY(check_dtype(bc_dtype));
   if (d_state != 16) return fail(JAMBA_ERR_UNSUPPORTED, "d_state must be 16");
@@ -905,6 +959,7 @@ jamba_status jamba_test_scan_missing_predecessor(const void* x, int ld_x, const 
 
 jamba_status jamba_rmsnorm(const void* x, const float* w, void* out, int rows, int cols, float eps, int dtype,
                            jamba_stream_t stream) {
+  JB_RANGE("jamba_rmsnorm");
   JB_TRY(check_dtype(dtype));
   if (rows <= 0 || cols <= 0) return fail(JAMBA_ERR_INVALID_ARG, "rmsnorm: sizes must be positive");
   JB_TRY(check_ptr(x, "x"));
@@ -916,6 +971,7 @@ jamba_status jamba_rmsnorm(const void* x, const float* w, void* out, int rows, i
 jamba_status jamba_causal_conv1d(const void* x, int ld_x, const void* w, const void* b, void* out,
                                  const float* state_in, float* state_out, int batch, int seqlen, int channels,
                                  int dtype, jamba_stream_t stream) {
+  JB_RANGE("jamba_causal_conv1d");
   JB_TRY(check_dtype(dtype));
   if (batch <= 0 || seqlen <= 0 || channels <= 0 || ld_x < channels)
     return fail(JAMBA_ERR_INVALID_ARG, "conv: bad sizes");
@@ -930,6 +986,7 @@ jamba_status jamba_causal_conv1d(const void* x, int ld_x, const void* w, const v
 
 jamba_status jamba_gemm(const void* a, const void* b, void* out, int ld_out, const void* residual, int m, int n,
                         int k, int dtype, int out_dtype, jamba_stream_t stream) {
+  JB_RANGE("jamba_gemm");
   JB_TRY(check_dtype(dtype));
   JB_TRY(check_dtype(out_dtype));
   if (m <= 0 || n <= 0 || k <= 0 || ld_out < n) return fail(JAMBA_ERR_INVALID_ARG, "gemm: bad sizes");
@@ -946,17 +1003,19 @@ jamba_status jamba_gemm(const void* a, const void* b, void* out, int ld_out, con
 namespace {
 struct MoeWs {
   int* counts; int* inv; void* xperm; void* act; float* Y;
+  int y_splits;   // k-split partial outputs of the down GEMM held in Y
   size_t total;
 };
 MoeWs carve_moe(const jamba_moe_config& c, int T, void* ws) {
   MoeWs m;
   const size_t rows = (size_t)T * c.top_k;
+  m.y_splits = c.expert_dtype == JAMBA_INT8 ? i8w_splits((int)rows, c.n_experts, c.d_model, c.d_ff) : 1;
   Carver cv(ws);
   m.counts = cv.take<int>(sizeof(int) * 64);
   m.inv = cv.take<int>(sizeof(int) * rows);
   m.xperm = cv.take(rows * c.d_model * 2);
   m.act = cv.take(rows * c.d_ff * 2);
-  m.Y = cv.take<float>(rows * c.d_model * 4);
+  m.Y = cv.take<float>(rows * c.d_model * 4 * m.y_splits);
   m.total = cv.off;
   return m;
 }
@@ -975,6 +1034,7 @@ jamba_status check_moe_cfg(const jamba_moe_config* c) {
 
 jamba_status jamba_quantize_int8_rows(const void* w, int dtype, long long rows, int cols, int8_t* q, float* scale,
                                       jamba_stream_t stream) {
+  JB_RANGE("jamba_quantize_int8_rows");
   JB_TRY(check_dtype(dtype));
   if (rows <= 0 || cols <= 0 || cols % 8) return fail(JAMBA_ERR_INVALID_ARG, "quantize: rows > 0, cols a positive multiple of 8");
   JB_TRY(check_ptr(w, "w"));
@@ -994,6 +1054,7 @@ jamba_status jamba_moe_forward(const jamba_moe_config* cfg, const jamba_moe_weig
                                const void* residual, void* y, int tokens, int32_t* topk_idx, float* topk_w,
                                int32_t* expert_offsets, int32_t* perm, void* ws, size_t ws_bytes,
                                jamba_stream_t stream) {
+  JB_RANGE("jamba_moe_forward");
   JB_TRY(check_moe_cfg(cfg));
   if (!w || tokens <= 0) return fail(JAMBA_ERR_INVALID_ARG, "moe: bad argument");
   JB_TRY(check_ptr(w->router, "router"));
@@ -1018,8 +1079,12 @@ jamba_status jamba_moe_forward(const jamba_moe_config* cfg, const jamba_moe_weig
   cudaStream_t s = cs(stream);
   const int E = c.n_experts, K = c.top_k, dm = c.d_model, dff = c.d_ff;
   const int rows = tokens * K;
+  NvtxSteps nv;
+  nv.next("router_top_k");
   JB_TRY(moe_route(x, w->router, tokens, dm, E, K, topk_idx, topk_w, m.counts, expert_offsets, perm, m.inv, s));
+  nv.next("gather");
   JB_TRY(moe_gather(x, perm, rows, K, dm, m.xperm, s));
+  nv.next("experts_gate_up_swiglu");
   // gate | up with SwiGLU: act = SiLU(x W_g^T) * (x W_u^T), per expert
   GemmDesc g1 = gdesc(m.xperm, dm, w->w_gate, dm, rows, dff, dm, EPI_SWIGLU, m.act, dff);
   g1.b2 = w->w_up;
@@ -1034,6 +1099,7 @@ jamba_status jamba_moe_forward(const jamba_moe_config* cfg, const jamba_moe_weig
   }
   JB_TRY(gemm_bf16(g1, s));
   // down: Y = act W_d^T, fp32 rows in routed order
+  nv.next("experts_down");
   GemmDesc g2 = gdesc(m.act, dff, w->w_down, dff, rows, dm, dff, EPI_F32, m.Y, dm);
   g2.grouped = 1;
   g2.offsets = expert_offsets;
@@ -1042,9 +1108,12 @@ jamba_status jamba_moe_forward(const jamba_moe_config* cfg, const jamba_moe_weig
   if (q8) {
     g2.b_int8 = 1;
     g2.scale_b = w->s_down;
+    g2.splits = m.y_splits;   // decode batches: k-split partials, summed by the combine
+    g2.split_stride = (long long)rows * dm;
   }
   JB_TRY(gemm_bf16(g2, s));
-  JB_TRY(moe_combine(m.Y, m.inv, topk_w, tokens, K, dm, residual, y, s));
+  nv.next("combine");
+  JB_TRY(moe_combine(m.Y, m.y_splits, (long long)rows * dm, m.inv, topk_w, tokens, K, dm, residual, y, s));
   return JAMBA_OK;
 }
 
@@ -1053,6 +1122,7 @@ jamba_status jamba_moe_forward(const jamba_moe_config* cfg, const jamba_moe_weig
 jamba_status jamba_moe_ep_dispatch(const jamba_moe_config* cfg, const void* router, const void* x, int tokens,
                                    int32_t* topk_idx, float* topk_w, int32_t* expert_offsets, int32_t* perm,
                                    void* send_rows, void* ws, size_t ws_bytes, jamba_stream_t stream) {
+  JB_RANGE("jamba_moe_ep_dispatch");
   JB_TRY(check_moe_cfg(cfg));
   if (tokens <= 0) return fail(JAMBA_ERR_INVALID_ARG, "moe ep dispatch: tokens must be positive");
   JB_TRY(check_ptr(router, "router"));
@@ -1082,6 +1152,7 @@ jamba_status jamba_moe_ep_experts_workspace_size(const jamba_moe_config* cfg, in
 jamba_status jamba_moe_ep_experts(const jamba_moe_config* cfg, const jamba_moe_weights* w, const void* rows_in,
                                   int rows, const int32_t* group_counts, int world, float* rows_out, void* ws,
                                   size_t ws_bytes, jamba_stream_t stream) {
+  JB_RANGE("jamba_moe_ep_experts");
   JB_TRY(check_moe_cfg(cfg));
   if (!w || rows < 0 || world <= 0 || world * cfg->n_experts > 4096)
     return fail(JAMBA_ERR_INVALID_ARG, "moe ep experts: bad argument");
@@ -1137,6 +1208,7 @@ jamba_status jamba_moe_ep_experts(const jamba_moe_config* cfg, const jamba_moe_w
 jamba_status jamba_moe_ep_combine(const jamba_moe_config* cfg, const float* rows_back, const float* topk_w,
                                   int tokens, const void* residual, void* y, void* ws, size_t ws_bytes,
                                   jamba_stream_t stream) {
+  JB_RANGE("jamba_moe_ep_combine");
   JB_TRY(check_moe_cfg(cfg));
   if (tokens <= 0) return fail(JAMBA_ERR_INVALID_ARG, "moe ep combine: tokens must be positive");
   JB_TRY(check_ptr(rows_back, "rows_back"));
@@ -1147,7 +1219,7 @@ jamba_status jamba_moe_ep_combine(const jamba_moe_config* cfg, const float* rows
   const jamba_moe_config& c = *cfg;
   MoeWs m = carve_moe(c, tokens, ws);
   if (ws_bytes < m.total) return fail(JAMBA_ERR_WORKSPACE, "moe ep combine: workspace too small");
-  return moe_combine(rows_back, m.inv, topk_w, tokens, c.top_k, c.d_model, residual, y, cs(stream));
+  return moe_combine(rows_back, 1, 0, m.inv, topk_w, tokens, c.top_k, c.d_model, residual, y, cs(stream));
 }
 
 }  // extern "C"
@@ -1213,6 +1285,7 @@ jamba_status jamba_attn_prefill_workspace_size(const jamba_attn_config* cfg, int
 jamba_status jamba_attn_prefill(const jamba_attn_config* cfg, const jamba_attn_weights* w, const void* x,
                                 const void* residual, void* out, int batch, int seqlen, void* k_cache,
                                 void* v_cache, int max_len, void* ws, size_t ws_bytes, jamba_stream_t stream) {
+  JB_RANGE("jamba_attn_prefill");
   JB_TRY(check_attn_cfg(cfg));
   if (!w || batch <= 0 || seqlen <= 0) return fail(JAMBA_ERR_INVALID_ARG, "attention prefill: bad argument");
   JB_TRY(check_ptr(w->w_qkv, "w_qkv"));
@@ -1253,6 +1326,7 @@ jamba_status jamba_attn_step_workspace_size(const jamba_attn_config* cfg, int ba
 jamba_status jamba_attn_step(const jamba_attn_config* cfg, const jamba_attn_weights* w, const void* x,
                              const void* residual, void* out, int batch, void* k_cache, void* v_cache,
                              int max_len, int32_t* lengths, void* ws, size_t ws_bytes, jamba_stream_t stream) {
+  JB_RANGE("jamba_attn_step");
   JB_TRY(check_attn_cfg(cfg));
   if (!w || batch <= 0 || max_len <= 0) return fail(JAMBA_ERR_INVALID_ARG, "attention step: bad argument");
   JB_TRY(check_ptr(w->w_qkv, "w_qkv"));

@@ -663,12 +663,13 @@ jamba_status attn_prefill_core(const void* qkv, void* vt, long long ldv, void* o
 // qkv [B, W]: k and v of the new token into the caches at position lengths[b]
 __global__ void __launch_bounds__(256)
 kv_append_kernel(const bf16* __restrict__ qkv, int H, int G, const int* __restrict__ lengths, bf16* __restrict__ kc,
-                 bf16* __restrict__ vc, int max_len) {
+                 bf16* __restrict__ vc, int max_len, int* err) {
   griddep_wait();
   griddep_launch();
   const int b = blockIdx.x;
   const int pos = lengths[b];
-  if (pos < 0 || pos >= max_len) return;   // out-of-range lengths append nothing
+  // out-of-range lengths append nothing (and are reported by the checked build)
+  if (!checked(pos >= 0 && pos < max_len, err) || pos < 0 || pos >= max_len) return;
   const long long W = (long long)(H + 2 * G) * ATT_D;
   for (int i = threadIdx.x; i < G * 16; i += 256) {
     const int g = i >> 4, ch = i & 15;
@@ -918,7 +919,7 @@ jamba_status attn_decode_core(const void* qkv, void* k_cache, void* v_cache, int
   if (H / G > DEC_REP) return fail(JAMBA_ERR_UNSUPPORTED, "attention step: at most 8 query heads per KV head");
   JB_CUDA(launch_pdl(kv_append_kernel, dim3(B), dim3(256), 0, s, reinterpret_cast<const bf16*>(qkv), H, G,
                      (const int*)lengths, reinterpret_cast<bf16*>(k_cache), reinterpret_cast<bf16*>(v_cache),
-                     max_len));
+                     max_len, device_error_word()));
   const float sl2 = 1.4426950408889634f / sqrtf((float)ATT_D);
   static std::atomic<bool> configured[64];
   int dev = 0;

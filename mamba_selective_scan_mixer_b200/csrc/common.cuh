@@ -33,6 +33,18 @@ __device__ __forceinline__ void set_error(int* err, int code) {
   if (err) atomicCAS(err, 0, code);
 }
 
+// Checked build (-DJAMBA_CHECKS): `checked(ok, err)` guards an access through
+// an index read from device data; when !ok it latches JAMBA_ERR_BOUNDS and the
+// caller skips the access.  In the normal build it is the constant true.
+#ifdef JAMBA_CHECKS
+__device__ __forceinline__ bool checked(bool ok, int* err) {
+  if (!ok) set_error(err, JAMBA_ERR_BOUNDS);
+  return ok;
+}
+#else
+__device__ __forceinline__ bool checked(bool, int*) { return true; }
+#endif
+
 __device__ __forceinline__ bool error_raised(const int* err) {
   return err && *(volatile const int*)err != 0;
 }

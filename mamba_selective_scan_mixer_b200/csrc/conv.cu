@@ -55,7 +55,7 @@ template <typename T>
 __global__ void __launch_bounds__(CONV_THREADS)
 conv_prefill_kernel(const T* __restrict__ x, long long ld_x, const T* __restrict__ w, const T* __restrict__ bias,
                     T* __restrict__ out, const float* __restrict__ st_in, float* __restrict__ st_out, int L,
-                    int C, const int* __restrict__ perm) {
+                    int C, const int* __restrict__ perm, int* err) {
   constexpr int V = Vec16<T>::N;
   griddep_wait();
   griddep_launch();
@@ -82,7 +82,7 @@ conv_prefill_kernel(const T* __restrict__ x, long long ld_x, const T* __restrict
 #pragma unroll
       for (int i = 0; i < V; ++i) {
         const int cn = perm ? __ldg(perm + c0 + i) : c0 + i;   // cache row of this channel
-        win[k][i] = st_in ? st_in[((long long)b * C + cn) * 3 + (3 + t)] : 0.f;
+        win[k][i] = st_in && checked(cn >= 0 && cn < C, err) ? st_in[((long long)b * C + cn) * 3 + (3 + t)] : 0.f;
       }
     }
   }
@@ -118,6 +118,7 @@ conv_prefill_kernel(const T* __restrict__ x, long long ld_x, const T* __restrict
 #pragma unroll
     for (int i = 0; i < V; ++i) {
       const int cn = perm ? __ldg(perm + c0 + i) : c0 + i;
+      if (!checked(cn >= 0 && cn < C, err)) continue;
 #pragma unroll
       for (int k = 0; k < 3; ++k) st_out[((long long)b * C + cn) * 3 + k] = win[k][i];
     }
@@ -183,11 +184,11 @@ jamba_status conv_prefill(const void* x, long long ld_x, const void* w, const vo
   if (dtype == JAMBA_BF16)
     JB_CUDA(launch_pdl(conv_prefill_kernel<bf16>, grid, dim3(CONV_THREADS), 0, s, reinterpret_cast<const bf16*>(x),
                        ld_x, reinterpret_cast<const bf16*>(w), reinterpret_cast<const bf16*>(b),
-                       reinterpret_cast<bf16*>(out), st_in, st_out, L, C, perm));
+                       reinterpret_cast<bf16*>(out), st_in, st_out, L, C, perm, device_error_word()));
   else
     JB_CUDA(launch_pdl(conv_prefill_kernel<float>, grid, dim3(CONV_THREADS), 0, s, reinterpret_cast<const float*>(x),
                        ld_x, reinterpret_cast<const float*>(w), reinterpret_cast<const float*>(b),
-                       reinterpret_cast<float*>(out), st_in, st_out, L, C, perm));
+                       reinterpret_cast<float*>(out), st_in, st_out, L, C, perm, device_error_word()));
   return JAMBA_OK;
 }
 
@@ -211,12 +212,14 @@ jamba_status conv_step(const void* x, long long ld_x, const void* w, const void*
 // else 2-byte elements (row_bytes is even for every weight reordered here).
 __global__ void __launch_bounds__(256)
 gather_rows_kernel(const uint8_t* __restrict__ src, uint8_t* __restrict__ dst, const int* __restrict__ perm,
-                   int rows, int row_bytes, int word) {
+                   int rows, int row_bytes, int word, int* err) {
   const int per_row = row_bytes / word;
   const long long n = (long long)rows * per_row;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
     const int r = (int)(i / per_row), e = (int)(i - (long long)r * per_row);
-    const long long so = (long long)__ldg(perm + r) * row_bytes + (long long)e * word;
+    const int pr = __ldg(perm + r);
+    if (!checked(pr >= 0 && pr < rows, err)) continue;
+    const long long so = (long long)pr * row_bytes + (long long)e * word;
     const long long d = (long long)r * row_bytes + (long long)e * word;
     if (word == 16) *reinterpret_cast<uint4*>(dst + d) = *reinterpret_cast<const uint4*>(src + so);
     else if (word == 4) *reinterpret_cast<uint32_t*>(dst + d) = *reinterpret_cast<const uint32_t*>(src + so);
@@ -227,11 +230,13 @@ gather_rows_kernel(const uint8_t* __restrict__ src, uint8_t* __restrict__ dst, c
 // dst[i, j] = src[i, perm[j]] for a [rows, cols] matrix of 2- or 4-byte elements
 __global__ void __launch_bounds__(256)
 gather_cols_kernel(const uint8_t* __restrict__ src, uint8_t* __restrict__ dst, const int* __restrict__ perm, int rows,
-                   int cols, int esize) {
+                   int cols, int esize, int* err) {
   const long long n = (long long)rows * cols;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
     const int r = (int)(i / cols), j = (int)(i - (long long)r * cols);
-    const long long so = ((long long)r * cols + __ldg(perm + j)) * esize;
+    const int pj = __ldg(perm + j);
+    if (!checked(pj >= 0 && pj < cols, err)) continue;
+    const long long so = ((long long)r * cols + pj) * esize;
     if (esize == 4) *reinterpret_cast<uint32_t*>(dst + i * 4) = *reinterpret_cast<const uint32_t*>(src + so);
     else *reinterpret_cast<uint16_t*>(dst + i * 2) = *reinterpret_cast<const uint16_t*>(src + so);
   }
@@ -251,7 +256,8 @@ jamba_status gather_rows(const void* src, void* dst, const int* perm, int rows, 
                   row_bytes % 4 == 0;
   const int word = a16 ? 16 : a4 ? 4 : 2;
   gather_rows_kernel<<<gather_grid((long long)rows * (row_bytes / word)), 256, 0, s>>>(
-      reinterpret_cast<const uint8_t*>(src), reinterpret_cast<uint8_t*>(dst), perm, rows, row_bytes, word);
+      reinterpret_cast<const uint8_t*>(src), reinterpret_cast<uint8_t*>(dst), perm, rows, row_bytes, word,
+      device_error_word());
   JB_CUDA(cudaGetLastError());
   return JAMBA_OK;
 }
@@ -260,7 +266,8 @@ jamba_status gather_cols(const void* src, void* dst, const int* perm, int rows, 
   if (!src || !dst || !perm || rows <= 0 || cols <= 0 || (esize != 2 && esize != 4))
     return fail(JAMBA_ERR_INVALID_ARG, "gather_cols: bad argument");
   gather_cols_kernel<<<gather_grid((long long)rows * cols), 256, 0, s>>>(
-      reinterpret_cast<const uint8_t*>(src), reinterpret_cast<uint8_t*>(dst), perm, rows, cols, esize);
+      reinterpret_cast<const uint8_t*>(src), reinterpret_cast<uint8_t*>(dst), perm, rows, cols, esize,
+      device_error_word());
   JB_CUDA(cudaGetLastError());
   return JAMBA_OK;
 }

@@ -88,8 +88,27 @@ static jamba_status launch_bn(int bn, const CUtensorMap& ma, const CUtensorMap& 
 // (decode batches: bound by streaming the codes); up to 255, 128-row tiles
 // with double-buffered accumulators; from 256, two 128-row halves share one
 // widened weight tile.
+// k-splits for the fp32 (down) expert GEMM with INT8 weights when the weights
+// take the M side: the split count (1 to 4, an even number of 64-deep steps
+// each) whose last wave of 128-row weight tiles over the SMs leaves the
+// fewest idle, assuming every group holds one token tile (decode batches).
+int i8w_splits(int M, int num_groups, int N, int K) {
+  if (num_groups <= 0 || M / num_groups > I8T_BNT || N % 128 || K % 128) return 1;
+  const long long tiles = (long long)(M < num_groups ? M : num_groups) * (N / 128);
+  const int k_tiles = K / 64, sms = num_sms();
+  int best = 1;
+  double best_cost = 1e30;
+  for (int sp = 1; sp <= 4; ++sp) {
+    if (k_tiles % (2 * sp)) continue;
+    const long long units = tiles * sp;
+    const double cost = (double)((units + sms - 1) / sms) / sp;   // waves, in whole-tile times
+    if (cost < best_cost - 1e-9) { best_cost = cost; best = sp; }
+  }
+  return best;
+}
+
 static jamba_status gemm_i8w(const GemmDesc& g, cudaStream_t s) {
-  if (!g.grouped || g.transpose_out || g.splits > 1 || g.residual || (g.epi != EPI_SWIGLU && g.epi != EPI_F32))
+  if (!g.grouped || g.transpose_out || g.residual || (g.epi != EPI_SWIGLU && g.epi != EPI_F32))
     return fail(JAMBA_ERR_UNSUPPORTED, "gemm: INT8 weights only in the grouped SwiGLU / fp32 expert GEMMs");
   if (!g.scale_b || (g.epi == EPI_SWIGLU && (!g.scale_b2 || !g.b2)) || !aligned16(g.scale_b) ||
       (g.scale_b2 && !aligned16(g.scale_b2)) || g.N % 4 || g.ldb % 16 || g.K % 16 || !aligned16(g.b) ||
@@ -117,8 +136,12 @@ static jamba_status gemm_i8w(const GemmDesc& g, cudaStream_t s) {
   p.N = g.N;
   p.K = g.K;
   p.k_tiles = (g.K + 63) / 64;
-  p.splits = 1;
-  p.k_tiles_per_split = p.k_tiles;
+  p.splits = g.splits < 1 ? 1 : g.splits;
+  if (p.splits > 1 && (!tok || g.epi != EPI_F32 || p.k_tiles % (2 * p.splits) || g.split_stride < (long long)g.M * g.ldo))
+    return fail(JAMBA_ERR_INVALID_ARG,
+                "gemm: INT8 k-splits only in the few-row fp32 GEMM, an even number of 64-deep steps per split");
+  p.k_tiles_per_split = p.k_tiles / p.splits;
+  p.split_stride = g.split_stride;
   p.n_tiles = (g.N + bn_out - 1) / bn_out;
   p.grouped = 1;
   p.offsets = g.offsets;
@@ -133,7 +156,7 @@ static jamba_status gemm_i8w(const GemmDesc& g, cudaStream_t s) {
   if (tok) {
     if (g.N % 128 || g.K % 128)
       return fail(JAMBA_ERR_INVALID_ARG, "gemm: INT8 weights with few rows need N and K multiples of 128");
-    const long long tiles = (long long)((g.M + I8T_BNT - 1) / I8T_BNT + g.num_groups) * p.n_tiles;
+    const long long tiles = (long long)((g.M + I8T_BNT - 1) / I8T_BNT + g.num_groups) * p.n_tiles * p.splits;
     const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
     return g.epi == EPI_SWIGLU ? launch_i8t<EPI_SWIGLU>(ma, mq, mq2, p, grid, s)
                                : launch_i8t<EPI_F32>(ma, mq, mq2, p, grid, s);
@@ -157,7 +180,7 @@ jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
     return fail(JAMBA_ERR_INVALID_ARG, "gemm: output leading dimension breaks 16-byte rows");
   if (g.residual && (g.transpose_out || g.epi != EPI_BF16 || g.ldr % 8 || !aligned16(g.residual)))
     return fail(JAMBA_ERR_INVALID_ARG, "gemm: residual only with aligned non-transposed bf16 output");
-  if (g.splits > 1 && (g.epi != EPI_F32 || g.grouped))
+  if (g.splits > 1 && (g.epi != EPI_F32 || (g.grouped && !g.b_int8)))
     return fail(JAMBA_ERR_INVALID_ARG, "gemm: split-K writes fp32 partials only");
   if (g.epi == EPI_SWIGLU && (!g.grouped || !g.b2))
     return fail(JAMBA_ERR_INVALID_ARG, "gemm: SwiGLU needs grouped gate and up weights");
@@ -212,6 +235,18 @@ jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
   p.splits = (p.k_tiles + p.k_tiles_per_split - 1) / p.k_tiles_per_split;
   p.m_tiles = (g.M + 127) / 128;
   p.n_tiles = (g.N + bn_out - 1) / bn_out;
+  {
+    // raster bands: as many m-tiles as keep their A rows within 32 MB, and
+    // at least 16.  Each wave sweeps the band's A rows once, so they stay in
+    // L2 only while they and a wave's B and C tiles fit it with room to
+    // spare: B bands of 64 MB (with ~20 MB of A and C per wave) were measured
+    // to miss on every wave, A bands of 16 and 24 MB to hit.  B is read once
+    // per band.
+    const long long band_bytes = 128ll * g.K * 2;
+    long long fit = (32ll << 20) / band_bytes;
+    if (fit < 16) fit = 16;
+    p.band_m = (int)(fit > p.m_tiles ? p.m_tiles : fit);
+  }
   p.grouped = g.grouped;
   p.offsets = g.offsets;
   p.num_groups = g.num_groups;

@@ -110,8 +110,9 @@ template <int MH>
 __device__ __forceinline__ int total_tiles_grouped(const GemmParams& p) {
   int tot = 0;
   for (int g = 0; g < p.num_groups; ++g) {
-    const int cnt = __ldg(p.offsets + g + 1) - __ldg(p.offsets + g);
-    tot += ((cnt + MH - 1) / MH) * p.n_tiles;
+    int o0, o1;
+    group_rows(p, g, o0, o1);
+    tot += ((o1 - o0 + MH - 1) / MH) * p.n_tiles;
   }
   return tot;
 }
@@ -120,7 +121,8 @@ __device__ __forceinline__ int total_tiles_grouped(const GemmParams& p) {
 template <int MH, int BN_OUT>
 __device__ __forceinline__ void decode_tile_grouped(const GemmParams& p, int t, TileInfo& ti) {
   for (int g = 0; g < p.num_groups; ++g) {
-    const int o0 = __ldg(p.offsets + g), o1 = __ldg(p.offsets + g + 1);
+    int o0, o1;
+    group_rows(p, g, o0, o1);
     const int mt = (o1 - o0 + MH - 1) / MH;
     const int tg = mt * p.n_tiles;
     if (t < tg) {
@@ -432,29 +434,35 @@ struct WidenPlan {
   }
 };
 
-// tile t -> (group, token rows m0.. clipped at m_end, weight rows n0..n0+127)
+// tile t -> (group, token rows m0.. clipped at m_end, weight rows n0..n0+127,
+// k-split); with p.splits > 1 (fp32 output only) split s covers 64-deep steps
+// [s k_tiles_per_split, (s + 1) k_tiles_per_split) and writes its partial sums
+// at out + s split_stride
 __device__ __forceinline__ int total_tiles_tok(const GemmParams& p) {
   int tot = 0;
   for (int g = 0; g < p.num_groups; ++g) {
-    const int cnt = __ldg(p.offsets + g + 1) - __ldg(p.offsets + g);
-    tot += ((cnt + I8T_BNT - 1) / I8T_BNT) * p.n_tiles;
+    int o0, o1;
+    group_rows(p, g, o0, o1);
+    tot += ((o1 - o0 + I8T_BNT - 1) / I8T_BNT) * p.n_tiles * p.splits;
   }
   return tot;
 }
 __device__ __forceinline__ void decode_tile_tok(const GemmParams& p, int t, TileInfo& ti) {
   for (int g = 0; g < p.num_groups; ++g) {
-    const int o0 = __ldg(p.offsets + g), o1 = __ldg(p.offsets + g + 1);
+    int o0, o1;
+    group_rows(p, g, o0, o1);
     const int nt = (o1 - o0 + I8T_BNT - 1) / I8T_BNT;
-    const int tg = nt * p.n_tiles;
+    const int tg = nt * p.n_tiles * p.splits;
     if (t < tg) {
-      const int tb = t % nt, wb = t / nt;   // token tiles of one weight tile are neighbours
+      // token tiles of one weight tile are neighbours, then its k-splits
+      const int tb = t % nt, r = t / nt, sp = r % p.splits, wb = r / p.splits;
       ti.m0 = o0 + tb * I8T_BNT;
       ti.m_end = o1;
       ti.n0 = wb * 128;
-      ti.kt0 = 0;
-      ti.kt1 = p.k_tiles;                   // 64-deep steps, an even number here
+      ti.kt0 = sp * p.k_tiles_per_split;    // 64-deep steps, even counts here
+      ti.kt1 = min(p.k_tiles, ti.kt0 + p.k_tiles_per_split);
       ti.group = p.group_mod > 0 ? g % p.group_mod : g;
-      ti.split = 0;
+      ti.split = sp;
       return;
     }
     t -= tg;
@@ -659,7 +667,7 @@ gemm_i8w_tok_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           }
         } else {
           tmem_wait_ld();
-          float* o = reinterpret_cast<float*>(p.out) + f;
+          float* o = reinterpret_cast<float*>(p.out) + ti.split * p.split_stride + f;
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             const int m = ti.m0 + j * 32 + c;

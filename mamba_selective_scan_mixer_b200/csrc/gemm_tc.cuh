@@ -31,6 +31,7 @@ struct GemmParams {
   int k_tiles;           // ceil(K / 64)
   int splits, k_tiles_per_split;
   int m_tiles, n_tiles;  // dense mode
+  int band_m;            // dense mode: m-tiles per raster band (their A rows stay in L2 while B streams)
   int grouped;           // A rows split by offsets[], B is [groups, rows, K]
   const int* offsets;
   int num_groups;
@@ -58,12 +59,24 @@ struct TileInfo {
   int m0, m_end, n0, kt0, kt1, group, split;
 };
 
+// Rows [o0, o1) of group g.  The offsets are device data (a caller's counts in
+// the expert-parallel path): they are clamped into [0, M] with o1 >= o0, so a
+// bad table gives empty or clipped groups, never rows past A or the output,
+// and every role of a kernel decodes the same tiles from it.
+__device__ __forceinline__ void group_rows(const GemmParams& p, int g, int& o0, int& o1) {
+  const int a = __ldg(p.offsets + g), b = __ldg(p.offsets + g + 1);
+  o0 = min(max(a, 0), p.M);
+  o1 = min(max(b, o0), p.M);
+  checked(o0 == a && o1 == b, p.err);
+}
+
 __device__ __forceinline__ int total_tiles(const GemmParams& p) {
   if (!p.grouped) return p.m_tiles * p.n_tiles * p.splits;
   int tot = 0;
   for (int g = 0; g < p.num_groups; ++g) {
-    const int cnt = __ldg(p.offsets + g + 1) - __ldg(p.offsets + g);
-    tot += ((cnt + 127) >> 7) * p.n_tiles;
+    int o0, o1;
+    group_rows(p, g, o0, o1);
+    tot += ((o1 - o0 + 127) >> 7) * p.n_tiles;
   }
   return tot;
 }
@@ -74,12 +87,13 @@ __device__ __forceinline__ void decode_tile(const GemmParams& p, int t, TileInfo
     const int per_split = p.m_tiles * p.n_tiles;
     const int s = t / per_split;
     const int r = t - s * per_split;
-    // rasterise in bands of 16 m-tiles so concurrent CTAs share A and B tiles in L2
-    constexpr int G = 16;
-    const int span = G * p.n_tiles;
+    // rasterise in bands of band_m m-tiles, m fastest within a band: the
+    // band's A rows (sized on the host to stay in L2) are read from DRAM
+    // once, the CTAs of a wave share each B tile, and B is read once per band
+    const int span = p.band_m * p.n_tiles;
     const int gi = r / span;
-    const int first_m = gi * G;
-    const int gsize = min(p.m_tiles - first_m, G);
+    const int first_m = gi * p.band_m;
+    const int gsize = min(p.m_tiles - first_m, p.band_m);
     const int rr = r - gi * span;
     const int mb = first_m + rr % gsize;
     const int nb = rr / gsize;
@@ -92,7 +106,8 @@ __device__ __forceinline__ void decode_tile(const GemmParams& p, int t, TileInfo
     ti.split = s;
   } else {
     for (int g = 0; g < p.num_groups; ++g) {
-      const int o0 = __ldg(p.offsets + g), o1 = __ldg(p.offsets + g + 1);
+      int o0, o1;
+      group_rows(p, g, o0, o1);
       const int mt = (o1 - o0 + 127) >> 7;
       const int tg = mt * p.n_tiles;
       if (t < tg) {
@@ -125,26 +140,43 @@ __device__ __forceinline__ float log1p_small(float e) {
   return e * (1.0f - e * (0.5f - e * (0.33333334f - e * (0.25f - e * (0.2f - e * (0.16666667f - e * 0.14285715f))))));
 }
 
-// softplus of 32 values in place: one ex2 each, the series when every e^v of
-// the warp is below 1/8 (the common case for dt), otherwise one lg2 as well.
-__device__ __forceinline__ void softplus32(float* w) {
+// log(1 + e) for two values at once (0 <= e <= 1/8): the same series in Horner
+// form with packed fp32x2 arithmetic.
+__device__ __forceinline__ float2 log1p_small2(float2 e) {
+  float2 p = ffma2(e, make_float2(0.14285715f, 0.14285715f), make_float2(-0.16666667f, -0.16666667f));
+  p = ffma2(p, e, make_float2(0.2f, 0.2f));
+  p = ffma2(p, e, make_float2(-0.25f, -0.25f));
+  p = ffma2(p, e, make_float2(0.33333334f, 0.33333334f));
+  p = ffma2(p, e, make_float2(-0.5f, -0.5f));
+  p = ffma2(p, e, make_float2(1.0f, 1.0f));
+  return fmul2(p, e);
+}
+
+// softplus of 32 values in place, each given as x = v * log2(e) (v the
+// pre-activation): one ex2 each, then the series when every e^v of the warp
+// is at most 1/8 (x <= -3: the common case for dt), otherwise one lg2 as well.
+__device__ __forceinline__ void softplus32_log2(float* w) {
   float e[32];
-  bool small = true;
+  float mx = w[0];
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
-    e[i] = ex2(1.4426950408889634f * w[i]);
-    small = small && e[i] < 0.125f;
+    e[i] = ex2(w[i]);
+    mx = fmaxf(mx, w[i]);
   }
-  if (__all_sync(0xffffffffu, small)) {
+  if (__all_sync(0xffffffffu, mx <= -3.0f)) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) w[i] = log1p_small(e[i]);
+    for (int i = 0; i < 32; i += 2) {
+      const float2 r = log1p_small2(make_float2(e[i], e[i + 1]));
+      w[i] = r.x; w[i + 1] = r.y;
+    }
   } else {
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       float l;
       asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(l) : "f"(1.0f + e[i]));
-      const float r = e[i] < 0.125f ? log1p_small(e[i]) : 0.6931471805599453f * l;
-      w[i] = w[i] > 15.0f ? w[i] : r;
+      const float v = 0.6931471805599453f * w[i];
+      const float r = e[i] <= 0.125f ? log1p_small(e[i]) : 0.6931471805599453f * l;
+      w[i] = v > 15.0f ? v : r;
     }
   }
 }
@@ -460,7 +492,8 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 #pragma unroll
         for (int jj = 0; jj < S::SB_CHUNKS; ++jj) {
           const int col = ti.n0 + (half + WPQ * jj) * 32 + lane;
-          bl[jj] = (half + WPQ * jj < BN / 32 && col < p.N) ? __ldg(p.bias + col) : 0.f;
+          // scaled by log2(e): the epilogue forms (acc + bias) * log2(e) in one FMA
+          bl[jj] = (half + WPQ * jj < BN / 32 && col < p.N) ? __ldg(p.bias + col) * 1.4426950408889634f : 0.f;
         }
       }
       if (!mbar_wait_warp(tfull0 + 8 * acc, use & 1, p.err)) break;
@@ -497,9 +530,12 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 #pragma unroll
           for (int c = 0; c < 32; c += 4) {
             const float4 b4 = *reinterpret_cast<const float4*>(sb + jj * 32 + c);
-            v[c] += b4.x; v[c + 1] += b4.y; v[c + 2] += b4.z; v[c + 3] += b4.w;
+            const float2 l2e = make_float2(1.4426950408889634f, 1.4426950408889634f);
+            const float2 lo = ffma2(make_float2(v[c], v[c + 1]), l2e, make_float2(b4.x, b4.y));
+            const float2 hi = ffma2(make_float2(v[c + 2], v[c + 3]), l2e, make_float2(b4.z, b4.w));
+            v[c] = lo.x; v[c + 1] = lo.y; v[c + 2] = hi.x; v[c + 3] = hi.y;
           }
-          softplus32(v);
+          softplus32_log2(v);
           uint8_t* buf = stg + (stg_count % NSTG) * 4096;
           if (lane == 0) bulk_wait_read<NSTG - 1>();   // this buffer's previous store has read it
           __syncwarp();

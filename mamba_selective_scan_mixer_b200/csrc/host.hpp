@@ -7,11 +7,38 @@
 #include <cudaTypedefs.h>
 #include <stdint.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include <string>
 
 #include "../../include/jamba.h"
 
 namespace jb {
+
+// NVTX ranges on the host timeline: one around every library call that
+// launches work (JB_RANGE, named after the entry point) and one per step of
+// the path inside it (NvtxSteps::next, named after the step).  They cost a
+// no-op call unless a profiler that collects NVTX is attached.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+#define JB_RANGE_CAT2(a, b) a##b
+#define JB_RANGE_CAT(a, b) JB_RANGE_CAT2(a, b)
+#define JB_RANGE(name) ::jb::NvtxRange JB_RANGE_CAT(jb_range_, __LINE__)(name)
+struct NvtxSteps {
+  bool open = false;
+  void next(const char* name) {
+    if (open) nvtxRangePop();
+    nvtxRangePushA(name);
+    open = true;
+  }
+  ~NvtxSteps() {
+    if (open) nvtxRangePop();
+  }
+};
 
 jamba_status fail(jamba_status st, const std::string& msg);
 const char* last_error();
@@ -91,6 +118,10 @@ struct GemmDesc {
   const void* conv_w; const void* conv_b; float* conv_state; void* xc_out; int conv_c;
 };
 jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s);
+// k-splits that balance the fp32 expert GEMM with INT8 weights over the SMs
+// when every expert holds few rows (1 otherwise); the caller gives the GEMM
+// that many fp32 partial outputs, split_stride elements apart.
+int i8w_splits(int M, int num_groups, int N, int K);
 jamba_status gemm_f32(const GemmDesc& g, cudaStream_t s);
 
 // Splits so that m_tiles * n_tiles * splits fills the SMs, each split keeping
@@ -180,8 +211,9 @@ jamba_status moe_gather(const void* x, const int* perm, int rows, int K, int dm,
 jamba_status group_offsets(const int* counts, int n, int* offsets, cudaStream_t s);   // exclusive prefix sum
 jamba_status quantize_int8_rows(const void* w, int dtype, long long rows, int cols, int8_t* q, float* scale,
                                 cudaStream_t s);
-jamba_status moe_combine(const float* Y, const int* inv, const float* w, int T, int K, int dm, const void* residual,
-                         void* out, cudaStream_t s);
+// out[t] = sum over slots k of w[t, k] * (sum over splits of Y[split][inv[t, k]]) (+ residual[t])
+jamba_status moe_combine(const float* Y, int splits, long long split_stride, const int* inv, const float* w, int T,
+                         int K, int dm, const void* residual, void* out, cudaStream_t s);
 
 // ---------------------------------------------------------------- attention
 jamba_status attn_prefill_core(const void* qkv, void* vt, long long ldv, void* o, void* k_cache, void* v_cache,

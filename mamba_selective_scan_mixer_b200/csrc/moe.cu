@@ -85,61 +85,72 @@ router_kernel(const bf16* __restrict__ x, const bf16* __restrict__ W, int T, int
   }
 }
 
-// Few tokens: one block per token, the d_model sum split over 8 warps (each
-// its own slice, partials added in warp order), so the logits of a decode
-// batch take a few microseconds instead of one warp's serial fp64 chain.
-__global__ void __launch_bounds__(256)
-router_split_kernel(const bf16* __restrict__ x, const bf16* __restrict__ W, int dm, int E, int K,
+// Few tokens: one block per token and one warp per expert (experts beyond the
+// warps loop), each lane summing its 1/32 of d_model in four fp64 partials;
+// then one warp takes the softmax and the top K with one expert per lane
+// (two when E > 32), so the decision costs a few shuffles instead of a
+// serial pass over the logits.
+__global__ void __launch_bounds__(512)
+router_token_kernel(const bf16* __restrict__ x, const bf16* __restrict__ W, int dm, int E, int K,
                     int* __restrict__ idx_out, float* __restrict__ w_out, int* __restrict__ counts) {
-  __shared__ double part[8][64];
   __shared__ double logit[64];
-  const int t = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int slice = dm / 8;   // a multiple of 32
+  const int t = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   const bf16* xr = x + (long long)t * dm;
-  for (int e0 = 0; e0 < E; e0 += ROUTER_EG) {
-    double acc[ROUTER_EG];
-#pragma unroll
-    for (int e = 0; e < ROUTER_EG; ++e) acc[e] = 0.0;
-    for (int k0 = warp * slice + lane * 8; k0 < (warp + 1) * slice; k0 += 256) {
+  for (int e = warp; e < E; e += nw) {
+    const bf16* wr = W + (long long)e * dm;
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll 4
+    for (int k0 = lane * 8; k0 < dm; k0 += 256) {
       const uint4 xv = *reinterpret_cast<const uint4*>(xr + k0);
+      const uint4 wv = __ldg(reinterpret_cast<const uint4*>(wr + k0));
       const __nv_bfloat162* xh = reinterpret_cast<const __nv_bfloat162*>(&xv);
-      float xf[8];
+      const __nv_bfloat162* wh = reinterpret_cast<const __nv_bfloat162*>(&wv);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float2 f = __bfloat1622float2(xh[i]);
-        xf[2 * i] = f.x;
-        xf[2 * i + 1] = f.y;
-      }
-#pragma unroll
-      for (int e = 0; e < ROUTER_EG; ++e) {
-        if (e0 + e >= E) break;
-        const uint4 wv = __ldg(reinterpret_cast<const uint4*>(W + (long long)(e0 + e) * dm + k0));
-        const __nv_bfloat162* wh = reinterpret_cast<const __nv_bfloat162*>(&wv);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 f = __bfloat1622float2(wh[i]);
-          acc[e] += (double)(xf[2 * i] * f.x);      // exact product of two bf16 values
-          acc[e] += (double)(xf[2 * i + 1] * f.y);
-        }
+        const float2 a = __bfloat1622float2(xh[i]), b = __bfloat1622float2(wh[i]);
+        acc[i] += (double)(a.x * b.x);      // exact product of two bf16 values
+        acc[i] += (double)(a.y * b.y);
       }
     }
+    double v = (acc[0] + acc[1]) + (acc[2] + acc[3]);
 #pragma unroll
-    for (int e = 0; e < ROUTER_EG; ++e) {
-      double v = acc[e];
-#pragma unroll
-      for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0 && e0 + e < E) part[warp][e0 + e] = v;
-    }
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) logit[e] = v;
   }
   __syncthreads();
-  if (warp == 0) {
-    for (int e = lane; e < E; e += 32) {
-      double v = part[0][e];
-      for (int w = 1; w < 8; ++w) v += part[w][e];
-      logit[e] = v;
+  if (warp != 0) return;
+  const double NEG = -1.0 / 0.0;
+  const bool v0 = lane < E, v1 = lane + 32 < E;
+  const double l0 = v0 ? logit[lane] : NEG, l1 = v1 ? logit[lane + 32] : NEG;
+  double mx = l0 > l1 ? l0 : l1;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    const double m2 = __shfl_xor_sync(0xffffffffu, mx, o);
+    mx = m2 > mx ? m2 : mx;
+  }
+  double den = (v0 ? exp(l0 - mx) : 0.0) + (v1 ? exp(l1 - mx) : 0.0);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  bool took0 = false, took1 = false;
+  for (int k = 0; k < K; ++k) {
+    // this lane's best untaken expert, then the warp's (ties: the lower index)
+    double bv = NEG;
+    int bi = 1 << 30;
+    if (v0 && !took0) { bv = l0; bi = lane; }
+    if (v1 && !took1 && (bi == (1 << 30) || l1 > bv)) { bv = l1; bi = lane + 32; }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
     }
-    __syncwarp();
-    if (lane == 0) route_token(logit, E, K, t, idx_out, w_out, counts);
+    took0 = took0 || bi == lane;
+    took1 = took1 || bi == lane + 32;
+    if (lane == 0) {
+      idx_out[(long long)t * K + k] = bi;
+      w_out[(long long)t * K + k] = (float)(exp(bv - mx) / den);
+      atomicAdd(counts + bi, 1);
+    }
   }
 }
 
@@ -196,9 +207,12 @@ permute_kernel(const int* __restrict__ idx, int TK, int E, const int* __restrict
 
 // routed row p <- token perm[p] / K
 __global__ void __launch_bounds__(256)
-gather_rows_kernel(const bf16* __restrict__ x, const int* __restrict__ perm, int K, int dm, bf16* __restrict__ out) {
+gather_rows_kernel(const bf16* __restrict__ x, const int* __restrict__ perm, int K, int dm, bf16* __restrict__ out,
+                   int* err) {
   const long long p = blockIdx.x;
-  const int t = perm[p] / K;
+  const int pp = perm[p];
+  if (!checked(pp >= 0 && pp < (int)gridDim.x, err)) return;
+  const int t = pp / K;
   const uint4* src = reinterpret_cast<const uint4*>(x + (long long)t * dm);
   uint4* dst = reinterpret_cast<uint4*>(out + p * dm);
   for (int i = threadIdx.x; i < dm / 8; i += 256) dst[i] = src[i];
@@ -206,14 +220,23 @@ gather_rows_kernel(const bf16* __restrict__ x, const int* __restrict__ perm, int
 
 // out[t] = residual[t] + sum_k w[t, k] * Y[inv[t K + k]], slot 0 first, fp32
 __global__ void __launch_bounds__(256)
-combine_kernel(const float* __restrict__ Y, const int* __restrict__ inv, const float* __restrict__ w, int K, int dm,
-               const bf16* __restrict__ residual, bf16* __restrict__ out) {
+combine_kernel(const float* __restrict__ Y, int splits, long long split_stride, const int* __restrict__ inv,
+               const float* __restrict__ w, int K, int dm, const bf16* __restrict__ residual, bf16* __restrict__ out,
+               int* err) {
   const long long t = blockIdx.x;
+  const int rows = (int)gridDim.x * K;
   for (int c = threadIdx.x * 4; c < dm; c += 1024) {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     for (int k = 0; k < K; ++k) {
       const float wk = w[t * K + k];
-      const float4 y = *reinterpret_cast<const float4*>(Y + (long long)inv[t * K + k] * dm + c);
+      const int j = inv[t * K + k];
+      if (!checked(j >= 0 && j < rows, err)) continue;
+      const float* yr = Y + (long long)j * dm + c;
+      float4 y = *reinterpret_cast<const float4*>(yr);
+      for (int sp = 1; sp < splits; ++sp) {   // k-split partial sums of the down GEMM, in split order
+        const float4 y2 = *reinterpret_cast<const float4*>(yr + sp * split_stride);
+        y.x += y2.x; y.y += y2.y; y.z += y2.z; y.w += y2.w;
+      }
       acc[0] = fmaf(wk, y.x, acc[0]);
       acc[1] = fmaf(wk, y.y, acc[1]);
       acc[2] = fmaf(wk, y.z, acc[2]);
@@ -307,8 +330,8 @@ jamba_status moe_route(const void* x, const void* W, int T, int dm, int E, int K
                        int* offsets, int* perm, int* inv, cudaStream_t s) {
   JB_CUDA(cudaMemsetAsync(counts, 0, sizeof(int) * E, s));
   if (T <= 4096) {
-    router_split_kernel<<<T, 256, 0, s>>>(reinterpret_cast<const bf16*>(x), reinterpret_cast<const bf16*>(W), dm, E,
-                                          K, idx, w, counts);
+    router_token_kernel<<<T, 32 * (E < 16 ? E : 16), 0, s>>>(reinterpret_cast<const bf16*>(x),
+                                                             reinterpret_cast<const bf16*>(W), dm, E, K, idx, w, counts);
   } else {
     int blocks = (T + 7) / 8;
     const int cap = 8 * num_sms();
@@ -341,15 +364,16 @@ jamba_status group_offsets(const int* counts, int n, int* offsets, cudaStream_t 
 }
 
 jamba_status moe_gather(const void* x, const int* perm, int rows, int K, int dm, void* out, cudaStream_t s) {
-  gather_rows_kernel<<<rows, 256, 0, s>>>(reinterpret_cast<const bf16*>(x), perm, K, dm, reinterpret_cast<bf16*>(out));
+  gather_rows_kernel<<<rows, 256, 0, s>>>(reinterpret_cast<const bf16*>(x), perm, K, dm, reinterpret_cast<bf16*>(out),
+                                          device_error_word());
   JB_CUDA(cudaGetLastError());
   return JAMBA_OK;
 }
 
-jamba_status moe_combine(const float* Y, const int* inv, const float* w, int T, int K, int dm, const void* residual,
-                         void* out, cudaStream_t s) {
-  combine_kernel<<<T, 256, 0, s>>>(Y, inv, w, K, dm, reinterpret_cast<const bf16*>(residual),
-                                   reinterpret_cast<bf16*>(out));
+jamba_status moe_combine(const float* Y, int splits, long long split_stride, const int* inv, const float* w, int T,
+                         int K, int dm, const void* residual, void* out, cudaStream_t s) {
+  combine_kernel<<<T, 256, 0, s>>>(Y, splits, split_stride, inv, w, K, dm, reinterpret_cast<const bf16*>(residual),
+                                   reinterpret_cast<bf16*>(out), device_error_word());
   JB_CUDA(cudaGetLastError());
   return JAMBA_OK;
 }

@@ -496,8 +496,10 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
       h[j][i] = make_float2(0.f, 0.f);
       if (known && a.h0 && valid) {
         const int cn = a.perm ? __ldg(a.perm + c + j) : c + j;
-        const float* src = a.h0 + ((long long)cx.b * a.di + cn) * NS + 2 * i;
-        h[j][i] = make_float2(src[0], src[1]);
+        if (checked(cn >= 0 && cn < a.di, a.err)) {
+          const float* src = a.h0 + ((long long)cx.b * a.di + cn) * NS + 2 * i;
+          h[j][i] = make_float2(src[0], src[1]);
+        }
       }
     }
   float R[CPT];
@@ -625,13 +627,15 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
           }
           if (last) {
             const int cn = a.perm ? __ldg(a.perm + c + j) : c + j;
-            *reinterpret_cast<float2*>(a.h_out + ((long long)cx.b * a.di + cn) * NS + 2 * n2) = he;
+            if (checked(cn >= 0 && cn < a.di, a.err))
+              *reinterpret_cast<float2*>(a.h_out + ((long long)cx.b * a.di + cn) * NS + 2 * n2) = he;
           }
           if (a.summary && valid) {
             const int cn = a.perm ? __ldg(a.perm + c + j) : c + j;
             const float2 pin = make_float2(sP[(cl + j) * NS + 2 * n2], sP[(cl + j) * NS + 2 * n2 + 1]);
-            *reinterpret_cast<float2*>(a.p_out + ((long long)cx.b * a.di + cn) * NS + 2 * n2) =
-                make_float2(pe[2 * n2] * pin.x, pe[2 * n2 + 1] * pin.y);
+            if (checked(cn >= 0 && cn < a.di, a.err))
+              *reinterpret_cast<float2*>(a.p_out + ((long long)cx.b * a.di + cn) * NS + 2 * n2) =
+                  make_float2(pe[2 * n2] * pin.x, pe[2 * n2 + 1] * pin.y);
           }
           h[j][n2] = hi;
         }
@@ -662,6 +666,7 @@ selective_scan_kernel(const __grid_constant__ CUtensorMap mx, const __grid_const
 #pragma unroll
     for (int j = 0; j < CPT; ++j) {
       const int cn = a.perm ? __ldg(a.perm + c + j) : c + j;
+      if (!checked(cn >= 0 && cn < a.di, a.err)) continue;
       float pe[16];
       chunk_decay<FAST>(R[j], P[j], pe);
 #pragma unroll
@@ -958,6 +963,13 @@ jamba_status scan_run(const ScanCall& s, cudaStream_t st) {
   if (s.summary ? (!s.h_out || !s.p_out || !aligned16(s.h_out) || !aligned16(s.p_out)) : (!s.z || !s.y))
     return fail(JAMBA_ERR_INVALID_ARG, "scan: null tensor");
   if (s.chunk <= 0 || s.chunk % 16) return fail(JAMBA_ERR_INVALID_ARG, "scan: chunk must be a positive multiple of 16");
+  if (s.h0 && s.h_out) {
+    // the first chunk reads h0 while the last one may already write h_out:
+    // nothing orders the two, so the ranges may not overlap
+    const uintptr_t a = reinterpret_cast<uintptr_t>(s.h0), b = reinterpret_cast<uintptr_t>(s.h_out);
+    const uintptr_t n = (uintptr_t)s.batch * s.di * NS * sizeof(float);
+    if (a < b + n && b < a + n) return fail(JAMBA_ERR_INVALID_ARG, "scan: h_out may not overlap h0");
+  }
   if (s.ld_x < s.di || s.ld_dt < s.di || s.ld_b < NS || s.ld_c < NS ||
       (!s.summary && (s.ld_z < s.di || s.ld_y < s.di)))
     return fail(JAMBA_ERR_INVALID_ARG, "scan: leading dimension below the row width");

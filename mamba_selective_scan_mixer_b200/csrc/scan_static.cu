@@ -82,6 +82,7 @@ extern "C" jamba_status jamba_selective_scan_static(const void* x, int ld_x, con
                                                     const float* D, const float* h0, void* y, int ld_y,
                                                     float* h_out, int batch, int seqlen, int d_inner,
                                                     int d_state, int dtype, int* status, jamba_stream_t stream) {
+  JB_RANGE("jamba_selective_scan_static");
   if ((dtype != JAMBA_BF16 && dtype != JAMBA_F32) || (bc_dtype != JAMBA_BF16 && bc_dtype != JAMBA_F32))
     return fail(JAMBA_ERR_UNSUPPORTED, "static scan: dtype must be JAMBA_F32 or JAMBA_BF16");
   if (d_state != 16) return fail(JAMBA_ERR_UNSUPPORTED, "static scan: d_state must be 16");

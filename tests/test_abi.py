@@ -31,7 +31,7 @@ def test_library_exports_every_header_symbol(lib):
 
 def test_binding_covers_every_header_symbol():
     from mamba_selective_scan_mixer_b200._abi import SIGNATURES
-    declared = set(header_symbols()) - {"jamba_last_error"}
+    declared = set(header_symbols()) - {"jamba_last_error", "jamba_checked_build"}   # not jamba_status
     assert declared == set(SIGNATURES), declared ^ set(SIGNATURES)
 
 
@@ -41,6 +41,19 @@ def test_exports_with_nm(lib):
                          capture_output=True, text=True).stdout
     for n in header_symbols():
         assert (" T " + n) in out, n
+
+
+def test_checked_build_exports_the_same_symbols_and_says_so(lib):
+    """libjamba_checked.so (-DJAMBA_CHECKS) exports every header symbol and
+    jamba_checked_build() tells the two builds apart (no GPU needed)."""
+    from mamba_selective_scan_mixer_b200 import build
+    path = build.build(checked=True)
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True).stdout
+    for n in header_symbols():
+        assert (" T " + n) in out, n
+    chk = ctypes.CDLL(path)
+    assert chk.jamba_checked_build() == 1
+    assert lib.jamba_checked_build() == 0
 
 
 def test_create_rejects_bad_config_without_gpu(lib):

@@ -187,6 +187,29 @@ def test_scan_repeated_calls_reuse_workspace(dev):
     J.device_status()
 
 
+def test_scan_rejects_state_out_overlapping_state_in(dev):
+    """h_out over h0 (whole or in part) is refused with INVALID_ARG before any
+    launch: the first chunk's reads of h0 and the last chunk's writes of h_out
+    are not ordered."""
+    import ctypes
+    import mamba_selective_scan_mixer_b200 as J
+    from mamba_selective_scan_mixer_b200 import _abi
+    s = {k: v.to(dev) for k, v in scan_inputs(1, 256, 256, 16, seed=22).items()}
+    y = torch.empty_like(s["x"])
+    h = torch.zeros(2, 256, 16, device=dev)
+    n = ctypes.c_size_t()
+    J.lib().jamba_selective_scan_workspace_size(1, 256, 256, 16, 64, ctypes.byref(n))
+    ws = torch.empty(n.value, dtype=torch.uint8, device=dev)
+    P = lambda t: ctypes.c_void_p(t.data_ptr())
+    for h0, ho in ((h[0], h[0]), (h[0], h.view(-1)[2048:6144].view(256, 16)), (h[0], h[1])):
+        st = J.lib().jamba_selective_scan(P(s["x"]), 256, P(s["z"]), 256, P(s["dt"]), 256, P(s["B"]), 16, P(s["C"]),
+                                          16, _abi.JAMBA_BF16, P(s["A"]), P(s["D"]), P(h0), P(y), 256, P(ho), 1, 256,
+                                          256, 16, _abi.JAMBA_BF16, 64, P(ws), ctypes.c_size_t(n.value), None)
+        assert st == (0 if ho.data_ptr() == h[1].data_ptr() else 1), st   # 1: JAMBA_ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    J.device_status()
+
+
 # ------------------------------------------------------------------ norm
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])

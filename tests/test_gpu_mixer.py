@@ -97,6 +97,16 @@ def test_bf16_prefill_reordered_channel_groups(dev):
     assert rel_l2(np.concatenate([to_np(out1), to_np(out2)], axis=1), ref["out"]) < TOL_BF16
     assert rel_l2(to_np(ss2), ref["ssm_state"]) < TOL_BF16
     assert rel_l2(to_np(cs2), ref["conv_state"]) < TOL_BF16
+    # in-place continuation over many time chunks: the state in is copied
+    # before the scan (its first chunk reads it while its last chunk writes
+    # it), so the result is the continuation into separate caches (up to the
+    # rounding order of the carries, which the look-back takes as they come)
+    cs3, ss3 = cs.clone(), ss.clone()
+    out3, _, _ = mix.prefill(ud[:, 700:].contiguous(), conv_state_in=cs3, ssm_state_in=ss3, conv_state_out=cs3,
+                             ssm_state_out=ss3)
+    assert rel_l2(to_np(out3), to_np(out2)) < 1e-5
+    assert rel_l2(to_np(ss3), to_np(ss2)) < 1e-6
+    assert torch.equal(cs3, cs2)
 
 
 def test_bf16_decode_steps_match_oracle_and_prefill(dev):
