@@ -34,7 +34,7 @@ PAIR_B, PAIR_L = 4, 8192
 ATTN_L = 32768
 METRIC = "Mamba-layer tokens/s (prefill 128K, decode) at d_model=4096; scan HBM GB/s vs peak"
 # DRAM bytes (read + write) of one in_proj launch at 131072 tokens: ncu capture at 16384 tokens
-# (1.209 GB read + 0.514 GB written) scaled by 8, since
+# (0.710 GB read + 0.518 GB written) scaled by 8, since
 # operand re-reads and the output all grow with the token count
 IN_PROJ_TRAFFIC_128K = 8 * (0.710058752e9 + 0.517750784e9)
 
