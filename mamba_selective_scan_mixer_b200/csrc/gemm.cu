@@ -236,15 +236,18 @@ jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
   p.m_tiles = (g.M + 127) / 128;
   p.n_tiles = (g.N + bn_out - 1) / bn_out;
   {
-    // raster bands: as many m-tiles as keep their A rows within 32 MB, and
-    // at least 16.  Each wave sweeps the band's A rows once, so they stay in
-    // L2 only while they and a wave's B and C tiles fit it with room to
-    // spare: B bands of 64 MB (with ~20 MB of A and C per wave) were measured
-    // to miss on every wave, A bands of 16 and 24 MB to hit.  B is read once
-    // per band.
+    // raster bands: as many m-tiles as keep their A rows within 32 MB, from
+    // 16 to 32 of them.  A wave of CTAs then spans the band's whole height
+    // and several n-tiles, and the next wave finds the same A rows in L2 as
+    // long as they and a wave's B and C tiles fit it with room to spare: B
+    // bands of 64 MB (with ~20 MB of A and C per wave) were measured to miss
+    // on every wave, A bands of 16, 24 and 32 MB to hit.  Taller bands (512
+    // m-tiles for dt_proj's K = 256) leave a wave inside one n-tile, and its
+    // large output pushes the band out of L2 before the next n-tile reuses
+    // it (dt_proj 0.95 -> 1.10 ms).  B is read once per band.
     const long long band_bytes = 128ll * g.K * 2;
     long long fit = (32ll << 20) / band_bytes;
-    if (fit < 16) fit = 16;
+    fit = fit < 16 ? 16 : fit > 32 ? 32 : fit;
     p.band_m = (int)(fit > p.m_tiles ? p.m_tiles : fit);
   }
   p.grouped = g.grouped;

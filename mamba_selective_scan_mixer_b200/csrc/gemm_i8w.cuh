@@ -90,14 +90,20 @@ struct WidenPlanLinear {
       dhi[i] = row * 128 + (((2 * g + 1) ^ (row & 7)) << 4);
     }
   }
-  // q, b: shared-memory addresses of the code tile and the widened tile
+  // q, b: shared-memory addresses of the code tile and the widened tile.  All
+  // loads go out before the first store: the accesses are ordered asm
+  // statements, so a load placed after a store would wait for the widening of
+  // the codes before it, one load latency per iteration.
   __device__ __forceinline__ void run(uint32_t q, uint32_t b) const {
+    uint4 v[IT];
+#pragma unroll
+    for (int i = 0; i < IT; ++i)
+      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(v[i].x), "=r"(v[i].y), "=r"(v[i].z), "=r"(v[i].w) : "r"(q + src0 + PER * 16 * i));
 #pragma unroll
     for (int i = 0; i < IT; ++i) {
-      uint4 v, lo, hi;
-      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                   : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(q + src0 + PER * 16 * i));
-      widen16(v, lo, hi);
+      uint4 lo, hi;
+      widen16(v[i], lo, hi);
       asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(b + dlo[i]), "r"(lo.x), "r"(lo.y), "r"(lo.z),
                    "r"(lo.w) : "memory");
       asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(b + dhi[i]), "r"(hi.x), "r"(hi.y), "r"(hi.z),
@@ -392,46 +398,6 @@ struct I8tSmem {
   static constexpr int USED = A_OFF + BSTAGES * A_COLS;
   static constexpr uint32_t TMEM_COLS = USED <= 32 ? 32 : USED <= 64 ? 64 : USED <= 128 ? 128 : USED <= 256 ? 256 : 512;
   static_assert(USED <= 512, "tensor memory");
-};
-
-// Codes h*64 .. h*64+63 of ROWS rows stored as 128-byte rows under the
-// 128-byte swizzle -> ROWS x 64 bf16 (swizzled K-major).  A quarter-warp
-// takes the rows pi and pi ^ 5 of an 8-row group (pi < 4): their loads fall
-// in opposite halves of the swizzled row and their stores in chunks of
-// opposite parity, so neither side has bank conflicts.  The byte offsets of a
-// thread's loads and stores are the same for every stage, so they are worked
-// out once (the second half's loads differ from the first's in bit 6 only).
-template <int ROWS, int DQ_WARPS>
-struct WidenPlan {
-  static constexpr int IT = ROWS * 4 / (32 * DQ_WARPS);
-  static_assert(IT * 32 * DQ_WARPS == ROWS * 4, "whole iterations");
-  uint32_t src[IT], dlo[IT], dhi[IT];
-  __device__ __forceinline__ explicit WidenPlan(int ct) {
-#pragma unroll
-    for (int i = 0; i < IT; ++i) {
-      const int idx = ct + 32 * DQ_WARPS * i;
-      const int g = idx & 3, sel = (idx >> 2) & 1, pi = (idx >> 3) & 3;
-      const int row = (idx >> 5) * 8 + (sel ? (pi ^ 5) : pi);
-      src[i] = row * 128 + ((g ^ (row & 7)) << 4);
-      dlo[i] = row * 128 + (((2 * g) ^ (row & 7)) << 4);
-      dhi[i] = row * 128 + (((2 * g + 1) ^ (row & 7)) << 4);
-    }
-  }
-  // q, b: shared-memory addresses of the code tile and the widened tile
-  __device__ __forceinline__ void run(uint32_t q, int h, uint32_t b) const {
-    const uint32_t hx = (uint32_t)h << 6;
-#pragma unroll
-    for (int i = 0; i < IT; ++i) {
-      uint4 v, lo, hi;
-      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                   : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(q + (src[i] ^ hx)));
-      widen16(v, lo, hi);
-      asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(b + dlo[i]), "r"(lo.x), "r"(lo.y), "r"(lo.z),
-                   "r"(lo.w) : "memory");
-      asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(b + dhi[i]), "r"(hi.x), "r"(hi.y), "r"(hi.z),
-                   "r"(hi.w) : "memory");
-    }
-  }
 };
 
 // tile t -> (group, token rows m0.. clipped at m_end, weight rows n0..n0+127,
