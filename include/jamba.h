@@ -140,8 +140,9 @@ jamba_status jamba_mamba_workspace_size(jamba_mamba_t h, int batch, int seqlen, 
  *   conv_state_out / ssm_state_out: same shapes, fp32 or NULL: the caches after
  *            the last token (conv: the last d_conv-1 pre-conv inputs, oldest first)
  *   ws / ws_bytes: device workspace of at least jamba_mamba_workspace_size bytes
- * The states may alias (in == out) for in-place continuation; an aliased
- * ssm state is copied to the workspace before the scan reads it. */
+ * The states may alias (in == out) for in-place continuation (the conv cache
+ * is copied to the workspace first; the scan orders its own in-place update),
+ * but may not overlap otherwise. */
 jamba_status jamba_mamba_prefill(jamba_mamba_t h, const void* u, const void* residual, void* out,
                                  int batch, int seqlen, const float* conv_state_in,
                                  const float* ssm_state_in, float* conv_state_out,
@@ -290,15 +291,16 @@ jamba_status jamba_selective_scan_workspace_size(int batch, int seqlen, int d_in
  *   h0     [batch, d_inner, d_state] fp32 or NULL (zeros)
  *   y      [batch, seqlen, *] dtype, row stride ld_y (a multiple of 4)
  *   h_out  [batch, d_inner, d_state] fp32 or NULL: state after the last step;
- *          may not overlap h0 (the first chunk's reads of h0 and the last
- *          chunk's writes of h_out are not ordered)
+ *          may be h0 itself (in-place update: the last time chunk writes only
+ *          after the first has published that it read h0), but may not
+ *          overlap it otherwise
  *   chunk  time steps per chunk (multiple of 16), 0 = automatic
  * Time is split into chunks scanned concurrently; the state entering each
  * chunk is passed between chunks with a decoupled look-back, which folds the
  * carries in the order they become available: repeated calls agree up to
  * that rounding order (last bits), not bit for bit.  Errors:
- * UNSUPPORTED for d_state != 16, INVALID_ARG for strides/alignment or h_out
- * overlapping h0. */
+ * UNSUPPORTED for d_state != 16, INVALID_ARG for strides/alignment or an
+ * h_out that overlaps h0 without being it. */
 jamba_status jamba_selective_scan(const void* x, int ld_x, const void* z, int ld_z, const float* dt,
                                   int ld_dt, const void* B, int ld_b, const void* C, int ld_c,
                                   int bc_dtype, const float* A, const float* D, const float* h0,

@@ -62,7 +62,6 @@ struct PrefillWs {
   // context-parallel prefill only: in_proj rows of the 3 input tokens before
   // the slice, the conv cache they make, and the state entering the slice
   void* xz_halo; float* conv_halo; float* h_in;
-  float* h_tmp;         // the state entering the scan, when the caller's in and out states are one buffer
   ScanSchedule sched;   // the scan's per-group time chunks (n == 0: uniform chunks of `chunk`)
   size_t total;
 };
@@ -94,7 +93,6 @@ PrefillWs carve_prefill(const jamba_mamba* h, int batch, int L, void* ws, bool c
   p.dt = cv.take<float>(T * c.d_inner * 4);
   p.y = cv.take(T * c.d_inner * es);
   p.conv_tmp = cv.take<float>((size_t)batch * c.d_inner * (c.d_conv - 1) * 4);
-  p.h_tmp = cv.take<float>((size_t)batch * c.d_inner * c.d_state * 4);
   plan_scan(h, batch, L, &p.sched);
   if (h->perm) {
     // a per-group plan never exceeds the resident CTAs; sized for that bound
@@ -336,22 +334,6 @@ ScanCall scan_call(const jamba_mamba& h, const PrefillWs& p, int batch, int seql
   return sc;
 }
 
-// The state the scan starts from: the caller's, or a copy of it in the
-// workspace when it shares memory with the state the scan writes (in-place
-// continuation: the scan's first chunk reads the state while its last chunk
-// may already write it).
-jamba_status scan_state_in(const jamba_mamba& h, const PrefillWs& p, int batch, const float* in, const float* out,
-                           cudaStream_t s, const float** use) {
-  *use = in;
-  const size_t n = sizeof(float) * (size_t)batch * h.cfg.d_inner * h.cfg.d_state;
-  const uint8_t *a = reinterpret_cast<const uint8_t*>(in), *b = reinterpret_cast<const uint8_t*>(out);
-  if (a && b && a < b + n && b < a + n) {
-    JB_CUDA(cudaMemcpyAsync(p.h_tmp, in, n, cudaMemcpyDeviceToDevice, s));
-    *use = p.h_tmp;
-  }
-  return JAMBA_OK;
-}
-
 // The prefill from the scan on: selective scan + D skip + SiLU(z) gate, out_proj (+ residual).
 jamba_status prefill_back(const jamba_mamba& h, const PrefillWs& p, int batch, int seqlen, const float* ssm_state_in,
                           float* ssm_state_out, const void* residual, void* out, cudaStream_t s) {
@@ -360,7 +342,7 @@ jamba_status prefill_back(const jamba_mamba& h, const PrefillWs& p, int batch, i
   NvtxSteps nv;
   nv.next("selective_scan");
   ScanCall sc = scan_call(h, p, batch, seqlen);
-  JB_TRY(scan_state_in(h, p, batch, ssm_state_in, ssm_state_out, s, &sc.h0));
+  sc.h0 = ssm_state_in;   // may be ssm_state_out itself: the scan orders the in-place update
   sc.h_out = ssm_state_out;
   JB_TRY(scan_run(sc, s));
   nv.next("out_proj");
@@ -557,7 +539,7 @@ jamba_status jamba_mamba_prefill_tp_finish(jamba_mamba_t h, const float* xproj_s
   const int T = batch * seqlen, di = c.d_inner, dm = c.d_model;
   JB_TRY(prefill_front_b(*h, p, xproj_sum, 1, batch, seqlen, s));
   ScanCall sc = scan_call(*h, p, batch, seqlen);
-  JB_TRY(scan_state_in(*h, p, batch, ssm_state_in, ssm_state_out, s, &sc.h0));
+  sc.h0 = ssm_state_in;
   sc.h_out = ssm_state_out;
   JB_TRY(scan_run(sc, s));
   // this rank's share of out_proj (its d_inner columns), fp32

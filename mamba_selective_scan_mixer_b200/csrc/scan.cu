@@ -963,12 +963,13 @@ jamba_status scan_run(const ScanCall& s, cudaStream_t st) {
   if (s.summary ? (!s.h_out || !s.p_out || !aligned16(s.h_out) || !aligned16(s.p_out)) : (!s.z || !s.y))
     return fail(JAMBA_ERR_INVALID_ARG, "scan: null tensor");
   if (s.chunk <= 0 || s.chunk % 16) return fail(JAMBA_ERR_INVALID_ARG, "scan: chunk must be a positive multiple of 16");
-  if (s.h0 && s.h_out) {
-    // the first chunk reads h0 while the last one may already write h_out:
-    // nothing orders the two, so the ranges may not overlap
+  if (s.h0 && s.h_out && s.h0 != s.h_out) {
+    // h_out == h0 (in place) is ordered in the kernel: the last chunk writes
+    // after chunk 0 has published its flag, long after reading h0.  A partial
+    // overlap would put other rows' reads and writes in conflict: refused.
     const uintptr_t a = reinterpret_cast<uintptr_t>(s.h0), b = reinterpret_cast<uintptr_t>(s.h_out);
     const uintptr_t n = (uintptr_t)s.batch * s.di * NS * sizeof(float);
-    if (a < b + n && b < a + n) return fail(JAMBA_ERR_INVALID_ARG, "scan: h_out may not overlap h0");
+    if (a < b + n && b < a + n) return fail(JAMBA_ERR_INVALID_ARG, "scan: h_out overlaps h0 without being it");
   }
   if (s.ld_x < s.di || s.ld_dt < s.di || s.ld_b < NS || s.ld_c < NS ||
       (!s.summary && (s.ld_z < s.di || s.ld_y < s.di)))

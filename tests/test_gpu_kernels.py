@@ -187,10 +187,11 @@ def test_scan_repeated_calls_reuse_workspace(dev):
     J.device_status()
 
 
-def test_scan_rejects_state_out_overlapping_state_in(dev):
-    """h_out over h0 (whole or in part) is refused with INVALID_ARG before any
-    launch: the first chunk's reads of h0 and the last chunk's writes of h_out
-    are not ordered."""
+def test_scan_state_in_place_and_partial_overlap(dev):
+    """h_out == h0 runs in place (the last time chunk writes after the first
+    has published that it read h0) and matches separate buffers up to the
+    carries' rounding order; an h_out that overlaps h0 without being it is
+    refused with INVALID_ARG before any launch."""
     import ctypes
     import mamba_selective_scan_mixer_b200 as J
     from mamba_selective_scan_mixer_b200 import _abi
@@ -201,12 +202,20 @@ def test_scan_rejects_state_out_overlapping_state_in(dev):
     J.lib().jamba_selective_scan_workspace_size(1, 256, 256, 16, 64, ctypes.byref(n))
     ws = torch.empty(n.value, dtype=torch.uint8, device=dev)
     P = lambda t: ctypes.c_void_p(t.data_ptr())
-    for h0, ho in ((h[0], h[0]), (h[0], h.view(-1)[2048:6144].view(256, 16)), (h[0], h[1])):
-        st = J.lib().jamba_selective_scan(P(s["x"]), 256, P(s["z"]), 256, P(s["dt"]), 256, P(s["B"]), 16, P(s["C"]),
-                                          16, _abi.JAMBA_BF16, P(s["A"]), P(s["D"]), P(h0), P(y), 256, P(ho), 1, 256,
-                                          256, 16, _abi.JAMBA_BF16, 64, P(ws), ctypes.c_size_t(n.value), None)
-        assert st == (0 if ho.data_ptr() == h[1].data_ptr() else 1), st   # 1: JAMBA_ERR_INVALID_ARG
+    h.normal_()
+    run = lambda h0, ho: J.lib().jamba_selective_scan(
+        P(s["x"]), 256, P(s["z"]), 256, P(s["dt"]), 256, P(s["B"]), 16, P(s["C"]), 16, _abi.JAMBA_BF16, P(s["A"]),
+        P(s["D"]), P(h0), P(y), 256, P(ho), 1, 256, 256, 16, _abi.JAMBA_BF16, 64, P(ws), ctypes.c_size_t(n.value), None)
+    h_sep = torch.empty(256, 16, device=dev)
+    assert run(h[0], h_sep) == 0                                  # separate buffers (4 time chunks of 64)
+    y_sep = y.clone()
+    h_in_place = h[0].clone()
+    assert run(h_in_place, h_in_place) == 0                       # in place
     torch.cuda.synchronize()
+    J.device_status()
+    assert rel_l2(to_np(h_in_place), to_np(h_sep)) < 1e-6
+    assert rel_l2(to_np(y), to_np(y_sep)) < 1e-5
+    assert run(h[0], h.view(-1)[2048:6144].view(256, 16)) == 1    # partial overlap: JAMBA_ERR_INVALID_ARG
     J.device_status()
 
 
