@@ -338,6 +338,8 @@ def run_product(args):
         for lm in layers:
             dcs, dss = lm.new_states(B)
             lm.prefill(u0, conv_state_out=dcs, ssm_state_out=dss)
+            torch.cuda.synchronize()
+            lm.release_workspace()   # the prefill's ~21 GB; the decode steps need a few MB
             caches.append((dcs, dss))
         steps_u = decode_inputs(sh, B, NST, seed=1, device=dev)
         dout = torch.empty(B, sh.d_model, dtype=torch.bfloat16, device=dev)

@@ -90,6 +90,11 @@ class MambaMixer:
         return (torch.zeros(batch, sh.d_inner, sh.d_conv - 1, device=self.device),
                 torch.zeros(batch, sh.d_inner, sh.d_state, device=self.device))
 
+    def release_workspace(self):
+        """Drop the cached device workspace (after the last call that used it
+        has completed); the next call allocates one of its own size again."""
+        self.ws = _Workspace()
+
     def prefill(self, u, residual=None, conv_state_in=None, ssm_state_in=None, conv_state_out=None,
                 ssm_state_out=None, out=None, stream=None):
         """u [B, L, d_model] -> (out, conv_state_out, ssm_state_out)."""
