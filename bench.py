@@ -33,10 +33,10 @@ SCAN_L, SCAN_DI = 131072, 8192
 PAIR_B, PAIR_L = 4, 8192
 ATTN_L = 32768
 METRIC = "Mamba-layer tokens/s (prefill 128K, decode) at d_model=4096; scan HBM GB/s vs peak"
-# DRAM bytes (read + write) of one in_proj launch at 131072 tokens: ncu capture at 16384 tokens
-# (0.710 GB read + 0.518 GB written) scaled by 8, since
-# operand re-reads and the output all grow with the token count
-IN_PROJ_TRAFFIC_128K = 8 * (0.710058752e9 + 0.517750784e9)
+# DRAM bytes (read + write) of one in_proj + conv launch pair at 131072 tokens: ncu at 16384 tokens
+# (GEMM 0.715 GB read + 0.542 GB written, slab-row kernel 0.050 + 0.0004 GB) scaled by 8, since
+# operand re-reads and the outputs all grow with the token count
+IN_PROJ_TRAFFIC_128K = 8 * (0.714592512e9 + 0.542140928e9 + 0.050384896e9 + 0.000403968e9)
 
 
 def parse():
@@ -270,26 +270,28 @@ def run_product(args):
                                   "d_state 16, dt_rank 256, inner RMSNorm, bf16 weights/activations, fp32 state" % L,
                       "global_batch": world, "seq_len": L, "parallelism": "replicas" if world > 1 else "single",
                       "l2": "512 MB buffer written before every timed step (outside the events)"},
-           # per prefill step: in_proj, conv, x_proj, x_proj sum + norms, dt_proj, scan, out_proj
+           # per prefill step: in_proj + conv, conv slab rows, x_proj, x_proj sum + norms, dt_proj, scan, out_proj
            "gpu_launches": None if ms is None else 7 * args.steps, "clocks": clk}
 
     if rank == 0 and "gemm" in parts:
-        # dominant kernel: in_proj GEMM on the tensor cores, same shape as inside the step
-        xz = torch.empty(L, 2 * sh.d_inner, dtype=torch.bfloat16, device=dev)
-        a2 = u.view(L, sh.d_model)
-        g = lambda: J.gemm(a2, params["in_proj"], out=xz)
+        # dominant kernel: in_proj on the tensor cores with the conv in its
+        # epilogue (+ the slab-row kernel after it), the same launches as inside the step
+        xz = torch.empty(1, L, 2 * sh.d_inner, dtype=torch.bfloat16, device=dev)
+        xc = torch.empty(1, L, sh.d_inner, dtype=torch.bfloat16, device=dev)
+        g = lambda: J.in_proj_conv1d(u, params["in_proj"], params["conv_w"], params["conv_b"], xz=xz, xc=xc)
         for _ in range(2):
             g()
         gms, _ = event_time_ms(g, 5, stream, flush)
         flops = 2.0 * L * 2 * sh.d_inner * sh.d_model
         ach = flops / (gms / 1e3) / 1e12
-        res["roofline"] = {"kernel": "in_proj gemm_bf16_tc_kernel<256,4> (%dx%dx%d)" % (L, 2 * sh.d_inner, sh.d_model),
+        res["roofline"] = {"kernel": "in_proj + conv1d: gemm_bf16_tc_kernel<256,4,EPI_CONVP> + conv_fixup_kernel "
+                                     "(%dx%dx%d)" % (L, 2 * sh.d_inner, sh.d_model),
                            "bound": "tensor", "achieved": round(ach, 1), "peak": pk["bf16"], "unit": "TFLOP/s",
                            "frac": round(ach / pk["bf16"], 4),
                            "traffic": IN_PROJ_TRAFFIC_128K if L == PREFILL_L else None,
                            "peak_source": "%s bf16 burst (kernel timed alone)" % pk["src"],
                            "ms": round(gms, 3)}
-        del xz
+        del xz, xc
     if rank == 0 and "scan" in parts:
         # selective scan alone at 128K context
         SL = args.scan_seqlen

@@ -375,6 +375,25 @@ jamba_status jamba_causal_conv1d(const void* x, int ld_x, const void* w, const v
                                  const float* state_in, float* state_out, int batch, int seqlen,
                                  int channels, int dtype, jamba_stream_t stream);
 
+/* in_proj with the causal conv1d + SiLU in its epilogue (bf16): the first step
+ * of jamba_mamba_prefill on a bf16 handle, as its own call (Jamba section 2's
+ * Mamba layer: in_proj, then the conv over the x half).  Two launches: the
+ * tcgen05 GEMM, whose epilogue runs the conv over each 32-token slab it
+ * holds, and a small kernel for the rows 0-2 of each slab whose window reaches
+ * the slab above.
+ *   u [batch * seqlen, d_model] bf16; w_in [2 * d_inner, d_model] bf16 (x rows, then z rows)
+ *   conv_w [d_inner, 4], conv_b [d_inner] bf16, 16-byte aligned
+ *   xz [batch * seqlen, 2 * d_inner] bf16: z in columns d_inner.. (its x
+ *      columns are scratch: raw x of six rows in every 32)
+ *   xc [batch * seqlen, d_inner] bf16: SiLU(conv(x)), x the bf16 in_proj output
+ *   state_in / state_out [batch, d_inner, 3] fp32 or NULL, not aliased (as in
+ *      jamba_mamba_prefill)
+ * JAMBA_ERR_UNSUPPORTED unless seqlen >= 3 and d_inner is a multiple of 32 of
+ * at least 128 (jamba_gemm then jamba_causal_conv1d compute the same). */
+jamba_status jamba_in_proj_conv1d(const void* u, const void* w_in, const void* conv_w, const void* conv_b,
+                                  void* xz, void* xc, const float* state_in, float* state_out, int batch,
+                                  int seqlen, int d_model, int d_inner, jamba_stream_t stream);
+
 /* Dense GEMM out = a @ b^T (+ residual) on the sm_100a tensor cores (bf16) or
  * the CUDA cores (fp32).  a [m, k], b [n, k] row-major; out [m, n] row stride
  * ld_out; residual NULL or [m, n] with the same stride.  out_dtype may differ

@@ -88,6 +88,7 @@ SIGNATURES = {
                                             ctypes.c_ulonglong, P, SZ, P],
     "jamba_rmsnorm": [P, P, P, I, I, F, I, P],
     "jamba_causal_conv1d": [P, I, P, P, P, P, P, I, I, I, I, P],
+    "jamba_in_proj_conv1d": [P, P, P, P, P, P, P, P, I, I, I, I, P],
     "jamba_gemm": [P, P, P, I, P, I, I, I, I, I, P],
     "jamba_quantize_int8_rows": [P, I, ctypes.c_longlong, I, P, P, P],
     "jamba_moe_workspace_size": [ctypes.POINTER(MoeConfig), I, ctypes.POINTER(SZ)],

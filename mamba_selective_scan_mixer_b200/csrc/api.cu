@@ -256,6 +256,19 @@ jamba_status reorder_channels(jamba_mamba* h) {
 // The weights the prefill runs on: the reordered copy when the handle has one.
 const jamba_mamba_weights& prefill_weights(const jamba_mamba& h) { return h.perm ? h.wp : h.w; }
 
+// bf16 in_proj with the conv + SiLU in its epilogue, then the slab rows it
+// deferred: z into xz (its x columns are scratch), SiLU(conv(x)) into xc.
+jamba_status in_proj_conv(const void* u, const void* w_in, const void* conv_w, const void* conv_b, void* xz, void* xc,
+                          const float* cin, float* cout, const int* perm, int T, int seqlen, int dm, int di,
+                          cudaStream_t s) {
+  GemmDesc g = gdesc(u, dm, w_in, dm, T, 2 * di, dm, EPI_CONVP, xz, 2 * di);
+  g.conv_w = conv_w; g.conv_b = conv_b; g.xc_out = xc; g.conv_c = di;
+  g.conv_in = cin; g.conv_out = cout; g.conv_perm = perm; g.conv_L = seqlen;
+  JB_TRY(gemm_bf16(g, s));
+  NvtxRange r("conv1d_slab_rows");
+  return conv_fixup(xz, 2 * di, conv_w, conv_b, xc, cin, T, seqlen, di, perm, s);
+}
+
 // The prefill's first steps: in_proj, conv + SiLU (cache in -> out), x_proj
 // into split-K partials (p.xpart, p.splits of them).
 jamba_status prefill_front_a(const jamba_mamba& h, const PrefillWs& p, const void* u, int batch, int seqlen,
@@ -265,19 +278,29 @@ jamba_status prefill_front_a(const jamba_mamba& h, const PrefillWs& p, const voi
   const int T = batch * seqlen, di = c.d_inner, dm = c.d_model, R = c.dt_rank, N = c.d_state;
   const int W = R + 2 * N;
   NvtxSteps nv;
-  // in_proj: xz = u W_in^T
-  nv.next("in_proj");
-  JB_TRY(gemm_any(c.dtype, gdesc(u, dm, w.in_proj, dm, T, 2 * di, dm, c.dtype == JAMBA_BF16 ? EPI_BF16 : EPI_F32,
-                                 p.xz, 2 * di), s));
-  // conv + SiLU (cache in -> out; an aliased cache is copied first)
-  nv.next("conv1d");
+  // the conv cache in: an aliased one is copied first (the new cache is
+  // written while the old one is still read)
   const float* cin = conv_state_in;
   if (cin && cin == conv_state_out) {
     JB_CUDA(cudaMemcpyAsync(p.conv_tmp, cin, sizeof(float) * (size_t)batch * di * 3, cudaMemcpyDeviceToDevice, s));
     cin = p.conv_tmp;
   }
-  JB_TRY(conv_prefill(p.xz, 2 * di, w.conv_w, w.conv_b, p.xc, cin, conv_state_out, batch, seqlen, di, c.dtype,
-                      h.perm, s));
+  if (c.dtype == JAMBA_BF16 && seqlen >= 3 && di % 32 == 0 && di >= 128 && aligned16(w.conv_w) &&
+      aligned16(w.conv_b)) {
+    // in_proj with the conv + SiLU in its epilogue: z into xz, xc directly;
+    // the few rows whose window crosses a 32-row slab are finished after it
+    nv.next("in_proj_conv1d");
+    JB_TRY(in_proj_conv(u, w.in_proj, w.conv_w, w.conv_b, p.xz, p.xc, cin, conv_state_out, h.perm, T, seqlen, dm,
+                        di, s));
+  } else {
+    // in_proj: xz = u W_in^T, then conv + SiLU (cache in -> out)
+    nv.next("in_proj");
+    JB_TRY(gemm_any(c.dtype, gdesc(u, dm, w.in_proj, dm, T, 2 * di, dm, c.dtype == JAMBA_BF16 ? EPI_BF16 : EPI_F32,
+                                   p.xz, 2 * di), s));
+    nv.next("conv1d");
+    JB_TRY(conv_prefill(p.xz, 2 * di, w.conv_w, w.conv_b, p.xc, cin, conv_state_out, batch, seqlen, di, c.dtype,
+                        h.perm, s));
+  }
   // x_proj (split-K partials) -> sum + inner RMSNorms
   nv.next("x_proj");
   GemmDesc gx = gdesc(p.xc, di, w.x_proj, di, T, W, di, EPI_F32, p.xpart, W);
@@ -964,6 +987,30 @@ jamba_status jamba_causal_conv1d(const void* x, int ld_x, const void* w, const v
   if (state_in && state_in == state_out)
     return fail(JAMBA_ERR_INVALID_ARG, "conv: state_in and state_out may not alias here");
   return conv_prefill(x, ld_x, w, b, out, state_in, state_out, batch, seqlen, channels, dtype, nullptr, cs(stream));
+}
+
+jamba_status jamba_in_proj_conv1d(const void* u, const void* w_in, const void* conv_w, const void* conv_b, void* xz,
+                                  void* xc, const float* state_in, float* state_out, int batch, int seqlen,
+                                  int d_model, int d_inner, jamba_stream_t stream) {
+  JB_RANGE("jamba_in_proj_conv1d");
+  if (batch <= 0 || seqlen <= 0 || d_model <= 0 || d_inner <= 0)
+    return fail(JAMBA_ERR_INVALID_ARG, "in_proj conv: sizes must be positive");
+  JB_TRY(check_ptr(u, "u"));
+  JB_TRY(check_ptr(w_in, "w_in"));
+  JB_TRY(check_ptr(conv_w, "conv_w"));
+  JB_TRY(check_ptr(conv_b, "conv_b"));
+  JB_TRY(check_ptr(xz, "xz"));
+  JB_TRY(check_ptr(xc, "xc"));
+  JB_TRY(check_ptr(state_in, "state_in", false));
+  JB_TRY(check_ptr(state_out, "state_out", false));
+  if (state_in && state_in == state_out)
+    return fail(JAMBA_ERR_INVALID_ARG, "in_proj conv: state_in and state_out may not alias here");
+  if ((long long)batch * seqlen > (1LL << 31) / 2) return fail(JAMBA_ERR_UNSUPPORTED, "in_proj conv: too many tokens");
+  if (seqlen < 3 || d_inner % 32 || d_inner < 128 || !aligned16(conv_w) || !aligned16(conv_b))
+    return fail(JAMBA_ERR_UNSUPPORTED, "in_proj conv: needs seqlen >= 3, d_inner a multiple of 32 (>= 128) and "
+                                       "16-byte aligned conv weights");
+  return in_proj_conv(u, w_in, conv_w, conv_b, xz, xc, state_in, state_out, nullptr, batch * seqlen, seqlen, d_model,
+                      d_inner, cs(stream));
 }
 
 jamba_status jamba_gemm(const void* a, const void* b, void* out, int ld_out, const void* residual, int m, int n,

@@ -162,6 +162,103 @@ conv_halo_kernel(const T* __restrict__ xz, long long ld, float* __restrict__ sta
   state[i] = to_f(xz[((long long)b * 3 + k) * ld + c]);
 }
 
+// The rows an EPI_CONVP in_proj epilogue deferred: in each 32-row slab, rows
+// j = 0..2 whose position t in their sequence exceeds j (their window reaches
+// the slab above).  The epilogue left the raw x of slab rows 0-2 and 29-31 in
+// the x columns of xz; taps before the sequence start come from the cache.
+// A thread owns 8 channels and walks the slabs s = blockIdx.y, += gridDim.y
+// (one wave of blocks), the six raw rows of the next slab in
+// flight while the current one is computed.
+constexpr int FIX_THREADS = 128;
+
+__device__ __forceinline__ void fix_load(const bf16* __restrict__ xz, long long ld, int c0, int T, int s,
+                                         uint4 (&raw)[6]) {
+#pragma unroll
+  for (int r = 0; r < 6; ++r) {
+    const int row = s * 32 - 3 + r;
+    raw[r] = row >= 0 && row < T ? *reinterpret_cast<const uint4*>(xz + (long long)row * ld + c0) : make_uint4(0, 0, 0, 0);
+  }
+}
+
+__global__ void __launch_bounds__(FIX_THREADS)
+conv_fixup_kernel(const bf16* __restrict__ xz, long long ld, const bf16* __restrict__ w, const bf16* __restrict__ bias,
+                  bf16* __restrict__ xc, const float* __restrict__ st_in, int T, int L, int C,
+                  const int* __restrict__ perm, int* err) {
+  griddep_wait();
+  griddep_launch();
+  const int c0 = (blockIdx.x * FIX_THREADS + threadIdx.x) * 8;
+  if (c0 >= C) return;
+  const int slabs = (T + 31) / 32;
+  int s = blockIdx.y;
+  if (s >= slabs) return;
+  uint4 cur[6], nxt[6];
+  fix_load(xz, ld, c0, T, s, cur);
+  float wk[4][8], bv[8];
+  {
+    const uint4* wq = reinterpret_cast<const uint4*>(w + (long long)c0 * 4);   // 8 channels x 4 taps
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float f[8];
+      Vec16<bf16>::load(reinterpret_cast<const bf16*>(wq + q), f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) wk[e & 3][2 * q + (e >> 2)] = f[e];
+    }
+    Vec16<bf16>::load(bias + c0, bv);
+  }
+  for (; s < slabs; s += gridDim.y) {
+    const int sn = s + gridDim.y;
+    if (sn < slabs) fix_load(xz, ld, c0, T, sn, nxt);
+    float xw[6][8];
+#pragma unroll
+    for (int r = 0; r < 6; ++r) Vec16<bf16>::load(reinterpret_cast<const bf16*>(&cur[r]), xw[r]);
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+      const int m = s * 32 + j;
+      if (m >= T) break;
+      const int b = m / L, t = m - b * L;
+      if (t <= j) continue;   // computed by the epilogue
+      float o[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float x[4];   // x[t-3], x[t-2], x[t-1], x[t]
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int tk = t - 3 + k;
+          if (tk >= 0) {
+            x[k] = xw[j + k][i];
+          } else {
+            const int cn = perm ? __ldg(perm + c0 + i) : c0 + i;
+            x[k] = st_in && checked(cn >= 0 && cn < C, err) ? st_in[((long long)b * C + cn) * 3 + (3 + tk)] : 0.f;
+          }
+        }
+        float acc = bv[i];
+        acc = fmaf(wk[0][i], x[0], acc);
+        acc = fmaf(wk[1][i], x[1], acc);
+        acc = fmaf(wk[2][i], x[2], acc);
+        acc = fmaf(wk[3][i], x[3], acc);
+        o[i] = silu(acc);
+      }
+      Vec16<bf16>::store(xc + (long long)m * C + c0, o);
+    }
+#pragma unroll
+    for (int r = 0; r < 6; ++r) cur[r] = nxt[r];
+  }
+}
+
+jamba_status conv_fixup(const void* xz, long long ld, const void* w, const void* b, void* xc, const float* st_in,
+                        int T, int L, int C, const int* perm, cudaStream_t s) {
+  if (C % 8 || ld % 8 || !aligned16(xz) || !aligned16(xc) || !aligned16(w) || !aligned16(b) || L < 1)
+    return fail(JAMBA_ERR_INVALID_ARG, "conv fix-up: channels and row stride must fill 16-byte vectors");
+  const int slabs = (T + 31) / 32;
+  const int cblocks = (C / 8 + FIX_THREADS - 1) / FIX_THREADS;
+  int sy = 3 * num_sms() / cblocks;   // one wave: three blocks per SM (156 registers a thread)
+  sy = sy < 1 ? 1 : sy > slabs ? slabs : sy;
+  JB_CUDA(launch_pdl(conv_fixup_kernel, dim3(cblocks, sy), dim3(FIX_THREADS), 0, s, reinterpret_cast<const bf16*>(xz),
+                     ld, reinterpret_cast<const bf16*>(w), reinterpret_cast<const bf16*>(b), reinterpret_cast<bf16*>(xc),
+                     st_in, T, L, C, perm, device_error_word()));
+  return JAMBA_OK;
+}
+
 jamba_status conv_halo_state(const void* xz, long long ld, float* state, int batch, int C, int dtype,
                              cudaStream_t s) {
   const long long n = (long long)batch * C * 3;

@@ -69,7 +69,7 @@ static jamba_status launch_bn(int bn, const CUtensorMap& ma, const CUtensorMap& 
     // short), fed; three ring stages and one TMA-store box per epilogue warp
     // share the 227 KB
     if (bn == 256) return launch_tc<256, 3, EPI, false, 16>(ma, mb, mb2, mc, p, grid, s);
-  } else if constexpr (EPI == EPI_SWIGLU) {
+  } else if constexpr (EPI == EPI_SWIGLU || EPI == EPI_CONVP) {
     if (bn == 256) return launch_tc<256, 4, EPI, false>(ma, mb, mb2, mc, p, grid, s);
   } else {
     switch (bn) {
@@ -176,7 +176,7 @@ jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
   if (g.K % 8 || g.lda % 8 || g.ldb % 8 || !aligned16(g.a) || !aligned16(g.b))
     return fail(JAMBA_ERR_INVALID_ARG, "gemm: K and leading dimensions must be multiples of 8, operands 16-byte aligned");
   if (!g.transpose_out && !aligned16(g.out)) return fail(JAMBA_ERR_INVALID_ARG, "gemm: output must be 16-byte aligned");
-  if (!g.transpose_out && ((g.epi == EPI_BF16 || g.epi == EPI_SWIGLU) ? g.ldo % 8 : g.ldo % 4))
+  if (!g.transpose_out && ((g.epi == EPI_BF16 || g.epi == EPI_SWIGLU || g.epi == EPI_CONVP) ? g.ldo % 8 : g.ldo % 4))
     return fail(JAMBA_ERR_INVALID_ARG, "gemm: output leading dimension breaks 16-byte rows");
   if (g.residual && (g.transpose_out || g.epi != EPI_BF16 || g.ldr % 8 || !aligned16(g.residual)))
     return fail(JAMBA_ERR_INVALID_ARG, "gemm: residual only with aligned non-transposed bf16 output");
@@ -188,8 +188,15 @@ jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
                             !g.xc_out || g.conv_c <= 0 || g.conv_c > g.M ||
                             (reinterpret_cast<uintptr_t>(g.conv_w) & 7)))
     return fail(JAMBA_ERR_INVALID_ARG, "gemm: the conv epilogue needs a swap-AB GEMM and its conv operands");
+  if (g.epi == EPI_CONVP &&
+      (g.transpose_out || g.grouped || g.splits > 1 || g.residual || !g.conv_w || !g.conv_b || !g.xc_out ||
+       g.conv_c <= 0 || g.conv_c % 32 || g.N != 2 * g.conv_c || g.conv_L < 3 || g.M % g.conv_L ||
+       !aligned16(g.conv_w) || (reinterpret_cast<uintptr_t>(g.conv_b) & 3) || !aligned16(g.xc_out) ||
+       (g.bn && g.bn != 256)))
+    return fail(JAMBA_ERR_INVALID_ARG, "gemm: the prefill conv epilogue needs x|z columns (2 x a multiple of 32), "
+                                       "sequences of at least 3 rows and aligned conv operands");
   if (g.b_int8) return gemm_i8w(g, s);
-  int bn = g.bn;
+  int bn = g.epi == EPI_CONVP ? 256 : g.bn;
   if (bn == 0) {
     if (g.epi == EPI_SWIGLU || g.epi == EPI_SOFTPLUS) bn = g.transpose_out ? 64 : 256;
     else if (g.transpose_out || g.N <= 64) bn = 64;
@@ -265,6 +272,10 @@ jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
   p.conv_state = g.conv_state;
   p.xc_out = reinterpret_cast<bf16*>(g.xc_out);
   p.conv_c = g.conv_c;
+  p.conv_in = g.conv_in;
+  p.conv_out = g.conv_out;
+  p.conv_perm = g.conv_perm;
+  p.conv_L = g.conv_L;
   p.err = device_error_word();
   if (!p.err) return fail(JAMBA_ERR_CUDA, "could not allocate the device status word");
 
@@ -285,6 +296,7 @@ jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s) {
       case EPI_F32: return launch_bn<EPI_F32, false>(bn, ma, mb, mb2, mc, p, grid, s);
       case EPI_SOFTPLUS: return launch_bn<EPI_SOFTPLUS, false>(bn, ma, mb, mb2, mc, p, grid, s);
       case EPI_SWIGLU: return launch_bn<EPI_SWIGLU, false>(bn, ma, mb, mb2, mc, p, grid, s);
+      case EPI_CONVP: return launch_bn<EPI_CONVP, false>(bn, ma, mb, mb2, mc, p, grid, s);
       default: break;
     }
   }

@@ -21,7 +21,7 @@
 
 namespace jb {
 
-enum EpiKind : int { EPI_BF16 = 0, EPI_F32 = 1, EPI_SOFTPLUS = 2, EPI_SWIGLU = 3, EPI_CONV = 4 };
+enum EpiKind : int { EPI_BF16 = 0, EPI_F32 = 1, EPI_SOFTPLUS = 2, EPI_SWIGLU = 3, EPI_CONV = 4, EPI_CONVP = 5 };
 
 constexpr int GEMM_THREADS = 320;
 constexpr int GEMM_EPI_WARPS = 8;
@@ -52,6 +52,16 @@ struct GemmParams {
   float* conv_state;
   bf16* xc_out;
   int conv_c;
+  // EPI_CONVP (prefill in_proj, rows = tokens b * conv_L + t, N = 2 conv_c):
+  // columns n < conv_c are x, the causal conv + SiLU of which goes to xc_out
+  // [M, conv_c]; columns >= conv_c (z) are stored into out as in EPI_BF16.
+  // conv_in [M / conv_L, conv_c, 3] (or null: zeros) holds the three inputs
+  // before each sequence, conv_out receives its last three; both indexed by
+  // the cache row conv_perm[c] of channel c (identity when null)
+  const float* conv_in;
+  float* conv_out;
+  const int* conv_perm;
+  int conv_L;
   int* err;
 };
 
@@ -196,9 +206,105 @@ __device__ __forceinline__ void scale32(float* v, const float* __restrict__ scal
   }
 }
 
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
+  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+
+template <int EPI, bool TRANS, int NC>
+__device__ __forceinline__ void epi_chunk(const GemmParams& p, const TileInfo& ti, int m, int n, const float* v);
+
+// EPI_CONVP, one 32-column chunk of row m (token t of sequence b).  The x
+// value is the bf16 activation, as an unfused conv would read it back.  A
+// warp holds 32 consecutive rows (a slab), so the three inputs before row m
+// are the lanes below it; where the window reaches above the slab inside the
+// same sequence (lanes 0-2 with t > lane) the row is deferred: its raw x, and
+// the raw x of lanes 29-31 of every slab, is stored into the x columns of out
+// for conv_fixup_kernel.  Taps before the sequence start come from conv_in.
+// The multiply-add order is the one of the standalone conv kernels.
+__device__ __forceinline__ void epi_conv_prefill(const GemmParams& p, const TileInfo& ti, int m, int n,
+                                                 const float* v) {
+  if (n >= p.conv_c) {   // z columns (the chunk is all x or all z: conv_c % 32 == 0)
+    epi_chunk<EPI_BF16, false, 32>(p, ti, m, n, v);
+    return;
+  }
+  const int lane = threadIdx.x & 31;
+  uint32_t r0[16], r1[16], r2[16], r3[16];   // bf16 pairs of rows m, m-1, m-2, m-3
+#pragma unroll
+  for (int i = 0; i < 16; ++i) r0[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    r1[i] = __shfl_up_sync(0xffffffffu, r0[i], 1);
+    r2[i] = __shfl_up_sync(0xffffffffu, r0[i], 2);
+    r3[i] = __shfl_up_sync(0xffffffffu, r0[i], 3);
+  }
+  if (m >= ti.m_end) return;
+  const int L = p.conv_L, C = p.conv_c;
+  const int b = m / L, t = m - b * L;
+  const bool deferred = lane < 3 && t > lane;
+  if (deferred || lane >= 29) {
+    uint4* xo = reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(p.out) + (long long)m * p.ldo + n);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) xo[k] = make_uint4(r0[4 * k], r0[4 * k + 1], r0[4 * k + 2], r0[4 * k + 3]);
+  }
+  if (p.conv_out && t >= L - 3) {   // the cache after this sequence: its last three inputs
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float2 x = unpack_bf16x2(r0[i]);
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int c = n + 2 * i + e;
+        const int cn = p.conv_perm ? __ldg(p.conv_perm + c) : c;
+        if (checked(cn >= 0 && cn < C, p.err)) p.conv_out[((long long)b * C + cn) * 3 + (t - (L - 3))] = e ? x.y : x.x;
+      }
+    }
+  }
+  if (deferred) return;
+  uint4* xc = reinterpret_cast<uint4*>(p.xc_out + (long long)m * C + n);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int i = 4 * k + q;
+      const uint4 wq = __ldg(reinterpret_cast<const uint4*>(p.conv_w + (long long)(n + 2 * i) * 4));
+      const float2 w01 = unpack_bf16x2(wq.x), w23 = unpack_bf16x2(wq.y);   // channel n + 2i
+      const float2 u01 = unpack_bf16x2(wq.z), u23 = unpack_bf16x2(wq.w);   // channel n + 2i + 1
+      float2 acc = unpack_bf16x2(__ldg(reinterpret_cast<const uint32_t*>(p.conv_b + n + 2 * i)));
+      float2 x3 = unpack_bf16x2(r3[i]), x2 = unpack_bf16x2(r2[i]), x1 = unpack_bf16x2(r1[i]);
+      if (t < 3) {   // taps before the sequence start: the cache (exact fp32 values)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int c = n + 2 * i + e;
+          const int cn = p.conv_perm ? __ldg(p.conv_perm + c) : c;
+          const float* ci = p.conv_in && checked(cn >= 0 && cn < C, p.err) ? p.conv_in + ((long long)b * C + cn) * 3
+                                                                           : nullptr;
+          const float s3 = ci ? ci[t] : 0.f, s2 = ci && t < 2 ? ci[t + 1] : 0.f, s1 = ci && t < 1 ? ci[t + 2] : 0.f;
+          if (e) { x3.y = s3; if (t < 2) x2.y = s2; if (t < 1) x1.y = s1; }
+          else   { x3.x = s3; if (t < 2) x2.x = s2; if (t < 1) x1.x = s1; }
+        }
+      }
+      acc = ffma2(make_float2(w01.x, u01.x), x3, acc);
+      acc = ffma2(make_float2(w01.y, u01.y), x2, acc);
+      acc = ffma2(make_float2(w23.x, u23.x), x1, acc);
+      acc = ffma2(make_float2(w23.y, u23.y), unpack_bf16x2(r0[i]), acc);
+      o[q] = pack_bf16x2(silu(acc.x), silu(acc.y));
+    }
+    xc[k] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
 // Epilogue of one 32-column chunk held by this thread (row m, columns n..n+NC-1).
 template <int EPI, bool TRANS, int NC>
 __device__ __forceinline__ void epi_chunk(const GemmParams& p, const TileInfo& ti, int m, int n, const float* v) {
+  if constexpr (EPI == EPI_CONVP) {
+    static_assert(!TRANS && NC == 32, "the prefill conv epilogue works on whole 32-column chunks");
+    epi_conv_prefill(p, ti, m, n, v);
+    return;
+  }
   if (m >= ti.m_end) return;
   if constexpr (!TRANS) {
     if constexpr (EPI == EPI_BF16) {

@@ -116,6 +116,11 @@ struct GemmDesc {
   const float* scale_b2;  // ... and of b2
   // EPI_CONV (swap-AB only): decode conv fused into in_proj's epilogue
   const void* conv_w; const void* conv_b; float* conv_state; void* xc_out; int conv_c;
+  // EPI_CONVP (prefill in_proj, bf16): the conv + SiLU of the x columns in the
+  // epilogue (conv_w, conv_b, xc_out, conv_c as above); caches in / out per
+  // sequence of conv_L rows, cache row of channel c = conv_perm[c]; rows 0-2
+  // of 32-row slabs are completed by conv_fixup
+  const float* conv_in; float* conv_out; const int* conv_perm; int conv_L;
 };
 jamba_status gemm_bf16(const GemmDesc& g, cudaStream_t s);
 // k-splits that balance the fp32 expert GEMM with INT8 weights over the SMs
@@ -188,6 +193,11 @@ jamba_status conv_prefill(const void* x, long long ld_x, const void* w, const vo
                           cudaStream_t s);
 jamba_status conv_step(const void* x, long long ld_x, const void* w, const void* b, void* out, float* state,
                        int batch, int C, int dtype, cudaStream_t s);
+// After an EPI_CONVP in_proj: rows 0-2 of each 32-row slab whose conv window
+// reaches the slab above within their sequence, from the raw x the epilogue
+// left in the x columns of xz (row stride ld).
+jamba_status conv_fixup(const void* xz, long long ld, const void* w, const void* b, void* xc, const float* st_in,
+                        int T, int L, int C, const int* perm, cudaStream_t s);
 jamba_status conv_halo_state(const void* xz, long long ld, float* state, int batch, int C, int dtype,
                              cudaStream_t s);
 // Row and column gathers for reordering channel-indexed weights:

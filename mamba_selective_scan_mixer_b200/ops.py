@@ -302,6 +302,24 @@ def causal_conv1d(x, w, b, state_in=None, want_state=True, stream=None):
     return out, st
 
 
+def in_proj_conv1d(u, w_in, conv_w, conv_b, state_in=None, state_out=None, xz=None, xc=None, stream=None):
+    """bf16 u [batch, L, d_model] -> (xc [batch, L, d_inner] = SiLU(conv(x)),
+    xz [batch, L, 2 d_inner] with z in its second half, state_out): in_proj
+    with the conv in its epilogue."""
+    _cuda(u, w_in, conv_w, conv_b, state_in, state_out, xz, xc)
+    _contig(u, "u")
+    _contig(w_in, "w_in")
+    batch, L, dm = u.shape
+    di = w_in.shape[0] // 2
+    xz = torch.empty(batch, L, 2 * di, dtype=u.dtype, device=u.device) if xz is None else xz
+    xc = torch.empty(batch, L, di, dtype=u.dtype, device=u.device) if xc is None else xc
+    _contig(xz, "xz")
+    _contig(xc, "xc")
+    check(lib().jamba_in_proj_conv1d(_p(u), _p(w_in), _p(conv_w), _p(conv_b), _p(xz), _p(xc), _p(state_in),
+                                     _p(state_out), batch, L, dm, di, _stream(stream)))
+    return xc, xz, state_out
+
+
 def gemm(a, b, residual=None, out_dtype=None, out=None, stream=None):
     """a [m, k] @ b[n, k]^T (+ residual) on the tensor cores (bf16) or CUDA cores (fp32)."""
     _cuda(a, b, residual, out)

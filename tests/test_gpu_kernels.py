@@ -85,6 +85,55 @@ def test_conv_prefill(dev, dtype, L, with_state):
     np.testing.assert_array_equal(to_np(st_out), want_st)   # cached inputs are copied exactly
 
 
+@pytest.mark.parametrize("batch,L,di", [(3, 37, 256), (1, 3, 128), (2, 100, 384), (5, 7, 256), (1, 300, 256)])
+def test_in_proj_conv1d(dev, batch, L, di):
+    """in_proj with the conv in its epilogue: against the oracle (x|z
+    projection, conv over the bf16 x, caches), row by row for the conv output
+    (rows 0-2 of each 32-row slab are finished by a second kernel; short
+    sequences put their starts at every lane), and bit for bit against
+    jamba_gemm followed by jamba_causal_conv1d, which round and add in the
+    same order.  The cache in holds arbitrary fp32 values."""
+    import mamba_selective_scan_mixer_b200 as J
+    g = _gen(1000 + L)
+    dm = 256
+    u = torch.randn(batch, L, dm, generator=g).to(torch.bfloat16)
+    w_in = (0.05 * torch.randn(2 * di, dm, generator=g)).to(torch.bfloat16)
+    w = (0.5 * torch.randn(di, 4, generator=g)).to(torch.bfloat16)
+    b = (0.5 * torch.randn(di, generator=g)).to(torch.bfloat16)
+    st = torch.randn(batch, di, 3, generator=g)
+    st_out = torch.empty(batch, di, 3, device=dev)
+    xc, xz, _ = J.in_proj_conv1d(u.to(dev), w_in.to(dev), w.to(dev), b.to(dev), state_in=st.to(dev),
+                                 state_out=st_out)
+    xz64 = to_np(u) @ to_np(w_in).T
+    pre, want_st = om.causal_conv1d(xz64[..., :di], to_np(w), to_np(b), to_np(st))
+    want = om.silu(pre)
+    got = to_np(xc)
+    assert rel_l2(got, want) < TOL_BF16
+    row_err = (np.linalg.norm(got - want, axis=2) / np.linalg.norm(want, axis=2)).ravel()
+    assert row_err.max() < 2e-2, (int(row_err.argmax()), float(row_err.max()))
+    assert rel_l2(to_np(xz)[..., di:], xz64[..., di:]) < TOL_BF16
+    assert rel_l2(to_np(st_out), want_st) < TOL_BF16
+    # the unfused path on the same device: identical bits
+    xz2 = J.gemm(u.to(dev).view(batch * L, dm), w_in.to(dev)).view(batch, L, 2 * di)
+    xc2, st2 = J.causal_conv1d(xz2[..., :di], w.to(dev), b.to(dev), st.to(dev))
+    assert torch.equal(xc, xc2)
+    assert torch.equal(xz[..., di:], xz2[..., di:])
+    assert torch.equal(st_out, st2)
+
+
+def test_in_proj_conv1d_refuses_short_or_narrow(dev):
+    import mamba_selective_scan_mixer_b200 as J
+    from mamba_selective_scan_mixer_b200 import _abi
+    for L, di in ((2, 256), (40, 96), (40, 272)):
+        u = torch.zeros(1, L, 64, dtype=torch.bfloat16, device=dev)
+        w_in = torch.zeros(2 * di, 64, dtype=torch.bfloat16, device=dev)
+        w = torch.zeros(di, 4, dtype=torch.bfloat16, device=dev)
+        b = torch.zeros(di, dtype=torch.bfloat16, device=dev)
+        with pytest.raises(_abi.JambaError) as e:
+            J.in_proj_conv1d(u, w_in, w, b)
+        assert e.value.status == 2   # JAMBA_ERR_UNSUPPORTED
+
+
 # ------------------------------------------------------------------ scan
 
 def _scan_case(dev, batch, L, di, seed, dtype="bf16", bc="bf16", a_init="structured", h0=False, chunk=0,

@@ -245,3 +245,27 @@ def test_decode_b64_full_width_sampled_rows(dev):
     ref = om.mamba_prefill(p64, to_np(full), sh, scan="c")
     assert rel_l2(to_np(outs[rows]), ref["out"][:, L0:]) < TOL_BF16
     assert rel_l2(to_np(ss[rows]), ref["ssm_state"]) < TOL_BF16
+
+
+@pytest.mark.parametrize("batch,L", [(3, 37), (2, 3), (4, 5), (1, 100), (2, 2)])
+def test_prefill_conv_rows_through_x_proj(dev, batch, L):
+    """The conv inside the bf16 in_proj epilogue, row by row: a warp holds 32
+    token rows, so rows 0-2 of every 32-row slab whose window reaches the slab
+    above are finished by a second kernel, and rows near a sequence start take
+    their taps from the conv cache (random fp32 values here).  The x_proj
+    output of the tensor-parallel first part is linear in the conv output, so
+    each of its rows is compared with the oracle's on its own; short and
+    ragged sequences put sequence starts at every lane position.  L = 2 takes
+    the unfused path (fewer rows than the conv cache)."""
+    sh = MambaShape(d_model=256, d_inner=256, dt_rank=16, dtype="bf16", inner_norm=False)
+    mix, p64 = _mixer(sh, 21, dev, a_init="random")
+    u = mamba_input(sh, batch, L, seed=21)
+    g = torch.Generator().manual_seed(22)
+    cs0 = torch.randn(batch, sh.d_inner, 3, generator=g)
+    part, cs = mix.prefill_tp_begin(u.to(dev), conv_state_in=cs0.to(dev))
+    ref = om.mamba_prefill(p64, to_np(u), sh, conv_state0=cs0.double().numpy(), keep=True)
+    want = ref["proj"].reshape(batch * L, -1)
+    got = to_np(part)
+    row_err = np.linalg.norm(got - want, axis=1) / np.linalg.norm(want, axis=1)
+    assert row_err.max() < 2e-2, (int(row_err.argmax()), float(row_err.max()))
+    assert rel_l2(to_np(cs), ref["conv_state"]) < TOL_BF16
