@@ -101,6 +101,52 @@ xproj_norm_kernel(const float* __restrict__ part, int splits, long long split_st
   }
 }
 
+// The same for one partial (the prefill's x_proj has no k-split at large T):
+// a warp per token, lane l holding columns l, l + 32, ... (at most 16 of them),
+// so there is no block barrier and a block covers eight tokens.
+template <typename TD>
+__global__ void __launch_bounds__(256)
+xproj_norm_rows_kernel(const float* __restrict__ x, int T, int R, int N, const float* __restrict__ w_dt,
+                       const float* __restrict__ w_B, const float* __restrict__ w_C, int inner_norm, float eps,
+                       TD* __restrict__ dtlow, float* __restrict__ bc) {
+  griddep_wait();
+  griddep_launch();
+  const long long t = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const int lane = threadIdx.x & 31, W = R + 2 * N;
+  const float* xr = x + t * W;
+  float v[16];
+  float sq[3] = {0.f, 0.f, 0.f};
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int col = lane + 32 * i;
+    v[i] = col < W ? xr[col] : 0.f;
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int col = lane + 32 * i;
+    const int seg = col < R ? 0 : (col < R + N ? 1 : 2);
+    if (col < W) sq[seg] = fmaf(v[i], v[i], sq[seg]);
+  }
+  float inv[3] = {1.f, 1.f, 1.f};
+  if (inner_norm) {
+#pragma unroll
+    for (int k = 0; k < 3; ++k) inv[k] = rsqrtf(warp_sum(sq[k]) / (float)(k == 0 ? R : N) + eps);
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int col = lane + 32 * i;
+    if (col >= W) break;
+    if (col < R) {
+      dtlow[t * R + col] = from_f<TD>(inner_norm ? v[i] * inv[0] * w_dt[col] : v[i]);
+    } else if (col < R + N) {
+      bc[t * 2 * N + (col - R)] = inner_norm ? v[i] * inv[1] * w_B[col - R] : v[i];
+    } else {
+      bc[t * 2 * N + (col - R)] = inner_norm ? v[i] * inv[2] * w_C[col - R - N] : v[i];
+    }
+  }
+}
+
 // out[r, c] = sum_s part[s][r][c] (+ residual[r, c])
 template <typename T>
 __global__ void __launch_bounds__(256)
@@ -138,6 +184,16 @@ jamba_status xproj_norm(const float* part, int splits, long long split_stride, i
                         const float* w_dt, const float* w_B, const float* w_C, int inner_norm, float eps,
                         void* dtlow, float* bc, int dtype, cudaStream_t s) {
   if (R + 2 * N > 512) return fail(JAMBA_ERR_UNSUPPORTED, "x_proj width above 512");
+  if (splits == 1 && T >= 1024) {
+    const unsigned grid = (unsigned)((T + 7) / 8);
+    if (dtype == JAMBA_BF16)
+      JB_CUDA(launch_pdl(xproj_norm_rows_kernel<bf16>, dim3(grid), dim3(256), 0, s, part, T, R, N, w_dt, w_B, w_C,
+                         inner_norm, eps, reinterpret_cast<bf16*>(dtlow), bc));
+    else
+      JB_CUDA(launch_pdl(xproj_norm_rows_kernel<float>, dim3(grid), dim3(256), 0, s, part, T, R, N, w_dt, w_B, w_C,
+                         inner_norm, eps, reinterpret_cast<float*>(dtlow), bc));
+    return JAMBA_OK;
+  }
   const int threads = ((R + 2 * N + 31) / 32) * 32;
   if (dtype == JAMBA_BF16)
     JB_CUDA(launch_pdl(xproj_norm_kernel<bf16>, dim3(T), dim3(threads), 0, s, part, splits, split_stride, T, R, N, w_dt,

@@ -269,3 +269,17 @@ def test_prefill_conv_rows_through_x_proj(dev, batch, L):
     row_err = np.linalg.norm(got - want, axis=1) / np.linalg.norm(want, axis=1)
     assert row_err.max() < 2e-2, (int(row_err.argmax()), float(row_err.max()))
     assert rel_l2(to_np(cs), ref["conv_state"]) < TOL_BF16
+
+
+def test_bf16_prefill_long_unsplit_x_proj(dev):
+    """20000 tokens at d_inner 512: x_proj has enough tiles to run without a
+    k-split, and its sum + inner norms take the warp-per-token kernel
+    (random norm weights, so each of the three segments is checked)."""
+    sh = MambaShape(d_model=256, d_inner=512, dt_rank=32, dtype="bf16", inner_norm=True)
+    mix, p64 = _mixer(sh, 31, dev, norm_init="random", a_init="random")
+    u = mamba_input(sh, 1, 20000, seed=31)
+    out, cs, ss = mix.prefill(u.to(dev))
+    ref = om.mamba_prefill(p64, to_np(u), sh)
+    assert rel_l2(to_np(out), ref["out"]) < TOL_BF16
+    assert rel_l2(to_np(ss), ref["ssm_state"]) < TOL_BF16
+    assert rel_l2(to_np(cs), ref["conv_state"]) < TOL_BF16
