@@ -509,7 +509,6 @@ jamba_status jamba_mamba_prefill(jamba_mamba_t h, const void* u, const void* res
   JB_TRY(check_ptr(ssm_state_out, "ssm_state_out", false));
   JB_TRY(check_ptr(ws, "workspace"));
   if (u == out) return fail(JAMBA_ERR_INVALID_ARG, "prefill: out may not alias u");
-  const jamba_mamba_config& c = h->cfg;
   if ((long long)batch * seqlen > (1LL << 31) / 2) return fail(JAMBA_ERR_UNSUPPORTED, "prefill: too many tokens");
   PrefillWs p = carve_prefill(h, batch, seqlen, ws);
   if (ws_bytes < p.total) return fail(JAMBA_ERR_WORKSPACE, "prefill: workspace too small");
