@@ -11,11 +11,11 @@
 //              32-column chunks between them; tcgen05.ld, fused elementwise
 //              op, stores to global memory.
 // The epilogue kind is a template parameter, so each instantiation carries
-// only its own epilogue code.  Used for in_proj, x_proj, dt_proj
-// (+bias+softplus), out_proj (+residual), the decode projections (swap-AB:
-// weights as A so the 64-row token batch is the N side, stored transposed)
-// and the grouped MoE expert GEMMs (SwiGLU epilogue).  Every wait is bounded
-// (see common.cuh).
+// only its own epilogue code.  Used for in_proj (+ causal conv + SiLU of the
+// x columns), x_proj, dt_proj (+bias+softplus), out_proj (+residual), the
+// decode projections (swap-AB: weights as A so the 64-row token batch is the
+// N side, stored transposed; in_proj + conv step) and the grouped MoE expert
+// GEMMs (SwiGLU epilogue).  Every wait is bounded (see common.cuh).
 #pragma once
 #include "common.cuh"
 
