@@ -150,6 +150,31 @@ def test_bf16_decode_shapes(dev, dt_rank, batch, inner_norm, a_init):
     assert rel_l2(to_np(cs), ref["conv_state"]) < TOL_BF16
 
 
+@pytest.mark.parametrize("batch", [65, 7])
+def test_bf16_decode_residual(dev, batch):
+    """decode steps with a residual (added in the split-K sum of out_proj;
+    batch 65: a ragged second token tile) and without one, against the
+    oracle; the caches are the same either way"""
+    sh = MambaShape(d_model=512, d_inner=1024, dt_rank=64, dtype="bf16", inner_norm=True)
+    mix, p64 = _mixer(sh, 17, dev, a_init="random", norm_init="random")
+    L0, S = 16, 4
+    u = mamba_input(sh, batch, L0, seed=17)
+    steps = decode_inputs(sh, batch, S, seed=17)
+    res = decode_inputs(sh, batch, S, seed=18)
+    _, cs, ss = mix.prefill(u.to(dev))
+    cs2, ss2 = cs.clone(), ss.clone()
+    outs, plain = [], []
+    for t in range(S):
+        outs.append(to_np(mix.step(steps[t].to(dev), cs, ss, residual=res[t].to(dev))))
+        plain.append(to_np(mix.step(steps[t].to(dev), cs2, ss2)))
+    full = torch.cat([u, steps.transpose(0, 1)], dim=1)
+    ref = om.mamba_prefill(p64, to_np(full), sh)
+    want = ref["out"][:, L0:] + np.stack([to_np(r) for r in res], 1)
+    assert rel_l2(np.stack(outs, 1), want) < TOL_BF16
+    assert rel_l2(np.stack(plain, 1), ref["out"][:, L0:]) < TOL_BF16
+    assert torch.equal(ss, ss2) and torch.equal(cs, cs2)
+
+
 def test_bf16_decode_mid_width(dev):
     """d_model 1024 / d_inner 2048, batch 8: the decode GEMMs at a width
     between the small cases and Jamba's"""
