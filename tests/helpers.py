@@ -20,6 +20,19 @@ def rel_l2(got, want):
     return float(np.linalg.norm((got - want).ravel()) / (den if den > 0 else 1.0))
 
 
+def bf16_steps(a, b):
+    """Largest distance between two arrays of bf16 values, in bf16 steps (the
+    spacing of bf16 numbers at the larger magnitude of each pair).  Two runs of
+    the scan whose chunk carries were folded in a different order round their
+    fp32 states differently in the last bits, so bf16 outputs may sit one step
+    apart."""
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    m = np.maximum(np.abs(a), np.abs(b))
+    step = 2.0 ** (np.floor(np.log2(np.where(m > 0, m, 1.0))) - 7)
+    return float((np.abs(a - b) / step).max()) if a.size else 0.0
+
+
 def to_np(t):
     return t.detach().to("cpu").double().numpy()
 

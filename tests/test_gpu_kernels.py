@@ -7,7 +7,7 @@ import torch
 
 from oracle import mamba as om
 from synthetic import scan_inputs
-from tests.helpers import TOL_BF16, TOL_F32, cuda_or_skip, rel_l2, to_np
+from tests.helpers import TOL_BF16, TOL_F32, bf16_steps, cuda_or_skip, rel_l2, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -263,7 +263,7 @@ def test_scan_state_in_place_and_partial_overlap(dev):
     torch.cuda.synchronize()
     J.device_status()
     assert rel_l2(to_np(h_in_place), to_np(h_sep)) < 1e-6
-    assert rel_l2(to_np(y), to_np(y_sep)) < 1e-5
+    assert bf16_steps(to_np(y), to_np(y_sep)) <= 1
     assert run(h[0], h.view(-1)[2048:6144].view(256, 16)) == 1    # partial overlap: JAMBA_ERR_INVALID_ARG
     J.device_status()
 

@@ -6,7 +6,7 @@ import torch
 
 from oracle import mamba as om
 from synthetic import MambaShape, decode_inputs, mamba_input, mamba_params, workload
-from tests.helpers import TOL_BF16, TOL_F32, cuda_or_skip, rel_l2, to_np
+from tests.helpers import TOL_BF16, TOL_F32, bf16_steps, cuda_or_skip, rel_l2, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -104,7 +104,7 @@ def test_bf16_prefill_reordered_channel_groups(dev):
     cs3, ss3 = cs.clone(), ss.clone()
     out3, _, _ = mix.prefill(ud[:, 700:].contiguous(), conv_state_in=cs3, ssm_state_in=ss3, conv_state_out=cs3,
                              ssm_state_out=ss3)
-    assert rel_l2(to_np(out3), to_np(out2)) < 1e-5
+    assert bf16_steps(to_np(out3), to_np(out2)) <= 1
     assert rel_l2(to_np(ss3), to_np(ss2)) < 1e-6
     assert torch.equal(cs3, cs2)
 
