@@ -167,8 +167,8 @@ conv_halo_kernel(const T* __restrict__ xz, long long ld, float* __restrict__ sta
 // the slab above).  The epilogue left the raw x of slab rows 0-2 and 29-31 in
 // the x columns of xz; taps before the sequence start come from the cache.
 // A thread owns 8 channels and walks the slabs s = blockIdx.y, += gridDim.y
-// (one wave of blocks), the six raw rows of the next two slabs in flight while
-// the current one is computed.
+// (one wave of blocks), the six raw rows of the next slab in
+// flight while the current one is computed.
 constexpr int FIX_THREADS = 128;
 
 __device__ __forceinline__ void fix_load(const bf16* __restrict__ xz, long long ld, int c0, int T, int s,
@@ -191,10 +191,8 @@ conv_fixup_kernel(const bf16* __restrict__ xz, long long ld, const bf16* __restr
   const int slabs = (T + 31) / 32;
   int s = blockIdx.y;
   if (s >= slabs) return;
-  const int G = gridDim.y;
-  uint4 cur[6], nx1[6], nx2[6];   // this slab's raw rows and the next two slabs' in flight
+  uint4 cur[6], nxt[6];
   fix_load(xz, ld, c0, T, s, cur);
-  if (s + G < slabs) fix_load(xz, ld, c0, T, s + G, nx1);
   float wk[4][8], bv[8];
   {
     const uint4* wq = reinterpret_cast<const uint4*>(w + (long long)c0 * 4);   // 8 channels x 4 taps
@@ -207,8 +205,12 @@ conv_fixup_kernel(const bf16* __restrict__ xz, long long ld, const bf16* __restr
     }
     Vec16<bf16>::load(bias + c0, bv);
   }
-  for (; s < slabs; s += G) {
-    if (s + 2 * G < slabs) fix_load(xz, ld, c0, T, s + 2 * G, nx2);
+  for (; s < slabs; s += gridDim.y) {
+    const int sn = s + gridDim.y;
+    if (sn < slabs) fix_load(xz, ld, c0, T, sn, nxt);
+    float xw[6][8];
+#pragma unroll
+    for (int r = 0; r < 6; ++r) Vec16<bf16>::load(reinterpret_cast<const bf16*>(&cur[r]), xw[r]);
 #pragma unroll
     for (int j = 0; j < 3; ++j) {
       const int m = s * 32 + j;
@@ -218,13 +220,12 @@ conv_fixup_kernel(const bf16* __restrict__ xz, long long ld, const bf16* __restr
       float o[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        float x[4];   // x[t-3], x[t-2], x[t-1], x[t]: raw rows j .. j + 3 of the window
+        float x[4];   // x[t-3], x[t-2], x[t-1], x[t]
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const int tk = t - 3 + k;
           if (tk >= 0) {
-            const uint32_t wd = (&cur[j + k].x)[i >> 1];
-            x[k] = __uint_as_float((i & 1) ? (wd & 0xffff0000u) : (wd << 16));
+            x[k] = xw[j + k][i];
           } else {
             const int cn = perm ? __ldg(perm + c0 + i) : c0 + i;
             x[k] = st_in && checked(cn >= 0 && cn < C, err) ? st_in[((long long)b * C + cn) * 3 + (3 + tk)] : 0.f;
@@ -240,10 +241,7 @@ conv_fixup_kernel(const bf16* __restrict__ xz, long long ld, const bf16* __restr
       Vec16<bf16>::store(xc + (long long)m * C + c0, o);
     }
 #pragma unroll
-    for (int r = 0; r < 6; ++r) {
-      cur[r] = nx1[r];
-      nx1[r] = nx2[r];
-    }
+    for (int r = 0; r < 6; ++r) cur[r] = nxt[r];
   }
 }
 
@@ -253,7 +251,7 @@ jamba_status conv_fixup(const void* xz, long long ld, const void* w, const void*
     return fail(JAMBA_ERR_INVALID_ARG, "conv fix-up: channels and row stride must fill 16-byte vectors");
   const int slabs = (T + 31) / 32;
   const int cblocks = (C / 8 + FIX_THREADS - 1) / FIX_THREADS;
-  int sy = 3 * num_sms() / cblocks;   // one wave: three blocks per SM (152 registers a thread)
+  int sy = 3 * num_sms() / cblocks;   // one wave: three blocks per SM (156 registers a thread)
   sy = sy < 1 ? 1 : sy > slabs ? slabs : sy;
   JB_CUDA(launch_pdl(conv_fixup_kernel, dim3(cblocks, sy), dim3(FIX_THREADS), 0, s, reinterpret_cast<const bf16*>(xz),
                      ld, reinterpret_cast<const bf16*>(w), reinterpret_cast<const bf16*>(b), reinterpret_cast<bf16*>(xc),
