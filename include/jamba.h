@@ -344,6 +344,18 @@ jamba_status jamba_selective_scan_static(const void* x, int ld_x, const void* z,
                                          void* y, int ld_y, float* h_out, int batch, int seqlen, int d_inner,
                                          int d_state, int dtype, int* status, jamba_stream_t stream);
 
+/* Test support for the host-side planner of the bf16 prefill's scan (no GPU
+ * needed): the per-group time chunks jamba_mamba_prefill gives `groups`
+ * channel groups of 256 for `batch` rows of `seqlen` steps when the channels
+ * of group g keep a carried state for about head[g] steps (groups ordered
+ * slowest first) and `slots` CTAs fit on the device at once.  On return
+ * *planned is the number of groups planned (0: the uniform chunking of
+ * jamba_selective_scan is used instead), chunks[g] and lens[g] (caller
+ * arrays of `groups` ints) their chunk count and length (a multiple of 16)
+ * for g < *planned.  Not part of the method. */
+jamba_status jamba_test_scan_plan(int batch, int seqlen, int groups, const float* head, int slots, int* chunks,
+                                  int* lens, int* planned);
+
 /* Test support for the bounded device waits (failure detection without a GPU
  * fault).  Runs jamba_selective_scan (same arguments, chunk > 0 and at least
  * two chunks) but launches no CTA for the first time chunk, so the flags of

@@ -927,6 +927,20 @@ jamba_status jamba_selective_scan(const void* x, int ld_x, const void* z, int ld
   return scan_run(sc, cs(stream));
 }
 
+jamba_status jamba_test_scan_plan(int batch, int seqlen, int groups, const float* head, int slots, int* chunks,
+                                  int* lens, int* planned) {
+  if (!head || !chunks || !lens || !planned || groups <= 0 || groups > SCAN_MAX_GROUPS)
+    return fail(JAMBA_ERR_INVALID_ARG, "scan plan: bad argument");
+  ScanSchedule sch;
+  scan_plan(batch, seqlen, groups, head, slots, &sch);
+  *planned = sch.n;
+  for (int g = 0; g < sch.n; ++g) {
+    chunks[g] = sch.chunks[g];
+    lens[g] = sch.len[g];
+  }
+  return JAMBA_OK;
+}
+
 jamba_status jamba_test_scan_missing_predecessor(const void* x, int ld_x, const void* z, int ld_z, const float* dt,
                                                  int ld_dt, const void* B, int ld_b, const void* C, int ld_c,
                                                  int bc_dtype, const float* A, const float* D, void* y, int ld_y,
