@@ -356,6 +356,15 @@ jamba_status jamba_selective_scan_static(const void* x, int ld_x, const void* z,
 jamba_status jamba_test_scan_plan(int batch, int seqlen, int groups, const float* head, int slots, int* chunks,
                                   int* lens, int* planned);
 
+/* Test support for the host-side k-split choices (no GPU needed; the SM count
+ * is the current device's, 148 without one): *splits is the k-split count of
+ * a dense M x N x K GEMM with N-wide tiles keeping at least min_k_tiles
+ * 64-deep steps per split (x_proj and out_proj at decode sizes), and
+ * *i8w_splits_out that of the ExpertsInt8 fp32 expert GEMM over num_groups
+ * experts whose weights take the M side.  Not part of the method. */
+jamba_status jamba_test_gemm_splits(int M, int N, int K, int bn, int min_k_tiles, int num_groups, int* splits,
+                                    int* i8w_splits_out);
+
 /* Test support for the bounded device waits (failure detection without a GPU
  * fault).  Runs jamba_selective_scan (same arguments, chunk > 0 and at least
  * two chunks) but launches no CTA for the first time chunk, so the flags of

@@ -941,6 +941,15 @@ jamba_status jamba_test_scan_plan(int batch, int seqlen, int groups, const float
   return JAMBA_OK;
 }
 
+jamba_status jamba_test_gemm_splits(int M, int N, int K, int bn, int min_k_tiles, int num_groups, int* splits,
+                                    int* i8w_splits_out) {
+  if (!splits || !i8w_splits_out || M <= 0 || N <= 0 || K <= 0 || bn <= 0 || num_groups <= 0)
+    return fail(JAMBA_ERR_INVALID_ARG, "gemm splits: bad argument");
+  *splits = choose_splits(M, N, K, bn, min_k_tiles);
+  *i8w_splits_out = i8w_splits(M, num_groups, N, K);
+  return JAMBA_OK;
+}
+
 jamba_status jamba_test_scan_missing_predecessor(const void* x, int ld_x, const void* z, int ld_z, const float* dt,
                                                  int ld_dt, const void* B, int ld_b, const void* C, int ld_c,
                                                  int bc_dtype, const float* A, const float* D, void* y, int ld_y,

@@ -1,6 +1,7 @@
 """Host-side logic of the library that needs no GPU: the planner that gives
 each channel group of the bf16 prefill's scan its own number of time chunks
-(through the test entry jamba_test_scan_plan).
+(through the test entry jamba_test_scan_plan), and the k-split choices of the
+decode-size GEMMs (jamba_test_gemm_splits).
 
 A CTA of the scan costs its chunk plus the head it replays: the steps until
 its slowest channel has lost the incoming state, at most the chunk.  The
@@ -96,3 +97,39 @@ def test_plan_rejects_bad_arguments(lib):
     n = ctypes.c_int()
     assert lib.jamba_test_scan_plan(1, 1000, 65, h, 444, c, c, ctypes.byref(n)) == 1   # more than 64 groups
     assert lib.jamba_test_scan_plan(1, 1000, 4, None, 444, c, c, ctypes.byref(n)) == 1
+
+
+def _splits(lib, M, N, K, bn, min_k, groups=1):
+    s, s8 = ctypes.c_int(), ctypes.c_int()
+    assert lib.jamba_test_gemm_splits(M, N, K, bn, min_k, groups, ctypes.byref(s), ctypes.byref(s8)) == 0
+    return s.value, s8.value
+
+
+def test_k_splits_fill_one_wave(lib):
+    """x_proj and out_proj at decode sizes: tiles x splits stay within one wave
+    of the 148 SMs, every split keeps its minimum of 64-deep steps, and a GEMM
+    whose tiles already fill the SMs is not split"""
+    sms = 148
+    for M, N, K, bn, mk in ((288, 64, 8192, 64, 4), (4096, 64, 8192, 64, 8), (131072, 288, 8192, 144, 8),
+                            (288, 1, 2048, 64, 4), (4096, 65, 1024, 64, 8), (128, 64, 64, 64, 4)):
+        s, _ = _splits(lib, M, N, K, bn, mk)
+        tiles = -(-M // 128) * -(-N // bn)
+        k_tiles = -(-K // 64)
+        assert 1 <= s <= 32
+        if tiles >= sms:
+            assert s == 1
+        else:
+            assert tiles * s <= sms
+            per = -(-k_tiles // s)
+            assert (s - 1) * per < k_tiles          # no empty split
+            assert s == 1 or per >= mk
+    assert _splits(lib, 4096, 64, 8192, 64, 8)[0] == 4   # decode out_proj: 32 weight tiles x 4
+
+
+def test_int8_k_splits(lib):
+    """ExpertsInt8 fp32 expert GEMM at decode batches: 1 to 4 splits of an even
+    number of 64-deep steps; none when the experts hold many rows"""
+    for M, groups, N, K in ((128, 16, 4096, 14336), (64, 16, 4096, 14336), (16, 16, 4096, 14336)):
+        _, s8 = _splits(lib, M, N, K, 64, 4, groups)
+        assert 1 <= s8 <= 4 and (K // 64) % (2 * s8) == 0
+    assert _splits(lib, 32768, 4096, 14336, 64, 4, 16)[1] == 1
