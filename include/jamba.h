@@ -365,6 +365,13 @@ jamba_status jamba_test_scan_plan(int batch, int seqlen, int groups, const float
 jamba_status jamba_test_gemm_splits(int M, int N, int K, int bn, int min_k_tiles, int num_groups, int* splits,
                                     int* i8w_splits_out);
 
+/* Test support for jamba_mamba_prefill_host (no GPU needed): the time-chunk
+ * lengths it cuts a sequence of `seqlen` steps into for a given chunk (chunk
+ * above seqlen counts as seqlen), written to lens (capacity ints); *count is
+ * their number (JAMBA_ERR_INVALID_ARG when above capacity).  Not part of the
+ * method. */
+jamba_status jamba_test_host_chunks(int seqlen, int chunk, int* lens, int capacity, int* count);
+
 /* Test support for the bounded device waits (failure detection without a GPU
  * fault).  Runs jamba_selective_scan (same arguments, chunk > 0 and at least
  * two chunks) but launches no CTA for the first time chunk, so the flags of

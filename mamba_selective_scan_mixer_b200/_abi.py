@@ -86,6 +86,7 @@ SIGNATURES = {
     "jamba_selective_scan_static": [P, I, P, I, P, I, P, I, P, I, I, P, P, P, P, I, P, I, I, I, I, I, P, P],
     "jamba_test_scan_plan": [I, I, I, P, I, P, P, P],
     "jamba_test_gemm_splits": [I, I, I, I, I, I, P, P],
+    "jamba_test_host_chunks": [I, I, P, I, P],
     "jamba_test_scan_missing_predecessor": [P, I, P, I, P, I, P, I, P, I, I, P, P, P, I, P, I, I, I, I, I, I,
                                             ctypes.c_ulonglong, P, SZ, P],
     "jamba_rmsnorm": [P, P, P, I, I, F, I, P],

@@ -781,7 +781,39 @@ cudaError_t copy_rows(void* dst, const void* src, size_t row_bytes, size_t src_p
   return cudaMemcpy2DAsync(dst, dst_pitch, src, src_pitch, row_bytes, (size_t)batch, kind, s);
 }
 
+// Time chunks of the host-memory prefill: the first and last chunks ramp
+// (chunk/4, chunk/2) so that the copy-in before the first prefill and the
+// copy-out after the last one, which nothing overlaps, stay short.
+std::vector<int> host_chunk_lengths(int seqlen, int chunk) {
+  std::vector<int> lens;
+  if (seqlen >= 4 * chunk && chunk >= 64) {
+    const int q = chunk / 4, hlf = chunk / 2;
+    lens.push_back(q);
+    lens.push_back(hlf);
+    int rem = seqlen - 2 * (q + hlf);
+    while (rem > 0) {
+      lens.push_back(rem < chunk ? rem : chunk);
+      rem -= lens.back();
+    }
+    lens.push_back(hlf);
+    lens.push_back(q);
+  } else {
+    for (int t = 0; t < seqlen; t += chunk) lens.push_back(seqlen - t < chunk ? seqlen - t : chunk);
+  }
+  return lens;
+}
+
 }  // namespace
+
+jamba_status jamba_test_host_chunks(int seqlen, int chunk, int* lens, int capacity, int* count) {
+  if (!lens || !count || seqlen <= 0 || chunk <= 0 || capacity < 0)
+    return fail(JAMBA_ERR_INVALID_ARG, "host chunks: bad argument");
+  const std::vector<int> v = host_chunk_lengths(seqlen, chunk < seqlen ? chunk : seqlen);
+  *count = (int)v.size();
+  if ((int)v.size() > capacity) return fail(JAMBA_ERR_INVALID_ARG, "host chunks: capacity too small");
+  for (size_t i = 0; i < v.size(); ++i) lens[i] = v[i];
+  return JAMBA_OK;
+}
 
 jamba_status jamba_mamba_host_workspace_size(jamba_mamba_t h, int batch, int chunk, size_t* bytes) {
   if (!h || !bytes || batch <= 0 || chunk < 0) return fail(JAMBA_ERR_INVALID_ARG, "host workspace_size: bad argument");
@@ -826,24 +858,7 @@ jamba_status jamba_mamba_prefill_host(jamba_mamba_t h, const void* u_host, const
   uint8_t* out_buf[2] = {base + al(pre) + 4 * cb, base + al(pre) + 5 * cb};
   cudaStream_t s = cs(stream);
   const size_t pitch = (size_t)seqlen * tok;   // host row pitch: one batch row of the whole sequence
-  // chunk lengths: the first and last chunks ramp (chunk/4, chunk/2) so that
-  // the copy-in before the first prefill and the copy-out after the last one,
-  // which nothing overlaps, stay short
-  std::vector<int> lens;
-  if (seqlen >= 4 * chunk && chunk >= 64) {
-    const int q = chunk / 4, hlf = chunk / 2;
-    lens.push_back(q);
-    lens.push_back(hlf);
-    int rem = seqlen - 2 * (q + hlf);
-    while (rem > 0) {
-      lens.push_back(rem < chunk ? rem : chunk);
-      rem -= lens.back();
-    }
-    lens.push_back(hlf);
-    lens.push_back(q);
-  } else {
-    for (int t = 0; t < seqlen; t += chunk) lens.push_back(seqlen - t < chunk ? seqlen - t : chunk);
-  }
+  const std::vector<int> lens = host_chunk_lengths(seqlen, chunk);
   const int n_chunks = (int)lens.size();
   // the copy streams start after the work already queued on `stream`
   JB_CUDA(cudaEventRecord(h->ev_comp[1], s));

@@ -1,7 +1,8 @@
 """Host-side logic of the library that needs no GPU: the planner that gives
 each channel group of the bf16 prefill's scan its own number of time chunks
-(through the test entry jamba_test_scan_plan), and the k-split choices of the
-decode-size GEMMs (jamba_test_gemm_splits).
+(through the test entry jamba_test_scan_plan), the k-split choices of the
+decode-size GEMMs (jamba_test_gemm_splits) and the time chunks of the
+host-memory prefill (jamba_test_host_chunks).
 
 A CTA of the scan costs its chunk plus the head it replays: the steps until
 its slowest channel has lost the incoming state, at most the chunk.  The
@@ -133,3 +134,29 @@ def test_int8_k_splits(lib):
         _, s8 = _splits(lib, M, N, K, 64, 4, groups)
         assert 1 <= s8 <= 4 and (K // 64) % (2 * s8) == 0
     assert _splits(lib, 32768, 4096, 14336, 64, 4, 16)[1] == 1
+
+
+def _chunks(lib, seqlen, chunk):
+    buf = (ctypes.c_int * 4096)()
+    n = ctypes.c_int()
+    assert lib.jamba_test_host_chunks(seqlen, chunk, buf, 4096, ctypes.byref(n)) == 0
+    return list(buf)[:n.value]
+
+
+def test_host_prefill_chunks(lib):
+    """the host-memory prefill's time chunks cover the sequence exactly, none
+    longer than the chunk; from four chunks on, the first two and last two
+    ramp (chunk/4, chunk/2) so the unoverlapped first copy-in and last
+    copy-out are short"""
+    assert _chunks(lib, 131072, 16384) == [4096, 8192] + [16384] * 6 + [8192, 8192, 4096]
+    for seqlen, chunk in ((200, 48), (300, 64), (4200, 1024), (131072, 16384), (100, 1000), (65, 64), (1, 16384)):
+        lens = _chunks(lib, seqlen, chunk)
+        c = min(chunk, seqlen)
+        assert sum(lens) == seqlen and all(1 <= n <= c for n in lens)
+        if seqlen >= 4 * c and c >= 64:
+            assert lens[:2] == [c // 4, c // 2] and lens[-2:] == [c // 2, c // 4]
+        else:
+            assert lens[:-1] == [c] * (len(lens) - 1)
+    buf = (ctypes.c_int * 2)()
+    n = ctypes.c_int()
+    assert lib.jamba_test_host_chunks(1000, 10, buf, 2, ctypes.byref(n)) == 1 and n.value == 100
