@@ -5,11 +5,15 @@
 // x at negative times taken from the cache (the last three pre-conv inputs,
 // oldest first) or zero.
 //
-// Prefill: each thread owns 16 bytes of channels (8 bf16 or 4 fp32) over a run
-// of 64 time steps, keeping the three previous inputs in registers, so every
-// input row is read once (plus a 3-row halo per run) with 16-byte loads that
-// are contiguous across the warp; eight rows are requested at a time so that
-// enough bytes are in flight to stream at HBM speed.
+// The bf16 prefill runs the conv in the in_proj GEMM's epilogue (gemm_tc.cuh,
+// EPI_CONVP); conv_fixup_kernel here finishes the few rows that epilogue
+// defers.  The standalone prefill kernel serves the fp32 path, sequences of
+// fewer than three steps and jamba_causal_conv1d: each thread owns 16 bytes
+// of channels (8 bf16 or 4 fp32) over a run of 64 time steps, keeping the
+// three previous inputs in registers, so every input row is read once (plus
+// a 3-row halo per run) with 16-byte loads that are contiguous across the
+// warp; eight rows are requested at a time so that enough bytes are in
+// flight to stream at HBM speed.
 #include "common.cuh"
 #include "host.hpp"
 
