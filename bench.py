@@ -91,14 +91,27 @@ class Clocks:
         self.sel = ["-i", uuid] if uuid else []
 
     def start(self):
+        """Start sampling and return once the sampler writes (at most ~5 s), so that
+        the samples taken from here on cover the timed region that follows: the
+        lines already written are skipped by stop()."""
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
+        self.skip = 0
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
                                           "-lms", "20"] + self.sel, stdout=open(self.path, "w"),
                                          stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+            return
+        t_end = time.time() + 5.0
+        while time.time() < t_end and self.proc.poll() is None:
+            with open(self.path) as f:
+                n = f.read().count("\n")
+            if n > 0:
+                self.skip = n
+                break
+            time.sleep(0.01)
 
     def stop(self):
         if self.proc is None:
@@ -110,7 +123,10 @@ class Clocks:
             self.proc.kill()
         sm, mx, reasons = [], 0.0, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
+        lines = open(self.path).read().splitlines()
+        # samples from the timed region (the last one before it as well when it was shorter than a sample period)
+        lines = lines[self.skip:] or lines[-1:]
+        for line in lines:
             f = [x.strip() for x in line.split(",")]
             if len(f) < 9:
                 continue
