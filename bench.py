@@ -266,9 +266,9 @@ def run_product(args):
         torch.cuda.synchronize()
         J.device_status()
         clocks = Clocks(dev)
+        clocks.start()   # returns once sampling runs; the barrier then lines the ranks up for the timed steps
         barrier(world)
         torch.cuda.synchronize()
-        clocks.start()
         ms, per = event_time_ms(step, args.steps, stream, flush)
         torch.cuda.synchronize()
         barrier(world)
