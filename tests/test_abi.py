@@ -115,6 +115,25 @@ def test_product_path_fails_loudly_without_library(tmp_path):
     assert "raised" in r.stdout, r.stdout + r.stderr
 
 
+def test_binding_refuses_host_tensors():
+    """no CPU path: every binding call with a host tensor raises before the library runs"""
+    import torch
+    import mamba_selective_scan_mixer_b200 as J
+    bf = torch.bfloat16
+    a = torch.zeros(128, 64, dtype=bf)
+    calls = [
+        lambda: J.gemm(a, a),
+        lambda: J.rmsnorm(a, torch.ones(64)),
+        lambda: J.causal_conv1d(torch.zeros(1, 8, 64, dtype=bf), torch.zeros(64, 4, dtype=bf), torch.zeros(64, dtype=bf)),
+        lambda: J.in_proj_conv1d(torch.zeros(1, 8, 64, dtype=bf), torch.zeros(256, 64, dtype=bf),
+                                 torch.zeros(128, 4, dtype=bf), torch.zeros(128, dtype=bf)),
+        lambda: J.quantize_int8_rows(a),
+    ]
+    for call in calls:
+        with pytest.raises(ValueError, match="CUDA tensors only"):
+            call()
+
+
 def test_no_product_module_imports_the_oracle():
     pkg = os.path.join(ROOT, "mamba_selective_scan_mixer_b200")
     for dirpath, _, files in os.walk(pkg):
